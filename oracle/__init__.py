@@ -1,0 +1,11 @@
+"""CPU oracle (fp64, numpy) for the SRFT-int4 KV-cache path.
+
+TEST INFRASTRUCTURE ONLY: imported by the tests, the package smoke check and
+the benchmark's CPU-baseline / reference arm, never by the library.
+"""
+from .srft_oracle import *  # noqa: F401,F403
+from .srft_oracle import (attend_decode, attend_decode_fp16, attend_decode_int4,  # noqa: F401
+                          attend_decode_int4_rotated, compressed_bytes_per_vector, decode,
+                          dequantize, encode, encode_into_cache, fp16_rne, group_scales,
+                          pack_nibbles, quantize, real_dft_basis, srft_forward, srft_inverse,
+                          srft_matrix, unpack_nibbles)

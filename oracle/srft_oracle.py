@@ -1,0 +1,281 @@
+"""Plain fp64 CPU oracle for SRFT-int4 KV-cache compression and decode attention.
+
+TEST INFRASTRUCTURE ONLY. Only the test suite, the package smoke check and the
+benchmark's CPU-baseline / reference arm may import, call or execute anything
+in this package. The library (``rotated_int4_kv_b200``) never imports it, and
+this module imports nothing from the library: the two share no code. Inputs
+come from ``kvgen`` (random draws only).
+
+Sources, cited by page and section (the pages are web renderings of the paper
+"When Quantization Is Free: An int4 KV Cache That Outruns fp16 on Apple
+Silicon", arXiv 2605.05699):
+
+  [ABS]  paperdance.org/p/2605.05699 -- the English abstract: the fused kernel is
+         "sign-randomized FFT + per-channel lambda + per-group abs-max + int4
+         nibble pack"; 3x persistent compression.
+  [M1]   gist.science/de/paper/2605.05699, "Methodik" 1 (SRFT): SRFT(x) =
+         pack(F . diag(s) . x), F the unitary DFT, s a fixed random sign vector.
+  [M2]   same page, "Methodik" 2 (fused kernel), its five steps: load and sign
+         multiply; FFT passes; Hermitian unpack into a real representation;
+         per-channel lambda, per-group abs-max reduction and rounding to signed
+         int4; two int4 values packed into one byte.
+  [M3]   same page, "Methodik" 3 (scaling strategies): per-channel factor (one
+         per coordinate) combined with per-group scaling.
+  [RES]  same page, "Wichtige Ergebnisse" / Speichereffizienz: 3.0-3.56x
+         persistent compression.
+
+Readings taken where the pages leave a step open:
+
+  * Real basis ("pack"): rows in the order DC, (cos_k, sin_k) for
+    k = 1..D/2-1, Nyquist; row 2k-1 = sqrt(2/D) cos(2 pi k n / D), row 2k =
+    sqrt(2/D) sin(2 pi k n / D), row 0 = 1/sqrt(D), row D-1 = (-1)^n/sqrt(D).
+  * lambda multiplies the rotated channels (after the transform) [M2].
+  * Group = G contiguous rotated channels (G = 32 in the product; any G | D
+    here). scale = fp16 round-to-nearest-even of absmax/7, clamped to 65504;
+    the quantiser divides by that stored fp16 scale.
+  * Codes: round half to even, clamped to [-7, 7]; a zero scale gives zero
+    codes. Two's-complement nibbles, even element in the low nibble.
+  * Decode: x_hat = diag(s) F_r^T (c * scale / lambda).
+  * Attention (not on the pages): softmax(sigma <q, x_hat_K>) weighted sum of
+    x_hat_V, sigma = 1/sqrt(D) by default; query head h reads KV head
+    h // (Hq / Hkv).
+
+Parity pins: every function here is checked in ``tests/test_oracle_pins.py``
+against closed forms, brute force and invariants (see that file).
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+FP16_MAX = 65504.0
+QMAX = 7
+
+
+# ---------------------------------------------------------------------------
+# The transform [M1], [M2]
+# ---------------------------------------------------------------------------
+
+def real_dft_basis(D: int) -> np.ndarray:
+    """F_r: the D x D orthonormal real DFT basis (rows = output channels).
+
+    F is the unitary DFT [M1]; "pack" turns its Hermitian-symmetric output into
+    D real numbers [M2]: DC, then (cos_k, sin_k) pairs, then Nyquist. Angles
+    are taken from the exact integer k*n mod D so each entry is accurate to
+    about 1e-16.
+    """
+    if D < 2 or D % 2:
+        raise ValueError("D must be even and >= 2")
+    n = np.arange(D)
+    F = np.zeros((D, D), dtype=np.float64)
+    F[0, :] = 1.0 / math.sqrt(D)
+    amp = math.sqrt(2.0 / D)
+    for k in range(1, D // 2):
+        ang = 2.0 * math.pi * ((k * n) % D) / D
+        F[2 * k - 1, :] = amp * np.cos(ang)
+        F[2 * k, :] = amp * np.sin(ang)
+    F[D - 1, :] = np.where(n % 2 == 0, 1.0, -1.0) / math.sqrt(D)
+    return F
+
+
+def srft_matrix(signs: np.ndarray) -> np.ndarray:
+    """R = F_r . diag(s) [M1]."""
+    s = np.asarray(signs, dtype=np.float64)
+    return real_dft_basis(s.shape[0]) * s[None, :]
+
+
+def srft_forward(x: np.ndarray, signs: np.ndarray, lam: np.ndarray) -> np.ndarray:
+    """y = lambda * (F_r . diag(s) . x), over the last axis, in fp64 [M1], [M2]."""
+    x = np.asarray(x, dtype=np.float64)
+    R = srft_matrix(signs)
+    lam64 = np.asarray(lam, dtype=np.float64)
+    return (x @ R.T) * lam64
+
+
+def srft_inverse(y: np.ndarray, signs: np.ndarray, lam: np.ndarray) -> np.ndarray:
+    """x = diag(s) . F_r^T . (y / lambda): the exact inverse of srft_forward."""
+    y = np.asarray(y, dtype=np.float64) / np.asarray(lam, dtype=np.float64)
+    R = srft_matrix(signs)
+    return y @ R
+
+
+# ---------------------------------------------------------------------------
+# The quantiser [M2], [M3]
+# ---------------------------------------------------------------------------
+
+def fp16_rne(v) -> np.ndarray:
+    """Round fp64 values to the nearest fp16 (ties to even); returned as fp64."""
+    return np.asarray(v, dtype=np.float64).astype(np.float16).astype(np.float64)
+
+
+def group_scales(y: np.ndarray, G: int) -> np.ndarray:
+    """Per-group abs-max scale: fp16_rne(min(absmax/7, 65504)); fp16 array [..., D/G]."""
+    y = np.asarray(y, dtype=np.float64)
+    D = y.shape[-1]
+    if D % G:
+        raise ValueError("G must divide D")
+    a = np.abs(y).reshape(y.shape[:-1] + (D // G, G)).max(axis=-1)
+    return np.minimum(a / QMAX, FP16_MAX).astype(np.float16)
+
+
+def quantize(y: np.ndarray, scales16: np.ndarray, G: int):
+    """Signed int4 codes c = clamp(rint(y / scale), -7, 7); 0 where scale == 0.
+
+    Returns (codes int8 [..., D], pre-rounding values y/scale fp64 [..., D]).
+    """
+    y = np.asarray(y, dtype=np.float64)
+    D = y.shape[-1]
+    sc = np.repeat(np.asarray(scales16, dtype=np.float64), G, axis=-1)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        u = np.where(sc > 0, y / np.where(sc > 0, sc, 1.0), 0.0)
+    codes = np.clip(np.rint(u), -QMAX, QMAX).astype(np.int8)
+    assert codes.shape[-1] == D
+    return codes, u
+
+
+def pack_nibbles(codes: np.ndarray) -> np.ndarray:
+    """Two int4 codes per byte [M2]: byte j = (c[2j] & 0xF) | (c[2j+1] & 0xF) << 4."""
+    c = np.asarray(codes, dtype=np.int64)
+    lo = c[..., 0::2] & 0xF
+    hi = c[..., 1::2] & 0xF
+    return (lo | (hi << 4)).astype(np.uint8)
+
+
+def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
+    """Inverse of pack_nibbles: signed codes in [-8, 7] (int8 [..., 2*nbytes])."""
+    b = np.asarray(packed, dtype=np.int64)
+    lo = b & 0xF
+    hi = (b >> 4) & 0xF
+    lo = np.where(lo >= 8, lo - 16, lo)
+    hi = np.where(hi >= 8, hi - 16, hi)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.int8)
+    out[..., 0::2] = lo
+    out[..., 1::2] = hi
+    return out
+
+
+def encode(x: np.ndarray, signs: np.ndarray, lam: np.ndarray, G: int = 32):
+    """The encode path of [ABS]/[M2] over the last axis.
+
+    Returns dict(packed=uint8 [..., D/2], scales=float16 [..., D/G],
+    codes=int8 [..., D], y=fp64 [..., D], u=fp64 pre-rounding y/scale).
+    """
+    y = srft_forward(x, signs, lam)
+    scales = group_scales(y, G)
+    codes, u = quantize(y, scales, G)
+    return {"packed": pack_nibbles(codes), "scales": scales, "codes": codes, "y": y, "u": u}
+
+
+def dequantize(codes: np.ndarray, scales16: np.ndarray, G: int) -> np.ndarray:
+    """c_hat = c * scale (fp64), scale taken from the stored fp16 value."""
+    sc = np.repeat(np.asarray(scales16, dtype=np.float64), G, axis=-1)
+    return np.asarray(codes, dtype=np.float64) * sc
+
+
+def decode(packed: np.ndarray, scales16: np.ndarray, signs: np.ndarray, lam: np.ndarray,
+           G: int = 32) -> np.ndarray:
+    """x_hat = diag(s) F_r^T (c*scale / lambda), fp64 [..., D]."""
+    return srft_inverse(dequantize(unpack_nibbles(packed), scales16, G), signs, lam)
+
+
+def compressed_bytes_per_vector(D: int, G: int) -> int:
+    """D/2 bytes of codes plus one fp16 scale per group [RES]."""
+    return D // 2 + 2 * (D // G)
+
+
+# ---------------------------------------------------------------------------
+# Cache helpers: the [B, H, T_cap, ...] layout written at token offset pos
+# ---------------------------------------------------------------------------
+
+def encode_into_cache(x: np.ndarray, signs, lam, G: int, codes_cache: np.ndarray,
+                      scales_cache: np.ndarray, pos: int) -> None:
+    """Encode x [B, H, n, D] and write rows pos..pos+n-1 of the cache in place."""
+    n = x.shape[2]
+    enc = encode(x, signs, lam, G)
+    codes_cache[:, :, pos:pos + n, :] = enc["packed"]
+    scales_cache[:, :, pos:pos + n, :] = enc["scales"]
+
+
+# ---------------------------------------------------------------------------
+# Decode attention (read path; not described on the pages)
+# ---------------------------------------------------------------------------
+
+def _softmax_weighted(scores: np.ndarray, values: np.ndarray) -> np.ndarray:
+    m = scores.max()
+    p = np.exp(scores - m)
+    return (p[:, None] * values).sum(axis=0) / p.sum()
+
+
+def attend_decode(q: np.ndarray, k_hat: np.ndarray, v_hat: np.ndarray, seq_lens,
+                  sigma: float | None = None) -> np.ndarray:
+    """One-query decode attention in the original domain, fp64.
+
+    q [B, Hq, D]; k_hat, v_hat [B, Hkv, T, D] (already decoded, fp64 or fp16);
+    seq_lens [B]. Query head h reads KV head h // (Hq // Hkv).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, D = q.shape
+    Hkv = k_hat.shape[1]
+    grp = Hq // Hkv
+    if sigma is None:
+        sigma = 1.0 / math.sqrt(D)
+    out = np.zeros((B, Hq, D), dtype=np.float64)
+    for b in range(B):
+        T = int(seq_lens[b])
+        for h in range(Hq):
+            kh = h // grp
+            K = np.asarray(k_hat[b, kh, :T], dtype=np.float64)
+            V = np.asarray(v_hat[b, kh, :T], dtype=np.float64)
+            out[b, h] = _softmax_weighted(sigma * (K @ q[b, h]), V)
+    return out
+
+
+def attend_decode_int4(q, k_packed, k_scales, v_packed, v_scales, k_params, v_params, seq_lens,
+                       G: int = 32, sigma: float | None = None) -> np.ndarray:
+    """Attention over a packed int4 cache: decode K and V, then attend_decode.
+
+    k_params / v_params = (signs, lambda) of the K and V transforms.
+    """
+    T = int(np.max(seq_lens))
+    kh = decode(k_packed[:, :, :T], k_scales[:, :, :T], k_params[0], k_params[1], G)
+    vh = decode(v_packed[:, :, :T], v_scales[:, :, :T], v_params[0], v_params[1], G)
+    return attend_decode(q, kh, vh, seq_lens, sigma)
+
+
+def attend_decode_int4_rotated(q, k_packed, k_scales, v_packed, v_scales, k_params, v_params,
+                               seq_lens, G: int = 32, sigma: float | None = None) -> np.ndarray:
+    """The same attention computed in the rotated domain.
+
+    q_t = Lambda_K^-1 R_K q; score_t = sigma * sum_g scale_{t,g} sum_{i in g} q_t[i] c_t[i];
+    o_t = sum_t p_t c_hat^V_t; o = R_V^T Lambda_V^-1 o_t. Equal to
+    attend_decode_int4 because R is orthogonal: <q, R^T L^-1 c_hat> =
+    <L^-1 R q, c_hat>.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    B, Hq, D = q.shape
+    Hkv = k_packed.shape[1]
+    grp = Hq // Hkv
+    if sigma is None:
+        sigma = 1.0 / math.sqrt(D)
+    Rk = srft_matrix(k_params[0])
+    Rv = srft_matrix(v_params[0])
+    lk = np.asarray(k_params[1], dtype=np.float64)
+    lv = np.asarray(v_params[1], dtype=np.float64)
+    out = np.zeros((B, Hq, D), dtype=np.float64)
+    for b in range(B):
+        T = int(seq_lens[b])
+        for h in range(Hq):
+            kv = h // grp
+            qt = (Rk @ q[b, h]) / lk
+            ck = dequantize(unpack_nibbles(k_packed[b, kv, :T]), k_scales[b, kv, :T], G)
+            cv = dequantize(unpack_nibbles(v_packed[b, kv, :T]), v_scales[b, kv, :T], G)
+            ot = _softmax_weighted(sigma * (ck @ qt), cv)
+            out[b, h] = Rv.T @ (ot / lv)
+    return out
+
+
+def attend_decode_fp16(q, k16, v16, seq_lens, sigma: float | None = None) -> np.ndarray:
+    """The fp16-cache comparator: the same attention on fp16 K/V, computed in fp64."""
+    return attend_decode(q, np.asarray(k16, dtype=np.float64), np.asarray(v16, dtype=np.float64),
+                         seq_lens, sigma)
