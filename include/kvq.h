@@ -1,0 +1,182 @@
+/*
+ * kvq.h -- C ABI of the SRFT-int4 KV-cache library for NVIDIA B200 (sm_100a).
+ *
+ * The method is the fused KV-cache compression of "When Quantization Is Free:
+ * An int4 KV Cache That Outruns fp16 on Apple Silicon" (arXiv 2605.05699):
+ *   [ABS] paperdance.org/p/2605.05699, abstract: sign-randomised FFT + per-channel
+ *         lambda + per-group abs-max + int4 nibble pack, in one fused kernel.
+ *   [M1]  gist.science/de/paper/2605.05699, "Methodik" 1: SRFT(x) = pack(F . diag(s) . x),
+ *         F the unitary DFT, s a fixed random +/-1 vector.
+ *   [M2]  same page, "Methodik" 2: load + sign, FFT passes, Hermitian unpack to a real
+ *         representation, per-channel lambda, per-group abs-max, signed int4
+ *         rounding, two codes per byte.
+ * The read path (decode, decode attention on the packed cache) is not on the
+ * pages; it is the inverse transform and softmax attention taken in the rotated
+ * domain, valid because F is unitary (<q, R^T y> = <R q, y>).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ *  - Element types are given by their bits: fp16 values are passed as uint16_t
+ *    (IEEE binary16), codes as uint8_t. No CUDA or torch types appear here.
+ *  - All data pointers are DEVICE pointers on the plan's device (the current
+ *    device for kvq_attend_decode_ref), except where a comment says "host".
+ *    The caller owns every buffer; no entry point allocates device memory
+ *    except kvq_plan_create. All pointers must be 16-byte aligned.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream). Every call is asynchronous on that stream and never synchronises.
+ *  - Errors: arguments are checked on the host before anything is launched; a
+ *    failed check returns a negative kvq_status and touches no memory. A CUDA
+ *    error at launch returns KVQ_ERR_CUDA. kvq_last_error() gives a one-line
+ *    description of the last failure on the calling thread.
+ *  - Layouts (row-major, innermost last):
+ *      x / out vectors   fp16 [B, H, n, D]
+ *      codes cache       u8   [B, H, T_cap, D/2]   two's-complement nibbles,
+ *                                                  channel 2j in the low nibble of byte j
+ *      scales cache      fp16 [B, H, T_cap, D/G]   scale of channels [gG, gG+G)
+ *      q                 fp16 [B, Hq, D]
+ *      attention out     fp16 [B, Hq, D]
+ *  - Rotated channel order: channel 0 = DC, channels 2k-1 / 2k = cos / sin of
+ *    frequency k (k = 1 .. D/2-1), channel D-1 = Nyquist. Row 2k-1 of the real
+ *    basis is sqrt(2/D) cos(2 pi k n / D), row 2k is sqrt(2/D) sin(2 pi k n / D).
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kvq_status {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = -1, /* null pointer, non-positive size, bad sign/lambda value */
+  KVQ_ERR_UNSUPPORTED = -2, /* head_dim not 128/256, group not 32/16, Hq % Hkv != 0   */
+  KVQ_ERR_ALIGNMENT = -3,   /* pointer not 16-byte aligned, or T_cap odd (attention)   */
+  KVQ_ERR_CAPACITY = -4,    /* pos + n > T_cap, t0 + n > T_cap, T_len > T_cap           */
+  KVQ_ERR_CUDA = -5,        /* a CUDA runtime call or launch failed                    */
+  KVQ_ERR_WORKSPACE = -6,   /* workspace missing or smaller than kvq_workspace_size    */
+  KVQ_ERR_DEVICE = -7       /* no sm_100 device, or plan used on another device        */
+} kvq_status;
+
+/* Opaque per-(s, lambda) transform plan. Immutable after creation; one plan may be
+ * used from several streams and host threads at once. */
+typedef struct kvq_plan kvq_plan;
+
+/*
+ * kvq_plan_create -- [M1] fixes s, [M2] lambda (one factor per rotated channel).
+ *   out         host: receives the new plan.
+ *   head_dim    D: 128 or 256.
+ *   group       G: channels per abs-max scale group (32; 16 also accepted).
+ *   signs_host  host int8[D], every entry +1 or -1 (the fixed random sign vector s).
+ *   lambda_host host float[D], every entry finite and > 0 (per-channel lambda).
+ * Allocates a small device block on the current device (the plan's device):
+ * s and lambda, and the rotation matrices the attention kernels use for the
+ * query rotation and the output un-rotation (2 x D x D fp16 pairs).
+ * Errors: INVALID_ARG, UNSUPPORTED, CUDA, DEVICE.
+ */
+kvq_status kvq_plan_create(kvq_plan** out, int head_dim, int group, const int8_t* signs_host,
+                           const float* lambda_host);
+
+/* Frees the plan and its device block. Passing NULL is a no-op. The caller must
+ * ensure no launch that uses the plan is still pending. */
+kvq_status kvq_plan_destroy(kvq_plan* plan);
+
+/* Plan properties (head_dim, group); -1 for a NULL plan. */
+int kvq_plan_head_dim(const kvq_plan* plan);
+int kvq_plan_group(const kvq_plan* plan);
+
+/*
+ * kvq_encode -- the fused encode of [ABS]/[M2]: for each fp16 vector x of
+ * x[B, H, n, D]: y = lambda * (F_r . diag(s) . x) (fp32), then per group of G
+ * rotated channels scale = fp16_rn(min(absmax/7, 65504)) and
+ * c = clamp(rint(y / scale), -7, 7) (0 where scale == 0), nibble-packed.
+ *   x        fp16 [B, H, n, D] contiguous.
+ *   codes    u8   [B, H, T_cap, D/2]; rows pos .. pos+n-1 of every (b, h) are written.
+ *   scales   fp16 [B, H, T_cap, D/G]; same rows written.
+ *   T_cap    capacity (tokens) of the cache; pos + n <= T_cap.
+ * No other cache row is touched. n == 0 is a no-op.
+ * Errors: INVALID_ARG, ALIGNMENT, CAPACITY, DEVICE, CUDA.
+ */
+kvq_status kvq_encode(const kvq_plan* plan, const uint16_t* x, int B, int H, int n, uint8_t* codes,
+                      uint16_t* scales, int T_cap, int pos, void* stream);
+
+/*
+ * kvq_decode -- the inverse: x_hat = diag(s) . F_r^T . (c * scale / lambda), rounded
+ * to fp16, for cache rows t0 .. t0+n-1 of every (b, h).
+ *   out  fp16 [B, H, n, D] contiguous.
+ * Errors: INVALID_ARG, ALIGNMENT, CAPACITY, DEVICE, CUDA.
+ */
+kvq_status kvq_decode(const kvq_plan* plan, const uint8_t* codes, const uint16_t* scales, int B,
+                      int H, int T_cap, int t0, int n, uint16_t* out, void* stream);
+
+/*
+ * kvq_workspace_size -- bytes of device workspace that kvq_attend_decode and
+ * kvq_attend_decode_ref need for these shapes (T_cap = the cache capacity; the
+ * split of the sequence is chosen from it). The workspace holds the per-split
+ * softmax partials and one completion counter per (b, kv head, head tile).
+ * The counters must be zero before the first call that uses a workspace (e.g.
+ * cudaMemsetAsync once after allocation); every completed call leaves them zero
+ * again. Two calls must not use the same workspace concurrently.
+ */
+size_t kvq_workspace_size(int B, int Hq, int Hkv, int head_dim, int T_cap);
+
+/*
+ * kvq_attend_decode -- one-query decode attention read straight from the packed
+ * int4 K/V cache, in the rotated domain (not on the pages; follows from [M1]):
+ *   q_t = Lambda_K^-1 R_K q (fp32, kept as an fp16 hi + lo pair),
+ *   score_t = sigma * sum_g scaleK[t,g] * sum_{i in g} q_t[i] * cK[t,i],
+ *   o_t = sum_t softmax(score)_t * (cV[t] * scaleV[t]) (split over the sequence,
+ *         combined with the log-sum-exp rule),
+ *   out = diag(s_V) F_r^T Lambda_V^-1 o_t  -> fp16.
+ *   pk, pv     plans of the K and V transforms (same head_dim and group).
+ *   q          fp16 [B, Hq, D]; query head h reads KV head h / (Hq / Hkv).
+ *   k_codes, v_codes    u8 [B, Hkv, T_cap, D/2];  k_scales, v_scales fp16 [B, Hkv, T_cap, D/G].
+ *   seq_lens   device int32[B] (tokens 0 .. seq_lens[b]-1 are attended; values are
+ *              clamped to [0, T_cap]), or NULL to use T_len for every batch entry.
+ *   softmax_scale  sigma; <= 0 selects 1/sqrt(D).
+ *   out        fp16 [B, Hq, D]. A batch entry with no tokens gets zeros.
+ *   workspace  device buffer of >= kvq_workspace_size(B, Hq, Hkv, D, T_cap) bytes.
+ * T_cap must be even (the scale rows are fetched by TMA in 16-byte units).
+ * Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, CAPACITY, WORKSPACE, DEVICE, CUDA.
+ */
+kvq_status kvq_attend_decode(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q,
+                             const uint8_t* k_codes, const uint16_t* k_scales,
+                             const uint8_t* v_codes, const uint16_t* v_scales, int B, int Hq,
+                             int Hkv, int T_cap, const int32_t* seq_lens, int T_len,
+                             float softmax_scale, uint16_t* out, void* workspace,
+                             size_t ws_bytes, void* stream);
+
+/*
+ * kvq_attend_decode_ref -- the fp16-cache comparator for the same shapes: the same
+ * split-sequence softmax attention over fp16 K/V [B, Hkv, T_cap, D] with no
+ * rotation. This is the uncompressed baseline the int4 path is measured against
+ * (the pages compare int4 with an fp16 cache, [ABS]).
+ * Same argument rules as kvq_attend_decode (head_dim = D is 128 or 256).
+ */
+kvq_status kvq_attend_decode_ref(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B,
+                                 int Hq, int Hkv, int head_dim, int T_cap,
+                                 const int32_t* seq_lens, int T_len, float softmax_scale,
+                                 uint16_t* out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * kvq_poll_device_errors -- synchronises the current device, then returns (in
+ * *flags, host, may be NULL) the bit flags raised by kernels of this library
+ * since the last poll, and clears them: 1 = a kernel gave up waiting for a TMA
+ * load (bounded wait of 1 s), 2 = a bulk store did not drain. 0 means none.
+ * Errors: CUDA.
+ */
+kvq_status kvq_poll_device_errors(uint32_t* flags);
+
+/* Static description of a status code. */
+const char* kvq_status_string(kvq_status status);
+
+/* One-line description of the last failed call on this host thread ("" if none). */
+const char* kvq_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

@@ -1,0 +1,159 @@
+"""torch-facing wrappers over the C ABI (argument marshalling only).
+
+Every call passes raw device pointers and the current CUDA stream to
+``libkvq.so``; all arithmetic runs in the library's CUDA kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import torch
+
+from ._lib import check, lib
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype, shape=None):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.device.type != "cuda":
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+class Plan:
+    """A (sign vector s, lambda) transform plan on the current CUDA device."""
+
+    def __init__(self, signs, lam, group: int = 32):
+        s = np.ascontiguousarray(np.asarray(signs, dtype=np.int8))
+        l = np.ascontiguousarray(np.asarray(lam, dtype=np.float32))
+        if s.ndim != 1 or l.shape != s.shape:
+            raise ValueError("signs and lambda must be 1-D arrays of the same length")
+        self.head_dim = int(s.shape[0])
+        self.group = int(group)
+        self._h = ctypes.c_void_p()
+        check(lib.kvq_plan_create(ctypes.byref(self._h), self.head_dim, self.group,
+                                  s.ctypes.data_as(ctypes.c_void_p), l.ctypes.data_as(ctypes.c_void_p)),
+              "kvq_plan_create")
+        self._lib = lib
+
+    @property
+    def handle(self) -> ctypes.c_void_p:
+        return self._h
+
+    def close(self) -> None:
+        if getattr(self, "_h", None) and self._h.value:
+            self._lib.kvq_plan_destroy(self._h)
+            self._h = ctypes.c_void_p()
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def encode(plan: Plan, x: torch.Tensor, codes: torch.Tensor, scales: torch.Tensor, pos: int = 0,
+           stream=None) -> None:
+    """Encode x [B, H, n, D] fp16 into cache rows pos..pos+n-1 of codes / scales."""
+    B, H, n, D = x.shape
+    T_cap = codes.shape[2]
+    _need(x, "x", torch.float16)
+    _need(codes, "codes", torch.uint8, (B, H, T_cap, D // 2))
+    _need(scales, "scales", torch.float16, (B, H, T_cap, D // plan.group))
+    check(lib.kvq_encode(plan.handle, _ptr(x), B, H, n, _ptr(codes), _ptr(scales), T_cap, int(pos),
+                         _stream(stream)), "kvq_encode")
+
+
+def decode(plan: Plan, codes: torch.Tensor, scales: torch.Tensor, t0: int, n: int, out: torch.Tensor = None,
+           stream=None) -> torch.Tensor:
+    """Decode cache rows t0..t0+n-1 into fp16 [B, H, n, D]."""
+    B, H, T_cap, half = codes.shape
+    D = 2 * half
+    _need(codes, "codes", torch.uint8)
+    _need(scales, "scales", torch.float16, (B, H, T_cap, D // plan.group))
+    if out is None:
+        out = torch.empty((B, H, n, D), dtype=torch.float16, device=codes.device)
+    _need(out, "out", torch.float16, (B, H, n, D))
+    check(lib.kvq_decode(plan.handle, _ptr(codes), _ptr(scales), B, H, T_cap, int(t0), int(n), _ptr(out),
+                         _stream(stream)), "kvq_decode")
+    return out
+
+
+def workspace_size(B: int, Hq: int, Hkv: int, head_dim: int, T_cap: int) -> int:
+    return int(lib.kvq_workspace_size(B, Hq, Hkv, head_dim, T_cap))
+
+
+def make_workspace(B: int, Hq: int, Hkv: int, head_dim: int, T_cap: int, device=None) -> torch.Tensor:
+    """A zero-initialised workspace (its counters must start at zero)."""
+    n = max(16, workspace_size(B, Hq, Hkv, head_dim, T_cap))
+    return torch.zeros(n, dtype=torch.uint8, device=device or torch.device("cuda"))
+
+
+def attend_decode(pk: Plan, pv: Plan, q, k_codes, k_scales, v_codes, v_scales, seq_lens=None, T_len=None,
+                  softmax_scale: float = 0.0, out=None, workspace=None, stream=None) -> torch.Tensor:
+    """One-query decode attention on the packed int4 cache (rotated domain)."""
+    B, Hq, D = q.shape
+    _, Hkv, T_cap, half = k_codes.shape
+    _need(q, "q", torch.float16)
+    for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
+        _need(t, name, torch.uint8, (B, Hkv, T_cap, D // 2))
+    for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+        _need(t, name, torch.float16, (B, Hkv, T_cap, D // pk.group))
+    if seq_lens is not None:
+        _need(seq_lens, "seq_lens", torch.int32, (B,))
+    if T_len is None:
+        T_len = T_cap if seq_lens is None else 0
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float16, device=q.device)
+    _need(out, "out", torch.float16, (B, Hq, D))
+    if workspace is None:
+        workspace = make_workspace(B, Hq, Hkv, D, T_cap, q.device)
+    check(lib.kvq_attend_decode(pk.handle, pv.handle, _ptr(q), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
+                                _ptr(v_scales), B, Hq, Hkv, T_cap, _ptr(seq_lens), int(T_len),
+                                float(softmax_scale), _ptr(out), _ptr(workspace), workspace.numel(),
+                                _stream(stream)), "kvq_attend_decode")
+    return out
+
+
+def attend_decode_ref(q, k, v, seq_lens=None, T_len=None, softmax_scale: float = 0.0, out=None, workspace=None,
+                      stream=None) -> torch.Tensor:
+    """The fp16-cache comparator kernel on the same shapes."""
+    B, Hq, D = q.shape
+    _, Hkv, T_cap, _ = k.shape
+    _need(q, "q", torch.float16)
+    _need(k, "k", torch.float16, (B, Hkv, T_cap, D))
+    _need(v, "v", torch.float16, (B, Hkv, T_cap, D))
+    if seq_lens is not None:
+        _need(seq_lens, "seq_lens", torch.int32, (B,))
+    if T_len is None:
+        T_len = T_cap if seq_lens is None else 0
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float16, device=q.device)
+    _need(out, "out", torch.float16, (B, Hq, D))
+    if workspace is None:
+        workspace = make_workspace(B, Hq, Hkv, D, T_cap, q.device)
+    check(lib.kvq_attend_decode_ref(_ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, D, T_cap, _ptr(seq_lens), int(T_len),
+                                    float(softmax_scale), _ptr(out), _ptr(workspace), workspace.numel(),
+                                    _stream(stream)), "kvq_attend_decode_ref")
+    return out
+
+
+def poll_device_errors() -> int:
+    flags = ctypes.c_uint32(0)
+    check(lib.kvq_poll_device_errors(ctypes.byref(flags)), "kvq_poll_device_errors")
+    return int(flags.value)

@@ -1,0 +1,326 @@
+// kvq_api.cu -- the C ABI: plan management, host-side argument checks, error
+// reporting and the driver entry point for TMA tensor maps.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "kvq_internal.h"
+
+namespace kvq {
+
+uint32_t codec_error_flags(bool clear);
+uint32_t attend_error_flags(bool clear);
+
+namespace {
+thread_local std::string t_last_error;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Per-channel normalisation of the real basis: dg_c = 1/sqrt(D) (DC, Nyquist),
+// sqrt(2/D) (cos rows), -sqrt(2/D) (sin rows: the spectrum slot holds Im X_k and
+// the sin row equals -sqrt(2/D) Im X_k).
+double basis_dg(int c, int D) {
+  if (c == 0 || c == D - 1) return 1.0 / std::sqrt((double)D);
+  return (c & 1) ? std::sqrt(2.0 / D) : -std::sqrt(2.0 / D);
+}
+
+// Row c of the orthonormal real basis at sample n (used only to build the
+// rotation matrices that the attention kernels apply with tensor cores).
+double basis_entry(int c, int n, int D) {
+  if (c == 0) return 1.0 / std::sqrt((double)D);
+  if (c == D - 1) return (n & 1) ? -1.0 / std::sqrt((double)D) : 1.0 / std::sqrt((double)D);
+  const int k = (c + 1) / 2;
+  const long m = ((long)k * n) % D;
+  const double ang = 2.0 * M_PI * (double)m / (double)D;
+  return (c & 1) ? std::sqrt(2.0 / D) * std::cos(ang) : std::sqrt(2.0 / D) * std::sin(ang);
+}
+
+uint16_t f2h_bits(float f) {
+  const __half h = __float2half_rn(f);
+  return __half_as_ushort(h);
+}
+float h2f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
+
+// Fragment order of an m16n8k16 A operand (row-major 16x16 tile) for lane = 4g + c:
+// a0 = A[g][2c..2c+1], a1 = A[g+8][2c..2c+1], a2 = A[g][2c+8..2c+9], a3 = A[g+8][2c+8..2c+9].
+void build_frag(const std::vector<double>& A, int D, std::vector<uint32_t>& out) {
+  const int MT = D / 16;
+  out.assign((size_t)MT * MT * 2 * 32 * 4, 0u);
+  for (int mt = 0; mt < MT; ++mt)
+    for (int kt = 0; kt < MT; ++kt)
+      for (int hl = 0; hl < 2; ++hl)
+        for (int lane = 0; lane < 32; ++lane) {
+          const int g = lane >> 2, c = lane & 3;
+          const int rows[4] = {g, g + 8, g, g + 8};
+          const int cols[4] = {2 * c, 2 * c, 2 * c + 8, 2 * c + 8};
+          for (int r = 0; r < 4; ++r) {
+            uint32_t w = 0;
+            for (int e = 0; e < 2; ++e) {
+              const double a = A[(size_t)(mt * 16 + rows[r]) * D + kt * 16 + cols[r] + e];
+              const float af = (float)a;
+              const uint16_t hi = f2h_bits(af);
+              const uint16_t lo = f2h_bits((float)(a - (double)h2f(hi)));
+              w |= (uint32_t)(hl == 0 ? hi : lo) << (16 * e);
+            }
+            out[((((size_t)mt * MT + kt) * 2 + hl) * 32 + lane) * 4 + r] = w;
+          }
+        }
+}
+}  // namespace
+
+void set_error(const std::string& msg) { t_last_error = msg; }
+
+kvq_status fail(kvq_status st, const std::string& msg) {
+  t_last_error = msg;
+  return st;
+}
+
+kvq_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+                        const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz,
+                        const char* what) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return fail(KVQ_ERR_CUDA, "cuTensorMapEncodeTiled not available from the driver");
+  cuuint64_t d[5];
+  cuuint64_t st[4];
+  cuuint32_t bx[5], es[5];
+  for (int i = 0; i < rank; ++i) {
+    d[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i + 1 < rank; ++i) st[i] = strides_bytes[i];
+  const CUresult r = fn(map, dt, (cuuint32_t)rank, const_cast<void*>(base), d, st, bx, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(KVQ_ERR_CUDA, std::string("tensor map for ") + what + " rejected by the driver");
+  return KVQ_OK;
+}
+
+int num_sms(int device) {
+  static int cache[64] = {0};
+  if (device < 0 || device >= 64) return 148;
+  if (cache[device] == 0) {
+    int v = 0;
+    cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, device);
+    cache[device] = v > 0 ? v : 148;
+  }
+  return cache[device];
+}
+
+kvq_status check_plan_device(const kvq_plan* p) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(KVQ_ERR_DEVICE, "no current CUDA device");
+  if (dev != p->device) return fail(KVQ_ERR_DEVICE, "plan belongs to another device");
+  return KVQ_OK;
+}
+
+}  // namespace kvq
+
+using kvq::fail;
+
+extern "C" {
+
+const char* kvq_status_string(kvq_status s) {
+  switch (s) {
+    case KVQ_OK: return "ok";
+    case KVQ_ERR_INVALID_ARG: return "invalid argument";
+    case KVQ_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KVQ_ERR_ALIGNMENT: return "misaligned pointer or size";
+    case KVQ_ERR_CAPACITY: return "cache capacity exceeded";
+    case KVQ_ERR_CUDA: return "CUDA error";
+    case KVQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case KVQ_ERR_DEVICE: return "device mismatch or unsupported device";
+  }
+  return "unknown status";
+}
+
+const char* kvq_last_error(void) { return kvq::t_last_error.c_str(); }
+
+kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, const float* lambda) {
+  if (!out || !signs || !lambda) return fail(KVQ_ERR_INVALID_ARG, "plan_create: null argument");
+  *out = nullptr;
+  if (D != 128 && D != 256) return fail(KVQ_ERR_UNSUPPORTED, "plan_create: head_dim must be 128 or 256");
+  if (G != 32 && G != 16) return fail(KVQ_ERR_UNSUPPORTED, "plan_create: group must be 32 or 16");
+  for (int i = 0; i < D; ++i) {
+    if (signs[i] != 1 && signs[i] != -1) return fail(KVQ_ERR_INVALID_ARG, "plan_create: signs must be +1/-1");
+    if (!(std::isfinite(lambda[i]) && lambda[i] > 0.0f))
+      return fail(KVQ_ERR_INVALID_ARG, "plan_create: lambda must be finite and > 0");
+  }
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(KVQ_ERR_DEVICE, "plan_create: no CUDA device");
+  cudaDeviceProp prop{};
+  if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess || prop.major != 10)
+    return fail(KVQ_ERR_DEVICE, "plan_create: needs a compute capability 10.x (sm_100) device");
+
+  kvq_plan* p = new kvq_plan();
+  p->D = D;
+  p->G = G;
+  p->device = dev;
+  for (int c = 0; c < D; ++c) {
+    const double dg = kvq::basis_dg(c, D);
+    p->enc.chan[c] = (float)((double)lambda[c] * dg);
+    p->dec.chan[c] = (float)(dg / (double)lambda[c]);
+  }
+  for (int w = 0; w < D / 2; ++w) {
+    const uint32_t m = (signs[2 * w] < 0 ? 0x8000u : 0u) | (signs[2 * w + 1] < 0 ? 0x80000000u : 0u);
+    p->enc.sgn[w] = m;
+    p->dec.sgn[w] = m;
+  }
+  // R' = Lambda^-1 F_r diag(s) and its transpose, as split-fp16 mma fragments
+  std::vector<double> R((size_t)D * D), RT((size_t)D * D);
+  for (int i = 0; i < D; ++i)
+    for (int j = 0; j < D; ++j) {
+      const double v = kvq::basis_entry(i, j, D) * (double)signs[j] / (double)lambda[i];
+      R[(size_t)i * D + j] = v;
+      RT[(size_t)j * D + i] = v;
+    }
+  std::vector<uint32_t> fq, fo;
+  kvq::build_frag(R, D, fq);
+  kvq::build_frag(RT, D, fo);
+  const size_t bytes = fq.size() * 4;
+  void* blk = nullptr;
+  if (cudaMalloc(&blk, 2 * bytes) != cudaSuccess) {
+    delete p;
+    return fail(KVQ_ERR_CUDA, "plan_create: cudaMalloc failed");
+  }
+  if (cudaMemcpy(blk, fq.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy((char*)blk + bytes, fo.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess) {
+    cudaFree(blk);
+    delete p;
+    return fail(KVQ_ERR_CUDA, "plan_create: upload failed");
+  }
+  p->dblock = blk;
+  p->rq_frag = reinterpret_cast<const uint4*>(blk);
+  p->ro_frag = reinterpret_cast<const uint4*>((char*)blk + bytes);
+  *out = p;
+  return KVQ_OK;
+}
+
+kvq_status kvq_plan_destroy(kvq_plan* p) {
+  if (!p) return KVQ_OK;
+  if (p->dblock) {
+    int cur = -1;
+    cudaGetDevice(&cur);
+    if (cur != p->device) cudaSetDevice(p->device);
+    cudaFree(p->dblock);
+    if (cur != p->device && cur >= 0) cudaSetDevice(cur);
+  }
+  delete p;
+  return KVQ_OK;
+}
+
+int kvq_plan_head_dim(const kvq_plan* p) { return p ? p->D : -1; }
+int kvq_plan_group(const kvq_plan* p) { return p ? p->G : -1; }
+
+kvq_status kvq_encode(const kvq_plan* p, const uint16_t* x, int B, int H, int n, uint8_t* codes, uint16_t* scales,
+                      int T_cap, int pos, void* stream) {
+  if (!p) return fail(KVQ_ERR_INVALID_ARG, "encode: null plan");
+  if (B < 0 || H < 0 || n < 0 || T_cap < 0 || pos < 0) return fail(KVQ_ERR_INVALID_ARG, "encode: negative size");
+  if ((long)pos + n > T_cap) return fail(KVQ_ERR_CAPACITY, "encode: pos + n > T_cap");
+  if (B == 0 || H == 0 || n == 0) return KVQ_OK;
+  if (!x || !codes || !scales) return fail(KVQ_ERR_INVALID_ARG, "encode: null buffer");
+  if (!kvq::aligned16(x) || !kvq::aligned16(codes) || !kvq::aligned16(scales))
+    return fail(KVQ_ERR_ALIGNMENT, "encode: buffers must be 16-byte aligned");
+  if ((long)B * H > (1L << 30) || (long)T_cap * B * H > (1L << 40)) return fail(KVQ_ERR_INVALID_ARG, "encode: too large");
+  kvq_status st = kvq::check_plan_device(p);
+  if (st != KVQ_OK) return st;
+  return kvq::launch_encode(p, x, B, H, n, codes, scales, T_cap, pos, (cudaStream_t)stream);
+}
+
+kvq_status kvq_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* scales, int B, int H, int T_cap,
+                      int t0, int n, uint16_t* out, void* stream) {
+  if (!p) return fail(KVQ_ERR_INVALID_ARG, "decode: null plan");
+  if (B < 0 || H < 0 || n < 0 || T_cap < 0 || t0 < 0) return fail(KVQ_ERR_INVALID_ARG, "decode: negative size");
+  if ((long)t0 + n > T_cap) return fail(KVQ_ERR_CAPACITY, "decode: t0 + n > T_cap");
+  if (B == 0 || H == 0 || n == 0) return KVQ_OK;
+  if (!out || !codes || !scales) return fail(KVQ_ERR_INVALID_ARG, "decode: null buffer");
+  if (!kvq::aligned16(out) || !kvq::aligned16(codes) || !kvq::aligned16(scales))
+    return fail(KVQ_ERR_ALIGNMENT, "decode: buffers must be 16-byte aligned");
+  if ((long)B * H > (1L << 30) || (long)T_cap * B * H > (1L << 40)) return fail(KVQ_ERR_INVALID_ARG, "decode: too large");
+  kvq_status st = kvq::check_plan_device(p);
+  if (st != KVQ_OK) return st;
+  return kvq::launch_decode(p, codes, scales, B, H, T_cap, t0, n, out, (cudaStream_t)stream);
+}
+
+size_t kvq_workspace_size(int B, int Hq, int Hkv, int D, int T_cap) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || T_cap < 0 || (D != 128 && D != 256) || Hq % Hkv) return 0;
+  return kvq::attend_workspace_bytes(B, Hq, Hkv, D, T_cap);
+}
+
+static kvq_status check_attend_common(int B, int Hq, int Hkv, int D, int T_cap, int T_len, const void* q,
+                                      const void* out, const void* ws, size_t ws_bytes) {
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || T_cap < 0) return fail(KVQ_ERR_INVALID_ARG, "attend: bad sizes");
+  if (Hq % Hkv) return fail(KVQ_ERR_UNSUPPORTED, "attend: Hq must be a multiple of Hkv");
+  if (T_cap & 1) return fail(KVQ_ERR_ALIGNMENT, "attend: T_cap must be even");
+  if (T_len < 0) return fail(KVQ_ERR_INVALID_ARG, "attend: T_len < 0");
+  if (T_len > T_cap) return fail(KVQ_ERR_CAPACITY, "attend: T_len > T_cap");
+  if (B == 0) return KVQ_OK;
+  if (!q || !out) return fail(KVQ_ERR_INVALID_ARG, "attend: null buffer");
+  if (!kvq::aligned16(q) || !kvq::aligned16(out)) return fail(KVQ_ERR_ALIGNMENT, "attend: q/out must be 16-byte aligned");
+  const size_t need = kvq::attend_workspace_bytes(B, Hq, Hkv, D, T_cap);
+  if (!ws || ws_bytes < need) return fail(KVQ_ERR_WORKSPACE, "attend: workspace missing or too small");
+  if (!kvq::aligned16(ws)) return fail(KVQ_ERR_ALIGNMENT, "attend: workspace must be 16-byte aligned");
+  return KVQ_OK;
+}
+
+kvq_status kvq_attend_decode(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q, const uint8_t* kc,
+                             const uint16_t* ks, const uint8_t* vc, const uint16_t* vs, int B, int Hq, int Hkv,
+                             int T_cap, const int32_t* seq_lens, int T_len, float sigma, uint16_t* out,
+                             void* ws, size_t ws_bytes, void* stream) {
+  if (!pk || !pv) return fail(KVQ_ERR_INVALID_ARG, "attend: null plan");
+  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device)
+    return fail(KVQ_ERR_INVALID_ARG, "attend: K and V plans differ in head_dim, group or device");
+  if (pk->G != 32) return fail(KVQ_ERR_UNSUPPORTED, "attend: group must be 32");
+  kvq_status st = check_attend_common(B, Hq, Hkv, pk->D, T_cap, T_len, q, out, ws, ws_bytes);
+  if (st != KVQ_OK || B == 0) return st;
+  if (!kc || !ks || !vc || !vs) return fail(KVQ_ERR_INVALID_ARG, "attend: null cache buffer");
+  if (!kvq::aligned16(kc) || !kvq::aligned16(ks) || !kvq::aligned16(vc) || !kvq::aligned16(vs))
+    return fail(KVQ_ERR_ALIGNMENT, "attend: cache buffers must be 16-byte aligned");
+  st = kvq::check_plan_device(pk);
+  if (st != KVQ_OK) return st;
+  return kvq::launch_attend_int4(pk, pv, q, kc, ks, vc, vs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, out, ws,
+                                 ws_bytes, (cudaStream_t)stream);
+}
+
+kvq_status kvq_attend_decode_ref(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq, int Hkv,
+                                 int D, int T_cap, const int32_t* seq_lens, int T_len, float sigma, uint16_t* out,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  if (D != 128 && D != 256) return fail(KVQ_ERR_UNSUPPORTED, "attend_ref: head_dim must be 128 or 256");
+  kvq_status st = check_attend_common(B, Hq, Hkv, D, T_cap, T_len, q, out, ws, ws_bytes);
+  if (st != KVQ_OK || B == 0) return st;
+  if (!k || !v) return fail(KVQ_ERR_INVALID_ARG, "attend_ref: null cache buffer");
+  if (!kvq::aligned16(k) || !kvq::aligned16(v)) return fail(KVQ_ERR_ALIGNMENT, "attend_ref: K/V must be 16-byte aligned");
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(KVQ_ERR_DEVICE, "attend_ref: no CUDA device");
+  return kvq::launch_attend_fp16(q, k, v, B, Hq, Hkv, D, T_cap, seq_lens, T_len, sigma, out, ws, ws_bytes,
+                                 (cudaStream_t)stream);
+}
+
+kvq_status kvq_poll_device_errors(uint32_t* flags) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return fail(KVQ_ERR_CUDA, "poll: device synchronize failed");
+  const uint32_t f = kvq::codec_error_flags(true) | kvq::attend_error_flags(true);
+  if (flags) *flags = f;
+  return KVQ_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,75 @@
+// kvq_internal.h -- definitions shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/kvq.h"
+
+namespace kvq {
+
+constexpr int kMaxD = 256;
+
+// Per-plan constants handed to the codec kernels by value (kernel parameter
+// space), so that every per-channel factor is a constant-bank operand.
+struct CodecConsts {
+  float chan[kMaxD];       // encode: lambda_c * dg_c ; decode: dg_c / lambda_c (rotated channel c)
+  uint32_t sgn[kMaxD / 2]; // XOR mask per fp16 pair of the original domain (0x8000 per negative s)
+};
+
+}  // namespace kvq
+
+struct kvq_plan {
+  int D = 0;
+  int G = 0;
+  int device = -1;
+  kvq::CodecConsts enc{};  // lambda_c * dg_c
+  kvq::CodecConsts dec{};  // dg_c / lambda_c
+  // Device block: the rotation R' = Lambda^-1 F_r diag(s) in mma fragment order,
+  // split into fp16 hi + lo parts, once as A = R' (query rotation, q_t = R' q)
+  // and once as A = R'^T (output un-rotation, o = R'^T o_t).
+  void* dblock = nullptr;
+  const uint4* rq_frag = nullptr;   // [D/16 m-tiles][D/16 k-tiles][2 hi/lo][32 lanes] uint4
+  const uint4* ro_frag = nullptr;   // same layout for R'^T
+};
+
+namespace kvq {
+
+// thread-local last-error text
+void set_error(const std::string& msg);
+kvq_status fail(kvq_status st, const std::string& msg);
+
+// driver entry point for tensor-map encoding (no link against libcuda)
+kvq_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base,
+                        const uint64_t* dims, const uint64_t* strides_bytes, const uint32_t* box,
+                        CUtensorMapSwizzle swz, const char* what);
+
+int num_sms(int device);
+
+kvq_status check_plan_device(const kvq_plan* p);
+
+// codec launchers (kvq_codec.cu)
+kvq_status launch_encode(const kvq_plan* p, const uint16_t* x, int B, int H, int n, uint8_t* codes,
+                         uint16_t* scales, int T_cap, int pos, cudaStream_t s);
+kvq_status launch_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* scales, int B, int H,
+                         int T_cap, int t0, int n, uint16_t* out, cudaStream_t s);
+
+// attention launchers (kvq_attend.cu)
+size_t attend_workspace_bytes(int B, int Hq, int Hkv, int D, int T_cap);
+kvq_status launch_attend_int4(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q,
+                              const uint8_t* kc, const uint16_t* ks, const uint8_t* vc, const uint16_t* vs,
+                              int B, int Hq, int Hkv, int T_cap, const int32_t* seq_lens, int T_len,
+                              float sigma, uint16_t* out, void* ws, size_t ws_bytes, cudaStream_t s);
+kvq_status launch_attend_fp16(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
+                              int Hkv, int D, int T_cap, const int32_t* seq_lens, int T_len, float sigma,
+                              uint16_t* out, void* ws, size_t ws_bytes, cudaStream_t s);
+
+// device error word (bit flags raised by kernels that gave up a bounded wait)
+uint32_t* device_error_word();
+
+}  // namespace kvq

@@ -1,0 +1,160 @@
+// srft_fft.cuh -- real DFT of a register-resident vector, for the SRFT of
+// "When Quantization Is Free" (gist.science/de/paper/2605.05699, "Methodik" 1-2:
+// SRFT(x) = pack(F . diag(s) . x); the FFT passes and the Hermitian unpack into a
+// real representation).
+//
+// The pages run log2(d/2) radix-2 Stockham passes on Metal SIMD groups. Here one
+// thread owns a whole vector in registers and runs a radix-2 decimation-in-time
+// real FFT whose twiddles are compile-time immediates, so no shuffles and no
+// shared-memory passes are needed.
+//
+// Slot layout of a size-N real spectrum (unnormalised, X_k = sum_n x_n e^{-2 pi i k n/N}):
+//   slot 0 = X_0 (DC), slot 1 = X_{N/2} (Nyquist), slot 2k = Re X_k, slot 2k+1 = Im X_k.
+// The transform of the samples v[OFF + S*j] (j < N) is written in place: slot j
+// lands in v[OFF + S*j]. A size-N stage combines the spectra E (even samples,
+// slots at v[OFF + 2S j]) and O (odd samples, at v[OFF + S + 2S j]):
+//   X_0 = E_0 + O_0, X_{N/2} = E_0 - O_0, X_{N/4} = E_{N/4} - i O_{N/4},
+//   X_k = E_k + W^k O_k, X_{N/2-k} = conj(E_k - W^k O_k), W = e^{-2 pi i / N},
+// with the k-butterfly written as four FMAs plus two (a+b, 2a-(a+b)) FMAs.
+// rdft_inv is the exact transpose of rdft_fwd (adjoint), so for the orthonormal
+// real basis F_r = P Dg A, F_r^T = A^T Dg P^T: decode runs the transpose after
+// applying the per-channel normalisation.
+#pragma once
+
+#include <cuda_runtime.h>
+
+namespace kvq {
+
+// ---------------------------------------------------------------- compile-time twiddles
+// cos / sin of 2 pi m / n, by exact rational octant reduction and a Taylor series
+// in double precision (all arguments end up in [0, pi/4]); rounded to float by the caller.
+__host__ __device__ constexpr double kTwoPi = 6.283185307179586476925286766559;
+
+__host__ __device__ constexpr double taylor_sin(double x) {
+  double term = x, sum = x;
+  const double x2 = x * x;
+  for (int i = 1; i < 16; ++i) {
+    term *= -x2 / double((2 * i) * (2 * i + 1));
+    sum += term;
+  }
+  return sum;
+}
+
+__host__ __device__ constexpr double taylor_cos(double x) {
+  double term = 1.0, sum = 1.0;
+  const double x2 = x * x;
+  for (int i = 1; i < 16; ++i) {
+    term *= -x2 / double((2 * i - 1) * (2 * i));
+    sum += term;
+  }
+  return sum;
+}
+
+// cos(2 pi m / n) for integers m, n > 0
+__host__ __device__ constexpr double cos2pi_frac(long m, long n) {
+  m %= n;
+  if (m < 0) m += n;
+  if (2 * m > n) m = n - m;                      // cos(2pi f) = cos(2pi (1-f)); f in [0, 1/2]
+  if (4 * m > n) return -cos2pi_frac(n - 2 * m, 2 * n);  // = -cos(2pi (1/2 - f))
+  if (8 * m > n) return taylor_sin(kTwoPi * double(n - 4 * m) / double(4 * n));  // = sin(2pi(1/4 - f))
+  return taylor_cos(kTwoPi * double(m) / double(n));
+}
+
+__host__ __device__ constexpr double sin2pi_frac(long m, long n) { return cos2pi_frac(n - 4 * m, 4 * n); }
+
+// ---------------------------------------------------------------- butterflies
+template <int N, int OFF, int S, int TOT, int K>
+struct RdftBfly {
+  static __device__ __forceinline__ void fwd(float (&v)[TOT], const float (&e)[N / 2], const float (&o)[N / 2]) {
+    if constexpr (K < N / 4) {
+      constexpr float c = static_cast<float>(cos2pi_frac(K, N));
+      constexpr float s = static_cast<float>(sin2pi_frac(K, N));
+      const float er = e[2 * K], ei = e[2 * K + 1], orr = o[2 * K], oi = o[2 * K + 1];
+      // W^K O = (c*or + s*oi) + i (c*oi - s*or)
+      const float xr = fmaf(c, orr, fmaf(s, oi, er));
+      const float xi = fmaf(c, oi, fmaf(-s, orr, ei));
+      v[OFF + S * (2 * K)] = xr;
+      v[OFF + S * (2 * K + 1)] = xi;
+      v[OFF + S * (N - 2 * K)] = fmaf(2.0f, er, -xr);      // Re(E - W O)
+      v[OFF + S * (N - 2 * K + 1)] = fmaf(-2.0f, ei, xi);  // -Im(E - W O)
+      RdftBfly<N, OFF, S, TOT, K + 1>::fwd(v, e, o);
+    }
+  }
+  static __device__ __forceinline__ void inv(const float (&v)[TOT], float (&e)[N / 2], float (&o)[N / 2]) {
+    if constexpr (K < N / 4) {
+      constexpr float c = static_cast<float>(cos2pi_frac(K, N));
+      constexpr float s = static_cast<float>(sin2pi_frac(K, N));
+      const float ar = v[OFF + S * (2 * K)], ai = v[OFF + S * (2 * K + 1)];
+      const float br = v[OFF + S * (N - 2 * K)], bi = v[OFF + S * (N - 2 * K + 1)];
+      e[2 * K] = ar + br;
+      e[2 * K + 1] = ai - bi;
+      const float dr = ar - br, di = ai + bi;
+      o[2 * K] = fmaf(c, dr, -s * di);
+      o[2 * K + 1] = fmaf(s, dr, c * di);
+      RdftBfly<N, OFF, S, TOT, K + 1>::inv(v, e, o);
+    }
+  }
+};
+
+template <int N, int OFF, int S, int TOT>
+struct Rdft {
+  static_assert(N >= 4 && (N & (N - 1)) == 0, "N must be a power of two >= 4");
+  static __device__ __forceinline__ void fwd(float (&v)[TOT]) {
+    Rdft<N / 2, OFF, 2 * S, TOT>::fwd(v);
+    Rdft<N / 2, OFF + S, 2 * S, TOT>::fwd(v);
+    constexpr int M = N / 2;
+    float e[M], o[M];
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+      e[j] = v[OFF + 2 * S * j];
+      o[j] = v[OFF + S + 2 * S * j];
+    }
+    v[OFF] = e[0] + o[0];
+    v[OFF + S] = e[0] - o[0];
+    v[OFF + S * M] = e[1];
+    v[OFF + S * (M + 1)] = -o[1];
+    RdftBfly<N, OFF, S, TOT, 1>::fwd(v, e, o);
+  }
+  static __device__ __forceinline__ void inv(float (&v)[TOT]) {
+    constexpr int M = N / 2;
+    float e[M], o[M];
+    const float x0 = v[OFF], xn = v[OFF + S];
+    e[0] = x0 + xn;
+    o[0] = x0 - xn;
+    e[1] = v[OFF + S * M];
+    o[1] = -v[OFF + S * (M + 1)];
+    RdftBfly<N, OFF, S, TOT, 1>::inv(v, e, o);
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+      v[OFF + 2 * S * j] = e[j];
+      v[OFF + S + 2 * S * j] = o[j];
+    }
+    Rdft<N / 2, OFF, 2 * S, TOT>::inv(v);
+    Rdft<N / 2, OFF + S, 2 * S, TOT>::inv(v);
+  }
+};
+
+template <int OFF, int S, int TOT>
+struct Rdft<2, OFF, S, TOT> {
+  static __device__ __forceinline__ void fwd(float (&v)[TOT]) {
+    const float a = v[OFF], b = v[OFF + S];
+    v[OFF] = a + b;
+    v[OFF + S] = a - b;
+  }
+  static __device__ __forceinline__ void inv(float (&v)[TOT]) { fwd(v); }
+};
+
+// Whole-vector transforms: slots of the size-N spectrum in v[0..N).
+template <int N>
+__device__ __forceinline__ void rdft_fwd(float (&v)[N]) {
+  Rdft<N, 0, 1, N>::fwd(v);
+}
+template <int N>
+__device__ __forceinline__ void rdft_inv(float (&v)[N]) {
+  Rdft<N, 0, 1, N>::inv(v);
+}
+
+// Rotated channel c (DC, cos1, sin1, ..., Nyquist order) <-> spectrum slot.
+__host__ __device__ constexpr int slot_of_channel(int c, int N) { return c == 0 ? 0 : (c == N - 1 ? 1 : c + 1); }
+
+}  // namespace kvq
