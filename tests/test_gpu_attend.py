@@ -1,0 +1,202 @@
+"""GPU parity of kvq_attend_decode (int4, rotated domain) and kvq_attend_decode_ref
+(fp16) against the oracle, through the C ABI. The int4 oracle runs on the GPU's
+own packed cache (codes and scales copied back), per the acceptance rule."""
+import numpy as np
+import pytest
+
+import kvgen
+import oracle
+from tests.parity import check_rel_l2
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def kvq():
+    import rotated_int4_kv_b200 as k
+    return k
+
+
+def _build_cache(kvq, wl, B, Hkv, T_cap, T_fill, seed=21, layer=0):
+    D = wl.head_dim
+    dev = torch.device("cuda")
+    out = {}
+    for kind in ("k", "v"):
+        s, lam = kvgen.plan_params(D, seed=seed, layer=layer, kind=kind)
+        plan = kvq.Plan(s, lam)
+        x = torch.from_numpy(kvgen.kv_numpy(wl, kind, (B, Hkv, T_fill, D), seed=seed, layer=layer)).to(dev)
+        codes = torch.zeros((B, Hkv, T_cap, D // 2), dtype=torch.uint8, device=dev)
+        scales = torch.zeros((B, Hkv, T_cap, D // 32), dtype=torch.float16, device=dev)
+        kvq.encode(plan, x, codes, scales, 0)
+        out[kind] = dict(plan=plan, params=(s, lam), x=x, codes=codes, scales=scales)
+    return out
+
+
+def _oracle_int4(q16, cache, lens, sigma=None):
+    k, v = cache["k"], cache["v"]
+    return oracle.attend_decode_int4(q16, k["codes"].cpu().numpy(), k["scales"].cpu().numpy(),
+                                     v["codes"].cpu().numpy(), v["scales"].cpu().numpy(), k["params"],
+                                     v["params"], lens, 32, sigma)
+
+
+CASES = [
+    # (workload, B, Hkv, Hq, T_cap, lens)  lens: None -> T_len = T_cap
+    ("toy", 1, 1, 1, 256, None),
+    ("qwen", 1, 2, 12, 1024, None),
+    ("qwen", 2, 2, 12, 1000, [1000, 531]),
+    ("qwen", 3, 2, 4, 130, [1, 0, 129]),
+    ("mistral", 2, 8, 32, 700, [700, 65]),
+    ("longctx", 1, 2, 16, 300, None),          # GQA 8
+    ("longctx", 1, 1, 16, 200, [77]),           # GQA 16: two head tiles
+    ("gemma", 1, 1, 4, 4096, None),             # D = 256
+    ("gemma", 2, 2, 6, 333, [333, 17]),         # D = 256, GQA 3, ragged
+]
+
+
+def _ids(cases):
+    return [f"{c[0]}-B{c[1]}kv{c[2]}q{c[3]}T{c[4]}" + ("" if c[5] is None else "ragged") for c in cases]
+
+
+@pytest.mark.parametrize("case", CASES, ids=_ids(CASES))
+def test_attend_int4_matches_oracle(kvq, case):
+    wl_name, B, Hkv, Hq, T_cap, lens = case
+    wl = kvgen.WORKLOADS[wl_name]
+    D = wl.head_dim
+    cache = _build_cache(kvq, wl, B, Hkv, T_cap, T_cap)
+    q16 = kvgen.q_numpy((B, Hq, D), salt=5)
+    q = torch.from_numpy(q16).cuda()
+    if lens is None:
+        out = kvq.attend_decode(cache["k"]["plan"], cache["v"]["plan"], q, cache["k"]["codes"],
+                                cache["k"]["scales"], cache["v"]["codes"], cache["v"]["scales"], T_len=T_cap)
+        lens_np = [T_cap] * B
+    else:
+        sl = torch.tensor(lens, dtype=torch.int32, device="cuda")
+        out = kvq.attend_decode(cache["k"]["plan"], cache["v"]["plan"], q, cache["k"]["codes"],
+                                cache["k"]["scales"], cache["v"]["codes"], cache["v"]["scales"], seq_lens=sl)
+        lens_np = lens
+    torch.cuda.synchronize()
+    assert kvq.poll_device_errors() == 0
+    got = out.cpu().numpy().astype(np.float64)
+    ref = np.zeros((B, Hq, D))
+    live = [i for i in range(B) if lens_np[i] > 0]
+    if live:
+        sub = _oracle_int4(q16[live], {k: dict(v, codes=v["codes"][live], scales=v["scales"][live])
+                                       for k, v in cache.items()}, [lens_np[i] for i in live])
+        ref[live] = sub
+    for i in range(B):
+        if lens_np[i] == 0:
+            assert not got[i].any(), "empty sequence must give zeros"
+    if live:
+        check_rel_l2(got[live].reshape(-1, D), ref[live].reshape(-1, D), label=str(case))
+
+
+@pytest.mark.parametrize("case", CASES, ids=_ids(CASES))
+def test_attend_fp16_ref_matches_oracle(kvq, case):
+    wl_name, B, Hkv, Hq, T_cap, lens = case
+    wl = kvgen.WORKLOADS[wl_name]
+    D = wl.head_dim
+    k16 = kvgen.kv_numpy(wl, "k", (B, Hkv, T_cap, D), seed=31)
+    v16 = kvgen.kv_numpy(wl, "v", (B, Hkv, T_cap, D), seed=31)
+    q16 = kvgen.q_numpy((B, Hq, D), salt=6)
+    k, v, q = (torch.from_numpy(a).cuda() for a in (k16, v16, q16))
+    if lens is None:
+        out = kvq.attend_decode_ref(q, k, v, T_len=T_cap)
+        lens_np = [T_cap] * B
+    else:
+        out = kvq.attend_decode_ref(q, k, v, seq_lens=torch.tensor(lens, dtype=torch.int32, device="cuda"))
+        lens_np = lens
+    torch.cuda.synchronize()
+    assert kvq.poll_device_errors() == 0
+    got = out.cpu().numpy().astype(np.float64)
+    live = [i for i in range(B) if lens_np[i] > 0]
+    for i in range(B):
+        if lens_np[i] == 0:
+            assert not got[i].any()
+    if live:
+        ref = oracle.attend_decode_fp16(q16[live], k16[live], v16[live], [lens_np[i] for i in live])
+        check_rel_l2(got[live].reshape(-1, D), ref.reshape(-1, D), label=str(case))
+
+
+def test_attend_split_independence_and_workspace_reuse(kvq):
+    """The same inputs through T_len (split chosen from T_len) and through seq_lens
+    (split chosen from T_cap), twice on one workspace, agree to fp32 noise."""
+    wl = kvgen.WORKLOADS["qwen"]
+    B, Hkv, Hq, T_cap, T = 1, 2, 12, 8192, 600
+    cache = _build_cache(kvq, wl, B, Hkv, T_cap, T_cap, seed=5)
+    q = torch.from_numpy(kvgen.q_numpy((B, Hq, 128), salt=9)).cuda()
+    ws = kvq.make_workspace(B, Hq, Hkv, 128, T_cap)
+    args = (cache["k"]["plan"], cache["v"]["plan"], q, cache["k"]["codes"], cache["k"]["scales"],
+            cache["v"]["codes"], cache["v"]["scales"])
+    a = kvq.attend_decode(*args, T_len=T, workspace=ws).float()
+    b = kvq.attend_decode(*args, seq_lens=torch.tensor([T], dtype=torch.int32, device="cuda"), workspace=ws).float()
+    c2 = kvq.attend_decode(*args, T_len=T, workspace=ws).float()
+    torch.cuda.synchronize()
+    assert torch.equal(a, c2)
+    assert float((a - b).norm() / a.norm()) < 1e-3
+    assert not torch.count_nonzero(ws[:64])  # counters left at zero
+
+
+def test_attend_errors(kvq):
+    wl = kvgen.WORKLOADS["toy"]
+    cache = _build_cache(kvq, wl, 1, 1, 64, 64)
+    q = torch.zeros((1, 1, 128), dtype=torch.float16, device="cuda")
+    args = (cache["k"]["plan"], cache["v"]["plan"], q, cache["k"]["codes"], cache["k"]["scales"],
+            cache["v"]["codes"], cache["v"]["scales"])
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.attend_decode(*args, T_len=65)
+    assert e.value.status == -4
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.attend_decode(*args, T_len=10, workspace=torch.zeros(8, dtype=torch.uint8, device="cuda"))
+    assert e.value.status == -6
+
+
+def test_mistral_full_size_sampled(kvq):
+    """Mistral-7B-shaped batched decode at full size (B=16, 8 KV heads, 32 query heads,
+    T=32768, D=128), one layer, in the bench's launch configuration; sampled
+    (b, q head) rows checked against the oracle on the same packed cache."""
+    wl = kvgen.WORKLOADS["mistral"]
+    B, Hkv, Hq, T, D = wl.batch, wl.h_kv, wl.h_q, wl.contexts[0], wl.head_dim
+    dev = torch.device("cuda")
+    plans, caches = {}, {}
+    for kind in ("k", "v"):
+        s, lam = kvgen.plan_params(D, layer=0, kind=kind)
+        plans[kind] = (kvq.Plan(s, lam), (s, lam))
+        codes = torch.empty((B, Hkv, T, D // 2), dtype=torch.uint8, device=dev)
+        scales = torch.empty((B, Hkv, T, D // 32), dtype=torch.float16, device=dev)
+        for b in range(B):
+            x = kvgen.kv_torch(wl, kind, (1, Hkv, T, D), dev, layer=0, salt=b)
+            kvq.encode(plans[kind][0], x, codes[b:b + 1], scales[b:b + 1], 0)
+            if kind == "k" and b == 3:
+                k16_b3 = x.clone()
+            if kind == "v" and b == 3:
+                v16_b3 = x.clone()
+        caches[kind] = (codes, scales)
+    q = kvgen.q_torch((B, Hq, D), dev)
+    out = kvq.attend_decode(plans["k"][0], plans["v"][0], q, caches["k"][0], caches["k"][1], caches["v"][0],
+                            caches["v"][1], T_len=T)
+    torch.cuda.synchronize()
+    assert kvq.poll_device_errors() == 0
+    q16 = q.cpu().numpy()
+    for b, kvh in ((0, 0), (3, 5), (15, 7)):
+        sl = slice(kvh, kvh + 1)
+        hq = slice(kvh * 4, kvh * 4 + 4)
+        kc = caches["k"][0][b:b + 1, sl].cpu().numpy()
+        ks = caches["k"][1][b:b + 1, sl].cpu().numpy()
+        vc = caches["v"][0][b:b + 1, sl].cpu().numpy()
+        vs = caches["v"][1][b:b + 1, sl].cpu().numpy()
+        ref = oracle.attend_decode_int4(q16[b:b + 1, hq], kc, ks, vc, vs, plans["k"][1], plans["v"][1], [T])
+        check_rel_l2(out[b:b + 1, hq].cpu().numpy().reshape(-1, D), ref.reshape(-1, D), label=f"b{b} kv{kvh}")
+    # the fp16 comparator on the same shapes (batch entry 3's real K/V; others random)
+    k16 = torch.empty((B, Hkv, T, D), dtype=torch.float16, device=dev)
+    v16 = torch.empty_like(k16)
+    kvgen.kv_torch(wl, "k", (B, Hkv, T, D), dev, layer=1, out=k16)
+    kvgen.kv_torch(wl, "v", (B, Hkv, T, D), dev, layer=1, out=v16)
+    k16[3], v16[3] = k16_b3[0], v16_b3[0]
+    o16 = kvq.attend_decode_ref(q, k16, v16, T_len=T)
+    torch.cuda.synchronize()
+    for kvh in (0, 6):
+        hq = slice(kvh * 4, kvh * 4 + 4)
+        ref = oracle.attend_decode_fp16(q16[3:4, hq], k16[3:4, kvh:kvh + 1].cpu().numpy(),
+                                        v16[3:4, kvh:kvh + 1].cpu().numpy(), [T])
+        check_rel_l2(o16[3:4, hq].cpu().numpy().reshape(-1, D), ref.reshape(-1, D), label=f"fp16 kv{kvh}")
