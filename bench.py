@@ -1,0 +1,400 @@
+#!/usr/bin/env python
+"""Benchmark of the SRFT-int4 KV-cache hot path on B200.
+
+Workload (default): Gemma-3-1B-shaped prefill -- 26 layers, 1 KV head, 4 query
+heads, D=256, batch 1, 4096-token prefix, group 32. One step = encode the full
+K and V cache of every layer (52 jobs x 4096 vectors, one grouped kvq_encode_batch
+launch) and then one 1-token int4 decode attention per layer (26 kvq_attend_decode
+launches on parallel streams). Both phases are replayed as CUDA graphs; inputs
+rotate over three distinct input sets so that every step reads its 109 MB of
+fp16 K/V from HBM, not from the 126 MB L2.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kvq|reference]
+
+Prints one JSON line (rank 0). Under torchrun each rank runs its own copy of the
+workload (weak scaling, no collective on the data path); the timed region is
+bracketed by a barrier and device synchronisation and the max over ranks is used.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import kvgen  # noqa: E402
+
+METRIC = "encode Mvec/s (ns/vec) and int4 decode-attn GB/s, % of B200 HBM roofline"
+WORKLOAD = "gemma"
+N_INPUT_SETS = 3
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def _algo_bytes(D: int, G: int = 32):
+    vec = 2 * D + D // 2 + 2 * (D // G)          # encode: fp16 in + codes + scales out
+    tok = 2 * (D // 2 + 2 * (D // G))            # int4 attention: K and V codes + scales per token x kv head
+    return vec, tok
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling in the background (100 ms period)."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.thread is not None:
+            self.thread.join(timeout=2)
+
+    def summary(self, t0: float, t1: float):
+        rows = []
+        for ts, line in self.lines:
+            if t0 <= ts <= t1:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+def oracle_sample(wl, seed: int, layer: int = 0):
+    """One layer of the step on the host: K and V encode (2 x T vectors) and the
+    1-token int4 decode attention over them, with the fp64 oracle as it stands."""
+    import oracle
+    D, T, G = wl.head_dim, wl.contexts[0], wl.group
+    ks, kl = kvgen.plan_params(D, seed=seed, layer=layer, kind="k")
+    vs, vl = kvgen.plan_params(D, seed=seed, layer=layer, kind="v")
+    k = kvgen.kv_numpy(wl, "k", (1, wl.h_kv, T, D), seed=seed, layer=layer)
+    v = kvgen.kv_numpy(wl, "v", (1, wl.h_kv, T, D), seed=seed, layer=layer)
+    q = kvgen.q_numpy((1, wl.h_q, D), seed=seed, layer=layer)
+    t0 = time.perf_counter()
+    ek = oracle.encode(k, ks, kl, G)
+    ev = oracle.encode(v, vs, vl, G)
+    oracle.attend_decode_int4(q, ek["packed"], ek["scales"], ev["packed"], ev["scales"], (ks, kl), (vs, vl), [T], G)
+    dt = time.perf_counter() - t0
+    return 2 * wl.h_kv * T, dt
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1])
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def cpu_baseline(wl, budget_s: float = 10.0):
+    vecs, secs, n = 0, 0.0, 0
+    while secs < budget_s or n < 1:
+        v, dt = oracle_sample(wl, seed=kvgen.DEFAULT_SEED, layer=n % wl.layers)
+        vecs += v
+        secs += dt
+        n += 1
+    return {"value": vecs / secs / 1e6, "unit": "Mvec/s", "cores": _blas_threads(), "kind": "oracle",
+            "sample": f"{n} x one layer of the step (K+V encode of {2 * wl.h_kv * wl.contexts[0]} vectors, D="
+                      f"{wl.head_dim}, plus the 1-token int4 attention over {wl.contexts[0]} tokens), "
+                      f"{secs:.1f} s of host time"}
+
+
+# ---------------------------------------------------------------- reference arm
+def run_reference(args, rank: int, world: int):
+    if rank != 0:
+        return 0
+    wl = kvgen.WORKLOADS[WORKLOAD]
+    for _ in range(args.warmup):
+        oracle_sample(wl, seed=kvgen.DEFAULT_SEED)
+    vecs, secs = 0, 0.0
+    for s in range(args.steps):
+        v, dt = oracle_sample(wl, seed=kvgen.DEFAULT_SEED, layer=s % wl.layers)
+        vecs += v
+        secs += dt
+    val = vecs / secs / 1e6
+    sample = (f"each step = one layer of the workload on the host (K+V encode of {2 * wl.h_kv * wl.contexts[0]} "
+              f"vectors + 1-token int4 attention over {wl.contexts[0]} tokens)")
+    line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "Mvec/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(1, args.steps),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": _config(wl),
+            "cpu_baseline": {"value": val, "unit": "Mvec/s", "cores": _blas_threads(), "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": val, "unit": "Mvec/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(wl):
+    return {"workload": "gemma3-1b-prefill: encode K+V of 26 layers x 4096 tokens, then 1-token int4 decode "
+                        "attention per layer",
+            "layers": wl.layers, "kv_heads": wl.h_kv, "q_heads": wl.h_q, "head_dim": wl.head_dim,
+            "batch": wl.batch, "prefix": wl.contexts[0], "group": wl.group,
+            "l2": f"inputs rotate over {N_INPUT_SETS} distinct input sets (3 x 109 MB) so each step reads HBM"}
+
+
+# ---------------------------------------------------------------- kvq arm
+def run_kvq(args, rank: int, world: int):
+    import torch
+
+    import rotated_int4_kv_b200 as kvq
+
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = kvgen.WORKLOADS[WORKLOAD]
+    L, Hkv, Hq, D, T, G = wl.layers, wl.h_kv, wl.h_q, wl.head_dim, wl.contexts[0], wl.group
+    seed = kvgen.DEFAULT_SEED + 1000 * rank
+    NJ = 2 * L
+    vec_b, tok_b = _algo_bytes(D, G)
+
+    # plans (per layer and K/V), inputs, caches
+    plans = []
+    for l in range(L):
+        for kind in ("k", "v"):
+            s, lam = kvgen.plan_params(D, seed=seed, layer=l, kind=kind)
+            plans.append(kvq.Plan(s, lam, group=G))
+    X = []
+    for i in range(N_INPUT_SETS):
+        x = torch.empty((NJ, Hkv, T, D), dtype=torch.float16, device=dev)
+        for j in range(NJ):
+            kvgen.kv_torch(wl, "kv"[j % 2], (1, Hkv, T, D), dev, seed=seed, layer=j // 2, salt=i, out=x[j:j + 1])
+        X.append(x)
+    codes = torch.empty((NJ, Hkv, T, D // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty((NJ, Hkv, T, D // G), dtype=torch.float16, device=dev)
+    q = torch.stack([kvgen.q_torch((1, Hq, D), dev, seed=seed, layer=l) for l in range(L)])  # [L, 1, Hq, D]
+    out = torch.empty((L, 1, Hq, D), dtype=torch.float16, device=dev)
+    ws = [kvq.make_workspace(1, Hq, Hkv, D, T, dev) for _ in range(L)]
+
+    def jobs_for(i):
+        return [(plans[j], X[i][j:j + 1], codes[j:j + 1], scales[j:j + 1], 0) for j in range(NJ)]
+
+    def attn(l, stream=None):
+        kvq.attend_decode(plans[2 * l], plans[2 * l + 1], q[l], codes[2 * l:2 * l + 1], scales[2 * l:2 * l + 1],
+                          codes[2 * l + 1:2 * l + 2], scales[2 * l + 1:2 * l + 2], T_len=T, out=out[l],
+                          workspace=ws[l], stream=stream)
+
+    n_side = 8
+    side = [torch.cuda.Stream(device=dev) for _ in range(n_side)]
+
+    def attn_phase():
+        main = torch.cuda.current_stream()
+        ev = torch.cuda.Event()
+        ev.record(main)
+        for s in side:
+            s.wait_event(ev)
+        for l in range(L):
+            attn(l, side[l % n_side])
+        for s in side:
+            e = torch.cuda.Event()
+            e.record(s)
+            main.wait_event(e)
+
+    # eager run first (one-time kernel attribute setup happens outside capture)
+    kvq.encode_batch(jobs_for(0))
+    attn_phase()
+    torch.cuda.synchronize()
+    assert kvq.poll_device_errors() == 0
+
+    g_enc, g_att = [], []
+    cap_stream = torch.cuda.Stream(device=dev)
+    for i in range(N_INPUT_SETS):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=cap_stream):
+            kvq.encode_batch(jobs_for(i))
+        g_enc.append(g)
+    ga = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(ga, stream=cap_stream):
+        attn_phase()
+    g_att.append(ga)
+    torch.cuda.synchronize()
+
+    def step(i, ev_a=None, ev_b=None):
+        if ev_a is not None:
+            ev_a.record()
+        g_enc[i % N_INPUT_SETS].replay()
+        if ev_b is not None:
+            ev_b.record()
+        g_att[0].replay()
+
+    clk = ClockSampler(local)
+    clk.start()
+    # soak so the clocks reach their loaded steady state before warm-up and timing
+    t_soak = time.time()
+    i = 0
+    while time.time() - t_soak < 1.5:
+        step(i)
+        i += 1
+        if i % 64 == 0:
+            torch.cuda.synchronize()
+    for w in range(args.warmup):
+        step(w)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    ev_a = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev_b = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    wall0 = time.time()
+    t_start.record()
+    for s in range(args.steps):
+        step(s, ev_a[s], ev_b[s])
+    t_end.record()
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    wall1 = time.time()
+    clk.stop()
+    ms = t_start.elapsed_time(t_end)
+    enc_ms = [a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]
+    att_ms = [ev_b[s].elapsed_time(ev_a[s + 1]) for s in range(args.steps - 1)] + [ev_b[-1].elapsed_time(t_end)]
+    if dist is not None:
+        t = torch.tensor([ms, float(np.mean(enc_ms)), float(np.mean(att_ms))], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, enc_avg, att_avg = (float(v) for v in t.tolist())
+    else:
+        enc_avg, att_avg = float(np.mean(enc_ms)), float(np.mean(att_ms))
+    assert kvq.poll_device_errors() == 0
+
+    # ---- end to end through the C ABI with host buffers (pinned), copies in the timed region
+    e2e_steps = max(3, min(args.steps, 10))
+    x_host = [torch.empty(X[0].shape, dtype=torch.float16, pin_memory=True) for _ in range(2)]
+    for hbuf in x_host:
+        hbuf.copy_(X[0])
+    q_host = q.cpu().pin_memory()
+    out_host = torch.empty(out.shape, dtype=torch.float16, pin_memory=True)
+    x_dev = X[0]
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(e2e_steps):
+        x_dev.copy_(x_host[s % 2], non_blocking=True)
+        q.copy_(q_host, non_blocking=True)
+        kvq.encode_batch(jobs_for(0))
+        attn_phase()
+        out_host.copy_(out, non_blocking=True)
+    e1.record()
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    h2d = x_dev.numel() * 2 + q.numel() * 2
+    d2h = out.numel() * 2
+
+    vec_step = NJ * Hkv * T
+    value = world * vec_step / (ms / args.steps * 1e-3) / 1e6
+    hbm, peak_kind = _peaks()
+    enc_gbs = vec_step * vec_b / (enc_avg * 1e-3) / 1e9
+    att_bytes = L * Hkv * T * tok_b
+    att_gbs = att_bytes / (att_avg * 1e-3) / 1e9
+    clocks = clk.summary(wall0 - 1.0, wall1 + 0.2)
+    res = None
+    if rank == 0:
+        cpu = cpu_baseline(wl) if world == 1 else None
+        res = {
+            "metric": METRIC, "value": value, "unit": "Mvec/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _config(wl),
+            "encode": {"kernel_us": 1e3 * enc_avg, "ns_per_vec": 1e6 * enc_avg / vec_step,
+                       "Mvec_s": vec_step / (enc_avg * 1e-3) / 1e6, "GB_s": enc_gbs,
+                       "frac_hbm": enc_gbs / hbm, "frac_hbm_8TBs_nominal": enc_gbs / 8000.0,
+                       "bytes_per_vec": vec_b},
+            "attention": {"phase_us": 1e3 * att_avg, "us_per_layer": 1e3 * att_avg / L,
+                          "tokens_heads_per_s": L * Hkv * T / (att_avg * 1e-3), "GB_s": att_gbs,
+                          "frac_hbm": att_gbs / hbm, "bytes_per_token_head": tok_b},
+            "roofline": {"bound": "hbm", "achieved": enc_gbs, "peak": hbm, "unit": "GB/s",
+                         "frac": enc_gbs / hbm, "traffic": None, "kernel": "encode_kernel<256,32,64>",
+                         "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs, burst copy)"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * vec_step / (e2e_ms * 1e-3) / 1e6, "unit": "Mvec/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": args.steps * (1 + L),
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],
+                       "samples": clocks["samples"]},
+        }
+    for g in g_enc + g_att:
+        g.reset()
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+    if res is not None:
+        print(json.dumps(res), flush=True)
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    return run_kvq(args, rank, world)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -103,6 +103,26 @@ kvq_status kvq_encode(const kvq_plan* plan, const uint16_t* x, int B, int H, int
                       uint16_t* scales, int T_cap, int pos, void* stream);
 
 /*
+ * kvq_encode_batch -- the same encode for many independent (plan, x, cache) jobs in
+ * one grouped launch, e.g. K and V of every layer of a prefill (each with its own
+ * s and lambda). Each job is exactly one kvq_encode call; jobs are processed in
+ * any order and must not write overlapping cache rows.
+ *   jobs    host array of njobs descriptors (read during the call only). All jobs
+ *           with work must use plans of one head_dim, group and device. Jobs with
+ *           B, H or n == 0 are skipped. Up to 64 jobs share one kernel launch.
+ * Errors: as kvq_encode, reported for the first offending job; nothing is launched.
+ */
+typedef struct kvq_encode_job {
+  const kvq_plan* plan;
+  const uint16_t* x;   /* fp16 [B, H, n, D] */
+  uint8_t* codes;      /* u8   [B, H, T_cap, D/2] */
+  uint16_t* scales;    /* fp16 [B, H, T_cap, D/G] */
+  int B, H, n, T_cap, pos;
+} kvq_encode_job;
+
+kvq_status kvq_encode_batch(const kvq_encode_job* jobs, int njobs, void* stream);
+
+/*
  * kvq_decode -- the inverse: x_hat = diag(s) . F_r^T . (c * scale / lambda), rounded
  * to fp16, for cache rows t0 .. t0+n-1 of every (b, h).
  *   out  fp16 [B, H, n, D] contiguous.

@@ -18,6 +18,13 @@ class KvqError(RuntimeError):
         super().__init__(f"{where}: {STATUS_NAMES.get(status, status)} ({detail})")
 
 
+class EncodeJob(ctypes.Structure):
+    """Mirror of ``kvq_encode_job`` in include/kvq.h."""
+    _fields_ = [("plan", ctypes.c_void_p), ("x", ctypes.c_void_p), ("codes", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("B", ctypes.c_int), ("H", ctypes.c_int), ("n", ctypes.c_int),
+                ("T_cap", ctypes.c_int), ("pos", ctypes.c_int)]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(f"{LIB_PATH} is missing: build it with `python -m rotated_int4_kv_b200.build` "
@@ -30,6 +37,7 @@ def _load() -> ctypes.CDLL:
         "kvq_plan_head_dim": (I, [P]),
         "kvq_plan_group": (I, [P]),
         "kvq_encode": (I, [P, P, I, I, I, P, P, I, I, P]),
+        "kvq_encode_batch": (I, [ctypes.POINTER(EncodeJob), I, P]),
         "kvq_decode": (I, [P, P, P, I, I, I, I, I, P, P]),
         "kvq_workspace_size": (S, [I, I, I, I, I]),
         "kvq_attend_decode": (I, [P, P, P, P, P, P, P, I, I, I, I, P, I, F, P, P, S, P]),

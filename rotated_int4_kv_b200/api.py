@@ -10,7 +10,7 @@ import ctypes
 import numpy as np
 import torch
 
-from ._lib import check, lib
+from ._lib import EncodeJob, check, lib
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -77,6 +77,21 @@ def encode(plan: Plan, x: torch.Tensor, codes: torch.Tensor, scales: torch.Tenso
     _need(scales, "scales", torch.float16, (B, H, T_cap, D // plan.group))
     check(lib.kvq_encode(plan.handle, _ptr(x), B, H, n, _ptr(codes), _ptr(scales), T_cap, int(pos),
                          _stream(stream)), "kvq_encode")
+
+
+def encode_batch(jobs, stream=None) -> None:
+    """Grouped encode: ``jobs`` is a sequence of (plan, x, codes, scales, pos) tuples,
+    each exactly what :func:`encode` takes; all run in one launch (up to 64 per launch)."""
+    arr = (EncodeJob * max(1, len(jobs)))()
+    for i, (plan, x, codes, scales, pos) in enumerate(jobs):
+        B, H, n, D = x.shape
+        T_cap = codes.shape[2]
+        _need(x, f"jobs[{i}].x", torch.float16)
+        _need(codes, f"jobs[{i}].codes", torch.uint8, (B, H, T_cap, D // 2))
+        _need(scales, f"jobs[{i}].scales", torch.float16, (B, H, T_cap, D // plan.group))
+        arr[i] = EncodeJob(plan.handle.value, x.data_ptr(), codes.data_ptr(), scales.data_ptr(), B, H, n, T_cap,
+                           int(pos))
+    check(lib.kvq_encode_batch(arr, len(jobs), _stream(stream)), "kvq_encode_batch")
 
 
 def decode(plan: Plan, codes: torch.Tensor, scales: torch.Tensor, t0: int, n: int, out: torch.Tensor = None,

@@ -5,6 +5,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <unordered_map>
 #include <vector>
 
 #include "kvq_internal.h"
@@ -95,9 +96,47 @@ kvq_status fail(kvq_status st, const std::string& msg) {
   return st;
 }
 
+namespace {
+// Small cache of encoded tensor maps: repeated calls on the same buffers (the
+// usual decode loop) skip the driver call. Keyed by every encoding input.
+struct MapKey {
+  uint64_t w[20];
+  bool operator==(const MapKey& o) const { return std::memcmp(w, o.w, sizeof(w)) == 0; }
+};
+struct MapKeyHash {
+  size_t operator()(const MapKey& k) const {
+    uint64_t h = 1469598103934665603ull;
+    for (uint64_t v : k.w) h = (h ^ v) * 1099511628211ull;
+    return (size_t)h;
+  }
+};
+std::mutex g_map_mu;
+std::unordered_map<MapKey, CUtensorMap, MapKeyHash> g_maps;
+constexpr size_t kMaxCachedMaps = 8192;
+}  // namespace
+
 kvq_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
                         const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle swz,
                         const char* what) {
+  MapKey key{};
+  key.w[0] = (uint64_t)dt | ((uint64_t)rank << 8) | ((uint64_t)swz << 16);
+  key.w[1] = reinterpret_cast<uint64_t>(base);
+  for (int i = 0; i < rank && i < 5; ++i) {
+    key.w[2 + i] = dims[i];
+    key.w[7 + i] = box[i];
+  }
+  for (int i = 0; i + 1 < rank && i < 4; ++i) key.w[12 + i] = strides_bytes[i];
+  int dev = -1;
+  cudaGetDevice(&dev);
+  key.w[16] = (uint64_t)(int64_t)dev;
+  {
+    std::lock_guard<std::mutex> lk(g_map_mu);
+    auto it = g_maps.find(key);
+    if (it != g_maps.end()) {
+      *map = it->second;
+      return KVQ_OK;
+    }
+  }
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return fail(KVQ_ERR_CUDA, "cuTensorMapEncodeTiled not available from the driver");
   cuuint64_t d[5];
@@ -113,6 +152,9 @@ kvq_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dt, int rank, cons
                         CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(KVQ_ERR_CUDA, std::string("tensor map for ") + what + " rejected by the driver");
+  std::lock_guard<std::mutex> lk(g_map_mu);
+  if (g_maps.size() >= kMaxCachedMaps) g_maps.clear();
+  g_maps.emplace(key, *map);
   return KVQ_OK;
 }
 
@@ -199,12 +241,13 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
   kvq::build_frag(RT, D, fo);
   const size_t bytes = fq.size() * 4;
   void* blk = nullptr;
-  if (cudaMalloc(&blk, 2 * bytes) != cudaSuccess) {
+  if (cudaMalloc(&blk, 2 * bytes + sizeof(kvq::CodecConsts)) != cudaSuccess) {
     delete p;
     return fail(KVQ_ERR_CUDA, "plan_create: cudaMalloc failed");
   }
   if (cudaMemcpy(blk, fq.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
-      cudaMemcpy((char*)blk + bytes, fo.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess) {
+      cudaMemcpy((char*)blk + bytes, fo.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy((char*)blk + 2 * bytes, &p->enc, sizeof(kvq::CodecConsts), cudaMemcpyHostToDevice) != cudaSuccess) {
     cudaFree(blk);
     delete p;
     return fail(KVQ_ERR_CUDA, "plan_create: upload failed");
@@ -212,6 +255,7 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
   p->dblock = blk;
   p->rq_frag = reinterpret_cast<const uint4*>(blk);
   p->ro_frag = reinterpret_cast<const uint4*>((char*)blk + bytes);
+  p->enc_dev = reinterpret_cast<const kvq::CodecConsts*>((char*)blk + 2 * bytes);
   *out = p;
   return KVQ_OK;
 }
@@ -244,7 +288,37 @@ kvq_status kvq_encode(const kvq_plan* p, const uint16_t* x, int B, int H, int n,
   if ((long)B * H > (1L << 30) || (long)T_cap * B * H > (1L << 40)) return fail(KVQ_ERR_INVALID_ARG, "encode: too large");
   kvq_status st = kvq::check_plan_device(p);
   if (st != KVQ_OK) return st;
-  return kvq::launch_encode(p, x, B, H, n, codes, scales, T_cap, pos, (cudaStream_t)stream);
+  kvq_encode_job job{p, x, codes, scales, B, H, n, T_cap, pos};
+  return kvq::launch_encode_jobs(&job, 1, (cudaStream_t)stream);
+}
+
+kvq_status kvq_encode_batch(const kvq_encode_job* jobs, int njobs, void* stream) {
+  if (njobs < 0 || (njobs > 0 && !jobs)) return fail(KVQ_ERR_INVALID_ARG, "encode_batch: bad job array");
+  std::vector<kvq_encode_job> live;
+  live.reserve(njobs);
+  const kvq_plan* p0 = nullptr;
+  for (int i = 0; i < njobs; ++i) {
+    const kvq_encode_job& j = jobs[i];
+    const std::string w = "encode_batch job " + std::to_string(i) + ": ";
+    if (!j.plan) return fail(KVQ_ERR_INVALID_ARG, w + "null plan");
+    if (j.B < 0 || j.H < 0 || j.n < 0 || j.T_cap < 0 || j.pos < 0) return fail(KVQ_ERR_INVALID_ARG, w + "negative size");
+    if ((long)j.pos + j.n > j.T_cap) return fail(KVQ_ERR_CAPACITY, w + "pos + n > T_cap");
+    if (j.B == 0 || j.H == 0 || j.n == 0) continue;
+    if (!j.x || !j.codes || !j.scales) return fail(KVQ_ERR_INVALID_ARG, w + "null buffer");
+    if (!kvq::aligned16(j.x) || !kvq::aligned16(j.codes) || !kvq::aligned16(j.scales))
+      return fail(KVQ_ERR_ALIGNMENT, w + "buffers must be 16-byte aligned");
+    if ((long)j.B * j.H > (1L << 30) || (long)j.T_cap * j.B * j.H > (1L << 40)) return fail(KVQ_ERR_INVALID_ARG, w + "too large");
+    if (!p0) {
+      p0 = j.plan;
+      kvq_status st = kvq::check_plan_device(p0);
+      if (st != KVQ_OK) return st;
+    } else if (j.plan->D != p0->D || j.plan->G != p0->G || j.plan->device != p0->device) {
+      return fail(KVQ_ERR_INVALID_ARG, w + "all jobs must share head_dim, group and device");
+    }
+    live.push_back(j);
+  }
+  if (live.empty()) return KVQ_OK;
+  return kvq::launch_encode_jobs(live.data(), (int)live.size(), (cudaStream_t)stream);
 }
 
 kvq_status kvq_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* scales, int B, int H, int T_cap,

@@ -19,7 +19,9 @@
 //     8- or 16-byte store per vector.
 // Decode is the exact transpose: TMA-load the code rows, unpack, scale by
 // scale * dg / lambda, inverse real FFT (transpose graph), sign, fp16, TMA store.
+#include <algorithm>
 #include <cstdio>
+#include <cstring>
 #include <mutex>
 
 #include "kvq_internal.h"
@@ -59,15 +61,40 @@ struct SmemLayout {
   static constexpr int kXStage = kNT * D * 2;        // fp16 x tile (D/64 swizzled boxes)
   static constexpr int kCTile = kNT * D / 2;         // packed code tile
   static constexpr int kStages = D == 128 ? 2 : 1;
-  static constexpr int kBytes = kStages * kXStage + kCTile + 64 + 1024;
+  static constexpr int kBytes = kStages * kXStage + kCTile + D * 4 + D * 2 + 64 + 1024;
 };
 
 // ---------------------------------------------------------------- encode
-template <int D, int G>
-__global__ void __launch_bounds__(kNT, kMinBlocks<D>) encode_kernel(const __grid_constant__ CUtensorMap xmap,
-                                                     const __grid_constant__ CUtensorMap cmap,
-                                                     const __grid_constant__ CodecConsts cc, TileGeom geom,
-                                                     uint16_t* __restrict__ scales, int T_cap, int pos) {
+// One launch walks the tiles of up to MAXJ independent jobs (kvq_encode = 1 job,
+// kvq_encode_batch = a grouped launch). A job's tensor maps live in the kernel
+// parameter block; its lambda/sign constants are staged in shared memory when a
+// CTA moves to a tile of another job.
+struct alignas(64) EncJob {
+  CUtensorMap xmap;           // x [BH, n, D] fp16, box {64, T_box, BH_box}, 128B swizzle
+  CUtensorMap cmap;           // codes [BH, pos+n, D/2] u8 (rows pos.. of the cache), box {D/2, T_box, BH_box}
+  const CodecConsts* cc;      // device: lambda*dg per channel, sign masks
+  uint16_t* scales;
+  int T_cap, pos, BH, n, T_box, BH_box, t_shift, n_ttiles, tile0;
+};
+
+template <int MAXJ>
+struct EncBatch {
+  EncJob jobs[MAXJ];
+  int njobs;
+  int total_tiles;
+};
+
+template <int MAXJ>
+__device__ __forceinline__ int job_of(const EncBatch<MAXJ>& P, int tile) {
+  int j = 0;
+  if constexpr (MAXJ > 1) {
+    while (j + 1 < P.njobs && tile >= P.jobs[j + 1].tile0) ++j;
+  }
+  return j;
+}
+
+template <int D, int G, int MAXJ>
+__global__ void __launch_bounds__(kNT, kMinBlocks<D>) encode_kernel(const __grid_constant__ EncBatch<MAXJ> P) {
   using L = SmemLayout<D>;
   constexpr int kBoxes = D / 64;
   constexpr int kBoxBytes = kNT * 128;
@@ -77,45 +104,61 @@ __global__ void __launch_bounds__(kNT, kMinBlocks<D>) encode_kernel(const __grid
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xs = smem;
   uint8_t* cs = smem + L::kStages * L::kXStage;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(cs + L::kCTile);
+  float* cchan = reinterpret_cast<float*>(cs + L::kCTile);          // [D]
+  uint32_t* csgn = reinterpret_cast<uint32_t*>(cchan + D);           // [D/2]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(csgn + D / 2);
 
   const int tid = threadIdx.x;
   const int first = blockIdx.x;
   const int stride = gridDim.x;
-  if (first >= geom.n_tiles) return;
+  if (first >= P.total_tiles) return;
 
   if (tid == 0) {
-    prefetch_tensormap(&xmap);
-    prefetch_tensormap(&cmap);
     for (int s = 0; s < L::kStages; ++s) mbar_init(&bar[s], 1);
     fence_mbarrier_init();
   }
   __syncthreads();
 
   auto issue = [&](int tile, int stage) {
-    int bh0, t0;
-    tile_origin(geom, tile, bh0, t0);
+    const EncJob& J = P.jobs[job_of(P, tile)];
+    const int lt = tile - J.tile0;
+    const int tb = lt / J.n_ttiles;
+    const int bh0 = tb * J.BH_box, t0 = (lt - tb * J.n_ttiles) * J.T_box;
     mbar_arrive_expect_tx(&bar[stage], L::kXStage);
 #pragma unroll
     for (int b = 0; b < kBoxes; ++b)
-      tma_load_3d(xs + stage * L::kXStage + b * kBoxBytes, &xmap, &bar[stage], b * 64, t0, bh0);
+      tma_load_3d(xs + stage * L::kXStage + b * kBoxBytes, &J.xmap, &bar[stage], b * 64, t0, bh0);
   };
   if (tid == 0) {
     for (int s = 0; s < L::kStages; ++s) {
       const int tile = first + s * stride;
-      if (tile < geom.n_tiles) issue(tile, s);
+      if (tile < P.total_tiles) issue(tile, s);
     }
   }
 
-  const int t_l = tid & (geom.T_box - 1);
-  const int bh_l = tid >> geom.t_shift;
+  int cur_job = -1;
   int it = 0;
-  for (int tile = first; tile < geom.n_tiles; tile += stride, ++it) {
+  for (int tile = first; tile < P.total_tiles; tile += stride, ++it) {
+    const int j = job_of(P, tile);
+    const EncJob& J = P.jobs[j];
+    if (j != cur_job) {  // CTA-uniform: stage this job's constants (previous readers finished before the last sync)
+      const float* src = J.cc->chan;
+      for (int i = tid; i < D; i += kNT) cchan[i] = src[i];
+      for (int i = tid; i < D / 2; i += kNT) csgn[i] = J.cc->sgn[i];
+      cur_job = j;
+      __syncthreads();
+    }
+    const int lt = tile - J.tile0;
+    const int tb = lt / J.n_ttiles;
+    const int bh0 = tb * J.BH_box, t0 = (lt - tb * J.n_ttiles) * J.T_box;
+    const int t_l = tid & (J.T_box - 1);
+    const int bh_l = tid >> J.t_shift;
+
     const int stage = it % L::kStages;
     const uint32_t parity = (it / L::kStages) & 1;
     if (!mbar_wait_bounded(&bar[stage], parity)) {
       atomicOr(&g_codec_err, kErrTimeoutLoad);
-      return;  // nothing else of ours is in flight on this barrier's stage only
+      return;
     }
     // ---- load own row (swizzled 128B boxes), apply signs, convert
     float v[D];
@@ -127,12 +170,12 @@ __global__ void __launch_bounds__(kNT, kMinBlocks<D>) encode_kernel(const __grid
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
           const uint4 w = *reinterpret_cast<const uint4*>(base + b * kBoxBytes + ((c ^ sw) << 4));
+          const uint4 m = *reinterpret_cast<const uint4*>(csgn + (b * 64 + c * 8) / 2);
           const int e0 = b * 64 + c * 8;
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+          const uint32_t ww[4] = {w.x ^ m.x, w.y ^ m.y, w.z ^ m.z, w.w ^ m.w};
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            uint32_t h2 = ww[q] ^ cc.sgn[e0 / 2 + q];
-            const float2 f = __half22float2(*reinterpret_cast<__half2*>(&h2));
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ww[q]));
             v[e0 + 2 * q] = f.x;
             v[e0 + 2 * q + 1] = f.y;
           }
@@ -142,7 +185,7 @@ __global__ void __launch_bounds__(kNT, kMinBlocks<D>) encode_kernel(const __grid
     __syncthreads();  // every thread has its row: the stage may be refilled
     if (tid == 0) {
       const int nxt = tile + L::kStages * stride;
-      if (nxt < geom.n_tiles) issue(nxt, stage);
+      if (nxt < P.total_tiles) issue(nxt, stage);
     }
 
     // ---- transform
@@ -156,10 +199,15 @@ __global__ void __launch_bounds__(kNT, kMinBlocks<D>) encode_kernel(const __grid
       float y[G];
       float a = 0.0f;
 #pragma unroll
-      for (int i = 0; i < G; ++i) {
-        const int c = g * G + i;
-        y[i] = v[slot_of_channel(c, D)] * cc.chan[c];
-        a = fmaxf(a, fabsf(y[i]));
+      for (int i4 = 0; i4 < G / 4; ++i4) {
+        const float4 l4 = *reinterpret_cast<const float4*>(cchan + g * G + 4 * i4);
+        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int i = 4 * i4 + e;
+          y[i] = v[slot_of_channel(g * G + i, D)] * lv[e];
+          a = fmaxf(a, fabsf(y[i]));
+        }
       }
       const float sf = fminf(__fdiv_rn(a, 7.0f), 65504.0f);
       const __half hs = __float2half_rn(sf);
@@ -188,12 +236,10 @@ __global__ void __launch_bounds__(kNT, kMinBlocks<D>) encode_kernel(const __grid
     }
 
     // ---- outputs
-    int bh0, t0;
-    tile_origin(geom, tile, bh0, t0);
     const int t = t0 + t_l, bh = bh0 + bh_l;
-    const bool valid = (t < geom.n) && (bh < geom.BH);
+    const bool valid = (t < J.n) && (bh < J.BH);
     if (valid) {
-      uint16_t* sp = scales + ((size_t)bh * T_cap + pos + t) * kNG;
+      uint16_t* sp = J.scales + ((size_t)bh * J.T_cap + J.pos + t) * kNG;
       if constexpr (kNG == 4) {
         *reinterpret_cast<uint2*>(sp) = make_uint2(sbits[0] | (sbits[1] << 16), sbits[2] | (sbits[3] << 16));
       } else {
@@ -219,7 +265,7 @@ __global__ void __launch_bounds__(kNT, kMinBlocks<D>) encode_kernel(const __grid
     fence_proxy_async_smem();
     __syncthreads();
     if (tid == 0) {
-      tma_store_3d(&cmap, cs, 0, pos + t0, bh0);
+      tma_store_3d(&J.cmap, cs, 0, J.pos + t0, bh0);
       bulk_commit_group();
     }
   }
@@ -402,39 +448,73 @@ int occupancy_blocks(K kernel, int smem_bytes) {
   return nb;
 }
 
-template <int D, int G>
-kvq_status run_encode(const kvq_plan* p, const uint16_t* x, int B, int H, int n, uint8_t* codes, uint16_t* scales,
-                      int T_cap, int pos, cudaStream_t s) {
-  const int BH = B * H;
-  TileGeom geom = make_geom(BH, n);
-  CUtensorMap xmap, cmap;
-  {
-    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)n, (uint64_t)BH};
-    const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)D * 2 * n};
-    const uint32_t box[3] = {64u, (uint32_t)geom.T_box, (uint32_t)geom.BH_box};
-    kvq_status st = encode_tiled(&xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, x, dims, strides, box,
-                                 CU_TENSOR_MAP_SWIZZLE_128B, "encode input");
-    if (st != KVQ_OK) return st;
+template <int D, int G, int MAXJ>
+kvq_status run_encode_chunk(const kvq_encode_job* jobs, int nj, cudaStream_t s) {
+  EncBatch<MAXJ> P;
+  memset(&P, 0, sizeof(P));
+  int tiles = 0;
+  for (int i = 0; i < nj; ++i) {
+    const kvq_encode_job& q = jobs[i];
+    EncJob& J = P.jobs[i];
+    const int BH = q.B * q.H;
+    TileGeom geom = make_geom(BH, q.n);
+    {
+      const uint64_t dims[3] = {(uint64_t)D, (uint64_t)q.n, (uint64_t)BH};
+      const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)D * 2 * q.n};
+      const uint32_t box[3] = {64u, (uint32_t)geom.T_box, (uint32_t)geom.BH_box};
+      kvq_status st = encode_tiled(&J.xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 3, q.x, dims, strides, box,
+                                   CU_TENSOR_MAP_SWIZZLE_128B, "encode input");
+      if (st != KVQ_OK) return st;
+    }
+    {
+      const uint64_t dims[3] = {(uint64_t)D / 2, (uint64_t)(q.pos + q.n), (uint64_t)BH};
+      const uint64_t strides[2] = {(uint64_t)D / 2, (uint64_t)(D / 2) * q.T_cap};
+      const uint32_t box[3] = {(uint32_t)D / 2, (uint32_t)geom.T_box, (uint32_t)geom.BH_box};
+      kvq_status st = encode_tiled(&J.cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q.codes, dims, strides, box,
+                                   D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, "code cache");
+      if (st != KVQ_OK) return st;
+    }
+    J.cc = q.plan->enc_dev;
+    J.scales = q.scales;
+    J.T_cap = q.T_cap;
+    J.pos = q.pos;
+    J.BH = BH;
+    J.n = q.n;
+    J.T_box = geom.T_box;
+    J.BH_box = geom.BH_box;
+    J.t_shift = geom.t_shift;
+    J.n_ttiles = geom.n_ttiles;
+    J.tile0 = tiles;
+    tiles += geom.n_tiles;
   }
-  {
-    const uint64_t dims[3] = {(uint64_t)D / 2, (uint64_t)(pos + n), (uint64_t)BH};
-    const uint64_t strides[2] = {(uint64_t)D / 2, (uint64_t)(D / 2) * T_cap};
-    const uint32_t box[3] = {(uint32_t)D / 2, (uint32_t)geom.T_box, (uint32_t)geom.BH_box};
-    kvq_status st = encode_tiled(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, codes, dims, strides, box,
-                                 D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, "code cache");
-    if (st != KVQ_OK) return st;
-  }
+  P.njobs = nj;
+  P.total_tiles = tiles;
   constexpr int smem = SmemLayout<D>::kBytes;
   static int blocks_per_sm = -1;
   static std::once_flag once;
   std::call_once(once, [&] {
-    cudaFuncSetAttribute(encode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    blocks_per_sm = occupancy_blocks(encode_kernel<D, G>, smem);
+    cudaFuncSetAttribute(encode_kernel<D, G, MAXJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    blocks_per_sm = occupancy_blocks(encode_kernel<D, G, MAXJ>, smem);
   });
-  const int grid = std::min(geom.n_tiles, blocks_per_sm * num_sms(p->device));
-  encode_kernel<D, G><<<grid, kNT, smem, s>>>(xmap, cmap, p->enc, geom, scales, T_cap, pos);
+  int dev = 0;
+  cudaGetDevice(&dev);
+  const int grid = std::min(tiles, blocks_per_sm * num_sms(dev));
+  encode_kernel<D, G, MAXJ><<<grid, kNT, smem, s>>>(P);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("encode launch: ") + cudaGetErrorString(e));
+  return KVQ_OK;
+}
+
+constexpr int kMaxJobs = 64;
+
+template <int D, int G>
+kvq_status run_encode(const kvq_encode_job* jobs, int njobs, cudaStream_t s) {
+  if (njobs == 1) return run_encode_chunk<D, G, 1>(jobs, 1, s);
+  for (int i = 0; i < njobs; i += kMaxJobs) {
+    const int nj = std::min(kMaxJobs, njobs - i);
+    kvq_status st = run_encode_chunk<D, G, kMaxJobs>(jobs + i, nj, s);
+    if (st != KVQ_OK) return st;
+  }
   return KVQ_OK;
 }
 
@@ -476,12 +556,12 @@ kvq_status run_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* s
 
 }  // namespace
 
-kvq_status launch_encode(const kvq_plan* p, const uint16_t* x, int B, int H, int n, uint8_t* codes,
-                         uint16_t* scales, int T_cap, int pos, cudaStream_t s) {
-  if (p->D == 128 && p->G == 32) return run_encode<128, 32>(p, x, B, H, n, codes, scales, T_cap, pos, s);
-  if (p->D == 256 && p->G == 32) return run_encode<256, 32>(p, x, B, H, n, codes, scales, T_cap, pos, s);
-  if (p->D == 128 && p->G == 16) return run_encode<128, 16>(p, x, B, H, n, codes, scales, T_cap, pos, s);
-  if (p->D == 256 && p->G == 16) return run_encode<256, 16>(p, x, B, H, n, codes, scales, T_cap, pos, s);
+kvq_status launch_encode_jobs(const kvq_encode_job* jobs, int njobs, cudaStream_t s) {
+  const int D = jobs[0].plan->D, G = jobs[0].plan->G;
+  if (D == 128 && G == 32) return run_encode<128, 32>(jobs, njobs, s);
+  if (D == 256 && G == 32) return run_encode<256, 32>(jobs, njobs, s);
+  if (D == 128 && G == 16) return run_encode<128, 16>(jobs, njobs, s);
+  if (D == 256 && G == 16) return run_encode<256, 16>(jobs, njobs, s);
   return fail(KVQ_ERR_UNSUPPORTED, "encode: unsupported (head_dim, group)");
 }
 

@@ -36,6 +36,7 @@ struct kvq_plan {
   void* dblock = nullptr;
   const uint4* rq_frag = nullptr;   // [D/16 m-tiles][D/16 k-tiles][2 hi/lo][32 lanes] uint4
   const uint4* ro_frag = nullptr;   // same layout for R'^T
+  const kvq::CodecConsts* enc_dev = nullptr;  // device copy of `enc` (read by the encode kernel)
 };
 
 namespace kvq {
@@ -54,8 +55,7 @@ int num_sms(int device);
 kvq_status check_plan_device(const kvq_plan* p);
 
 // codec launchers (kvq_codec.cu)
-kvq_status launch_encode(const kvq_plan* p, const uint16_t* x, int B, int H, int n, uint8_t* codes,
-                         uint16_t* scales, int T_cap, int pos, cudaStream_t s);
+kvq_status launch_encode_jobs(const kvq_encode_job* jobs, int njobs, cudaStream_t s);
 kvq_status launch_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* scales, int B, int H,
                          int T_cap, int t0, int n, uint16_t* out, cudaStream_t s);
 

@@ -50,7 +50,7 @@ CASES = [
     ("longctx", 1, 2, 16, 300, None),          # GQA 8
     ("longctx", 1, 1, 16, 200, [77]),           # GQA 16: two head tiles
     ("gemma", 1, 1, 4, 4096, None),             # D = 256
-    ("gemma", 2, 2, 6, 333, [333, 17]),         # D = 256, GQA 3, ragged
+    ("gemma", 2, 2, 6, 334, [333, 17]),         # D = 256, GQA 3, ragged (odd lengths)
 ]
 
 

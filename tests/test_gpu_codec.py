@@ -139,3 +139,48 @@ def test_gemma_full_size_sampled(kvq):
             check_encode(x16, s, lam, 32, codes[0, 0].cpu().numpy()[idx], scales[0, 0].cpu().numpy()[idx],
                          label=f"gemma L{layer}{kind}")
     assert kvq.poll_device_errors() == 0
+
+
+def test_encode_batch_matches_single_calls(kvq):
+    """Grouped encode of many (plan, x, cache) jobs with different shapes equals the
+    single-call encode of each job, bit for bit, and matches the oracle."""
+    dev = torch.device("cuda")
+    jobs, singles, inputs = [], [], []
+    shapes = [("qwen", 1, 2, 1, 8, 3), ("qwen", 2, 2, 200, 256, 40), ("toy", 1, 1, 256, 256, 0),
+              ("mistral", 3, 8, 17, 20, 2), ("qwen", 1, 2, 130, 130, 0)] * 14  # 70 jobs: two launches
+    for i, (wl_name, B, H, n, T_cap, pos) in enumerate(shapes):
+        wl = kvgen.WORKLOADS[wl_name]
+        s, lam = kvgen.plan_params(128, layer=i, kind="k")
+        plan = kvq.Plan(s, lam)
+        x16 = kvgen.kv_numpy(wl, "k", (B, H, n, 128), layer=i)
+        x = torch.from_numpy(x16).to(dev)
+        mk = lambda: (torch.full((B, H, T_cap, 64), 0x5A, dtype=torch.uint8, device=dev),
+                      torch.full((B, H, T_cap, 4), 3.0, dtype=torch.float16, device=dev))
+        c1, s1 = mk()
+        c2, s2 = mk()
+        jobs.append((plan, x, c1, s1, pos))
+        singles.append((plan, x, c2, s2, pos))
+        inputs.append((x16, s, lam, pos, n))
+    kvq.encode_batch(jobs)
+    for j in singles:
+        kvq.encode(*j)
+    torch.cuda.synchronize()
+    assert kvq.poll_device_errors() == 0
+    for (_, _, c1, s1, _), (_, _, c2, s2, _), (x16, s, lam, pos, n) in zip(jobs, singles, inputs):
+        assert torch.equal(c1, c2) and torch.equal(s1, s2)
+        check_encode(x16, s, lam, 32, c1.cpu().numpy()[:, :, pos:pos + n], s1.cpu().numpy()[:, :, pos:pos + n])
+
+
+def test_encode_batch_rejects_mixed_head_dims(kvq):
+    dev = torch.device("cuda")
+    p1 = kvq.Plan(*kvgen.plan_params(128))
+    p2 = kvq.Plan(*kvgen.plan_params(256))
+    j1 = (p1, torch.zeros((1, 1, 4, 128), dtype=torch.float16, device=dev),
+          torch.zeros((1, 1, 4, 64), dtype=torch.uint8, device=dev),
+          torch.zeros((1, 1, 4, 4), dtype=torch.float16, device=dev), 0)
+    j2 = (p2, torch.zeros((1, 1, 4, 256), dtype=torch.float16, device=dev),
+          torch.zeros((1, 1, 4, 128), dtype=torch.uint8, device=dev),
+          torch.zeros((1, 1, 4, 8), dtype=torch.float16, device=dev), 0)
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.encode_batch([j1, j2])
+    assert e.value.status == -1
