@@ -252,6 +252,14 @@ def run_kvq(args, rank: int, world: int):
     attn_phase()
     torch.cuda.synchronize()
     assert kvq.poll_device_errors() == 0
+    if args.ncu:
+        # profiling mode: a few eager steps, nothing timed (the launches an ncu capture selects from)
+        for s in range(args.steps):
+            kvq.encode_batch(jobs_for(s % N_INPUT_SETS))
+            attn_phase()
+        torch.cuda.synchronize()
+        print(json.dumps({"ncu_mode": True, "steps": args.steps, "launches_per_step": 1 + L}), flush=True)
+        return 0
 
     g_enc, g_att = [], []
     cap_stream = torch.cuda.Stream(device=dev)
@@ -386,6 +394,8 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--ncu", action="store_true",
+                    help="profiling mode: run --steps eager steps without timing, for ncu captures")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         args.warmup = 3

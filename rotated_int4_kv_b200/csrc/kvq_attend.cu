@@ -73,9 +73,61 @@ struct AttnParams {
   float sl2;                                   // softmax scale * log2(e)
   float* part;                                 // [units][S][2*8 + 8*D]
   int* cnt;                                    // [units]
-  const uint4* rq;                             // R'_K fragments (int4 only)
+  const float* qt;                             // rotated queries [units][8][D] (int4 only; from qrot_kernel)
   const uint4* ro;                             // R'_V^T fragments (int4 only)
 };
+
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Query rotation, once per (b, kv head, head tile): q_t[h][i] = sum_j R'[i][j] q[h][j]
+// with R' = Lambda_K^-1 F_r diag(s_K) as split fp16 (hi + lo) A fragments and q
+// (exact fp16) as B; fp32 accumulate. Every fragment load of a warp's m-tile is
+// issued before its mma chain. The attention kernel is launched as a programmatic
+// dependent of this one and waits for it only before reading q_t.
+template <int D>
+__global__ void __launch_bounds__(256) qrot_kernel(const uint16_t* __restrict__ q, const uint4* __restrict__ rq,
+                                                   float* __restrict__ qt, int Hq, int Hkv, int G, int HT) {
+  griddep_launch_dependents();
+  constexpr int MT = D / 16;
+  const int unit = blockIdx.x;
+  const int bk = unit / HT, ht = unit - bk * HT;
+  const int b = bk / Hkv, kvh = bk - b * Hkv;
+  const int heads = min(kHT, G - ht * kHT);
+  const int hq0 = kvh * G + ht * kHT;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;
+  const uint16_t* qb = q + ((size_t)b * Hq + hq0) * D;
+  float* out = qt + (size_t)unit * kHT * D;
+  uint32_t bq0[MT], bq1[MT];
+#pragma unroll
+  for (int kt = 0; kt < MT; ++kt) {
+    bq0[kt] = bq1[kt] = 0u;
+    if (g < heads) {
+      const uint16_t* qh = qb + (size_t)g * D + kt * 16 + 2 * c;
+      bq0[kt] = __ldg(reinterpret_cast<const uint32_t*>(qh));
+      bq1[kt] = __ldg(reinterpret_cast<const uint32_t*>(qh + 8));
+    }
+  }
+  for (int mt = warp; mt < MT; mt += 8) {
+    uint4 ah[MT], al[MT];
+#pragma unroll
+    for (int kt = 0; kt < MT; ++kt) {
+      ah[kt] = __ldg(rq + (((size_t)mt * MT + kt) * 2 + 0) * 32 + lane);
+      al[kt] = __ldg(rq + (((size_t)mt * MT + kt) * 2 + 1) * 32 + lane);
+    }
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int kt = 0; kt < MT; ++kt) {
+      mma_16816(acc, ah[kt].x, ah[kt].y, ah[kt].z, ah[kt].w, bq0[kt], bq1[kt]);
+      mma_16816(acc, al[kt].x, al[kt].y, al[kt].z, al[kt].w, bq0[kt], bq1[kt]);
+    }
+    out[(2 * c) * D + mt * 16 + g] = acc[0];
+    out[(2 * c + 1) * D + mt * 16 + g] = acc[1];
+    out[(2 * c) * D + mt * 16 + g + 8] = acc[2];
+    out[(2 * c + 1) * D + mt * 16 + g + 8] = acc[3];
+  }
+}
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
@@ -202,31 +254,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
     }
   } else {
     // ------------------------------------------------------------ consumers
-    // (1) query rotation: q_t[h][i] = sum_j R'[i][j] q[h][j]  (int4) or q_t = q (fp16)
-    const uint16_t* qb = p.q + ((size_t)b * p.Hq + hq0) * D;
+    // (1) rotated query (int4: written by qrot_kernel, waited for here) or q itself (fp16)
     if constexpr (INT4) {
-      // B operand: q (k = input channel j, n = head); A = R' fragments (hi, lo) from the plan
-      for (int mt = warp; mt < MT; mt += kCWarps) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int kt = 0; kt < MT; ++kt) {
-          uint32_t b0 = 0u, b1 = 0u;
-          if (g < heads) {
-            const uint16_t* qh = qb + (size_t)g * D + kt * 16 + 2 * c;
-            b0 = __ldg(reinterpret_cast<const uint32_t*>(qh));
-            b1 = __ldg(reinterpret_cast<const uint32_t*>(qh + 8));
-          }
-          const uint4 ah = __ldg(p.rq + (((size_t)mt * MT + kt) * 2 + 0) * 32 + lane);
-          const uint4 al = __ldg(p.rq + (((size_t)mt * MT + kt) * 2 + 1) * 32 + lane);
-          mma_16816(acc, ah.x, ah.y, ah.z, ah.w, b0, b1);
-          mma_16816(acc, al.x, al.y, al.z, al.w, b0, b1);
-        }
-        // C: rows = output channel (mt*16 + g, +8), cols = head (2c, 2c+1)
-        qt[(2 * c) * D + mt * 16 + g] = acc[0];
-        qt[(2 * c + 1) * D + mt * 16 + g] = acc[1];
-        qt[(2 * c) * D + mt * 16 + g + 8] = acc[2];
-        qt[(2 * c + 1) * D + mt * 16 + g + 8] = acc[3];
-      }
+      griddep_wait();
+      const float4* src = reinterpret_cast<const float4*>(p.qt + (size_t)unit * kHT * D);
+      for (int i = threadIdx.x; i < kHT * D / 4; i += kCWarps * 32)
+        reinterpret_cast<float4*>(qt)[i] = __ldcg(src + i);
     } else {
+      const uint16_t* qb = p.q + ((size_t)b * p.Hq + hq0) * D;
       for (int i = threadIdx.x; i < kHT * D; i += kCWarps * 32) {
         const int h = i / D;
         qt[i] = h < heads ? __half2float(__ushort_as_half(__ldg(qb + i))) : 0.0f;
@@ -538,56 +573,76 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
   __threadfence();
   const float* parts = p.part + (size_t)unit * p.S * PART;
   float* om = qt;  // merged o_t [8][D] (fp32)
-  for (int idx = threadIdx.x; idx < kHT * D; idx += kThreads) {
-    const int h = idx / D;
+  // per-head merge weights, computed once: wsm[s][h] = 2^(m_s - M) / L (0 for empty splits)
+  float* wsm = reinterpret_cast<float*>(ring);  // [S][8] (ring is free)
+  float* hm = wsm + p.S * kHT;                  // [8] head max
+  if (threadIdx.x < kHT) {
+    const int h = threadIdx.x;
     float M = -INFINITY;
     for (int s2 = 0; s2 < p.S; ++s2) M = fmaxf(M, __ldcg(parts + (size_t)s2 * PART + h));
-    float o = 0.0f, L = 0.0f;
-    if (M != -INFINITY) {
-      for (int s2 = 0; s2 < p.S; ++s2) {
-        const float* ps = parts + (size_t)s2 * PART;
-        const float ms = __ldcg(ps + h);
-        if (ms == -INFINITY) continue;
-        const float w = fast_exp2(ms - M);
-        o += __ldcg(ps + 2 * kHT + idx) * w;
-        L += __ldcg(ps + kHT + h) * w;
-      }
+    hm[h] = M;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < p.S * kHT; i += kThreads) {
+    const int s2 = i / kHT, h = i - s2 * kHT;
+    const float ms = __ldcg(parts + (size_t)s2 * PART + h);
+    const float M = hm[h];
+    wsm[i] = (M == -INFINITY || ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
+  }
+  __syncthreads();
+  if (threadIdx.x < kHT) {
+    const int h = threadIdx.x;
+    float L = 0.0f;
+    for (int s2 = 0; s2 < p.S; ++s2) L += wsm[s2 * kHT + h] * __ldcg(parts + (size_t)s2 * PART + kHT + h);
+    hm[h] = L > 0.0f ? 1.0f / L : 0.0f;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < p.S * kHT; i += kThreads) wsm[i] *= hm[i % kHT];
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < kHT * D; idx += kThreads) {
+    const int h = idx / D;
+    const float* po = parts + 2 * kHT + idx;
+    float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
+    int s2 = 0;
+    for (; s2 + 4 <= p.S; s2 += 4) {
+      o0 += wsm[(s2 + 0) * kHT + h] * __ldcg(po + (size_t)(s2 + 0) * PART);
+      o1 += wsm[(s2 + 1) * kHT + h] * __ldcg(po + (size_t)(s2 + 1) * PART);
+      o2 += wsm[(s2 + 2) * kHT + h] * __ldcg(po + (size_t)(s2 + 2) * PART);
+      o3 += wsm[(s2 + 3) * kHT + h] * __ldcg(po + (size_t)(s2 + 3) * PART);
     }
-    om[idx] = L > 0.0f ? o / L : 0.0f;
+    for (; s2 < p.S; ++s2) o0 += wsm[s2 * kHT + h] * __ldcg(po + (size_t)s2 * PART);
+    om[idx] = (o0 + o1) + (o2 + o3);
   }
   if (threadIdx.x == 0) p.cnt[unit] = 0;  // leave the counter at zero for the next call
   __syncthreads();
   uint16_t* ob = p.out + ((size_t)b * p.Hq + hq0) * D;
   if constexpr (INT4) {
-    // o[h][n] = sum_i R'^T[n][i] o_t[h][i]: A = R'^T (hi, lo), B = o_t split into hi + lo
-    if (warp < kCWarps) {
-      for (int mt = warp; mt < MT; mt += kCWarps) {
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int kt = 0; kt < MT; ++kt) {
-          const float* oh = om + g * D + kt * 16 + 2 * c;
-          __half h0, l0, h1, l1, h8, l8, h9, l9;
-          split_h(oh[0], h0, l0);
-          split_h(oh[1], h1, l1);
-          split_h(oh[8], h8, l8);
-          split_h(oh[9], h9, l9);
-          const uint32_t bh0 = h2_bits(__halves2half2(h0, h1)), bh1 = h2_bits(__halves2half2(h8, h9));
-          const uint32_t bl0 = h2_bits(__halves2half2(l0, l1)), bl1 = h2_bits(__halves2half2(l8, l9));
-          const uint4 ah = __ldg(p.ro + (((size_t)mt * MT + kt) * 2 + 0) * 32 + lane);
-          const uint4 al = __ldg(p.ro + (((size_t)mt * MT + kt) * 2 + 1) * 32 + lane);
-          mma_16816(acc, ah.x, ah.y, ah.z, ah.w, bh0, bh1);
-          mma_16816(acc, ah.x, ah.y, ah.z, ah.w, bl0, bl1);
-          mma_16816(acc, al.x, al.y, al.z, al.w, bh0, bh1);
-        }
-        // C: rows n = mt*16 + g (+8), cols head 2c, 2c+1
-        const int n0 = mt * 16 + g;
-        if (2 * c < heads) {
-          ob[(size_t)(2 * c) * D + n0] = __half_as_ushort(__float2half_rn(acc[0]));
-          ob[(size_t)(2 * c) * D + n0 + 8] = __half_as_ushort(__float2half_rn(acc[2]));
-        }
-        if (2 * c + 1 < heads) {
-          ob[(size_t)(2 * c + 1) * D + n0] = __half_as_ushort(__float2half_rn(acc[1]));
-          ob[(size_t)(2 * c + 1) * D + n0 + 8] = __half_as_ushort(__float2half_rn(acc[3]));
-        }
+    // o[h][n] = sum_i R'^T[n][i] o_t[h][i] with fp16 operands (R'^T hi part, o_t rounded to
+    // fp16; the result is rounded to fp16 anyway) and fp32 accumulate; the B
+    // fragments are shared by all m-tiles, and each m-tile's A loads are issued together.
+    uint32_t bo0[MT], bo1[MT];
+#pragma unroll
+    for (int kt = 0; kt < MT; ++kt) {
+      const float* oh = om + g * D + kt * 16 + 2 * c;
+      bo0[kt] = pack_half2(oh[0], oh[1]);
+      bo1[kt] = pack_half2(oh[8], oh[9]);
+    }
+    for (int mt = warp; mt < MT; mt += kCWarps + 1) {
+      uint4 ah[MT];
+#pragma unroll
+      for (int kt = 0; kt < MT; ++kt) ah[kt] = __ldg(p.ro + (((size_t)mt * MT + kt) * 2 + 0) * 32 + lane);
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int kt = 0; kt < MT; ++kt) mma_16816(acc, ah[kt].x, ah[kt].y, ah[kt].z, ah[kt].w, bo0[kt], bo1[kt]);
+      // C: rows n = mt*16 + g (+8), cols head 2c, 2c+1
+      const int n0 = mt * 16 + g;
+      if (2 * c < heads) {
+        ob[(size_t)(2 * c) * D + n0] = __half_as_ushort(__float2half_rn(acc[0]));
+        ob[(size_t)(2 * c) * D + n0 + 8] = __half_as_ushort(__float2half_rn(acc[2]));
+      }
+      if (2 * c + 1 < heads) {
+        ob[(size_t)(2 * c + 1) * D + n0] = __half_as_ushort(__float2half_rn(acc[1]));
+        ob[(size_t)(2 * c + 1) * D + n0 + 8] = __half_as_ushort(__float2half_rn(acc[3]));
       }
     }
   } else {
@@ -617,20 +672,43 @@ int ctas_per_sm() {
   return v;
 }
 
-// Split of the token range: enough CTAs to fill the GPU about twice, at least
-// one 64-token stage per split. Monotone in T (so the workspace size computed
-// from T_cap bounds every call with T <= T_cap).
+// Split of the token range. Each split keeps at least kMinTilesPerSplit stages so
+// that its TMA pipeline streams; among the split counts that give at least one
+// full wave of CTAs, the smallest one whose last wave is >= 85% full is taken
+// (else the best-filled one). Non-decreasing in T, so the workspace size computed
+// from T_cap bounds every call with T <= T_cap.
+constexpr int kMinTilesPerSplit = 2;
+constexpr int kMaxSplits = 256;
+
 SplitPlan choose_split(int B, int Hq, int Hkv, int T, int sms, int per_sm) {
   SplitPlan sp{};
   const int G = Hq / Hkv;
   sp.HT = (G + kHT - 1) / kHT;
   const long units = (long)B * Hkv * sp.HT;
   const int ntile = T > 0 ? (T + kTileT - 1) / kTileT : 1;
-  const long target = 2L * sms * per_sm;
-  int S = (int)((target + units - 1) / units);
-  S = S < 1 ? 1 : S;
-  S = S > ntile ? ntile : S;
-  const int tiles_per = (ntile + S - 1) / S;
+  const long slots = (long)sms * per_sm;
+  int s_cap = std::max(1, ntile / kMinTilesPerSplit);
+  s_cap = std::min(s_cap, kMaxSplits);
+  int best = 1;
+  double best_eff = -1.0;
+  const int s_lo = (int)std::min<long>(s_cap, std::max<long>(1, (slots + units - 1) / units));
+  for (int S = s_lo; S <= s_cap; ++S) {
+    const int tiles_per = (ntile + S - 1) / S;
+    const int Sr = (ntile + tiles_per - 1) / tiles_per;
+    const long ctas = units * Sr;
+    const long waves = (ctas + slots - 1) / slots;
+    const double eff = (double)ctas / (double)(waves * slots);
+    if (eff >= 0.85) {
+      best = S;
+      best_eff = eff;
+      break;
+    }
+    if (eff > best_eff + 1e-9) {
+      best_eff = eff;
+      best = S;
+    }
+  }
+  const int tiles_per = (ntile + best - 1) / best;
   sp.tps = tiles_per * kTileT;
   sp.S = (ntile + tiles_per - 1) / tiles_per;
   return sp;
@@ -638,11 +716,14 @@ SplitPlan choose_split(int B, int Hq, int Hkv, int T, int sms, int per_sm) {
 
 constexpr int kMaxPerSmForSizing = 4;
 
+// workspace: [counters (units ints, 256-aligned)] [rotated queries units x 8 x D fp32] [partials]
+size_t ws_cnt_bytes(size_t units) { return ((units * 4 + 255) / 256) * 256; }
+size_t ws_qt_bytes(size_t units, int D) { return units * kHT * D * 4; }
+
 size_t ws_bytes_for(int B, int Hq, int Hkv, int D, int S_max, int HT) {
   const size_t units = (size_t)B * Hkv * HT;
-  const size_t cnt = ((units * 4 + 255) / 256) * 256;
   const size_t part = units * (size_t)S_max * (2 * kHT + kHT * D) * 4;
-  return cnt + part;
+  return ws_cnt_bytes(units) + ws_qt_bytes(units, D) + part;
 }
 
 template <int D, bool INT4>
@@ -704,28 +785,48 @@ kvq_status run_attend(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q,
   prm.tps = sp.tps;
   const float sg = sigma > 0.0f ? sigma : 1.0f / sqrtf((float)D);
   prm.sl2 = sg * kLog2e;
-  const size_t cnt_bytes = ((units * 4 + 255) / 256) * 256;
-  prm.cnt = reinterpret_cast<int*>(ws);
-  prm.part = reinterpret_cast<float*>(reinterpret_cast<char*>(ws) + cnt_bytes);
-  prm.rq = INT4 ? pk->rq_frag : nullptr;
+  char* wsb = reinterpret_cast<char*>(ws);
+  prm.cnt = reinterpret_cast<int*>(wsb);
+  float* qt_ws = reinterpret_cast<float*>(wsb + ws_cnt_bytes(units));
+  prm.qt = qt_ws;
+  prm.part = reinterpret_cast<float*>(wsb + ws_cnt_bytes(units) + ws_qt_bytes(units, D));
   prm.ro = INT4 ? pv->ro_frag : nullptr;
   dim3 grid(sp.S, sp.HT, B * Hkv);
   if (grid.z > 65535u) return fail(KVQ_ERR_UNSUPPORTED, "attend: B * Hkv > 65535");
-  attend_kernel<D, INT4><<<grid, kThreads, C::kSmem, strm>>>(kmap, vmap, ksmap, vsmap, prm);
-  const cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
+  if constexpr (INT4) {
+    qrot_kernel<D><<<(unsigned)units, 256, 0, strm>>>(q, pk->rq_frag, qt_ws, Hq, Hkv, Hq / Hkv, sp.HT);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("qrot launch: ") + cudaGetErrorString(e));
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = C::kSmem;
+    cfg.stream = strm;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, attend_kernel<D, INT4>, kmap, vmap, ksmap, vsmap, prm);
+    if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
+  } else {
+    attend_kernel<D, INT4><<<grid, kThreads, C::kSmem, strm>>>(kmap, vmap, ksmap, vsmap, prm);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
+  }
   return KVQ_OK;
 }
 
 }  // namespace
 
 size_t attend_workspace_bytes(int B, int Hq, int Hkv, int D, int T_cap) {
-  int dev = 0;
-  int sms = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess) sms = num_sms(dev);
-  SplitPlan sp = choose_split(B, Hq, Hkv, T_cap, sms, kMaxPerSmForSizing);
-  // the launch uses per_sm <= kMaxPerSmForSizing, hence S <= this S
-  return ws_bytes_for(B, Hq, Hkv, D, sp.S, sp.HT);
+  // Bound over every split the launch can choose for T <= T_cap: S never exceeds
+  // min(kMaxSplits, ntile(T_cap) / kMinTilesPerSplit) (at least 1).
+  const int G = Hq / Hkv;
+  const int HT = (G + kHT - 1) / kHT;
+  const int ntile = T_cap > 0 ? (T_cap + kTileT - 1) / kTileT : 1;
+  const int s_max = std::max(1, std::min(kMaxSplits, ntile / kMinTilesPerSplit));
+  return ws_bytes_for(B, Hq, Hkv, D, s_max, HT);
 }
 
 kvq_status launch_attend_int4(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q, const uint8_t* kc,

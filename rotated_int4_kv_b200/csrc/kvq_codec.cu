@@ -50,31 +50,27 @@ __device__ __forceinline__ void tile_origin(const TileGeom& g, int tile, int& bh
   t0 = tt * g.T_box;
 }
 
-// D=128: 2 prefetch stages, 3 CTAs per SM (<= 170 registers); D=256: the vector
-// needs ~255 registers, so 2 CTAs per SM with one stage each (the next tile's
-// load is issued as soon as the current one is in registers).
+// decode: D=128 fits 3 CTAs per SM (<= 170 registers); D=256 needs ~255 registers.
 template <int D>
 constexpr int kMinBlocks = D == 128 ? 3 : 2;
-
-template <int D>
-struct SmemLayout {
-  static constexpr int kXStage = kNT * D * 2;        // fp16 x tile (D/64 swizzled boxes)
-  static constexpr int kCTile = kNT * D / 2;         // packed code tile
-  static constexpr int kStages = D == 128 ? 2 : 1;
-  static constexpr int kBytes = kStages * kXStage + kCTile + D * 4 + D * 2 + 64 + 1024;
-};
 
 // ---------------------------------------------------------------- encode
 // One launch walks the tiles of up to MAXJ independent jobs (kvq_encode = 1 job,
 // kvq_encode_batch = a grouped launch). A job's tensor maps live in the kernel
-// parameter block; its lambda/sign constants are staged in shared memory when a
-// CTA moves to a tile of another job.
+// parameter block; its lambda/sign constants are read through L1 (uniform loads).
+//
+// Pipeline: no producer warp and no CTA-wide barrier in the steady state. A tile
+// (128 vectors at D=128, 64 at D=256) is one TMA load into one of two stages;
+// each of the four warps reads its 32 (or 16) rows, and the warp that finishes
+// reading a stage last (found with an acq_rel shared-memory counter) issues the
+// stage's next load. Each warp stages its own packed codes and stores them with
+// its own TMA box, so warps drift freely within the two-stage window.
 struct alignas(64) EncJob {
   CUtensorMap xmap;           // x [BH, n, D] fp16, box {64, T_box, BH_box}, 128B swizzle
-  CUtensorMap cmap;           // codes [BH, pos+n, D/2] u8 (rows pos.. of the cache), box {D/2, T_box, BH_box}
+  CUtensorMap cmap;           // codes [BH, pos+n, D/2] u8, box = one warp's rows {D/2, Tw, Bw}
   const CodecConsts* cc;      // device: lambda*dg per channel, sign masks
   uint16_t* scales;
-  int T_cap, pos, BH, n, T_box, BH_box, t_shift, n_ttiles, tile0;
+  int T_cap, pos, BH, n, T_box, BH_box, t_shift, n_ttiles, tile0, Tw, w_shift;
 };
 
 template <int MAXJ>
@@ -93,183 +89,298 @@ __device__ __forceinline__ int job_of(const EncBatch<MAXJ>& P, int tile) {
   return j;
 }
 
+__device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
+  uint32_t old;
+  asm volatile("atom.acq_rel.cta.shared::cta.add.u32 %0, [%1], %2;" : "=r"(old) : "r"(smem_u32(p)), "r"(v) : "memory");
+  return old;
+}
+
+// D = 256 pair combine: thread p of a pair holds the size-128 spectrum of the samples
+// x[2j + p] (E for p = 0, O for p = 1) in slot order; it forms X_k and X_{128-k} for
+// k = 32p + J, J = 0..32, exchanging one value per component with its partner.
+// Thread 0 then owns channels [0, 64) and [192, 256), thread 1 channels [64, 192);
+// local value L of both threads maps to the same (J, X or X_{128-k}, Re or Im), except L = 0.
+template <int S_>
+struct TwPair {  // W_256^(32p + J) for p = 0, 1
+  static constexpr float c0 = static_cast<float>(cos2pi_frac(S_, 256));
+  static constexpr float s0 = static_cast<float>(sin2pi_frac(S_, 256));
+  static constexpr float c1 = static_cast<float>(cos2pi_frac(S_ + 32, 256));
+  static constexpr float s1 = static_cast<float>(sin2pi_frac(S_ + 32, 256));
+};
+
+__device__ __forceinline__ float slotv(const float2 (&u)[64], int sl) { return (sl & 1) ? u[sl >> 1].y : u[sl >> 1].x; }
+
+template <int J>
+__device__ __forceinline__ void pair_combine(const float2 (&u)[64], float (&o)[128], const bool p) {
+  if constexpr (J <= 32) {
+    constexpr int k0 = J, k1 = 32 + J;
+    constexpr int re0 = k0 == 0 ? 0 : 2 * k0, im0 = k0 == 0 ? -1 : 2 * k0 + 1;
+    constexpr int re1 = k1 == 64 ? 1 : 2 * k1, im1 = k1 == 64 ? -1 : 2 * k1 + 1;
+    const float u_re0 = slotv(u, re0), u_re1 = slotv(u, re1);
+    const float u_im0 = im0 < 0 ? 0.0f : slotv(u, im0 < 0 ? 0 : im0);
+    const float u_im1 = im1 < 0 ? 0.0f : slotv(u, im1 < 0 ? 0 : im1);
+    const float mine_re = p ? u_re1 : u_re0, send_re = p ? u_re0 : u_re1;
+    const float mine_im = p ? u_im1 : u_im0, send_im = p ? u_im0 : u_im1;
+    const float recv_re = __shfl_xor_sync(0xffffffffu, send_re, 1);
+    const float recv_im = __shfl_xor_sync(0xffffffffu, send_im, 1);
+    const float er = p ? recv_re : mine_re, ei = p ? recv_im : mine_im;
+    const float orr = p ? mine_re : recv_re, oi = p ? mine_im : recv_im;
+    const float c = p ? TwPair<J>::c1 : TwPair<J>::c0;
+    const float sn = p ? TwPair<J>::s1 : TwPair<J>::s0;
+    const float xr = fmaf(c, orr, fmaf(sn, oi, er));  // X_k = E + W O
+    const float xi = fmaf(c, oi, fmaf(-sn, orr, ei));
+    const float yr = fmaf(2.0f, er, -xr);              // X_{128-k} = conj(E - W O)
+    const float yi = fmaf(-2.0f, ei, xi);
+    if constexpr (J == 0) {
+      o[0] = p ? xi : xr;
+      o[127] = yr;
+    } else if constexpr (J < 32) {
+      o[2 * J - 1] = xr;
+      o[2 * J] = xi;
+      o[127 - 2 * J] = yr;
+      o[128 - 2 * J] = yi;
+    } else {
+      o[63] = xr;
+      o[64] = yi;
+    }
+    pair_combine<J + 1>(u, o, p);
+  }
+}
+
+// lambda, per-group abs-max, fp16 scale, int4 rounding and nibble packing of
+// NV channel values (NV/G groups); lam points at the lambda*dg of those channels.
+template <int NV, int G>
+__device__ __forceinline__ void quantize_pack(const float (&v)[NV], const float* __restrict__ lam,
+                                              uint32_t (&words)[NV / 8], uint32_t (&sbits)[NV / G]) {
+#pragma unroll
+  for (int g = 0; g < NV / G; ++g) {
+    float y[G];
+    float a = 0.0f;
+#pragma unroll
+    for (int i4 = 0; i4 < G / 4; ++i4) {
+      const float4 l4 = __ldg(reinterpret_cast<const float4*>(lam + g * G) + i4);
+      const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int i = 4 * i4 + e;
+        y[i] = v[g * G + i] * lv[e];
+        a = fmaxf(a, fabsf(y[i]));
+      }
+    }
+    const float sf = fminf(__fdiv_rn(a, 7.0f), 65504.0f);
+    const __half hs = __float2half_rn(sf);
+    const float sq = __half2float(hs);
+    const float inv = sq > 0.0f ? __frcp_rn(sq) : 0.0f;
+    sbits[g] = __half_as_ushort(hs);
+    const bool clampit = a * inv >= 7.5f;
+    uint32_t b[G];
+#pragma unroll
+    for (int i = 0; i < G; i += 2) {
+      float2 q = __ffma2_rn(make_float2(y[i], y[i + 1]), make_float2(inv, inv), make_float2(kMagic, kMagic));
+      if (clampit) {
+        q.x = fminf(fmaxf(q.x, kMagicLo), kMagicHi);
+        q.y = fminf(fmaxf(q.y, kMagicLo), kMagicHi);
+      }
+      b[i] = __float_as_uint(q.x);
+      b[i + 1] = __float_as_uint(q.y);
+    }
+#pragma unroll
+    for (int w = 0; w < G / 8; ++w) {
+      const uint32_t* bb = b + 8 * w;
+      const uint32_t x01 = bb[0] + (bb[1] << 4);
+      const uint32_t x23 = bb[2] + (bb[3] << 4);
+      const uint32_t x45 = bb[4] + (bb[5] << 4);
+      const uint32_t x67 = bb[6] + (bb[7] << 4);
+      words[g * (G / 8) + w] = prmt(x01 + (x23 << 8), x45 + (x67 << 8), 0x5410u) ^ 0x88888888u;
+    }
+  }
+}
+
+template <int D>
+struct EncCfg {
+  static constexpr int kTPV = D / 128;                 // threads per vector
+  static constexpr int kRows = kNT / kTPV;             // vectors per tile
+  static constexpr int kRowsW = 32 / kTPV;             // vectors per warp
+  static constexpr int kXStage = kRows * D * 2;        // 32 KB
+  static constexpr int kBoxBytes = kRows * 128;        // one 64-half box
+  static constexpr int kStages = 2;
+  static constexpr int kCWarp = kRowsW * D / 2;        // per-warp code staging (2 KB)
+  static constexpr int kBytes = kStages * kXStage + 4 * kCWarp + 64 + 1024;
+};
+
 template <int D, int G, int MAXJ>
-__global__ void __launch_bounds__(kNT, kMinBlocks<D>) encode_kernel(const __grid_constant__ EncBatch<MAXJ> P) {
-  using L = SmemLayout<D>;
-  constexpr int kBoxes = D / 64;
-  constexpr int kBoxBytes = kNT * 128;
-  constexpr int kNG = D / G;
-  constexpr int kWords = D / 8;  // packed code words per vector
+__global__ void __launch_bounds__(kNT, 3) encode_kernel(const __grid_constant__ EncBatch<MAXJ> P) {
+  using C = EncCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xs = smem;
-  uint8_t* cs = smem + L::kStages * L::kXStage;
-  float* cchan = reinterpret_cast<float*>(cs + L::kCTile);          // [D]
-  uint32_t* csgn = reinterpret_cast<uint32_t*>(cchan + D);           // [D/2]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(csgn + D / 2);
+  uint8_t* cs_all = smem + C::kStages * C::kXStage;
+  uint64_t* full = reinterpret_cast<uint64_t*>(cs_all + 4 * C::kCWarp);
+  uint32_t* rd_cnt = reinterpret_cast<uint32_t*>(full + C::kStages);
 
   const int tid = threadIdx.x;
+  const int warp = tid >> 5, lane = tid & 31;
   const int first = blockIdx.x;
   const int stride = gridDim.x;
   if (first >= P.total_tiles) return;
-
   if (tid == 0) {
-    for (int s = 0; s < L::kStages; ++s) mbar_init(&bar[s], 1);
+    for (int s2 = 0; s2 < C::kStages; ++s2) {
+      mbar_init(&full[s2], 1);
+      rd_cnt[s2] = 0;
+    }
     fence_mbarrier_init();
   }
   __syncthreads();
-
   auto issue = [&](int tile, int stage) {
     const EncJob& J = P.jobs[job_of(P, tile)];
     const int lt = tile - J.tile0;
     const int tb = lt / J.n_ttiles;
     const int bh0 = tb * J.BH_box, t0 = (lt - tb * J.n_ttiles) * J.T_box;
-    mbar_arrive_expect_tx(&bar[stage], L::kXStage);
+    mbar_arrive_expect_tx(&full[stage], C::kXStage);
 #pragma unroll
-    for (int b = 0; b < kBoxes; ++b)
-      tma_load_3d(xs + stage * L::kXStage + b * kBoxBytes, &J.xmap, &bar[stage], b * 64, t0, bh0);
+    for (int b = 0; b < D / 64; ++b)
+      tma_load_3d(xs + stage * C::kXStage + b * C::kBoxBytes, &J.xmap, &full[stage], b * 64, t0, bh0);
   };
   if (tid == 0) {
-    for (int s = 0; s < L::kStages; ++s) {
-      const int tile = first + s * stride;
-      if (tile < P.total_tiles) issue(tile, s);
+    for (int s2 = 0; s2 < C::kStages; ++s2) {
+      const int tile = first + s2 * stride;
+      if (tile < P.total_tiles) issue(tile, s2);
     }
   }
-
-  int cur_job = -1;
+  uint8_t* cs = cs_all + warp * C::kCWarp;
+  const int r = warp * C::kRowsW + (C::kTPV == 2 ? (lane >> 1) : lane);  // tile row of this thread
+  const bool p = C::kTPV == 2 && (lane & 1);
   int it = 0;
   for (int tile = first; tile < P.total_tiles; tile += stride, ++it) {
-    const int j = job_of(P, tile);
-    const EncJob& J = P.jobs[j];
-    if (j != cur_job) {  // CTA-uniform: stage this job's constants (previous readers finished before the last sync)
-      const float* src = J.cc->chan;
-      for (int i = tid; i < D; i += kNT) cchan[i] = src[i];
-      for (int i = tid; i < D / 2; i += kNT) csgn[i] = J.cc->sgn[i];
-      cur_job = j;
-      __syncthreads();
-    }
+    const EncJob& J = P.jobs[job_of(P, tile)];
     const int lt = tile - J.tile0;
     const int tb = lt / J.n_ttiles;
     const int bh0 = tb * J.BH_box, t0 = (lt - tb * J.n_ttiles) * J.T_box;
-    const int t_l = tid & (J.T_box - 1);
-    const int bh_l = tid >> J.t_shift;
-
-    const int stage = it % L::kStages;
-    const uint32_t parity = (it / L::kStages) & 1;
-    if (!mbar_wait_bounded(&bar[stage], parity)) {
+    const int stage = it % C::kStages;
+    if (!mbar_wait_bounded(&full[stage], (it / C::kStages) & 1)) {
       atomicOr(&g_codec_err, kErrTimeoutLoad);
       return;
     }
-    // ---- load own row (swizzled 128B boxes), apply signs, convert
-    float v[D];
+    // ---- own row (128B-swizzled boxes) -> fp32 pairs, signs applied on the fp16 bits
+    float2 v[64];
     {
-      const uint8_t* base = xs + stage * L::kXStage + tid * 128;
-      const int sw = tid & 7;
+      const uint8_t* base = xs + stage * C::kXStage + r * 128;
+      const int sw = r & 7;
+      if constexpr (C::kTPV == 1) {
+        const uint4* sg = reinterpret_cast<const uint4*>(J.cc->sgn);
 #pragma unroll
-      for (int b = 0; b < kBoxes; ++b) {
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint4 w = *reinterpret_cast<const uint4*>(base + b * kBoxBytes + ((c ^ sw) << 4));
-          const uint4 m = *reinterpret_cast<const uint4*>(csgn + (b * 64 + c * 8) / 2);
-          const int e0 = b * 64 + c * 8;
+        for (int cc = 0; cc < 16; ++cc) {  // x[8cc .. 8cc+7]
+          const uint4 w = *reinterpret_cast<const uint4*>(base + (cc >> 3) * C::kBoxBytes + (((cc & 7) ^ sw) << 4));
+          const uint4 m = __ldg(sg + cc);
           const uint32_t ww[4] = {w.x ^ m.x, w.y ^ m.y, w.z ^ m.z, w.w ^ m.w};
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&ww[q]));
-            v[e0 + 2 * q] = f.x;
-            v[e0 + 2 * q + 1] = f.y;
-          }
+          for (int q = 0; q < 4; ++q) v[4 * cc + q] = __half22float2(*reinterpret_cast<const __half2*>(&ww[q]));
         }
-      }
-    }
-    __syncthreads();  // every thread has its row: the stage may be refilled
-    if (tid == 0) {
-      const int nxt = tile + L::kStages * stride;
-      if (nxt < P.total_tiles) issue(nxt, stage);
-    }
-
-    // ---- transform
-    rdft_fwd<D>(v);
-
-    // ---- lambda, group abs-max, fp16 scale, int4 rounding, nibble packing
-    uint32_t words[kWords];
-    uint32_t sbits[kNG];
-#pragma unroll
-    for (int g = 0; g < kNG; ++g) {
-      float y[G];
-      float a = 0.0f;
-#pragma unroll
-      for (int i4 = 0; i4 < G / 4; ++i4) {
-        const float4 l4 = *reinterpret_cast<const float4*>(cchan + g * G + 4 * i4);
-        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int i = 4 * i4 + e;
-          y[i] = v[slot_of_channel(g * G + i, D)] * lv[e];
-          a = fmaxf(a, fabsf(y[i]));
-        }
-      }
-      const float sf = fminf(__fdiv_rn(a, 7.0f), 65504.0f);
-      const __half hs = __float2half_rn(sf);
-      const float sq = __half2float(hs);
-      const float inv = sq > 0.0f ? __frcp_rn(sq) : 0.0f;
-      sbits[g] = __half_as_ushort(hs);
-      const bool clampit = a * inv >= 7.5f;
-      uint32_t b[G];
-#pragma unroll
-      for (int i = 0; i < G; ++i) {
-        float qv = fmaf(y[i], inv, kMagic);
-        if (clampit) qv = fminf(fmaxf(qv, kMagicLo), kMagicHi);
-        b[i] = __float_as_uint(qv);
-      }
-#pragma unroll
-      for (int w = 0; w < G / 8; ++w) {
-        const uint32_t* bb = b + 8 * w;
-        const uint32_t x01 = bb[0] + (bb[1] << 4);
-        const uint32_t x23 = bb[2] + (bb[3] << 4);
-        const uint32_t x45 = bb[4] + (bb[5] << 4);
-        const uint32_t x67 = bb[6] + (bb[7] << 4);
-        const uint32_t lo = x01 + (x23 << 8);
-        const uint32_t hi = x45 + (x67 << 8);
-        words[g * (G / 8) + w] = prmt(lo, hi, 0x5410u) ^ 0x88888888u;
-      }
-    }
-
-    // ---- outputs
-    const int t = t0 + t_l, bh = bh0 + bh_l;
-    const bool valid = (t < J.n) && (bh < J.BH);
-    if (valid) {
-      uint16_t* sp = J.scales + ((size_t)bh * J.T_cap + J.pos + t) * kNG;
-      if constexpr (kNG == 4) {
-        *reinterpret_cast<uint2*>(sp) = make_uint2(sbits[0] | (sbits[1] << 16), sbits[2] | (sbits[3] << 16));
       } else {
+        const uint32_t sel = p ? 0x7632u : 0x5410u;
+        const uint32_t* sg = J.cc->sgn;
 #pragma unroll
-        for (int q = 0; q < kNG / 8; ++q)
-          reinterpret_cast<uint4*>(sp)[q] =
-              make_uint4(sbits[8 * q + 0] | (sbits[8 * q + 1] << 16), sbits[8 * q + 2] | (sbits[8 * q + 3] << 16),
-                         sbits[8 * q + 4] | (sbits[8 * q + 5] << 16), sbits[8 * q + 6] | (sbits[8 * q + 7] << 16));
+        for (int cc = 0; cc < 32; ++cc) {  // thread p takes x[8cc + p + 2i], i = 0..3
+          const uint4 w = *reinterpret_cast<const uint4*>(base + (cc >> 3) * C::kBoxBytes + (((cc & 7) ^ sw) << 4));
+          const uint4 m = __ldg(reinterpret_cast<const uint4*>(sg) + cc);
+          uint32_t h0 = prmt(w.x ^ m.x, w.y ^ m.y, sel);
+          uint32_t h1 = prmt(w.z ^ m.z, w.w ^ m.w, sel);
+          v[2 * cc] = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+          v[2 * cc + 1] = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+        }
       }
     }
-    if (tid == 0) bulk_wait_group_read0();  // the previous tile's code store has left the staging tile
-    __syncthreads();
-    {
-      // code row: D/2 bytes = D/32 chunks of 16 B; 64B swizzle for D=128, 128B for D=256
-      uint8_t* row = cs + tid * (D / 2);
+    __syncwarp();
+    if (lane == 0) {
+      // the warp that reads this stage last refills it with the stage's next tile
+      if (atom_add_acq_rel(&rd_cnt[stage], 1u) % 4u == 3u) {
+        const int nxt = tile + C::kStages * stride;
+        if (nxt < P.total_tiles) {
+          fence_proxy_async_smem();
+          issue(nxt, stage);
+        }
+      }
+    }
+    // ---- transform (packed f32x2 halves + scalar top stage), lambda, quantise, pack
+    rdft_fwd_packed<128>(v);
+    uint32_t words[16];
+    uint32_t sbits[128 / G];
+    int cb_lo, cb_hi;  // first channels of the two 64-channel halves this thread owns
+    if constexpr (C::kTPV == 1) {
+      float vv[128];
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        const int pc = (D == 128) ? (c ^ ((tid >> 1) & 3)) : (c ^ (tid & 7));
-        *reinterpret_cast<uint4*>(row + pc * 16) =
-            make_uint4(words[4 * c], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
+      for (int c = 0; c < 128; ++c) vv[c] = slotv(v, slot_of_channel(c, 128));
+      quantize_pack<128, G>(vv, J.cc->chan, words, sbits);
+      cb_lo = 0;
+      cb_hi = 64;
+    } else {
+      float vv[128];
+      pair_combine<0>(v, vv, p);
+      cb_lo = p ? 64 : 0;
+      cb_hi = p ? 128 : 192;
+      float lo[64], hi[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        lo[i] = vv[i];
+        hi[i] = vv[64 + i];
+      }
+      uint32_t wl[8], wh[8], sl[64 / G], sh[64 / G];
+      quantize_pack<64, G>(lo, J.cc->chan + cb_lo, wl, sl);
+      quantize_pack<64, G>(hi, J.cc->chan + cb_hi, wh, sh);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        words[i] = wl[i];
+        words[8 + i] = wh[i];
+      }
+#pragma unroll
+      for (int i = 0; i < 64 / G; ++i) {
+        sbits[i] = sl[i];
+        sbits[64 / G + i] = sh[i];
+      }
+    }
+    // ---- scales: one store per owned half (groups are contiguous within a half)
+    const int t_l = r & (J.T_box - 1), bh_l = r >> J.t_shift;
+    const int t = t0 + t_l, bh = bh0 + bh_l;
+    if (t < J.n && bh < J.BH) {
+      uint16_t* sp = J.scales + ((size_t)bh * J.T_cap + J.pos + t) * (D / G);
+      constexpr int NH = 64 / G;  // scales per 64-channel half (2 or 4)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int g0 = (h ? cb_hi : cb_lo) / G;
+        if constexpr (NH == 2) {
+          *reinterpret_cast<uint32_t*>(sp + g0) = sbits[h * NH] | (sbits[h * NH + 1] << 16);
+        } else {
+          *reinterpret_cast<uint2*>(sp + g0) = make_uint2(sbits[h * NH] | (sbits[h * NH + 1] << 16),
+                                                          sbits[h * NH + 2] | (sbits[h * NH + 3] << 16));
+        }
+      }
+    }
+    // ---- codes: this warp's rows -> its staging slice -> its own TMA store
+    if (lane == 0) bulk_wait_group_read0();
+    __syncwarp();
+    {
+      const int rw = r - warp * C::kRowsW;  // row within the warp's slice
+      uint8_t* row = cs + rw * (D / 2);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+#pragma unroll
+        for (int c2 = 0; c2 < 2; ++c2) {  // 16-byte chunks = 32 channels
+          const int ch = (h ? cb_hi : cb_lo) / 32 + c2;
+          const int pc = (D == 128) ? (ch ^ ((rw >> 1) & 3)) : (ch ^ (rw & 7));
+          const int wi = 8 * h + 4 * c2;
+          *reinterpret_cast<uint4*>(row + pc * 16) = make_uint4(words[wi], words[wi + 1], words[wi + 2], words[wi + 3]);
+        }
       }
     }
     fence_proxy_async_smem();
-    __syncthreads();
-    if (tid == 0) {
-      tma_store_3d(&J.cmap, cs, 0, J.pos + t0, bh0);
+    __syncwarp();
+    if (lane == 0) {
+      const int r0 = warp * C::kRowsW;  // the warp's rows: a {Tw, RowsW/Tw} box of the tile
+      tma_store_3d(&J.cmap, cs, 0, J.pos + t0 + (r0 & (J.T_box - 1)), bh0 + (r0 >> J.t_shift));
       bulk_commit_group();
     }
   }
-  if (tid == 0) bulk_wait_group0();
+  if (lane == 0) bulk_wait_group0();
 }
 
 // ---------------------------------------------------------------- decode
@@ -425,14 +536,14 @@ __global__ void __launch_bounds__(kNT, kMinBlocks<D>) decode_kernel(const __grid
 }
 
 // ---------------------------------------------------------------- host side
-TileGeom make_geom(int BH, int n) {
+TileGeom make_geom(int BH, int n, int rows = kNT) {
   TileGeom g{};
   g.BH = BH;
   g.n = n;
   int tb = 1;
-  while (tb < n && tb < kNT) tb <<= 1;
+  while (tb < n && tb < rows) tb <<= 1;
   g.T_box = tb;
-  g.BH_box = kNT / tb;
+  g.BH_box = rows / tb;
   int sh = 0;
   while ((1 << sh) < tb) ++sh;
   g.t_shift = sh;
@@ -457,7 +568,9 @@ kvq_status run_encode_chunk(const kvq_encode_job* jobs, int nj, cudaStream_t s) 
     const kvq_encode_job& q = jobs[i];
     EncJob& J = P.jobs[i];
     const int BH = q.B * q.H;
-    TileGeom geom = make_geom(BH, q.n);
+    TileGeom geom = make_geom(BH, q.n, EncCfg<D>::kRows);
+    const int RW = EncCfg<D>::kRowsW;
+    const int Tw = std::min(geom.T_box, RW);
     {
       const uint64_t dims[3] = {(uint64_t)D, (uint64_t)q.n, (uint64_t)BH};
       const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)D * 2 * q.n};
@@ -469,7 +582,7 @@ kvq_status run_encode_chunk(const kvq_encode_job* jobs, int nj, cudaStream_t s) 
     {
       const uint64_t dims[3] = {(uint64_t)D / 2, (uint64_t)(q.pos + q.n), (uint64_t)BH};
       const uint64_t strides[2] = {(uint64_t)D / 2, (uint64_t)(D / 2) * q.T_cap};
-      const uint32_t box[3] = {(uint32_t)D / 2, (uint32_t)geom.T_box, (uint32_t)geom.BH_box};
+      const uint32_t box[3] = {(uint32_t)D / 2, (uint32_t)Tw, (uint32_t)(RW / Tw)};
       kvq_status st = encode_tiled(&J.cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q.codes, dims, strides, box,
                                    D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, "code cache");
       if (st != KVQ_OK) return st;
@@ -485,21 +598,23 @@ kvq_status run_encode_chunk(const kvq_encode_job* jobs, int nj, cudaStream_t s) 
     J.t_shift = geom.t_shift;
     J.n_ttiles = geom.n_ttiles;
     J.tile0 = tiles;
+    J.Tw = Tw;
     tiles += geom.n_tiles;
   }
   P.njobs = nj;
   P.total_tiles = tiles;
-  constexpr int smem = SmemLayout<D>::kBytes;
+  void (*kern)(const EncBatch<MAXJ>) = encode_kernel<D, G, MAXJ>;
+  const int smem = EncCfg<D>::kBytes;
   static int blocks_per_sm = -1;
   static std::once_flag once;
   std::call_once(once, [&] {
-    cudaFuncSetAttribute(encode_kernel<D, G, MAXJ>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    blocks_per_sm = occupancy_blocks(encode_kernel<D, G, MAXJ>, smem);
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    blocks_per_sm = occupancy_blocks(kern, smem);
   });
   int dev = 0;
   cudaGetDevice(&dev);
   const int grid = std::min(tiles, blocks_per_sm * num_sms(dev));
-  encode_kernel<D, G, MAXJ><<<grid, kNT, smem, s>>>(P);
+  kern<<<grid, kNT, smem, s>>>(P);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("encode launch: ") + cudaGetErrorString(e));
   return KVQ_OK;

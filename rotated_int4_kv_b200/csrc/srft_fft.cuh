@@ -154,6 +154,165 @@ __device__ __forceinline__ void rdft_inv(float (&v)[N]) {
   Rdft<N, 0, 1, N>::inv(v);
 }
 
+// ---------------------------------------------------------------- packed (f32x2) transforms
+// Two independent real sequences per float2 (.x and .y); every butterfly runs as
+// Blackwell packed fp32 instructions (fma/add/sub .f32x2), i.e. one issue slot
+// for two scalar operations. Used for the two halves of the first decimation:
+// with v[m] = (x[2m], x[2m+1]), a packed size-N/2 transform gives E (even
+// samples) in .x and O (odd samples) in .y; rdft_top_* then forms the size-N
+// spectrum with scalar butterflies.
+__device__ __forceinline__ float2 p2fma(float2 a, float2 b, float2 c) { return __ffma2_rn(a, b, c); }
+__device__ __forceinline__ float2 p2add(float2 a, float2 b) { return __fadd2_rn(a, b); }
+__device__ __forceinline__ float2 p2mul(float2 a, float2 b) { return __fmul2_rn(a, b); }
+__device__ __forceinline__ float2 p2sub(float2 a, float2 b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<unsigned long long*>(&a)), "l"(*reinterpret_cast<unsigned long long*>(&b)));
+  return *reinterpret_cast<float2*>(&d);
+}
+__device__ __forceinline__ float2 p2bc(float x) { return make_float2(x, x); }
+
+template <int N, int OFF, int S, int TOT, int K>
+struct RdftBflyP {
+  static __device__ __forceinline__ void fwd(float2 (&v)[TOT], const float2 (&e)[N / 2], const float2 (&o)[N / 2]) {
+    if constexpr (K < N / 4) {
+      constexpr float c = static_cast<float>(cos2pi_frac(K, N));
+      constexpr float s = static_cast<float>(sin2pi_frac(K, N));
+      const float2 er = e[2 * K], ei = e[2 * K + 1], orr = o[2 * K], oi = o[2 * K + 1];
+      const float2 xr = p2fma(p2bc(c), orr, p2fma(p2bc(s), oi, er));
+      const float2 xi = p2fma(p2bc(c), oi, p2fma(p2bc(-s), orr, ei));
+      v[OFF + S * (2 * K)] = xr;
+      v[OFF + S * (2 * K + 1)] = xi;
+      v[OFF + S * (N - 2 * K)] = p2fma(p2bc(-c), orr, p2fma(p2bc(-s), oi, er));  // Re(E - W O)
+      v[OFF + S * (N - 2 * K + 1)] = p2fma(p2bc(-2.0f), ei, xi);                 // -Im(E - W O)
+      RdftBflyP<N, OFF, S, TOT, K + 1>::fwd(v, e, o);
+    }
+  }
+  static __device__ __forceinline__ void inv(const float2 (&v)[TOT], float2 (&e)[N / 2], float2 (&o)[N / 2]) {
+    if constexpr (K < N / 4) {
+      constexpr float c = static_cast<float>(cos2pi_frac(K, N));
+      constexpr float s = static_cast<float>(sin2pi_frac(K, N));
+      const float2 ar = v[OFF + S * (2 * K)], ai = v[OFF + S * (2 * K + 1)];
+      const float2 br = v[OFF + S * (N - 2 * K)], bi = v[OFF + S * (N - 2 * K + 1)];
+      e[2 * K] = p2add(ar, br);
+      e[2 * K + 1] = p2sub(ai, bi);
+      const float2 dr = p2sub(ar, br), di = p2add(ai, bi);
+      o[2 * K] = p2fma(p2bc(c), dr, p2mul(p2bc(-s), di));
+      o[2 * K + 1] = p2fma(p2bc(s), dr, p2mul(p2bc(c), di));
+      RdftBflyP<N, OFF, S, TOT, K + 1>::inv(v, e, o);
+    }
+  }
+};
+
+template <int N, int OFF, int S, int TOT>
+struct RdftP {
+  static_assert(N >= 4 && (N & (N - 1)) == 0, "N must be a power of two >= 4");
+  static __device__ __forceinline__ void fwd(float2 (&v)[TOT]) {
+    RdftP<N / 2, OFF, 2 * S, TOT>::fwd(v);
+    RdftP<N / 2, OFF + S, 2 * S, TOT>::fwd(v);
+    constexpr int M = N / 2;
+    float2 e[M], o[M];
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+      e[j] = v[OFF + 2 * S * j];
+      o[j] = v[OFF + S + 2 * S * j];
+    }
+    v[OFF] = p2add(e[0], o[0]);
+    v[OFF + S] = p2sub(e[0], o[0]);
+    v[OFF + S * M] = e[1];
+    v[OFF + S * (M + 1)] = p2sub(make_float2(0.0f, 0.0f), o[1]);
+    RdftBflyP<N, OFF, S, TOT, 1>::fwd(v, e, o);
+  }
+  static __device__ __forceinline__ void inv(float2 (&v)[TOT]) {
+    constexpr int M = N / 2;
+    float2 e[M], o[M];
+    const float2 x0 = v[OFF], xn = v[OFF + S];
+    e[0] = p2add(x0, xn);
+    o[0] = p2sub(x0, xn);
+    e[1] = v[OFF + S * M];
+    o[1] = p2sub(make_float2(0.0f, 0.0f), v[OFF + S * (M + 1)]);
+    RdftBflyP<N, OFF, S, TOT, 1>::inv(v, e, o);
+#pragma unroll
+    for (int j = 0; j < M; ++j) {
+      v[OFF + 2 * S * j] = e[j];
+      v[OFF + S + 2 * S * j] = o[j];
+    }
+    RdftP<N / 2, OFF, 2 * S, TOT>::inv(v);
+    RdftP<N / 2, OFF + S, 2 * S, TOT>::inv(v);
+  }
+};
+
+template <int OFF, int S, int TOT>
+struct RdftP<2, OFF, S, TOT> {
+  static __device__ __forceinline__ void fwd(float2 (&v)[TOT]) {
+    const float2 a = v[OFF], b = v[OFF + S];
+    v[OFF] = p2add(a, b);
+    v[OFF + S] = p2sub(a, b);
+  }
+  static __device__ __forceinline__ void inv(float2 (&v)[TOT]) { fwd(v); }
+};
+
+// Top stage (scalar) of a size-N transform whose even/odd halves were transformed
+// packed: in v[j] = (E slot j, O slot j), out v[k] = (Re X_k, Im X_k) for
+// 1 <= k < N/2 and v[0] = (X_0, X_{N/2}) -- the same slot order as rdft_fwd.
+template <int N, int K>
+__device__ __forceinline__ void rdft_top_bfly(float2 (&v)[N / 2], const float (&e)[N / 2], const float (&o)[N / 2]) {
+  if constexpr (K < N / 4) {
+    constexpr float c = static_cast<float>(cos2pi_frac(K, N));
+    constexpr float s = static_cast<float>(sin2pi_frac(K, N));
+    const float er = e[2 * K], ei = e[2 * K + 1], orr = o[2 * K], oi = o[2 * K + 1];
+    const float xr = fmaf(c, orr, fmaf(s, oi, er));
+    const float xi = fmaf(c, oi, fmaf(-s, orr, ei));
+    v[K] = make_float2(xr, xi);
+    v[N / 2 - K] = make_float2(fmaf(2.0f, er, -xr), fmaf(-2.0f, ei, xi));
+    rdft_top_bfly<N, K + 1>(v, e, o);
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void rdft_fwd_packed(float2 (&v)[N / 2]) {
+  RdftP<N / 2, 0, 1, N / 2>::fwd(v);
+  float e[N / 2], o[N / 2];
+#pragma unroll
+  for (int j = 0; j < N / 2; ++j) {
+    e[j] = v[j].x;
+    o[j] = v[j].y;
+  }
+  v[0] = make_float2(e[0] + o[0], e[0] - o[0]);
+  v[N / 4] = make_float2(e[1], -o[1]);
+  rdft_top_bfly<N, 1>(v, e, o);
+}
+
+// Exact transpose of rdft_fwd_packed: slots in, (x[2m], x[2m+1]) pairs out.
+template <int N, int K>
+__device__ __forceinline__ void rdft_top_bfly_inv(const float2 (&v)[N / 2], float (&e)[N / 2], float (&o)[N / 2]) {
+  if constexpr (K < N / 4) {
+    constexpr float c = static_cast<float>(cos2pi_frac(K, N));
+    constexpr float s = static_cast<float>(sin2pi_frac(K, N));
+    const float ar = v[K].x, ai = v[K].y, br = v[N / 2 - K].x, bi = v[N / 2 - K].y;
+    e[2 * K] = ar + br;
+    e[2 * K + 1] = ai - bi;
+    const float dr = ar - br, di = ai + bi;
+    o[2 * K] = fmaf(c, dr, -s * di);
+    o[2 * K + 1] = fmaf(s, dr, c * di);
+    rdft_top_bfly_inv<N, K + 1>(v, e, o);
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void rdft_inv_packed(float2 (&v)[N / 2]) {
+  float e[N / 2], o[N / 2];
+  e[0] = v[0].x + v[0].y;
+  o[0] = v[0].x - v[0].y;
+  e[1] = v[N / 4].x;
+  o[1] = -v[N / 4].y;
+  rdft_top_bfly_inv<N, 1>(v, e, o);
+#pragma unroll
+  for (int j = 0; j < N / 2; ++j) v[j] = make_float2(e[j], o[j]);
+  RdftP<N / 2, 0, 1, N / 2>::inv(v);
+}
+
 // Rotated channel c (DC, cos1, sin1, ..., Nyquist order) <-> spectrum slot.
 __host__ __device__ constexpr int slot_of_channel(int c, int N) { return c == 0 ? 0 : (c == N - 1 ? 1 : c + 1); }
 
