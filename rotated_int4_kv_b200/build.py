@@ -1,6 +1,7 @@
 """Build the in-tree shared library ``libkvq.so`` (CUDA C++ for sm_100a) with nvcc.
 
-Usage: ``python -m rotated_int4_kv_b200.build [--force] [--verbose]``. Object files
+Usage: ``python rotated_int4_kv_b200/build.py [--force] [--verbose]`` (run it as a script:
+importing the package loads the library it builds). Object files
 go to ``_build/`` at the repository root; the library is written next to this file.
 """
 from __future__ import annotations
