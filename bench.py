@@ -53,6 +53,22 @@ def _algo_bytes(D: int, G: int = 32):
     return vec, tok
 
 
+# ---------------------------------------------------------------- multi-rank helpers
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise max of per-rank timings (all ranks call it, in the same order)."""
+    if dist is None:
+        return [float(v) for v in values]
+    import torch
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_throughput(world: int, units_per_rank: int, ms_total: float, steps: int) -> float:
+    """Whole-job units/s (in millions) for weak scaling: every rank processes units_per_rank per step."""
+    return world * units_per_rank / (ms_total / steps * 1e-3) / 1e6
+
+
 # ---------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi clock/throttle sampling in the background (100 ms period)."""
@@ -315,12 +331,7 @@ def run_kvq(args, rank: int, world: int):
     ms = t_start.elapsed_time(t_end)
     enc_ms = [a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]
     att_ms = [ev_b[s].elapsed_time(ev_a[s + 1]) for s in range(args.steps - 1)] + [ev_b[-1].elapsed_time(t_end)]
-    if dist is not None:
-        t = torch.tensor([ms, float(np.mean(enc_ms)), float(np.mean(att_ms))], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, enc_avg, att_avg = (float(v) for v in t.tolist())
-    else:
-        enc_avg, att_avg = float(np.mean(enc_ms)), float(np.mean(att_ms))
+    ms, enc_avg, att_avg = max_over_ranks([ms, float(np.mean(enc_ms)), float(np.mean(att_ms))], dist, dev)
     assert kvq.poll_device_errors() == 0
 
     # ---- end to end through the C ABI with host buffers (pinned), copies in the timed region
@@ -348,7 +359,7 @@ def run_kvq(args, rank: int, world: int):
     d2h = out.numel() * 2
 
     vec_step = NJ * Hkv * T
-    value = world * vec_step / (ms / args.steps * 1e-3) / 1e6
+    value = job_throughput(world, vec_step, ms, args.steps)
     hbm, peak_kind = _peaks()
     enc_gbs = vec_step * vec_b / (enc_avg * 1e-3) / 1e9
     att_bytes = L * Hkv * T * tok_b
