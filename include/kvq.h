@@ -169,6 +169,32 @@ kvq_status kvq_attend_decode(const kvq_plan* pk, const kvq_plan* pv, const uint1
                              size_t ws_bytes, void* stream);
 
 /*
+ * kvq_attend_decode_noalloc -- kvq_attend_decode for callers that cannot allocate
+ * device memory: a serving runtime whose memory is planned up front, code that
+ * runs while a stream is being captured (cudaMalloc is not allowed there), or a
+ * host where another component owns the allocator. The paper has no counterpart;
+ * this is a library convenience.
+ * Same arguments and results as kvq_attend_decode, without the workspace: the
+ * scratch is one file-scope device array of 8 MiB inside the library (every GPU
+ * that loads the library holds it until the process exits). Shapes whose split
+ * needs more than 8 MiB of scratch are rejected with KVQ_ERR_WORKSPACE before
+ * anything is launched (use kvq_attend_decode for those).
+ * No cudaMalloc, cudaFree or allocating library call is made. The first call on
+ * a device looks up the array's device address (cudaGetSymbolAddress with that
+ * device current); make that first call before any stream capture. Each call
+ * clears the array's counters with a stream-ordered memset before its kernels.
+ * All calls share the one array and it keeps the last call's contents, so calls
+ * whose executions overlap on the GPU (other streams, other host threads, or
+ * graph branches) race and must be serialised by the caller.
+ * Errors: as kvq_attend_decode.
+ */
+kvq_status kvq_attend_decode_noalloc(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q,
+                                     const uint8_t* k_codes, const uint16_t* k_scales,
+                                     const uint8_t* v_codes, const uint16_t* v_scales, int B, int Hq,
+                                     int Hkv, int T_cap, const int32_t* seq_lens, int T_len,
+                                     float softmax_scale, uint16_t* out, void* stream);
+
+/*
  * kvq_attend_decode_ref -- the fp16-cache comparator for the same shapes: the same
  * split-sequence softmax attention over fp16 K/V [B, Hkv, T_cap, D] with no
  * rotation. This is the uncompressed baseline the int4 path is measured against

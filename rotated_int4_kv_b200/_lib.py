@@ -42,6 +42,7 @@ def _load() -> ctypes.CDLL:
         "kvq_workspace_size": (S, [I, I, I, I, I]),
         "kvq_attend_decode": (I, [P, P, P, P, P, P, P, I, I, I, I, P, I, F, P, P, S, P]),
         "kvq_attend_decode_ref": (I, [P, P, P, I, I, I, I, I, P, I, F, P, P, S, P]),
+        "kvq_attend_decode_noalloc": (I, [P, P, P, P, P, P, P, I, I, I, I, P, I, F, P, P]),
         "kvq_poll_device_errors": (I, [U32P]),
         "kvq_status_string": (ctypes.c_char_p, [I]),
         "kvq_last_error": (ctypes.c_char_p, []),

@@ -145,6 +145,32 @@ def attend_decode(pk: Plan, pv: Plan, q, k_codes, k_scales, v_codes, v_scales, s
     return out
 
 
+def attend_decode_noalloc(pk: Plan, pv: Plan, q, k_codes, k_scales, v_codes, v_scales, seq_lens=None, T_len=None,
+                          softmax_scale: float = 0.0, out=None, stream=None) -> torch.Tensor:
+    """kvq_attend_decode_noalloc: the int4 decode attention for callers that cannot
+    allocate device memory; its scratch is a static array inside the library
+    (8 MiB, shared by all calls: calls that overlap on the GPU race)."""
+    B, Hq, D = q.shape
+    _, Hkv, T_cap, half = k_codes.shape
+    _need(q, "q", torch.float16)
+    for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
+        _need(t, name, torch.uint8, (B, Hkv, T_cap, D // 2))
+    for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+        _need(t, name, torch.float16, (B, Hkv, T_cap, D // pk.group))
+    if seq_lens is not None:
+        _need(seq_lens, "seq_lens", torch.int32, (B,))
+    if T_len is None:
+        T_len = T_cap if seq_lens is None else 0
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float16, device=q.device)
+    _need(out, "out", torch.float16, (B, Hq, D))
+    check(lib.kvq_attend_decode_noalloc(pk.handle, pv.handle, _ptr(q), _ptr(k_codes), _ptr(k_scales),
+                                        _ptr(v_codes), _ptr(v_scales), B, Hq, Hkv, T_cap, _ptr(seq_lens),
+                                        int(T_len), float(softmax_scale), _ptr(out), _stream(stream)),
+          "kvq_attend_decode_noalloc")
+    return out
+
+
 def attend_decode_ref(q, k, v, seq_lens=None, T_len=None, softmax_scale: float = 0.0, out=None, workspace=None,
                       stream=None) -> torch.Tensor:
     """The fp16-cache comparator kernel on the same shapes."""

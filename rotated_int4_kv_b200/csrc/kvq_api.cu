@@ -376,6 +376,30 @@ kvq_status kvq_attend_decode(const kvq_plan* pk, const kvq_plan* pv, const uint1
                                  ws_bytes, (cudaStream_t)stream);
 }
 
+kvq_status kvq_attend_decode_noalloc(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q, const uint8_t* kc,
+                                     const uint16_t* ks, const uint8_t* vc, const uint16_t* vs, int B, int Hq,
+                                     int Hkv, int T_cap, const int32_t* seq_lens, int T_len, float sigma,
+                                     uint16_t* out, void* stream) {
+  if (!pk || !pv) return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: null plan");
+  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device)
+    return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: K and V plans differ in head_dim, group or device");
+  if (pk->G != 32) return fail(KVQ_ERR_UNSUPPORTED, "attend_noalloc: group must be 32");
+  if (B < 0 || Hq <= 0 || Hkv <= 0 || T_cap < 0) return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: bad sizes");
+  if (Hq % Hkv) return fail(KVQ_ERR_UNSUPPORTED, "attend_noalloc: Hq must be a multiple of Hkv");
+  if (T_cap & 1) return fail(KVQ_ERR_ALIGNMENT, "attend_noalloc: T_cap must be even");
+  if (T_len < 0) return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: T_len < 0");
+  if (T_len > T_cap) return fail(KVQ_ERR_CAPACITY, "attend_noalloc: T_len > T_cap");
+  if (B == 0) return KVQ_OK;
+  if (!q || !out || !kc || !ks || !vc || !vs) return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: null buffer");
+  if (!kvq::aligned16(q) || !kvq::aligned16(out) || !kvq::aligned16(kc) || !kvq::aligned16(ks) ||
+      !kvq::aligned16(vc) || !kvq::aligned16(vs))
+    return fail(KVQ_ERR_ALIGNMENT, "attend_noalloc: buffers must be 16-byte aligned");
+  kvq_status st = kvq::check_plan_device(pk);
+  if (st != KVQ_OK) return st;
+  return kvq::launch_attend_int4_noalloc(pk, pv, q, kc, ks, vc, vs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, out,
+                                         (cudaStream_t)stream);
+}
+
 kvq_status kvq_attend_decode_ref(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq, int Hkv,
                                  int D, int T_cap, const int32_t* seq_lens, int T_len, float sigma, uint16_t* out,
                                  void* ws, size_t ws_bytes, void* stream) {

@@ -850,6 +850,67 @@ kvq_status launch_attend_fp16(const uint16_t* q, const uint16_t* k, const uint16
                                 out, ws, ws_bytes, s);
 }
 
+// ---------------------------------------------------------------- allocation-free variant
+// Callers that cannot allocate device memory (a serving runtime whose memory is
+// planned up front, code that runs while a stream is being captured, where
+// cudaMalloc is not allowed, or hosts where another component owns the
+// allocator) use kvq_attend_decode_noalloc. Its workspace is this file-scope
+// array: every GPU that loads the library holds it until the process exits,
+// and every call shares it.
+constexpr size_t kNoAllocScratchBytes = 8u << 20;  // 8 MiB
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_scratch_mu;
+void* g_scratch_ptr[64] = {nullptr};
+
+// The host-side name of g_noalloc_scratch is not a device address: resolve the
+// real one once per device, with that device current.
+kvq_status noalloc_scratch(int dev, void** out) {
+  if (dev < 0 || dev >= 64) return fail(KVQ_ERR_DEVICE, "attend_noalloc: device index out of range");
+  std::lock_guard<std::mutex> lk(g_scratch_mu);
+  if (!g_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+    if (e != cudaSuccess || !ptr)
+      return fail(KVQ_ERR_CUDA, std::string("attend_noalloc: cudaGetSymbolAddress failed: ") + cudaGetErrorString(e));
+    g_scratch_ptr[dev] = ptr;
+  }
+  *out = g_scratch_ptr[dev];
+  return KVQ_OK;
+}
+}  // namespace
+
+kvq_status launch_attend_int4_noalloc(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q, const uint8_t* kc,
+                                      const uint16_t* ks, const uint8_t* vc, const uint16_t* vs, int B, int Hq,
+                                      int Hkv, int T_cap, const int32_t* seq_lens, int T_len, float sigma,
+                                      uint16_t* out, cudaStream_t s) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return fail(KVQ_ERR_DEVICE, "attend_noalloc: no current device");
+  const int D = pk->D;
+  // the exact split the launch will choose, hence the exact scratch it needs
+  const int per_sm = D == 128 ? std::min(ctas_per_sm<128, true>(), kMaxPerSmForSizing)
+                              : std::min(ctas_per_sm<256, true>(), kMaxPerSmForSizing);
+  const SplitPlan sp = choose_split(B, Hq, Hkv, seq_lens ? T_cap : T_len, num_sms(dev), per_sm);
+  const size_t need = ws_bytes_for(B, Hq, Hkv, D, sp.S, sp.HT);
+  if (need > kNoAllocScratchBytes)
+    return fail(KVQ_ERR_WORKSPACE, "attend_noalloc: these shapes need " + std::to_string(need) +
+                                       " bytes of scratch; the static scratch holds " +
+                                       std::to_string(kNoAllocScratchBytes) + " (use kvq_attend_decode)");
+  void* scratch = nullptr;
+  kvq_status st = noalloc_scratch(dev, &scratch);
+  if (st != KVQ_OK) return st;
+  // the split counters must start at zero; the array keeps the previous call's contents
+  const size_t units = (size_t)B * Hkv * sp.HT;
+  const cudaError_t e = cudaMemsetAsync(scratch, 0, ws_cnt_bytes(units), s);
+  if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("attend_noalloc: memset: ") + cudaGetErrorString(e));
+  if (D == 128)
+    return run_attend<128, true>(pk, pv, q, kc, ks, vc, vs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, out, scratch,
+                                 kNoAllocScratchBytes, s);
+  return run_attend<256, true>(pk, pv, q, kc, ks, vc, vs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, out, scratch,
+                               kNoAllocScratchBytes, s);
+}
+
 uint32_t attend_error_flags(bool clear) {
   uint32_t v = 0;
   cudaMemcpyFromSymbol(&v, g_attend_err, sizeof(v));

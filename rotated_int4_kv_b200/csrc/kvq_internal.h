@@ -65,6 +65,11 @@ kvq_status launch_attend_int4(const kvq_plan* pk, const kvq_plan* pv, const uint
                               const uint8_t* kc, const uint16_t* ks, const uint8_t* vc, const uint16_t* vs,
                               int B, int Hq, int Hkv, int T_cap, const int32_t* seq_lens, int T_len,
                               float sigma, uint16_t* out, void* ws, size_t ws_bytes, cudaStream_t s);
+kvq_status launch_attend_int4_noalloc(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q,
+                                      const uint8_t* kc, const uint16_t* ks, const uint8_t* vc,
+                                      const uint16_t* vs, int B, int Hq, int Hkv, int T_cap,
+                                      const int32_t* seq_lens, int T_len, float sigma, uint16_t* out,
+                                      cudaStream_t s);
 kvq_status launch_attend_fp16(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
                               int Hkv, int D, int T_cap, const int32_t* seq_lens, int T_len, float sigma,
                               uint16_t* out, void* ws, size_t ws_bytes, cudaStream_t s);

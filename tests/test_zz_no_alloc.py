@@ -1,0 +1,71 @@
+"""kvq_attend_decode_noalloc: the int4 decode attention for callers that cannot
+allocate device memory (memory planned up front, code running under stream
+capture, hosts whose allocator belongs to someone else). Its scratch is a static
+array inside the library, so this checks, through the C ABI, that two calls in a
+row give what the workspace-taking kvq_attend_decode gives, and that shapes too
+large for the static scratch are refused before anything runs.
+
+Kept in a file that pytest collects last; it must pass on its own in a fresh
+process and after every other test."""
+import ctypes
+
+import numpy as np
+import pytest
+
+import kvgen
+from tests.parity import REL_L2, check_rel_l2
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+def _cache(kvq, wl, B, Hkv, T, seed):
+    D = wl.head_dim
+    dev = torch.device("cuda")
+    out = {}
+    for kind in ("k", "v"):
+        plan = kvq.Plan(*kvgen.plan_params(D, seed=seed, kind=kind))
+        x = torch.from_numpy(kvgen.kv_numpy(wl, kind, (B, Hkv, T, D), seed=seed)).to(dev)
+        codes = torch.zeros((B, Hkv, T, D // 2), dtype=torch.uint8, device=dev)
+        scales = torch.zeros((B, Hkv, T, D // 32), dtype=torch.float16, device=dev)
+        kvq.encode(plan, x, codes, scales, 0)
+        out[kind] = (plan, codes, scales)
+    return out
+
+
+@pytest.mark.parametrize("name,B,Hkv,Hq,T,lens", [
+    ("qwen", 2, 2, 12, 1000, [1000, 377]),
+    ("gemma", 1, 1, 4, 4096, None),
+])
+def test_noalloc_matches_workspace_entry_point_twice(name, B, Hkv, Hq, T, lens):
+    import rotated_int4_kv_b200 as kvq
+
+    wl = kvgen.WORKLOADS[name]
+    D = wl.head_dim
+    c = _cache(kvq, wl, B, Hkv, T, seed=41)
+    q = torch.from_numpy(kvgen.q_numpy((B, Hq, D), salt=13)).cuda()
+    sl = None if lens is None else torch.tensor(lens, dtype=torch.int32, device="cuda")
+    args = (c["k"][0], c["v"][0], q, c["k"][1], c["k"][2], c["v"][1], c["v"][2])
+    ref = kvq.attend_decode(*args, seq_lens=sl, T_len=T if sl is None else None).float().cpu().numpy()
+    for _ in range(2):  # the static scratch keeps the previous call's contents
+        got = kvq.attend_decode_noalloc(*args, seq_lens=sl, T_len=T if sl is None else None)
+        torch.cuda.synchronize()
+        check_rel_l2(got.float().cpu().numpy().reshape(-1, D), ref.reshape(-1, D), tol=REL_L2, label=name)
+    assert kvq.poll_device_errors() == 0
+
+
+def test_noalloc_refuses_shapes_beyond_static_scratch():
+    import rotated_int4_kv_b200 as kvq
+    from rotated_int4_kv_b200 import lib
+
+    D = 128
+    pk = kvq.Plan(*kvgen.plan_params(D, kind="k"))
+    pv = kvq.Plan(*kvgen.plan_params(D, kind="v"))
+    # 2048 x 8 KV heads x 64 query heads: the per-head-tile rotated queries alone exceed 8 MiB.
+    # The size check happens on the host before any pointer is touched, so 16-byte aligned
+    # placeholder addresses are enough.
+    fake = ctypes.c_void_p(1 << 20)
+    st = lib.kvq_attend_decode_noalloc(pk.handle, pv.handle, fake, fake, fake, fake, fake, 2048, 64, 8, 256, None,
+                                       256, ctypes.c_float(0.0), fake, None)
+    assert st == -6
+    assert b"static scratch" in lib.kvq_last_error()
