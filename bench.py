@@ -399,12 +399,147 @@ def run_kvq(args, rank: int, world: int):
     return 0
 
 
+# ---------------------------------------------------------------- other workloads (decode-attention table)
+def _graph_time(torch, fn, steps, warmup):
+    """Capture fn() (one step) in a CUDA graph and time `steps` replays (ms per step)."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.graph(g, stream=s):
+        fn()
+    for _ in range(warmup):
+        g.replay()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(steps):
+        g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    g.reset()
+    return a.elapsed_time(b) / steps
+
+
+def run_decode_workload(args, rank: int, world: int):
+    """Decode-step workloads: per layer, append-encode one token of K and V (one grouped
+    launch) and run one-query decode attention, int4 against the fp16 comparator
+    (fp16 step = one-token K/V append copy + fp16 attention). Steps are CUDA graphs."""
+    import torch
+
+    import rotated_int4_kv_b200 as kvq
+
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = kvgen.WORKLOADS[args.workload]
+    D, Hkv, Hq, B, G = wl.head_dim, wl.h_kv, wl.h_q, wl.batch, wl.group
+    seed = kvgen.DEFAULT_SEED + 1000 * rank
+    hbm, _ = _peaks()
+    vec_b, tok_b = _algo_bytes(D, G)
+    contexts = wl.contexts if args.contexts is None else tuple(int(c) for c in args.contexts.split(","))
+    layers = wl.layers if args.layers is None else args.layers
+    distinct = min(layers, max(1, args.distinct_layers))
+    cases = []
+    for T in contexts:
+        T_cap = T + 2
+        plans, caches, caches16 = [], [], []
+        for l in range(distinct):
+            pk = kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=l, kind="k"))
+            pv = kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=l, kind="v"))
+            plans.append((pk, pv))
+            c = {}
+            for kind, pl in (("k", pk), ("v", pv)):
+                codes = torch.zeros((B, Hkv, T_cap, D // 2), dtype=torch.uint8, device=dev)
+                scales = torch.zeros((B, Hkv, T_cap, D // G), dtype=torch.float16, device=dev)
+                x16 = torch.zeros((B, Hkv, T_cap, D), dtype=torch.float16, device=dev)
+                for b in range(B):
+                    kvgen.kv_torch(wl, kind, (1, Hkv, T, D), dev, seed=seed, layer=l, salt=b, out=x16[b:b + 1, :, :T])
+                    kvq.encode(pl, x16[b:b + 1, :, :T].contiguous(), codes[b:b + 1], scales[b:b + 1], 0)
+                c[kind] = (codes, scales)
+                caches16.append(x16) if kind == "k" else caches16.append(x16)
+            caches.append(c)
+        k16s = caches16[0::2]
+        v16s = caches16[1::2]
+        q = [kvgen.q_torch((B, Hq, D), dev, seed=seed, layer=l) for l in range(distinct)]
+        newk = [kvgen.kv_torch(wl, "k", (B, Hkv, 1, D), dev, seed=seed, layer=l, salt=99) for l in range(distinct)]
+        newv = [kvgen.kv_torch(wl, "v", (B, Hkv, 1, D), dev, seed=seed, layer=l, salt=98) for l in range(distinct)]
+        out = torch.empty((B, Hq, D), dtype=torch.float16, device=dev)
+        ws = [kvq.make_workspace(B, Hq, Hkv, D, T_cap, dev) for _ in range(distinct)]
+
+        def step_int4():
+            for l in range(layers):
+                d = l % distinct
+                pk, pv = plans[d]
+                kc, ks = caches[d]["k"]
+                vc, vs = caches[d]["v"]
+                kvq.encode_batch([(pk, newk[d], kc, ks, T), (pv, newv[d], vc, vs, T)])
+                kvq.attend_decode(pk, pv, q[d], kc, ks, vc, vs, T_len=T + 1, out=out, workspace=ws[d])
+
+        def step_fp16():
+            for l in range(layers):
+                d = l % distinct
+                k16s[d][:, :, T:T + 1].copy_(newk[d])
+                v16s[d][:, :, T:T + 1].copy_(newv[d])
+                kvq.attend_decode_ref(q[d], k16s[d], v16s[d], T_len=T + 1, out=out, workspace=ws[d])
+
+        def attn_only_int4():
+            for l in range(layers):
+                d = l % distinct
+                pk, pv = plans[d]
+                kvq.attend_decode(pk, pv, q[d], *caches[d]["k"], *caches[d]["v"], T_len=T + 1, out=out,
+                                  workspace=ws[d])
+
+        def attn_only_fp16():
+            for l in range(layers):
+                d = l % distinct
+                kvq.attend_decode_ref(q[d], k16s[d], v16s[d], T_len=T + 1, out=out, workspace=ws[d])
+
+        ms4 = _graph_time(torch, step_int4, args.steps, args.warmup)
+        ms16 = _graph_time(torch, step_fp16, args.steps, args.warmup)
+        a4 = _graph_time(torch, attn_only_int4, args.steps, args.warmup)
+        a16 = _graph_time(torch, attn_only_fp16, args.steps, args.warmup)
+        assert kvq.poll_device_errors() == 0
+        tokheads = layers * B * Hkv * (T + 1)
+        cases.append({
+            "T": T, "layers": layers, "distinct_layer_caches": distinct,
+            "int4_step_ms": ms4, "fp16_step_ms": ms16, "step_speedup": ms16 / ms4,
+            "int4_attn_ms": a4, "fp16_attn_ms": a16, "attn_speedup": a16 / a4,
+            "int4_tokens_heads_per_s": tokheads / (a4 * 1e-3),
+            "int4_attn_GB_s": tokheads * tok_b / (a4 * 1e-3) / 1e9,
+            "int4_frac_hbm": tokheads * tok_b / (a4 * 1e-3) / 1e9 / hbm,
+            "fp16_attn_GB_s": tokheads * 4 * D / (a16 * 1e-3) / 1e9,
+            "fp16_frac_hbm": tokheads * 4 * D / (a16 * 1e-3) / 1e9 / hbm,
+            "l2": ("working set > L2 (HBM-bound)" if distinct * B * Hkv * T * tok_b > 126e6
+                   else "working set fits in L2: latency of an L2-warm decode loop"),
+        })
+        del caches, caches16, k16s, v16s
+        torch.cuda.empty_cache()
+    big = cases[-1]
+    line = {"metric": METRIC, "value": big["int4_attn_GB_s"], "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": big["int4_step_ms"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": args.workload, "layers": layers, "kv_heads": Hkv, "q_heads": Hq, "head_dim": D,
+                       "batch": B, "contexts": list(contexts), "group": G},
+            "cases": cases}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="kvq", choices=["kvq", "reference"])
+    ap.add_argument("--workload", default=WORKLOAD, choices=["gemma", "mistral", "qwen", "longctx"],
+                    help="gemma (default) = the headline prefill-encode step; the others time decode steps")
+    ap.add_argument("--contexts", default=None, help="comma-separated context lengths (decode workloads)")
+    ap.add_argument("--layers", type=int, default=None, help="layers per decode step (default: the model's)")
+    ap.add_argument("--distinct-layers", type=int, default=4,
+                    help="distinct per-layer caches cycled through a decode step (each > L2 for the big shapes)")
     ap.add_argument("--ncu", action="store_true",
                     help="profiling mode: run --steps eager steps without timing, for ncu captures")
     args = ap.parse_args(argv)
@@ -414,6 +549,8 @@ def main(argv=None):
     world = int(os.environ.get("WORLD_SIZE", "1"))
     if args.impl == "reference":
         return run_reference(args, rank, world)
+    if args.workload != WORKLOAD:
+        return run_decode_workload(args, rank, world)
     return run_kvq(args, rank, world)
 
 

@@ -71,9 +71,8 @@ typedef struct kvq_plan kvq_plan;
  *   group       G: channels per abs-max scale group (32; 16 also accepted).
  *   signs_host  host int8[D], every entry +1 or -1 (the fixed random sign vector s).
  *   lambda_host host float[D], every entry finite and > 0 (per-channel lambda).
- * Allocates a small device block on the current device (the plan's device):
- * s and lambda, and the rotation matrices the attention kernels use for the
- * query rotation and the output un-rotation (2 x D x D fp16 pairs).
+ * Allocates a small device block (under 4 KB) on the current device, the plan's
+ * device: the per-channel factors and sign masks derived from s and lambda.
  * Errors: INVALID_ARG, UNSUPPORTED, CUDA, DEVICE.
  */
 kvq_status kvq_plan_create(kvq_plan** out, int head_dim, int group, const int8_t* signs_host,

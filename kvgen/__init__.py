@@ -158,6 +158,10 @@ def kv_torch(wl: Workload, which: str, shape, device, seed: int = DEFAULT_SEED, 
     dist = wl.k_dist if which == "k" else wl.v_dist
     gains = torch.tensor(channel_gains(wl, which, seed, layer), dtype=torch.float32, device=device)
     shape = tuple(shape)
+    if out is not None and not out.is_contiguous():
+        tmp = kv_torch(wl, which, shape, device, seed=seed, layer=layer, salt=salt)
+        out.copy_(tmp)
+        return out
     if out is None:
         out = torch.empty(shape, dtype=torch.float16, device=device)
     # draw in slabs along the leading dims to bound the fp32 temporaries

@@ -45,48 +45,6 @@ double basis_dg(int c, int D) {
   return (c & 1) ? std::sqrt(2.0 / D) : -std::sqrt(2.0 / D);
 }
 
-// Row c of the orthonormal real basis at sample n (used only to build the
-// rotation matrices that the attention kernels apply with tensor cores).
-double basis_entry(int c, int n, int D) {
-  if (c == 0) return 1.0 / std::sqrt((double)D);
-  if (c == D - 1) return (n & 1) ? -1.0 / std::sqrt((double)D) : 1.0 / std::sqrt((double)D);
-  const int k = (c + 1) / 2;
-  const long m = ((long)k * n) % D;
-  const double ang = 2.0 * M_PI * (double)m / (double)D;
-  return (c & 1) ? std::sqrt(2.0 / D) * std::cos(ang) : std::sqrt(2.0 / D) * std::sin(ang);
-}
-
-uint16_t f2h_bits(float f) {
-  const __half h = __float2half_rn(f);
-  return __half_as_ushort(h);
-}
-float h2f(uint16_t b) { return __half2float(__ushort_as_half(b)); }
-
-// Fragment order of an m16n8k16 A operand (row-major 16x16 tile) for lane = 4g + c:
-// a0 = A[g][2c..2c+1], a1 = A[g+8][2c..2c+1], a2 = A[g][2c+8..2c+9], a3 = A[g+8][2c+8..2c+9].
-void build_frag(const std::vector<double>& A, int D, std::vector<uint32_t>& out) {
-  const int MT = D / 16;
-  out.assign((size_t)MT * MT * 2 * 32 * 4, 0u);
-  for (int mt = 0; mt < MT; ++mt)
-    for (int kt = 0; kt < MT; ++kt)
-      for (int hl = 0; hl < 2; ++hl)
-        for (int lane = 0; lane < 32; ++lane) {
-          const int g = lane >> 2, c = lane & 3;
-          const int rows[4] = {g, g + 8, g, g + 8};
-          const int cols[4] = {2 * c, 2 * c, 2 * c + 8, 2 * c + 8};
-          for (int r = 0; r < 4; ++r) {
-            uint32_t w = 0;
-            for (int e = 0; e < 2; ++e) {
-              const double a = A[(size_t)(mt * 16 + rows[r]) * D + kt * 16 + cols[r] + e];
-              const float af = (float)a;
-              const uint16_t hi = f2h_bits(af);
-              const uint16_t lo = f2h_bits((float)(a - (double)h2f(hi)));
-              w |= (uint32_t)(hl == 0 ? hi : lo) << (16 * e);
-            }
-            out[((((size_t)mt * MT + kt) * 2 + hl) * 32 + lane) * 4 + r] = w;
-          }
-        }
-}
 }  // namespace
 
 void set_error(const std::string& msg) { t_last_error = msg; }
@@ -228,34 +186,21 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
     p->enc.sgn[w] = m;
     p->dec.sgn[w] = m;
   }
-  // R' = Lambda^-1 F_r diag(s) and its transpose, as split-fp16 mma fragments
-  std::vector<double> R((size_t)D * D), RT((size_t)D * D);
-  for (int i = 0; i < D; ++i)
-    for (int j = 0; j < D; ++j) {
-      const double v = kvq::basis_entry(i, j, D) * (double)signs[j] / (double)lambda[i];
-      R[(size_t)i * D + j] = v;
-      RT[(size_t)j * D + i] = v;
-    }
-  std::vector<uint32_t> fq, fo;
-  kvq::build_frag(R, D, fq);
-  kvq::build_frag(RT, D, fo);
-  const size_t bytes = fq.size() * 4;
   void* blk = nullptr;
-  if (cudaMalloc(&blk, 2 * bytes + sizeof(kvq::CodecConsts)) != cudaSuccess) {
+  if (cudaMalloc(&blk, 2 * sizeof(kvq::CodecConsts)) != cudaSuccess) {
     delete p;
     return fail(KVQ_ERR_CUDA, "plan_create: cudaMalloc failed");
   }
-  if (cudaMemcpy(blk, fq.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
-      cudaMemcpy((char*)blk + bytes, fo.data(), bytes, cudaMemcpyHostToDevice) != cudaSuccess ||
-      cudaMemcpy((char*)blk + 2 * bytes, &p->enc, sizeof(kvq::CodecConsts), cudaMemcpyHostToDevice) != cudaSuccess) {
+  if (cudaMemcpy(blk, &p->enc, sizeof(kvq::CodecConsts), cudaMemcpyHostToDevice) != cudaSuccess ||
+      cudaMemcpy((char*)blk + sizeof(kvq::CodecConsts), &p->dec, sizeof(kvq::CodecConsts), cudaMemcpyHostToDevice) !=
+          cudaSuccess) {
     cudaFree(blk);
     delete p;
     return fail(KVQ_ERR_CUDA, "plan_create: upload failed");
   }
   p->dblock = blk;
-  p->rq_frag = reinterpret_cast<const uint4*>(blk);
-  p->ro_frag = reinterpret_cast<const uint4*>((char*)blk + bytes);
-  p->enc_dev = reinterpret_cast<const kvq::CodecConsts*>((char*)blk + 2 * bytes);
+  p->enc_dev = reinterpret_cast<const kvq::CodecConsts*>(blk);
+  p->dec_dev = reinterpret_cast<const kvq::CodecConsts*>((char*)blk + sizeof(kvq::CodecConsts));
   *out = p;
   return KVQ_OK;
 }

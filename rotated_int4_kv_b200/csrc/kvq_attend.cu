@@ -24,16 +24,18 @@
 //     into P per group. Online softmax runs in base 2;
 //   * warps merge in shared memory, the CTA writes (m, l, o) to the workspace,
 //     and the last CTA of a (b, kv head, head tile) -- found with an atomic
-//     counter, no waiting -- merges the splits, un-rotates with R'_V^T on the
-//     tensor cores (split-fp16 operands, fp32 accumulate) and writes fp16.
-// The query rotation uses the same split-fp16 mma on R'_K. Tensor cores are used
-// for issue rate, not throughput: the kernel is bound by HBM bandwidth.
+//     counter, no waiting -- merges the splits and un-rotates with the inverse
+//     register FFT (o = diag(s_V) F_r^T Lambda_V^-1 o_t), then writes fp16.
+// The query is rotated inside every CTA with the forward register FFT while the
+// producer's first loads are in flight. Tensor cores are used for issue rate,
+// not throughput: the kernel is bound by HBM bandwidth.
 #include <algorithm>
 #include <cstdio>
 #include <mutex>
 
 #include "kvq_internal.h"
 #include "kvq_ptx.cuh"
+#include "srft_fft.cuh"
 
 namespace kvq {
 
@@ -46,6 +48,7 @@ constexpr int kThreads = (kCWarps + 1) * 32;
 constexpr int kTileT = 16 * kCWarps;       // tokens per stage
 constexpr int kHT = 8;                     // query heads per CTA (mma N)
 constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kMaxSplitsCfg = 256;          // upper bound on splits per unit
 
 template <int D, bool INT4>
 struct Cfg {
@@ -60,7 +63,9 @@ struct Cfg {
   // warp-merge scratch (reuses the stage ring): per warp m[8], l[8], o[8][D]
   static constexpr int kWarpState = (2 * kHT + kHT * D) * 4;
   static constexpr int kRing = kStages * kStageBytes;
-  static constexpr int kScratch = kCWarps * kWarpState > kRing ? kCWarps * kWarpState : kRing;
+  static constexpr int kTail = (2 * kMaxSplitsCfg * kHT + kHT * D) * 4;  // merge m/l/weights + un-rotated output
+  static constexpr int kScratch0 = kCWarps * kWarpState > kRing ? kCWarps * kWarpState : kRing;
+  static constexpr int kScratch = kScratch0 > kTail ? kScratch0 : kTail;
   static constexpr int kQt = kHT * D * 4;                  // fp32 q_t (or merged o_t) [8][D]
   static constexpr int kSmem = kScratch + kQt + 64 + 1024;
 };
@@ -73,61 +78,10 @@ struct AttnParams {
   float sl2;                                   // softmax scale * log2(e)
   float* part;                                 // [units][S][2*8 + 8*D]
   int* cnt;                                    // [units]
-  const float* qt;                             // rotated queries [units][8][D] (int4 only; from qrot_kernel)
-  const uint4* ro;                             // R'_V^T fragments (int4 only)
+  const CodecConsts* ke;                       // K plan: sign masks (int4 only)
+  const CodecConsts* kd;                       // K plan: dg / lambda per channel
+  const CodecConsts* vd;                       // V plan: dg / lambda per channel, sign masks
 };
-
-__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void griddep_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
-// Query rotation, once per (b, kv head, head tile): q_t[h][i] = sum_j R'[i][j] q[h][j]
-// with R' = Lambda_K^-1 F_r diag(s_K) as split fp16 (hi + lo) A fragments and q
-// (exact fp16) as B; fp32 accumulate. Every fragment load of a warp's m-tile is
-// issued before its mma chain. The attention kernel is launched as a programmatic
-// dependent of this one and waits for it only before reading q_t.
-template <int D>
-__global__ void __launch_bounds__(256) qrot_kernel(const uint16_t* __restrict__ q, const uint4* __restrict__ rq,
-                                                   float* __restrict__ qt, int Hq, int Hkv, int G, int HT) {
-  griddep_launch_dependents();
-  constexpr int MT = D / 16;
-  const int unit = blockIdx.x;
-  const int bk = unit / HT, ht = unit - bk * HT;
-  const int b = bk / Hkv, kvh = bk - b * Hkv;
-  const int heads = min(kHT, G - ht * kHT);
-  const int hq0 = kvh * G + ht * kHT;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int g = lane >> 2, c = lane & 3;
-  const uint16_t* qb = q + ((size_t)b * Hq + hq0) * D;
-  float* out = qt + (size_t)unit * kHT * D;
-  uint32_t bq0[MT], bq1[MT];
-#pragma unroll
-  for (int kt = 0; kt < MT; ++kt) {
-    bq0[kt] = bq1[kt] = 0u;
-    if (g < heads) {
-      const uint16_t* qh = qb + (size_t)g * D + kt * 16 + 2 * c;
-      bq0[kt] = __ldg(reinterpret_cast<const uint32_t*>(qh));
-      bq1[kt] = __ldg(reinterpret_cast<const uint32_t*>(qh + 8));
-    }
-  }
-  for (int mt = warp; mt < MT; mt += 8) {
-    uint4 ah[MT], al[MT];
-#pragma unroll
-    for (int kt = 0; kt < MT; ++kt) {
-      ah[kt] = __ldg(rq + (((size_t)mt * MT + kt) * 2 + 0) * 32 + lane);
-      al[kt] = __ldg(rq + (((size_t)mt * MT + kt) * 2 + 1) * 32 + lane);
-    }
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int kt = 0; kt < MT; ++kt) {
-      mma_16816(acc, ah[kt].x, ah[kt].y, ah[kt].z, ah[kt].w, bq0[kt], bq1[kt]);
-      mma_16816(acc, al[kt].x, al[kt].y, al[kt].z, al[kt].w, bq0[kt], bq1[kt]);
-    }
-    out[(2 * c) * D + mt * 16 + g] = acc[0];
-    out[(2 * c + 1) * D + mt * 16 + g] = acc[1];
-    out[(2 * c) * D + mt * 16 + g + 8] = acc[2];
-    out[(2 * c + 1) * D + mt * 16 + g + 8] = acc[3];
-  }
-}
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
@@ -164,8 +118,137 @@ __device__ __forceinline__ void split_h(float x, __half& hi, __half& lo) {
   lo = __float2half_rn(x - __half2float(hi));
 }
 
+// q_t = Lambda_K^-1 F_r diag(s_K) q for the real heads of a tile, by the register
+// FFT: one lane per head at D = 128, a lane pair per head at D = 256 (all 32
+// lanes of the calling warp execute it; lanes beyond the real heads work on zeros).
+template <int D>
+__device__ __forceinline__ void rotate_query(const uint16_t* __restrict__ qb, int heads, const CodecConsts* ke,
+                                             const CodecConsts* kd, float* qt, int lane) {
+  float2 v[64];
+  if constexpr (D == 128) {
+    const int h = lane;
+    const bool live = h < heads;
+    const uint4* src = reinterpret_cast<const uint4*>(qb + (size_t)(live ? h : 0) * D);
+#pragma unroll
+    for (int cc = 0; cc < 16; ++cc) {
+      uint4 w = live ? __ldg(src + cc) : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 m = __ldg(reinterpret_cast<const uint4*>(ke->sgn) + cc);
+      const uint32_t ww[4] = {w.x ^ m.x, w.y ^ m.y, w.z ^ m.z, w.w ^ m.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) v[4 * cc + q] = __half22float2(*reinterpret_cast<const __half2*>(&ww[q]));
+    }
+    rdft_fwd_packed<128>(v);
+    if (live) {
+#pragma unroll
+      for (int c4 = 0; c4 < 32; ++c4) {
+        const float4 k4 = __ldg(reinterpret_cast<const float4*>(kd->chan) + c4);
+        float4 o;
+        o.x = slotv(v, slot_of_channel(4 * c4 + 0, 128)) * k4.x;
+        o.y = slotv(v, slot_of_channel(4 * c4 + 1, 128)) * k4.y;
+        o.z = slotv(v, slot_of_channel(4 * c4 + 2, 128)) * k4.z;
+        o.w = slotv(v, slot_of_channel(4 * c4 + 3, 128)) * k4.w;
+        reinterpret_cast<float4*>(qt + h * D)[c4] = o;
+      }
+    }
+  } else {
+    const int h = lane >> 1;
+    const bool p = (lane & 1) != 0;
+    const bool live = h < heads;
+    const uint32_t sel = p ? 0x7632u : 0x5410u;
+    const uint4* src = reinterpret_cast<const uint4*>(qb + (size_t)(live ? h : 0) * D);
+#pragma unroll
+    for (int cc = 0; cc < 32; ++cc) {  // thread p takes q[8cc + p + 2i]
+      const uint4 w = live ? __ldg(src + cc) : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 m = __ldg(reinterpret_cast<const uint4*>(ke->sgn) + cc);
+      uint32_t h0 = prmt(w.x ^ m.x, w.y ^ m.y, sel);
+      uint32_t h1 = prmt(w.z ^ m.z, w.w ^ m.w, sel);
+      v[2 * cc] = __half22float2(*reinterpret_cast<const __half2*>(&h0));
+      v[2 * cc + 1] = __half22float2(*reinterpret_cast<const __half2*>(&h1));
+    }
+    rdft_fwd_packed<128>(v);
+    float o[128];
+    pair_combine<0>(v, o, p);
+    if (live) {
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int cb = half ? (p ? 128 : 192) : (p ? 64 : 0);
+#pragma unroll
+        for (int c4 = 0; c4 < 16; ++c4) {
+          const float4 k4 = __ldg(reinterpret_cast<const float4*>(kd->chan + cb) + c4);
+          const int L = 64 * half + 4 * c4;
+          reinterpret_cast<float4*>(qt + h * D + cb)[c4] =
+              make_float4(o[L] * k4.x, o[L + 1] * k4.y, o[L + 2] * k4.z, o[L + 3] * k4.w);
+        }
+      }
+    }
+  }
+}
+
+// x = F_r^T Lambda_V^-1 o_t (without the sign, applied at the fp16 store) for the
+// real heads, by the inverse register FFT; writes fp32 x[h][n] to xb.
+template <int D>
+__device__ __forceinline__ void unrotate_out(const float* om, int heads, const CodecConsts* vd, float* xb, int lane) {
+  float2 u[64];
+  if constexpr (D == 128) {
+    const int h = lane;
+    const bool live = h < heads;
+    const float* oh = om + (live ? h : 0) * D;
+#pragma unroll
+    for (int c4 = 0; c4 < 32; ++c4) {
+      const float4 k4 = __ldg(reinterpret_cast<const float4*>(vd->chan) + c4);
+      const float4 o4 = live ? reinterpret_cast<const float4*>(oh)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float ov[4] = {o4.x * k4.x, o4.y * k4.y, o4.z * k4.z, o4.w * k4.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int sl = slot_of_channel(4 * c4 + e, 128);
+        if (sl & 1)
+          u[sl >> 1].y = ov[e];
+        else
+          u[sl >> 1].x = ov[e];
+      }
+    }
+    rdft_inv_packed<128>(u);
+    if (live) {
+#pragma unroll
+      for (int m = 0; m < 64; m += 2)
+        reinterpret_cast<float4*>(xb + h * D)[m >> 1] = make_float4(u[m].x, u[m].y, u[m + 1].x, u[m + 1].y);
+    }
+  } else {
+    const int h = lane >> 1;
+    const bool p = (lane & 1) != 0;
+    const bool live = h < heads;
+    const float* oh = om + (live ? h : 0) * D;
+    float o[128];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const int cb = half ? (p ? 128 : 192) : (p ? 64 : 0);
+#pragma unroll
+      for (int c4 = 0; c4 < 16; ++c4) {
+        const float4 k4 = __ldg(reinterpret_cast<const float4*>(vd->chan + cb) + c4);
+        const float4 o4 = live ? reinterpret_cast<const float4*>(oh + cb)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int L = 64 * half + 4 * c4;
+        o[L] = o4.x * k4.x;
+        o[L + 1] = o4.y * k4.y;
+        o[L + 2] = o4.z * k4.z;
+        o[L + 3] = o4.w * k4.w;
+      }
+    }
+#pragma unroll
+    for (int m = 0; m < 64; ++m) u[m] = make_float2(0.f, 0.f);
+    pair_combine_inv<0>(o, u, p);
+    rdft_inv_packed<128>(u);
+    if (live) {
+#pragma unroll
+      for (int m = 0; m < 64; ++m) {  // u[m] = (x[4m + p], x[4m + 2 + p])
+        xb[h * D + 4 * m + (p ? 1 : 0)] = u[m].x;
+        xb[h * D + 4 * m + 2 + (p ? 1 : 0)] = u[m].y;
+      }
+    }
+  }
+}
+
 template <int D, bool INT4>
-__global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_constant__ CUtensorMap kmap,
+__global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(const __grid_constant__ CUtensorMap kmap,
                                                              const __grid_constant__ CUtensorMap vmap,
                                                              const __grid_constant__ CUtensorMap ksmap,
                                                              const __grid_constant__ CUtensorMap vsmap,
@@ -254,17 +337,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
     }
   } else {
     // ------------------------------------------------------------ consumers
-    // (1) rotated query (int4: written by qrot_kernel, waited for here) or q itself (fp16)
+    // (1) the query in the K transform's rotated domain (int4) or q itself (fp16)
+    const uint16_t* qb = p.q + ((size_t)b * p.Hq + hq0) * D;
     if constexpr (INT4) {
-      griddep_wait();
-      const float4* src = reinterpret_cast<const float4*>(p.qt + (size_t)unit * kHT * D);
-      for (int i = threadIdx.x; i < kHT * D / 4; i += kCWarps * 32)
-        reinterpret_cast<float4*>(qt)[i] = __ldcg(src + i);
+      if (warp == 0) rotate_query<D>(qb, heads, p.ke, p.kd, qt, lane);
+      for (int i = threadIdx.x; i < (kHT - heads) * D; i += kCWarps * 32) qt[heads * D + i] = 0.0f;
     } else {
-      const uint16_t* qb = p.q + ((size_t)b * p.Hq + hq0) * D;
-      for (int i = threadIdx.x; i < kHT * D; i += kCWarps * 32) {
-        const int h = i / D;
-        qt[i] = h < heads ? __half2float(__ushort_as_half(__ldg(qb + i))) : 0.0f;
+      for (int i = threadIdx.x; i < kHT * D / 2; i += kCWarps * 32) {
+        const int h = (2 * i) / D;
+        const float2 f = h < heads ? __half22float2(__ldg(reinterpret_cast<const __half2*>(qb) + i))
+                                   : make_float2(0.0f, 0.0f);
+        reinterpret_cast<float2*>(qt)[i] = f;
       }
     }
     consumer_sync();
@@ -533,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
   float* mypart = p.part + ((size_t)unit * p.S + split) * PART;
   {
     // CTA partial: M = max_w m_w, L = sum_w l_w 2^(m_w - M), O = sum_w o_w 2^(m_w - M)
-    for (int idx = threadIdx.x; idx < kHT * D; idx += kThreads) {
+    for (int idx = threadIdx.x; idx < heads * D; idx += kThreads) {
       const int h = idx / D;
       float M = -INFINITY;
 #pragma unroll
@@ -562,92 +645,84 @@ __global__ void __launch_bounds__(kThreads, 1) attend_kernel(const __grid_consta
     }
   }
   // ------------------------------------------------------------ last CTA of the unit merges the splits
-  __threadfence();
+  // bar.sync orders every thread's partial stores before thread 0's device-scope
+  // fence and counter increment (release); the last CTA's thread 0 fences again
+  // after seeing the count (acquire) before the block reads the other partials.
   __syncthreads();
   if (threadIdx.x == 0) {
+    __threadfence();
     const int prev = atomicAdd(p.cnt + unit, 1);
-    *flag = (prev == p.S - 1) ? 1 : 0;
+    const int last = (prev == p.S - 1) ? 1 : 0;
+    if (last) __threadfence();
+    *flag = last;
   }
   __syncthreads();
   if (*flag == 0) return;
-  __threadfence();
   const float* parts = p.part + (size_t)unit * p.S * PART;
   float* om = qt;  // merged o_t [8][D] (fp32)
-  // per-head merge weights, computed once: wsm[s][h] = 2^(m_s - M) / L (0 for empty splits)
-  float* wsm = reinterpret_cast<float*>(ring);  // [S][8] (ring is free)
-  float* hm = wsm + p.S * kHT;                  // [8] head max
+  // per-head merge weights: wsm[s][h] = 2^(m_s - M) / L (0 for empty splits). One parallel
+  // pass loads every split's (m, l); one thread per head then reduces in shared memory.
+  float* wsm = reinterpret_cast<float*>(ring);  // [S][8] m, then weights
+  float* lsm = wsm + p.S * kHT;                 // [S][8] l
+  float* xb = lsm + p.S * kHT;                  // [8][D] un-rotated output (fp32)
+  for (int i = threadIdx.x; i < p.S * kHT; i += kThreads) {
+    const int s2 = i / kHT, h = i - s2 * kHT;
+    wsm[i] = __ldcg(parts + (size_t)s2 * PART + h);
+    lsm[i] = __ldcg(parts + (size_t)s2 * PART + kHT + h);
+  }
+  __syncthreads();
   if (threadIdx.x < kHT) {
     const int h = threadIdx.x;
     float M = -INFINITY;
-    for (int s2 = 0; s2 < p.S; ++s2) M = fmaxf(M, __ldcg(parts + (size_t)s2 * PART + h));
-    hm[h] = M;
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < p.S * kHT; i += kThreads) {
-    const int s2 = i / kHT, h = i - s2 * kHT;
-    const float ms = __ldcg(parts + (size_t)s2 * PART + h);
-    const float M = hm[h];
-    wsm[i] = (M == -INFINITY || ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
-  }
-  __syncthreads();
-  if (threadIdx.x < kHT) {
-    const int h = threadIdx.x;
+    for (int s2 = 0; s2 < p.S; ++s2) M = fmaxf(M, wsm[s2 * kHT + h]);
     float L = 0.0f;
-    for (int s2 = 0; s2 < p.S; ++s2) L += wsm[s2 * kHT + h] * __ldcg(parts + (size_t)s2 * PART + kHT + h);
-    hm[h] = L > 0.0f ? 1.0f / L : 0.0f;
+    for (int s2 = 0; s2 < p.S; ++s2) {
+      const float ms = wsm[s2 * kHT + h];
+      const float w = (M == -INFINITY || ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
+      wsm[s2 * kHT + h] = w;
+      L += w * lsm[s2 * kHT + h];
+    }
+    const float invL = L > 0.0f ? 1.0f / L : 0.0f;
+    for (int s2 = 0; s2 < p.S; ++s2) wsm[s2 * kHT + h] *= invL;
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < p.S * kHT; i += kThreads) wsm[i] *= hm[i % kHT];
-  __syncthreads();
-  for (int idx = threadIdx.x; idx < kHT * D; idx += kThreads) {
-    const int h = idx / D;
-    const float* po = parts + 2 * kHT + idx;
-    float o0 = 0.f, o1 = 0.f, o2 = 0.f, o3 = 0.f;
-    int s2 = 0;
-    for (; s2 + 4 <= p.S; s2 += 4) {
-      o0 += wsm[(s2 + 0) * kHT + h] * __ldcg(po + (size_t)(s2 + 0) * PART);
-      o1 += wsm[(s2 + 1) * kHT + h] * __ldcg(po + (size_t)(s2 + 1) * PART);
-      o2 += wsm[(s2 + 2) * kHT + h] * __ldcg(po + (size_t)(s2 + 2) * PART);
-      o3 += wsm[(s2 + 3) * kHT + h] * __ldcg(po + (size_t)(s2 + 3) * PART);
+  {
+    // o_t[h][c] = sum_s w_s[h] o_s[h][c], four channels per thread and four splits in flight
+    const float4* po4 = reinterpret_cast<const float4*>(parts + 2 * kHT);
+    constexpr int P4 = (2 * kHT + kHT * D) / 4;
+    for (int i = threadIdx.x; i < heads * D / 4; i += kThreads) {
+      const int h = (4 * i) / D;
+      float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
+      int s2 = 0;
+      for (; s2 + 2 <= p.S; s2 += 2) {
+        const float w0 = wsm[s2 * kHT + h], w1 = wsm[(s2 + 1) * kHT + h];
+        const float4 v0 = __ldcg(po4 + (size_t)s2 * P4 + i), v1 = __ldcg(po4 + (size_t)(s2 + 1) * P4 + i);
+        a0.x = fmaf(w0, v0.x, a0.x); a0.y = fmaf(w0, v0.y, a0.y); a0.z = fmaf(w0, v0.z, a0.z); a0.w = fmaf(w0, v0.w, a0.w);
+        a1.x = fmaf(w1, v1.x, a1.x); a1.y = fmaf(w1, v1.y, a1.y); a1.z = fmaf(w1, v1.z, a1.z); a1.w = fmaf(w1, v1.w, a1.w);
+      }
+      if (s2 < p.S) {
+        const float w0 = wsm[s2 * kHT + h];
+        const float4 v0 = __ldcg(po4 + (size_t)s2 * P4 + i);
+        a0.x = fmaf(w0, v0.x, a0.x); a0.y = fmaf(w0, v0.y, a0.y); a0.z = fmaf(w0, v0.z, a0.z); a0.w = fmaf(w0, v0.w, a0.w);
+      }
+      reinterpret_cast<float4*>(om)[i] = make_float4(a0.x + a1.x, a0.y + a1.y, a0.z + a1.z, a0.w + a1.w);
     }
-    for (; s2 < p.S; ++s2) o0 += wsm[s2 * kHT + h] * __ldcg(po + (size_t)s2 * PART);
-    om[idx] = (o0 + o1) + (o2 + o3);
   }
   if (threadIdx.x == 0) p.cnt[unit] = 0;  // leave the counter at zero for the next call
   __syncthreads();
   uint16_t* ob = p.out + ((size_t)b * p.Hq + hq0) * D;
   if constexpr (INT4) {
-    // o[h][n] = sum_i R'^T[n][i] o_t[h][i] with fp16 operands (R'^T hi part, o_t rounded to
-    // fp16; the result is rounded to fp16 anyway) and fp32 accumulate; the B
-    // fragments are shared by all m-tiles, and each m-tile's A loads are issued together.
-    uint32_t bo0[MT], bo1[MT];
-#pragma unroll
-    for (int kt = 0; kt < MT; ++kt) {
-      const float* oh = om + g * D + kt * 16 + 2 * c;
-      bo0[kt] = pack_half2(oh[0], oh[1]);
-      bo1[kt] = pack_half2(oh[8], oh[9]);
-    }
-    for (int mt = warp; mt < MT; mt += kCWarps + 1) {
-      uint4 ah[MT];
-#pragma unroll
-      for (int kt = 0; kt < MT; ++kt) ah[kt] = __ldg(p.ro + (((size_t)mt * MT + kt) * 2 + 0) * 32 + lane);
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int kt = 0; kt < MT; ++kt) mma_16816(acc, ah[kt].x, ah[kt].y, ah[kt].z, ah[kt].w, bo0[kt], bo1[kt]);
-      // C: rows n = mt*16 + g (+8), cols head 2c, 2c+1
-      const int n0 = mt * 16 + g;
-      if (2 * c < heads) {
-        ob[(size_t)(2 * c) * D + n0] = __half_as_ushort(__float2half_rn(acc[0]));
-        ob[(size_t)(2 * c) * D + n0 + 8] = __half_as_ushort(__float2half_rn(acc[2]));
-      }
-      if (2 * c + 1 < heads) {
-        ob[(size_t)(2 * c + 1) * D + n0] = __half_as_ushort(__float2half_rn(acc[1]));
-        ob[(size_t)(2 * c + 1) * D + n0 + 8] = __half_as_ushort(__float2half_rn(acc[3]));
-      }
+    if (warp == 0) unrotate_out<D>(om, heads, p.vd, xb, lane);
+    __syncthreads();
+    // fp16 with the V sign folded in as an XOR on the sign bits
+    for (int i = threadIdx.x; i < heads * D / 2; i += kThreads) {
+      const int j = i % (D / 2);
+      const uint32_t hv = pack_half2(xb[2 * i], xb[2 * i + 1]) ^ __ldg(&p.vd->sgn[j]);
+      reinterpret_cast<uint32_t*>(ob)[i] = hv;
     }
   } else {
-    for (int idx = threadIdx.x; idx < heads * D; idx += kThreads)
-      ob[idx] = __half_as_ushort(__float2half_rn(om[idx]));
+    for (int i = threadIdx.x; i < heads * D / 2; i += kThreads)
+      reinterpret_cast<uint32_t*>(ob)[i] = pack_half2(om[2 * i], om[2 * i + 1]);
   }
 }
 
@@ -672,13 +747,15 @@ int ctas_per_sm() {
   return v;
 }
 
-// Split of the token range. Each split keeps at least kMinTilesPerSplit stages so
-// that its TMA pipeline streams; among the split counts that give at least one
-// full wave of CTAs, the smallest one whose last wave is >= 85% full is taken
-// (else the best-filled one). Non-decreasing in T, so the workspace size computed
-// from T_cap bounds every call with T <= T_cap.
+// Split of the token range. When splits of ~4 stages cannot fill the GPU (few
+// units, short context) the kernel is latency-bound: take ~4 stages per split,
+// which keeps the final merge short. Otherwise (throughput regime) take, among
+// split counts giving at least one full wave, the smallest whose last wave is
+// >= 85% full. Every split keeps >= kMinTilesPerSplit stages, S <= kMaxSplits, and
+// S is non-decreasing in T, so a workspace sized from T_cap bounds every call.
 constexpr int kMinTilesPerSplit = 2;
-constexpr int kMaxSplits = 256;
+constexpr int kMaxSplits = kMaxSplitsCfg;
+constexpr int kLatencyTilesPerSplit = 4;
 
 SplitPlan choose_split(int B, int Hq, int Hkv, int T, int sms, int per_sm) {
   SplitPlan sp{};
@@ -690,22 +767,25 @@ SplitPlan choose_split(int B, int Hq, int Hkv, int T, int sms, int per_sm) {
   int s_cap = std::max(1, ntile / kMinTilesPerSplit);
   s_cap = std::min(s_cap, kMaxSplits);
   int best = 1;
-  double best_eff = -1.0;
-  const int s_lo = (int)std::min<long>(s_cap, std::max<long>(1, (slots + units - 1) / units));
-  for (int S = s_lo; S <= s_cap; ++S) {
-    const int tiles_per = (ntile + S - 1) / S;
-    const int Sr = (ntile + tiles_per - 1) / tiles_per;
-    const long ctas = units * Sr;
-    const long waves = (ctas + slots - 1) / slots;
-    const double eff = (double)ctas / (double)(waves * slots);
-    if (eff >= 0.85) {
-      best = S;
-      best_eff = eff;
-      break;
-    }
-    if (eff > best_eff + 1e-9) {
-      best_eff = eff;
-      best = S;
+  if (units * std::max(1, ntile / kLatencyTilesPerSplit) < slots) {
+    best = std::max(1, std::min(ntile / kLatencyTilesPerSplit, s_cap));
+  } else {
+    double best_eff = -1.0;
+    const int s_lo = (int)std::min<long>(s_cap, std::max<long>(1, (slots + units - 1) / units));
+    for (int S = s_lo; S <= s_cap; ++S) {
+      const int tiles_per = (ntile + S - 1) / S;
+      const int Sr = (ntile + tiles_per - 1) / tiles_per;
+      const long ctas = units * Sr;
+      const long waves = (ctas + slots - 1) / slots;
+      const double eff = (double)ctas / (double)(waves * slots);
+      if (eff >= 0.85) {
+        best = S;
+        break;
+      }
+      if (eff > best_eff + 1e-9) {
+        best_eff = eff;
+        best = S;
+      }
     }
   }
   const int tiles_per = (ntile + best - 1) / best;
@@ -716,14 +796,13 @@ SplitPlan choose_split(int B, int Hq, int Hkv, int T, int sms, int per_sm) {
 
 constexpr int kMaxPerSmForSizing = 4;
 
-// workspace: [counters (units ints, 256-aligned)] [rotated queries units x 8 x D fp32] [partials]
+// workspace: [counters (units ints, 256-aligned)] [partials units x S x (m[8], l[8], o[8][D]) fp32]
 size_t ws_cnt_bytes(size_t units) { return ((units * 4 + 255) / 256) * 256; }
-size_t ws_qt_bytes(size_t units, int D) { return units * kHT * D * 4; }
 
 size_t ws_bytes_for(int B, int Hq, int Hkv, int D, int S_max, int HT) {
   const size_t units = (size_t)B * Hkv * HT;
   const size_t part = units * (size_t)S_max * (2 * kHT + kHT * D) * 4;
-  return ws_cnt_bytes(units) + ws_qt_bytes(units, D) + part;
+  return ws_cnt_bytes(units) + part;
 }
 
 template <int D, bool INT4>
@@ -787,33 +866,15 @@ kvq_status run_attend(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q,
   prm.sl2 = sg * kLog2e;
   char* wsb = reinterpret_cast<char*>(ws);
   prm.cnt = reinterpret_cast<int*>(wsb);
-  float* qt_ws = reinterpret_cast<float*>(wsb + ws_cnt_bytes(units));
-  prm.qt = qt_ws;
-  prm.part = reinterpret_cast<float*>(wsb + ws_cnt_bytes(units) + ws_qt_bytes(units, D));
-  prm.ro = INT4 ? pv->ro_frag : nullptr;
+  prm.part = reinterpret_cast<float*>(wsb + ws_cnt_bytes(units));
+  prm.ke = INT4 ? pk->enc_dev : nullptr;
+  prm.kd = INT4 ? pk->dec_dev : nullptr;
+  prm.vd = INT4 ? pv->dec_dev : nullptr;
   dim3 grid(sp.S, sp.HT, B * Hkv);
   if (grid.z > 65535u) return fail(KVQ_ERR_UNSUPPORTED, "attend: B * Hkv > 65535");
-  if constexpr (INT4) {
-    qrot_kernel<D><<<(unsigned)units, 256, 0, strm>>>(q, pk->rq_frag, qt_ws, Hq, Hkv, Hq / Hkv, sp.HT);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("qrot launch: ") + cudaGetErrorString(e));
-    cudaLaunchConfig_t cfg{};
-    cfg.gridDim = grid;
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = C::kSmem;
-    cfg.stream = strm;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, attend_kernel<D, INT4>, kmap, vmap, ksmap, vsmap, prm);
-    if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
-  } else {
-    attend_kernel<D, INT4><<<grid, kThreads, C::kSmem, strm>>>(kmap, vmap, ksmap, vsmap, prm);
-    const cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
-  }
+  attend_kernel<D, INT4><<<grid, kThreads, C::kSmem, strm>>>(kmap, vmap, ksmap, vsmap, prm);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
   return KVQ_OK;
 }
 

@@ -95,58 +95,6 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
   return old;
 }
 
-// D = 256 pair combine: thread p of a pair holds the size-128 spectrum of the samples
-// x[2j + p] (E for p = 0, O for p = 1) in slot order; it forms X_k and X_{128-k} for
-// k = 32p + J, J = 0..32, exchanging one value per component with its partner.
-// Thread 0 then owns channels [0, 64) and [192, 256), thread 1 channels [64, 192);
-// local value L of both threads maps to the same (J, X or X_{128-k}, Re or Im), except L = 0.
-template <int S_>
-struct TwPair {  // W_256^(32p + J) for p = 0, 1
-  static constexpr float c0 = static_cast<float>(cos2pi_frac(S_, 256));
-  static constexpr float s0 = static_cast<float>(sin2pi_frac(S_, 256));
-  static constexpr float c1 = static_cast<float>(cos2pi_frac(S_ + 32, 256));
-  static constexpr float s1 = static_cast<float>(sin2pi_frac(S_ + 32, 256));
-};
-
-__device__ __forceinline__ float slotv(const float2 (&u)[64], int sl) { return (sl & 1) ? u[sl >> 1].y : u[sl >> 1].x; }
-
-template <int J>
-__device__ __forceinline__ void pair_combine(const float2 (&u)[64], float (&o)[128], const bool p) {
-  if constexpr (J <= 32) {
-    constexpr int k0 = J, k1 = 32 + J;
-    constexpr int re0 = k0 == 0 ? 0 : 2 * k0, im0 = k0 == 0 ? -1 : 2 * k0 + 1;
-    constexpr int re1 = k1 == 64 ? 1 : 2 * k1, im1 = k1 == 64 ? -1 : 2 * k1 + 1;
-    const float u_re0 = slotv(u, re0), u_re1 = slotv(u, re1);
-    const float u_im0 = im0 < 0 ? 0.0f : slotv(u, im0 < 0 ? 0 : im0);
-    const float u_im1 = im1 < 0 ? 0.0f : slotv(u, im1 < 0 ? 0 : im1);
-    const float mine_re = p ? u_re1 : u_re0, send_re = p ? u_re0 : u_re1;
-    const float mine_im = p ? u_im1 : u_im0, send_im = p ? u_im0 : u_im1;
-    const float recv_re = __shfl_xor_sync(0xffffffffu, send_re, 1);
-    const float recv_im = __shfl_xor_sync(0xffffffffu, send_im, 1);
-    const float er = p ? recv_re : mine_re, ei = p ? recv_im : mine_im;
-    const float orr = p ? mine_re : recv_re, oi = p ? mine_im : recv_im;
-    const float c = p ? TwPair<J>::c1 : TwPair<J>::c0;
-    const float sn = p ? TwPair<J>::s1 : TwPair<J>::s0;
-    const float xr = fmaf(c, orr, fmaf(sn, oi, er));  // X_k = E + W O
-    const float xi = fmaf(c, oi, fmaf(-sn, orr, ei));
-    const float yr = fmaf(2.0f, er, -xr);              // X_{128-k} = conj(E - W O)
-    const float yi = fmaf(-2.0f, ei, xi);
-    if constexpr (J == 0) {
-      o[0] = p ? xi : xr;
-      o[127] = yr;
-    } else if constexpr (J < 32) {
-      o[2 * J - 1] = xr;
-      o[2 * J] = xi;
-      o[127 - 2 * J] = yr;
-      o[128 - 2 * J] = yi;
-    } else {
-      o[63] = xr;
-      o[64] = yi;
-    }
-    pair_combine<J + 1>(u, o, p);
-  }
-}
-
 // lambda, per-group abs-max, fp16 scale, int4 rounding and nibble packing of
 // NV channel values (NV/G groups); lam points at the lambda*dg of those channels.
 template <int NV, int G>

@@ -30,13 +30,11 @@ struct kvq_plan {
   int device = -1;
   kvq::CodecConsts enc{};  // lambda_c * dg_c
   kvq::CodecConsts dec{};  // dg_c / lambda_c
-  // Device block: the rotation R' = Lambda^-1 F_r diag(s) in mma fragment order,
-  // split into fp16 hi + lo parts, once as A = R' (query rotation, q_t = R' q)
-  // and once as A = R'^T (output un-rotation, o = R'^T o_t).
+  // Device block: copies of `enc` and `dec` for kernels that serve several plans
+  // in one launch (grouped encode) or two plans at once (attention: K and V).
   void* dblock = nullptr;
-  const uint4* rq_frag = nullptr;   // [D/16 m-tiles][D/16 k-tiles][2 hi/lo][32 lanes] uint4
-  const uint4* ro_frag = nullptr;   // same layout for R'^T
-  const kvq::CodecConsts* enc_dev = nullptr;  // device copy of `enc` (read by the encode kernel)
+  const kvq::CodecConsts* enc_dev = nullptr;
+  const kvq::CodecConsts* dec_dev = nullptr;
 };
 
 namespace kvq {
