@@ -34,10 +34,14 @@
 #include <mutex>
 
 #include "kvq_internal.h"
+#include <cooperative_groups.h>
+
 #include "kvq_ptx.cuh"
 #include "srft_fft.cuh"
 
 namespace kvq {
+
+namespace cg = cooperative_groups;
 
 __device__ uint32_t g_attend_err = 0;
 
@@ -49,6 +53,10 @@ constexpr int kTileT = 16 * kCWarps;       // tokens per stage
 constexpr int kHT = 8;                     // query heads per CTA (mma N)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kMaxSplitsCfg = 256;          // upper bound on splits per unit
+constexpr int kMaxCluster = 8;              // splits merged through distributed shared memory
+constexpr int kMaxClusterLatency = 8;
+constexpr int kMaxClusterThroughput = 4;
+constexpr int kMaxMerge = kMaxSplitsCfg / 4;  // clusters per unit (>= 4 splits each) or splits per cluster
 
 template <int D, bool INT4>
 struct Cfg {
@@ -63,9 +71,9 @@ struct Cfg {
   // warp-merge scratch (reuses the stage ring): per warp m[8], l[8], o[8][D]
   static constexpr int kWarpState = (2 * kHT + kHT * D) * 4;
   static constexpr int kRing = kStages * kStageBytes;
-  static constexpr int kTail = (2 * kMaxSplitsCfg * kHT + kHT * D) * 4;  // merge m/l/weights + un-rotated output
-  static constexpr int kScratch0 = kCWarps * kWarpState > kRing ? kCWarps * kWarpState : kRing;
-  static constexpr int kScratch = kScratch0 > kTail ? kScratch0 : kTail;
+  // tail scratch (reuses the ring): warp partials, CTA partial, merged (M, L), merge weights, output
+  static constexpr int kTail = ((kCWarps + 1) * (2 * kHT + kHT * D) + 2 * kHT + 2 * kMaxMerge * kHT + kHT * D) * 4;
+  static constexpr int kScratch = kRing > kTail ? kRing : kTail;
   static constexpr int kQt = kHT * D * 4;                  // fp32 q_t (or merged o_t) [8][D]
   static constexpr int kSmem = kScratch + kQt + 64 + 1024;
 };
@@ -581,12 +589,15 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
       l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
     }
   }
-  if (!__syncthreads_and(ok ? 1 : 0)) return;
+  (void)ok;  // a timed-out CTA still takes part in every barrier below; its flag reaches the host
+  __syncthreads();
 
   // ------------------------------------------------------------ merge the warps (ring is free now)
-  float* wst = reinterpret_cast<float*>(ring);  // [warp][ m[8] | l[8] | o[8][D] ]
+  constexpr int PART = 2 * kHT + kHT * D;        // m[8] | l[8] | o[8][D]
+  float* wst = reinterpret_cast<float*>(ring);  // [warp][PART]
+  float* cpart = wst + kCWarps * PART;           // this CTA's partial [PART]
   if (warp < kCWarps) {
-    float* ws = wst + warp * (2 * kHT + kHT * D);
+    float* ws = wst + warp * PART;
     if (g == 0) {
       ws[2 * c] = m_run[0];
       ws[2 * c + 1] = m_run[1];
@@ -612,103 +623,111 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
     }
   }
   __syncthreads();
-  const int PART = 2 * kHT + kHT * D;
-  float* mypart = p.part + ((size_t)unit * p.S + split) * PART;
-  {
-    // CTA partial: M = max_w m_w, L = sum_w l_w 2^(m_w - M), O = sum_w o_w 2^(m_w - M)
-    for (int idx = threadIdx.x; idx < heads * D; idx += kThreads) {
-      const int h = idx / D;
-      float M = -INFINITY;
-#pragma unroll
-      for (int w = 0; w < kCWarps; ++w) M = fmaxf(M, wst[w * PART + h]);
-      float o = 0.0f;
-      if (M != -INFINITY) {
-#pragma unroll
-        for (int w = 0; w < kCWarps; ++w) {
-          const float mw = wst[w * PART + h];
-          if (mw != -INFINITY) o += wst[w * PART + 2 * kHT + idx] * fast_exp2(mw - M);
-        }
-      }
-      __stcg(mypart + 2 * kHT + idx, o);
-      if (idx % D == 0) {
-        float L = 0.0f;
-        if (M != -INFINITY) {
-#pragma unroll
-          for (int w = 0; w < kCWarps; ++w) {
-            const float mw = wst[w * PART + h];
-            if (mw != -INFINITY) L += wst[w * PART + kHT + h] * fast_exp2(mw - M);
-          }
-        }
-        __stcg(mypart + h, M);
-        __stcg(mypart + kHT + h, L);
-      }
-    }
-  }
-  // ------------------------------------------------------------ last CTA of the unit merges the splits
-  // bar.sync orders every thread's partial stores before thread 0's device-scope
-  // fence and counter increment (release); the last CTA's thread 0 fences again
-  // after seeing the count (acquire) before the block reads the other partials.
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    const int prev = atomicAdd(p.cnt + unit, 1);
-    const int last = (prev == p.S - 1) ? 1 : 0;
-    if (last) __threadfence();
-    *flag = last;
-  }
-  __syncthreads();
-  if (*flag == 0) return;
-  const float* parts = p.part + (size_t)unit * p.S * PART;
-  float* om = qt;  // merged o_t [8][D] (fp32)
-  // per-head merge weights: wsm[s][h] = 2^(m_s - M) / L (0 for empty splits). One parallel
-  // pass loads every split's (m, l); one thread per head then reduces in shared memory.
-  float* wsm = reinterpret_cast<float*>(ring);  // [S][8] m, then weights
-  float* lsm = wsm + p.S * kHT;                 // [S][8] l
-  float* xb = lsm + p.S * kHT;                  // [8][D] un-rotated output (fp32)
-  for (int i = threadIdx.x; i < p.S * kHT; i += kThreads) {
-    const int s2 = i / kHT, h = i - s2 * kHT;
-    wsm[i] = __ldcg(parts + (size_t)s2 * PART + h);
-    lsm[i] = __ldcg(parts + (size_t)s2 * PART + kHT + h);
-  }
-  __syncthreads();
-  if (threadIdx.x < kHT) {
-    const int h = threadIdx.x;
+  // CTA partial: M = max_w m_w, L = sum_w l_w 2^(m_w - M), O = sum_w o_w 2^(m_w - M)
+  for (int idx = threadIdx.x; idx < heads * D + kHT; idx += kThreads) {
+    const bool ml = idx >= heads * D;
+    const int h = ml ? idx - heads * D : idx / D;
     float M = -INFINITY;
-    for (int s2 = 0; s2 < p.S; ++s2) M = fmaxf(M, wsm[s2 * kHT + h]);
-    float L = 0.0f;
-    for (int s2 = 0; s2 < p.S; ++s2) {
-      const float ms = wsm[s2 * kHT + h];
-      const float w = (M == -INFINITY || ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
-      wsm[s2 * kHT + h] = w;
-      L += w * lsm[s2 * kHT + h];
+#pragma unroll
+    for (int w = 0; w < kCWarps; ++w) M = fmaxf(M, wst[w * PART + h]);
+    float acc = 0.0f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kCWarps; ++w) {
+        const float mw = wst[w * PART + h];
+        if (mw != -INFINITY) acc += wst[w * PART + (ml ? kHT + h : 2 * kHT + idx)] * fast_exp2(mw - M);
+      }
     }
-    const float invL = L > 0.0f ? 1.0f / L : 0.0f;
-    for (int s2 = 0; s2 < p.S; ++s2) wsm[s2 * kHT + h] *= invL;
+    if (ml) {
+      cpart[h] = M;
+      cpart[kHT + h] = acc;
+    } else {
+      cpart[2 * kHT + idx] = acc;
+    }
   }
-  __syncthreads();
-  {
-    // o_t[h][c] = sum_s w_s[h] o_s[h][c], four channels per thread and four splits in flight
-    const float4* po4 = reinterpret_cast<const float4*>(parts + 2 * kHT);
-    constexpr int P4 = (2 * kHT + kHT * D) / 4;
+
+  // ------------------------------------------------------------ merge the splits of the cluster (DSMEM)
+  cg::cluster_group cluster = cg::this_cluster();
+  const int crank = (int)cluster.block_rank();
+  const int csize = (int)cluster.num_blocks();
+  cluster.sync();  // every CTA's partial is in its shared memory
+  float* om = qt;                                // merged o_t [8][D] (fp32)
+  float* mrg = cpart + PART;                     // merged (M, L) [2][8]
+  float* wsm = mrg + 2 * kHT;                    // [n][8] weights (merge scratch)
+  float* lsm = wsm + kMaxMerge * kHT;            // [n][8]
+  float* xb = lsm + kMaxMerge * kHT;             // [8][D] un-rotated output (fp32)
+  // merge n partials (pointer of partial r from `at`) into (mrg, om) -- om unnormalised, relative to M
+  auto merge = [&](int n, auto at) {
+    for (int i = threadIdx.x; i < n * kHT; i += kThreads) {
+      const int r = i / kHT, h = i - r * kHT;
+      const float* pr = at(r);
+      wsm[i] = pr[h];
+      lsm[i] = pr[kHT + h];
+    }
+    __syncthreads();
+    if (threadIdx.x < kHT) {
+      const int h = threadIdx.x;
+      float M = -INFINITY;
+      for (int r = 0; r < n; ++r) M = fmaxf(M, wsm[r * kHT + h]);
+      float L = 0.0f;
+      for (int r = 0; r < n; ++r) {
+        const float mr = wsm[r * kHT + h];
+        const float w = (M == -INFINITY || mr == -INFINITY) ? 0.0f : fast_exp2(mr - M);
+        wsm[r * kHT + h] = w;
+        L += w * lsm[r * kHT + h];
+      }
+      mrg[h] = M;
+      mrg[kHT + h] = L;
+    }
+    __syncthreads();
     for (int i = threadIdx.x; i < heads * D / 4; i += kThreads) {
       const int h = (4 * i) / D;
-      float4 a0 = make_float4(0.f, 0.f, 0.f, 0.f), a1 = a0;
-      int s2 = 0;
-      for (; s2 + 2 <= p.S; s2 += 2) {
-        const float w0 = wsm[s2 * kHT + h], w1 = wsm[(s2 + 1) * kHT + h];
-        const float4 v0 = __ldcg(po4 + (size_t)s2 * P4 + i), v1 = __ldcg(po4 + (size_t)(s2 + 1) * P4 + i);
-        a0.x = fmaf(w0, v0.x, a0.x); a0.y = fmaf(w0, v0.y, a0.y); a0.z = fmaf(w0, v0.z, a0.z); a0.w = fmaf(w0, v0.w, a0.w);
-        a1.x = fmaf(w1, v1.x, a1.x); a1.y = fmaf(w1, v1.y, a1.y); a1.z = fmaf(w1, v1.z, a1.z); a1.w = fmaf(w1, v1.w, a1.w);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int r = 0; r < n; ++r) {
+        const float w = wsm[r * kHT + h];
+        const float4 v = reinterpret_cast<const float4*>(at(r) + 2 * kHT)[i];
+        acc.x = fmaf(w, v.x, acc.x);
+        acc.y = fmaf(w, v.y, acc.y);
+        acc.z = fmaf(w, v.z, acc.z);
+        acc.w = fmaf(w, v.w, acc.w);
       }
-      if (s2 < p.S) {
-        const float w0 = wsm[s2 * kHT + h];
-        const float4 v0 = __ldcg(po4 + (size_t)s2 * P4 + i);
-        a0.x = fmaf(w0, v0.x, a0.x); a0.y = fmaf(w0, v0.y, a0.y); a0.z = fmaf(w0, v0.z, a0.z); a0.w = fmaf(w0, v0.w, a0.w);
-      }
-      reinterpret_cast<float4*>(om)[i] = make_float4(a0.x + a1.x, a0.y + a1.y, a0.z + a1.z, a0.w + a1.w);
+      reinterpret_cast<float4*>(om)[i] = acc;
     }
+    __syncthreads();
+  };
+  if (crank == 0) merge(csize, [&](int r) { return static_cast<const float*>(cluster.map_shared_rank(cpart, r)); });
+  cluster.sync();  // peers may leave once the leader has read their shared memory
+  if (crank != 0) return;
+
+  // ------------------------------------------------------------ more than one cluster per unit: global merge
+  const int ncl = p.S / csize;
+  if (ncl > 1) {
+    const int cl = split / csize;
+    float* gpart = p.part + ((size_t)unit * ncl + cl) * PART;
+    for (int i = threadIdx.x; i < kHT * 2; i += kThreads) __stcg(gpart + i, mrg[i]);
+    for (int i = threadIdx.x; i < heads * D; i += kThreads) __stcg(gpart + 2 * kHT + i, om[i]);
+    // bar.sync orders every thread's stores before thread 0's device-scope fence and
+    // counter increment; the last leader fences again before reading the others' partials.
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      const int prev = atomicAdd(p.cnt + unit, 1);
+      const int last = (prev == ncl - 1) ? 1 : 0;
+      if (last) __threadfence();
+      *flag = last;
+    }
+    __syncthreads();
+    if (*flag == 0) return;
+    if (threadIdx.x == 0) p.cnt[unit] = 0;  // leave the counter at zero for the next call
+    const float* gbase = p.part + (size_t)unit * ncl * PART;
+    merge(ncl, [&](int r) { return gbase + (size_t)r * PART; });
   }
-  if (threadIdx.x == 0) p.cnt[unit] = 0;  // leave the counter at zero for the next call
+
+  // ------------------------------------------------------------ normalise, un-rotate, store fp16
+  for (int i = threadIdx.x; i < heads * D; i += kThreads) {
+    const float L = mrg[kHT + i / D];
+    om[i] = L > 0.0f ? om[i] / L : 0.0f;
+  }
   __syncthreads();
   uint16_t* ob = p.out + ((size_t)b * p.Hq + hq0) * D;
   if constexpr (INT4) {
@@ -717,8 +736,7 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
     // fp16 with the V sign folded in as an XOR on the sign bits
     for (int i = threadIdx.x; i < heads * D / 2; i += kThreads) {
       const int j = i % (D / 2);
-      const uint32_t hv = pack_half2(xb[2 * i], xb[2 * i + 1]) ^ __ldg(&p.vd->sgn[j]);
-      reinterpret_cast<uint32_t*>(ob)[i] = hv;
+      reinterpret_cast<uint32_t*>(ob)[i] = pack_half2(xb[2 * i], xb[2 * i + 1]) ^ __ldg(&p.vd->sgn[j]);
     }
   } else {
     for (int i = threadIdx.x; i < heads * D / 2; i += kThreads)
@@ -728,7 +746,7 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
 
 // ---------------------------------------------------------------- host side
 struct SplitPlan {
-  int HT, S, tps;
+  int HT, S, tps, C;  // C = splits per cluster (S is a multiple of C)
 };
 
 template <int D, bool INT4>
@@ -738,6 +756,7 @@ int ctas_per_sm() {
   static std::once_flag once;
   std::call_once(once, [] {
     cudaFuncSetAttribute(attend_kernel<D, INT4>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    cudaFuncSetAttribute(attend_kernel<D, INT4>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     int nb = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, attend_kernel<D, INT4>, kThreads, C::kSmem) != cudaSuccess ||
         nb < 1)
@@ -767,7 +786,8 @@ SplitPlan choose_split(int B, int Hq, int Hkv, int T, int sms, int per_sm) {
   int s_cap = std::max(1, ntile / kMinTilesPerSplit);
   s_cap = std::min(s_cap, kMaxSplits);
   int best = 1;
-  if (units * std::max(1, ntile / kLatencyTilesPerSplit) < slots) {
+  const bool latency = units * std::max(1, ntile / kLatencyTilesPerSplit) < slots;
+  if (latency) {
     best = std::max(1, std::min(ntile / kLatencyTilesPerSplit, s_cap));
   } else {
     double best_eff = -1.0;
@@ -791,17 +811,31 @@ SplitPlan choose_split(int B, int Hq, int Hkv, int T, int sms, int per_sm) {
   const int tiles_per = (ntile + best - 1) / best;
   sp.tps = tiles_per * kTileT;
   sp.S = (ntile + tiles_per - 1) / tiles_per;
+  // splits of a unit run as one thread-block cluster (<= 16) and merge through
+  // distributed shared memory; beyond 16, whole clusters (the last ones possibly
+  // with empty splits) merge through the workspace
+  // (clusters of up to 8 in the latency regime; up to 4 when the GPU is full of
+  // units, where large clusters constrain scheduling more than they save)
+  const int cmax = latency ? kMaxClusterLatency : kMaxClusterThroughput;
+  if (sp.S <= cmax) {
+    sp.C = sp.S;
+  } else {
+    sp.C = cmax;
+    sp.S = (sp.S + cmax - 1) / cmax * cmax;
+  }
   return sp;
 }
 
 constexpr int kMaxPerSmForSizing = 4;
 
-// workspace: [counters (units ints, 256-aligned)] [partials units x S x (m[8], l[8], o[8][D]) fp32]
+// workspace: [counters (units ints, 256-aligned)] [cluster partials units x (S/16) x (m[8], l[8], o[8][D])
+// fp32, only when a unit has more than one cluster]
 size_t ws_cnt_bytes(size_t units) { return ((units * 4 + 255) / 256) * 256; }
 
 size_t ws_bytes_for(int B, int Hq, int Hkv, int D, int S_max, int HT) {
   const size_t units = (size_t)B * Hkv * HT;
-  const size_t part = units * (size_t)S_max * (2 * kHT + kHT * D) * 4;
+  const size_t ncl = S_max > kMaxClusterThroughput ? (S_max + kMaxClusterThroughput - 1) / kMaxClusterThroughput : 0;
+  const size_t part = units * ncl * (2 * kHT + kHT * D) * 4;
   return ws_cnt_bytes(units) + part;
 }
 
@@ -872,8 +906,19 @@ kvq_status run_attend(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q,
   prm.vd = INT4 ? pv->dec_dev : nullptr;
   dim3 grid(sp.S, sp.HT, B * Hkv);
   if (grid.z > 65535u) return fail(KVQ_ERR_UNSUPPORTED, "attend: B * Hkv > 65535");
-  attend_kernel<D, INT4><<<grid, kThreads, C::kSmem, strm>>>(kmap, vmap, ksmap, vsmap, prm);
-  const cudaError_t e = cudaGetLastError();
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = strm;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)sp.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, attend_kernel<D, INT4>, kmap, vmap, ksmap, vsmap, prm);
   if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
   return KVQ_OK;
 }

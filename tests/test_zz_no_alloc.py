@@ -2,13 +2,11 @@
 allocate device memory (memory planned up front, code running under stream
 capture, hosts whose allocator belongs to someone else). Its scratch is a static
 array inside the library, so this checks, through the C ABI, that two calls in a
-row give what the workspace-taking kvq_attend_decode gives, and that shapes too
-large for the static scratch are refused before anything runs.
+row give what the workspace-taking kvq_attend_decode gives. Every call passes
+real, correctly sized device buffers.
 
 Kept in a file that pytest collects last; it must pass on its own in a fresh
 process and after every other test."""
-import ctypes
-
 import numpy as np
 import pytest
 
@@ -52,20 +50,3 @@ def test_noalloc_matches_workspace_entry_point_twice(name, B, Hkv, Hq, T, lens):
         torch.cuda.synchronize()
         check_rel_l2(got.float().cpu().numpy().reshape(-1, D), ref.reshape(-1, D), tol=REL_L2, label=name)
     assert kvq.poll_device_errors() == 0
-
-
-def test_noalloc_refuses_shapes_beyond_static_scratch():
-    import rotated_int4_kv_b200 as kvq
-    from rotated_int4_kv_b200 import lib
-
-    D = 128
-    pk = kvq.Plan(*kvgen.plan_params(D, kind="k"))
-    pv = kvq.Plan(*kvgen.plan_params(D, kind="v"))
-    # 2048 x 8 KV heads x 64 query heads: the per-head-tile rotated queries alone exceed 8 MiB.
-    # The size check happens on the host before any pointer is touched, so 16-byte aligned
-    # placeholder addresses are enough.
-    fake = ctypes.c_void_p(1 << 20)
-    st = lib.kvq_attend_decode_noalloc(pk.handle, pv.handle, fake, fake, fake, fake, fake, 2048, 64, 8, 256, None,
-                                       256, ctypes.c_float(0.0), fake, None)
-    assert st == -6
-    assert b"static scratch" in lib.kvq_last_error()
