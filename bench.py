@@ -247,7 +247,7 @@ def run_kvq(args, rank: int, world: int):
                           codes[2 * l + 1:2 * l + 2], scales[2 * l + 1:2 * l + 2], T_len=T, out=out[l],
                           workspace=ws[l], stream=stream)
 
-    n_side = 8
+    n_side = L  # one stream per layer: the layers' attentions are independent in this step
     side = [torch.cuda.Stream(device=dev) for _ in range(n_side)]
 
     def attn_phase():

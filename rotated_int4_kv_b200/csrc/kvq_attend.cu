@@ -325,9 +325,10 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
         uint8_t* st = ring + s * C::kStageBytes;
         const int t0 = t_begin + i * kTileT;
         mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+        const uint64_t pol = l2_evict_first_policy();
         if constexpr (INT4) {
-          tma_load_2d(st, &kmap, &full[s], 0, row0 + t0);
-          tma_load_2d(st + C::kKBytes, &vmap, &full[s], 0, row0 + t0);
+          tma_load_2d_hint(st, &kmap, &full[s], 0, row0 + t0, pol);
+          tma_load_2d_hint(st + C::kKBytes, &vmap, &full[s], 0, row0 + t0, pol);
 #pragma unroll
           for (int j = 0; j < C::kScaleLoads; ++j) {
             tma_load_2d(st + 2 * C::kKBytes + j * C::kScaleBox * 2, &ksmap, &full[s], t0 * NG + j * C::kScaleBox, bk);
@@ -337,8 +338,8 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
         } else {
 #pragma unroll
           for (int j = 0; j < D / 64; ++j) {
-            tma_load_2d(st + j * kTileT * 128, &kmap, &full[s], 64 * j, row0 + t0);
-            tma_load_2d(st + C::kKBytes + j * kTileT * 128, &vmap, &full[s], 64 * j, row0 + t0);
+            tma_load_2d_hint(st + j * kTileT * 128, &kmap, &full[s], 64 * j, row0 + t0, pol);
+            tma_load_2d_hint(st + C::kKBytes + j * kTileT * 128, &vmap, &full[s], 64 * j, row0 + t0, pol);
           }
         }
       }

@@ -185,9 +185,10 @@ __global__ void __launch_bounds__(kNT, 3) encode_kernel(const __grid_constant__ 
     const int tb = lt / J.n_ttiles;
     const int bh0 = tb * J.BH_box, t0 = (lt - tb * J.n_ttiles) * J.T_box;
     mbar_arrive_expect_tx(&full[stage], C::kXStage);
+    const uint64_t pol = l2_evict_first_policy();
 #pragma unroll
     for (int b = 0; b < D / 64; ++b)
-      tma_load_3d(xs + stage * C::kXStage + b * C::kBoxBytes, &J.xmap, &full[stage], b * 64, t0, bh0);
+      tma_load_3d_hint(xs + stage * C::kXStage + b * C::kBoxBytes, &J.xmap, &full[stage], b * 64, t0, bh0, pol);
   };
   if (tid == 0) {
     for (int s2 = 0; s2 < C::kStages; ++s2) {
