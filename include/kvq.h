@@ -168,6 +168,36 @@ kvq_status kvq_attend_decode(const kvq_plan* pk, const kvq_plan* pv, const uint1
                              size_t ws_bytes, void* stream);
 
 /*
+ * kvq_attend_decode_batch -- kvq_attend_decode for many independent problems of one
+ * shape in one grouped launch (up to 32 per launch; more are run as consecutive
+ * launches on the stream), e.g. the decode attention of every layer of a model
+ * step when the layers' queries are already known, or several caches of one
+ * shape. Each job is exactly one kvq_attend_decode call with the shared sizes.
+ *   jobs     host array of njobs descriptors (read during the call only). All plans
+ *            share one head_dim, group (32) and device.
+ *   B, Hq, Hkv, T_cap, seq_lens, T_len, softmax_scale   shared by every job.
+ *   workspace  >= kvq_workspace_size(min(njobs, 32) * B, Hq, Hkv, D, T_cap) bytes,
+ *            counters zero before the first use (every call leaves them zero).
+ * Errors: as kvq_attend_decode, reported for the first offending job; nothing is
+ * launched when any job fails validation.
+ */
+typedef struct kvq_attend_job {
+  const kvq_plan* pk;        /* K plan */
+  const kvq_plan* pv;        /* V plan */
+  const uint16_t* q;         /* fp16 [B, Hq, D] */
+  const uint8_t* k_codes;    /* u8   [B, Hkv, T_cap, D/2] */
+  const uint16_t* k_scales;  /* fp16 [B, Hkv, T_cap, D/32] */
+  const uint8_t* v_codes;
+  const uint16_t* v_scales;
+  uint16_t* out;             /* fp16 [B, Hq, D] */
+} kvq_attend_job;
+
+kvq_status kvq_attend_decode_batch(const kvq_attend_job* jobs, int njobs, int B, int Hq, int Hkv,
+                                   int T_cap, const int32_t* seq_lens, int T_len,
+                                   float softmax_scale, void* workspace, size_t ws_bytes,
+                                   void* stream);
+
+/*
  * kvq_attend_decode_noalloc -- kvq_attend_decode for callers that cannot allocate
  * device memory: a serving runtime whose memory is planned up front, code that
  * runs while a stream is being captured (cudaMalloc is not allowed there), or a

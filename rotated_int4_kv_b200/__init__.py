@@ -4,8 +4,9 @@ The compute path lives in ``libkvq.so`` (hand-written CUDA for sm_100a, C ABI in
 ``include/kvq.h``); this package only marshals torch tensors into it.
 """
 from ._lib import LIB_PATH, KvqError, lib  # noqa: F401
-from .api import (Plan, attend_decode, attend_decode_noalloc, attend_decode_ref, decode, encode,  # noqa: F401
-                  encode_batch, make_workspace, poll_device_errors, workspace_size)
+from .api import (Plan, attend_decode, attend_decode_batch, attend_decode_noalloc, attend_decode_ref,  # noqa: F401
+                  decode, encode, encode_batch, make_workspace, poll_device_errors, workspace_size)
 
-__all__ = ["Plan", "encode", "encode_batch", "decode", "attend_decode", "attend_decode_noalloc", "attend_decode_ref", "workspace_size", "make_workspace",
-           "poll_device_errors", "KvqError", "LIB_PATH", "lib"]
+__all__ = ["Plan", "encode", "encode_batch", "decode", "attend_decode", "attend_decode_batch",
+           "attend_decode_noalloc", "attend_decode_ref", "workspace_size", "make_workspace", "poll_device_errors",
+           "KvqError", "LIB_PATH", "lib"]

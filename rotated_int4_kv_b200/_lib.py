@@ -25,9 +25,16 @@ class EncodeJob(ctypes.Structure):
                 ("T_cap", ctypes.c_int), ("pos", ctypes.c_int)]
 
 
+class AttendJob(ctypes.Structure):
+    """Mirror of ``kvq_attend_job`` in include/kvq.h."""
+    _fields_ = [("pk", ctypes.c_void_p), ("pv", ctypes.c_void_p), ("q", ctypes.c_void_p),
+                ("k_codes", ctypes.c_void_p), ("k_scales", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
+                ("v_scales", ctypes.c_void_p), ("out", ctypes.c_void_p)]
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
-        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m rotated_int4_kv_b200.build` "
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python rotated_int4_kv_b200/build.py` "
                           "(nvcc, sm_100a). There is no fallback implementation.")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, F, S, U32P = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.POINTER(ctypes.c_uint32)
@@ -43,6 +50,7 @@ def _load() -> ctypes.CDLL:
         "kvq_attend_decode": (I, [P, P, P, P, P, P, P, I, I, I, I, P, I, F, P, P, S, P]),
         "kvq_attend_decode_ref": (I, [P, P, P, I, I, I, I, I, P, I, F, P, P, S, P]),
         "kvq_attend_decode_noalloc": (I, [P, P, P, P, P, P, P, I, I, I, I, P, I, F, P, P]),
+        "kvq_attend_decode_batch": (I, [ctypes.POINTER(AttendJob), I, I, I, I, I, P, I, F, P, S, P]),
         "kvq_poll_device_errors": (I, [U32P]),
         "kvq_status_string": (ctypes.c_char_p, [I]),
         "kvq_last_error": (ctypes.c_char_p, []),

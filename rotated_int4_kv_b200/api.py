@@ -10,7 +10,7 @@ import ctypes
 import numpy as np
 import torch
 
-from ._lib import EncodeJob, check, lib
+from ._lib import AttendJob, EncodeJob, check, lib
 
 
 def _stream(stream) -> ctypes.c_void_p:
@@ -143,6 +143,44 @@ def attend_decode(pk: Plan, pv: Plan, q, k_codes, k_scales, v_codes, v_scales, s
                                 float(softmax_scale), _ptr(out), _ptr(workspace), workspace.numel(),
                                 _stream(stream)), "kvq_attend_decode")
     return out
+
+
+def attend_decode_batch(jobs, seq_lens=None, T_len=None, softmax_scale: float = 0.0, workspace=None,
+                        stream=None) -> list:
+    """Grouped int4 decode attention: ``jobs`` is a sequence of
+    (pk, pv, q, k_codes, k_scales, v_codes, v_scales[, out]) tuples of one shape,
+    each exactly what :func:`attend_decode` takes; up to 32 run per launch.
+    Returns the list of outputs."""
+    if not jobs:
+        return []
+    q0, kc0 = jobs[0][2], jobs[0][3]
+    B, Hq, D = q0.shape
+    _, Hkv, T_cap, _ = kc0.shape
+    arr = (AttendJob * len(jobs))()
+    outs = []
+    for i, job in enumerate(jobs):
+        pk, pv, q, k_codes, k_scales, v_codes, v_scales = job[:7]
+        out = job[7] if len(job) > 7 and job[7] is not None else torch.empty((B, Hq, D), dtype=torch.float16,
+                                                                             device=q.device)
+        _need(q, f"jobs[{i}].q", torch.float16, (B, Hq, D))
+        for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
+            _need(t, f"jobs[{i}].{name}", torch.uint8, (B, Hkv, T_cap, D // 2))
+        for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+            _need(t, f"jobs[{i}].{name}", torch.float16, (B, Hkv, T_cap, D // pk.group))
+        _need(out, f"jobs[{i}].out", torch.float16, (B, Hq, D))
+        arr[i] = AttendJob(pk.handle.value, pv.handle.value, q.data_ptr(), k_codes.data_ptr(), k_scales.data_ptr(),
+                           v_codes.data_ptr(), v_scales.data_ptr(), out.data_ptr())
+        outs.append(out)
+    if seq_lens is not None:
+        _need(seq_lens, "seq_lens", torch.int32, (B,))
+    if T_len is None:
+        T_len = T_cap if seq_lens is None else 0
+    if workspace is None:
+        workspace = make_workspace(min(len(jobs), 32) * B, Hq, Hkv, D, T_cap, q0.device)
+    check(lib.kvq_attend_decode_batch(arr, len(jobs), B, Hq, Hkv, T_cap, _ptr(seq_lens), int(T_len),
+                                      float(softmax_scale), _ptr(workspace), workspace.numel(), _stream(stream)),
+          "kvq_attend_decode_batch")
+    return outs
 
 
 def attend_decode_noalloc(pk: Plan, pv: Plan, q, k_codes, k_scales, v_codes, v_scales, seq_lens=None, T_len=None,

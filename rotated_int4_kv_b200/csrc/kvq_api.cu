@@ -321,6 +321,41 @@ kvq_status kvq_attend_decode(const kvq_plan* pk, const kvq_plan* pv, const uint1
                                  ws_bytes, (cudaStream_t)stream);
 }
 
+kvq_status kvq_attend_decode_batch(const kvq_attend_job* jobs, int njobs, int B, int Hq, int Hkv, int T_cap,
+                                   const int32_t* seq_lens, int T_len, float sigma, void* ws, size_t ws_bytes,
+                                   void* stream) {
+  if (njobs < 0 || (njobs > 0 && !jobs)) return fail(KVQ_ERR_INVALID_ARG, "attend_batch: bad job array");
+  if (njobs == 0) return KVQ_OK;
+  const kvq_plan* p0 = jobs[0].pk;
+  if (!p0) return fail(KVQ_ERR_INVALID_ARG, "attend_batch: job 0: null plan");
+  std::vector<kvq::AttendJobHost> hj((size_t)njobs);
+  for (int i = 0; i < njobs; ++i) {
+    const kvq_attend_job& j = jobs[i];
+    const std::string tag = "attend_batch: job " + std::to_string(i) + ": ";
+    if (!j.pk || !j.pv) return fail(KVQ_ERR_INVALID_ARG, tag + "null plan");
+    if (j.pk->D != p0->D || j.pv->D != p0->D || j.pk->G != p0->G || j.pv->G != p0->G ||
+        j.pk->device != p0->device || j.pv->device != p0->device)
+      return fail(KVQ_ERR_INVALID_ARG, tag + "plans differ in head_dim, group or device");
+    if (j.pk->G != 32) return fail(KVQ_ERR_UNSUPPORTED, tag + "group must be 32");
+    kvq_status st = check_attend_common(B, Hq, Hkv, p0->D, T_cap, T_len, j.q, j.out, ws, ws_bytes);
+    if (st != KVQ_OK) return fail(st, tag + kvq_last_error());
+    if (B == 0) continue;
+    if (!j.k_codes || !j.k_scales || !j.v_codes || !j.v_scales) return fail(KVQ_ERR_INVALID_ARG, tag + "null cache buffer");
+    if (!kvq::aligned16(j.k_codes) || !kvq::aligned16(j.k_scales) || !kvq::aligned16(j.v_codes) ||
+        !kvq::aligned16(j.v_scales))
+      return fail(KVQ_ERR_ALIGNMENT, tag + "cache buffers must be 16-byte aligned");
+    hj[(size_t)i] = kvq::AttendJobHost{j.pk, j.pv, j.q, j.k_codes, j.k_scales, j.v_codes, j.v_scales, j.out};
+  }
+  if (B == 0) return KVQ_OK;
+  if ((size_t)B * std::min(njobs, 32) * Hkv > 65535u) return fail(KVQ_ERR_UNSUPPORTED, "attend_batch: 32 * B * Hkv > 65535");
+  const size_t need = kvq::attend_workspace_bytes(B * std::min(njobs, 32), Hq, Hkv, p0->D, T_cap);
+  if (ws_bytes < need) return fail(KVQ_ERR_WORKSPACE, "attend_batch: workspace too small (size it for min(njobs, 32) * B)");
+  kvq_status st = kvq::check_plan_device(p0);
+  if (st != KVQ_OK) return st;
+  return kvq::launch_attend_int4_batch(hj.data(), njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes,
+                                       (cudaStream_t)stream);
+}
+
 kvq_status kvq_attend_decode_noalloc(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q, const uint8_t* kc,
                                      const uint16_t* ks, const uint8_t* vc, const uint16_t* vs, int B, int Hq,
                                      int Hkv, int T_cap, const int32_t* seq_lens, int T_len, float sigma,

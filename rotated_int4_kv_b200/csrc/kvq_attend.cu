@@ -56,7 +56,8 @@ constexpr int kMaxSplitsCfg = 256;          // upper bound on splits per unit
 constexpr int kMaxCluster = 8;              // splits merged through distributed shared memory
 constexpr int kMaxClusterLatency = 8;
 constexpr int kMaxClusterThroughput = 4;
-constexpr int kMaxMerge = kMaxSplitsCfg / 4;  // clusters per unit (>= 4 splits each) or splits per cluster
+constexpr int kMaxMerge = kMaxSplitsCfg / 4;  // cluster partials per unit merged through the workspace
+constexpr int kMaxJobs = 32;                // problems per launch of a batch (job table in parameter space)
 
 template <int D, bool INT4>
 struct Cfg {
@@ -75,20 +76,45 @@ struct Cfg {
   static constexpr int kTail = ((kCWarps + 1) * (2 * kHT + kHT * D) + 2 * kHT + 2 * kMaxMerge * kHT + kHT * D) * 4;
   static constexpr int kScratch = kRing > kTail ? kRing : kTail;
   static constexpr int kQt = kHT * D * 4;                  // fp32 q_t (or merged o_t) [8][D]
-  static constexpr int kSmem = kScratch + kQt + 64 + 1024;
+  // staged at kernel start by bulk copies: the tile's query rows (fp16 [8][D]) and,
+  // for int4, the plans' per-channel factors and sign masks (K: dg/lambda, masks;
+  // V: dg/lambda, masks)
+  static constexpr int kQs = kHT * D * 2;
+  static constexpr int kChanBytes = D * 4;
+  static constexpr int kSgnBytes = D * 2;  // one u32 mask per fp16 pair
+  static constexpr int kConsts = INT4 ? 2 * (kChanBytes + kSgnBytes) : 0;
+  // B fragments of the score product, one 16-byte entry per (k step, lane):
+  // (hi01, hi23, lo01, lo23) -- read from shared memory at each use
+  static constexpr int kKSteps = INT4 ? 2 * NG : D / 16;
+  static constexpr int kQf = kKSteps * 32 * 16;
+  static constexpr int kBars = 128;        // full[], empty[], const barrier, flag
+  static constexpr int kSmem = kScratch + kQt + kQs + kConsts + kQf + kBars + 1024;
+  static_assert(2 * kStages * 8 + 8 + 4 <= kBars, "barrier region");
 };
 
 struct AttnParams {
-  const uint16_t* q;
-  uint16_t* out;
   const int32_t* seq_lens;
   int T_len, B, Hq, Hkv, T_cap, G, HT, S, tps;  // tps = tokens per split (multiple of kTileT)
   float sl2;                                   // softmax scale * log2(e)
   float* part;                                 // [units][S][2*8 + 8*D]
   int* cnt;                                    // [units]
-  const CodecConsts* ke;                       // K plan: sign masks (int4 only)
-  const CodecConsts* kd;                       // K plan: dg / lambda per channel
-  const CodecConsts* vd;                       // V plan: dg / lambda per channel, sign masks
+};
+
+// One attention problem of a launch: its caches (as tensor maps), query, output
+// and the two plans' constants. A launch runs MAXJ of them with shared shapes;
+// blockIdx.z = job * (B * Hkv) + b * Hkv + kv head.
+struct alignas(64) AttnJob {
+  CUtensorMap kmap, vmap, ksmap, vsmap;  // K/V codes (or fp16 K/V) and scale rows
+  const uint16_t* q;
+  uint16_t* out;
+  const CodecConsts* ke;  // K plan: sign masks (int4 only)
+  const CodecConsts* kd;  // K plan: dg / lambda per channel
+  const CodecConsts* vd;  // V plan: dg / lambda per channel, sign masks
+};
+
+template <int MAXJ>
+struct AttnJobs {
+  AttnJob j[MAXJ];
 };
 
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
@@ -130,17 +156,17 @@ __device__ __forceinline__ void split_h(float x, __half& hi, __half& lo) {
 // FFT: one lane per head at D = 128, a lane pair per head at D = 256 (all 32
 // lanes of the calling warp execute it; lanes beyond the real heads work on zeros).
 template <int D>
-__device__ __forceinline__ void rotate_query(const uint16_t* __restrict__ qb, int heads, const CodecConsts* ke,
-                                             const CodecConsts* kd, float* qt, int lane) {
+__device__ __forceinline__ void rotate_query(const uint16_t* qs, int heads, const uint32_t* ksg, const float* kch,
+                                             float* qt, int lane) {
   float2 v[64];
   if constexpr (D == 128) {
     const int h = lane;
     const bool live = h < heads;
-    const uint4* src = reinterpret_cast<const uint4*>(qb + (size_t)(live ? h : 0) * D);
+    const uint4* src = reinterpret_cast<const uint4*>(qs + (live ? h : 0) * D);
 #pragma unroll
     for (int cc = 0; cc < 16; ++cc) {
-      uint4 w = live ? __ldg(src + cc) : make_uint4(0u, 0u, 0u, 0u);
-      const uint4 m = __ldg(reinterpret_cast<const uint4*>(ke->sgn) + cc);
+      uint4 w = live ? src[cc] : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 m = reinterpret_cast<const uint4*>(ksg)[cc];
       const uint32_t ww[4] = {w.x ^ m.x, w.y ^ m.y, w.z ^ m.z, w.w ^ m.w};
 #pragma unroll
       for (int q = 0; q < 4; ++q) v[4 * cc + q] = __half22float2(*reinterpret_cast<const __half2*>(&ww[q]));
@@ -149,7 +175,7 @@ __device__ __forceinline__ void rotate_query(const uint16_t* __restrict__ qb, in
     if (live) {
 #pragma unroll
       for (int c4 = 0; c4 < 32; ++c4) {
-        const float4 k4 = __ldg(reinterpret_cast<const float4*>(kd->chan) + c4);
+        const float4 k4 = reinterpret_cast<const float4*>(kch)[c4];
         float4 o;
         o.x = slotv(v, slot_of_channel(4 * c4 + 0, 128)) * k4.x;
         o.y = slotv(v, slot_of_channel(4 * c4 + 1, 128)) * k4.y;
@@ -163,11 +189,11 @@ __device__ __forceinline__ void rotate_query(const uint16_t* __restrict__ qb, in
     const bool p = (lane & 1) != 0;
     const bool live = h < heads;
     const uint32_t sel = p ? 0x7632u : 0x5410u;
-    const uint4* src = reinterpret_cast<const uint4*>(qb + (size_t)(live ? h : 0) * D);
+    const uint4* src = reinterpret_cast<const uint4*>(qs + (live ? h : 0) * D);
 #pragma unroll
     for (int cc = 0; cc < 32; ++cc) {  // thread p takes q[8cc + p + 2i]
-      const uint4 w = live ? __ldg(src + cc) : make_uint4(0u, 0u, 0u, 0u);
-      const uint4 m = __ldg(reinterpret_cast<const uint4*>(ke->sgn) + cc);
+      const uint4 w = live ? src[cc] : make_uint4(0u, 0u, 0u, 0u);
+      const uint4 m = reinterpret_cast<const uint4*>(ksg)[cc];
       uint32_t h0 = prmt(w.x ^ m.x, w.y ^ m.y, sel);
       uint32_t h1 = prmt(w.z ^ m.z, w.w ^ m.w, sel);
       v[2 * cc] = __half22float2(*reinterpret_cast<const __half2*>(&h0));
@@ -182,7 +208,7 @@ __device__ __forceinline__ void rotate_query(const uint16_t* __restrict__ qb, in
         const int cb = half ? (p ? 128 : 192) : (p ? 64 : 0);
 #pragma unroll
         for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 k4 = __ldg(reinterpret_cast<const float4*>(kd->chan + cb) + c4);
+          const float4 k4 = reinterpret_cast<const float4*>(kch + cb)[c4];
           const int L = 64 * half + 4 * c4;
           reinterpret_cast<float4*>(qt + h * D + cb)[c4] =
               make_float4(o[L] * k4.x, o[L + 1] * k4.y, o[L + 2] * k4.z, o[L + 3] * k4.w);
@@ -192,20 +218,24 @@ __device__ __forceinline__ void rotate_query(const uint16_t* __restrict__ qb, in
   }
 }
 
-// x = F_r^T Lambda_V^-1 o_t (without the sign, applied at the fp16 store) for the
-// real heads, by the inverse register FFT; writes fp32 x[h][n] to xb.
+// x = F_r^T Lambda_V^-1 o_t / L_h (without the sign, applied at the fp16 store)
+// for the real heads, by the inverse register FFT; writes fp32 x[h][n] to xb.
+// vch: dg / lambda per rotated channel (shared memory); Lh: softmax denominators.
 template <int D>
-__device__ __forceinline__ void unrotate_out(const float* om, int heads, const CodecConsts* vd, float* xb, int lane) {
+__device__ __forceinline__ void unrotate_out(const float* om, int heads, const float* vch, const float* Lh, float* xb,
+                                             int lane) {
   float2 u[64];
   if constexpr (D == 128) {
     const int h = lane;
     const bool live = h < heads;
     const float* oh = om + (live ? h : 0) * D;
+    const float L = live ? Lh[h] : 0.0f;
+    const float r = L > 0.0f ? 1.0f / L : 0.0f;
 #pragma unroll
     for (int c4 = 0; c4 < 32; ++c4) {
-      const float4 k4 = __ldg(reinterpret_cast<const float4*>(vd->chan) + c4);
+      const float4 k4 = reinterpret_cast<const float4*>(vch)[c4];
       const float4 o4 = live ? reinterpret_cast<const float4*>(oh)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float ov[4] = {o4.x * k4.x, o4.y * k4.y, o4.z * k4.z, o4.w * k4.w};
+      const float ov[4] = {o4.x * k4.x * r, o4.y * k4.y * r, o4.z * k4.z * r, o4.w * k4.w * r};
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int sl = slot_of_channel(4 * c4 + e, 128);
@@ -226,19 +256,21 @@ __device__ __forceinline__ void unrotate_out(const float* om, int heads, const C
     const bool p = (lane & 1) != 0;
     const bool live = h < heads;
     const float* oh = om + (live ? h : 0) * D;
+    const float L = live ? Lh[h] : 0.0f;
+    const float r = L > 0.0f ? 1.0f / L : 0.0f;
     float o[128];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
       const int cb = half ? (p ? 128 : 192) : (p ? 64 : 0);
 #pragma unroll
       for (int c4 = 0; c4 < 16; ++c4) {
-        const float4 k4 = __ldg(reinterpret_cast<const float4*>(vd->chan + cb) + c4);
+        const float4 k4 = reinterpret_cast<const float4*>(vch + cb)[c4];
         const float4 o4 = live ? reinterpret_cast<const float4*>(oh + cb)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
-        const int L = 64 * half + 4 * c4;
-        o[L] = o4.x * k4.x;
-        o[L + 1] = o4.y * k4.y;
-        o[L + 2] = o4.z * k4.z;
-        o[L + 3] = o4.w * k4.w;
+        const int m = 64 * half + 4 * c4;
+        o[m] = o4.x * k4.x * r;
+        o[m + 1] = o4.y * k4.y * r;
+        o[m + 2] = o4.z * k4.z * r;
+        o[m + 3] = o4.w * k4.w * r;
       }
     }
 #pragma unroll
@@ -255,12 +287,9 @@ __device__ __forceinline__ void unrotate_out(const float* om, int heads, const C
   }
 }
 
-template <int D, bool INT4>
-__global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(const __grid_constant__ CUtensorMap kmap,
-                                                             const __grid_constant__ CUtensorMap vmap,
-                                                             const __grid_constant__ CUtensorMap ksmap,
-                                                             const __grid_constant__ CUtensorMap vsmap,
-                                                             const AttnParams p) {
+template <int D, bool INT4, int MAXJ>
+__global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
+    attend_kernel(const __grid_constant__ AttnJobs<MAXJ> jt, const __grid_constant__ AttnParams p) {
   using C = Cfg<D, INT4>;
   constexpr int NG = C::NG;
   constexpr int MT = D / 16;  // channel m-tiles of the PV product
@@ -268,18 +297,29 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
   float* qt = reinterpret_cast<float*>(smem + C::kScratch);      // [8][D]
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kScratch + C::kQt);
+  uint16_t* qs = reinterpret_cast<uint16_t*>(smem + C::kScratch + C::kQt);  // fp16 [heads][D]
+  uint8_t* cst = smem + C::kScratch + C::kQt + C::kQs;
+  const float* kch = reinterpret_cast<const float*>(cst);
+  const uint32_t* ksg = reinterpret_cast<const uint32_t*>(cst + C::kChanBytes);
+  const float* vch = reinterpret_cast<const float*>(cst + C::kChanBytes + C::kSgnBytes);
+  const uint32_t* vsg = reinterpret_cast<const uint32_t*>(cst + 2 * C::kChanBytes + C::kSgnBytes);
+  uint4* qf = reinterpret_cast<uint4*>(smem + C::kScratch + C::kQt + C::kQs + C::kConsts);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kScratch + C::kQt + C::kQs + C::kConsts + C::kQf);
   uint64_t* empty = full + C::kStages;
-  int* flag = reinterpret_cast<int*>(empty + C::kStages);
+  uint64_t* cbar = empty + C::kStages;
+  int* flag = reinterpret_cast<int*>(cbar + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
-  const int split = blockIdx.x, ht = blockIdx.y, bk = blockIdx.z;
+  const int split = blockIdx.x, ht = blockIdx.y;
+  const int job = MAXJ == 1 ? 0 : (int)blockIdx.z / (p.B * p.Hkv);
+  const int bk = (int)blockIdx.z - job * (p.B * p.Hkv);
+  const AttnJob& J = jt.j[job];
   const int b = bk / p.Hkv, kvh = bk - b * p.Hkv;
   const int heads = min(kHT, p.G - ht * kHT);  // real heads in this tile
   const int hq0 = kvh * p.G + ht * kHT;        // first query head
-  const int unit = bk * p.HT + ht;
+  const int unit = (int)blockIdx.z * p.HT + ht;  // workspace slot (over all jobs)
 
   int T_b = p.T_len;
   if (p.seq_lens) T_b = min(max(__ldg(p.seq_lens + b), 0), p.T_cap);
@@ -293,6 +333,7 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kCWarps);
     }
+    mbar_init(cbar, 1);
     fence_mbarrier_init();
   }
   __syncthreads();
@@ -308,11 +349,21 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
   if (warp == kCWarps) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      prefetch_tensormap(&kmap);
-      prefetch_tensormap(&vmap);
+      // query rows of the tile and the plans' constants: one round trip, one barrier
+      const uint32_t qbytes = (uint32_t)(heads * D * 2);
+      mbar_arrive_expect_tx(cbar, qbytes + (INT4 ? (uint32_t)C::kConsts : 0u));
+      bulk_load(qs, J.q + ((size_t)b * p.Hq + hq0) * D, qbytes, cbar);
       if constexpr (INT4) {
-        prefetch_tensormap(&ksmap);
-        prefetch_tensormap(&vsmap);
+        bulk_load(cst, J.kd->chan, C::kChanBytes, cbar);
+        bulk_load(cst + C::kChanBytes, J.ke->sgn, C::kSgnBytes, cbar);
+        bulk_load(cst + C::kChanBytes + C::kSgnBytes, J.vd->chan, C::kChanBytes, cbar);
+        bulk_load(cst + 2 * C::kChanBytes + C::kSgnBytes, J.vd->sgn, C::kSgnBytes, cbar);
+      }
+      prefetch_tensormap(&J.kmap);
+      prefetch_tensormap(&J.vmap);
+      if constexpr (INT4) {
+        prefetch_tensormap(&J.ksmap);
+        prefetch_tensormap(&J.vsmap);
       }
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % C::kStages;
@@ -327,19 +378,19 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
         mbar_arrive_expect_tx(&full[s], C::kStageBytes);
         const uint64_t pol = l2_evict_first_policy();
         if constexpr (INT4) {
-          tma_load_2d_hint(st, &kmap, &full[s], 0, row0 + t0, pol);
-          tma_load_2d_hint(st + C::kKBytes, &vmap, &full[s], 0, row0 + t0, pol);
+          tma_load_2d_hint(st, &J.kmap, &full[s], 0, row0 + t0, pol);
+          tma_load_2d_hint(st + C::kKBytes, &J.vmap, &full[s], 0, row0 + t0, pol);
 #pragma unroll
           for (int j = 0; j < C::kScaleLoads; ++j) {
-            tma_load_2d(st + 2 * C::kKBytes + j * C::kScaleBox * 2, &ksmap, &full[s], t0 * NG + j * C::kScaleBox, bk);
-            tma_load_2d(st + 2 * C::kKBytes + C::kSBytes + j * C::kScaleBox * 2, &vsmap, &full[s],
+            tma_load_2d(st + 2 * C::kKBytes + j * C::kScaleBox * 2, &J.ksmap, &full[s], t0 * NG + j * C::kScaleBox, bk);
+            tma_load_2d(st + 2 * C::kKBytes + C::kSBytes + j * C::kScaleBox * 2, &J.vsmap, &full[s],
                         t0 * NG + j * C::kScaleBox, bk);
           }
         } else {
 #pragma unroll
           for (int j = 0; j < D / 64; ++j) {
-            tma_load_2d_hint(st + j * kTileT * 128, &kmap, &full[s], 64 * j, row0 + t0, pol);
-            tma_load_2d_hint(st + C::kKBytes + j * kTileT * 128, &vmap, &full[s], 64 * j, row0 + t0, pol);
+            tma_load_2d_hint(st + j * kTileT * 128, &J.kmap, &full[s], 64 * j, row0 + t0, pol);
+            tma_load_2d_hint(st + C::kKBytes + j * kTileT * 128, &J.vmap, &full[s], 64 * j, row0 + t0, pol);
           }
         }
       }
@@ -347,27 +398,28 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
   } else {
     // ------------------------------------------------------------ consumers
     // (1) the query in the K transform's rotated domain (int4) or q itself (fp16)
-    const uint16_t* qb = p.q + ((size_t)b * p.Hq + hq0) * D;
+    if (!mbar_wait_bounded(cbar, 0)) {
+      atomicOr(&g_attend_err, kErrTimeoutLoad);
+      ok = false;
+    }
     if constexpr (INT4) {
-      if (warp == 0) rotate_query<D>(qb, heads, p.ke, p.kd, qt, lane);
+      if (warp == 0) rotate_query<D>(qs, heads, ksg, kch, qt, lane);
       for (int i = threadIdx.x; i < (kHT - heads) * D; i += kCWarps * 32) qt[heads * D + i] = 0.0f;
     } else {
       for (int i = threadIdx.x; i < kHT * D / 2; i += kCWarps * 32) {
         const int h = (2 * i) / D;
-        const float2 f = h < heads ? __half22float2(__ldg(reinterpret_cast<const __half2*>(qb) + i))
-                                   : make_float2(0.0f, 0.0f);
+        const float2 f = h < heads ? __half22float2(reinterpret_cast<const __half2*>(qs)[i]) : make_float2(0.0f, 0.0f);
         reinterpret_cast<float2*>(qt)[i] = f;
       }
     }
     consumer_sync();
 
-    // (2) B fragments of the score product (n = head g)
-    constexpr int kKSteps = INT4 ? 2 * NG : D / 16;
-    uint32_t qb_hi[kKSteps][2], qb_lo[kKSteps][2];
+    // (2) B fragments of the score product (n = head g), built once per CTA into
+    // shared memory (warp w takes k steps w, w + 4, ...)
+    constexpr int kKSteps = C::kKSteps;
     {
       const float* qh = qt + g * D;
-#pragma unroll
-      for (int ks = 0; ks < kKSteps; ++ks) {
+      for (int ks = warp; ks < kKSteps; ks += kCWarps) {
         int ch[4];
         if constexpr (INT4) {
           // group G = ks/2; step A: (8c, 8c+4 | 8c+1, 8c+5); step B: (8c+2, 8c+6 | 8c+3, 8c+7)
@@ -385,12 +437,11 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
         __half hi[4], lo[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) split_h(qh[ch[e]], hi[e], lo[e]);
-        qb_hi[ks][0] = h2_bits(__halves2half2(hi[0], hi[1]));
-        qb_hi[ks][1] = h2_bits(__halves2half2(hi[2], hi[3]));
-        qb_lo[ks][0] = h2_bits(__halves2half2(lo[0], lo[1]));
-        qb_lo[ks][1] = h2_bits(__halves2half2(lo[2], lo[3]));
+        qf[ks * 32 + lane] = make_uint4(h2_bits(__halves2half2(hi[0], hi[1])), h2_bits(__halves2half2(hi[2], hi[3])),
+                                        h2_bits(__halves2half2(lo[0], lo[1])), h2_bits(__halves2half2(lo[2], lo[3])));
       }
     }
+    consumer_sync();
 
     // (3) stream the token range
     const int lane_a = 4 * (2 * c) + (g >> 1);
@@ -442,14 +493,16 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
           nib8_to_h2(w3, hB1);
           const int G0 = 2 * gp, G1 = 2 * gp + 1;
           float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-          mma_16816(a0, hA0[0], hB0[0], hA0[1], hB0[1], qb_hi[2 * G0][0], qb_hi[2 * G0][1]);
-          mma_16816(a0, hA0[0], hB0[0], hA0[1], hB0[1], qb_lo[2 * G0][0], qb_lo[2 * G0][1]);
-          mma_16816(a0, hA0[2], hB0[2], hA0[3], hB0[3], qb_hi[2 * G0 + 1][0], qb_hi[2 * G0 + 1][1]);
-          mma_16816(a0, hA0[2], hB0[2], hA0[3], hB0[3], qb_lo[2 * G0 + 1][0], qb_lo[2 * G0 + 1][1]);
-          mma_16816(a1, hA1[0], hB1[0], hA1[1], hB1[1], qb_hi[2 * G1][0], qb_hi[2 * G1][1]);
-          mma_16816(a1, hA1[0], hB1[0], hA1[1], hB1[1], qb_lo[2 * G1][0], qb_lo[2 * G1][1]);
-          mma_16816(a1, hA1[2], hB1[2], hA1[3], hB1[3], qb_hi[2 * G1 + 1][0], qb_hi[2 * G1 + 1][1]);
-          mma_16816(a1, hA1[2], hB1[2], hA1[3], hB1[3], qb_lo[2 * G1 + 1][0], qb_lo[2 * G1 + 1][1]);
+          const uint4 f0 = qf[(2 * G0) * 32 + lane], f1 = qf[(2 * G0 + 1) * 32 + lane];
+          const uint4 f2 = qf[(2 * G1) * 32 + lane], f3 = qf[(2 * G1 + 1) * 32 + lane];
+          mma_16816(a0, hA0[0], hB0[0], hA0[1], hB0[1], f0.x, f0.y);
+          mma_16816(a0, hA0[0], hB0[0], hA0[1], hB0[1], f0.z, f0.w);
+          mma_16816(a0, hA0[2], hB0[2], hA0[3], hB0[3], f1.x, f1.y);
+          mma_16816(a0, hA0[2], hB0[2], hA0[3], hB0[3], f1.z, f1.w);
+          mma_16816(a1, hA1[0], hB1[0], hA1[1], hB1[1], f2.x, f2.y);
+          mma_16816(a1, hA1[0], hB1[0], hA1[1], hB1[1], f2.z, f2.w);
+          mma_16816(a1, hA1[2], hB1[2], hA1[3], hB1[3], f3.x, f3.y);
+          mma_16816(a1, hA1[2], hB1[2], hA1[3], hB1[3], f3.z, f3.w);
           sc[0] = fmaf(skA[G0], a0[0], fmaf(skA[G1], a1[0], sc[0]));
           sc[1] = fmaf(skA[G0], a0[1], fmaf(skA[G1], a1[1], sc[1]));
           sc[2] = fmaf(skB[G0], a0[2], fmaf(skB[G1], a1[2], sc[2]));
@@ -467,7 +520,8 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
           const int box = cc >> 3, ch = cc & 7;
           uint32_t a0, a1, a2, a3;
           ldmatrix_x4(a0, a1, a2, a3, smem_u32(kt + box * kTileT * 128 + row * 128 + ((ch ^ (row & 7)) << 4)));
-          mma_16816(sc, a0, a1, a2, a3, qb_hi[ks][0], qb_hi[ks][1]);
+          const uint4 f = qf[ks * 32 + lane];
+          mma_16816(sc, a0, a1, a2, a3, f.x, f.y);
         }
       }
       // base-2 scores with masking of tokens outside [t_begin, t_end)
@@ -699,6 +753,8 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
   if (crank == 0) merge(csize, [&](int r) { return static_cast<const float*>(cluster.map_shared_rank(cpart, r)); });
   cluster.sync();  // peers may leave once the leader has read their shared memory
   if (crank != 0) return;
+  // the producer warp reads staged constants below: observe their barrier too
+  if (warp == kCWarps && !mbar_wait_bounded(cbar, 0)) atomicOr(&g_attend_err, kErrTimeoutLoad);
 
   // ------------------------------------------------------------ more than one cluster per unit: global merge
   const int ncl = p.S / csize;
@@ -725,23 +781,21 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1) attend_kernel(cons
   }
 
   // ------------------------------------------------------------ normalise, un-rotate, store fp16
-  for (int i = threadIdx.x; i < heads * D; i += kThreads) {
-    const float L = mrg[kHT + i / D];
-    om[i] = L > 0.0f ? om[i] / L : 0.0f;
-  }
-  __syncthreads();
-  uint16_t* ob = p.out + ((size_t)b * p.Hq + hq0) * D;
+  uint16_t* ob = J.out + ((size_t)b * p.Hq + hq0) * D;
   if constexpr (INT4) {
-    if (warp == 0) unrotate_out<D>(om, heads, p.vd, xb, lane);
+    if (warp == 0) unrotate_out<D>(om, heads, vch, mrg + kHT, xb, lane);
     __syncthreads();
     // fp16 with the V sign folded in as an XOR on the sign bits
     for (int i = threadIdx.x; i < heads * D / 2; i += kThreads) {
       const int j = i % (D / 2);
-      reinterpret_cast<uint32_t*>(ob)[i] = pack_half2(xb[2 * i], xb[2 * i + 1]) ^ __ldg(&p.vd->sgn[j]);
+      reinterpret_cast<uint32_t*>(ob)[i] = pack_half2(xb[2 * i], xb[2 * i + 1]) ^ vsg[j];
     }
   } else {
-    for (int i = threadIdx.x; i < heads * D / 2; i += kThreads)
-      reinterpret_cast<uint32_t*>(ob)[i] = pack_half2(om[2 * i], om[2 * i + 1]);
+    for (int i = threadIdx.x; i < heads * D / 2; i += kThreads) {
+      const float L = mrg[kHT + (2 * i) / D];
+      const float r = L > 0.0f ? 1.0f / L : 0.0f;
+      reinterpret_cast<uint32_t*>(ob)[i] = pack_half2(om[2 * i] * r, om[2 * i + 1] * r);
+    }
   }
 }
 
@@ -750,61 +804,108 @@ struct SplitPlan {
   int HT, S, tps, C;  // C = splits per cluster (S is a multiple of C)
 };
 
-template <int D, bool INT4>
-int ctas_per_sm() {
+constexpr int kMaxPerSmForSizing = 4;
+
+// Occupancy of one kernel instantiation: CTAs per SM, and for every cluster size
+// c <= kMaxCluster the CTAs that can be resident at once in clusters of c (whole
+// clusters must fit in one GPC, so this can be well below SMs x CTAs per SM).
+struct Occupancy {
+  int per_sm;
+  int cap[kMaxCluster + 1];
+};
+
+template <int D, bool INT4, int MAXJ>
+const Occupancy& occupancy() {
   using C = Cfg<D, INT4>;
-  static int v = -1;
+  static Occupancy occ{};
   static std::once_flag once;
   std::call_once(once, [] {
-    cudaFuncSetAttribute(attend_kernel<D, INT4>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
-    cudaFuncSetAttribute(attend_kernel<D, INT4>, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    auto kern = attend_kernel<D, INT4, MAXJ>;
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, attend_kernel<D, INT4>, kThreads, C::kSmem) != cudaSuccess ||
-        nb < 1)
-      nb = 1;
-    v = nb;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, C::kSmem) != cudaSuccess || nb < 1) nb = 1;
+    occ.per_sm = std::min(nb, kMaxPerSmForSizing);
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const int slots = num_sms(dev) * occ.per_sm;
+    for (int c = 1; c <= kMaxCluster; ++c) {
+      cudaLaunchConfig_t cfg{};
+      cfg.gridDim = dim3(c, 1, 1);
+      cfg.blockDim = dim3(kThreads);
+      cfg.dynamicSmemBytes = C::kSmem;
+      cudaLaunchAttribute attr[1];
+      attr[0].id = cudaLaunchAttributeClusterDimension;
+      attr[0].val.clusterDim.x = (unsigned)c;
+      attr[0].val.clusterDim.y = 1;
+      attr[0].val.clusterDim.z = 1;
+      cfg.attrs = attr;
+      cfg.numAttrs = 1;
+      int ncl = 0;
+      if (cudaOccupancyMaxActiveClusters(&ncl, kern, &cfg) != cudaSuccess || ncl < 1) ncl = std::max(1, slots / c);
+      occ.cap[c] = std::min(slots, ncl * c);
+    }
+    occ.cap[0] = slots;
+    (void)cudaGetLastError();  // a refused query leaves no sticky error behind
   });
-  return v;
+  return occ;
 }
 
 // Split of the token range. When splits of ~4 stages cannot fill the GPU (few
 // units, short context) the kernel is latency-bound: take ~4 stages per split,
-// which keeps the final merge short. Otherwise (throughput regime) take, among
-// split counts giving at least one full wave, the smallest whose last wave is
-// >= 85% full. Every split keeps >= kMinTilesPerSplit stages, S <= kMaxSplits, and
-// S is non-decreasing in T, so a workspace sized from T_cap bounds every call.
+// which keeps the final merge short. Otherwise (throughput regime) take the split
+// count with the least estimated time (rounds of resident CTAs times the stages
+// per split plus a fixed per-CTA cost). Every split keeps >= kMinTilesPerSplit
+// stages and S <= kMaxSplits. The splits of a unit form clusters of C CTAs
+// (C = the largest divisor of S up to 8 in the latency regime, up to 4 in the
+// throughput regime, where large clusters constrain scheduling more than they
+// save) that merge through distributed shared memory; when S > C the S / C
+// cluster partials (<= kMaxMerge) merge through the workspace.
 constexpr int kMinTilesPerSplit = 2;
 constexpr int kMaxSplits = kMaxSplitsCfg;
 constexpr int kLatencyTilesPerSplit = 4;
+constexpr int kFixedTiles = 12;  // per-CTA fixed cost (query rotation, merges) in stage-times
+constexpr int kMergeTiles = 6;   // workspace merge of cluster partials, in stage-times
 
-SplitPlan choose_split(int B, int Hq, int Hkv, int T, int sms, int per_sm) {
+int cluster_for(int S, int cmax) {
+  for (int c = std::min(S, cmax); c > 1; --c)
+    if (S % c == 0) return c;
+  return 1;
+}
+
+SplitPlan choose_split(int B, int Hq, int Hkv, int T, const Occupancy& occ) {
   SplitPlan sp{};
   const int G = Hq / Hkv;
   sp.HT = (G + kHT - 1) / kHT;
   const long units = (long)B * Hkv * sp.HT;
   const int ntile = T > 0 ? (T + kTileT - 1) / kTileT : 1;
-  const long slots = (long)sms * per_sm;
+  const long slots = occ.cap[0];
   int s_cap = std::max(1, ntile / kMinTilesPerSplit);
   s_cap = std::min(s_cap, kMaxSplits);
-  int best = 1;
   const bool latency = units * std::max(1, ntile / kLatencyTilesPerSplit) < slots;
+  const int cmax = latency ? kMaxClusterLatency : kMaxClusterThroughput;
+  // S as launched: each split takes ceil(ntile / S) stages, so fewer splits may be nonempty
+  auto realised = [&](int S) {
+    const int tiles_per = (ntile + S - 1) / S;
+    return (ntile + tiles_per - 1) / tiles_per;
+  };
+  auto mergeable = [&](int S) { return S / cluster_for(S, cmax) <= kMaxMerge; };
+  int best = 1;
   if (latency) {
     best = std::max(1, std::min(ntile / kLatencyTilesPerSplit, s_cap));
+    while (best > 1 && !mergeable(realised(best))) --best;
   } else {
-    double best_eff = -1.0;
-    const int s_lo = (int)std::min<long>(s_cap, std::max<long>(1, (slots + units - 1) / units));
-    for (int S = s_lo; S <= s_cap; ++S) {
-      const int tiles_per = (ntile + S - 1) / S;
-      const int Sr = (ntile + tiles_per - 1) / tiles_per;
-      const long ctas = units * Sr;
-      const long waves = (ctas + slots - 1) / slots;
-      const double eff = (double)ctas / (double)(waves * slots);
-      if (eff >= 0.85) {
-        best = S;
-        break;
-      }
-      if (eff > best_eff + 1e-9) {
-        best_eff = eff;
+    // estimated time in stage-times: rounds of resident CTAs x (stages per split +
+    // the per-CTA fixed cost), plus the workspace merge when a unit has several clusters
+    long best_t = -1;
+    for (int S = 1; S <= s_cap; ++S) {
+      const int Sr = realised(S);
+      if (!mergeable(Sr)) continue;
+      const int C = cluster_for(Sr, cmax);
+      const long rounds = (units * Sr + occ.cap[C] - 1) / occ.cap[C];
+      const long t = rounds * ((ntile + S - 1) / S + kFixedTiles) + (Sr / C > 1 ? kMergeTiles : 0);
+      if (best_t < 0 || t < best_t) {
+        best_t = t;
         best = S;
       }
     }
@@ -812,81 +913,82 @@ SplitPlan choose_split(int B, int Hq, int Hkv, int T, int sms, int per_sm) {
   const int tiles_per = (ntile + best - 1) / best;
   sp.tps = tiles_per * kTileT;
   sp.S = (ntile + tiles_per - 1) / tiles_per;
-  // splits of a unit run as one thread-block cluster (<= 16) and merge through
-  // distributed shared memory; beyond 16, whole clusters (the last ones possibly
-  // with empty splits) merge through the workspace
-  // (clusters of up to 8 in the latency regime; up to 4 when the GPU is full of
-  // units, where large clusters constrain scheduling more than they save)
-  const int cmax = latency ? kMaxClusterLatency : kMaxClusterThroughput;
-  if (sp.S <= cmax) {
-    sp.C = sp.S;
-  } else {
-    sp.C = cmax;
-    sp.S = (sp.S + cmax - 1) / cmax * cmax;
-  }
+  sp.C = cluster_for(sp.S, cmax);
   return sp;
 }
 
-constexpr int kMaxPerSmForSizing = 4;
-
-// workspace: [counters (units ints, 256-aligned)] [cluster partials units x (S/16) x (m[8], l[8], o[8][D])
+// workspace: [counters (units ints, 256-aligned)] [cluster partials units x ncl x (m[8], l[8], o[8][D])
 // fp32, only when a unit has more than one cluster]
 size_t ws_cnt_bytes(size_t units) { return ((units * 4 + 255) / 256) * 256; }
 
-size_t ws_bytes_for(int B, int Hq, int Hkv, int D, int S_max, int HT) {
+size_t ws_bytes_for(int B, int Hq, int Hkv, int D, int ncl, int HT) {
   const size_t units = (size_t)B * Hkv * HT;
-  const size_t ncl = S_max > kMaxClusterThroughput ? (S_max + kMaxClusterThroughput - 1) / kMaxClusterThroughput : 0;
-  const size_t part = units * ncl * (2 * kHT + kHT * D) * 4;
+  const size_t part = units * (size_t)(ncl > 1 ? ncl : 0) * (2 * kHT + kHT * D) * 4;
   return ws_cnt_bytes(units) + part;
 }
 
+// Tensor maps and pointers of one problem. Rows of the code (or fp16) maps are
+// (b, kv head, token) rows; scale maps have one row of T_cap * D/32 halves per (b, kv head).
 template <int D, bool INT4>
-kvq_status run_attend(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q, const void* kc, const uint16_t* ks,
-                      const void* vc, const uint16_t* vs, int B, int Hq, int Hkv, int T_cap, const int32_t* seq_lens,
-                      int T_len, float sigma, uint16_t* out, void* ws, size_t ws_bytes, cudaStream_t strm) {
+kvq_status make_job(const AttendJobHost& h, int B, int Hkv, int T_cap, AttnJob* j) {
   using C = Cfg<D, INT4>;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  const int sms = num_sms(dev);
-  const int per_sm = std::min(ctas_per_sm<D, INT4>(), kMaxPerSmForSizing);
-  const int T_split = seq_lens ? T_cap : T_len;
-  SplitPlan sp = choose_split(B, Hq, Hkv, T_split, sms, per_sm);
-  const size_t units = (size_t)B * Hkv * sp.HT;
-  const size_t need = ws_bytes_for(B, Hq, Hkv, D, sp.S, sp.HT);
-  if (ws_bytes < need) return fail(KVQ_ERR_WORKSPACE, "attend: workspace too small for this split");
-  CUtensorMap kmap, vmap, ksmap, vsmap;
   const uint64_t rows = (uint64_t)B * Hkv * T_cap;
+  kvq_status st;
   if (INT4) {
     const uint64_t dims[2] = {(uint64_t)D / 2, rows};
     const uint64_t strides[1] = {(uint64_t)D / 2};
     const uint32_t box[2] = {(uint32_t)D / 2, (uint32_t)kTileT};
     const CUtensorMapSwizzle sw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
-    kvq_status st = encode_tiled(&kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, kc, dims, strides, box, sw, "K codes");
-    if (st == KVQ_OK) st = encode_tiled(&vmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, vc, dims, strides, box, sw, "V codes");
+    st = encode_tiled(&j->kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, h.kc, dims, strides, box, sw, "K codes");
+    if (st == KVQ_OK) st = encode_tiled(&j->vmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, h.vc, dims, strides, box, sw, "V codes");
     if (st != KVQ_OK) return st;
     const uint64_t sd[2] = {(uint64_t)T_cap * C::NG, (uint64_t)B * Hkv};
     const uint64_t ss[1] = {(uint64_t)T_cap * C::NG * 2};
     const uint32_t sb[2] = {(uint32_t)C::kScaleBox, 1u};
-    st = encode_tiled(&ksmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, ks, sd, ss, sb, CU_TENSOR_MAP_SWIZZLE_NONE, "K scales");
+    st = encode_tiled(&j->ksmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h.ks, sd, ss, sb, CU_TENSOR_MAP_SWIZZLE_NONE,
+                      "K scales");
     if (st == KVQ_OK)
-      st = encode_tiled(&vsmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, vs, sd, ss, sb, CU_TENSOR_MAP_SWIZZLE_NONE, "V scales");
+      st = encode_tiled(&j->vsmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h.vs, sd, ss, sb, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        "V scales");
     if (st != KVQ_OK) return st;
   } else {
     const uint64_t dims[2] = {(uint64_t)D, rows};
     const uint64_t strides[1] = {(uint64_t)D * 2};
     const uint32_t box[2] = {64u, (uint32_t)kTileT};
-    kvq_status st = encode_tiled(&kmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, kc, dims, strides, box,
-                                 CU_TENSOR_MAP_SWIZZLE_128B, "K cache");
+    st = encode_tiled(&j->kmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h.kc, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
+                      "K cache");
     if (st == KVQ_OK)
-      st = encode_tiled(&vmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, vc, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
-                        "V cache");
+      st = encode_tiled(&j->vmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h.vc, dims, strides, box,
+                        CU_TENSOR_MAP_SWIZZLE_128B, "V cache");
     if (st != KVQ_OK) return st;
-    ksmap = kmap;
-    vsmap = vmap;
+    j->ksmap = j->kmap;
+    j->vsmap = j->vmap;
+  }
+  j->q = h.q;
+  j->out = h.out;
+  j->ke = INT4 ? h.pk->enc_dev : nullptr;
+  j->kd = INT4 ? h.pk->dec_dev : nullptr;
+  j->vd = INT4 ? h.pv->dec_dev : nullptr;
+  return KVQ_OK;
+}
+
+// One launch over nj <= MAXJ problems of equal shape.
+template <int D, bool INT4, int MAXJ>
+kvq_status launch_chunk(const AttendJobHost* jobs, int nj, int B, int Hq, int Hkv, int T_cap, const int32_t* seq_lens,
+                        int T_len, float sigma, void* ws, size_t ws_bytes, cudaStream_t strm) {
+  using C = Cfg<D, INT4>;
+  const int T_split = seq_lens ? T_cap : T_len;
+  const int Bj = nj * B;  // the jobs of a launch split like a larger batch
+  SplitPlan sp = choose_split(Bj, Hq, Hkv, T_split, occupancy<D, INT4, MAXJ>());
+  const size_t units = (size_t)Bj * Hkv * sp.HT;
+  const size_t need = ws_bytes_for(Bj, Hq, Hkv, D, sp.S / sp.C, sp.HT);
+  if (ws_bytes < need) return fail(KVQ_ERR_WORKSPACE, "attend: workspace too small for this split");
+  AttnJobs<MAXJ> jt;
+  for (int i = 0; i < nj; ++i) {
+    const kvq_status st = make_job<D, INT4>(jobs[i], B, Hkv, T_cap, &jt.j[i]);
+    if (st != KVQ_OK) return st;
   }
   AttnParams prm{};
-  prm.q = q;
-  prm.out = out;
   prm.seq_lens = seq_lens;
   prm.T_len = T_len;
   prm.B = B;
@@ -902,11 +1004,8 @@ kvq_status run_attend(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q,
   char* wsb = reinterpret_cast<char*>(ws);
   prm.cnt = reinterpret_cast<int*>(wsb);
   prm.part = reinterpret_cast<float*>(wsb + ws_cnt_bytes(units));
-  prm.ke = INT4 ? pk->enc_dev : nullptr;
-  prm.kd = INT4 ? pk->dec_dev : nullptr;
-  prm.vd = INT4 ? pv->dec_dev : nullptr;
-  dim3 grid(sp.S, sp.HT, B * Hkv);
-  if (grid.z > 65535u) return fail(KVQ_ERR_UNSUPPORTED, "attend: B * Hkv > 65535");
+  dim3 grid(sp.S, sp.HT, Bj * Hkv);
+  if (grid.z > 65535u) return fail(KVQ_ERR_UNSUPPORTED, "attend: jobs * B * Hkv > 65535");
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
   cfg.blockDim = dim3(kThreads);
@@ -919,8 +1018,24 @@ kvq_status run_attend(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q,
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, attend_kernel<D, INT4>, kmap, vmap, ksmap, vsmap, prm);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, attend_kernel<D, INT4, MAXJ>, jt, prm);
   if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
+  return KVQ_OK;
+}
+
+// Launches of up to kMaxJobs problems each, in stream order; they reuse the
+// workspace from its start (every launch leaves its counters at zero).
+template <int D, bool INT4>
+kvq_status run_attend(const AttendJobHost* jobs, int njobs, int B, int Hq, int Hkv, int T_cap,
+                      const int32_t* seq_lens, int T_len, float sigma, void* ws, size_t ws_bytes, cudaStream_t strm) {
+  if (njobs == 1)
+    return launch_chunk<D, INT4, 1>(jobs, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, strm);
+  for (int j0 = 0; j0 < njobs; j0 += kMaxJobs) {
+    const int nj = std::min(kMaxJobs, njobs - j0);
+    const kvq_status st =
+        launch_chunk<D, INT4, kMaxJobs>(jobs + j0, nj, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, strm);
+    if (st != KVQ_OK) return st;
+  }
   return KVQ_OK;
 }
 
@@ -928,33 +1043,37 @@ kvq_status run_attend(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q,
 
 size_t attend_workspace_bytes(int B, int Hq, int Hkv, int D, int T_cap) {
   // Bound over every split the launch can choose for T <= T_cap: S never exceeds
-  // min(kMaxSplits, ntile(T_cap) / kMinTilesPerSplit) (at least 1).
+  // min(kMaxSplits, ntile(T_cap) / kMinTilesPerSplit) (at least 1), and a unit never
+  // has more than min(S, kMaxMerge) cluster partials.
   const int G = Hq / Hkv;
   const int HT = (G + kHT - 1) / kHT;
   const int ntile = T_cap > 0 ? (T_cap + kTileT - 1) / kTileT : 1;
   const int s_max = std::max(1, std::min(kMaxSplits, ntile / kMinTilesPerSplit));
-  return ws_bytes_for(B, Hq, Hkv, D, s_max, HT);
+  return ws_bytes_for(B, Hq, Hkv, D, std::min(s_max, kMaxMerge), HT);
 }
 
 kvq_status launch_attend_int4(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q, const uint8_t* kc,
                               const uint16_t* ks, const uint8_t* vc, const uint16_t* vs, int B, int Hq, int Hkv,
                               int T_cap, const int32_t* seq_lens, int T_len, float sigma, uint16_t* out, void* ws,
                               size_t ws_bytes, cudaStream_t s) {
-  if (pk->D == 128)
-    return run_attend<128, true>(pk, pv, q, kc, ks, vc, vs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, out, ws,
-                                 ws_bytes, s);
-  return run_attend<256, true>(pk, pv, q, kc, ks, vc, vs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, out, ws,
-                               ws_bytes, s);
+  const AttendJobHost job{pk, pv, q, kc, ks, vc, vs, out};
+  return launch_attend_int4_batch(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
+}
+
+kvq_status launch_attend_int4_batch(const AttendJobHost* jobs, int njobs, int B, int Hq, int Hkv, int T_cap,
+                                    const int32_t* seq_lens, int T_len, float sigma, void* ws, size_t ws_bytes,
+                                    cudaStream_t s) {
+  if (jobs[0].pk->D == 128)
+    return run_attend<128, true>(jobs, njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
+  return run_attend<256, true>(jobs, njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
 }
 
 kvq_status launch_attend_fp16(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq, int Hkv, int D,
                               int T_cap, const int32_t* seq_lens, int T_len, float sigma, uint16_t* out, void* ws,
                               size_t ws_bytes, cudaStream_t s) {
-  if (D == 128)
-    return run_attend<128, false>(nullptr, nullptr, q, k, nullptr, v, nullptr, B, Hq, Hkv, T_cap, seq_lens, T_len,
-                                  sigma, out, ws, ws_bytes, s);
-  return run_attend<256, false>(nullptr, nullptr, q, k, nullptr, v, nullptr, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma,
-                                out, ws, ws_bytes, s);
+  const AttendJobHost job{nullptr, nullptr, q, k, nullptr, v, nullptr, out};
+  if (D == 128) return run_attend<128, false>(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
+  return run_attend<256, false>(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
 }
 
 // ---------------------------------------------------------------- allocation-free variant
@@ -996,10 +1115,9 @@ kvq_status launch_attend_int4_noalloc(const kvq_plan* pk, const kvq_plan* pv, co
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(KVQ_ERR_DEVICE, "attend_noalloc: no current device");
   const int D = pk->D;
   // the exact split the launch will choose, hence the exact scratch it needs
-  const int per_sm = D == 128 ? std::min(ctas_per_sm<128, true>(), kMaxPerSmForSizing)
-                              : std::min(ctas_per_sm<256, true>(), kMaxPerSmForSizing);
-  const SplitPlan sp = choose_split(B, Hq, Hkv, seq_lens ? T_cap : T_len, num_sms(dev), per_sm);
-  const size_t need = ws_bytes_for(B, Hq, Hkv, D, sp.S, sp.HT);
+  const Occupancy& occ = D == 128 ? occupancy<128, true, 1>() : occupancy<256, true, 1>();
+  const SplitPlan sp = choose_split(B, Hq, Hkv, seq_lens ? T_cap : T_len, occ);
+  const size_t need = ws_bytes_for(B, Hq, Hkv, D, sp.S / sp.C, sp.HT);
   if (need > kNoAllocScratchBytes)
     return fail(KVQ_ERR_WORKSPACE, "attend_noalloc: these shapes need " + std::to_string(need) +
                                        " bytes of scratch; the static scratch holds " +
@@ -1011,11 +1129,10 @@ kvq_status launch_attend_int4_noalloc(const kvq_plan* pk, const kvq_plan* pv, co
   const size_t units = (size_t)B * Hkv * sp.HT;
   const cudaError_t e = cudaMemsetAsync(scratch, 0, ws_cnt_bytes(units), s);
   if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("attend_noalloc: memset: ") + cudaGetErrorString(e));
+  const AttendJobHost job{pk, pv, q, kc, ks, vc, vs, out};
   if (D == 128)
-    return run_attend<128, true>(pk, pv, q, kc, ks, vc, vs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, out, scratch,
-                                 kNoAllocScratchBytes, s);
-  return run_attend<256, true>(pk, pv, q, kc, ks, vc, vs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, out, scratch,
-                               kNoAllocScratchBytes, s);
+    return run_attend<128, true>(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, scratch, kNoAllocScratchBytes, s);
+  return run_attend<256, true>(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, scratch, kNoAllocScratchBytes, s);
 }
 
 uint32_t attend_error_flags(bool clear) {

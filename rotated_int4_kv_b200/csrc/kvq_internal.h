@@ -58,7 +58,21 @@ kvq_status launch_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t
                          int T_cap, int t0, int n, uint16_t* out, cudaStream_t s);
 
 // attention launchers (kvq_attend.cu)
+// One decode-attention problem: plans (int4 only), query, caches, output.
+struct AttendJobHost {
+  const kvq_plan* pk;
+  const kvq_plan* pv;
+  const uint16_t* q;
+  const void* kc;   // K codes (int4) or fp16 K
+  const uint16_t* ks;
+  const void* vc;   // V codes (int4) or fp16 V
+  const uint16_t* vs;
+  uint16_t* out;
+};
 size_t attend_workspace_bytes(int B, int Hq, int Hkv, int D, int T_cap);
+kvq_status launch_attend_int4_batch(const AttendJobHost* jobs, int njobs, int B, int Hq, int Hkv, int T_cap,
+                                    const int32_t* seq_lens, int T_len, float sigma, void* ws, size_t ws_bytes,
+                                    cudaStream_t s);
 kvq_status launch_attend_int4(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q,
                               const uint8_t* kc, const uint16_t* ks, const uint8_t* vc, const uint16_t* vs,
                               int B, int Hq, int Hkv, int T_cap, const int32_t* seq_lens, int T_len,

@@ -20,7 +20,8 @@ def test_header_declares_the_boundary():
     names = _declared()
     for n in ("kvq_plan_create", "kvq_plan_destroy", "kvq_encode", "kvq_encode_batch", "kvq_decode",
               "kvq_workspace_size", "kvq_attend_decode", "kvq_attend_decode_ref", "kvq_status_string",
-              "kvq_last_error", "kvq_poll_device_errors"):
+              "kvq_last_error", "kvq_poll_device_errors", "kvq_attend_decode_batch",
+              "kvq_attend_decode_noalloc"):
         assert n in names
 
 
@@ -33,6 +34,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_status_strings_and_host_checks():
+    from rotated_int4_kv_b200 import _lib as kvq_lib
     from rotated_int4_kv_b200 import lib
 
     assert lib.kvq_status_string(0) == b"ok"
@@ -47,6 +49,11 @@ def test_status_strings_and_host_checks():
                                      0, None) == -2
     assert lib.kvq_encode_batch(None, -1, None) == -1
     assert lib.kvq_encode_batch(None, 0, None) == 0
+    assert lib.kvq_attend_decode_batch(None, -1, 1, 4, 1, 64, None, 64, ctypes.c_float(0), None, 0, None) == -1
+    assert lib.kvq_attend_decode_batch(None, 0, 1, 4, 1, 64, None, 64, ctypes.c_float(0), None, 0, None) == 0
+    jobs = (kvq_lib.AttendJob * 2)()  # null plans: refused before any CUDA call
+    assert lib.kvq_attend_decode_batch(jobs, 2, 1, 4, 1, 64, None, 64, ctypes.c_float(0), None, 0, None) == -1
+    assert b"job 0" in lib.kvq_last_error()
     h = P()
     signs = (ctypes.c_int8 * 128)(*([1] * 128))
     lam = (ctypes.c_float * 128)(*([1.0] * 128))

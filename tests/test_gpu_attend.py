@@ -200,3 +200,48 @@ def test_mistral_full_size_sampled(kvq):
         ref = oracle.attend_decode_fp16(q16[3:4, hq], k16[3:4, kvh:kvh + 1].cpu().numpy(),
                                         v16[3:4, kvh:kvh + 1].cpu().numpy(), [T])
         check_rel_l2(o16[3:4, hq].cpu().numpy().reshape(-1, D), ref.reshape(-1, D), label=f"fp16 kv{kvh}")
+
+
+BATCH_CASES = [
+    # (workload, njobs, B, Hkv, Hq, T_cap, lens): each job its own layer (plans, cache, query)
+    ("gemma", 5, 1, 1, 4, 1024, None),          # D = 256, one launch
+    ("qwen", 35, 1, 2, 12, 256, [200]),         # D = 128, two launches (32 + 3 jobs)
+    ("mistral", 3, 2, 8, 32, 514, [514, 3]),    # ragged batch entries
+]
+
+
+@pytest.mark.parametrize("case", BATCH_CASES, ids=[f"{c[0]}-x{c[1]}" for c in BATCH_CASES])
+def test_attend_batch_matches_oracle_per_job(kvq, case):
+    wl_name, nj, B, Hkv, Hq, T_cap, lens = case
+    wl = kvgen.WORKLOADS[wl_name]
+    D = wl.head_dim
+    caches = [_build_cache(kvq, wl, B, Hkv, T_cap, T_cap, seed=31, layer=j) for j in range(nj)]
+    qs16 = [kvgen.q_numpy((B, Hq, D), salt=100 + j) for j in range(nj)]
+    jobs = [(c["k"]["plan"], c["v"]["plan"], torch.from_numpy(q).cuda(), c["k"]["codes"], c["k"]["scales"],
+             c["v"]["codes"], c["v"]["scales"]) for c, q in zip(caches, qs16)]
+    sl = None if lens is None else torch.tensor(lens * (B // len(lens)) if len(lens) < B else lens,
+                                                dtype=torch.int32, device="cuda")
+    lens_np = [T_cap] * B if sl is None else sl.cpu().tolist()
+    outs = kvq.attend_decode_batch(jobs, seq_lens=sl, T_len=T_cap if sl is None else None)
+    singles = [kvq.attend_decode(*j, seq_lens=sl, T_len=T_cap if sl is None else None) for j in jobs]
+    torch.cuda.synchronize()
+    assert kvq.poll_device_errors() == 0
+    for j in range(nj):
+        got = outs[j].cpu().numpy().astype(np.float64)
+        one = singles[j].cpu().numpy().astype(np.float64)
+        # another split of the same sums: equal to fp32 noise
+        check_rel_l2(got.reshape(-1, D), one.reshape(-1, D), tol=1e-3, label=f"job {j} vs single call")
+        if j in (0, nj - 1):
+            ref = _oracle_int4(qs16[j], caches[j], lens_np)
+            check_rel_l2(got.reshape(-1, D), ref.reshape(-1, D), tol=2e-3, label=f"job {j} vs oracle")
+
+
+def test_attend_batch_rejects_mixed_head_dims(kvq):
+    g, q = kvgen.WORKLOADS["gemma"], kvgen.WORKLOADS["qwen"]
+    cg_ = _build_cache(kvq, g, 1, 1, 64, 64)
+    cq = _build_cache(kvq, q, 1, 1, 64, 64)
+    jobs = [(c["k"]["plan"], c["v"]["plan"], torch.zeros((1, 4, w.head_dim), dtype=torch.float16, device="cuda"),
+             c["k"]["codes"], c["k"]["scales"], c["v"]["codes"], c["v"]["scales"])
+            for c, w in ((cg_, g), (cq, q))]
+    with pytest.raises(Exception):
+        kvq.attend_decode_batch(jobs, T_len=64)
