@@ -53,6 +53,7 @@ def _peaks():
 # until a new capture. Summaries and commands: profiles/.
 KERNEL_SOURCES = {
     "encode": ["kvq_codec.cu", "kvq_ptx.cuh", "srft_fft.cuh", "kvq_internal.h"],
+    "encode_tc": ["kvq_encode_tc.cu", "kvq_ptx.cuh", "kvq_quant.cuh", "kvq_internal.h"],
     "attend": ["kvq_attend.cu", "kvq_ptx.cuh", "srft_fft.cuh", "kvq_internal.h"],
 }
 NCU_TRAFFIC = {
@@ -383,8 +384,11 @@ def run_kvq(args, rank: int, world: int):
     # roofline of the kernel with the larger share of the step (each phase is one launch)
     src = "measured (MEASURED_PEAKS.json hbm_gbs, burst copy)" if peak_kind == "measured" else "fallback 6.65 TB/s"
     if enc_avg >= att_avg:
+        tc = kvq.get_encode_path() != "fft" and G == 32
         roof = {"bound": "hbm", "achieved": enc_gbs, "peak": hbm, "unit": "GB/s", "frac": enc_gbs / hbm,
-                "traffic": _ncu_traffic("encode"), "kernel": f"encode_kernel<{D},{G},64>",
+                "traffic": _ncu_traffic("encode_tc" if tc else "encode"),
+                "kernel": ("encode_tc256_kernel<64>" if D == 256 else "encode_tc_kernel<128,64>") if tc
+                else f"encode_kernel<{D},{G},64>",
                 "share": enc_avg / (enc_avg + att_avg), "peak_source": src}
     else:
         roof = {"bound": "hbm", "achieved": att_gbs, "peak": hbm, "unit": "GB/s", "frac": att_gbs / hbm,

@@ -122,6 +122,22 @@ typedef struct kvq_encode_job {
 kvq_status kvq_encode_batch(const kvq_encode_job* jobs, int njobs, void* stream);
 
 /*
+ * kvq_set_encode_path / kvq_get_encode_path -- which kernel kvq_encode and
+ * kvq_encode_batch run (process-wide setting; not on the pages):
+ *   0  default: the tensor-core encode (tcgen05 GEMM against W = Lambda F_r diag(s)
+ *      held as an fp16 hi + lo pair) where it exists (head_dim 128, group 32),
+ *      else the register-FFT encode;
+ *   1  always the register-FFT encode (one radix-2 real FFT per vector in registers);
+ *   2  always the tensor-core encode (KVQ_ERR_UNSUPPORTED where it does not exist).
+ * Both produce codes and scales that meet the same acceptance rule against the
+ * fp64 definition; they may differ from each other only at rounding boundaries.
+ * Set it between launches, not while another thread is encoding.
+ * Errors: INVALID_ARG for a value other than 0, 1, 2.
+ */
+kvq_status kvq_set_encode_path(int path);
+int kvq_get_encode_path(void);
+
+/*
  * kvq_decode -- the inverse: x_hat = diag(s) . F_r^T . (c * scale / lambda), rounded
  * to fp16, for cache rows t0 .. t0+n-1 of every (b, h).
  *   out  fp16 [B, H, n, D] contiguous.

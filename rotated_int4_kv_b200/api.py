@@ -94,6 +94,20 @@ def encode_batch(jobs, stream=None) -> None:
     check(lib.kvq_encode_batch(arr, len(jobs), _stream(stream)), "kvq_encode_batch")
 
 
+ENCODE_PATHS = {"auto": 0, "fft": 1, "tensor": 2}
+
+
+def set_encode_path(path: str) -> None:
+    """Select the encode kernel: "auto" (tensor cores where supported), "fft"
+    (register FFT) or "tensor" (tensor cores only)."""
+    check(lib.kvq_set_encode_path(ENCODE_PATHS[path]), "kvq_set_encode_path")
+
+
+def get_encode_path() -> str:
+    v = int(lib.kvq_get_encode_path())
+    return {n: k for k, n in ENCODE_PATHS.items()}[v]
+
+
 def decode(plan: Plan, codes: torch.Tensor, scales: torch.Tensor, t0: int, n: int, out: torch.Tensor = None,
            stream=None) -> torch.Tensor:
     """Decode cache rows t0..t0+n-1 into fp16 [B, H, n, D]."""

@@ -1,5 +1,6 @@
 // kvq_api.cu -- the C ABI: plan management, host-side argument checks, error
 // reporting and the driver entry point for TMA tensor maps.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -40,6 +41,20 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // Per-channel normalisation of the real basis: dg_c = 1/sqrt(D) (DC, Nyquist),
 // sqrt(2/D) (cos rows), -sqrt(2/D) (sin rows: the spectrum slot holds Im X_k and
 // the sin row equals -sqrt(2/D) Im X_k).
+// Row c of the orthonormal real basis in channel order, at sample n: DC, then
+// (cos_k, +sin_k) pairs, then Nyquist; angles from the exact residue k n mod D.
+double basis_value(int c, int n, int D) {
+  const double pi2 = 6.283185307179586476925286766559;
+  if (c == 0) return 1.0 / std::sqrt((double)D);
+  if (c == D - 1) return ((n & 1) ? -1.0 : 1.0) / std::sqrt((double)D);
+  const int k = (c + 1) / 2;
+  const double ang = pi2 * (double)((long)k * n % D) / (double)D;
+  return std::sqrt(2.0 / D) * ((c & 1) ? std::cos(ang) : std::sin(ang));
+}
+
+uint16_t half_bits(float f) { return __half_as_ushort(__float2half_rn(f)); }
+float half_value(uint16_t b) { return __half2float(__ushort_as_half(b)); }
+
 double basis_dg(int c, int D) {
   if (c == 0 || c == D - 1) return 1.0 / std::sqrt((double)D);
   return (c & 1) ? std::sqrt(2.0 / D) : -std::sqrt(2.0 / D);
@@ -52,6 +67,21 @@ void set_error(const std::string& msg) { t_last_error = msg; }
 kvq_status fail(kvq_status st, const std::string& msg) {
   t_last_error = msg;
   return st;
+}
+
+std::atomic<int> g_encode_path{0};
+
+int encode_path() { return g_encode_path.load(); }
+
+// All jobs share head_dim and group (checked by the callers).
+kvq_status dispatch_encode(const kvq_encode_job* jobs, int njobs, cudaStream_t s) {
+  const kvq_plan* p = jobs[0].plan;
+  const int path = g_encode_path.load();
+  const bool tc = encode_tc_supported(p->D, p->G) && p->wt_dev != nullptr;
+  if (path == 2 && !tc)
+    return fail(KVQ_ERR_UNSUPPORTED, "encode: the tensor-core path supports head_dim 128 with group 32 only");
+  if (tc && path != 1) return launch_encode_tc(jobs, njobs, s);
+  return launch_encode_jobs(jobs, njobs, s);
 }
 
 namespace {
@@ -186,14 +216,56 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
     p->enc.sgn[w] = m;
     p->dec.sgn[w] = m;
   }
+  // tensor-core encode operand, fp16 hi rows then lo rows (value = hi + lo to ~2^-22):
+  //   D = 128: W = Lambda F_r diag(s) [128 x 128] (channel order);
+  //   D = 256: the unnormalised 128-point real DFT in slot order [128 x 128] (row 0: 1,
+  //            row 1: (-1)^m, row 2k: cos(2 pi k m / 128), row 2k+1: -sin(2 pi k m / 128)),
+  //            applied to the even and the odd samples of s (.) x.
+  std::vector<uint16_t> wt;
+  if (D == 256) {
+    const int M = 128;
+    wt.resize((size_t)2 * M * M);
+    const double pi2 = 6.283185307179586476925286766559;
+    for (int j = 0; j < M; ++j)
+      for (int m = 0; m < M; ++m) {
+        double w;
+        if (j == 0) w = 1.0;
+        else if (j == 1) w = (m & 1) ? -1.0 : 1.0;
+        else {
+          const int k = j / 2;
+          const double ang = pi2 * (double)((long)k * m % M) / (double)M;
+          w = (j & 1) ? -std::sin(ang) : std::cos(ang);
+        }
+        const uint16_t hi = kvq::half_bits((float)w);
+        const uint16_t lo = kvq::half_bits((float)(w - (double)kvq::half_value(hi)));
+        wt[(size_t)j * M + m] = hi;
+        wt[(size_t)(M + j) * M + m] = lo;
+      }
+  }
+  if (D == 128) {
+    wt.resize((size_t)2 * D * D);
+    for (int c = 0; c < D; ++c)
+      for (int n = 0; n < D; ++n) {
+        const double w = (double)lambda[c] * kvq::basis_value(c, n, D) * (double)signs[n];
+        const uint16_t hi = kvq::half_bits((float)w);
+        const uint16_t lo = kvq::half_bits((float)(w - (double)kvq::half_value(hi)));
+        wt[(size_t)c * D + n] = hi;
+        wt[(size_t)(D + c) * D + n] = lo;
+      }
+  }
+  constexpr size_t kWtOff = 4096;  // after the two CodecConsts copies, 16-byte aligned for TMA
+  static_assert(2 * sizeof(kvq::CodecConsts) <= kWtOff, "plan block layout");
+  const size_t bytes = wt.empty() ? 2 * sizeof(kvq::CodecConsts) : kWtOff + wt.size() * 2;
   void* blk = nullptr;
-  if (cudaMalloc(&blk, 2 * sizeof(kvq::CodecConsts)) != cudaSuccess) {
+  if (cudaMalloc(&blk, bytes) != cudaSuccess) {
     delete p;
     return fail(KVQ_ERR_CUDA, "plan_create: cudaMalloc failed");
   }
   if (cudaMemcpy(blk, &p->enc, sizeof(kvq::CodecConsts), cudaMemcpyHostToDevice) != cudaSuccess ||
       cudaMemcpy((char*)blk + sizeof(kvq::CodecConsts), &p->dec, sizeof(kvq::CodecConsts), cudaMemcpyHostToDevice) !=
-          cudaSuccess) {
+          cudaSuccess ||
+      (!wt.empty() &&
+       cudaMemcpy((char*)blk + kWtOff, wt.data(), wt.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess)) {
     cudaFree(blk);
     delete p;
     return fail(KVQ_ERR_CUDA, "plan_create: upload failed");
@@ -201,6 +273,7 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
   p->dblock = blk;
   p->enc_dev = reinterpret_cast<const kvq::CodecConsts*>(blk);
   p->dec_dev = reinterpret_cast<const kvq::CodecConsts*>((char*)blk + sizeof(kvq::CodecConsts));
+  p->wt_dev = wt.empty() ? nullptr : reinterpret_cast<const uint16_t*>((char*)blk + kWtOff);
   *out = p;
   return KVQ_OK;
 }
@@ -234,7 +307,7 @@ kvq_status kvq_encode(const kvq_plan* p, const uint16_t* x, int B, int H, int n,
   kvq_status st = kvq::check_plan_device(p);
   if (st != KVQ_OK) return st;
   kvq_encode_job job{p, x, codes, scales, B, H, n, T_cap, pos};
-  return kvq::launch_encode_jobs(&job, 1, (cudaStream_t)stream);
+  return kvq::dispatch_encode(&job, 1, (cudaStream_t)stream);
 }
 
 kvq_status kvq_encode_batch(const kvq_encode_job* jobs, int njobs, void* stream) {
@@ -263,8 +336,16 @@ kvq_status kvq_encode_batch(const kvq_encode_job* jobs, int njobs, void* stream)
     live.push_back(j);
   }
   if (live.empty()) return KVQ_OK;
-  return kvq::launch_encode_jobs(live.data(), (int)live.size(), (cudaStream_t)stream);
+  return kvq::dispatch_encode(live.data(), (int)live.size(), (cudaStream_t)stream);
 }
+
+kvq_status kvq_set_encode_path(int path) {
+  if (path < 0 || path > 2) return fail(KVQ_ERR_INVALID_ARG, "set_encode_path: path must be 0, 1 or 2");
+  kvq::g_encode_path.store(path);
+  return KVQ_OK;
+}
+
+int kvq_get_encode_path(void) { return kvq::g_encode_path.load(); }
 
 kvq_status kvq_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* scales, int B, int H, int T_cap,
                       int t0, int n, uint16_t* out, void* stream) {
@@ -396,7 +477,7 @@ kvq_status kvq_attend_decode_ref(const uint16_t* q, const uint16_t* k, const uin
 
 kvq_status kvq_poll_device_errors(uint32_t* flags) {
   if (cudaDeviceSynchronize() != cudaSuccess) return fail(KVQ_ERR_CUDA, "poll: device synchronize failed");
-  const uint32_t f = kvq::codec_error_flags(true) | kvq::attend_error_flags(true);
+  const uint32_t f = kvq::codec_error_flags(true) | kvq::attend_error_flags(true) | kvq::encode_tc_error_flags(true);
   if (flags) *flags = f;
   return KVQ_OK;
 }

@@ -138,10 +138,6 @@ __device__ __forceinline__ void nib8_to_h2(uint32_t w, uint32_t (&h)[4]) {
   h[3] = h2_bits(__hfma2(bits_h2(d), k16, k72));
 }
 
-__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
 __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kCWarps * 32) : "memory"); }
 
 __device__ __forceinline__ float fast_exp2(float x) { return ex2_approx(x); }

@@ -26,6 +26,7 @@
 
 #include "kvq_internal.h"
 #include "kvq_ptx.cuh"
+#include "kvq_quant.cuh"
 #include "srft_fft.cuh"
 
 namespace kvq {
@@ -35,9 +36,6 @@ __device__ uint32_t g_codec_err = 0;
 namespace {
 
 constexpr int kNT = 128;            // threads (= vectors) per CTA
-constexpr float kMagic = 12582920.0f;  // 1.5 * 2^23 + 8: bits = 0x4B400008 + code
-constexpr float kMagicLo = 12582913.0f;  // code -7
-constexpr float kMagicHi = 12582927.0f;  // code +7
 
 struct TileGeom {
   int BH, n, T_box, BH_box, n_ttiles, n_tiles, t_shift;
@@ -103,44 +101,18 @@ __device__ __forceinline__ void quantize_pack(const float (&v)[NV], const float*
 #pragma unroll
   for (int g = 0; g < NV / G; ++g) {
     float y[G];
-    float a = 0.0f;
 #pragma unroll
     for (int i4 = 0; i4 < G / 4; ++i4) {
       const float4 l4 = __ldg(reinterpret_cast<const float4*>(lam + g * G) + i4);
-      const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int i = 4 * i4 + e;
-        y[i] = v[g * G + i] * lv[e];
-        a = fmaxf(a, fabsf(y[i]));
-      }
+      y[4 * i4 + 0] = v[g * G + 4 * i4 + 0] * l4.x;
+      y[4 * i4 + 1] = v[g * G + 4 * i4 + 1] * l4.y;
+      y[4 * i4 + 2] = v[g * G + 4 * i4 + 2] * l4.z;
+      y[4 * i4 + 3] = v[g * G + 4 * i4 + 3] * l4.w;
     }
-    const float sf = fminf(__fdiv_rn(a, 7.0f), 65504.0f);
-    const __half hs = __float2half_rn(sf);
-    const float sq = __half2float(hs);
-    const float inv = sq > 0.0f ? __frcp_rn(sq) : 0.0f;
-    sbits[g] = __half_as_ushort(hs);
-    const bool clampit = a * inv >= 7.5f;
-    uint32_t b[G];
+    uint32_t w[G / 8];
+    quantize_group<G>(y, w, sbits[g]);
 #pragma unroll
-    for (int i = 0; i < G; i += 2) {
-      float2 q = __ffma2_rn(make_float2(y[i], y[i + 1]), make_float2(inv, inv), make_float2(kMagic, kMagic));
-      if (clampit) {
-        q.x = fminf(fmaxf(q.x, kMagicLo), kMagicHi);
-        q.y = fminf(fmaxf(q.y, kMagicLo), kMagicHi);
-      }
-      b[i] = __float_as_uint(q.x);
-      b[i + 1] = __float_as_uint(q.y);
-    }
-#pragma unroll
-    for (int w = 0; w < G / 8; ++w) {
-      const uint32_t* bb = b + 8 * w;
-      const uint32_t x01 = bb[0] + (bb[1] << 4);
-      const uint32_t x23 = bb[2] + (bb[3] << 4);
-      const uint32_t x45 = bb[4] + (bb[5] << 4);
-      const uint32_t x67 = bb[6] + (bb[7] << 4);
-      words[g * (G / 8) + w] = prmt(x01 + (x23 << 8), x45 + (x67 << 8), 0x5410u) ^ 0x88888888u;
-    }
+    for (int i = 0; i < G / 8; ++i) words[g * (G / 8) + i] = w[i];
   }
 }
 

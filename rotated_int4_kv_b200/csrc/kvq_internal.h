@@ -35,6 +35,10 @@ struct kvq_plan {
   void* dblock = nullptr;
   const kvq::CodecConsts* enc_dev = nullptr;
   const kvq::CodecConsts* dec_dev = nullptr;
+  // Tensor-core encode operand in the same block, fp16 hi rows then lo rows
+  // (value = hi + lo to ~2^-22): D = 128: W = Lambda F_r diag(s) [128][128];
+  // D = 256: the 128-point real DFT in slot order [128][128].
+  const uint16_t* wt_dev = nullptr;
 };
 
 namespace kvq {
@@ -51,6 +55,14 @@ kvq_status encode_tiled(CUtensorMap* map, CUtensorMapDataType dt, int rank, cons
 int num_sms(int device);
 
 kvq_status check_plan_device(const kvq_plan* p);
+
+// tensor-core encode (kvq_encode_tc.cu)
+bool encode_tc_supported(int D, int G);
+kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t s);
+uint32_t encode_tc_error_flags(bool clear);
+// encode path: 0 = tensor cores where supported, else the register FFT; 1 = register FFT; 2 = tensor cores
+int encode_path();
+kvq_status dispatch_encode(const kvq_encode_job* jobs, int njobs, cudaStream_t s);
 
 // codec launchers (kvq_codec.cu)
 kvq_status launch_encode_jobs(const kvq_encode_job* jobs, int njobs, cudaStream_t s);
