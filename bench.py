@@ -387,7 +387,7 @@ def run_kvq(args, rank: int, world: int):
         tc = kvq.get_encode_path() != "fft" and G == 32
         roof = {"bound": "hbm", "achieved": enc_gbs, "peak": hbm, "unit": "GB/s", "frac": enc_gbs / hbm,
                 "traffic": _ncu_traffic("encode_tc" if tc else "encode"),
-                "kernel": ("encode_tc256_kernel<64>" if D == 256 else "encode_tc_kernel<128,64>") if tc
+                "kernel": f"encode_tc_kernel<{D},64>" if tc
                 else f"encode_kernel<{D},{G},64>",
                 "share": enc_avg / (enc_avg + att_avg), "peak_source": src}
     else:

@@ -216,42 +216,20 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
     p->enc.sgn[w] = m;
     p->dec.sgn[w] = m;
   }
-  // tensor-core encode operand, fp16 hi rows then lo rows (value = hi + lo to ~2^-22):
-  //   D = 128: W = Lambda F_r diag(s) [128 x 128] (channel order);
-  //   D = 256: the unnormalised 128-point real DFT in slot order [128 x 128] (row 0: 1,
-  //            row 1: (-1)^m, row 2k: cos(2 pi k m / 128), row 2k+1: -sin(2 pi k m / 128)),
-  //            applied to the even and the odd samples of s (.) x.
-  std::vector<uint16_t> wt;
-  if (D == 256) {
-    const int M = 128;
-    wt.resize((size_t)2 * M * M);
-    const double pi2 = 6.283185307179586476925286766559;
-    for (int j = 0; j < M; ++j)
-      for (int m = 0; m < M; ++m) {
-        double w;
-        if (j == 0) w = 1.0;
-        else if (j == 1) w = (m & 1) ? -1.0 : 1.0;
-        else {
-          const int k = j / 2;
-          const double ang = pi2 * (double)((long)k * m % M) / (double)M;
-          w = (j & 1) ? -std::sin(ang) : std::cos(ang);
-        }
-        const uint16_t hi = kvq::half_bits((float)w);
-        const uint16_t lo = kvq::half_bits((float)(w - (double)kvq::half_value(hi)));
-        wt[(size_t)j * M + m] = hi;
-        wt[(size_t)(M + j) * M + m] = lo;
-      }
-  }
-  if (D == 128) {
-    wt.resize((size_t)2 * D * D);
-    for (int c = 0; c < D; ++c)
-      for (int n = 0; n < D; ++n) {
-        const double w = (double)lambda[c] * kvq::basis_value(c, n, D) * (double)signs[n];
-        const uint16_t hi = kvq::half_bits((float)w);
-        const uint16_t lo = kvq::half_bits((float)(w - (double)kvq::half_value(hi)));
-        wt[(size_t)c * D + n] = hi;
-        wt[(size_t)(D + c) * D + n] = lo;
-      }
+  // tensor-core encode operand: W = Lambda F_r diag(s) (channel rows, D columns) as an
+  // fp16 pair (value = hi + lo to ~2^-22 |W|), laid out per 128-channel half h as
+  // 128 hi rows then 128 lo rows: row 256 h + r = hi of channel 128 h + r,
+  // row 256 h + 128 + r = lo of the same channel.
+  std::vector<uint16_t> wt((size_t)2 * D * D);
+  for (int c = 0; c < D; ++c) {
+    const int h = c / 128, rr = c % 128;
+    for (int n = 0; n < D; ++n) {
+      const double w = (double)lambda[c] * kvq::basis_value(c, n, D) * (double)signs[n];
+      const uint16_t hi = kvq::half_bits((float)w);
+      const uint16_t lo = kvq::half_bits((float)(w - (double)kvq::half_value(hi)));
+      wt[(size_t)(256 * h + rr) * D + n] = hi;
+      wt[(size_t)(256 * h + 128 + rr) * D + n] = lo;
+    }
   }
   constexpr size_t kWtOff = 4096;  // after the two CodecConsts copies, 16-byte aligned for TMA
   static_assert(2 * sizeof(kvq::CodecConsts) <= kWtOff, "plan block layout");

@@ -35,9 +35,8 @@ struct kvq_plan {
   void* dblock = nullptr;
   const kvq::CodecConsts* enc_dev = nullptr;
   const kvq::CodecConsts* dec_dev = nullptr;
-  // Tensor-core encode operand in the same block, fp16 hi rows then lo rows
-  // (value = hi + lo to ~2^-22): D = 128: W = Lambda F_r diag(s) [128][128];
-  // D = 256: the 128-point real DFT in slot order [128][128].
+  // Tensor-core encode operand in the same block: W = Lambda F_r diag(s) as fp16
+  // hi + lo, per 128-channel half 128 hi rows then 128 lo rows, D columns.
   const uint16_t* wt_dev = nullptr;
 };
 

@@ -20,44 +20,64 @@ constexpr float kMagic = 12582920.0f;    // 1.5 * 2^23 + 8: bits = 0x4B400008 + 
 constexpr float kMagicLo = 12582913.0f;  // code -7
 constexpr float kMagicHi = 12582927.0f;  // code +7
 
+// max |y_i| (max is exact, so the order of the reduction does not matter): a tree
+// of three-input maxima, the first level on absolute values.
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ float max3_abs(float a, float b, float c) {
+  float d;
+  asm("max.abs.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+template <int G>
+__device__ __forceinline__ float absmax(const float (&y)[G]) {
+  static_assert(G == 16 || G == 32, "group size");
+  constexpr int L1 = (G + 2) / 3;  // 11 (G = 32) or 6 (G = 16)
+  float m[L1];
+#pragma unroll
+  for (int i = 0; i < G / 3; ++i) m[i] = max3_abs(y[3 * i], y[3 * i + 1], y[3 * i + 2]);
+  if constexpr (G % 3 == 2) m[L1 - 1] = fmaxf(fabsf(y[G - 2]), fabsf(y[G - 1]));
+  if constexpr (G % 3 == 1) m[L1 - 1] = fabsf(y[G - 1]);
+  // 11 -> 4 -> 2 -> 1, or 6 -> 2 -> 1
+  if constexpr (L1 == 11) {
+    const float a0 = max3(m[0], m[1], m[2]), a1 = max3(m[3], m[4], m[5]), a2 = max3(m[6], m[7], m[8]);
+    const float a3 = fmaxf(m[9], m[10]);
+    return fmaxf(max3(a0, a1, a2), a3);
+  } else {
+    return fmaxf(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]));
+  }
+}
+
 // One group of G values (already lambda-scaled): G/8 packed code words and the
 // fp16 scale bits.
 template <int G>
 __device__ __forceinline__ void quantize_group(const float (&y)[G], uint32_t (&words)[G / 8], uint32_t& sbits) {
-  // abs-max as a pairwise tree (max is exact, so the order does not matter)
-  float m[G / 2];
-#pragma unroll
-  for (int i = 0; i < G / 2; ++i) m[i] = fmaxf(fabsf(y[2 * i]), fabsf(y[2 * i + 1]));
-#pragma unroll
-  for (int w = G / 4; w >= 1; w >>= 1)
-#pragma unroll
-    for (int i = 0; i < w; ++i) m[i] = fmaxf(m[i], m[i + w]);
-  const float a = m[0];
+  const float a = absmax<G>(y);
   const float sf = fminf(__fdiv_rn(a, 7.0f), 65504.0f);
   const __half hs = __float2half_rn(sf);
   const float sq = __half2float(hs);
   const float inv = sq > 0.0f ? __frcp_rn(sq) : 0.0f;
   sbits = __half_as_ushort(hs);
-  const bool clampit = a * inv >= 7.5f;
-  uint32_t b[G];
+  // |y| * inv can reach 7.5 only when the scale lost precision (fp16 subnormal or the
+  // 65504 cap): then clamp to the +-7 codes before packing
+  uint32_t bits[G];
+  if (a * inv < 7.5f) {
 #pragma unroll
-  for (int i = 0; i < G; i += 2) {
-    float2 q = __ffma2_rn(make_float2(y[i], y[i + 1]), make_float2(inv, inv), make_float2(kMagic, kMagic));
-    if (clampit) {
-      q.x = fminf(fmaxf(q.x, kMagicLo), kMagicHi);
-      q.y = fminf(fmaxf(q.y, kMagicLo), kMagicHi);
-    }
-    b[i] = __float_as_uint(q.x);
-    b[i + 1] = __float_as_uint(q.y);
+    for (int i = 0; i < G; ++i) bits[i] = __float_as_uint(fmaf(y[i], inv, kMagic));
+  } else {
+#pragma unroll
+    for (int i = 0; i < G; ++i) bits[i] = __float_as_uint(fminf(fmaxf(fmaf(y[i], inv, kMagic), kMagicLo), kMagicHi));
   }
+  // low byte of each word = code + 8 (0..15): two nibbles per byte, four bytes per word
 #pragma unroll
   for (int w = 0; w < G / 8; ++w) {
-    const uint32_t* bb = b + 8 * w;
-    const uint32_t x01 = bb[0] + (bb[1] << 4);
-    const uint32_t x23 = bb[2] + (bb[3] << 4);
-    const uint32_t x45 = bb[4] + (bb[5] << 4);
-    const uint32_t x67 = bb[6] + (bb[7] << 4);
-    words[w] = prmt(x01 + (x23 << 8), x45 + (x67 << 8), 0x5410u) ^ 0x88888888u;
+    const uint32_t* bb = bits + 8 * w;
+    const uint32_t lo = bb[0] + (bb[1] << 4) + ((bb[2] + (bb[3] << 4)) << 8);
+    const uint32_t hi = bb[4] + (bb[5] << 4) + ((bb[6] + (bb[7] << 4)) << 8);
+    words[w] = prmt(lo, hi, 0x5410u) ^ 0x88888888u;
   }
 }
 
