@@ -58,7 +58,9 @@ KERNEL_SOURCES = {
 }
 NCU_TRAFFIC = {
     # kernel -> (source digest at capture time, bytes per launch)
-    "encode": ("800dad8c026c", 115282176),
+    "encode": ("800dad8c026c", 115282176),       # register-FFT encode, Gemma step (52 jobs)
+    "encode_tc": ("cafe5c0e8a7f", 127376384),    # tensor-core encode, Gemma step (52 jobs)
+    "attend": ("f95f7ac4b9ec", 30920960),        # grouped int4 attention, Gemma step (26 jobs)
 }
 
 
@@ -409,6 +411,13 @@ def run_kvq(args, rank: int, world: int):
                           "tokens_heads_per_s": L * Hkv * T / (att_avg * 1e-3), "GB_s": att_gbs,
                           "frac_hbm": att_gbs / hbm, "bytes_per_token_head": tok_b},
             "roofline": roof,
+            "kernels": {  # both launches of the step, each timed with CUDA events on its stream
+                "encode": {"kernel": roof["kernel"] if enc_avg >= att_avg else "encode", "us": 1e3 * enc_avg,
+                           "achieved_GB_s": enc_gbs, "frac": enc_gbs / hbm, "share": enc_avg / (enc_avg + att_avg)},
+                "attention": {"kernel": f"attend_kernel<{D},int4,32>", "us": 1e3 * att_avg, "achieved_GB_s": att_gbs,
+                              "frac": att_gbs / hbm, "share": att_avg / (enc_avg + att_avg),
+                              "traffic": _ncu_traffic("attend")},
+            },
             "cpu_baseline": cpu,
             "e2e": {"value": world * vec_step / (e2e_ms * 1e-3) / 1e6, "unit": "Mvec/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
