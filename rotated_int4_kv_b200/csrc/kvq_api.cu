@@ -231,9 +231,25 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
       wt[(size_t)(256 * h + 128 + rr) * D + n] = lo;
     }
   }
+  // D = 128 attention operands: M = Lambda^-1 F_r (hi, lo) and its transpose (hi, lo)
+  std::vector<uint16_t> rot;
+  if (D == 128) {
+    rot.resize((size_t)4 * D * D);
+    for (int c = 0; c < D; ++c)
+      for (int n = 0; n < D; ++n) {
+        const double m = kvq::basis_value(c, n, D) / (double)lambda[c];
+        const uint16_t hi = kvq::half_bits((float)m);
+        const uint16_t lo = kvq::half_bits((float)(m - (double)kvq::half_value(hi)));
+        rot[(size_t)c * D + n] = hi;                      // rq hi [c][n]
+        rot[(size_t)(D + c) * D + n] = lo;                // rq lo
+        rot[(size_t)(2 * D + n) * D + c] = hi;            // ru hi [n][c]
+        rot[(size_t)(3 * D + n) * D + c] = lo;            // ru lo
+      }
+  }
   constexpr size_t kWtOff = 4096;  // after the two CodecConsts copies, 16-byte aligned for TMA
   static_assert(2 * sizeof(kvq::CodecConsts) <= kWtOff, "plan block layout");
-  const size_t bytes = wt.empty() ? 2 * sizeof(kvq::CodecConsts) : kWtOff + wt.size() * 2;
+  const size_t rot_off = kWtOff + wt.size() * 2;
+  const size_t bytes = rot_off + rot.size() * 2;
   void* blk = nullptr;
   if (cudaMalloc(&blk, bytes) != cudaSuccess) {
     delete p;
@@ -243,7 +259,9 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
       cudaMemcpy((char*)blk + sizeof(kvq::CodecConsts), &p->dec, sizeof(kvq::CodecConsts), cudaMemcpyHostToDevice) !=
           cudaSuccess ||
       (!wt.empty() &&
-       cudaMemcpy((char*)blk + kWtOff, wt.data(), wt.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess)) {
+       cudaMemcpy((char*)blk + kWtOff, wt.data(), wt.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess) ||
+      (!rot.empty() &&
+       cudaMemcpy((char*)blk + rot_off, rot.data(), rot.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess)) {
     cudaFree(blk);
     delete p;
     return fail(KVQ_ERR_CUDA, "plan_create: upload failed");
@@ -252,6 +270,8 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
   p->enc_dev = reinterpret_cast<const kvq::CodecConsts*>(blk);
   p->dec_dev = reinterpret_cast<const kvq::CodecConsts*>((char*)blk + sizeof(kvq::CodecConsts));
   p->wt_dev = wt.empty() ? nullptr : reinterpret_cast<const uint16_t*>((char*)blk + kWtOff);
+  p->rq_dev = rot.empty() ? nullptr : reinterpret_cast<const uint16_t*>((char*)blk + rot_off);
+  p->ru_dev = rot.empty() ? nullptr : reinterpret_cast<const uint16_t*>((char*)blk + rot_off + (size_t)2 * D * D * 2);
   *out = p;
   return KVQ_OK;
 }

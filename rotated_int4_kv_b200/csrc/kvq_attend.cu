@@ -87,8 +87,13 @@ struct Cfg {
   // (hi01, hi23, lo01, lo23) -- read from shared memory at each use
   static constexpr int kKSteps = INT4 ? 2 * NG : D / 16;
   static constexpr int kQf = kKSteps * 32 * 16;
-  static constexpr int kBars = 128;        // full[], empty[], const barrier, flag
-  static constexpr int kSmem = kScratch + kQt + kQs + kConsts + kQf + kBars + 1024;
+  static constexpr int kBars = 128;        // full[], empty[], const barrier, rotation barrier, flag
+  // D = 128 int4: the plan's rotation matrix (hi, lo) for the query, then the V plan's
+  // transpose for the output, as [hi/lo][64-column chunk][128 rows][128 B] (128-byte swizzle)
+  static constexpr bool kMmaRot = INT4 && D == 128;
+  static constexpr int kRotOff = (kScratch + kQt + kQs + kConsts + kQf + kBars + 1023) / 1024 * 1024;
+  static constexpr int kRot = kMmaRot ? 4 * 128 * 128 : 0;
+  static constexpr int kSmem = kRotOff + kRot + 1024;
   static_assert(2 * kStages * 8 + 8 + 4 <= kBars, "barrier region");
 };
 
@@ -105,6 +110,7 @@ struct AttnParams {
 // blockIdx.z = job * (B * Hkv) + b * Hkv + kv head.
 struct alignas(64) AttnJob {
   CUtensorMap kmap, vmap, ksmap, vsmap;  // K/V codes (or fp16 K/V) and scale rows
+  CUtensorMap rqmap, rumap;              // D = 128 int4: K plan rotation, V plan un-rotation (hi/lo rows)
   const uint16_t* q;
   uint16_t* out;
   const CodecConsts* ke;  // K plan: sign masks (int4 only)
@@ -283,6 +289,103 @@ __device__ __forceinline__ void unrotate_out(const float* om, int heads, const f
   }
 }
 
+// D = 128: q_t[h][c] = sum_n M[c][n] q'[h][n] with q' = s (.) q (fp16, exact) and
+// M = Lambda^-1 F_r held as fp16 hi + lo in shared memory ([hi/lo][64-column chunk]
+// [128 rows][128 B], 128-byte swizzle), on the tensor cores: mma.m16n8k16 with 16
+// channels as M, the 8 heads as N, samples as K; the four consumer warps take two
+// channel tiles each. Heads beyond `heads` get zero rows.
+__device__ __forceinline__ uint32_t rot_addr(const uint8_t* base, int hl, int row, int col) {
+  // element (row, col) of matrix hl (0 = hi, 1 = lo); col multiple of 8
+  const int kc = col >> 6, ch = (col & 63) >> 3;
+  return smem_u32(base + (2 * hl + kc) * 16384 + row * 128 + ((ch ^ (row & 7)) << 4));
+}
+
+__device__ __forceinline__ void rotate_query_mma(const uint16_t* qs, int heads, const uint32_t* ksg,
+                                                 const uint8_t* srot, float* qt, int warp, int lane) {
+  const int g = lane >> 2, cq = lane & 3;
+  const int mi = lane >> 3;
+  // B fragments (k = samples, n = head g): q'[g][16 ks + 2 cq (+1)], [.. + 8 (+9)]
+  uint32_t bq[8][2];
+  const uint32_t* qrow = reinterpret_cast<const uint32_t*>(qs + (g < heads ? g : 0) * 128);
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+    const int w0 = 8 * ks + cq, w1 = w0 + 4;  // fp16-pair words of the row
+    bq[ks][0] = g < heads ? (qrow[w0] ^ ksg[w0]) : 0u;
+    bq[ks][1] = g < heads ? (qrow[w1] ^ ksg[w1]) : 0u;
+  }
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int mt = 2 * warp + t;  // channels 16 mt .. 16 mt + 15
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int row = 16 * mt + ((mi & 1) << 3) + (lane & 7);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int col = 16 * ks + ((mi >> 1) << 3);
+      uint32_t a0, a1, a2, a3;
+      ldmatrix_x4(a0, a1, a2, a3, rot_addr(srot, 0, row, col));
+      mma_16816(acc, a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
+      ldmatrix_x4(a0, a1, a2, a3, rot_addr(srot, 1, row, col));
+      mma_16816(acc, a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
+    }
+    // C layout: rows g, g + 8 (channels), columns 2 cq, 2 cq + 1 (heads)
+    const int c0 = 16 * mt + g;
+    qt[(2 * cq) * 128 + c0] = acc[0];
+    qt[(2 * cq + 1) * 128 + c0] = acc[1];
+    qt[(2 * cq) * 128 + c0 + 8] = acc[2];
+    qt[(2 * cq + 1) * 128 + c0 + 8] = acc[3];
+  }
+}
+
+// D = 128: x[h][n] = sum_c M^T[n][c] o_t[h][c] / L_h (the sign is applied at the fp16
+// store), with M^T held like M above; o_t (fp32) enters as an fp16 hi + lo pair, so
+// three products per step (hi.hi, hi.lo, lo.hi) keep ~2^-22 relative precision.
+__device__ __forceinline__ void unrotate_out_mma(const float* om, int heads, const float* Lh, const uint8_t* srot,
+                                                 float* xb, int warp, int lane) {
+  const int g = lane >> 2, cq = lane & 3;
+  const int mi = lane >> 3;
+  const float L = g < heads ? Lh[g] : 0.0f;
+  const float r = L > 0.0f ? 1.0f / L : 0.0f;
+  const float* orow = om + (g < heads ? g : 0) * 128;
+  uint32_t bh[8][2], bl[8][2];
+#pragma unroll
+  for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int k0 = 16 * ks + 2 * cq + 8 * e;
+      const float v0 = orow[k0] * r, v1 = orow[k0 + 1] * r;
+      const __half h0 = __float2half_rn(v0), h1 = __float2half_rn(v1);
+      const __half l0 = __float2half_rn(v0 - __half2float(h0)), l1 = __float2half_rn(v1 - __half2float(h1));
+      bh[ks][e] = g < heads ? h2_bits(__halves2half2(h0, h1)) : 0u;
+      bl[ks][e] = g < heads ? h2_bits(__halves2half2(l0, l1)) : 0u;
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    const int mt = 2 * warp + t;  // samples 16 mt .. 16 mt + 15
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    const int row = 16 * mt + ((mi & 1) << 3) + (lane & 7);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+      const int col = 16 * ks + ((mi >> 1) << 3);
+      uint32_t a0, a1, a2, a3;
+      ldmatrix_x4(a0, a1, a2, a3, rot_addr(srot, 0, row, col));
+      mma_16816(acc, a0, a1, a2, a3, bh[ks][0], bh[ks][1]);
+      mma_16816(acc, a0, a1, a2, a3, bl[ks][0], bl[ks][1]);
+      ldmatrix_x4(a0, a1, a2, a3, rot_addr(srot, 1, row, col));
+      mma_16816(acc, a0, a1, a2, a3, bh[ks][0], bh[ks][1]);
+    }
+    const int n0 = 16 * mt + g;
+    if (2 * cq < heads) {
+      xb[(2 * cq) * 128 + n0] = acc[0];
+      xb[(2 * cq) * 128 + n0 + 8] = acc[2];
+    }
+    if (2 * cq + 1 < heads) {
+      xb[(2 * cq + 1) * 128 + n0] = acc[1];
+      xb[(2 * cq + 1) * 128 + n0 + 8] = acc[3];
+    }
+  }
+}
+
 template <int D, bool INT4, int MAXJ>
 __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
     attend_kernel(const __grid_constant__ AttnJobs<MAXJ> jt, const __grid_constant__ AttnParams p) {
@@ -303,7 +406,9 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kScratch + C::kQt + C::kQs + C::kConsts + C::kQf);
   uint64_t* empty = full + C::kStages;
   uint64_t* cbar = empty + C::kStages;
-  int* flag = reinterpret_cast<int*>(cbar + 1);
+  uint64_t* ubar = cbar + 1;  // un-rotation matrix landed (D = 128 int4)
+  int* flag = reinterpret_cast<int*>(ubar + 1);
+  uint8_t* srot = smem + C::kRotOff;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -330,6 +435,7 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
       mbar_init(&empty[s], kCWarps);
     }
     mbar_init(cbar, 1);
+    mbar_init(ubar, 1);
     fence_mbarrier_init();
   }
   __syncthreads();
@@ -347,13 +453,19 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
     if (lane == 0) {
       // query rows of the tile and the plans' constants: one round trip, one barrier
       const uint32_t qbytes = (uint32_t)(heads * D * 2);
-      mbar_arrive_expect_tx(cbar, qbytes + (INT4 ? (uint32_t)C::kConsts : 0u));
+      mbar_arrive_expect_tx(cbar, qbytes + (INT4 ? (uint32_t)C::kConsts : 0u) + (uint32_t)C::kRot);
       bulk_load(qs, J.q + ((size_t)b * p.Hq + hq0) * D, qbytes, cbar);
       if constexpr (INT4) {
         bulk_load(cst, J.kd->chan, C::kChanBytes, cbar);
         bulk_load(cst + C::kChanBytes, J.ke->sgn, C::kSgnBytes, cbar);
         bulk_load(cst + C::kChanBytes + C::kSgnBytes, J.vd->chan, C::kChanBytes, cbar);
         bulk_load(cst + 2 * C::kChanBytes + C::kSgnBytes, J.vd->sgn, C::kSgnBytes, cbar);
+      }
+      if constexpr (C::kMmaRot) {
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int kc = 0; kc < 2; ++kc) tma_load_2d(srot + (2 * hl + kc) * 16384, &J.rqmap, cbar, 64 * kc, 128 * hl);
       }
       prefetch_tensormap(&J.kmap);
       prefetch_tensormap(&J.vmap);
@@ -398,7 +510,9 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
       atomicOr(&g_attend_err, kErrTimeoutLoad);
       ok = false;
     }
-    if constexpr (INT4) {
+    if constexpr (C::kMmaRot) {
+      rotate_query_mma(qs, heads, ksg, srot, qt, warp, lane);
+    } else if constexpr (INT4) {
       if (warp == 0) rotate_query<D>(qs, heads, ksg, kch, qt, lane);
       for (int i = threadIdx.x; i < (kHT - heads) * D; i += kCWarps * 32) qt[heads * D + i] = 0.0f;
     } else {
@@ -409,6 +523,18 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
       }
     }
     consumer_sync();
+    if constexpr (C::kMmaRot) {
+      // the rotation matrix is consumed: a cluster leader (the only CTA that can run the
+      // final merge) prefetches the V plan's un-rotation matrix into the same buffer
+      if (threadIdx.x == 0 && cg::this_cluster().block_rank() == 0) {
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(ubar, (uint32_t)C::kRot);
+#pragma unroll
+        for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+          for (int kc = 0; kc < 2; ++kc) tma_load_2d(srot + (2 * hl + kc) * 16384, &J.rumap, ubar, 64 * kc, 128 * hl);
+      }
+    }
 
     // (2) B fragments of the score product (n = head g), built once per CTA into
     // shared memory (warp w takes k steps w, w + 4, ...)
@@ -749,6 +875,9 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
   if (crank == 0) merge(csize, [&](int r) { return static_cast<const float*>(cluster.map_shared_rank(cpart, r)); });
   cluster.sync();  // peers may leave once the leader has read their shared memory
   if (crank != 0) return;
+  // (D = 128 int4) the leader's un-rotation matrix prefetch must land before the CTA may exit
+  bool rot_ok = true;
+  if constexpr (C::kMmaRot) rot_ok = mbar_wait_bounded(ubar, 0);
   // the producer warp reads staged constants below: observe their barrier too
   if (warp == kCWarps && !mbar_wait_bounded(cbar, 0)) atomicOr(&g_attend_err, kErrTimeoutLoad);
 
@@ -778,7 +907,15 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
 
   // ------------------------------------------------------------ normalise, un-rotate, store fp16
   uint16_t* ob = J.out + ((size_t)b * p.Hq + hq0) * D;
-  if constexpr (INT4) {
+  if constexpr (C::kMmaRot) {
+    if (!rot_ok && threadIdx.x == 0) atomicOr(&g_attend_err, kErrTimeoutLoad);
+    if (warp < kCWarps) unrotate_out_mma(om, heads, mrg + kHT, srot, xb, warp, lane);
+    __syncthreads();
+    for (int i = threadIdx.x; i < heads * D / 2; i += kThreads) {
+      const int j = i % (D / 2);
+      reinterpret_cast<uint32_t*>(ob)[i] = pack_half2(xb[2 * i], xb[2 * i + 1]) ^ vsg[j];
+    }
+  } else if constexpr (INT4) {
     if (warp == 0) unrotate_out<D>(om, heads, vch, mrg + kHT, xb, lane);
     __syncthreads();
     // fp16 with the V sign folded in as an XOR on the sign bits
@@ -959,6 +1096,17 @@ kvq_status make_job(const AttendJobHost& h, int B, int Hkv, int T_cap, AttnJob* 
     if (st != KVQ_OK) return st;
     j->ksmap = j->kmap;
     j->vsmap = j->vmap;
+  }
+  if constexpr (INT4 && D == 128) {
+    const uint64_t rd[2] = {128u, 256u};
+    const uint64_t rs[1] = {256u};
+    const uint32_t rb[2] = {64u, 128u};
+    st = encode_tiled(&j->rqmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h.pk->rq_dev, rd, rs, rb,
+                      CU_TENSOR_MAP_SWIZZLE_128B, "K rotation");
+    if (st == KVQ_OK)
+      st = encode_tiled(&j->rumap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h.pv->ru_dev, rd, rs, rb,
+                        CU_TENSOR_MAP_SWIZZLE_128B, "V un-rotation");
+    if (st != KVQ_OK) return st;
   }
   j->q = h.q;
   j->out = h.out;
