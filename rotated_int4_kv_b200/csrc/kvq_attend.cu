@@ -126,18 +126,26 @@ struct AttnJobs {
 __device__ __forceinline__ uint32_t h2_bits(__half2 h) { return *reinterpret_cast<uint32_t*>(&h); }
 __device__ __forceinline__ __half2 bits_h2(uint32_t u) { return *reinterpret_cast<__half2*>(&u); }
 
+// (a & mask) ^ c on the mask bits, c elsewhere: one lop3 (truth table b ? a ^ c : c).
+__device__ __forceinline__ uint32_t lop3_xor_in_mask(uint32_t a, uint32_t mask, uint32_t c) {
+  uint32_t d;
+  asm("lop3.b32 %0, %1, %2, %3, 0x6A;" : "=r"(d) : "r"(a), "r"(mask), "r"(c));
+  return d;
+}
+
 // Four fp16x2 pairs of exact integer codes from one word of eight nibbles
 // (two's complement). Output pairs: (n0,n4), (n1,n5), (n2,n6), (n3,n7).
+// Each lop3 forms 0x6400 | (nibble ^ 8) per half, i.e. the fp16 value 1024 + code + 8
+// (or 1024 + 16 (code + 8) for the high nibbles); one fp16 op removes the offset.
 __device__ __forceinline__ void nib8_to_h2(uint32_t w, uint32_t (&h)[4]) {
-  const uint32_t u = w ^ 0x88888888u;  // offset binary: code + 8
   const __half2 k1032 = __floats2half2_rn(1032.0f, 1032.0f);
   const __half2 k16 = __floats2half2_rn(0.0625f, 0.0625f);
   const __half2 k72 = __floats2half2_rn(-72.0f, -72.0f);
-  const uint32_t a = lop3_and_or(u, 0x000F000Fu, 0x64006400u);
-  const uint32_t b = lop3_and_or(u, 0x00F000F0u, 0x64006400u);
-  const uint32_t u8 = u >> 8;
-  const uint32_t c = lop3_and_or(u8, 0x000F000Fu, 0x64006400u);
-  const uint32_t d = lop3_and_or(u8, 0x00F000F0u, 0x64006400u);
+  const uint32_t a = lop3_xor_in_mask(w, 0x000F000Fu, 0x64086408u);
+  const uint32_t b = lop3_xor_in_mask(w, 0x00F000F0u, 0x64806480u);
+  const uint32_t w8 = w >> 8;
+  const uint32_t c = lop3_xor_in_mask(w8, 0x000F000Fu, 0x64086408u);
+  const uint32_t d = lop3_xor_in_mask(w8, 0x00F000F0u, 0x64806480u);
   h[0] = h2_bits(__hsub2(bits_h2(a), k1032));
   h[1] = h2_bits(__hfma2(bits_h2(b), k16, k72));
   h[2] = h2_bits(__hsub2(bits_h2(c), k1032));
