@@ -231,8 +231,29 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
       wt[(size_t)(256 * h + 128 + rr) * D + n] = lo;
     }
   }
-  // D = 128 attention operands: M = Lambda^-1 F_r (hi, lo) and its transpose (hi, lo)
+  // attention operands. D = 128: M = Lambda^-1 F_r (hi, lo) and its transpose (hi, lo).
+  // D = 256: the unnormalised 128-point real DFT in slot order, F128 (hi, lo): row 0 = 1,
+  // row 1 = (-1)^m, row 2k = cos(2 pi k m / 128), row 2k+1 = -sin(2 pi k m / 128).
   std::vector<uint16_t> rot;
+  if (D == 256) {
+    const int M = 128;
+    rot.resize((size_t)2 * M * M);
+    const double pi2 = 6.283185307179586476925286766559;
+    for (int j = 0; j < M; ++j)
+      for (int m = 0; m < M; ++m) {
+        double v;
+        if (j == 0) v = 1.0;
+        else if (j == 1) v = (m & 1) ? -1.0 : 1.0;
+        else {
+          const double ang = pi2 * (double)((long)(j / 2) * m % M) / (double)M;
+          v = (j & 1) ? -std::sin(ang) : std::cos(ang);
+        }
+        const uint16_t hi = kvq::half_bits((float)v);
+        const uint16_t lo = kvq::half_bits((float)(v - (double)kvq::half_value(hi)));
+        rot[(size_t)j * M + m] = hi;
+        rot[(size_t)(M + j) * M + m] = lo;
+      }
+  }
   if (D == 128) {
     rot.resize((size_t)4 * D * D);
     for (int c = 0; c < D; ++c)
@@ -271,7 +292,8 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
   p->dec_dev = reinterpret_cast<const kvq::CodecConsts*>((char*)blk + sizeof(kvq::CodecConsts));
   p->wt_dev = wt.empty() ? nullptr : reinterpret_cast<const uint16_t*>((char*)blk + kWtOff);
   p->rq_dev = rot.empty() ? nullptr : reinterpret_cast<const uint16_t*>((char*)blk + rot_off);
-  p->ru_dev = rot.empty() ? nullptr : reinterpret_cast<const uint16_t*>((char*)blk + rot_off + (size_t)2 * D * D * 2);
+  p->ru_dev = D != 128 || rot.empty() ? nullptr
+                                      : reinterpret_cast<const uint16_t*>((char*)blk + rot_off + (size_t)2 * D * D * 2);
   *out = p;
   return KVQ_OK;
 }

@@ -22,13 +22,18 @@
 //     group's fp32 partial. P is transposed with four shuffles into the B operand
 //     of the PV product (channels as M, tokens as K), with the V scale folded
 //     into P per group. Online softmax runs in base 2;
-//   * warps merge in shared memory, the CTA writes (m, l, o) to the workspace,
-//     and the last CTA of a (b, kv head, head tile) -- found with an atomic
-//     counter, no waiting -- merges the splits and un-rotates with the inverse
-//     register FFT (o = diag(s_V) F_r^T Lambda_V^-1 o_t), then writes fp16.
-// The query is rotated inside every CTA with the forward register FFT while the
-// producer's first loads are in flight. Tensor cores are used for issue rate,
-// not throughput: the kernel is bound by HBM bandwidth.
+//   * warps merge in shared memory; the splits of a (b, kv head, head tile) form a
+//     thread-block cluster and merge through distributed shared memory; when the
+//     splits span several clusters, the cluster leaders write (m, l, o) to the
+//     workspace and the last one -- found with an atomic counter, no waiting --
+//     merges them; the final leader un-rotates and writes fp16.
+// The query rotation and the output un-rotation run on the tensor cores with
+// matrices precomputed per plan and TMA-loaded into shared memory (fp16 hi + lo
+// pairs, ~2^-22 relative): at D = 128 the dense Lambda^-1 F_r (query) and its
+// transpose for the V plan (output, prefetched during the token loop); at D = 256
+// the 128-point real DFT applied to the even and odd samples, joined by one
+// radix-2 step (the even/odd split of the length-256 transform). Tensor cores are
+// used for issue rate, not throughput: the token loop is bound by HBM bandwidth.
 #include <algorithm>
 #include <cstdio>
 #include <mutex>
@@ -37,7 +42,6 @@
 #include <cooperative_groups.h>
 
 #include "kvq_ptx.cuh"
-#include "srft_fft.cuh"
 
 namespace kvq {
 
@@ -90,7 +94,7 @@ struct Cfg {
   static constexpr int kBars = 128;        // full[], empty[], const barrier, rotation barrier, flag
   // D = 128 int4: the plan's rotation matrix (hi, lo) for the query, then the V plan's
   // transpose for the output, as [hi/lo][64-column chunk][128 rows][128 B] (128-byte swizzle)
-  static constexpr bool kMmaRot = INT4 && D == 128;
+  static constexpr bool kMmaRot = INT4;   // D = 128: Lambda^-1 F_r; D = 256: F128 (even/odd split)
   static constexpr int kRotOff = (kScratch + kQt + kQs + kConsts + kQf + kBars + 1023) / 1024 * 1024;
   static constexpr int kRot = kMmaRot ? 4 * 128 * 128 : 0;
   static constexpr int kSmem = kRotOff + kRot + 1024;
@@ -160,141 +164,6 @@ __device__ __forceinline__ float fast_exp2(float x) { return ex2_approx(x); }
 __device__ __forceinline__ void split_h(float x, __half& hi, __half& lo) {
   hi = __float2half_rn(x);
   lo = __float2half_rn(x - __half2float(hi));
-}
-
-// q_t = Lambda_K^-1 F_r diag(s_K) q for the real heads of a tile, by the register
-// FFT: one lane per head at D = 128, a lane pair per head at D = 256 (all 32
-// lanes of the calling warp execute it; lanes beyond the real heads work on zeros).
-template <int D>
-__device__ __forceinline__ void rotate_query(const uint16_t* qs, int heads, const uint32_t* ksg, const float* kch,
-                                             float* qt, int lane) {
-  float2 v[64];
-  if constexpr (D == 128) {
-    const int h = lane;
-    const bool live = h < heads;
-    const uint4* src = reinterpret_cast<const uint4*>(qs + (live ? h : 0) * D);
-#pragma unroll
-    for (int cc = 0; cc < 16; ++cc) {
-      uint4 w = live ? src[cc] : make_uint4(0u, 0u, 0u, 0u);
-      const uint4 m = reinterpret_cast<const uint4*>(ksg)[cc];
-      const uint32_t ww[4] = {w.x ^ m.x, w.y ^ m.y, w.z ^ m.z, w.w ^ m.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) v[4 * cc + q] = __half22float2(*reinterpret_cast<const __half2*>(&ww[q]));
-    }
-    rdft_fwd_packed<128>(v);
-    if (live) {
-#pragma unroll
-      for (int c4 = 0; c4 < 32; ++c4) {
-        const float4 k4 = reinterpret_cast<const float4*>(kch)[c4];
-        float4 o;
-        o.x = slotv(v, slot_of_channel(4 * c4 + 0, 128)) * k4.x;
-        o.y = slotv(v, slot_of_channel(4 * c4 + 1, 128)) * k4.y;
-        o.z = slotv(v, slot_of_channel(4 * c4 + 2, 128)) * k4.z;
-        o.w = slotv(v, slot_of_channel(4 * c4 + 3, 128)) * k4.w;
-        reinterpret_cast<float4*>(qt + h * D)[c4] = o;
-      }
-    }
-  } else {
-    const int h = lane >> 1;
-    const bool p = (lane & 1) != 0;
-    const bool live = h < heads;
-    const uint32_t sel = p ? 0x7632u : 0x5410u;
-    const uint4* src = reinterpret_cast<const uint4*>(qs + (live ? h : 0) * D);
-#pragma unroll
-    for (int cc = 0; cc < 32; ++cc) {  // thread p takes q[8cc + p + 2i]
-      const uint4 w = live ? src[cc] : make_uint4(0u, 0u, 0u, 0u);
-      const uint4 m = reinterpret_cast<const uint4*>(ksg)[cc];
-      uint32_t h0 = prmt(w.x ^ m.x, w.y ^ m.y, sel);
-      uint32_t h1 = prmt(w.z ^ m.z, w.w ^ m.w, sel);
-      v[2 * cc] = __half22float2(*reinterpret_cast<const __half2*>(&h0));
-      v[2 * cc + 1] = __half22float2(*reinterpret_cast<const __half2*>(&h1));
-    }
-    rdft_fwd_packed<128>(v);
-    float o[128];
-    pair_combine<0>(v, o, p);
-    if (live) {
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int cb = half ? (p ? 128 : 192) : (p ? 64 : 0);
-#pragma unroll
-        for (int c4 = 0; c4 < 16; ++c4) {
-          const float4 k4 = reinterpret_cast<const float4*>(kch + cb)[c4];
-          const int L = 64 * half + 4 * c4;
-          reinterpret_cast<float4*>(qt + h * D + cb)[c4] =
-              make_float4(o[L] * k4.x, o[L + 1] * k4.y, o[L + 2] * k4.z, o[L + 3] * k4.w);
-        }
-      }
-    }
-  }
-}
-
-// x = F_r^T Lambda_V^-1 o_t / L_h (without the sign, applied at the fp16 store)
-// for the real heads, by the inverse register FFT; writes fp32 x[h][n] to xb.
-// vch: dg / lambda per rotated channel (shared memory); Lh: softmax denominators.
-template <int D>
-__device__ __forceinline__ void unrotate_out(const float* om, int heads, const float* vch, const float* Lh, float* xb,
-                                             int lane) {
-  float2 u[64];
-  if constexpr (D == 128) {
-    const int h = lane;
-    const bool live = h < heads;
-    const float* oh = om + (live ? h : 0) * D;
-    const float L = live ? Lh[h] : 0.0f;
-    const float r = L > 0.0f ? 1.0f / L : 0.0f;
-#pragma unroll
-    for (int c4 = 0; c4 < 32; ++c4) {
-      const float4 k4 = reinterpret_cast<const float4*>(vch)[c4];
-      const float4 o4 = live ? reinterpret_cast<const float4*>(oh)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
-      const float ov[4] = {o4.x * k4.x * r, o4.y * k4.y * r, o4.z * k4.z * r, o4.w * k4.w * r};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int sl = slot_of_channel(4 * c4 + e, 128);
-        if (sl & 1)
-          u[sl >> 1].y = ov[e];
-        else
-          u[sl >> 1].x = ov[e];
-      }
-    }
-    rdft_inv_packed<128>(u);
-    if (live) {
-#pragma unroll
-      for (int m = 0; m < 64; m += 2)
-        reinterpret_cast<float4*>(xb + h * D)[m >> 1] = make_float4(u[m].x, u[m].y, u[m + 1].x, u[m + 1].y);
-    }
-  } else {
-    const int h = lane >> 1;
-    const bool p = (lane & 1) != 0;
-    const bool live = h < heads;
-    const float* oh = om + (live ? h : 0) * D;
-    const float L = live ? Lh[h] : 0.0f;
-    const float r = L > 0.0f ? 1.0f / L : 0.0f;
-    float o[128];
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      const int cb = half ? (p ? 128 : 192) : (p ? 64 : 0);
-#pragma unroll
-      for (int c4 = 0; c4 < 16; ++c4) {
-        const float4 k4 = reinterpret_cast<const float4*>(vch + cb)[c4];
-        const float4 o4 = live ? reinterpret_cast<const float4*>(oh + cb)[c4] : make_float4(0.f, 0.f, 0.f, 0.f);
-        const int m = 64 * half + 4 * c4;
-        o[m] = o4.x * k4.x * r;
-        o[m + 1] = o4.y * k4.y * r;
-        o[m + 2] = o4.z * k4.z * r;
-        o[m + 3] = o4.w * k4.w * r;
-      }
-    }
-#pragma unroll
-    for (int m = 0; m < 64; ++m) u[m] = make_float2(0.f, 0.f);
-    pair_combine_inv<0>(o, u, p);
-    rdft_inv_packed<128>(u);
-    if (live) {
-#pragma unroll
-      for (int m = 0; m < 64; ++m) {  // u[m] = (x[4m + p], x[4m + 2 + p])
-        xb[h * D + 4 * m + (p ? 1 : 0)] = u[m].x;
-        xb[h * D + 4 * m + 2 + (p ? 1 : 0)] = u[m].y;
-      }
-    }
-  }
 }
 
 // D = 128: q_t[h][c] = sum_n M[c][n] q'[h][n] with q' = s (.) q (fp16, exact) and
@@ -390,6 +259,208 @@ __device__ __forceinline__ void unrotate_out_mma(const float* om, int heads, con
     if (2 * cq + 1 < heads) {
       xb[(2 * cq + 1) * 128 + n0] = acc[1];
       xb[(2 * cq + 1) * 128 + n0 + 8] = acc[3];
+    }
+  }
+}
+
+// D = 256 by one radix-2 decimation in time: E = F128 q'_even, O = F128 q'_odd on the
+// tensor cores (F128 = the unnormalised 128-point real DFT in slot order, fp16 hi + lo
+// in shared memory, same layout as above), then X_k = E_k + W^k O_k, X_{128-k} =
+// conj(E_k - W^k O_k) (W = e^{-2 pi i / 256}) and q_t[c] = (dg / lambda)_c X(c).
+// eo: fp32 scratch [E, O][8 heads][128 slots]. Called by the four consumer warps.
+__device__ __forceinline__ void rotate_query_eo(const uint16_t* qs, int heads, const uint32_t* ksg, const float* kch,
+                                                const uint8_t* srot, float* eo, float* qt, int warp, int lane) {
+  const int g = lane >> 2, cq = lane & 3;
+  const int mi = lane >> 3;
+  {
+    // B fragments (k = m, n = head g): even samples 2m and odd samples 2m + 1 of q' = s (.) q
+    uint32_t be[8][2], bo[8][2];
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(qs + (g < heads ? g : 0) * 256);
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int m0 = 16 * ks + 2 * cq + 8 * e;  // words m0, m0 + 1 hold samples 2 m0 .. 2 m0 + 3
+        const uint32_t wa = qrow[m0] ^ ksg[m0], wb = qrow[m0 + 1] ^ ksg[m0 + 1];
+        be[ks][e] = g < heads ? prmt(wa, wb, 0x5410u) : 0u;
+        bo[ks][e] = g < heads ? prmt(wa, wb, 0x7632u) : 0u;
+      }
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int mt = 2 * warp + t;  // slots 16 mt .. 16 mt + 15
+      float ae[4] = {0.f, 0.f, 0.f, 0.f}, ao[4] = {0.f, 0.f, 0.f, 0.f};
+      const int row = 16 * mt + ((mi & 1) << 3) + (lane & 7);
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        const int col = 16 * ks + ((mi >> 1) << 3);
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4(a0, a1, a2, a3, rot_addr(srot, 0, row, col));
+        mma_16816(ae, a0, a1, a2, a3, be[ks][0], be[ks][1]);
+        mma_16816(ao, a0, a1, a2, a3, bo[ks][0], bo[ks][1]);
+        ldmatrix_x4(a0, a1, a2, a3, rot_addr(srot, 1, row, col));
+        mma_16816(ae, a0, a1, a2, a3, be[ks][0], be[ks][1]);
+        mma_16816(ao, a0, a1, a2, a3, bo[ks][0], bo[ks][1]);
+      }
+      const int j0 = 16 * mt + g;
+      eo[(2 * cq) * 128 + j0] = ae[0];
+      eo[(2 * cq + 1) * 128 + j0] = ae[1];
+      eo[(2 * cq) * 128 + j0 + 8] = ae[2];
+      eo[(2 * cq + 1) * 128 + j0 + 8] = ae[3];
+      eo[1024 + (2 * cq) * 128 + j0] = ao[0];
+      eo[1024 + (2 * cq + 1) * 128 + j0] = ao[1];
+      eo[1024 + (2 * cq) * 128 + j0 + 8] = ao[2];
+      eo[1024 + (2 * cq + 1) * 128 + j0 + 8] = ao[3];
+    }
+  }
+  consumer_sync();
+  // radix-2 combine into channels: thread t takes channels t and t + 128 of every head
+  const int t = threadIdx.x;  // 0 .. 127 (consumer warps)
+#pragma unroll
+  for (int half = 0; half < 2; ++half) {
+    const int ch = t + 128 * half;
+    int k, slot_re, slot_im;
+    bool mirror = false, re;
+    if (ch == 0) {
+      k = 0; re = true;
+    } else if (ch == 255) {
+      k = 0; re = true; mirror = true;  // X_128 = E_0 - O_0
+    } else {
+      const int kk = (ch + 1) >> 1;
+      re = (ch & 1) != 0;
+      if (kk <= 64) {
+        k = kk;
+      } else {
+        k = 128 - kk;
+        mirror = true;
+      }
+    }
+    slot_re = k == 0 ? 0 : (k == 64 ? 1 : 2 * k);
+    slot_im = (k == 0 || k == 64) ? -1 : 2 * k + 1;
+    float sn, cs;
+    sincospif((float)k / 128.0f, &sn, &cs);
+    const float f = kch[ch];
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      float v = 0.0f;
+      if (h < heads) {
+        const float* E = eo + h * 128;
+        const float* O = eo + 1024 + h * 128;
+        const float er = E[slot_re], orr = O[slot_re];
+        const float ei = slot_im >= 0 ? E[slot_im] : 0.0f, oi = slot_im >= 0 ? O[slot_im] : 0.0f;
+        float tr = fmaf(cs, orr, sn * oi), ti = fmaf(cs, oi, -sn * orr);
+        if (k == 64) {  // W^64 = -i and E_64, O_64 real: X_64 = E_64 - i O_64
+          tr = 0.0f;
+          ti = -orr;
+        }
+        const float xr = mirror ? er - tr : er + tr;
+        const float xi = mirror ? ti - ei : ei + ti;
+        v = (re ? xr : xi) * f;
+      }
+      qt[h * 256 + ch] = v;
+    }
+  }
+}
+
+// Transpose of rotate_query_eo for the output (sign applied at the fp16 store):
+// Z_c = (dg / lambda)_c o_t[c] / L; (E', O') = combine^T(Z); x_even = F128^T E',
+// x_odd = F128^T O' on the tensor cores (ldmatrix.trans of the resident F128; E', O'
+// enter as fp16 hi + lo). eo: fp32 scratch [2][8][128]. All 160 threads call it.
+__device__ __forceinline__ void unrotate_out_eo(const float* om, int heads, const float* Lh, const float* vch,
+                                                const uint8_t* srot, float* eo, float* xb, int warp, int lane) {
+  const int t = threadIdx.x;
+  if (t <= 64) {  // k = t
+    const int k = t;
+    float sn, cs;
+    sincospif((float)k / 128.0f, &sn, &cs);
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+      float* E = eo + h * 128;
+      float* O = eo + 1024 + h * 128;
+      if (h >= heads) {
+        if (k == 0) { E[0] = O[0] = 0.0f; }
+        else if (k == 64) { E[1] = O[1] = 0.0f; }
+        else { E[2 * k] = E[2 * k + 1] = O[2 * k] = O[2 * k + 1] = 0.0f; }
+        continue;
+      }
+      const float L = Lh[h];
+      const float r = L > 0.0f ? 1.0f / L : 0.0f;
+      const float* o = om + h * 256;
+      auto Z = [&](int c) { return o[c] * vch[c] * r; };
+      if (k == 0) {
+        const float z0 = Z(0), z128 = Z(255);
+        E[0] = z0 + z128;
+        O[0] = z0 - z128;
+      } else if (k == 64) {
+        E[1] = Z(127);   // Re X_64
+        O[1] = -Z(128);  // -Im X_64
+      } else {
+        const int m = 128 - k;
+        const float zrk = Z(2 * k - 1), zik = Z(2 * k), zrm = Z(2 * m - 1), zim = Z(2 * m);
+        const float dr = zrk - zrm, si = zik + zim;
+        E[2 * k] = zrk + zrm;
+        E[2 * k + 1] = zik - zim;
+        O[2 * k] = fmaf(cs, dr, -sn * si);
+        O[2 * k + 1] = fmaf(sn, dr, cs * si);
+      }
+    }
+  }
+  __syncthreads();
+  if (warp < kCWarps) {
+    const int g = lane >> 2, cq = lane & 3;
+    const int mi = lane >> 3;
+    const float* Er = eo + g * 128;
+    const float* Or = eo + 1024 + g * 128;
+    uint32_t eh[8][2], el[8][2], oh[8][2], ol[8][2];
+#pragma unroll
+    for (int ks = 0; ks < 8; ++ks) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int j0 = 16 * ks + 2 * cq + 8 * e;
+        __half h0 = __float2half_rn(Er[j0]), h1 = __float2half_rn(Er[j0 + 1]);
+        __half l0 = __float2half_rn(Er[j0] - __half2float(h0)), l1 = __float2half_rn(Er[j0 + 1] - __half2float(h1));
+        eh[ks][e] = h2_bits(__halves2half2(h0, h1));
+        el[ks][e] = h2_bits(__halves2half2(l0, l1));
+        h0 = __float2half_rn(Or[j0]);
+        h1 = __float2half_rn(Or[j0 + 1]);
+        l0 = __float2half_rn(Or[j0] - __half2float(h0));
+        l1 = __float2half_rn(Or[j0 + 1] - __half2float(h1));
+        oh[ks][e] = h2_bits(__halves2half2(h0, h1));
+        ol[ks][e] = h2_bits(__halves2half2(l0, l1));
+      }
+    }
+#pragma unroll
+    for (int tt = 0; tt < 2; ++tt) {
+      const int mt = 2 * warp + tt;  // samples m = 16 mt .. 16 mt + 15 of each half
+      float xe[4] = {0.f, 0.f, 0.f, 0.f}, xo[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ks = 0; ks < 8; ++ks) {
+        // A = F128^T (rows m, columns j): transposed 8x8 blocks of F128 rows j
+        const int jrow = 16 * ks + ((mi >> 1) << 3) + (lane & 7);
+        const int mcol = 16 * mt + ((mi & 1) << 3);
+        uint32_t a0, a1, a2, a3;
+        ldmatrix_x4_trans(a0, a1, a2, a3, rot_addr(srot, 0, jrow, mcol));
+        mma_16816(xe, a0, a1, a2, a3, eh[ks][0], eh[ks][1]);
+        mma_16816(xe, a0, a1, a2, a3, el[ks][0], el[ks][1]);
+        mma_16816(xo, a0, a1, a2, a3, oh[ks][0], oh[ks][1]);
+        mma_16816(xo, a0, a1, a2, a3, ol[ks][0], ol[ks][1]);
+        ldmatrix_x4_trans(a0, a1, a2, a3, rot_addr(srot, 1, jrow, mcol));
+        mma_16816(xe, a0, a1, a2, a3, eh[ks][0], eh[ks][1]);
+        mma_16816(xo, a0, a1, a2, a3, oh[ks][0], oh[ks][1]);
+      }
+      const int m0 = 16 * mt + g;
+      if (2 * cq < heads) {
+        xb[(2 * cq) * 256 + 2 * m0] = xe[0];
+        xb[(2 * cq) * 256 + 2 * m0 + 1] = xo[0];
+        xb[(2 * cq) * 256 + 2 * (m0 + 8)] = xe[2];
+        xb[(2 * cq) * 256 + 2 * (m0 + 8) + 1] = xo[2];
+      }
+      if (2 * cq + 1 < heads) {
+        xb[(2 * cq + 1) * 256 + 2 * m0] = xe[1];
+        xb[(2 * cq + 1) * 256 + 2 * m0 + 1] = xo[1];
+        xb[(2 * cq + 1) * 256 + 2 * (m0 + 8)] = xe[3];
+        xb[(2 * cq + 1) * 256 + 2 * (m0 + 8) + 1] = xo[3];
+      }
     }
   }
 }
@@ -518,11 +589,10 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
       atomicOr(&g_attend_err, kErrTimeoutLoad);
       ok = false;
     }
-    if constexpr (C::kMmaRot) {
+    if constexpr (C::kMmaRot && D == 128) {
       rotate_query_mma(qs, heads, ksg, srot, qt, warp, lane);
-    } else if constexpr (INT4) {
-      if (warp == 0) rotate_query<D>(qs, heads, ksg, kch, qt, lane);
-      for (int i = threadIdx.x; i < (kHT - heads) * D; i += kCWarps * 32) qt[heads * D + i] = 0.0f;
+    } else if constexpr (C::kMmaRot) {
+      rotate_query_eo(qs, heads, ksg, kch, srot, reinterpret_cast<float*>(qf), qt, warp, lane);
     } else {
       for (int i = threadIdx.x; i < kHT * D / 2; i += kCWarps * 32) {
         const int h = (2 * i) / D;
@@ -531,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
       }
     }
     consumer_sync();
-    if constexpr (C::kMmaRot) {
+    if constexpr (C::kMmaRot && D == 128) {
       // the rotation matrix is consumed: a cluster leader (the only CTA that can run the
       // final merge) prefetches the V plan's un-rotation matrix into the same buffer
       if (threadIdx.x == 0 && cg::this_cluster().block_rank() == 0) {
@@ -885,7 +955,7 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
   if (crank != 0) return;
   // (D = 128 int4) the leader's un-rotation matrix prefetch must land before the CTA may exit
   bool rot_ok = true;
-  if constexpr (C::kMmaRot) rot_ok = mbar_wait_bounded(ubar, 0);
+  if constexpr (C::kMmaRot && D == 128) rot_ok = mbar_wait_bounded(ubar, 0);
   // the producer warp reads staged constants below: observe their barrier too
   if (warp == kCWarps && !mbar_wait_bounded(cbar, 0)) atomicOr(&g_attend_err, kErrTimeoutLoad);
 
@@ -917,16 +987,12 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
   uint16_t* ob = J.out + ((size_t)b * p.Hq + hq0) * D;
   if constexpr (C::kMmaRot) {
     if (!rot_ok && threadIdx.x == 0) atomicOr(&g_attend_err, kErrTimeoutLoad);
-    if (warp < kCWarps) unrotate_out_mma(om, heads, mrg + kHT, srot, xb, warp, lane);
-    __syncthreads();
-    for (int i = threadIdx.x; i < heads * D / 2; i += kThreads) {
-      const int j = i % (D / 2);
-      reinterpret_cast<uint32_t*>(ob)[i] = pack_half2(xb[2 * i], xb[2 * i + 1]) ^ vsg[j];
+    if constexpr (D == 128) {
+      if (warp < kCWarps) unrotate_out_mma(om, heads, mrg + kHT, srot, xb, warp, lane);
+    } else {
+      unrotate_out_eo(om, heads, mrg + kHT, vch, srot, reinterpret_cast<float*>(qf), xb, warp, lane);
     }
-  } else if constexpr (INT4) {
-    if (warp == 0) unrotate_out<D>(om, heads, vch, mrg + kHT, xb, lane);
     __syncthreads();
-    // fp16 with the V sign folded in as an XOR on the sign bits
     for (int i = threadIdx.x; i < heads * D / 2; i += kThreads) {
       const int j = i % (D / 2);
       reinterpret_cast<uint32_t*>(ob)[i] = pack_half2(xb[2 * i], xb[2 * i + 1]) ^ vsg[j];
@@ -1104,6 +1170,15 @@ kvq_status make_job(const AttendJobHost& h, int B, int Hkv, int T_cap, AttnJob* 
     if (st != KVQ_OK) return st;
     j->ksmap = j->kmap;
     j->vsmap = j->vmap;
+  }
+  if constexpr (INT4 && D == 256) {
+    const uint64_t rd[2] = {128u, 256u};
+    const uint64_t rs[1] = {256u};
+    const uint32_t rb[2] = {64u, 128u};
+    st = encode_tiled(&j->rqmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h.pk->rq_dev, rd, rs, rb,
+                      CU_TENSOR_MAP_SWIZZLE_128B, "F128");
+    if (st != KVQ_OK) return st;
+    j->rumap = j->rqmap;
   }
   if constexpr (INT4 && D == 128) {
     const uint64_t rd[2] = {128u, 256u};
