@@ -53,7 +53,6 @@ namespace {
 
 constexpr int kCWarps = 4;                 // consumer warps
 constexpr int kThreads = (kCWarps + 1) * 32;
-constexpr int kTileT = 16 * kCWarps;       // tokens per stage
 constexpr int kHT = 8;                     // query heads per CTA (mma N)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kMaxSplitsCfg = 256;          // upper bound on splits per unit
@@ -67,12 +66,16 @@ template <int D, bool INT4>
 struct Cfg {
   static constexpr int NG = D / 32;                        // scale groups (int4)
   static constexpr int kRowBytes = INT4 ? D / 2 : 2 * D;   // bytes per token row of K (and V)
-  static constexpr int kKBytes = kTileT * kRowBytes;
-  static constexpr int kSBytes = INT4 ? kTileT * NG * 2 : 0;
+  // each consumer warp takes kSub subtiles of 16 tokens per stage (two independent
+  // instruction streams for the int4 path, whose per-token work is latency-bound)
+  static constexpr int kSub = INT4 ? 2 : 1;
+  static constexpr int kTile = 16 * kCWarps * kSub;        // tokens per stage
+  static constexpr int kKBytes = kTile * kRowBytes;
+  static constexpr int kSBytes = INT4 ? kTile * NG * 2 : 0;
   static constexpr int kStageBytes = 2 * kKBytes + 2 * kSBytes;
-  static constexpr int kStages = INT4 ? 4 : (D == 128 ? 3 : 2);
-  static constexpr int kScaleBox = (kTileT * NG) < 256 ? kTileT * NG : 256;  // halves per scale TMA box
-  static constexpr int kScaleLoads = INT4 ? (kTileT * NG) / kScaleBox : 0;
+  static constexpr int kStages = INT4 ? 2 : (D == 128 ? 3 : 2);
+  static constexpr int kScaleBox = (kTile * NG) < 256 ? kTile * NG : 256;  // halves per scale TMA box
+  static constexpr int kScaleLoads = INT4 ? (kTile * NG) / kScaleBox : 0;
   // warp-merge scratch (reuses the stage ring): per warp m[8], l[8], o[8][D]
   static constexpr int kWarpState = (2 * kHT + kHT * D) * 4;
   static constexpr int kRing = kStages * kStageBytes;
@@ -103,7 +106,7 @@ struct Cfg {
 
 struct AttnParams {
   const int32_t* seq_lens;
-  int T_len, B, Hq, Hkv, T_cap, G, HT, S, tps;  // tps = tokens per split (multiple of kTileT)
+  int T_len, B, Hq, Hkv, T_cap, G, HT, S, tps;  // tps = tokens per split (multiple of the stage)
   float sl2;                                   // softmax scale * log2(e)
   float* part;                                 // [units][S][2*8 + 8*D]
   int* cnt;                                    // [units]
@@ -466,7 +469,7 @@ __device__ __forceinline__ void unrotate_out_eo(const float* om, int heads, cons
 }
 
 template <int D, bool INT4, int MAXJ>
-__global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
+__global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
     attend_kernel(const __grid_constant__ AttnJobs<MAXJ> jt, const __grid_constant__ AttnParams p) {
   using C = Cfg<D, INT4>;
   constexpr int NG = C::NG;
@@ -505,7 +508,7 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
   if (p.seq_lens) T_b = min(max(__ldg(p.seq_lens + b), 0), p.T_cap);
   const int t_begin = split * p.tps;
   const int t_end = min(t_begin + p.tps, T_b);
-  const int ntiles = t_end > t_begin ? (t_end - t_begin + kTileT - 1) / kTileT : 0;
+  const int ntiles = t_end > t_begin ? (t_end - t_begin + C::kTile - 1) / C::kTile : 0;
   const int row0 = bk * p.T_cap;  // first cache row of this (b, kv head)
 
   if (threadIdx.x == 0) {
@@ -561,7 +564,7 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
           }
         }
         uint8_t* st = ring + s * C::kStageBytes;
-        const int t0 = t_begin + i * kTileT;
+        const int t0 = t_begin + i * C::kTile;
         mbar_arrive_expect_tx(&full[s], C::kStageBytes);
         const uint64_t pol = l2_evict_first_policy();
         if constexpr (INT4) {
@@ -576,8 +579,8 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
         } else {
 #pragma unroll
           for (int j = 0; j < D / 64; ++j) {
-            tma_load_2d_hint(st + j * kTileT * 128, &J.kmap, &full[s], 64 * j, row0 + t0, pol);
-            tma_load_2d_hint(st + C::kKBytes + j * kTileT * 128, &J.vmap, &full[s], 64 * j, row0 + t0, pol);
+            tma_load_2d_hint(st + j * C::kTile * 128, &J.kmap, &full[s], 64 * j, row0 + t0, pol);
+            tma_load_2d_hint(st + C::kKBytes + j * C::kTile * 128, &J.vmap, &full[s], 64 * j, row0 + t0, pol);
           }
         }
       }
@@ -654,87 +657,105 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
         break;
       }
       const uint8_t* st = ring + s * C::kStageBytes;
-      const int tw0 = t_begin + i * kTileT + warp * 16;  // first token of this warp
-      const bool partial = tw0 + 16 > t_end;
-      const int r0 = warp * 16;                            // stage row of that token
-
-      // ---- scores S^T[token][head] (C layout: rows g, g+8; cols 2c, 2c+1)
-      float sc[4] = {0.f, 0.f, 0.f, 0.f};
-      if constexpr (INT4) {
-        const uint8_t* kt = st;
-        const uint8_t* ks = st + 2 * C::kKBytes;
-        // scales of tokens r0+g and r0+g+8
-        float skA[NG], skB[NG];
-        {
-          const uint16_t* sa = reinterpret_cast<const uint16_t*>(ks) + (r0 + g) * NG;
-          const uint16_t* sb = reinterpret_cast<const uint16_t*>(ks) + (r0 + g + 8) * NG;
+      // this warp's SUB subtiles of 16 tokens: stage rows (SUB warp + sb) 16 .. + 15
+      constexpr int SUB = C::kSub;
+      int tw0[SUB];
+      bool partial[SUB];
+      float sc[SUB][4];
 #pragma unroll
-          for (int q2 = 0; q2 < NG / 2; ++q2) {
-            const float2 fa = __half22float2(bits_h2(reinterpret_cast<const uint32_t*>(sa)[q2]));
-            const float2 fb = __half22float2(bits_h2(reinterpret_cast<const uint32_t*>(sb)[q2]));
-            skA[2 * q2] = fa.x;
-            skA[2 * q2 + 1] = fa.y;
-            skB[2 * q2] = fb.x;
-            skB[2 * q2 + 1] = fb.y;
+      for (int sb = 0; sb < SUB; ++sb) {
+        const int r0s = (warp * SUB + sb) * 16;
+        tw0[sb] = t_begin + i * C::kTile + r0s;
+        partial[sb] = tw0[sb] + 16 > t_end;
+        float scs[4] = {0.f, 0.f, 0.f, 0.f};
+        // ---- scores S^T[token][head] (C layout: rows g, g+8; cols 2c, 2c+1)
+        if constexpr (INT4) {
+          const uint8_t* kt = st;
+          const uint8_t* ks = st + 2 * C::kKBytes;
+          // scales of tokens r0+g and r0+g+8
+          float skA[NG], skB[NG];
+          {
+            const uint16_t* sa = reinterpret_cast<const uint16_t*>(ks) + (r0s + g) * NG;
+            const uint16_t* sb = reinterpret_cast<const uint16_t*>(ks) + (r0s + g + 8) * NG;
+  #pragma unroll
+            for (int q2 = 0; q2 < NG / 2; ++q2) {
+              const float2 fa = __half22float2(bits_h2(reinterpret_cast<const uint32_t*>(sa)[q2]));
+              const float2 fb = __half22float2(bits_h2(reinterpret_cast<const uint32_t*>(sb)[q2]));
+              skA[2 * q2] = fa.x;
+              skA[2 * q2 + 1] = fa.y;
+              skB[2 * q2] = fb.x;
+              skB[2 * q2 + 1] = fb.y;
+            }
+          }
+  #pragma unroll
+          for (int gp = 0; gp < NG / 2; ++gp) {  // two groups per ldmatrix.x4
+            const int mi = lane >> 3;
+            const int row = r0s + ((mi & 1) << 3) + (lane & 7);
+            const int chunk = 2 * gp + (mi >> 1);
+            const int pch = (D == 128) ? (chunk ^ ((row >> 1) & 3)) : (chunk ^ (row & 7));
+            uint32_t w0, w1, w2, w3;  // (tok g, G0) (tok g+8, G0) (tok g, G1) (tok g+8, G1)
+            ldmatrix_x4(w0, w1, w2, w3, smem_u32(kt + row * C::kRowBytes + pch * 16));
+            uint32_t hA0[4], hB0[4], hA1[4], hB1[4];
+            nib8_to_h2(w0, hA0);
+            nib8_to_h2(w1, hB0);
+            nib8_to_h2(w2, hA1);
+            nib8_to_h2(w3, hB1);
+            const int G0 = 2 * gp, G1 = 2 * gp + 1;
+            float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint4 f0 = qf[(2 * G0) * 32 + lane], f1 = qf[(2 * G0 + 1) * 32 + lane];
+            const uint4 f2 = qf[(2 * G1) * 32 + lane], f3 = qf[(2 * G1 + 1) * 32 + lane];
+            mma_16816(a0, hA0[0], hB0[0], hA0[1], hB0[1], f0.x, f0.y);
+            mma_16816(a0, hA0[0], hB0[0], hA0[1], hB0[1], f0.z, f0.w);
+            mma_16816(a0, hA0[2], hB0[2], hA0[3], hB0[3], f1.x, f1.y);
+            mma_16816(a0, hA0[2], hB0[2], hA0[3], hB0[3], f1.z, f1.w);
+            mma_16816(a1, hA1[0], hB1[0], hA1[1], hB1[1], f2.x, f2.y);
+            mma_16816(a1, hA1[0], hB1[0], hA1[1], hB1[1], f2.z, f2.w);
+            mma_16816(a1, hA1[2], hB1[2], hA1[3], hB1[3], f3.x, f3.y);
+            mma_16816(a1, hA1[2], hB1[2], hA1[3], hB1[3], f3.z, f3.w);
+            scs[0] = fmaf(skA[G0], a0[0], fmaf(skA[G1], a1[0], scs[0]));
+            scs[1] = fmaf(skA[G0], a0[1], fmaf(skA[G1], a1[1], scs[1]));
+            scs[2] = fmaf(skB[G0], a0[2], fmaf(skB[G1], a1[2], scs[2]));
+            scs[3] = fmaf(skB[G0], a0[3], fmaf(skB[G1], a1[3], scs[3]));
+          }
+        } else {
+          const uint8_t* kt = st;
+  #pragma unroll
+          for (int ks = 0; ks < D / 16; ++ks) {
+            // A = K rows (tokens) x 16 channels: matrices (tok 0-7, ch 0-7) (tok 8-15, ch 0-7)
+            // (tok 0-7, ch 8-15) (tok 8-15, ch 8-15)
+            const int mi = lane >> 3;
+            const int row = r0s + ((mi & 1) << 3) + (lane & 7);
+            const int cc = 2 * ks + (mi >> 1);  // 16-byte chunk (8 channels)
+            const int box = cc >> 3, ch = cc & 7;
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4(a0, a1, a2, a3, smem_u32(kt + box * C::kTile * 128 + row * 128 + ((ch ^ (row & 7)) << 4)));
+            const uint4 f = qf[ks * 32 + lane];
+            mma_16816(scs, a0, a1, a2, a3, f.x, f.y);
           }
         }
+
 #pragma unroll
-        for (int gp = 0; gp < NG / 2; ++gp) {  // two groups per ldmatrix.x4
-          const int mi = lane >> 3;
-          const int row = r0 + ((mi & 1) << 3) + (lane & 7);
-          const int chunk = 2 * gp + (mi >> 1);
-          const int pch = (D == 128) ? (chunk ^ ((row >> 1) & 3)) : (chunk ^ (row & 7));
-          uint32_t w0, w1, w2, w3;  // (tok g, G0) (tok g+8, G0) (tok g, G1) (tok g+8, G1)
-          ldmatrix_x4(w0, w1, w2, w3, smem_u32(kt + row * C::kRowBytes + pch * 16));
-          uint32_t hA0[4], hB0[4], hA1[4], hB1[4];
-          nib8_to_h2(w0, hA0);
-          nib8_to_h2(w1, hB0);
-          nib8_to_h2(w2, hA1);
-          nib8_to_h2(w3, hB1);
-          const int G0 = 2 * gp, G1 = 2 * gp + 1;
-          float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
-          const uint4 f0 = qf[(2 * G0) * 32 + lane], f1 = qf[(2 * G0 + 1) * 32 + lane];
-          const uint4 f2 = qf[(2 * G1) * 32 + lane], f3 = qf[(2 * G1 + 1) * 32 + lane];
-          mma_16816(a0, hA0[0], hB0[0], hA0[1], hB0[1], f0.x, f0.y);
-          mma_16816(a0, hA0[0], hB0[0], hA0[1], hB0[1], f0.z, f0.w);
-          mma_16816(a0, hA0[2], hB0[2], hA0[3], hB0[3], f1.x, f1.y);
-          mma_16816(a0, hA0[2], hB0[2], hA0[3], hB0[3], f1.z, f1.w);
-          mma_16816(a1, hA1[0], hB1[0], hA1[1], hB1[1], f2.x, f2.y);
-          mma_16816(a1, hA1[0], hB1[0], hA1[1], hB1[1], f2.z, f2.w);
-          mma_16816(a1, hA1[2], hB1[2], hA1[3], hB1[3], f3.x, f3.y);
-          mma_16816(a1, hA1[2], hB1[2], hA1[3], hB1[3], f3.z, f3.w);
-          sc[0] = fmaf(skA[G0], a0[0], fmaf(skA[G1], a1[0], sc[0]));
-          sc[1] = fmaf(skA[G0], a0[1], fmaf(skA[G1], a1[1], sc[1]));
-          sc[2] = fmaf(skB[G0], a0[2], fmaf(skB[G1], a1[2], sc[2]));
-          sc[3] = fmaf(skB[G0], a0[3], fmaf(skB[G1], a1[3], sc[3]));
-        }
-      } else {
-        const uint8_t* kt = st;
-#pragma unroll
-        for (int ks = 0; ks < D / 16; ++ks) {
-          // A = K rows (tokens) x 16 channels: matrices (tok 0-7, ch 0-7) (tok 8-15, ch 0-7)
-          // (tok 0-7, ch 8-15) (tok 8-15, ch 8-15)
-          const int mi = lane >> 3;
-          const int row = r0 + ((mi & 1) << 3) + (lane & 7);
-          const int cc = 2 * ks + (mi >> 1);  // 16-byte chunk (8 channels)
-          const int box = cc >> 3, ch = cc & 7;
-          uint32_t a0, a1, a2, a3;
-          ldmatrix_x4(a0, a1, a2, a3, smem_u32(kt + box * kTileT * 128 + row * 128 + ((ch ^ (row & 7)) << 4)));
-          const uint4 f = qf[ks * 32 + lane];
-          mma_16816(sc, a0, a1, a2, a3, f.x, f.y);
-        }
+        for (int e = 0; e < 4; ++e) sc[sb][e] = scs[e];
       }
       // base-2 scores with masking of tokens outside [t_begin, t_end)
-      float s2[4];
+      float s2[SUB][4];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) s2[e] = sc[e] * p.sl2;
-      if (partial) {
-        const bool va = tw0 + g < t_end, vb = tw0 + g + 8 < t_end;
-        if (!va) s2[0] = s2[1] = -INFINITY;
-        if (!vb) s2[2] = s2[3] = -INFINITY;
+      for (int sb = 0; sb < SUB; ++sb) {
+#pragma unroll
+        for (int e = 0; e < 4; ++e) s2[sb][e] = sc[sb][e] * p.sl2;
+        if (partial[sb]) {
+          const bool va = tw0[sb] + g < t_end, vb = tw0[sb] + g + 8 < t_end;
+          if (!va) s2[sb][0] = s2[sb][1] = -INFINITY;
+          if (!vb) s2[sb][2] = s2[sb][3] = -INFINITY;
+        }
       }
-      // ---- online softmax (exact running max per head column)
-      float mx0 = fmaxf(s2[0], s2[2]), mx1 = fmaxf(s2[1], s2[3]);
+      // ---- online softmax over the warp's SUB x 16 tokens (exact running max per head column)
+      float mx0 = fmaxf(s2[0][0], s2[0][2]), mx1 = fmaxf(s2[0][1], s2[0][3]);
+#pragma unroll
+      for (int sb = 1; sb < SUB; ++sb) {
+        mx0 = fmaxf(mx0, fmaxf(s2[sb][0], s2[sb][2]));
+        mx1 = fmaxf(mx1, fmaxf(s2[sb][1], s2[sb][3]));
+      }
 #pragma unroll
       for (int off = 4; off < 32; off <<= 1) {
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
@@ -759,79 +780,83 @@ __global__ void __launch_bounds__(kThreads, INT4 ? 2 : (D == 128 ? 2 : 1))
       }
       const float ms0 = m_run[0] == -INFINITY ? 0.0f : m_run[0];
       const float ms1 = m_run[1] == -INFINITY ? 0.0f : m_run[1];
-      const float p0 = fast_exp2(s2[0] - ms0), p1 = fast_exp2(s2[1] - ms1);
-      const float p2 = fast_exp2(s2[2] - ms0), p3 = fast_exp2(s2[3] - ms1);
-      l_run[0] += p0 + p2;
-      l_run[1] += p1 + p3;
-      // ---- transpose P into the PV B operand: b0 = (tok 2c, 2c+1; head g), b1 = (tok 2c+8, 2c+9; head g)
-      const uint32_t X0 = pack_half2(p0, p2);  // (tok g, tok g+8) of head 2c
-      const uint32_t X1 = pack_half2(p1, p3);  // of head 2c+1
-      const uint32_t ya0 = __shfl_sync(0xffffffffu, X0, lane_a), ya1 = __shfl_sync(0xffffffffu, X1, lane_a);
-      const uint32_t yb0 = __shfl_sync(0xffffffffu, X0, lane_b), yb1 = __shfl_sync(0xffffffffu, X1, lane_b);
-      const uint32_t ya = (g & 1) ? ya1 : ya0;  // (P[2c][g], P[2c+8][g])
-      const uint32_t yb = (g & 1) ? yb1 : yb0;  // (P[2c+1][g], P[2c+9][g])
-      const uint32_t pb0 = prmt(ya, yb, 0x5410u);  // (P[2c][g], P[2c+1][g])
-      const uint32_t pb1 = prmt(ya, yb, 0x7632u);  // (P[2c+8][g], P[2c+9][g])
-
-      // ---- PV: O^T[channel][head] += V^T[channel][token] P[token][head]
-      if constexpr (INT4) {
-        const uint8_t* vt = st + C::kKBytes;
-        const uint16_t* vs = reinterpret_cast<const uint16_t*>(st + 2 * C::kKBytes + C::kSBytes);
-        // V scales of tokens 2c, 2c+1, 2c+8, 2c+9 (rows of this warp), paired per group
-        uint32_t sw[4][NG / 2];
-        {
-          const int toks[4] = {2 * c, 2 * c + 1, 2 * c + 8, 2 * c + 9};
+      // ---- P, transposed into the PV B operand: b0 = (tok 2c, 2c+1; head g), b1 = (tok 2c+8, 2c+9; head g)
+      uint32_t pb0[SUB], pb1[SUB];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t* sp = reinterpret_cast<const uint32_t*>(vs + (r0 + toks[e]) * NG);
-            const bool valid = !partial || (tw0 + toks[e] < t_end);
+      for (int sb = 0; sb < SUB; ++sb) {
+        const float p0 = fast_exp2(s2[sb][0] - ms0), p1 = fast_exp2(s2[sb][1] - ms1);
+        const float p2 = fast_exp2(s2[sb][2] - ms0), p3 = fast_exp2(s2[sb][3] - ms1);
+        l_run[0] += p0 + p2;
+        l_run[1] += p1 + p3;
+        const uint32_t X0 = pack_half2(p0, p2);  // (tok g, tok g+8) of head 2c
+        const uint32_t X1 = pack_half2(p1, p3);  // of head 2c+1
+        const uint32_t ya0 = __shfl_sync(0xffffffffu, X0, lane_a), ya1 = __shfl_sync(0xffffffffu, X1, lane_a);
+        const uint32_t yb0 = __shfl_sync(0xffffffffu, X0, lane_b), yb1 = __shfl_sync(0xffffffffu, X1, lane_b);
+        const uint32_t ya = (g & 1) ? ya1 : ya0;  // (P[2c][g], P[2c+8][g])
+        const uint32_t yb = (g & 1) ? yb1 : yb0;  // (P[2c+1][g], P[2c+9][g])
+        pb0[sb] = prmt(ya, yb, 0x5410u);           // (P[2c][g], P[2c+1][g])
+        pb1[sb] = prmt(ya, yb, 0x7632u);           // (P[2c+8][g], P[2c+9][g])
+      }
 #pragma unroll
-            for (int q2 = 0; q2 < NG / 2; ++q2) sw[e][q2] = valid ? sp[q2] : 0u;
+      for (int sb = 0; sb < SUB; ++sb) {
+        const int r0s = (warp * SUB + sb) * 16;
+        // ---- PV: O^T[channel][head] += V^T[channel][token] P[token][head]
+        if constexpr (INT4) {
+          const uint8_t* vt = st + C::kKBytes;
+          const uint16_t* vs = reinterpret_cast<const uint16_t*>(st + 2 * C::kKBytes + C::kSBytes);
+          // V scales of tokens 2c, 2c+1, 2c+8, 2c+9 (rows of this warp), paired per group
+          uint32_t sw[4][NG / 2];
+          {
+            const int toks[4] = {2 * c, 2 * c + 1, 2 * c + 8, 2 * c + 9};
+  #pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t* sp = reinterpret_cast<const uint32_t*>(vs + (r0s + toks[e]) * NG);
+              const bool valid = !partial[sb] || (tw0[sb] + toks[e] < t_end);
+  #pragma unroll
+              for (int q2 = 0; q2 < NG / 2; ++q2) sw[e][q2] = valid ? sp[q2] : 0u;
+            }
           }
-        }
-#pragma unroll
-        for (int gp = 0; gp < NG / 2; ++gp) {
-          const int mi = lane >> 3;
-          const int row = r0 + ((mi & 1) << 3) + (lane & 7);
-          const int chunk = 2 * gp + (mi >> 1);
-          const int pch = (D == 128) ? (chunk ^ ((row >> 1) & 3)) : (chunk ^ (row & 7));
-          uint32_t w0, w1, w2, w3;  // (tok 0-7, G0) (tok 8-15, G0) (tok 0-7, G1) (tok 8-15, G1), transposed
-          ldmatrix_x4_trans(w0, w1, w2, w3, smem_u32(vt + row * C::kRowBytes + pch * 16));
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const int G = 2 * gp + h;
-            // V-scale pairs for this group: (s[2c], s[2c+1]) and (s[2c+8], s[2c+9])
-            const uint32_t sel = (G & 1) ? 0x7632u : 0x5410u;
-            const uint32_t s01 = prmt(sw[0][G >> 1], sw[1][G >> 1], sel);
-            const uint32_t s89 = prmt(sw[2][G >> 1], sw[3][G >> 1], sel);
-            const uint32_t b0 = h2_bits(__hmul2(bits_h2(pb0), bits_h2(s01)));
-            const uint32_t b1 = h2_bits(__hmul2(bits_h2(pb1), bits_h2(s89)));
-            uint32_t lo[4], hi[4];
-            nib8_to_h2(h ? w2 : w0, lo);  // tokens 2c, 2c+1: channels 4g .. 4g+3 of group G
-            nib8_to_h2(h ? w3 : w1, hi);  // tokens 2c+8, 2c+9
-            // M-tile X: rows g -> ch 4g, g+8 -> ch 4g+1 ; M-tile Y: ch 4g+2, 4g+3
-            mma_16816(o_acc[2 * G], lo[0], lo[1], hi[0], hi[1], b0, b1);
-            mma_16816(o_acc[2 * G + 1], lo[2], lo[3], hi[2], hi[3], b0, b1);
+  #pragma unroll
+          for (int gp = 0; gp < NG / 2; ++gp) {
+            const int mi = lane >> 3;
+            const int row = r0s + ((mi & 1) << 3) + (lane & 7);
+            const int chunk = 2 * gp + (mi >> 1);
+            const int pch = (D == 128) ? (chunk ^ ((row >> 1) & 3)) : (chunk ^ (row & 7));
+            uint32_t w0, w1, w2, w3;  // (tok 0-7, G0) (tok 8-15, G0) (tok 0-7, G1) (tok 8-15, G1), transposed
+            ldmatrix_x4_trans(w0, w1, w2, w3, smem_u32(vt + row * C::kRowBytes + pch * 16));
+  #pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int G = 2 * gp + h;
+              // V-scale pairs for this group: (s[2c], s[2c+1]) and (s[2c+8], s[2c+9])
+              const uint32_t sel = (G & 1) ? 0x7632u : 0x5410u;
+              const uint32_t s01 = prmt(sw[0][G >> 1], sw[1][G >> 1], sel);
+              const uint32_t s89 = prmt(sw[2][G >> 1], sw[3][G >> 1], sel);
+              const uint32_t b0 = h2_bits(__hmul2(bits_h2(pb0[sb]), bits_h2(s01)));
+              const uint32_t b1 = h2_bits(__hmul2(bits_h2(pb1[sb]), bits_h2(s89)));
+              uint32_t lo[4], hi[4];
+              nib8_to_h2(h ? w2 : w0, lo);  // tokens 2c, 2c+1: channels 4g .. 4g+3 of group G
+              nib8_to_h2(h ? w3 : w1, hi);  // tokens 2c+8, 2c+9
+              // M-tile X: rows g -> ch 4g, g+8 -> ch 4g+1 ; M-tile Y: ch 4g+2, 4g+3
+              mma_16816(o_acc[2 * G], lo[0], lo[1], hi[0], hi[1], b0, b1);
+              mma_16816(o_acc[2 * G + 1], lo[2], lo[3], hi[2], hi[3], b0, b1);
+            }
           }
-        }
-      } else {
-        const uint8_t* vt = st + C::kKBytes;
-        uint32_t b0 = pb0, b1 = pb1;
-        if (partial) {
-          // masked tokens have P = 0 already (scores -inf); V rows there are finite or zero-filled
-        }
-#pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
-          // A = V^T (16 channels x 16 tokens): ldmatrix.trans of (tok 0-7, ch 0-7) (tok 0-7, ch 8-15)
-          // (tok 8-15, ch 0-7) (tok 8-15, ch 8-15)
-          const int mi = lane >> 3;
-          const int row = r0 + ((mi >> 1) << 3) + (lane & 7);
-          const int cc = 2 * mt + (mi & 1);
-          const int box = cc >> 3, ch = cc & 7;
-          uint32_t a0, a1, a2, a3;
-          ldmatrix_x4_trans(a0, a1, a2, a3,
-                            smem_u32(vt + box * kTileT * 128 + row * 128 + ((ch ^ (row & 7)) << 4)));
-          mma_16816(o_acc[mt], a0, a1, a2, a3, b0, b1);
+        } else {
+          const uint8_t* vt = st + C::kKBytes;
+          uint32_t b0 = pb0[sb], b1 = pb1[sb];
+  #pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            // A = V^T (16 channels x 16 tokens): ldmatrix.trans of (tok 0-7, ch 0-7) (tok 0-7, ch 8-15)
+            // (tok 8-15, ch 0-7) (tok 8-15, ch 8-15)
+            const int mi = lane >> 3;
+            const int row = r0s + ((mi >> 1) << 3) + (lane & 7);
+            const int cc = 2 * mt + (mi & 1);
+            const int box = cc >> 3, ch = cc & 7;
+            uint32_t a0, a1, a2, a3;
+            ldmatrix_x4_trans(a0, a1, a2, a3,
+                              smem_u32(vt + box * C::kTile * 128 + row * 128 + ((ch ^ (row & 7)) << 4)));
+            mma_16816(o_acc[mt], a0, a1, a2, a3, b0, b1);
+          }
         }
       }
       __syncwarp();
@@ -1058,21 +1083,22 @@ const Occupancy& occupancy() {
   return occ;
 }
 
-// Split of the token range. When splits of ~4 stages cannot fill the GPU (few
-// units, short context) the kernel is latency-bound: take ~4 stages per split,
+// Split of the token range. When splits of ~256 tokens cannot fill the GPU (few
+// units, short context) the kernel is latency-bound: take ~256 tokens per split,
 // which keeps the final merge short. Otherwise (throughput regime) take the split
 // count with the least estimated time (rounds of resident CTAs times the stages
-// per split plus a fixed per-CTA cost). Every split keeps >= kMinTilesPerSplit
-// stages and S <= kMaxSplits. The splits of a unit form clusters of C CTAs
+// per split plus a fixed per-CTA cost). Every split keeps >= kMinTokensPerSplit
+// tokens and S <= kMaxSplits. The splits of a unit form clusters of C CTAs
 // (C = the largest divisor of S up to 8 in the latency regime, up to 4 in the
 // throughput regime, where large clusters constrain scheduling more than they
 // save) that merge through distributed shared memory; when S > C the S / C
 // cluster partials (<= kMaxMerge) merge through the workspace.
-constexpr int kMinTilesPerSplit = 2;
+// (all in tokens; a stage is 64 or 128 tokens depending on the kernel)
+constexpr int kMinTokensPerSplit = 128;
 constexpr int kMaxSplits = kMaxSplitsCfg;
-constexpr int kLatencyTilesPerSplit = 4;
-constexpr int kFixedTiles = 12;  // per-CTA fixed cost (query rotation, merges) in stage-times
-constexpr int kMergeTiles = 6;   // workspace merge of cluster partials, in stage-times
+constexpr int kLatencyTokensPerSplit = 256;
+constexpr int kFixedTokens = 768;  // per-CTA fixed cost (query rotation, merges) in token-times
+constexpr int kMergeTokens = 384;  // workspace merge of cluster partials, in token-times
 
 int cluster_for(int S, int cmax) {
   for (int c = std::min(S, cmax); c > 1; --c)
@@ -1080,13 +1106,16 @@ int cluster_for(int S, int cmax) {
   return 1;
 }
 
-SplitPlan choose_split(int B, int Hq, int Hkv, int T, const Occupancy& occ) {
+SplitPlan choose_split(int B, int Hq, int Hkv, int T, const Occupancy& occ, int tile) {
   SplitPlan sp{};
   const int G = Hq / Hkv;
   sp.HT = (G + kHT - 1) / kHT;
   const long units = (long)B * Hkv * sp.HT;
-  const int ntile = T > 0 ? (T + kTileT - 1) / kTileT : 1;
+  const int ntile = T > 0 ? (T + tile - 1) / tile : 1;
   const long slots = occ.cap[0];
+  const int kMinTilesPerSplit = std::max(1, kMinTokensPerSplit / tile);
+  const int kLatencyTilesPerSplit = std::max(1, kLatencyTokensPerSplit / tile);
+  const int kFixedTiles = kFixedTokens / tile, kMergeTiles = kMergeTokens / tile;
   int s_cap = std::max(1, ntile / kMinTilesPerSplit);
   s_cap = std::min(s_cap, kMaxSplits);
   const bool latency = units * std::max(1, ntile / kLatencyTilesPerSplit) < slots;
@@ -1118,7 +1147,7 @@ SplitPlan choose_split(int B, int Hq, int Hkv, int T, const Occupancy& occ) {
     }
   }
   const int tiles_per = (ntile + best - 1) / best;
-  sp.tps = tiles_per * kTileT;
+  sp.tps = tiles_per * tile;
   sp.S = (ntile + tiles_per - 1) / tiles_per;
   sp.C = cluster_for(sp.S, cmax);
   return sp;
@@ -1144,7 +1173,7 @@ kvq_status make_job(const AttendJobHost& h, int B, int Hkv, int T_cap, AttnJob* 
   if (INT4) {
     const uint64_t dims[2] = {(uint64_t)D / 2, rows};
     const uint64_t strides[1] = {(uint64_t)D / 2};
-    const uint32_t box[2] = {(uint32_t)D / 2, (uint32_t)kTileT};
+    const uint32_t box[2] = {(uint32_t)D / 2, (uint32_t)C::kTile};
     const CUtensorMapSwizzle sw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     st = encode_tiled(&j->kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, h.kc, dims, strides, box, sw, "K codes");
     if (st == KVQ_OK) st = encode_tiled(&j->vmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, h.vc, dims, strides, box, sw, "V codes");
@@ -1161,7 +1190,7 @@ kvq_status make_job(const AttendJobHost& h, int B, int Hkv, int T_cap, AttnJob* 
   } else {
     const uint64_t dims[2] = {(uint64_t)D, rows};
     const uint64_t strides[1] = {(uint64_t)D * 2};
-    const uint32_t box[2] = {64u, (uint32_t)kTileT};
+    const uint32_t box[2] = {64u, (uint32_t)C::kTile};
     st = encode_tiled(&j->kmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h.kc, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B,
                       "K cache");
     if (st == KVQ_OK)
@@ -1206,7 +1235,7 @@ kvq_status launch_chunk(const AttendJobHost* jobs, int nj, int B, int Hq, int Hk
   using C = Cfg<D, INT4>;
   const int T_split = seq_lens ? T_cap : T_len;
   const int Bj = nj * B;  // the jobs of a launch split like a larger batch
-  SplitPlan sp = choose_split(Bj, Hq, Hkv, T_split, occupancy<D, INT4, MAXJ>());
+  SplitPlan sp = choose_split(Bj, Hq, Hkv, T_split, occupancy<D, INT4, MAXJ>(), C::kTile);
   const size_t units = (size_t)Bj * Hkv * sp.HT;
   const size_t need = ws_bytes_for(Bj, Hq, Hkv, D, sp.S / sp.C, sp.HT);
   if (ws_bytes < need) return fail(KVQ_ERR_WORKSPACE, "attend: workspace too small for this split");
@@ -1269,13 +1298,12 @@ kvq_status run_attend(const AttendJobHost* jobs, int njobs, int B, int Hq, int H
 }  // namespace
 
 size_t attend_workspace_bytes(int B, int Hq, int Hkv, int D, int T_cap) {
-  // Bound over every split the launch can choose for T <= T_cap: S never exceeds
-  // min(kMaxSplits, ntile(T_cap) / kMinTilesPerSplit) (at least 1), and a unit never
-  // has more than min(S, kMaxMerge) cluster partials.
+  // Bound over every split the launch can choose for T <= T_cap: every split keeps at
+  // least kMinTokensPerSplit tokens, so S <= min(kMaxSplits, T_cap / kMinTokensPerSplit)
+  // (at least 1), and a unit never has more than min(S, kMaxMerge) cluster partials.
   const int G = Hq / Hkv;
   const int HT = (G + kHT - 1) / kHT;
-  const int ntile = T_cap > 0 ? (T_cap + kTileT - 1) / kTileT : 1;
-  const int s_max = std::max(1, std::min(kMaxSplits, ntile / kMinTilesPerSplit));
+  const int s_max = std::max(1, std::min(kMaxSplits, T_cap / kMinTokensPerSplit));
   return ws_bytes_for(B, Hq, Hkv, D, std::min(s_max, kMaxMerge), HT);
 }
 
@@ -1343,7 +1371,7 @@ kvq_status launch_attend_int4_noalloc(const kvq_plan* pk, const kvq_plan* pv, co
   const int D = pk->D;
   // the exact split the launch will choose, hence the exact scratch it needs
   const Occupancy& occ = D == 128 ? occupancy<128, true, 1>() : occupancy<256, true, 1>();
-  const SplitPlan sp = choose_split(B, Hq, Hkv, seq_lens ? T_cap : T_len, occ);
+  const SplitPlan sp = choose_split(B, Hq, Hkv, seq_lens ? T_cap : T_len, occ, Cfg<128, true>::kTile);
   const size_t need = ws_bytes_for(B, Hq, Hkv, D, sp.S / sp.C, sp.HT);
   if (need > kNoAllocScratchBytes)
     return fail(KVQ_ERR_WORKSPACE, "attend_noalloc: these shapes need " + std::to_string(need) +
