@@ -255,7 +255,8 @@ kvq_status kvq_attend_decode_ref(const uint16_t* q, const uint16_t* k, const uin
  * kvq_poll_device_errors -- synchronises the current device, then returns (in
  * *flags, host, may be NULL) the bit flags raised by kernels of this library
  * since the last poll, and clears them: 1 = a kernel gave up waiting for a TMA
- * load (bounded wait of 1 s), 2 = a bulk store did not drain. 0 means none.
+ * load (bounded wait of 1 s), 2 = a bulk store did not drain, 4 = an attention
+ * cluster merge did not receive (or release) a partial within 1 s. 0 means none.
  * Errors: CUDA.
  */
 kvq_status kvq_poll_device_errors(uint32_t* flags);

@@ -39,13 +39,11 @@
 #include <mutex>
 
 #include "kvq_internal.h"
-#include <cooperative_groups.h>
 
 #include "kvq_ptx.cuh"
 
 namespace kvq {
 
-namespace cg = cooperative_groups;
 
 __device__ uint32_t g_attend_err = 0;
 
@@ -76,11 +74,10 @@ struct Cfg {
   static constexpr int kStages = INT4 ? 2 : (D == 128 ? 3 : 2);
   static constexpr int kScaleBox = (kTile * NG) < 256 ? kTile * NG : 256;  // halves per scale TMA box
   static constexpr int kScaleLoads = INT4 ? (kTile * NG) / kScaleBox : 0;
-  // warp-merge scratch (reuses the stage ring): per warp m[8], l[8], o[8][D]
-  static constexpr int kWarpState = (2 * kHT + kHT * D) * 4;
   static constexpr int kRing = kStages * kStageBytes;
-  // tail scratch (reuses the ring): warp partials, CTA partial, merged (M, L), merge weights, output
-  static constexpr int kTail = ((kCWarps + 1) * (2 * kHT + kHT * D) + 2 * kHT + 2 * kMaxMerge * kHT + kHT * D) * 4;
+  // tail scratch (reuses the ring): the warps' partials, this CTA's partial, the merged
+  // (M, L) and the warps' (m, l); the un-rotated output reuses the warp partials
+  static constexpr int kTail = ((kCWarps + 1) * (2 * kHT + kHT * D) + 2 * kHT + kCWarps * 2 * kHT) * 4;
   static constexpr int kScratch = kRing > kTail ? kRing : kTail;
   static constexpr int kQt = kHT * D * 4;                  // fp32 q_t (or merged o_t) [8][D]
   // staged at kernel start by bulk copies: the tile's query rows (fp16 [8][D]) and,
@@ -94,14 +91,17 @@ struct Cfg {
   // (hi01, hi23, lo01, lo23) -- read from shared memory at each use
   static constexpr int kKSteps = INT4 ? 2 * NG : D / 16;
   static constexpr int kQf = kKSteps * 32 * 16;
-  static constexpr int kBars = 128;        // full[], empty[], const barrier, rotation barrier, flag
+  static constexpr int kBars = 128;        // full[], empty[], const, rotation, cluster rdy / got barriers, flag
   // D = 128 int4: the plan's rotation matrix (hi, lo) for the query, then the V plan's
   // transpose for the output, as [hi/lo][64-column chunk][128 rows][128 B] (128-byte swizzle)
   static constexpr bool kMmaRot = INT4;   // D = 128: Lambda^-1 F_r; D = 256: F128 (even/odd split)
   static constexpr int kRotOff = (kScratch + kQt + kQs + kConsts + kQf + kBars + 1023) / 1024 * 1024;
   static constexpr int kRot = kMmaRot ? 4 * 128 * 128 : 0;
   static constexpr int kSmem = kRotOff + kRot + 1024;
-  static_assert(2 * kStages * 8 + 8 + 4 <= kBars, "barrier region");
+  static_assert(2 * kStages * 8 + 4 * 8 + 4 <= kBars, "barrier region");
+  // the merge weights of up to kMaxMerge partials reuse the (dead) B fragments
+  static_assert(kQf >= 2 * kMaxMerge * kHT * 4, "merge scratch");
+  static_assert(kHT * D <= kCWarps * (2 * kHT + kHT * D), "output scratch");
 };
 
 struct AttnParams {
@@ -196,7 +196,8 @@ __device__ __forceinline__ void rotate_query_mma(const uint16_t* qs, int heads, 
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int mt = 2 * warp + t;  // channels 16 mt .. 16 mt + 15
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    // hi and lo products in separate accumulators: two short dependency chains
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, acl[4] = {0.f, 0.f, 0.f, 0.f};
     const int row = 16 * mt + ((mi & 1) << 3) + (lane & 7);
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
@@ -205,14 +206,14 @@ __device__ __forceinline__ void rotate_query_mma(const uint16_t* qs, int heads, 
       ldmatrix_x4(a0, a1, a2, a3, rot_addr(srot, 0, row, col));
       mma_16816(acc, a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
       ldmatrix_x4(a0, a1, a2, a3, rot_addr(srot, 1, row, col));
-      mma_16816(acc, a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
+      mma_16816(acl, a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
     }
     // C layout: rows g, g + 8 (channels), columns 2 cq, 2 cq + 1 (heads)
     const int c0 = 16 * mt + g;
-    qt[(2 * cq) * 128 + c0] = acc[0];
-    qt[(2 * cq + 1) * 128 + c0] = acc[1];
-    qt[(2 * cq) * 128 + c0 + 8] = acc[2];
-    qt[(2 * cq + 1) * 128 + c0 + 8] = acc[3];
+    qt[(2 * cq) * 128 + c0] = acc[0] + acl[0];
+    qt[(2 * cq + 1) * 128 + c0] = acc[1] + acl[1];
+    qt[(2 * cq) * 128 + c0 + 8] = acc[2] + acl[2];
+    qt[(2 * cq + 1) * 128 + c0 + 8] = acc[3] + acl[3];
   }
 }
 
@@ -242,7 +243,8 @@ __device__ __forceinline__ void unrotate_out_mma(const float* om, int heads, con
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int mt = 2 * warp + t;  // samples 16 mt .. 16 mt + 15
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    // the three products in separate accumulators: short dependency chains
+    float acc[4] = {0.f, 0.f, 0.f, 0.f}, ahl[4] = {0.f, 0.f, 0.f, 0.f}, alh[4] = {0.f, 0.f, 0.f, 0.f};
     const int row = 16 * mt + ((mi & 1) << 3) + (lane & 7);
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
@@ -250,10 +252,12 @@ __device__ __forceinline__ void unrotate_out_mma(const float* om, int heads, con
       uint32_t a0, a1, a2, a3;
       ldmatrix_x4(a0, a1, a2, a3, rot_addr(srot, 0, row, col));
       mma_16816(acc, a0, a1, a2, a3, bh[ks][0], bh[ks][1]);
-      mma_16816(acc, a0, a1, a2, a3, bl[ks][0], bl[ks][1]);
+      mma_16816(ahl, a0, a1, a2, a3, bl[ks][0], bl[ks][1]);
       ldmatrix_x4(a0, a1, a2, a3, rot_addr(srot, 1, row, col));
-      mma_16816(acc, a0, a1, a2, a3, bh[ks][0], bh[ks][1]);
+      mma_16816(alh, a0, a1, a2, a3, bh[ks][0], bh[ks][1]);
     }
+#pragma unroll
+    for (int e = 0; e < 4; ++e) acc[e] += ahl[e] + alh[e];
     const int n0 = 16 * mt + g;
     if (2 * cq < heads) {
       xb[(2 * cq) * 128 + n0] = acc[0];
@@ -292,7 +296,9 @@ __device__ __forceinline__ void rotate_query_eo(const uint16_t* qs, int heads, c
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       const int mt = 2 * warp + t;  // slots 16 mt .. 16 mt + 15
+      // products with the hi and lo halves of F128 in separate accumulators
       float ae[4] = {0.f, 0.f, 0.f, 0.f}, ao[4] = {0.f, 0.f, 0.f, 0.f};
+      float ael[4] = {0.f, 0.f, 0.f, 0.f}, aol[4] = {0.f, 0.f, 0.f, 0.f};
       const int row = 16 * mt + ((mi & 1) << 3) + (lane & 7);
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
@@ -302,8 +308,13 @@ __device__ __forceinline__ void rotate_query_eo(const uint16_t* qs, int heads, c
         mma_16816(ae, a0, a1, a2, a3, be[ks][0], be[ks][1]);
         mma_16816(ao, a0, a1, a2, a3, bo[ks][0], bo[ks][1]);
         ldmatrix_x4(a0, a1, a2, a3, rot_addr(srot, 1, row, col));
-        mma_16816(ae, a0, a1, a2, a3, be[ks][0], be[ks][1]);
-        mma_16816(ao, a0, a1, a2, a3, bo[ks][0], bo[ks][1]);
+        mma_16816(ael, a0, a1, a2, a3, be[ks][0], be[ks][1]);
+        mma_16816(aol, a0, a1, a2, a3, bo[ks][0], bo[ks][1]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        ae[e] += ael[e];
+        ao[e] += aol[e];
       }
       const int j0 = 16 * mt + g;
       eo[(2 * cq) * 128 + j0] = ae[0];
@@ -435,7 +446,9 @@ __device__ __forceinline__ void unrotate_out_eo(const float* om, int heads, cons
 #pragma unroll
     for (int tt = 0; tt < 2; ++tt) {
       const int mt = 2 * warp + tt;  // samples m = 16 mt .. 16 mt + 15 of each half
+      // products with the hi and lo halves of F128 in separate accumulators
       float xe[4] = {0.f, 0.f, 0.f, 0.f}, xo[4] = {0.f, 0.f, 0.f, 0.f};
+      float xel[4] = {0.f, 0.f, 0.f, 0.f}, xol[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int ks = 0; ks < 8; ++ks) {
         // A = F128^T (rows m, columns j): transposed 8x8 blocks of F128 rows j
@@ -444,12 +457,17 @@ __device__ __forceinline__ void unrotate_out_eo(const float* om, int heads, cons
         uint32_t a0, a1, a2, a3;
         ldmatrix_x4_trans(a0, a1, a2, a3, rot_addr(srot, 0, jrow, mcol));
         mma_16816(xe, a0, a1, a2, a3, eh[ks][0], eh[ks][1]);
-        mma_16816(xe, a0, a1, a2, a3, el[ks][0], el[ks][1]);
         mma_16816(xo, a0, a1, a2, a3, oh[ks][0], oh[ks][1]);
+        mma_16816(xe, a0, a1, a2, a3, el[ks][0], el[ks][1]);
         mma_16816(xo, a0, a1, a2, a3, ol[ks][0], ol[ks][1]);
         ldmatrix_x4_trans(a0, a1, a2, a3, rot_addr(srot, 1, jrow, mcol));
-        mma_16816(xe, a0, a1, a2, a3, eh[ks][0], eh[ks][1]);
-        mma_16816(xo, a0, a1, a2, a3, oh[ks][0], oh[ks][1]);
+        mma_16816(xel, a0, a1, a2, a3, eh[ks][0], eh[ks][1]);
+        mma_16816(xol, a0, a1, a2, a3, oh[ks][0], oh[ks][1]);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        xe[e] += xel[e];
+        xo[e] += xol[e];
       }
       const int m0 = 16 * mt + g;
       if (2 * cq < heads) {
@@ -489,7 +507,9 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
   uint64_t* empty = full + C::kStages;
   uint64_t* cbar = empty + C::kStages;
   uint64_t* ubar = cbar + 1;  // un-rotation matrix landed (D = 128 int4)
-  int* flag = reinterpret_cast<int*>(ubar + 1);
+  uint64_t* rdy = ubar + 1;   // cluster peers: the leader has read this CTA's partial
+  uint64_t* got = rdy + 1;    // cluster leader: every peer's partial is complete
+  int* flag = reinterpret_cast<int*>(got + 1);
   uint8_t* srot = smem + C::kRotOff;
 
   const int warp = threadIdx.x >> 5;
@@ -504,11 +524,6 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
   const int hq0 = kvh * p.G + ht * kHT;        // first query head
   const int unit = (int)blockIdx.z * p.HT + ht;  // workspace slot (over all jobs)
 
-  int T_b = p.T_len;
-  if (p.seq_lens) T_b = min(max(__ldg(p.seq_lens + b), 0), p.T_cap);
-  const int t_begin = split * p.tps;
-  const int t_end = min(t_begin + p.tps, T_b);
-  const int ntiles = t_end > t_begin ? (t_end - t_begin + C::kTile - 1) / C::kTile : 0;
   const int row0 = bk * p.T_cap;  // first cache row of this (b, kv head)
 
   if (threadIdx.x == 0) {
@@ -518,9 +533,49 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
     }
     mbar_init(cbar, 1);
     mbar_init(ubar, 1);
+    mbar_init(rdy, 1);
+    mbar_init(got, cluster_nctarank() > 1 ? cluster_nctarank() - 1 : 1);
     fence_mbarrier_init();
   }
+  // the next kernel in the stream may start its prologue now: everything it reads that
+  // this kernel writes, it reads after its own grid_dep_wait()
+  grid_dep_launch();
   __syncthreads();
+  cluster_arrive_relaxed();  // published barrier initialisation; waited on before the merge
+  if (warp == kCWarps && lane == 0) {
+    // the plans' constants (written once when a plan is made, never by a kernel) need
+    // not wait for the previous kernel: staged while it finishes. The query rows come
+    // on the same barrier after the wait below.
+    const uint32_t qbytes = (uint32_t)(heads * D * 2);
+    mbar_arrive_expect_tx(cbar, qbytes + (INT4 ? (uint32_t)C::kConsts : 0u) + (uint32_t)C::kRot);
+    if constexpr (INT4) {
+      bulk_load(cst, J.kd->chan, C::kChanBytes, cbar);
+      bulk_load(cst + C::kChanBytes, J.ke->sgn, C::kSgnBytes, cbar);
+      bulk_load(cst + C::kChanBytes + C::kSgnBytes, J.vd->chan, C::kChanBytes, cbar);
+      bulk_load(cst + 2 * C::kChanBytes + C::kSgnBytes, J.vd->sgn, C::kSgnBytes, cbar);
+    }
+    if constexpr (C::kMmaRot) {
+#pragma unroll
+      for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+        for (int kc = 0; kc < 2; ++kc) tma_load_2d(srot + (2 * hl + kc) * 16384, &J.rqmap, cbar, 64 * kc, 128 * hl);
+    }
+    prefetch_tensormap(&J.kmap);
+    prefetch_tensormap(&J.vmap);
+    if constexpr (INT4) {
+      prefetch_tensormap(&J.ksmap);
+      prefetch_tensormap(&J.vsmap);
+    }
+  }
+  // from here on: the query, the caches, the sequence lengths, the workspace and the
+  // output, which earlier kernels in the stream may write
+  grid_dep_wait();
+
+  int T_b = p.T_len;
+  if (p.seq_lens) T_b = min(max(__ldg(p.seq_lens + b), 0), p.T_cap);
+  const int t_begin = split * p.tps;
+  const int t_end = min(t_begin + p.tps, T_b);
+  const int ntiles = t_end > t_begin ? (t_end - t_begin + C::kTile - 1) / C::kTile : 0;
 
   // per-warp softmax state (consumer warps): heads 2c, 2c+1
   float m_run[2] = {-INFINITY, -INFINITY};
@@ -533,28 +588,8 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
   if (warp == kCWarps) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      // query rows of the tile and the plans' constants: one round trip, one barrier
-      const uint32_t qbytes = (uint32_t)(heads * D * 2);
-      mbar_arrive_expect_tx(cbar, qbytes + (INT4 ? (uint32_t)C::kConsts : 0u) + (uint32_t)C::kRot);
-      bulk_load(qs, J.q + ((size_t)b * p.Hq + hq0) * D, qbytes, cbar);
-      if constexpr (INT4) {
-        bulk_load(cst, J.kd->chan, C::kChanBytes, cbar);
-        bulk_load(cst + C::kChanBytes, J.ke->sgn, C::kSgnBytes, cbar);
-        bulk_load(cst + C::kChanBytes + C::kSgnBytes, J.vd->chan, C::kChanBytes, cbar);
-        bulk_load(cst + 2 * C::kChanBytes + C::kSgnBytes, J.vd->sgn, C::kSgnBytes, cbar);
-      }
-      if constexpr (C::kMmaRot) {
-#pragma unroll
-        for (int hl = 0; hl < 2; ++hl)
-#pragma unroll
-          for (int kc = 0; kc < 2; ++kc) tma_load_2d(srot + (2 * hl + kc) * 16384, &J.rqmap, cbar, 64 * kc, 128 * hl);
-      }
-      prefetch_tensormap(&J.kmap);
-      prefetch_tensormap(&J.vmap);
-      if constexpr (INT4) {
-        prefetch_tensormap(&J.ksmap);
-        prefetch_tensormap(&J.vsmap);
-      }
+      // the query rows of the tile (their bytes are in the barrier's count already)
+      bulk_load(qs, J.q + ((size_t)b * p.Hq + hq0) * D, (uint32_t)(heads * D * 2), cbar);
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % C::kStages;
         if (i >= C::kStages) {
@@ -607,7 +642,7 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
     if constexpr (C::kMmaRot && D == 128) {
       // the rotation matrix is consumed: a cluster leader (the only CTA that can run the
       // final merge) prefetches the V plan's un-rotation matrix into the same buffer
-      if (threadIdx.x == 0 && cg::this_cluster().block_rank() == 0) {
+      if (threadIdx.x == 0 && cluster_ctarank() == 0) {
         fence_proxy_async_smem();
         mbar_arrive_expect_tx(ubar, (uint32_t)C::kRot);
 #pragma unroll
@@ -873,18 +908,31 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
   __syncthreads();
 
   // ------------------------------------------------------------ merge the warps (ring is free now)
+  // Each warp rescales its (m, l, o) to the CTA maximum M = max_w m_w, then the CTA
+  // partial is O = sum_w o_w 2^(m_w - M), L = sum_w l_w 2^(m_w - M).
   constexpr int PART = 2 * kHT + kHT * D;        // m[8] | l[8] | o[8][D]
-  float* wst = reinterpret_cast<float*>(ring);  // [warp][PART]
+  float* wst = reinterpret_cast<float*>(ring);  // [warp][PART] (o only)
   float* cpart = wst + kCWarps * PART;           // this CTA's partial [PART]
+  float* mrg = cpart + PART;                     // merged (M, L) [2][8]
+  float* wml = mrg + 2 * kHT;                    // the warps' (m, l) [warp][2][8]
+  if (warp < kCWarps && g == 0) {
+    wml[warp * 2 * kHT + 2 * c] = m_run[0];
+    wml[warp * 2 * kHT + 2 * c + 1] = m_run[1];
+    wml[warp * 2 * kHT + kHT + 2 * c] = l_run[0];
+    wml[warp * 2 * kHT + kHT + 2 * c + 1] = l_run[1];
+  }
+  __syncthreads();
   if (warp < kCWarps) {
-    float* ws = wst + warp * PART;
-    if (g == 0) {
-      ws[2 * c] = m_run[0];
-      ws[2 * c + 1] = m_run[1];
-      ws[kHT + 2 * c] = l_run[0];
-      ws[kHT + 2 * c + 1] = l_run[1];
+    float sc[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int h = 2 * c + e;
+      float M = -INFINITY;
+#pragma unroll
+      for (int w = 0; w < kCWarps; ++w) M = fmaxf(M, wml[w * 2 * kHT + h]);
+      sc[e] = m_run[e] == -INFINITY ? 0.0f : fast_exp2(m_run[e] - M);
     }
-    float* wo = ws + 2 * kHT;
+    float* wo = wst + warp * PART + 2 * kHT;
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
       int ch0, ch1;  // channels held in rows g and g+8 of m-tile mt
@@ -896,46 +944,108 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
         ch0 = mt * 16 + g;
         ch1 = ch0 + 8;
       }
-      wo[(2 * c) * D + ch0] = o_acc[mt][0];
-      wo[(2 * c + 1) * D + ch0] = o_acc[mt][1];
-      wo[(2 * c) * D + ch1] = o_acc[mt][2];
-      wo[(2 * c + 1) * D + ch1] = o_acc[mt][3];
+      wo[(2 * c) * D + ch0] = o_acc[mt][0] * sc[0];
+      wo[(2 * c + 1) * D + ch0] = o_acc[mt][1] * sc[1];
+      wo[(2 * c) * D + ch1] = o_acc[mt][2] * sc[0];
+      wo[(2 * c + 1) * D + ch1] = o_acc[mt][3] * sc[1];
     }
-  }
-  __syncthreads();
-  // CTA partial: M = max_w m_w, L = sum_w l_w 2^(m_w - M), O = sum_w o_w 2^(m_w - M)
-  for (int idx = threadIdx.x; idx < heads * D + kHT; idx += kThreads) {
-    const bool ml = idx >= heads * D;
-    const int h = ml ? idx - heads * D : idx / D;
+  } else if (lane < kHT) {
+    const int h = lane;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kCWarps; ++w) M = fmaxf(M, wst[w * PART + h]);
-    float acc = 0.0f;
+    for (int w = 0; w < kCWarps; ++w) M = fmaxf(M, wml[w * 2 * kHT + h]);
+    float L = 0.0f;
     if (M != -INFINITY) {
 #pragma unroll
       for (int w = 0; w < kCWarps; ++w) {
-        const float mw = wst[w * PART + h];
-        if (mw != -INFINITY) acc += wst[w * PART + (ml ? kHT + h : 2 * kHT + idx)] * fast_exp2(mw - M);
+        const float mw = wml[w * 2 * kHT + h];
+        if (mw != -INFINITY) L += wml[w * 2 * kHT + kHT + h] * fast_exp2(mw - M);
       }
     }
-    if (ml) {
-      cpart[h] = M;
-      cpart[kHT + h] = acc;
-    } else {
-      cpart[2 * kHT + idx] = acc;
+    cpart[h] = M;
+    cpart[kHT + h] = L;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < heads * D / 4; i += kThreads) {
+    float4 acc = reinterpret_cast<const float4*>(wst + 2 * kHT)[i];
+#pragma unroll
+    for (int w = 1; w < kCWarps; ++w) {
+      const float4 v = reinterpret_cast<const float4*>(wst + w * PART + 2 * kHT)[i];
+      acc.x += v.x;
+      acc.y += v.y;
+      acc.z += v.z;
+      acc.w += v.w;
     }
+    reinterpret_cast<float4*>(cpart + 2 * kHT)[i] = acc;
   }
 
   // ------------------------------------------------------------ merge the splits of the cluster (DSMEM)
-  cg::cluster_group cluster = cg::this_cluster();
-  const int crank = (int)cluster.block_rank();
-  const int csize = (int)cluster.num_blocks();
-  cluster.sync();  // every CTA's partial is in its shared memory
-  float* om = qt;                                // merged o_t [8][D] (fp32)
-  float* mrg = cpart + PART;                     // merged (M, L) [2][8]
-  float* wsm = mrg + 2 * kHT;                    // [n][8] weights (merge scratch)
-  float* lsm = wsm + kMaxMerge * kHT;            // [n][8]
-  float* xb = lsm + kMaxMerge * kHT;             // [8][D] un-rotated output (fp32)
+  // Each peer publishes its partial with one arrival on the leader's (cluster rank 0)
+  // `got` barrier; the leader reads all partials from distributed shared memory in one
+  // pass and then arrives on each peer's `rdy`, after which the peer may exit.
+  const int crank = (int)cluster_ctarank();
+  const int csize = (int)cluster_nctarank();
+  fence_acq_rel_cluster();  // this thread's partial writes, for the leader's reads
+  __syncthreads();
+  cluster_wait();  // every CTA of the cluster has initialised its barriers
+  if (crank != 0) {
+    if (threadIdx.x == 0) {
+      mbar_arrive_remote(mapa_shared(smem_u32(got), 0));
+      if (!mbar_wait_cluster_bounded(rdy, 0)) atomicOr(&g_attend_err, kErrTimeoutCombine);
+    }
+    return;
+  }
+  if (csize > 1 && !mbar_wait_cluster_bounded(got, 0) && threadIdx.x == 0) atomicOr(&g_attend_err, kErrTimeoutCombine);
+  float* om = qt;                                  // merged o_t [8][D] (fp32)
+  {
+    const uint32_t cbase = smem_u32(cpart);
+    for (int i = threadIdx.x; i < heads * D / 4; i += kThreads) {
+      const int h = (4 * i) / D;
+      float mr[kMaxCluster], lr[kMaxCluster];
+      float4 vr[kMaxCluster];
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r) {
+        if (r < csize) {
+          const uint32_t a = mapa_shared(cbase, (uint32_t)r);
+          mr[r] = ld_dsmem_f32(a + 4 * h);
+          lr[r] = ld_dsmem_f32(a + 4 * (kHT + h));
+          vr[r] = ld_dsmem_f32x4(a + 4 * (2 * kHT) + 16 * i);
+        }
+      }
+      float M = -INFINITY;
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r)
+        if (r < csize) M = fmaxf(M, mr[r]);
+      float L = 0.0f;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r) {
+        if (r < csize) {
+          const float w = (M == -INFINITY || mr[r] == -INFINITY) ? 0.0f : fast_exp2(mr[r] - M);
+          L = fmaf(w, lr[r], L);
+          acc.x = fmaf(w, vr[r].x, acc.x);
+          acc.y = fmaf(w, vr[r].y, acc.y);
+          acc.z = fmaf(w, vr[r].z, acc.z);
+          acc.w = fmaf(w, vr[r].w, acc.w);
+        }
+      }
+      reinterpret_cast<float4*>(om)[i] = acc;
+      if ((4 * i) % D == 0) {
+        mrg[h] = M;
+        mrg[kHT + h] = L;
+      }
+    }
+    if (threadIdx.x >= heads && threadIdx.x < kHT) {  // head rows past the group: empty
+      mrg[threadIdx.x] = -INFINITY;
+      mrg[kHT + threadIdx.x] = 0.0f;
+    }
+    __syncthreads();
+    if (csize > 1 && threadIdx.x == 0)
+      for (int r = 1; r < csize; ++r) mbar_arrive_remote(mapa_shared(smem_u32(rdy), (uint32_t)r));
+  }
+  float* wsm = reinterpret_cast<float*>(qf);       // [n][8] weights (workspace merge scratch)
+  float* lsm = wsm + kMaxMerge * kHT;              // [n][8]
+  float* xb = wst;                                 // [8][D] un-rotated output (fp32), over the dead warp partials
   // merge n partials (pointer of partial r from `at`) into (mrg, om) -- om unnormalised, relative to M
   auto merge = [&](int n, auto at) {
     for (int i = threadIdx.x; i < n * kHT; i += kThreads) {
@@ -975,9 +1085,6 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
     }
     __syncthreads();
   };
-  if (crank == 0) merge(csize, [&](int r) { return static_cast<const float*>(cluster.map_shared_rank(cpart, r)); });
-  cluster.sync();  // peers may leave once the leader has read their shared memory
-  if (crank != 0) return;
   // (D = 128 int4) the leader's un-rotation matrix prefetch must land before the CTA may exit
   bool rot_ok = true;
   if constexpr (C::kMmaRot && D == 128) rot_ok = mbar_wait_bounded(ubar, 0);
@@ -1267,13 +1374,17 @@ kvq_status launch_chunk(const AttendJobHost* jobs, int nj, int B, int Hq, int Hk
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = strm;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = (unsigned)sp.C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  // programmatic dependent launch: the kernel stages the plans' constants while the
+  // previous kernel in the stream finishes, and reads nothing else before it completes
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, attend_kernel<D, INT4, MAXJ>, jt, prm);
   if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
   return KVQ_OK;
