@@ -72,6 +72,8 @@ struct Cfg {
   static constexpr int kSBytes = INT4 ? kTile * NG * 2 : 0;
   static constexpr int kStageBytes = 2 * kKBytes + 2 * kSBytes;
   static constexpr int kStages = INT4 ? 2 : (D == 128 ? 3 : 2);
+  // latency of one stage when the kernel is latency-bound (ns, measured; split planning)
+  static constexpr long kStageNs = INT4 ? (D == 128 ? 750 : 1350) : (D == 128 ? 200 : 570);
   static constexpr int kScaleBox = (kTile * NG) < 256 ? kTile * NG : 256;  // halves per scale TMA box
   static constexpr int kScaleLoads = INT4 ? (kTile * NG) / kScaleBox : 0;
   static constexpr int kRing = kStages * kStageBytes;
@@ -1051,8 +1053,8 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
     for (int i = threadIdx.x; i < n * kHT; i += kThreads) {
       const int r = i / kHT, h = i - r * kHT;
       const float* pr = at(r);
-      wsm[i] = pr[h];
-      lsm[i] = pr[kHT + h];
+      wsm[i] = __ldcg(pr + h);
+      lsm[i] = __ldcg(pr + kHT + h);
     }
     __syncthreads();
     if (threadIdx.x < kHT) {
@@ -1073,13 +1075,22 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
     for (int i = threadIdx.x; i < heads * D / 4; i += kThreads) {
       const int h = (4 * i) / D;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int r = 0; r < n; ++r) {
-        const float w = wsm[r * kHT + h];
-        const float4 v = reinterpret_cast<const float4*>(at(r) + 2 * kHT)[i];
-        acc.x = fmaf(w, v.x, acc.x);
-        acc.y = fmaf(w, v.y, acc.y);
-        acc.z = fmaf(w, v.z, acc.z);
-        acc.w = fmaf(w, v.w, acc.w);
+      // eight partials' loads in flight at a time (one L2 round trip per eight)
+      for (int r0 = 0; r0 < n; r0 += 8) {
+        float4 v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          if (r0 + j < n) v[j] = __ldcg(reinterpret_cast<const float4*>(at(r0 + j) + 2 * kHT) + i);
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (r0 + j < n) {
+            const float w = wsm[(r0 + j) * kHT + h];
+            acc.x = fmaf(w, v[j].x, acc.x);
+            acc.y = fmaf(w, v[j].y, acc.y);
+            acc.z = fmaf(w, v[j].z, acc.z);
+            acc.w = fmaf(w, v[j].w, acc.w);
+          }
+        }
       }
       reinterpret_cast<float4*>(om)[i] = acc;
     }
@@ -1097,7 +1108,8 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
     const int cl = split / csize;
     float* gpart = p.part + ((size_t)unit * ncl + cl) * PART;
     for (int i = threadIdx.x; i < kHT * 2; i += kThreads) __stcg(gpart + i, mrg[i]);
-    for (int i = threadIdx.x; i < heads * D; i += kThreads) __stcg(gpart + 2 * kHT + i, om[i]);
+    for (int i = threadIdx.x; i < heads * D / 4; i += kThreads)
+      __stcg(reinterpret_cast<float4*>(gpart + 2 * kHT) + i, reinterpret_cast<const float4*>(om)[i]);
     // bar.sync orders every thread's stores before thread 0's device-scope fence and
     // counter increment; the last leader fences again before reading the others' partials.
     __syncthreads();
@@ -1191,11 +1203,12 @@ const Occupancy& occupancy() {
 }
 
 // Split of the token range. When splits of ~256 tokens cannot fill the GPU (few
-// units, short context) the kernel is latency-bound: take ~256 tokens per split,
-// which keeps the final merge short. Otherwise (throughput regime) take the split
-// count with the least estimated time (rounds of resident CTAs times the stages
-// per split plus a fixed per-CTA cost). Every split keeps >= kMinTokensPerSplit
-// tokens and S <= kMaxSplits. The splits of a unit form clusters of C CTAs
+// units, short context) the kernel is latency-bound: every candidate runs in one
+// round, and the (S, C) with the least estimated latency wins (stages per split,
+// the cluster merge, a workspace merge when a unit spans several clusters). Otherwise
+// (throughput regime) take the split count with the least estimated time (rounds of
+// resident CTAs times the stages per split plus a fixed per-CTA cost). Every split
+// keeps >= kMinTokensPerSplit tokens and S <= kMaxSplits. The splits of a unit form clusters of C CTAs
 // (C = the largest divisor of S up to 8 in the latency regime, up to 4 in the
 // throughput regime, where large clusters constrain scheduling more than they
 // save) that merge through distributed shared memory; when S > C the S / C
@@ -1213,7 +1226,13 @@ int cluster_for(int S, int cmax) {
   return 1;
 }
 
-SplitPlan choose_split(int B, int Hq, int Hkv, int T, const Occupancy& occ, int tile) {
+// Latency-regime costs (ns): merging the partials of a cluster of c CTAs (distributed
+// shared memory; clusters of 8 span more of a GPC and cost more), and merging n > 1
+// cluster partials through the workspace (counter, fences, one more L2 round trip).
+inline long cluster_ns(int c) { return c == 1 ? 0 : (c <= 4 ? 300 : 950); }
+inline long workspace_merge_ns(int n) { return n > 1 ? 2500 + 150L * n : 0; }
+
+SplitPlan choose_split(int B, int Hq, int Hkv, int T, const Occupancy& occ, int tile, long stage_ns) {
   SplitPlan sp{};
   const int G = Hq / Hkv;
   sp.HT = (G + kHT - 1) / kHT;
@@ -1234,9 +1253,25 @@ SplitPlan choose_split(int B, int Hq, int Hkv, int T, const Occupancy& occ, int 
   };
   auto mergeable = [&](int S) { return S / cluster_for(S, cmax) <= kMaxMerge; };
   int best = 1;
+  int best_c = 0;  // latency regime: the cluster size chosen with S (0: the default rule)
   if (latency) {
-    best = std::max(1, std::min(ntile / kLatencyTilesPerSplit, s_cap));
-    while (best > 1 && !mergeable(realised(best))) --best;
+    // every candidate runs in one round: estimated time = stages per split x the
+    // stage latency + the cluster merge + a workspace merge when the unit has more
+    // than one cluster (all in ns, measured on the kernels)
+    // S need not divide the stages: the last splits may be empty (an empty CTA's
+    // partial has m = -inf and drops out of the merges), so C = S stays available
+    long best_t = -1;
+    for (int S = 1; S <= s_cap; ++S) {
+      for (int Cc = 1; Cc <= kMaxClusterLatency && Cc <= S; Cc *= 2) {
+        if (S % Cc != 0 || S / Cc > kMaxMerge || units * S > occ.cap[Cc]) continue;
+        const long t = (long)((ntile + S - 1) / S) * stage_ns + cluster_ns(Cc) + workspace_merge_ns(S / Cc);
+        if (best_t < 0 || t < best_t) {
+          best_t = t;
+          best = S;
+          best_c = Cc;
+        }
+      }
+    }
   } else {
     // estimated time in stage-times: rounds of resident CTAs x (stages per split +
     // the per-CTA fixed cost), plus the workspace merge when a unit has several clusters
@@ -1255,8 +1290,13 @@ SplitPlan choose_split(int B, int Hq, int Hkv, int T, const Occupancy& occ, int 
   }
   const int tiles_per = (ntile + best - 1) / best;
   sp.tps = tiles_per * tile;
-  sp.S = (ntile + tiles_per - 1) / tiles_per;
-  sp.C = cluster_for(sp.S, cmax);
+  if (best_c > 0) {
+    sp.S = best;
+    sp.C = best_c;
+  } else {
+    sp.S = (ntile + tiles_per - 1) / tiles_per;
+    sp.C = cluster_for(sp.S, cmax);
+  }
   return sp;
 }
 
@@ -1342,7 +1382,7 @@ kvq_status launch_chunk(const AttendJobHost* jobs, int nj, int B, int Hq, int Hk
   using C = Cfg<D, INT4>;
   const int T_split = seq_lens ? T_cap : T_len;
   const int Bj = nj * B;  // the jobs of a launch split like a larger batch
-  SplitPlan sp = choose_split(Bj, Hq, Hkv, T_split, occupancy<D, INT4, MAXJ>(), C::kTile);
+  SplitPlan sp = choose_split(Bj, Hq, Hkv, T_split, occupancy<D, INT4, MAXJ>(), C::kTile, C::kStageNs);
   const size_t units = (size_t)Bj * Hkv * sp.HT;
   const size_t need = ws_bytes_for(Bj, Hq, Hkv, D, sp.S / sp.C, sp.HT);
   if (ws_bytes < need) return fail(KVQ_ERR_WORKSPACE, "attend: workspace too small for this split");
@@ -1409,12 +1449,13 @@ kvq_status run_attend(const AttendJobHost* jobs, int njobs, int B, int Hq, int H
 }  // namespace
 
 size_t attend_workspace_bytes(int B, int Hq, int Hkv, int D, int T_cap) {
-  // Bound over every split the launch can choose for T <= T_cap: every split keeps at
-  // least kMinTokensPerSplit tokens, so S <= min(kMaxSplits, T_cap / kMinTokensPerSplit)
-  // (at least 1), and a unit never has more than min(S, kMaxMerge) cluster partials.
+  // Bound over every split the launch can choose for T <= T_cap: S never exceeds the
+  // stage count over the minimum stages per split, at most ceil(T_cap / kMinTokensPerSplit)
+  // for every kernel (capped by kMaxSplits, at least 1), and a unit never has more than
+  // min(S, kMaxMerge) cluster partials.
   const int G = Hq / Hkv;
   const int HT = (G + kHT - 1) / kHT;
-  const int s_max = std::max(1, std::min(kMaxSplits, T_cap / kMinTokensPerSplit));
+  const int s_max = std::max(1, std::min(kMaxSplits, (T_cap + kMinTokensPerSplit - 1) / kMinTokensPerSplit));
   return ws_bytes_for(B, Hq, Hkv, D, std::min(s_max, kMaxMerge), HT);
 }
 
@@ -1482,7 +1523,8 @@ kvq_status launch_attend_int4_noalloc(const kvq_plan* pk, const kvq_plan* pv, co
   const int D = pk->D;
   // the exact split the launch will choose, hence the exact scratch it needs
   const Occupancy& occ = D == 128 ? occupancy<128, true, 1>() : occupancy<256, true, 1>();
-  const SplitPlan sp = choose_split(B, Hq, Hkv, seq_lens ? T_cap : T_len, occ, Cfg<128, true>::kTile);
+  const SplitPlan sp = choose_split(B, Hq, Hkv, seq_lens ? T_cap : T_len, occ, Cfg<128, true>::kTile,
+                                    D == 128 ? Cfg<128, true>::kStageNs : Cfg<256, true>::kStageNs);
   const size_t need = ws_bytes_for(B, Hq, Hkv, D, sp.S / sp.C, sp.HT);
   if (need > kNoAllocScratchBytes)
     return fail(KVQ_ERR_WORKSPACE, "attend_noalloc: these shapes need " + std::to_string(need) +
