@@ -49,8 +49,6 @@ __device__ uint32_t g_attend_err = 0;
 
 namespace {
 
-constexpr int kCWarps = 4;                 // consumer warps
-constexpr int kThreads = (kCWarps + 1) * 32;
 constexpr int kHT = 8;                     // query heads per CTA (mma N)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kMaxSplitsCfg = 256;          // upper bound on splits per unit
@@ -64,6 +62,10 @@ template <int D, bool INT4>
 struct Cfg {
   static constexpr int NG = D / 32;                        // scale groups (int4)
   static constexpr int kRowBytes = INT4 ? D / 2 : 2 * D;   // bytes per token row of K (and V)
+  // consumer warps (plus one producer warp); resident CTAs per SM for the launch bounds
+  static constexpr int kCWarps = 4;
+  static constexpr int kThreads = (kCWarps + 1) * 32;
+  static constexpr int kMinBlocks = D == 128 ? 2 : 1;
   // each consumer warp takes kSub subtiles of 16 tokens per stage (two independent
   // instruction streams for the int4 path, whose per-token work is latency-bound)
   static constexpr int kSub = INT4 ? 2 : 1;
@@ -161,7 +163,8 @@ __device__ __forceinline__ void nib8_to_h2(uint32_t w, uint32_t (&h)[4]) {
   h[3] = h2_bits(__hfma2(bits_h2(d), k16, k72));
 }
 
-__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kCWarps * 32) : "memory"); }
+template <int NW>
+__device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NW * 32) : "memory"); }
 
 __device__ __forceinline__ float fast_exp2(float x) { return ex2_approx(x); }
 
@@ -277,6 +280,7 @@ __device__ __forceinline__ void unrotate_out_mma(const float* om, int heads, con
 // in shared memory, same layout as above), then X_k = E_k + W^k O_k, X_{128-k} =
 // conj(E_k - W^k O_k) (W = e^{-2 pi i / 256}) and q_t[c] = (dg / lambda)_c X(c).
 // eo: fp32 scratch [E, O][8 heads][128 slots]. Called by the four consumer warps.
+template <int NW>
 __device__ __forceinline__ void rotate_query_eo(const uint16_t* qs, int heads, const uint32_t* ksg, const float* kch,
                                                 const uint8_t* srot, float* eo, float* qt, int warp, int lane) {
   const int g = lane >> 2, cq = lane & 3;
@@ -296,8 +300,8 @@ __device__ __forceinline__ void rotate_query_eo(const uint16_t* qs, int heads, c
       }
     }
 #pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const int mt = 2 * warp + t;  // slots 16 mt .. 16 mt + 15
+    for (int t = 0; t < 8 / NW; ++t) {
+      const int mt = (8 / NW) * warp + t;  // slots 16 mt .. 16 mt + 15
       // products with the hi and lo halves of F128 in separate accumulators
       float ae[4] = {0.f, 0.f, 0.f, 0.f}, ao[4] = {0.f, 0.f, 0.f, 0.f};
       float ael[4] = {0.f, 0.f, 0.f, 0.f}, aol[4] = {0.f, 0.f, 0.f, 0.f};
@@ -329,12 +333,12 @@ __device__ __forceinline__ void rotate_query_eo(const uint16_t* qs, int heads, c
       eo[1024 + (2 * cq + 1) * 128 + j0 + 8] = ao[3];
     }
   }
-  consumer_sync();
-  // radix-2 combine into channels: thread t takes channels t and t + 128 of every head
-  const int t = threadIdx.x;  // 0 .. 127 (consumer warps)
+  consumer_sync<NW>();
+  // radix-2 combine into channels: consumer thread t takes channels t, t + 32 NW, ...
+  const int t = threadIdx.x;  // 0 .. 32 NW - 1 (consumer warps)
 #pragma unroll
-  for (int half = 0; half < 2; ++half) {
-    const int ch = t + 128 * half;
+  for (int half = 0; half < 256 / (32 * NW); ++half) {
+    const int ch = t + 32 * NW * half;
     int k, slot_re, slot_im;
     bool mirror = false, re;
     if (ch == 0) {
@@ -382,6 +386,7 @@ __device__ __forceinline__ void rotate_query_eo(const uint16_t* qs, int heads, c
 // Z_c = (dg / lambda)_c o_t[c] / L; (E', O') = combine^T(Z); x_even = F128^T E',
 // x_odd = F128^T O' on the tensor cores (ldmatrix.trans of the resident F128; E', O'
 // enter as fp16 hi + lo). eo: fp32 scratch [2][8][128]. All 160 threads call it.
+template <int NW>
 __device__ __forceinline__ void unrotate_out_eo(const float* om, int heads, const float* Lh, const float* vch,
                                                 const uint8_t* srot, float* eo, float* xb, int warp, int lane) {
   const int t = threadIdx.x;
@@ -422,7 +427,7 @@ __device__ __forceinline__ void unrotate_out_eo(const float* om, int heads, cons
     }
   }
   __syncthreads();
-  if (warp < kCWarps) {
+  if (warp < NW) {
     const int g = lane >> 2, cq = lane & 3;
     const int mi = lane >> 3;
     const float* Er = eo + g * 128;
@@ -446,8 +451,8 @@ __device__ __forceinline__ void unrotate_out_eo(const float* om, int heads, cons
       }
     }
 #pragma unroll
-    for (int tt = 0; tt < 2; ++tt) {
-      const int mt = 2 * warp + tt;  // samples m = 16 mt .. 16 mt + 15 of each half
+    for (int tt = 0; tt < 8 / NW; ++tt) {
+      const int mt = (8 / NW) * warp + tt;  // samples m = 16 mt .. 16 mt + 15 of each half
       // products with the hi and lo halves of F128 in separate accumulators
       float xe[4] = {0.f, 0.f, 0.f, 0.f}, xo[4] = {0.f, 0.f, 0.f, 0.f};
       float xel[4] = {0.f, 0.f, 0.f, 0.f}, xol[4] = {0.f, 0.f, 0.f, 0.f};
@@ -489,9 +494,12 @@ __device__ __forceinline__ void unrotate_out_eo(const float* om, int heads, cons
 }
 
 template <int D, bool INT4, int MAXJ>
-__global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
+__global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinBlocks))
     attend_kernel(const __grid_constant__ AttnJobs<MAXJ> jt, const __grid_constant__ AttnParams p) {
   using C = Cfg<D, INT4>;
+  constexpr int kCWarps = C::kCWarps;
+  constexpr int kThreads = C::kThreads;
+  static_assert(D == 256 || kCWarps == 4, "the D = 128 rotation helpers take four consumer warps");
   constexpr int NG = C::NG;
   constexpr int MT = D / 16;  // channel m-tiles of the PV product
   extern __shared__ uint8_t smem_raw[];
@@ -632,7 +640,7 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
     if constexpr (C::kMmaRot && D == 128) {
       rotate_query_mma(qs, heads, ksg, srot, qt, warp, lane);
     } else if constexpr (C::kMmaRot) {
-      rotate_query_eo(qs, heads, ksg, kch, srot, reinterpret_cast<float*>(qf), qt, warp, lane);
+      rotate_query_eo<kCWarps>(qs, heads, ksg, kch, srot, reinterpret_cast<float*>(qf), qt, warp, lane);
     } else {
       for (int i = threadIdx.x; i < kHT * D / 2; i += kCWarps * 32) {
         const int h = (2 * i) / D;
@@ -640,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
         reinterpret_cast<float2*>(qt)[i] = f;
       }
     }
-    consumer_sync();
+    consumer_sync<kCWarps>();
     if constexpr (C::kMmaRot && D == 128) {
       // the rotation matrix is consumed: a cluster leader (the only CTA that can run the
       // final merge) prefetches the V plan's un-rotation matrix into the same buffer
@@ -681,7 +689,7 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
                                         h2_bits(__halves2half2(lo[0], lo[1])), h2_bits(__halves2half2(lo[2], lo[3])));
       }
     }
-    consumer_sync();
+    consumer_sync<kCWarps>();
 
     // (3) stream the token range
     const int lane_a = 4 * (2 * c) + (g >> 1);
@@ -696,6 +704,12 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
       const uint8_t* st = ring + s * C::kStageBytes;
       // this warp's SUB subtiles of 16 tokens: stage rows (SUB warp + sb) 16 .. + 15
       constexpr int SUB = C::kSub;
+      if (t_begin + i * C::kTile + warp * SUB * 16 >= t_end) {
+        // none of the warp's tokens is in range (the ragged last stage): nothing to add
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&empty[s]);
+        continue;
+      }
       int tw0[SUB];
       bool partial[SUB];
       float sc[SUB][4];
@@ -1134,7 +1148,7 @@ __global__ void __launch_bounds__(kThreads, D == 128 ? 2 : 1)
     if constexpr (D == 128) {
       if (warp < kCWarps) unrotate_out_mma(om, heads, mrg + kHT, srot, xb, warp, lane);
     } else {
-      unrotate_out_eo(om, heads, mrg + kHT, vch, srot, reinterpret_cast<float*>(qf), xb, warp, lane);
+      unrotate_out_eo<kCWarps>(om, heads, mrg + kHT, vch, srot, reinterpret_cast<float*>(qf), xb, warp, lane);
     }
     __syncthreads();
     for (int i = threadIdx.x; i < heads * D / 2; i += kThreads) {
@@ -1175,7 +1189,7 @@ const Occupancy& occupancy() {
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     int nb = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, kThreads, C::kSmem) != cudaSuccess || nb < 1) nb = 1;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, kern, C::kThreads, C::kSmem) != cudaSuccess || nb < 1) nb = 1;
     occ.per_sm = std::min(nb, kMaxPerSmForSizing);
     int dev = 0;
     cudaGetDevice(&dev);
@@ -1183,7 +1197,7 @@ const Occupancy& occupancy() {
     for (int c = 1; c <= kMaxCluster; ++c) {
       cudaLaunchConfig_t cfg{};
       cfg.gridDim = dim3(c, 1, 1);
-      cfg.blockDim = dim3(kThreads);
+      cfg.blockDim = dim3(C::kThreads);
       cfg.dynamicSmemBytes = C::kSmem;
       cudaLaunchAttribute attr[1];
       attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1411,7 +1425,7 @@ kvq_status launch_chunk(const AttendJobHost* jobs, int nj, int B, int Hq, int Hk
   if (grid.z > 65535u) return fail(KVQ_ERR_UNSUPPORTED, "attend: jobs * B * Hkv > 65535");
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = grid;
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(C::kThreads);
   cfg.dynamicSmemBytes = C::kSmem;
   cfg.stream = strm;
   cudaLaunchAttribute attr[2];
