@@ -59,8 +59,8 @@ KERNEL_SOURCES = {
 NCU_TRAFFIC = {
     # kernel -> (source digest at capture time, bytes per launch)
     "encode": ("800dad8c026c", 115282176),       # register-FFT encode, Gemma step (52 jobs)
-    "encode_tc": ("cafe5c0e8a7f", 127376384),    # tensor-core encode, Gemma step (52 jobs)
-    "attend": ("f95f7ac4b9ec", 30920960),        # grouped int4 attention, Gemma step (26 jobs)
+    "encode_tc": ("424d112ae180", 124641024),    # tensor-core encode, Gemma step (52 jobs)
+    "attend": ("71f8ac5bccce", 32592896),        # grouped int4 attention, Gemma step (26 jobs)
 }
 
 
