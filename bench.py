@@ -64,6 +64,17 @@ NCU_TRAFFIC = {
 }
 
 
+def _tensor_peak() -> float:
+    """Measured sustained dense bf16 TFLOP/s (the encode runs inside a long step), else 1400."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        if "bf16_tflops_sustained" in d:
+            return float(d["bf16_tflops_sustained"])
+    return 1400.0
+
+
 def _source_digest(kind: str) -> str:
     import hashlib
 
@@ -385,8 +396,16 @@ def run_kvq(args, rank: int, world: int):
     clocks = clk.summary(wall0 - 1.0, wall1 + 0.2)
     # roofline of the kernel with the larger share of the step (each phase is one launch)
     src = "measured (MEASURED_PEAKS.json hbm_gbs, burst copy)" if peak_kind == "measured" else "fallback 6.65 TB/s"
+    tc = kvq.get_encode_path() != "fft" and G == 32
+    # the tensor-core encode's own work: Y = X [W_hi; W_lo]^T, 2 x D x 2D flops per vector
+    # (context for the HBM roofline: at D = 256 this product, not HBM, bounds the kernel)
+    tensor = None
+    if tc:
+        tflops = vec_step * 4 * D * D / (enc_avg * 1e-3) / 1e12
+        tensor = {"flops_per_vec": 4 * D * D, "achieved_TFLOP_s": tflops,
+                  "peak_TFLOP_s": _tensor_peak(), "frac": tflops / _tensor_peak(),
+                  "peak_source": "measured (MEASURED_PEAKS.json bf16_tflops_sustained; fp16 runs at the bf16 rate)"}
     if enc_avg >= att_avg:
-        tc = kvq.get_encode_path() != "fft" and G == 32
         roof = {"bound": "hbm", "achieved": enc_gbs, "peak": hbm, "unit": "GB/s", "frac": enc_gbs / hbm,
                 "traffic": _ncu_traffic("encode_tc" if tc else "encode"),
                 "kernel": f"encode_tc_kernel<{D},64>" if tc
@@ -413,7 +432,8 @@ def run_kvq(args, rank: int, world: int):
             "roofline": roof,
             "kernels": {  # both launches of the step, each timed with CUDA events on its stream
                 "encode": {"kernel": roof["kernel"] if enc_avg >= att_avg else "encode", "us": 1e3 * enc_avg,
-                           "achieved_GB_s": enc_gbs, "frac": enc_gbs / hbm, "share": enc_avg / (enc_avg + att_avg)},
+                           "achieved_GB_s": enc_gbs, "frac": enc_gbs / hbm, "share": enc_avg / (enc_avg + att_avg),
+                           "tensor": tensor},
                 "attention": {"kernel": f"attend_kernel<{D},int4,32>", "us": 1e3 * att_avg, "achieved_GB_s": att_gbs,
                               "frac": att_gbs / hbm, "share": att_avg / (enc_avg + att_avg),
                               "traffic": _ncu_traffic("attend")},
