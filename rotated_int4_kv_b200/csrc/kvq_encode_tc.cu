@@ -122,6 +122,9 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
     mbar_init(mdone, 1);
     fence_mbarrier_init();
   }
+  // programmatic dependent launch: the next kernel in the stream may start its own
+  // prologue now (it reads what this kernel writes only after its grid dependency wait)
+  grid_dep_launch();
   if (warp == 1) {
     tmem_alloc(tmem_slot, C::kTmemCols);
     tmem_relinquish();
@@ -136,6 +139,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
     if (lane == 0 && ntile > 0) {
       const uint64_t pol = l2_evict_first_policy();
       int job = job_of(bt.j, bt.njobs, 0, t_begin), wjob = -1, nw = 0;
+      // the first job's W (a plan constant, written once when the plan is made) is
+      // loaded while the previous kernel in the stream finishes; the inputs after it
+      mbar_arrive_expect_tx(wfull, C::kW);
+#pragma unroll
+      for (int kc = 0; kc < C::KC; ++kc) tma_load_2d(sW + kc * C::kChunkW, &bt.j[job].wmap, wfull, kc * 64, 256 * half);
+      wjob = job;
+      nw = 1;
+      grid_dep_wait();
       for (int i = 0; i < ntile; ++i) {
         const int t = t_begin + i;
         job = job_of(bt.j, bt.njobs, job, t);
@@ -351,14 +362,28 @@ kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t 
     int dev = 0;
     cudaGetDevice(&dev);
     const int sms = num_sms(dev);
+    // programmatic dependent launch: the kernel loads its first W and allocates TMEM
+    // while the previous kernel in the stream finishes (grid dependency wait before the
+    // inputs and every global write)
+    cudaLaunchConfig_t cfg{};
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.stream = strm;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e;
     if (D == 128) {
-      const int grid = std::min(tiles, sms);
-      encode_tc_kernel<128, kTcMaxJobs><<<grid, kTcThreads, TcCfg<128>::kSmem, strm>>>(bt);
+      cfg.gridDim = dim3(std::min(tiles, sms));
+      cfg.dynamicSmemBytes = TcCfg<128>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, encode_tc_kernel<128, kTcMaxJobs>, bt);
     } else {
-      const int grid = 2 * std::min(tiles, sms / 2);
-      encode_tc_kernel<256, kTcMaxJobs><<<grid, kTcThreads, TcCfg<256>::kSmem, strm>>>(bt);
+      cfg.gridDim = dim3(2 * std::min(tiles, sms / 2));
+      cfg.dynamicSmemBytes = TcCfg<256>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, encode_tc_kernel<256, kTcMaxJobs>, bt);
     }
-    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("encode (tensor cores) launch: ") + cudaGetErrorString(e));
   }
   return KVQ_OK;
