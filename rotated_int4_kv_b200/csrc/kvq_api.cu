@@ -231,11 +231,12 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
       wt[(size_t)(256 * h + 128 + rr) * D + n] = lo;
     }
   }
-  // attention operands. D = 128: M = Lambda^-1 F_r (hi, lo) and its transpose (hi, lo).
-  // D = 256: the unnormalised 128-point real DFT in slot order, F128 (hi, lo): row 0 = 1,
-  // row 1 = (-1)^m, row 2k = cos(2 pi k m / 128), row 2k+1 = -sin(2 pi k m / 128).
+  // attention operand (both head dims): the unnormalised 128-point real DFT in slot
+  // order, F128 (hi, lo): row 0 = 1, row 1 = (-1)^m, row 2k = cos(2 pi k m / 128),
+  // row 2k+1 = -sin(2 pi k m / 128). D = 128 applies it directly, D = 256 to the even
+  // and odd samples; the plan's signs and per-channel factors are applied around it.
   std::vector<uint16_t> rot;
-  if (D == 256) {
+  {
     const int M = 128;
     rot.resize((size_t)2 * M * M);
     const double pi2 = 6.283185307179586476925286766559;
@@ -252,19 +253,6 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
         const uint16_t lo = kvq::half_bits((float)(v - (double)kvq::half_value(hi)));
         rot[(size_t)j * M + m] = hi;
         rot[(size_t)(M + j) * M + m] = lo;
-      }
-  }
-  if (D == 128) {
-    rot.resize((size_t)4 * D * D);
-    for (int c = 0; c < D; ++c)
-      for (int n = 0; n < D; ++n) {
-        const double m = kvq::basis_value(c, n, D) / (double)lambda[c];
-        const uint16_t hi = kvq::half_bits((float)m);
-        const uint16_t lo = kvq::half_bits((float)(m - (double)kvq::half_value(hi)));
-        rot[(size_t)c * D + n] = hi;                      // rq hi [c][n]
-        rot[(size_t)(D + c) * D + n] = lo;                // rq lo
-        rot[(size_t)(2 * D + n) * D + c] = hi;            // ru hi [n][c]
-        rot[(size_t)(3 * D + n) * D + c] = lo;            // ru lo
       }
   }
   constexpr size_t kWtOff = 4096;  // after the two CodecConsts copies, 16-byte aligned for TMA
@@ -291,9 +279,7 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
   p->enc_dev = reinterpret_cast<const kvq::CodecConsts*>(blk);
   p->dec_dev = reinterpret_cast<const kvq::CodecConsts*>((char*)blk + sizeof(kvq::CodecConsts));
   p->wt_dev = wt.empty() ? nullptr : reinterpret_cast<const uint16_t*>((char*)blk + kWtOff);
-  p->rq_dev = rot.empty() ? nullptr : reinterpret_cast<const uint16_t*>((char*)blk + rot_off);
-  p->ru_dev = D != 128 || rot.empty() ? nullptr
-                                      : reinterpret_cast<const uint16_t*>((char*)blk + rot_off + (size_t)2 * D * D * 2);
+  p->rot_dev = reinterpret_cast<const uint16_t*>((char*)blk + rot_off);
   *out = p;
   return KVQ_OK;
 }

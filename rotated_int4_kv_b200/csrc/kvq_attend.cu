@@ -98,11 +98,11 @@ struct Cfg {
   static constexpr int kBars = 128;        // full[], empty[], const, rotation, cluster rdy / got barriers, flag
   // D = 128 int4: the plan's rotation matrix (hi, lo) for the query, then the V plan's
   // transpose for the output, as [hi/lo][64-column chunk][128 rows][128 B] (128-byte swizzle)
-  static constexpr bool kMmaRot = INT4;   // D = 128: Lambda^-1 F_r; D = 256: F128 (even/odd split)
+  static constexpr bool kMmaRot = INT4;   // F128 (D = 256: even/odd split)
   static constexpr int kRotOff = (kScratch + kQt + kQs + kConsts + kQf + kBars + 1023) / 1024 * 1024;
   static constexpr int kRot = kMmaRot ? 4 * 128 * 128 : 0;
   static constexpr int kSmem = kRotOff + kRot + 1024;
-  static_assert(2 * kStages * 8 + 4 * 8 + 4 <= kBars, "barrier region");
+  static_assert(2 * kStages * 8 + 3 * 8 + 4 <= kBars, "barrier region");
   // the merge weights of up to kMaxMerge partials reuse the (dead) B fragments
   static_assert(kQf >= 2 * kMaxMerge * kHT * 4, "merge scratch");
   static_assert(kHT * D <= kCWarps * (2 * kHT + kHT * D), "output scratch");
@@ -121,7 +121,7 @@ struct AttnParams {
 // blockIdx.z = job * (B * Hkv) + b * Hkv + kv head.
 struct alignas(64) AttnJob {
   CUtensorMap kmap, vmap, ksmap, vsmap;  // K/V codes (or fp16 K/V) and scale rows
-  CUtensorMap rqmap, rumap;              // D = 128 int4: K plan rotation, V plan un-rotation (hi/lo rows)
+  CUtensorMap rotmap;                    // int4: F128 (hi/lo rows), from the K plan
   const uint16_t* q;
   uint16_t* out;
   const CodecConsts* ke;  // K plan: sign masks (int4 only)
@@ -174,34 +174,43 @@ __device__ __forceinline__ void split_h(float x, __half& hi, __half& lo) {
   lo = __float2half_rn(x - __half2float(hi));
 }
 
-// D = 128: q_t[h][c] = sum_n M[c][n] q'[h][n] with q' = s (.) q (fp16, exact) and
-// M = Lambda^-1 F_r held as fp16 hi + lo in shared memory ([hi/lo][64-column chunk]
-// [128 rows][128 B], 128-byte swizzle), on the tensor cores: mma.m16n8k16 with 16
-// channels as M, the 8 heads as N, samples as K; the four consumer warps take two
-// channel tiles each. Heads beyond `heads` get zero rows.
+// The attention kernels hold F128, the unnormalised 128-point real DFT in slot order
+// (row 0 = DC, row 1 = Nyquist, rows 2k / 2k+1 = Re / Im X_k), as fp16 hi + lo in shared
+// memory ([hi/lo][64-column chunk][128 rows][128 B], 128-byte swizzle). At D = 128 the
+// real basis row of channel c is dg_c F128[slot(c)] with slot(0) = 0, slot(127) = 1 and
+// slot(c) = c + 1 otherwise; D = 256 applies F128 to the even and odd samples.
 __device__ __forceinline__ uint32_t rot_addr(const uint8_t* base, int hl, int row, int col) {
   // element (row, col) of matrix hl (0 = hi, 1 = lo); col multiple of 8
   const int kc = col >> 6, ch = (col & 63) >> 3;
   return smem_u32(base + (2 * hl + kc) * 16384 + row * 128 + ((ch ^ (row & 7)) << 4));
 }
+__device__ __forceinline__ int chan_of_slot128(int j) { return j == 0 ? 0 : (j == 1 ? 127 : j - 1); }
+__device__ __forceinline__ int slot_of_chan128(int c) { return c == 0 ? 0 : (c == 127 ? 1 : c + 1); }
 
-__device__ __forceinline__ void rotate_query_mma(const uint16_t* qs, int heads, const uint32_t* ksg,
-                                                 const uint8_t* srot, float* qt, int warp, int lane) {
+// X[j][r] = sum_m F128[j][m] x'_r[m] for up to eight fp16 rows x_r (x'_r = x_r with the
+// sign mask sgn_of(r) applied to its fp16 pairs, exact), on the tensor cores:
+// mma.m16n8k16 with 16 slots as M, the rows as N, samples as K; hi and lo products in
+// separate accumulators. Rows past nrows are zero. The four consumer warps take two
+// slot tiles each and hand every result to out(slot, row, value).
+template <typename SgnOf, typename Out>
+__device__ __forceinline__ void f128_forward(const uint16_t* rows, int nrows, SgnOf sgn_of, const uint8_t* srot,
+                                             int warp, int lane, Out out) {
   const int g = lane >> 2, cq = lane & 3;
   const int mi = lane >> 3;
-  // B fragments (k = samples, n = head g): q'[g][16 ks + 2 cq (+1)], [.. + 8 (+9)]
+  // B fragments (k = samples, n = row g): x'[g][16 ks + 2 cq (+1)], [.. + 8 (+9)]
   uint32_t bq[8][2];
-  const uint32_t* qrow = reinterpret_cast<const uint32_t*>(qs + (g < heads ? g : 0) * 128);
+  const int gr = g < nrows ? g : 0;
+  const uint32_t* xrow = reinterpret_cast<const uint32_t*>(rows + gr * 128);
+  const uint32_t* sg = sgn_of(gr);
 #pragma unroll
   for (int ks = 0; ks < 8; ++ks) {
     const int w0 = 8 * ks + cq, w1 = w0 + 4;  // fp16-pair words of the row
-    bq[ks][0] = g < heads ? (qrow[w0] ^ ksg[w0]) : 0u;
-    bq[ks][1] = g < heads ? (qrow[w1] ^ ksg[w1]) : 0u;
+    bq[ks][0] = g < nrows ? (xrow[w0] ^ sg[w0]) : 0u;
+    bq[ks][1] = g < nrows ? (xrow[w1] ^ sg[w1]) : 0u;
   }
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    const int mt = 2 * warp + t;  // channels 16 mt .. 16 mt + 15
-    // hi and lo products in separate accumulators: two short dependency chains
+    const int mt = 2 * warp + t;  // slots 16 mt .. 16 mt + 15
     float acc[4] = {0.f, 0.f, 0.f, 0.f}, acl[4] = {0.f, 0.f, 0.f, 0.f};
     const int row = 16 * mt + ((mi & 1) << 3) + (lane & 7);
 #pragma unroll
@@ -213,20 +222,30 @@ __device__ __forceinline__ void rotate_query_mma(const uint16_t* qs, int heads, 
       ldmatrix_x4(a0, a1, a2, a3, rot_addr(srot, 1, row, col));
       mma_16816(acl, a0, a1, a2, a3, bq[ks][0], bq[ks][1]);
     }
-    // C layout: rows g, g + 8 (channels), columns 2 cq, 2 cq + 1 (heads)
-    const int c0 = 16 * mt + g;
-    qt[(2 * cq) * 128 + c0] = acc[0] + acl[0];
-    qt[(2 * cq + 1) * 128 + c0] = acc[1] + acl[1];
-    qt[(2 * cq) * 128 + c0 + 8] = acc[2] + acl[2];
-    qt[(2 * cq + 1) * 128 + c0 + 8] = acc[3] + acl[3];
+    // C layout: rows g, g + 8 (slots), columns 2 cq, 2 cq + 1 (input rows)
+    const int j0 = 16 * mt + g;
+    out(j0, 2 * cq, acc[0] + acl[0]);
+    out(j0, 2 * cq + 1, acc[1] + acl[1]);
+    out(j0 + 8, 2 * cq, acc[2] + acl[2]);
+    out(j0 + 8, 2 * cq + 1, acc[3] + acl[3]);
   }
 }
 
-// D = 128: x[h][n] = sum_c M^T[n][c] o_t[h][c] / L_h (the sign is applied at the fp16
-// store), with M^T held like M above; o_t (fp32) enters as an fp16 hi + lo pair, so
-// three products per step (hi.hi, hi.lo, lo.hi) keep ~2^-22 relative precision.
-__device__ __forceinline__ void unrotate_out_mma(const float* om, int heads, const float* Lh, const uint8_t* srot,
-                                                 float* xb, int warp, int lane) {
+// D = 128: q_t[h][c] = (dg / lambda)_c X[slot(c)][h] with X = F128 (s (.) q_h).
+__device__ __forceinline__ void rotate_query_f128(const uint16_t* qs, int heads, const uint32_t* ksg, const float* kch,
+                                                  const uint8_t* srot, float* qt, int warp, int lane) {
+  f128_forward(qs, heads, [&](int) { return ksg; }, srot, warp, lane, [&](int j, int h, float v) {
+    const int c = chan_of_slot128(j);
+    qt[h * 128 + c] = kch[c] * v;
+  });
+}
+
+// D = 128: x[h][n] = sum_j F128[j][n] Z[h][j] with Z[h][slot(c)] = (dg / lambda)_c o_t[h][c] / L_h
+// (the sign is applied at the fp16 store); Z (fp32) enters as an fp16 hi + lo pair, so
+// three products per step (hi.hi, hi.lo, lo.hi) keep ~2^-22 relative precision. A =
+// F128^T by ldmatrix.trans of the resident F128. Called by the four consumer warps.
+__device__ __forceinline__ void unrotate_out_f128(const float* om, int heads, const float* Lh, const float* vch,
+                                                  const uint8_t* srot, float* xb, int warp, int lane) {
   const int g = lane >> 2, cq = lane & 3;
   const int mi = lane >> 3;
   const float L = g < heads ? Lh[g] : 0.0f;
@@ -237,8 +256,9 @@ __device__ __forceinline__ void unrotate_out_mma(const float* om, int heads, con
   for (int ks = 0; ks < 8; ++ks) {
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const int k0 = 16 * ks + 2 * cq + 8 * e;
-      const float v0 = orow[k0] * r, v1 = orow[k0 + 1] * r;
+      const int j0 = 16 * ks + 2 * cq + 8 * e;
+      const int c0 = chan_of_slot128(j0), c1 = chan_of_slot128(j0 + 1);
+      const float v0 = orow[c0] * vch[c0] * r, v1 = orow[c1] * vch[c1] * r;
       const __half h0 = __float2half_rn(v0), h1 = __float2half_rn(v1);
       const __half l0 = __float2half_rn(v0 - __half2float(h0)), l1 = __float2half_rn(v1 - __half2float(h1));
       bh[ks][e] = g < heads ? h2_bits(__halves2half2(h0, h1)) : 0u;
@@ -250,15 +270,16 @@ __device__ __forceinline__ void unrotate_out_mma(const float* om, int heads, con
     const int mt = 2 * warp + t;  // samples 16 mt .. 16 mt + 15
     // the three products in separate accumulators: short dependency chains
     float acc[4] = {0.f, 0.f, 0.f, 0.f}, ahl[4] = {0.f, 0.f, 0.f, 0.f}, alh[4] = {0.f, 0.f, 0.f, 0.f};
-    const int row = 16 * mt + ((mi & 1) << 3) + (lane & 7);
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
-      const int col = 16 * ks + ((mi >> 1) << 3);
+      // A = F128^T (rows n, columns j): transposed 8x8 blocks of F128 rows j
+      const int jrow = 16 * ks + ((mi >> 1) << 3) + (lane & 7);
+      const int ncol = 16 * mt + ((mi & 1) << 3);
       uint32_t a0, a1, a2, a3;
-      ldmatrix_x4(a0, a1, a2, a3, rot_addr(srot, 0, row, col));
+      ldmatrix_x4_trans(a0, a1, a2, a3, rot_addr(srot, 0, jrow, ncol));
       mma_16816(acc, a0, a1, a2, a3, bh[ks][0], bh[ks][1]);
       mma_16816(ahl, a0, a1, a2, a3, bl[ks][0], bl[ks][1]);
-      ldmatrix_x4(a0, a1, a2, a3, rot_addr(srot, 1, row, col));
+      ldmatrix_x4_trans(a0, a1, a2, a3, rot_addr(srot, 1, jrow, ncol));
       mma_16816(alh, a0, a1, a2, a3, bh[ks][0], bh[ks][1]);
     }
 #pragma unroll
@@ -516,8 +537,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kScratch + C::kQt + C::kQs + C::kConsts + C::kQf);
   uint64_t* empty = full + C::kStages;
   uint64_t* cbar = empty + C::kStages;
-  uint64_t* ubar = cbar + 1;  // un-rotation matrix landed (D = 128 int4)
-  uint64_t* rdy = ubar + 1;   // cluster peers: the leader has read this CTA's partial
+  uint64_t* rdy = cbar + 1;   // cluster peers: the leader has read this CTA's partial
   uint64_t* got = rdy + 1;    // cluster leader: every peer's partial is complete
   int* flag = reinterpret_cast<int*>(got + 1);
   uint8_t* srot = smem + C::kRotOff;
@@ -542,7 +562,6 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
       mbar_init(&empty[s], kCWarps);
     }
     mbar_init(cbar, 1);
-    mbar_init(ubar, 1);
     mbar_init(rdy, 1);
     mbar_init(got, cluster_nctarank() > 1 ? cluster_nctarank() - 1 : 1);
     fence_mbarrier_init();
@@ -568,7 +587,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
 #pragma unroll
       for (int hl = 0; hl < 2; ++hl)
 #pragma unroll
-        for (int kc = 0; kc < 2; ++kc) tma_load_2d(srot + (2 * hl + kc) * 16384, &J.rqmap, cbar, 64 * kc, 128 * hl);
+        for (int kc = 0; kc < 2; ++kc) tma_load_2d(srot + (2 * hl + kc) * 16384, &J.rotmap, cbar, 64 * kc, 128 * hl);
     }
     prefetch_tensormap(&J.kmap);
     prefetch_tensormap(&J.vmap);
@@ -638,7 +657,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
       ok = false;
     }
     if constexpr (C::kMmaRot && D == 128) {
-      rotate_query_mma(qs, heads, ksg, srot, qt, warp, lane);
+      rotate_query_f128(qs, heads, ksg, kch, srot, qt, warp, lane);
     } else if constexpr (C::kMmaRot) {
       rotate_query_eo<kCWarps>(qs, heads, ksg, kch, srot, reinterpret_cast<float*>(qf), qt, warp, lane);
     } else {
@@ -649,19 +668,6 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
       }
     }
     consumer_sync<kCWarps>();
-    if constexpr (C::kMmaRot && D == 128) {
-      // the rotation matrix is consumed: a cluster leader (the only CTA that can run the
-      // final merge) prefetches the V plan's un-rotation matrix into the same buffer
-      if (threadIdx.x == 0 && cluster_ctarank() == 0) {
-        fence_proxy_async_smem();
-        mbar_arrive_expect_tx(ubar, (uint32_t)C::kRot);
-#pragma unroll
-        for (int hl = 0; hl < 2; ++hl)
-#pragma unroll
-          for (int kc = 0; kc < 2; ++kc) tma_load_2d(srot + (2 * hl + kc) * 16384, &J.rumap, ubar, 64 * kc, 128 * hl);
-      }
-    }
-
     // (2) B fragments of the score product (n = head g), built once per CTA into
     // shared memory (warp w takes k steps w, w + 4, ...)
     constexpr int kKSteps = C::kKSteps;
@@ -1110,9 +1116,6 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
     }
     __syncthreads();
   };
-  // (D = 128 int4) the leader's un-rotation matrix prefetch must land before the CTA may exit
-  bool rot_ok = true;
-  if constexpr (C::kMmaRot && D == 128) rot_ok = mbar_wait_bounded(ubar, 0);
   // the producer warp reads staged constants below: observe their barrier too
   if (warp == kCWarps && !mbar_wait_bounded(cbar, 0)) atomicOr(&g_attend_err, kErrTimeoutLoad);
 
@@ -1144,9 +1147,8 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
   // ------------------------------------------------------------ normalise, un-rotate, store fp16
   uint16_t* ob = J.out + ((size_t)b * p.Hq + hq0) * D;
   if constexpr (C::kMmaRot) {
-    if (!rot_ok && threadIdx.x == 0) atomicOr(&g_attend_err, kErrTimeoutLoad);
     if constexpr (D == 128) {
-      if (warp < kCWarps) unrotate_out_mma(om, heads, mrg + kHT, srot, xb, warp, lane);
+      if (warp < kCWarps) unrotate_out_f128(om, heads, mrg + kHT, vch, srot, xb, warp, lane);
     } else {
       unrotate_out_eo<kCWarps>(om, heads, mrg + kHT, vch, srot, reinterpret_cast<float*>(qf), xb, warp, lane);
     }
@@ -1361,24 +1363,12 @@ kvq_status make_job(const AttendJobHost& h, int B, int Hkv, int T_cap, AttnJob* 
     j->ksmap = j->kmap;
     j->vsmap = j->vmap;
   }
-  if constexpr (INT4 && D == 256) {
+  if constexpr (INT4) {
     const uint64_t rd[2] = {128u, 256u};
     const uint64_t rs[1] = {256u};
     const uint32_t rb[2] = {64u, 128u};
-    st = encode_tiled(&j->rqmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h.pk->rq_dev, rd, rs, rb,
+    st = encode_tiled(&j->rotmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h.pk->rot_dev, rd, rs, rb,
                       CU_TENSOR_MAP_SWIZZLE_128B, "F128");
-    if (st != KVQ_OK) return st;
-    j->rumap = j->rqmap;
-  }
-  if constexpr (INT4 && D == 128) {
-    const uint64_t rd[2] = {128u, 256u};
-    const uint64_t rs[1] = {256u};
-    const uint32_t rb[2] = {64u, 128u};
-    st = encode_tiled(&j->rqmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h.pk->rq_dev, rd, rs, rb,
-                      CU_TENSOR_MAP_SWIZZLE_128B, "K rotation");
-    if (st == KVQ_OK)
-      st = encode_tiled(&j->rumap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, h.pv->ru_dev, rd, rs, rb,
-                        CU_TENSOR_MAP_SWIZZLE_128B, "V un-rotation");
     if (st != KVQ_OK) return st;
   }
   j->q = h.q;

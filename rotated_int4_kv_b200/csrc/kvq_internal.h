@@ -38,12 +38,10 @@ struct kvq_plan {
   // Tensor-core encode operand in the same block: W = Lambda F_r diag(s) as fp16
   // hi + lo, per 128-channel half 128 hi rows then 128 lo rows, D columns.
   const uint16_t* wt_dev = nullptr;
-  // Attention operands in the same block, fp16 hi rows [128] then lo rows [128]:
-  // D = 128: rq = Lambda^-1 F_r (rows: rotated channels, columns: samples) rotates a
-  // (signed) query; ru = rq^T un-rotates an output (the sign is applied separately).
-  // D = 256: rq = the unnormalised 128-point real DFT in slot order (ru unused).
-  const uint16_t* rq_dev = nullptr;
-  const uint16_t* ru_dev = nullptr;
+  // Attention operand in the same block: F128, the unnormalised 128-point real DFT in
+  // slot order, fp16 hi rows [128] then lo rows [128] (plan-independent; the attention
+  // kernels apply the plans' signs and per-channel factors around it).
+  const uint16_t* rot_dev = nullptr;
 };
 
 namespace kvq {
