@@ -184,6 +184,28 @@ kvq_status kvq_attend_decode(const kvq_plan* pk, const kvq_plan* pv, const uint1
                              size_t ws_bytes, void* stream);
 
 /*
+ * kvq_attend_decode_append -- one decode step of one layer in one launch: the new
+ * token's K and V rows are encoded into the caches at token `pos` (exactly what
+ * kvq_encode with n = 1 at `pos` stores, up to fp32 rounding of the transform: a
+ * code may differ only where the pre-rounding value lies at a rounding boundary),
+ * and the query attends over tokens 0 .. pos, the new one included, as
+ * kvq_attend_decode with T_len = pos + 1 (the SURVEY's "fused append"; the pages
+ * encode each new token with the same fused kernel as a prefill, [M2]).
+ *   k_new, v_new   fp16 [B, Hkv, D], the new token's rows (original domain).
+ *   k_codes, k_scales, v_codes, v_scales   the caches as in kvq_attend_decode,
+ *              written at token pos (every (b, kv head)), read at tokens < pos.
+ *   pos        0 <= pos < T_cap, the same for every batch entry.
+ *   q, out, softmax_scale, workspace   as in kvq_attend_decode.
+ * The other tokens of the caches are only read. Errors: as kvq_attend_decode;
+ * CAPACITY when pos >= T_cap.
+ */
+kvq_status kvq_attend_decode_append(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q,
+                                    const uint16_t* k_new, const uint16_t* v_new, uint8_t* k_codes,
+                                    uint16_t* k_scales, uint8_t* v_codes, uint16_t* v_scales, int B,
+                                    int Hq, int Hkv, int T_cap, int pos, float softmax_scale,
+                                    uint16_t* out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
  * kvq_attend_decode_batch -- kvq_attend_decode for many independent problems of one
  * shape in one grouped launch (up to 32 per launch; more are run as consecutive
  * launches on the stream), e.g. the decode attention of every layer of a model

@@ -159,6 +159,34 @@ def attend_decode(pk: Plan, pv: Plan, q, k_codes, k_scales, v_codes, v_scales, s
     return out
 
 
+def attend_decode_append(pk: Plan, pv: Plan, q, k_new, v_new, k_codes, k_scales, v_codes, v_scales, pos: int,
+                         softmax_scale: float = 0.0, out=None, workspace=None, stream=None) -> torch.Tensor:
+    """One decode step in one launch: encode the new token's K and V rows (fp16
+    [B, Hkv, D] or [B, Hkv, 1, D]) into the caches at token ``pos`` and attend over
+    tokens 0 .. pos (see kvq_attend_decode_append)."""
+    B, Hq, D = q.shape
+    _, Hkv, T_cap, _ = k_codes.shape
+    _need(q, "q", torch.float16)
+    for name, t in (("k_new", k_new), ("v_new", v_new)):
+        if tuple(t.shape) not in ((B, Hkv, D), (B, Hkv, 1, D)):
+            raise ValueError(f"{name}: expected shape {(B, Hkv, D)}, got {tuple(t.shape)}")
+        _need(t, name, torch.float16)
+    for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
+        _need(t, name, torch.uint8, (B, Hkv, T_cap, D // 2))
+    for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+        _need(t, name, torch.float16, (B, Hkv, T_cap, D // pk.group))
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float16, device=q.device)
+    _need(out, "out", torch.float16, (B, Hq, D))
+    if workspace is None:
+        workspace = make_workspace(B, Hq, Hkv, D, T_cap, q.device)
+    check(lib.kvq_attend_decode_append(pk.handle, pv.handle, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_codes),
+                                       _ptr(k_scales), _ptr(v_codes), _ptr(v_scales), B, Hq, Hkv, T_cap, int(pos),
+                                       float(softmax_scale), _ptr(out), _ptr(workspace), workspace.numel(),
+                                       _stream(stream)), "kvq_attend_decode_append")
+    return out
+
+
 def attend_decode_batch(jobs, seq_lens=None, T_len=None, softmax_scale: float = 0.0, workspace=None,
                         stream=None) -> list:
     """Grouped int4 decode attention: ``jobs`` is a sequence of

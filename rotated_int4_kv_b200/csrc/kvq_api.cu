@@ -408,6 +408,29 @@ kvq_status kvq_attend_decode(const kvq_plan* pk, const kvq_plan* pv, const uint1
                                  ws_bytes, (cudaStream_t)stream);
 }
 
+kvq_status kvq_attend_decode_append(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q, const uint16_t* k_new,
+                                    const uint16_t* v_new, uint8_t* kc, uint16_t* ks, uint8_t* vc, uint16_t* vs, int B,
+                                    int Hq, int Hkv, int T_cap, int pos, float sigma, uint16_t* out, void* ws,
+                                    size_t ws_bytes, void* stream) {
+  if (!pk || !pv) return fail(KVQ_ERR_INVALID_ARG, "attend_append: null plan");
+  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device)
+    return fail(KVQ_ERR_INVALID_ARG, "attend_append: K and V plans differ in head_dim, group or device");
+  if (pk->G != 32) return fail(KVQ_ERR_UNSUPPORTED, "attend_append: group must be 32");
+  if (pos < 0) return fail(KVQ_ERR_INVALID_ARG, "attend_append: pos < 0");
+  if (pos >= T_cap) return fail(KVQ_ERR_CAPACITY, "attend_append: pos + 1 > T_cap");
+  kvq_status st = check_attend_common(B, Hq, Hkv, pk->D, T_cap, pos + 1, q, out, ws, ws_bytes);
+  if (st != KVQ_OK || B == 0) return st;
+  if (!kc || !ks || !vc || !vs) return fail(KVQ_ERR_INVALID_ARG, "attend_append: null cache buffer");
+  if (!k_new || !v_new) return fail(KVQ_ERR_INVALID_ARG, "attend_append: null new K/V row");
+  if (!kvq::aligned16(kc) || !kvq::aligned16(ks) || !kvq::aligned16(vc) || !kvq::aligned16(vs) ||
+      !kvq::aligned16(k_new) || !kvq::aligned16(v_new))
+    return fail(KVQ_ERR_ALIGNMENT, "attend_append: buffers must be 16-byte aligned");
+  st = kvq::check_plan_device(pk);
+  if (st != KVQ_OK) return st;
+  return kvq::launch_attend_int4_append(pk, pv, q, k_new, v_new, kc, ks, vc, vs, B, Hq, Hkv, T_cap, pos, sigma, out,
+                                        ws, ws_bytes, (cudaStream_t)stream);
+}
+
 kvq_status kvq_attend_decode_batch(const kvq_attend_job* jobs, int njobs, int B, int Hq, int Hkv, int T_cap,
                                    const int32_t* seq_lens, int T_len, float sigma, void* ws, size_t ws_bytes,
                                    void* stream) {

@@ -41,6 +41,7 @@
 #include "kvq_internal.h"
 
 #include "kvq_ptx.cuh"
+#include "kvq_quant.cuh"
 
 namespace kvq {
 
@@ -95,11 +96,15 @@ struct Cfg {
   // (hi01, hi23, lo01, lo23) -- read from shared memory at each use
   static constexpr int kKSteps = INT4 ? 2 * NG : D / 16;
   static constexpr int kQf = kKSteps * 32 * 16;
+  // fused append: the new K and V rows (fp16 [2][D]); at D = 128 they are staged in the
+  // B-fragment buffer (built only after the append's encode), at D = 256 (whose query
+  // rotation uses that buffer as scratch) in a region of their own
+  static constexpr int kApp = (INT4 && D == 256) ? 2 * D * 2 : 0;
   static constexpr int kBars = 128;        // full[], empty[], const, rotation, cluster rdy / got barriers, flag
   // D = 128 int4: the plan's rotation matrix (hi, lo) for the query, then the V plan's
   // transpose for the output, as [hi/lo][64-column chunk][128 rows][128 B] (128-byte swizzle)
   static constexpr bool kMmaRot = INT4;   // F128 (D = 256: even/odd split)
-  static constexpr int kRotOff = (kScratch + kQt + kQs + kConsts + kQf + kBars + 1023) / 1024 * 1024;
+  static constexpr int kRotOff = (kScratch + kQt + kQs + kConsts + kQf + kApp + kBars + 1023) / 1024 * 1024;
   static constexpr int kRot = kMmaRot ? 4 * 128 * 128 : 0;
   static constexpr int kSmem = kRotOff + kRot + 1024;
   static_assert(2 * kStages * 8 + 3 * 8 + 4 <= kBars, "barrier region");
@@ -114,6 +119,17 @@ struct AttnParams {
   float sl2;                                   // softmax scale * log2(e)
   float* part;                                 // [units][S][2*8 + 8*D]
   int* cnt;                                    // [units]
+  // fused append (single-problem int4 launches; append_pos < 0: none): the new token's
+  // K and V rows (fp16 [B][Hkv][D]) are encoded into the caches at token append_pos by
+  // the last split of every unit, which also adds that token to its partial; the
+  // splits stream tokens [0, T_len) with T_len = append_pos.
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  uint8_t* kc_out;
+  uint16_t* ks_out;
+  uint8_t* vc_out;
+  uint16_t* vs_out;
+  int append_pos;
 };
 
 // One attention problem of a launch: its caches (as tensor maps), query, output
@@ -296,28 +312,32 @@ __device__ __forceinline__ void unrotate_out_f128(const float* om, int heads, co
   }
 }
 
-// D = 256 by one radix-2 decimation in time: E = F128 q'_even, O = F128 q'_odd on the
+// D = 256 by one radix-2 decimation in time: E = F128 x'_even, O = F128 x'_odd on the
 // tensor cores (F128 = the unnormalised 128-point real DFT in slot order, fp16 hi + lo
 // in shared memory, same layout as above), then X_k = E_k + W^k O_k, X_{128-k} =
-// conj(E_k - W^k O_k) (W = e^{-2 pi i / 256}) and q_t[c] = (dg / lambda)_c X(c).
-// eo: fp32 scratch [E, O][8 heads][128 slots]. Called by the four consumer warps.
-template <int NW>
-__device__ __forceinline__ void rotate_query_eo(const uint16_t* qs, int heads, const uint32_t* ksg, const float* kch,
-                                                const uint8_t* srot, float* eo, float* qt, int warp, int lane) {
+// conj(E_k - W^k O_k) (W = e^{-2 pi i / 256}); out(c, r, X(c)) for every channel c and
+// every row r < 8 (0 for rows past nrows), X(c) in the real basis' slot of channel c
+// (before its factor dg_c). x'_r = x_r with the sign mask sgn_of(r) applied. eo: fp32
+// scratch [E, O][8 rows][128 slots]. Called by the NW consumer warps.
+template <int NW, typename SgnOf, typename Out>
+__device__ __forceinline__ void f256_forward(const uint16_t* rows, int nrows, SgnOf sgn_of, const uint8_t* srot,
+                                             float* eo, int warp, int lane, Out out) {
   const int g = lane >> 2, cq = lane & 3;
   const int mi = lane >> 3;
   {
-    // B fragments (k = m, n = head g): even samples 2m and odd samples 2m + 1 of q' = s (.) q
+    // B fragments (k = m, n = row g): even samples 2m and odd samples 2m + 1 of x'
     uint32_t be[8][2], bo[8][2];
-    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(qs + (g < heads ? g : 0) * 256);
+    const int gr = g < nrows ? g : 0;
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(rows + gr * 256);
+    const uint32_t* sg = sgn_of(gr);
 #pragma unroll
     for (int ks = 0; ks < 8; ++ks) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int m0 = 16 * ks + 2 * cq + 8 * e;  // words m0, m0 + 1 hold samples 2 m0 .. 2 m0 + 3
-        const uint32_t wa = qrow[m0] ^ ksg[m0], wb = qrow[m0 + 1] ^ ksg[m0 + 1];
-        be[ks][e] = g < heads ? prmt(wa, wb, 0x5410u) : 0u;
-        bo[ks][e] = g < heads ? prmt(wa, wb, 0x7632u) : 0u;
+        const uint32_t wa = qrow[m0] ^ sg[m0], wb = qrow[m0 + 1] ^ sg[m0 + 1];
+        be[ks][e] = g < nrows ? prmt(wa, wb, 0x5410u) : 0u;
+        bo[ks][e] = g < nrows ? prmt(wa, wb, 0x7632u) : 0u;
       }
     }
 #pragma unroll
@@ -380,11 +400,10 @@ __device__ __forceinline__ void rotate_query_eo(const uint16_t* qs, int heads, c
     slot_im = (k == 0 || k == 64) ? -1 : 2 * k + 1;
     float sn, cs;
     sincospif((float)k / 128.0f, &sn, &cs);
-    const float f = kch[ch];
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
       float v = 0.0f;
-      if (h < heads) {
+      if (h < nrows) {
         const float* E = eo + h * 128;
         const float* O = eo + 1024 + h * 128;
         const float er = E[slot_re], orr = O[slot_re];
@@ -396,11 +415,19 @@ __device__ __forceinline__ void rotate_query_eo(const uint16_t* qs, int heads, c
         }
         const float xr = mirror ? er - tr : er + tr;
         const float xi = mirror ? ti - ei : ei + ti;
-        v = (re ? xr : xi) * f;
+        v = re ? xr : xi;
       }
-      qt[h * 256 + ch] = v;
+      out(ch, h, v);
     }
   }
+}
+
+// D = 256: q_t[h][c] = (dg / lambda)_c X(c) with X = F256 (s (.) q_h) by the even/odd split.
+template <int NW>
+__device__ __forceinline__ void rotate_query_eo(const uint16_t* qs, int heads, const uint32_t* ksg, const float* kch,
+                                                const uint8_t* srot, float* eo, float* qt, int warp, int lane) {
+  f256_forward<NW>(qs, heads, [&](int) { return ksg; }, srot, eo, warp, lane,
+                   [&](int c, int h, float v) { qt[h * 256 + c] = v * kch[c]; });
 }
 
 // Transpose of rotate_query_eo for the output (sign applied at the fp16 store):
@@ -534,7 +561,9 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
   const float* vch = reinterpret_cast<const float*>(cst + C::kChanBytes + C::kSgnBytes);
   const uint32_t* vsg = reinterpret_cast<const uint32_t*>(cst + 2 * C::kChanBytes + C::kSgnBytes);
   uint4* qf = reinterpret_cast<uint4*>(smem + C::kScratch + C::kQt + C::kQs + C::kConsts);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kScratch + C::kQt + C::kQs + C::kConsts + C::kQf);
+  uint16_t* app_in = reinterpret_cast<uint16_t*>(D == 128 ? smem + C::kScratch + C::kQt + C::kQs + C::kConsts
+                                                                : smem + C::kScratch + C::kQt + C::kQs + C::kConsts + C::kQf);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kScratch + C::kQt + C::kQs + C::kConsts + C::kQf + C::kApp);
   uint64_t* empty = full + C::kStages;
   uint64_t* cbar = empty + C::kStages;
   uint64_t* rdy = cbar + 1;   // cluster peers: the leader has read this CTA's partial
@@ -553,6 +582,8 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
   const int heads = min(kHT, p.G - ht * kHT);  // real heads in this tile
   const int hq0 = kvh * p.G + ht * kHT;        // first query head
   const int unit = (int)blockIdx.z * p.HT + ht;  // workspace slot (over all jobs)
+  // fused append: the last split of the unit encodes and adds the new token
+  const bool app = INT4 && p.append_pos >= 0 && split == p.S - 1;
 
   const int row0 = bk * p.T_cap;  // first cache row of this (b, kv head)
 
@@ -576,7 +607,8 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
     // not wait for the previous kernel: staged while it finishes. The query rows come
     // on the same barrier after the wait below.
     const uint32_t qbytes = (uint32_t)(heads * D * 2);
-    mbar_arrive_expect_tx(cbar, qbytes + (INT4 ? (uint32_t)C::kConsts : 0u) + (uint32_t)C::kRot);
+    mbar_arrive_expect_tx(cbar, qbytes + (INT4 ? (uint32_t)C::kConsts : 0u) + (uint32_t)C::kRot +
+                                    (app ? (uint32_t)(2 * D * 2) : 0u));
     if constexpr (INT4) {
       bulk_load(cst, J.kd->chan, C::kChanBytes, cbar);
       bulk_load(cst + C::kChanBytes, J.ke->sgn, C::kSgnBytes, cbar);
@@ -619,6 +651,10 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
     if (lane == 0) {
       // the query rows of the tile (their bytes are in the barrier's count already)
       bulk_load(qs, J.q + ((size_t)b * p.Hq + hq0) * D, (uint32_t)(heads * D * 2), cbar);
+      if (app) {  // the new K and V rows of this (b, kv head)
+        bulk_load(app_in, p.k_new + (size_t)bk * D, (uint32_t)(D * 2), cbar);
+        bulk_load(app_in + D, p.v_new + (size_t)bk * D, (uint32_t)(D * 2), cbar);
+      }
       for (int i = 0; i < ntiles; ++i) {
         const int s = i % C::kStages;
         if (i >= C::kStages) {
@@ -668,6 +704,68 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
       }
     }
     consumer_sync<kCWarps>();
+    // (1b) fused append: encode the new K and V rows with the resident F128 (the plans'
+    // signs, then the factors lambda dg = dg^2 / (dg / lambda)), quantise them as the
+    // encode kernels do, write them into the caches at append_pos (query-head tile 0 of
+    // the unit), and keep the dequantised rows (rotated domain) and the new token's
+    // base-2 scores per head for the end of the token loop (in qs, consumed by now)
+    float* ybuf = reinterpret_cast<float*>(qs);  // [K, V][D] fp32, then [8] scores
+    if constexpr (INT4) {
+      if (app) {
+        auto sgn_of = [&](int r) { return r ? vsg : ksg; };
+        auto enc_f = [&](int r, int c) {
+          const float d2 = (c == 0 || c == D - 1) ? 1.0f / D : 2.0f / D;
+          return d2 / (r ? vch[c] : kch[c]);
+        };
+        if constexpr (D == 128) {
+          f128_forward(app_in, 2, sgn_of, srot, warp, lane, [&](int j, int r, float v) {
+            if (r < 2) {
+              const int c = chan_of_slot128(j);
+              ybuf[r * D + c] = v * enc_f(r, c);
+            }
+          });
+        } else {
+          f256_forward<kCWarps>(app_in, 2, sgn_of, srot, reinterpret_cast<float*>(qf), warp, lane,
+                                [&](int c, int r, float v) {
+                                  if (r < 2) ybuf[r * D + c] = v * enc_f(r, c);
+                                });
+        }
+        consumer_sync<kCWarps>();
+        if (threadIdx.x < 2 * NG) {
+          const int r = threadIdx.x / NG, grp = threadIdx.x - r * NG;
+          float* yg = ybuf + r * D + 32 * grp;
+          float y[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) y[i] = yg[i];
+          uint32_t wd[4], sb;
+          quantize_group<32>(y, wd, sb);
+          if (ht == 0) {
+            const size_t crow = (size_t)bk * p.T_cap + p.append_pos;
+            *reinterpret_cast<uint4*>((r ? p.vc_out : p.kc_out) + crow * (D / 2) + 16 * grp) =
+                make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            (r ? p.vs_out : p.ks_out)[crow * NG + grp] = (uint16_t)sb;
+          }
+          const float sc = __half2float(__ushort_as_half((unsigned short)sb));
+#pragma unroll
+          for (int w = 0; w < 4; ++w) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int nib = (int)((wd[w] >> (4 * e)) & 15u);
+              yg[8 * w + e] = (float)(nib >= 8 ? nib - 16 : nib) * sc;
+            }
+          }
+        }
+        consumer_sync<kCWarps>();
+        for (int h = warp; h < kHT; h += kCWarps) {
+          float acc = 0.0f;
+          for (int c2 = lane; c2 < D; c2 += 32) acc = fmaf(qt[h * D + c2], ybuf[c2], acc);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+          if (lane == 0) ybuf[2 * D + h] = acc * p.sl2;
+        }
+        consumer_sync<kCWarps>();
+      }
+    }
     // (2) B fragments of the score product (n = head g), built once per CTA into
     // shared memory (warp w takes k steps w, w + 4, ...)
     constexpr int kKSteps = C::kKSteps;
@@ -924,6 +1022,31 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
     for (int off = 4; off < 32; off <<= 1) {
       l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
       l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
+    }
+    if constexpr (INT4) {
+      if (app && warp == 0) {
+        // the appended token: one more element of warp 0's online softmax (scores and
+        // dequantised V row from (1b); l is the warp total here, so every lane adds p)
+        const float* vhat = ybuf + D;
+        float pn[2], al[2];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float sn = ybuf[2 * D + 2 * c + e];
+          const float mn = fmaxf(m_run[e], sn);
+          al[e] = m_run[e] == -INFINITY ? 0.0f : fast_exp2(m_run[e] - mn);
+          pn[e] = fast_exp2(sn - mn);
+          l_run[e] = fmaf(l_run[e], al[e], pn[e]);
+          m_run[e] = mn;
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+          const int ch0 = (mt >> 1) * 32 + 4 * g + ((mt & 1) ? 2 : 0), ch1 = ch0 + 1;
+          o_acc[mt][0] = fmaf(o_acc[mt][0], al[0], pn[0] * vhat[ch0]);
+          o_acc[mt][1] = fmaf(o_acc[mt][1], al[1], pn[1] * vhat[ch0]);
+          o_acc[mt][2] = fmaf(o_acc[mt][2], al[0], pn[0] * vhat[ch1]);
+          o_acc[mt][3] = fmaf(o_acc[mt][3], al[1], pn[1] * vhat[ch1]);
+        }
+      }
     }
   }
   (void)ok;  // a timed-out CTA still takes part in every barrier below; its flag reaches the host
@@ -1379,10 +1502,23 @@ kvq_status make_job(const AttendJobHost& h, int B, int Hkv, int T_cap, AttnJob* 
   return KVQ_OK;
 }
 
-// One launch over nj <= MAXJ problems of equal shape.
+// The fused append of a single-problem launch: the new K and V rows and where they go.
+struct AppendHost {
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  uint8_t* kc;
+  uint16_t* ks;
+  uint8_t* vc;
+  uint16_t* vs;
+  int pos;
+};
+
+// One launch over nj <= MAXJ problems of equal shape (with app: the fused append, T_len =
+// the tokens already cached = app->pos).
 template <int D, bool INT4, int MAXJ>
 kvq_status launch_chunk(const AttendJobHost* jobs, int nj, int B, int Hq, int Hkv, int T_cap, const int32_t* seq_lens,
-                        int T_len, float sigma, void* ws, size_t ws_bytes, cudaStream_t strm) {
+                        int T_len, float sigma, void* ws, size_t ws_bytes, cudaStream_t strm,
+                        const AppendHost* app = nullptr) {
   using C = Cfg<D, INT4>;
   const int T_split = seq_lens ? T_cap : T_len;
   const int Bj = nj * B;  // the jobs of a launch split like a larger batch
@@ -1411,6 +1547,16 @@ kvq_status launch_chunk(const AttendJobHost* jobs, int nj, int B, int Hq, int Hk
   char* wsb = reinterpret_cast<char*>(ws);
   prm.cnt = reinterpret_cast<int*>(wsb);
   prm.part = reinterpret_cast<float*>(wsb + ws_cnt_bytes(units));
+  prm.append_pos = -1;
+  if (app) {
+    prm.k_new = app->k_new;
+    prm.v_new = app->v_new;
+    prm.kc_out = app->kc;
+    prm.ks_out = app->ks;
+    prm.vc_out = app->vc;
+    prm.vs_out = app->vs;
+    prm.append_pos = app->pos;
+  }
   dim3 grid(sp.S, sp.HT, Bj * Hkv);
   if (grid.z > 65535u) return fail(KVQ_ERR_UNSUPPORTED, "attend: jobs * B * Hkv > 65535");
   cudaLaunchConfig_t cfg{};
@@ -1477,6 +1623,17 @@ kvq_status launch_attend_int4_batch(const AttendJobHost* jobs, int njobs, int B,
   if (jobs[0].pk->D == 128)
     return run_attend<128, true>(jobs, njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
   return run_attend<256, true>(jobs, njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
+}
+
+kvq_status launch_attend_int4_append(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q, const uint16_t* k_new,
+                                     const uint16_t* v_new, uint8_t* kc, uint16_t* ks, uint8_t* vc, uint16_t* vs, int B,
+                                     int Hq, int Hkv, int T_cap, int pos, float sigma, uint16_t* out, void* ws,
+                                     size_t ws_bytes, cudaStream_t s) {
+  const AttendJobHost job{pk, pv, q, kc, ks, vc, vs, out};
+  const AppendHost app{k_new, v_new, kc, ks, vc, vs, pos};
+  if (pk->D == 128)
+    return launch_chunk<128, true, 1>(&job, 1, B, Hq, Hkv, T_cap, nullptr, pos, sigma, ws, ws_bytes, s, &app);
+  return launch_chunk<256, true, 1>(&job, 1, B, Hq, Hkv, T_cap, nullptr, pos, sigma, ws, ws_bytes, s, &app);
 }
 
 kvq_status launch_attend_fp16(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq, int Hkv, int D,

@@ -21,7 +21,7 @@ def test_header_declares_the_boundary():
     for n in ("kvq_plan_create", "kvq_plan_destroy", "kvq_encode", "kvq_encode_batch", "kvq_decode",
               "kvq_workspace_size", "kvq_attend_decode", "kvq_attend_decode_ref", "kvq_status_string",
               "kvq_last_error", "kvq_poll_device_errors", "kvq_attend_decode_batch",
-              "kvq_attend_decode_noalloc"):
+              "kvq_attend_decode_noalloc", "kvq_attend_decode_append"):
         assert n in names
 
 
@@ -47,6 +47,9 @@ def test_status_strings_and_host_checks():
                                  ctypes.c_float(0), None, None, 0, None) == -1
     assert lib.kvq_attend_decode_ref(None, None, None, 1, 4, 1, 100, 64, None, 64, ctypes.c_float(0), None, None,
                                      0, None) == -2
+    assert lib.kvq_attend_decode_append(None, None, None, None, None, None, None, None, None, 1, 4, 1, 64, 10,
+                                        ctypes.c_float(0), None, None, 0, None) == -1
+    assert b"null plan" in lib.kvq_last_error()
     assert lib.kvq_encode_batch(None, -1, None) == -1
     assert lib.kvq_encode_batch(None, 0, None) == 0
     assert lib.kvq_attend_decode_batch(None, -1, 1, 4, 1, 64, None, 64, ctypes.c_float(0), None, 0, None) == -1

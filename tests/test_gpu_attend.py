@@ -245,3 +245,88 @@ def test_attend_batch_rejects_mixed_head_dims(kvq):
             for c, w in ((cg_, g), (cq, q))]
     with pytest.raises(Exception):
         kvq.attend_decode_batch(jobs, T_len=64)
+
+
+APPEND_CASES = [
+    # (workload, B, Hkv, Hq, T_cap, pos): the new token goes to row pos, tokens 0 .. pos attended
+    ("toy", 1, 1, 1, 256, 255),
+    ("qwen", 1, 2, 12, 1026, 1024),
+    ("qwen", 1, 2, 12, 64, 0),                  # empty cache: only the new token
+    ("qwen", 3, 2, 12, 200, 130),               # ragged last stage
+    ("mistral", 2, 8, 32, 700, 513),
+    ("longctx", 1, 1, 16, 200, 77),             # GQA 16: two head tiles append the same token
+    ("gemma", 1, 1, 4, 4098, 4096),             # D = 256
+    ("gemma", 2, 2, 6, 334, 333),               # D = 256, GQA 3
+]
+
+
+@pytest.mark.parametrize("case", APPEND_CASES, ids=[f"{c[0]}-B{c[1]}kv{c[2]}q{c[3]}pos{c[5]}" for c in APPEND_CASES])
+def test_attend_append_matches_encode_then_attend(kvq, case):
+    """kvq_attend_decode_append = kvq_encode of the new token at pos + kvq_attend_decode
+    over pos + 1 tokens: the row it writes passes the encode acceptance rule against the
+    oracle, no other row changes, and its output matches the oracle on the GPU's own
+    cache and the two-call path."""
+    from tests.parity import BOUNDARY_TALLY, check_encode
+
+    wl_name, B, Hkv, Hq, T_cap, pos = case
+    wl = kvgen.WORKLOADS[wl_name]
+    D = wl.head_dim
+    dev = torch.device("cuda")
+    cache = {}
+    for kind in ("k", "v"):
+        s, lam = kvgen.plan_params(D, seed=23, layer=1, kind=kind)
+        plan = kvq.Plan(s, lam)
+        x = kvgen.kv_numpy(wl, kind, (B, Hkv, pos + 1, D), seed=23, layer=1)
+        codes = torch.full((B, Hkv, T_cap, D // 2), 0x5A, dtype=torch.uint8, device=dev)
+        scales = torch.full((B, Hkv, T_cap, D // 32), 3.0, dtype=torch.float16, device=dev)
+        if pos > 0:
+            kvq.encode(plan, torch.from_numpy(np.ascontiguousarray(x[:, :, :pos])).to(dev), codes, scales, 0)
+        cache[kind] = dict(plan=plan, params=(s, lam), x=x, codes=codes, scales=scales,
+                           new=torch.from_numpy(np.ascontiguousarray(x[:, :, pos])).to(dev))
+    q16 = kvgen.q_numpy((B, Hq, D), salt=9)
+    q = torch.from_numpy(q16).to(dev)
+    k, v = cache["k"], cache["v"]
+    # the two-call path on copies of the caches
+    kc2, ks2, vc2, vs2 = (t.clone() for t in (k["codes"], k["scales"], v["codes"], v["scales"]))
+    kvq.encode(k["plan"], k["new"].unsqueeze(2), kc2, ks2, pos)
+    kvq.encode(v["plan"], v["new"].unsqueeze(2), vc2, vs2, pos)
+    out2 = kvq.attend_decode(k["plan"], v["plan"], q, kc2, ks2, vc2, vs2, T_len=pos + 1)
+    before = [t.clone() for t in (k["codes"], k["scales"], v["codes"], v["scales"])]
+    out = kvq.attend_decode_append(k["plan"], v["plan"], q, k["new"], v["new"], k["codes"], k["scales"],
+                                   v["codes"], v["scales"], pos)
+    torch.cuda.synchronize()
+    assert kvq.poll_device_errors() == 0
+    # the appended rows: encode acceptance against the oracle
+    for kind in ("k", "v"):
+        c = cache[kind]
+        s, lam = c["params"]
+        nb, na = check_encode(c["x"][:, :, pos:pos + 1], s, lam, 32, c["codes"][:, :, pos:pos + 1].cpu().numpy(),
+                              c["scales"][:, :, pos:pos + 1].cpu().numpy(), label=f"{case} {kind}", count_only=True)
+        BOUNDARY_TALLY["bad"] += nb
+        BOUNDARY_TALLY["all"] += na
+    # every other row untouched
+    for t_after, t_before in zip((k["codes"], k["scales"], v["codes"], v["scales"]), before):
+        keep = torch.ones(T_cap, dtype=torch.bool, device=dev)
+        keep[pos] = False
+        assert torch.equal(t_after[:, :, keep], t_before[:, :, keep])
+    got = out.cpu().numpy().astype(np.float64)
+    ref = _oracle_int4(q16, cache, [pos + 1] * B)
+    check_rel_l2(got.reshape(-1, D), ref.reshape(-1, D), label=str(case))
+    check_rel_l2(got.reshape(-1, D), out2.cpu().numpy().astype(np.float64).reshape(-1, D), label=f"{case} vs two calls")
+
+
+def test_attend_append_rejects_bad_positions(kvq):
+    wl = kvgen.WORKLOADS["qwen"]
+    D, B, Hkv, Hq, T_cap = wl.head_dim, 1, 2, 12, 64
+    s, lam = kvgen.plan_params(D, kind="k")
+    pk = kvq.Plan(s, lam)
+    pv = kvq.Plan(*kvgen.plan_params(D, kind="v"))
+    dev = torch.device("cuda")
+    q = torch.zeros((B, Hq, D), dtype=torch.float16, device=dev)
+    kn = torch.zeros((B, Hkv, D), dtype=torch.float16, device=dev)
+    codes = torch.zeros((B, Hkv, T_cap, D // 2), dtype=torch.uint8, device=dev)
+    scales = torch.zeros((B, Hkv, T_cap, D // 32), dtype=torch.float16, device=dev)
+    with pytest.raises(kvq.KvqError, match="CAPACITY"):
+        kvq.attend_decode_append(pk, pv, q, kn, kn, codes, scales, codes.clone(), scales.clone(), T_cap)
+    with pytest.raises(kvq.KvqError, match="INVALID_ARG"):
+        kvq.attend_decode_append(pk, pv, q, kn, kn, codes, scales, codes.clone(), scales.clone(), -1)

@@ -6,7 +6,7 @@ import pytest
 
 import kvgen
 import oracle
-from tests.parity import MAX_BOUNDARY_FRAC, check_encode, check_rel_l2
+from tests.parity import BOUNDARY_TALLY, MAX_BOUNDARY_FRAC, check_encode, check_rel_l2
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -44,9 +44,7 @@ CASES = [
 ]
 
 
-# boundary mismatches and elements over every case of this module: the 1e-5 bound
-# applies to the fraction over all elements encoded, not to each small case
-_TALLY = {"bad": 0, "all": 0}
+_TALLY = BOUNDARY_TALLY  # shared with the fused-append tests
 PATHS = ["fft", "tensor"]
 
 
