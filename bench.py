@@ -584,6 +584,29 @@ def run_decode_workload(args, rank: int, world: int):
         })
         del caches, caches16, k16s, v16s
         torch.cuda.empty_cache()
+    stream_enc = None
+    sb = wl.extra.get("stream_batch") if wl.extra else None
+    if sb:
+        # streaming encode: one token per step for each of sb sequences x Hkv heads x {K, V}
+        # (one grouped launch per step; a few MB, so this measures latency, not HBM)
+        pk, pv = (kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=0, kind=k)) for k in ("k", "v"))
+        xk = kvgen.kv_torch(wl, "k", (sb, Hkv, 1, D), dev, seed=seed, layer=0, salt=77)
+        xv = kvgen.kv_torch(wl, "v", (sb, Hkv, 1, D), dev, seed=seed, layer=0, salt=78)
+        kc = torch.zeros((sb, Hkv, 2, D // 2), dtype=torch.uint8, device=dev)
+        ks = torch.zeros((sb, Hkv, 2, D // G), dtype=torch.float16, device=dev)
+        vc, vs = torch.zeros_like(kc), torch.zeros_like(ks)
+        nvec = 2 * sb * Hkv
+        stream_enc = {"sequences": sb, "vectors_per_step": nvec, "l2": "inputs fit in L2: launch latency"}
+        for path in ("tensor", "fft"):
+            kvq.set_encode_path(path)
+            try:
+                ms_e = _graph_time(torch, lambda: kvq.encode_batch([(pk, xk, kc, ks, 0), (pv, xv, vc, vs, 0)]),
+                                   args.steps, args.warmup)
+            finally:
+                kvq.set_encode_path("auto")
+            stream_enc[path] = {"us_per_step": ms_e * 1e3, "ns_per_vec": ms_e * 1e6 / nvec,
+                                "GB_s": nvec * vec_b / (ms_e * 1e-3) / 1e9}
+        assert kvq.poll_device_errors() == 0
     big = cases[-1]
     line = {"metric": METRIC, "value": big["int4_attn_GB_s"], "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": big["int4_step_ms"],
@@ -591,6 +614,8 @@ def run_decode_workload(args, rank: int, world: int):
             "config": {"workload": args.workload, "layers": layers, "kv_heads": Hkv, "q_heads": Hq, "head_dim": D,
                        "batch": B, "contexts": list(contexts), "group": G},
             "cases": cases}
+    if stream_enc is not None:
+        line["streaming_encode"] = stream_enc
     if rank == 0:
         print(json.dumps(line), flush=True)
     return 0
