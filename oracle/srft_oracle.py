@@ -39,6 +39,13 @@ Readings taken where the pages leave a step open:
   * Attention (not on the pages): softmax(sigma <q, x_hat_K>) weighted sum of
     x_hat_V, sigma = 1/sqrt(D) by default; query head h reads KV head
     h // (Hq / Hkv).
+  * SRHT variant ([M1] "Begruendung"/"Ergebnis": the Hadamard transform is the
+    common alternative, statistically indistinguishable in quality; the pages
+    define it no further): R = H_D diag(s) / sqrt(D) with H_D the Sylvester
+    Hadamard matrix in natural order, H[i][j] = (-1)^popcount(i & j); the same
+    sign vector, lambda after the rotation, and the same group, scale, code and
+    pack steps. Every function taking ``transform`` accepts "srft" (default)
+    or "srht".
 
 Parity pins: every function here is checked in ``tests/test_oracle_pins.py``
 against closed forms, brute force and invariants (see that file).
@@ -85,18 +92,45 @@ def srft_matrix(signs: np.ndarray) -> np.ndarray:
     return real_dft_basis(s.shape[0]) * s[None, :]
 
 
-def srft_forward(x: np.ndarray, signs: np.ndarray, lam: np.ndarray) -> np.ndarray:
-    """y = lambda * (F_r . diag(s) . x), over the last axis, in fp64 [M1], [M2]."""
+def hadamard_matrix(D: int) -> np.ndarray:
+    """The Sylvester Hadamard matrix of order D (a power of two), natural order:
+    H_1 = [1], H_2n = [[H_n, H_n], [H_n, -H_n]] (entries +-1, fp64)."""
+    if D < 1 or D & (D - 1):
+        raise ValueError("the Hadamard transform needs a power-of-two length")
+    H = np.ones((1, 1))
+    while H.shape[0] < D:
+        H = np.block([[H, H], [H, -H]])
+    return H
+
+
+def srht_matrix(signs: np.ndarray) -> np.ndarray:
+    """R = H_D . diag(s) / sqrt(D) (the SRHT reading above)."""
+    s = np.asarray(signs, dtype=np.float64)
+    D = s.shape[0]
+    return hadamard_matrix(D) * s[None, :] / math.sqrt(D)
+
+
+def rotation_matrix(signs: np.ndarray, transform: str = "srft") -> np.ndarray:
+    if transform == "srft":
+        return srft_matrix(signs)
+    if transform == "srht":
+        return srht_matrix(signs)
+    raise ValueError(f"unknown transform {transform!r}")
+
+
+def srft_forward(x: np.ndarray, signs: np.ndarray, lam: np.ndarray, transform: str = "srft") -> np.ndarray:
+    """y = lambda * (R . x) over the last axis in fp64, R = F_r diag(s) [M1], [M2]
+    (or the SRHT's H diag(s) / sqrt(D))."""
     x = np.asarray(x, dtype=np.float64)
-    R = srft_matrix(signs)
+    R = rotation_matrix(signs, transform)
     lam64 = np.asarray(lam, dtype=np.float64)
     return (x @ R.T) * lam64
 
 
-def srft_inverse(y: np.ndarray, signs: np.ndarray, lam: np.ndarray) -> np.ndarray:
-    """x = diag(s) . F_r^T . (y / lambda): the exact inverse of srft_forward."""
+def srft_inverse(y: np.ndarray, signs: np.ndarray, lam: np.ndarray, transform: str = "srft") -> np.ndarray:
+    """x = R^T . (y / lambda): the exact inverse of srft_forward."""
     y = np.asarray(y, dtype=np.float64) / np.asarray(lam, dtype=np.float64)
-    R = srft_matrix(signs)
+    R = rotation_matrix(signs, transform)
     return y @ R
 
 
@@ -155,13 +189,13 @@ def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
     return out
 
 
-def encode(x: np.ndarray, signs: np.ndarray, lam: np.ndarray, G: int = 32):
+def encode(x: np.ndarray, signs: np.ndarray, lam: np.ndarray, G: int = 32, transform: str = "srft"):
     """The encode path of [ABS]/[M2] over the last axis.
 
     Returns dict(packed=uint8 [..., D/2], scales=float16 [..., D/G],
     codes=int8 [..., D], y=fp64 [..., D], u=fp64 pre-rounding y/scale).
     """
-    y = srft_forward(x, signs, lam)
+    y = srft_forward(x, signs, lam, transform)
     scales = group_scales(y, G)
     codes, u = quantize(y, scales, G)
     return {"packed": pack_nibbles(codes), "scales": scales, "codes": codes, "y": y, "u": u}
@@ -174,9 +208,9 @@ def dequantize(codes: np.ndarray, scales16: np.ndarray, G: int) -> np.ndarray:
 
 
 def decode(packed: np.ndarray, scales16: np.ndarray, signs: np.ndarray, lam: np.ndarray,
-           G: int = 32) -> np.ndarray:
-    """x_hat = diag(s) F_r^T (c*scale / lambda), fp64 [..., D]."""
-    return srft_inverse(dequantize(unpack_nibbles(packed), scales16, G), signs, lam)
+           G: int = 32, transform: str = "srft") -> np.ndarray:
+    """x_hat = R^T (c*scale / lambda), fp64 [..., D]."""
+    return srft_inverse(dequantize(unpack_nibbles(packed), scales16, G), signs, lam, transform)
 
 
 def compressed_bytes_per_vector(D: int, G: int) -> int:
@@ -232,19 +266,20 @@ def attend_decode(q: np.ndarray, k_hat: np.ndarray, v_hat: np.ndarray, seq_lens,
 
 
 def attend_decode_int4(q, k_packed, k_scales, v_packed, v_scales, k_params, v_params, seq_lens,
-                       G: int = 32, sigma: float | None = None) -> np.ndarray:
+                       G: int = 32, sigma: float | None = None, transform: str = "srft") -> np.ndarray:
     """Attention over a packed int4 cache: decode K and V, then attend_decode.
 
     k_params / v_params = (signs, lambda) of the K and V transforms.
     """
     T = int(np.max(seq_lens))
-    kh = decode(k_packed[:, :, :T], k_scales[:, :, :T], k_params[0], k_params[1], G)
-    vh = decode(v_packed[:, :, :T], v_scales[:, :, :T], v_params[0], v_params[1], G)
+    kh = decode(k_packed[:, :, :T], k_scales[:, :, :T], k_params[0], k_params[1], G, transform)
+    vh = decode(v_packed[:, :, :T], v_scales[:, :, :T], v_params[0], v_params[1], G, transform)
     return attend_decode(q, kh, vh, seq_lens, sigma)
 
 
 def attend_decode_int4_rotated(q, k_packed, k_scales, v_packed, v_scales, k_params, v_params,
-                               seq_lens, G: int = 32, sigma: float | None = None) -> np.ndarray:
+                               seq_lens, G: int = 32, sigma: float | None = None,
+                               transform: str = "srft") -> np.ndarray:
     """The same attention computed in the rotated domain.
 
     q_t = Lambda_K^-1 R_K q; score_t = sigma * sum_g scale_{t,g} sum_{i in g} q_t[i] c_t[i];
@@ -258,8 +293,8 @@ def attend_decode_int4_rotated(q, k_packed, k_scales, v_packed, v_scales, k_para
     grp = Hq // Hkv
     if sigma is None:
         sigma = 1.0 / math.sqrt(D)
-    Rk = srft_matrix(k_params[0])
-    Rv = srft_matrix(v_params[0])
+    Rk = rotation_matrix(k_params[0], transform)
+    Rv = rotation_matrix(v_params[0], transform)
     lk = np.asarray(k_params[1], dtype=np.float64)
     lv = np.asarray(v_params[1], dtype=np.float64)
     out = np.zeros((B, Hq, D), dtype=np.float64)
