@@ -64,19 +64,37 @@ typedef enum kvq_status {
  * used from several streams and host threads at once. */
 typedef struct kvq_plan kvq_plan;
 
+/* The rotation R of a plan: the SRFT of [M1], R = F_r diag(s) (the default), or the
+ * SRHT the pages compare it with ([M1] "Begruendung" / "Ergebnis": equal quality),
+ * read here as R = H diag(s) / sqrt(D), H the Sylvester Hadamard matrix in natural
+ * order, H[i][j] = (-1)^popcount(i & j). */
+typedef enum { KVQ_TRANSFORM_SRFT = 0, KVQ_TRANSFORM_SRHT = 1 } kvq_transform;
+
 /*
- * kvq_plan_create -- [M1] fixes s, [M2] lambda (one factor per rotated channel).
+ * kvq_plan_create -- [M1] fixes s, [M2] lambda (one factor per rotated channel); the
+ * SRFT plan (kvq_plan_create_transform with KVQ_TRANSFORM_SRFT).
  *   out         host: receives the new plan.
  *   head_dim    D: 128 or 256.
  *   group       G: channels per abs-max scale group (32; 16 also accepted).
  *   signs_host  host int8[D], every entry +1 or -1 (the fixed random sign vector s).
  *   lambda_host host float[D], every entry finite and > 0 (per-channel lambda).
- * Allocates a small device block (under 4 KB) on the current device, the plan's
- * device: the per-channel factors and sign masks derived from s and lambda.
+ * Allocates one device block on the current device, the plan's device: the
+ * per-channel factors and sign masks derived from s and lambda, the tensor-core
+ * encode's operand Lambda R as an fp16 hi/lo pair (2 D^2 halves) and the attention
+ * kernels' 128-point transform (64 KB).
  * Errors: INVALID_ARG, UNSUPPORTED, CUDA, DEVICE.
  */
 kvq_status kvq_plan_create(kvq_plan** out, int head_dim, int group, const int8_t* signs_host,
                            const float* lambda_host);
+
+/* kvq_plan_create with the rotation chosen: transform is a kvq_transform value
+ * (UNSUPPORTED otherwise). Every entry point accepts either kind; the two plans of
+ * an attention call must use the same kind. */
+kvq_status kvq_plan_create_transform(kvq_plan** out, int head_dim, int group, const int8_t* signs_host,
+                                     const float* lambda_host, int transform);
+
+/* The plan's kvq_transform value; -1 for a NULL plan. */
+int kvq_plan_transform(const kvq_plan* plan);
 
 /* Frees the plan and its device block. Passing NULL is a no-op. The caller must
  * ensure no launch that uses the plan is still pending. */

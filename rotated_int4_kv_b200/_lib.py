@@ -40,6 +40,8 @@ def _load() -> ctypes.CDLL:
     P, I, F, S, U32P = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t, ctypes.POINTER(ctypes.c_uint32)
     sig = {
         "kvq_plan_create": (I, [ctypes.POINTER(P), I, I, P, P]),
+        "kvq_plan_create_transform": (I, [ctypes.POINTER(P), I, I, P, P, I]),
+        "kvq_plan_transform": (I, [P]),
         "kvq_plan_destroy": (I, [P]),
         "kvq_plan_head_dim": (I, [P]),
         "kvq_plan_group": (I, [P]),

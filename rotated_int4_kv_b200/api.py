@@ -35,20 +35,28 @@ def _need(t: torch.Tensor, name: str, dtype, shape=None):
         raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
 
 
-class Plan:
-    """A (sign vector s, lambda) transform plan on the current CUDA device."""
+TRANSFORMS = {"srft": 0, "srht": 1}
 
-    def __init__(self, signs, lam, group: int = 32):
+
+class Plan:
+    """A (sign vector s, lambda) transform plan on the current CUDA device; transform
+    "srft" (the pages' method, default) or "srht" (the Hadamard variant)."""
+
+    def __init__(self, signs, lam, group: int = 32, transform: str = "srft"):
         s = np.ascontiguousarray(np.asarray(signs, dtype=np.int8))
         l = np.ascontiguousarray(np.asarray(lam, dtype=np.float32))
         if s.ndim != 1 or l.shape != s.shape:
             raise ValueError("signs and lambda must be 1-D arrays of the same length")
+        if transform not in TRANSFORMS:
+            raise ValueError(f"transform must be one of {sorted(TRANSFORMS)}")
         self.head_dim = int(s.shape[0])
         self.group = int(group)
+        self.transform = transform
         self._h = ctypes.c_void_p()
-        check(lib.kvq_plan_create(ctypes.byref(self._h), self.head_dim, self.group,
-                                  s.ctypes.data_as(ctypes.c_void_p), l.ctypes.data_as(ctypes.c_void_p)),
-              "kvq_plan_create")
+        check(lib.kvq_plan_create_transform(ctypes.byref(self._h), self.head_dim, self.group,
+                                            s.ctypes.data_as(ctypes.c_void_p), l.ctypes.data_as(ctypes.c_void_p),
+                                            TRANSFORMS[transform]),
+              "kvq_plan_create_transform")
         self._lib = lib
 
     @property

@@ -19,12 +19,12 @@ class Int4KVCache:
     """Per-layer int4 K and V caches of ``capacity`` tokens for ``batch`` sequences.
 
     ``k_params`` / ``v_params``: one (signs, lambda) pair for every layer, or a list of
-    ``layers`` pairs (K and V get separate transforms). All sequences of the batch share
-    the write position of a layer.
+    ``layers`` pairs (K and V get separate transforms); ``transform`` "srft" or "srht".
+    All sequences of the batch share the write position of a layer.
     """
 
     def __init__(self, layers: int, batch: int, kv_heads: int, head_dim: int, capacity: int, k_params, v_params,
-                 device=None, group: int = 32):
+                 device=None, group: int = 32, transform: str = "srft"):
         if layers <= 0 or batch <= 0 or kv_heads <= 0 or capacity <= 0:
             raise ValueError("layers, batch, kv_heads and capacity must be positive")
         self.device = torch.device(device) if device is not None else torch.device("cuda")
@@ -41,8 +41,8 @@ class Int4KVCache:
             return list(params)
 
         with torch.cuda.device(self.device):
-            self.k_plans = [Plan(s, lam, group) for s, lam in per_layer(k_params)]
-            self.v_plans = [Plan(s, lam, group) for s, lam in per_layer(v_params)]
+            self.k_plans = [Plan(s, lam, group, transform) for s, lam in per_layer(k_params)]
+            self.v_plans = [Plan(s, lam, group, transform) for s, lam in per_layer(v_params)]
         shape_c = (batch, kv_heads, self.capacity, head_dim // 2)
         shape_s = (batch, kv_heads, self.capacity, head_dim // group)
         self.k_codes = [torch.zeros(shape_c, dtype=torch.uint8, device=self.device) for _ in range(layers)]

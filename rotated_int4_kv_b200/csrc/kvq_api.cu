@@ -52,6 +52,9 @@ double basis_value(int c, int n, int D) {
   return std::sqrt(2.0 / D) * ((c & 1) ? std::cos(ang) : std::sin(ang));
 }
 
+// Entry (i, j) of the Sylvester Hadamard matrix in natural order: (-1)^popcount(i & j).
+double hadamard_value(int i, int j) { return (__builtin_popcount((unsigned)(i & j)) & 1) ? -1.0 : 1.0; }
+
 uint16_t half_bits(float f) { return __half_as_ushort(__float2half_rn(f)); }
 float half_value(uint16_t b) { return __half2float(__ushort_as_half(b)); }
 
@@ -187,8 +190,18 @@ const char* kvq_status_string(kvq_status s) {
 const char* kvq_last_error(void) { return kvq::t_last_error.c_str(); }
 
 kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, const float* lambda) {
+  return kvq_plan_create_transform(out, D, G, signs, lambda, KVQ_TRANSFORM_SRFT);
+}
+
+int kvq_plan_transform(const kvq_plan* p) { return p ? p->xform : -1; }
+
+kvq_status kvq_plan_create_transform(kvq_plan** out, int D, int G, const int8_t* signs, const float* lambda,
+                                     int transform) {
   if (!out || !signs || !lambda) return fail(KVQ_ERR_INVALID_ARG, "plan_create: null argument");
   *out = nullptr;
+  if (transform != KVQ_TRANSFORM_SRFT && transform != KVQ_TRANSFORM_SRHT)
+    return fail(KVQ_ERR_UNSUPPORTED, "plan_create: transform must be KVQ_TRANSFORM_SRFT or KVQ_TRANSFORM_SRHT");
+  const bool hadamard = transform == KVQ_TRANSFORM_SRHT;
   if (D != 128 && D != 256) return fail(KVQ_ERR_UNSUPPORTED, "plan_create: head_dim must be 128 or 256");
   if (G != 32 && G != 16) return fail(KVQ_ERR_UNSUPPORTED, "plan_create: group must be 32 or 16");
   for (int i = 0; i < D; ++i) {
@@ -206,8 +219,11 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
   p->D = D;
   p->G = G;
   p->device = dev;
+  p->xform = transform;
+  // per-channel factor of the rotation's unnormalised rows: the real DFT's dg_c, or
+  // 1/sqrt(D) for every Hadamard row
   for (int c = 0; c < D; ++c) {
-    const double dg = kvq::basis_dg(c, D);
+    const double dg = hadamard ? 1.0 / std::sqrt((double)D) : kvq::basis_dg(c, D);
     p->enc.chan[c] = (float)((double)lambda[c] * dg);
     p->dec.chan[c] = (float)(dg / (double)lambda[c]);
   }
@@ -224,7 +240,8 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
   for (int c = 0; c < D; ++c) {
     const int h = c / 128, rr = c % 128;
     for (int n = 0; n < D; ++n) {
-      const double w = (double)lambda[c] * kvq::basis_value(c, n, D) * (double)signs[n];
+      const double r = hadamard ? kvq::hadamard_value(c, n) / std::sqrt((double)D) : kvq::basis_value(c, n, D);
+      const double w = (double)lambda[c] * r * (double)signs[n];
       const uint16_t hi = kvq::half_bits((float)w);
       const uint16_t lo = kvq::half_bits((float)(w - (double)kvq::half_value(hi)));
       wt[(size_t)(256 * h + rr) * D + n] = hi;
@@ -233,8 +250,9 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
   }
   // attention operand (both head dims): the unnormalised 128-point real DFT in slot
   // order, F128 (hi, lo): row 0 = 1, row 1 = (-1)^m, row 2k = cos(2 pi k m / 128),
-  // row 2k+1 = -sin(2 pi k m / 128). D = 128 applies it directly, D = 256 to the even
-  // and odd samples; the plan's signs and per-channel factors are applied around it.
+  // row 2k+1 = -sin(2 pi k m / 128); for the SRHT the 128-point Hadamard matrix (exact
+  // in fp16, lo = 0). D = 128 applies it directly, D = 256 to the even and odd samples;
+  // the plan's signs and per-channel factors are applied around it.
   std::vector<uint16_t> rot;
   {
     const int M = 128;
@@ -243,7 +261,8 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
     for (int j = 0; j < M; ++j)
       for (int m = 0; m < M; ++m) {
         double v;
-        if (j == 0) v = 1.0;
+        if (hadamard) v = kvq::hadamard_value(j, m);
+        else if (j == 0) v = 1.0;
         else if (j == 1) v = (m & 1) ? -1.0 : 1.0;
         else {
           const double ang = pi2 * (double)((long)(j / 2) * m % M) / (double)M;
@@ -336,8 +355,9 @@ kvq_status kvq_encode_batch(const kvq_encode_job* jobs, int njobs, void* stream)
       p0 = j.plan;
       kvq_status st = kvq::check_plan_device(p0);
       if (st != KVQ_OK) return st;
-    } else if (j.plan->D != p0->D || j.plan->G != p0->G || j.plan->device != p0->device) {
-      return fail(KVQ_ERR_INVALID_ARG, w + "all jobs must share head_dim, group and device");
+    } else if (j.plan->D != p0->D || j.plan->G != p0->G || j.plan->device != p0->device ||
+               j.plan->xform != p0->xform) {
+      return fail(KVQ_ERR_INVALID_ARG, w + "all jobs must share head_dim, group, transform and device");
     }
     live.push_back(j);
   }
@@ -394,8 +414,8 @@ kvq_status kvq_attend_decode(const kvq_plan* pk, const kvq_plan* pv, const uint1
                              int T_cap, const int32_t* seq_lens, int T_len, float sigma, uint16_t* out,
                              void* ws, size_t ws_bytes, void* stream) {
   if (!pk || !pv) return fail(KVQ_ERR_INVALID_ARG, "attend: null plan");
-  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device)
-    return fail(KVQ_ERR_INVALID_ARG, "attend: K and V plans differ in head_dim, group or device");
+  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device || pk->xform != pv->xform)
+    return fail(KVQ_ERR_INVALID_ARG, "attend: K and V plans differ in head_dim, group, transform or device");
   if (pk->G != 32) return fail(KVQ_ERR_UNSUPPORTED, "attend: group must be 32");
   kvq_status st = check_attend_common(B, Hq, Hkv, pk->D, T_cap, T_len, q, out, ws, ws_bytes);
   if (st != KVQ_OK || B == 0) return st;
@@ -413,8 +433,8 @@ kvq_status kvq_attend_decode_append(const kvq_plan* pk, const kvq_plan* pv, cons
                                     int Hq, int Hkv, int T_cap, int pos, float sigma, uint16_t* out, void* ws,
                                     size_t ws_bytes, void* stream) {
   if (!pk || !pv) return fail(KVQ_ERR_INVALID_ARG, "attend_append: null plan");
-  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device)
-    return fail(KVQ_ERR_INVALID_ARG, "attend_append: K and V plans differ in head_dim, group or device");
+  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device || pk->xform != pv->xform)
+    return fail(KVQ_ERR_INVALID_ARG, "attend_append: K and V plans differ in head_dim, group, transform or device");
   if (pk->G != 32) return fail(KVQ_ERR_UNSUPPORTED, "attend_append: group must be 32");
   if (pos < 0) return fail(KVQ_ERR_INVALID_ARG, "attend_append: pos < 0");
   if (pos >= T_cap) return fail(KVQ_ERR_CAPACITY, "attend_append: pos + 1 > T_cap");
@@ -444,8 +464,9 @@ kvq_status kvq_attend_decode_batch(const kvq_attend_job* jobs, int njobs, int B,
     const std::string tag = "attend_batch: job " + std::to_string(i) + ": ";
     if (!j.pk || !j.pv) return fail(KVQ_ERR_INVALID_ARG, tag + "null plan");
     if (j.pk->D != p0->D || j.pv->D != p0->D || j.pk->G != p0->G || j.pv->G != p0->G ||
-        j.pk->device != p0->device || j.pv->device != p0->device)
-      return fail(KVQ_ERR_INVALID_ARG, tag + "plans differ in head_dim, group or device");
+        j.pk->device != p0->device || j.pv->device != p0->device || j.pk->xform != p0->xform ||
+        j.pv->xform != p0->xform)
+      return fail(KVQ_ERR_INVALID_ARG, tag + "plans differ in head_dim, group, transform or device");
     if (j.pk->G != 32) return fail(KVQ_ERR_UNSUPPORTED, tag + "group must be 32");
     kvq_status st = check_attend_common(B, Hq, Hkv, p0->D, T_cap, T_len, j.q, j.out, ws, ws_bytes);
     if (st != KVQ_OK) return fail(st, tag + kvq_last_error());
@@ -471,8 +492,8 @@ kvq_status kvq_attend_decode_noalloc(const kvq_plan* pk, const kvq_plan* pv, con
                                      int Hkv, int T_cap, const int32_t* seq_lens, int T_len, float sigma,
                                      uint16_t* out, void* stream) {
   if (!pk || !pv) return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: null plan");
-  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device)
-    return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: K and V plans differ in head_dim, group or device");
+  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device || pk->xform != pv->xform)
+    return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: K and V plans differ in head_dim, group, transform or device");
   if (pk->G != 32) return fail(KVQ_ERR_UNSUPPORTED, "attend_noalloc: group must be 32");
   if (B < 0 || Hq <= 0 || Hkv <= 0 || T_cap < 0) return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: bad sizes");
   if (Hq % Hkv) return fail(KVQ_ERR_UNSUPPORTED, "attend_noalloc: Hq must be a multiple of Hkv");

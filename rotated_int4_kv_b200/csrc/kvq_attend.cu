@@ -130,6 +130,7 @@ struct AttnParams {
   uint8_t* vc_out;
   uint16_t* vs_out;
   int append_pos;
+  int xform;  // the plans' kvq_transform (0 SRFT, 1 SRHT)
 };
 
 // One attention problem of a launch: its caches (as tensor maps), query, output
@@ -201,6 +202,9 @@ __device__ __forceinline__ uint32_t rot_addr(const uint8_t* base, int hl, int ro
   return smem_u32(base + (2 * hl + kc) * 16384 + row * 128 + ((ch ^ (row & 7)) << 4));
 }
 __device__ __forceinline__ int chan_of_slot128(int j) { return j == 0 ? 0 : (j == 1 ? 127 : j - 1); }
+// the channel of row j of the resident matrix: the real DFT's slot order, or (hada:
+// SRHT plans, the matrix is the Hadamard matrix) the identity
+__device__ __forceinline__ int chan_of_row128(int j, bool hada) { return hada ? j : chan_of_slot128(j); }
 __device__ __forceinline__ int slot_of_chan128(int c) { return c == 0 ? 0 : (c == 127 ? 1 : c + 1); }
 
 // X[j][r] = sum_m F128[j][m] x'_r[m] for up to eight fp16 rows x_r (x'_r = x_r with the
@@ -247,11 +251,12 @@ __device__ __forceinline__ void f128_forward(const uint16_t* rows, int nrows, Sg
   }
 }
 
-// D = 128: q_t[h][c] = (dg / lambda)_c X[slot(c)][h] with X = F128 (s (.) q_h).
+// D = 128: q_t[h][c] = (dg / lambda)_c X[slot(c)][h] with X = F128 (s (.) q_h) (hada: the
+// Hadamard matrix, rows in channel order, dg = 1/sqrt(D)).
 __device__ __forceinline__ void rotate_query_f128(const uint16_t* qs, int heads, const uint32_t* ksg, const float* kch,
-                                                  const uint8_t* srot, float* qt, int warp, int lane) {
+                                                  const uint8_t* srot, float* qt, int warp, int lane, bool hada) {
   f128_forward(qs, heads, [&](int) { return ksg; }, srot, warp, lane, [&](int j, int h, float v) {
-    const int c = chan_of_slot128(j);
+    const int c = chan_of_row128(j, hada);
     qt[h * 128 + c] = kch[c] * v;
   });
 }
@@ -261,7 +266,7 @@ __device__ __forceinline__ void rotate_query_f128(const uint16_t* qs, int heads,
 // three products per step (hi.hi, hi.lo, lo.hi) keep ~2^-22 relative precision. A =
 // F128^T by ldmatrix.trans of the resident F128. Called by the four consumer warps.
 __device__ __forceinline__ void unrotate_out_f128(const float* om, int heads, const float* Lh, const float* vch,
-                                                  const uint8_t* srot, float* xb, int warp, int lane) {
+                                                  const uint8_t* srot, float* xb, int warp, int lane, bool hada) {
   const int g = lane >> 2, cq = lane & 3;
   const int mi = lane >> 3;
   const float L = g < heads ? Lh[g] : 0.0f;
@@ -273,7 +278,7 @@ __device__ __forceinline__ void unrotate_out_f128(const float* om, int heads, co
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
       const int j0 = 16 * ks + 2 * cq + 8 * e;
-      const int c0 = chan_of_slot128(j0), c1 = chan_of_slot128(j0 + 1);
+      const int c0 = chan_of_row128(j0, hada), c1 = chan_of_row128(j0 + 1, hada);
       const float v0 = orow[c0] * vch[c0] * r, v1 = orow[c1] * vch[c1] * r;
       const __half h0 = __float2half_rn(v0), h1 = __float2half_rn(v1);
       const __half l0 = __float2half_rn(v0 - __half2float(h0)), l1 = __float2half_rn(v1 - __half2float(h1));
@@ -321,7 +326,7 @@ __device__ __forceinline__ void unrotate_out_f128(const float* om, int heads, co
 // scratch [E, O][8 rows][128 slots]. Called by the NW consumer warps.
 template <int NW, typename SgnOf, typename Out>
 __device__ __forceinline__ void f256_forward(const uint16_t* rows, int nrows, SgnOf sgn_of, const uint8_t* srot,
-                                             float* eo, int warp, int lane, Out out) {
+                                             float* eo, int warp, int lane, bool hada, Out out) {
   const int g = lane >> 2, cq = lane & 3;
   const int mi = lane >> 3;
   {
@@ -375,8 +380,25 @@ __device__ __forceinline__ void f256_forward(const uint16_t* rows, int nrows, Sg
     }
   }
   consumer_sync<NW>();
-  // radix-2 combine into channels: consumer thread t takes channels t, t + 32 NW, ...
   const int t = threadIdx.x;  // 0 .. 32 NW - 1 (consumer warps)
+  if (hada) {
+    // Hadamard (SRHT plans): X[2k + b] = E_k + (-1)^b O_k
+#pragma unroll
+    for (int half = 0; half < 256 / (32 * NW); ++half) {
+      const int ch = t + 32 * NW * half, k = ch >> 1;
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        float v = 0.0f;
+        if (h < nrows) {
+          const float e = eo[h * 128 + k], o = eo[1024 + h * 128 + k];
+          v = (ch & 1) ? e - o : e + o;
+        }
+        out(ch, h, v);
+      }
+    }
+    return;
+  }
+  // radix-2 combine into channels: consumer thread t takes channels t, t + 32 NW, ...
 #pragma unroll
   for (int half = 0; half < 256 / (32 * NW); ++half) {
     const int ch = t + 32 * NW * half;
@@ -425,8 +447,9 @@ __device__ __forceinline__ void f256_forward(const uint16_t* rows, int nrows, Sg
 // D = 256: q_t[h][c] = (dg / lambda)_c X(c) with X = F256 (s (.) q_h) by the even/odd split.
 template <int NW>
 __device__ __forceinline__ void rotate_query_eo(const uint16_t* qs, int heads, const uint32_t* ksg, const float* kch,
-                                                const uint8_t* srot, float* eo, float* qt, int warp, int lane) {
-  f256_forward<NW>(qs, heads, [&](int) { return ksg; }, srot, eo, warp, lane,
+                                                const uint8_t* srot, float* eo, float* qt, int warp, int lane,
+                                                bool hada) {
+  f256_forward<NW>(qs, heads, [&](int) { return ksg; }, srot, eo, warp, lane, hada,
                    [&](int c, int h, float v) { qt[h * 256 + c] = v * kch[c]; });
 }
 
@@ -436,9 +459,29 @@ __device__ __forceinline__ void rotate_query_eo(const uint16_t* qs, int heads, c
 // enter as fp16 hi + lo). eo: fp32 scratch [2][8][128]. All 160 threads call it.
 template <int NW>
 __device__ __forceinline__ void unrotate_out_eo(const float* om, int heads, const float* Lh, const float* vch,
-                                                const uint8_t* srot, float* eo, float* xb, int warp, int lane) {
+                                                const uint8_t* srot, float* eo, float* xb, int warp, int lane,
+                                                bool hada) {
   const int t = threadIdx.x;
-  if (t <= 64) {  // k = t
+  if (hada) {
+    // Hadamard (SRHT plans), the transpose of X[2k + b] = E_k + (-1)^b O_k:
+    // E'_k = Z_2k + Z_2k+1, O'_k = Z_2k - Z_2k+1
+    if (t < 128) {
+      const int k = t;
+#pragma unroll
+      for (int h = 0; h < 8; ++h) {
+        float e = 0.0f, o = 0.0f;
+        if (h < heads) {
+          const float L = Lh[h];
+          const float r = L > 0.0f ? 1.0f / L : 0.0f;
+          const float z0 = om[h * 256 + 2 * k] * vch[2 * k] * r, z1 = om[h * 256 + 2 * k + 1] * vch[2 * k + 1] * r;
+          e = z0 + z1;
+          o = z0 - z1;
+        }
+        eo[h * 128 + k] = e;
+        eo[1024 + h * 128 + k] = o;
+      }
+    }
+  } else if (t <= 64) {  // k = t
     const int k = t;
     float sn, cs;
     sincospif((float)k / 128.0f, &sn, &cs);
@@ -584,6 +627,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
   const int unit = (int)blockIdx.z * p.HT + ht;  // workspace slot (over all jobs)
   // fused append: the last split of the unit encodes and adds the new token
   const bool app = INT4 && p.append_pos >= 0 && split == p.S - 1;
+  const bool hada = p.xform == 1;  // SRHT plans: the resident matrix is the Hadamard matrix
 
   const int row0 = bk * p.T_cap;  // first cache row of this (b, kv head)
 
@@ -693,9 +737,9 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
       ok = false;
     }
     if constexpr (C::kMmaRot && D == 128) {
-      rotate_query_f128(qs, heads, ksg, kch, srot, qt, warp, lane);
+      rotate_query_f128(qs, heads, ksg, kch, srot, qt, warp, lane, hada);
     } else if constexpr (C::kMmaRot) {
-      rotate_query_eo<kCWarps>(qs, heads, ksg, kch, srot, reinterpret_cast<float*>(qf), qt, warp, lane);
+      rotate_query_eo<kCWarps>(qs, heads, ksg, kch, srot, reinterpret_cast<float*>(qf), qt, warp, lane, hada);
     } else {
       for (int i = threadIdx.x; i < kHT * D / 2; i += kCWarps * 32) {
         const int h = (2 * i) / D;
@@ -714,18 +758,18 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
       if (app) {
         auto sgn_of = [&](int r) { return r ? vsg : ksg; };
         auto enc_f = [&](int r, int c) {
-          const float d2 = (c == 0 || c == D - 1) ? 1.0f / D : 2.0f / D;
+          const float d2 = (hada || c == 0 || c == D - 1) ? 1.0f / D : 2.0f / D;  // dg_c^2
           return d2 / (r ? vch[c] : kch[c]);
         };
         if constexpr (D == 128) {
           f128_forward(app_in, 2, sgn_of, srot, warp, lane, [&](int j, int r, float v) {
             if (r < 2) {
-              const int c = chan_of_slot128(j);
+              const int c = chan_of_row128(j, hada);
               ybuf[r * D + c] = v * enc_f(r, c);
             }
           });
         } else {
-          f256_forward<kCWarps>(app_in, 2, sgn_of, srot, reinterpret_cast<float*>(qf), warp, lane,
+          f256_forward<kCWarps>(app_in, 2, sgn_of, srot, reinterpret_cast<float*>(qf), warp, lane, hada,
                                 [&](int c, int r, float v) {
                                   if (r < 2) ybuf[r * D + c] = v * enc_f(r, c);
                                 });
@@ -1271,9 +1315,9 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
   uint16_t* ob = J.out + ((size_t)b * p.Hq + hq0) * D;
   if constexpr (C::kMmaRot) {
     if constexpr (D == 128) {
-      if (warp < kCWarps) unrotate_out_f128(om, heads, mrg + kHT, vch, srot, xb, warp, lane);
+      if (warp < kCWarps) unrotate_out_f128(om, heads, mrg + kHT, vch, srot, xb, warp, lane, hada);
     } else {
-      unrotate_out_eo<kCWarps>(om, heads, mrg + kHT, vch, srot, reinterpret_cast<float*>(qf), xb, warp, lane);
+      unrotate_out_eo<kCWarps>(om, heads, mrg + kHT, vch, srot, reinterpret_cast<float*>(qf), xb, warp, lane, hada);
     }
     __syncthreads();
     for (int i = threadIdx.x; i < heads * D / 2; i += kThreads) {
@@ -1548,6 +1592,7 @@ kvq_status launch_chunk(const AttendJobHost* jobs, int nj, int B, int Hq, int Hk
   prm.cnt = reinterpret_cast<int*>(wsb);
   prm.part = reinterpret_cast<float*>(wsb + ws_cnt_bytes(units));
   prm.append_pos = -1;
+  prm.xform = INT4 ? jobs[0].pk->xform : 0;
   if (app) {
     prm.k_new = app->k_new;
     prm.v_new = app->v_new;

@@ -52,6 +52,49 @@ __device__ __forceinline__ void tile_origin(const TileGeom& g, int tile, int& bh
 template <int D>
 constexpr int kMinBlocks = D == 128 ? 3 : 2;
 
+// ---------------------------------------------------------------- Walsh-Hadamard (SRHT plans)
+// Unnormalised Sylvester-order Hadamard transform (H[i][j] = (-1)^popcount(i & j)) by
+// the in-place butterflies (a, b) -> (a + b, a - b) at distances 1, 2, 4, ... of 128
+// values held as 64 packed pairs v[j] = (y[2j], y[2j+1]): distance 1 inside each pair,
+// the others between pairs j and j + h/2, componentwise on packed f32x2 operations.
+__device__ __forceinline__ void fwht128_packed(float2 (&v)[64]) {
+#pragma unroll
+  for (int j = 0; j < 64; ++j) {
+    const float a = v[j].x, b = v[j].y;
+    v[j] = make_float2(a + b, a - b);
+  }
+  const float2 m1 = make_float2(-1.0f, -1.0f);
+#pragma unroll
+  for (int st = 0; st < 6; ++st) {  // pair distance hh = 2^st
+    const int hh = 1 << st;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {   // the 32 butterflies of the stage
+      const int k = ((j >> st) << (st + 1)) | (j & (hh - 1));
+      const float2 a = v[k], b = v[k + hh];
+      v[k] = __fadd2_rn(a, b);
+      v[k + hh] = __ffma2_rn(b, m1, a);
+    }
+  }
+}
+
+// The same transform of N values in a scalar array (decode).
+template <int N>
+__device__ __forceinline__ void fwht_scalar(float (&v)[N]) {
+  constexpr int LOG = N == 256 ? 8 : 7;
+  static_assert(N == 128 || N == 256, "length");
+#pragma unroll
+  for (int st = 0; st < LOG; ++st) {  // distance h = 2^st
+    const int h = 1 << st;
+#pragma unroll
+    for (int j = 0; j < N / 2; ++j) {  // the N/2 butterflies of the stage
+      const int k = ((j >> st) << (st + 1)) | (j & (h - 1));
+      const float a = v[k], b = v[k + h];
+      v[k] = a + b;
+      v[k + h] = a - b;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- encode
 // One launch walks the tiles of up to MAXJ independent jobs (kvq_encode = 1 job,
 // kvq_encode_batch = a grouped launch). A job's tensor maps live in the kernel
@@ -128,7 +171,8 @@ struct EncCfg {
   static constexpr int kBytes = kStages * kXStage + 4 * kCWarp + 64 + 1024;
 };
 
-template <int D, int G, int MAXJ>
+// XF: 0 = SRFT (real FFT in registers), 1 = SRHT (Walsh-Hadamard butterflies).
+template <int D, int G, int XF, int MAXJ>
 __global__ void __launch_bounds__(kNT, 3) encode_kernel(const __grid_constant__ EncBatch<MAXJ> P) {
   using C = EncCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -223,11 +267,60 @@ __global__ void __launch_bounds__(kNT, 3) encode_kernel(const __grid_constant__ 
       }
     }
     // ---- transform (packed f32x2 halves + scalar top stage), lambda, quantise, pack
-    rdft_fwd_packed<128>(v);
     uint32_t words[16];
     uint32_t sbits[128 / G];
     int cb_lo, cb_hi;  // first channels of the two 64-channel halves this thread owns
-    if constexpr (C::kTPV == 1) {
+    if constexpr (XF == 1) {
+      // SRHT: channel c = Hadamard row c. D = 128: the thread's 128 samples directly.
+      // D = 256: thread p holds the samples 2m + p; with A_p = H128 of them,
+      // X[2k + b] = A_0[k] + (-1)^b A_1[k], and thread p owns channels 128 p .. 128 p + 127
+      // (k in [64 p, 64 p + 64)): it trades the other half of its A with its partner.
+      fwht128_packed(v);
+      float vv[128];
+      if constexpr (C::kTPV == 1) {
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+          vv[2 * j] = v[j].x;
+          vv[2 * j + 1] = v[j].y;
+        }
+        cb_lo = 0;
+        cb_hi = 64;
+      } else {
+#pragma unroll
+        for (int i = 0; i < 64; i += 2) {
+          const float2 own = p ? v[32 + i / 2] : v[i / 2];   // A[64 p + i], A[64 p + i + 1]
+          const float2 snd = p ? v[i / 2] : v[32 + i / 2];   // A[64 (1 - p) + i], ...
+          const float2 rcv = make_float2(__shfl_xor_sync(0xffffffffu, snd.x, 1), __shfl_xor_sync(0xffffffffu, snd.y, 1));
+          const float2 u = p ? rcv : own, w = p ? own : rcv;
+          vv[2 * i] = u.x + w.x;
+          vv[2 * i + 1] = u.x - w.x;
+          vv[2 * i + 2] = u.y + w.y;
+          vv[2 * i + 3] = u.y - w.y;
+        }
+        cb_lo = p ? 128 : 0;
+        cb_hi = cb_lo + 64;
+      }
+      float lo[64], hi[64];
+#pragma unroll
+      for (int i = 0; i < 64; ++i) {
+        lo[i] = vv[i];
+        hi[i] = vv[64 + i];
+      }
+      uint32_t wl[8], wh[8], sl[64 / G], sh[64 / G];
+      quantize_pack<64, G>(lo, J.cc->chan + cb_lo, wl, sl);
+      quantize_pack<64, G>(hi, J.cc->chan + cb_hi, wh, sh);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        words[i] = wl[i];
+        words[8 + i] = wh[i];
+      }
+#pragma unroll
+      for (int i = 0; i < 64 / G; ++i) {
+        sbits[i] = sl[i];
+        sbits[64 / G + i] = sh[i];
+      }
+    } else if constexpr (C::kTPV == 1) {
+      rdft_fwd_packed<128>(v);
       float vv[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) vv[c] = slotv(v, slot_of_channel(c, 128));
@@ -235,6 +328,7 @@ __global__ void __launch_bounds__(kNT, 3) encode_kernel(const __grid_constant__ 
       cb_lo = 0;
       cb_hi = 64;
     } else {
+      rdft_fwd_packed<128>(v);
       float vv[128];
       pair_combine<0>(v, vv, p);
       cb_lo = p ? 64 : 0;
@@ -313,7 +407,7 @@ struct DecSmem {
   static constexpr int kBytes = kStages * kCStage + kXTile + 64 + 1024;
 };
 
-template <int D, int G>
+template <int D, int G, int XF>
 __global__ void __launch_bounds__(kNT, kMinBlocks<D>) decode_kernel(const __grid_constant__ CUtensorMap cmap,
                                                      const __grid_constant__ CUtensorMap omap,
                                                      const __grid_constant__ CodecConsts cc, TileGeom geom,
@@ -423,10 +517,14 @@ __global__ void __launch_bounds__(kNT, kMinBlocks<D>) decode_kernel(const __grid
       for (int j = 0; j < 8; ++j) {
         const int c = 8 * w + j;
         const float code = __uint_as_float(((u >> (4 * j)) & 0xFu) | 0x4B400000u) - 12582920.0f;
-        v[slot_of_channel(c, D)] = code * (sc[c / G] * cc.chan[c]);
+        v[XF == 1 ? c : slot_of_channel(c, D)] = code * (sc[c / G] * cc.chan[c]);
       }
     }
-    rdft_inv<D>(v);
+    if constexpr (XF == 1) {
+      fwht_scalar<D>(v);  // H is symmetric: the inverse is the same butterflies
+    } else {
+      rdft_inv<D>(v);
+    }
     // sign, fp16, stage for the TMA store
     if (tid == 0) bulk_wait_group_read0();
     __syncthreads();
@@ -480,7 +578,7 @@ int occupancy_blocks(K kernel, int smem_bytes) {
   return nb;
 }
 
-template <int D, int G, int MAXJ>
+template <int D, int G, int XF, int MAXJ>
 kvq_status run_encode_chunk(const kvq_encode_job* jobs, int nj, cudaStream_t s) {
   EncBatch<MAXJ> P;
   memset(&P, 0, sizeof(P));
@@ -524,7 +622,7 @@ kvq_status run_encode_chunk(const kvq_encode_job* jobs, int nj, cudaStream_t s) 
   }
   P.njobs = nj;
   P.total_tiles = tiles;
-  void (*kern)(const EncBatch<MAXJ>) = encode_kernel<D, G, MAXJ>;
+  void (*kern)(const EncBatch<MAXJ>) = encode_kernel<D, G, XF, MAXJ>;
   const int smem = EncCfg<D>::kBytes;
   static int blocks_per_sm = -1;
   static std::once_flag once;
@@ -543,18 +641,18 @@ kvq_status run_encode_chunk(const kvq_encode_job* jobs, int nj, cudaStream_t s) 
 
 constexpr int kMaxJobs = 64;
 
-template <int D, int G>
+template <int D, int G, int XF>
 kvq_status run_encode(const kvq_encode_job* jobs, int njobs, cudaStream_t s) {
-  if (njobs == 1) return run_encode_chunk<D, G, 1>(jobs, 1, s);
+  if (njobs == 1) return run_encode_chunk<D, G, XF, 1>(jobs, 1, s);
   for (int i = 0; i < njobs; i += kMaxJobs) {
     const int nj = std::min(kMaxJobs, njobs - i);
-    kvq_status st = run_encode_chunk<D, G, kMaxJobs>(jobs + i, nj, s);
+    kvq_status st = run_encode_chunk<D, G, XF, kMaxJobs>(jobs + i, nj, s);
     if (st != KVQ_OK) return st;
   }
   return KVQ_OK;
 }
 
-template <int D, int G>
+template <int D, int G, int XF>
 kvq_status run_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* scales, int B, int H, int T_cap,
                       int t0, int n, uint16_t* out, cudaStream_t s) {
   const int BH = B * H;
@@ -580,11 +678,11 @@ kvq_status run_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* s
   static int blocks_per_sm = -1;
   static std::once_flag once;
   std::call_once(once, [&] {
-    cudaFuncSetAttribute(decode_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    blocks_per_sm = occupancy_blocks(decode_kernel<D, G>, smem);
+    cudaFuncSetAttribute(decode_kernel<D, G, XF>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    blocks_per_sm = occupancy_blocks(decode_kernel<D, G, XF>, smem);
   });
   const int grid = std::min(geom.n_tiles, blocks_per_sm * num_sms(p->device));
-  decode_kernel<D, G><<<grid, kNT, smem, s>>>(cmap, omap, p->dec, geom, scales, T_cap, t0);
+  decode_kernel<D, G, XF><<<grid, kNT, smem, s>>>(cmap, omap, p->dec, geom, scales, T_cap, t0);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("decode launch: ") + cudaGetErrorString(e));
   return KVQ_OK;
@@ -592,22 +690,34 @@ kvq_status run_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* s
 
 }  // namespace
 
+template <int XF>
+kvq_status launch_encode_xf(const kvq_encode_job* jobs, int njobs, int D, int G, cudaStream_t s) {
+  if (D == 128 && G == 32) return run_encode<128, 32, XF>(jobs, njobs, s);
+  if (D == 256 && G == 32) return run_encode<256, 32, XF>(jobs, njobs, s);
+  if (D == 128 && G == 16) return run_encode<128, 16, XF>(jobs, njobs, s);
+  if (D == 256 && G == 16) return run_encode<256, 16, XF>(jobs, njobs, s);
+  return fail(KVQ_ERR_UNSUPPORTED, "encode: unsupported (head_dim, group)");
+}
+
 kvq_status launch_encode_jobs(const kvq_encode_job* jobs, int njobs, cudaStream_t s) {
   const int D = jobs[0].plan->D, G = jobs[0].plan->G;
-  if (D == 128 && G == 32) return run_encode<128, 32>(jobs, njobs, s);
-  if (D == 256 && G == 32) return run_encode<256, 32>(jobs, njobs, s);
-  if (D == 128 && G == 16) return run_encode<128, 16>(jobs, njobs, s);
-  if (D == 256 && G == 16) return run_encode<256, 16>(jobs, njobs, s);
-  return fail(KVQ_ERR_UNSUPPORTED, "encode: unsupported (head_dim, group)");
+  return jobs[0].plan->xform == 1 ? launch_encode_xf<1>(jobs, njobs, D, G, s) : launch_encode_xf<0>(jobs, njobs, D, G, s);
+}
+
+template <int XF>
+kvq_status launch_decode_xf(const kvq_plan* p, const uint8_t* codes, const uint16_t* scales, int B, int H, int T_cap,
+                            int t0, int n, uint16_t* out, cudaStream_t s) {
+  if (p->D == 128 && p->G == 32) return run_decode<128, 32, XF>(p, codes, scales, B, H, T_cap, t0, n, out, s);
+  if (p->D == 256 && p->G == 32) return run_decode<256, 32, XF>(p, codes, scales, B, H, T_cap, t0, n, out, s);
+  if (p->D == 128 && p->G == 16) return run_decode<128, 16, XF>(p, codes, scales, B, H, T_cap, t0, n, out, s);
+  if (p->D == 256 && p->G == 16) return run_decode<256, 16, XF>(p, codes, scales, B, H, T_cap, t0, n, out, s);
+  return fail(KVQ_ERR_UNSUPPORTED, "decode: unsupported (head_dim, group)");
 }
 
 kvq_status launch_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* scales, int B, int H, int T_cap,
                          int t0, int n, uint16_t* out, cudaStream_t s) {
-  if (p->D == 128 && p->G == 32) return run_decode<128, 32>(p, codes, scales, B, H, T_cap, t0, n, out, s);
-  if (p->D == 256 && p->G == 32) return run_decode<256, 32>(p, codes, scales, B, H, T_cap, t0, n, out, s);
-  if (p->D == 128 && p->G == 16) return run_decode<128, 16>(p, codes, scales, B, H, T_cap, t0, n, out, s);
-  if (p->D == 256 && p->G == 16) return run_decode<256, 16>(p, codes, scales, B, H, T_cap, t0, n, out, s);
-  return fail(KVQ_ERR_UNSUPPORTED, "decode: unsupported (head_dim, group)");
+  return p->xform == 1 ? launch_decode_xf<1>(p, codes, scales, B, H, T_cap, t0, n, out, s)
+                       : launch_decode_xf<0>(p, codes, scales, B, H, T_cap, t0, n, out, s);
 }
 
 uint32_t codec_error_flags(bool clear) {

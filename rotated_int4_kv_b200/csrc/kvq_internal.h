@@ -28,6 +28,7 @@ struct kvq_plan {
   int D = 0;
   int G = 0;
   int device = -1;
+  int xform = 0;           // kvq_transform: 0 SRFT, 1 SRHT
   kvq::CodecConsts enc{};  // lambda_c * dg_c
   kvq::CodecConsts dec{};  // dg_c / lambda_c
   // Device block: copies of `enc` and `dec` for kernels that serve several plans

@@ -21,7 +21,8 @@ def test_header_declares_the_boundary():
     for n in ("kvq_plan_create", "kvq_plan_destroy", "kvq_encode", "kvq_encode_batch", "kvq_decode",
               "kvq_workspace_size", "kvq_attend_decode", "kvq_attend_decode_ref", "kvq_status_string",
               "kvq_last_error", "kvq_poll_device_errors", "kvq_attend_decode_batch",
-              "kvq_attend_decode_noalloc", "kvq_attend_decode_append"):
+              "kvq_attend_decode_noalloc", "kvq_attend_decode_append", "kvq_plan_create_transform",
+              "kvq_plan_transform"):
         assert n in names
 
 
@@ -62,6 +63,8 @@ def test_status_strings_and_host_checks():
     lam = (ctypes.c_float * 128)(*([1.0] * 128))
     assert lib.kvq_plan_create(ctypes.byref(h), 96, 32, signs, lam) == -2      # head_dim
     assert lib.kvq_plan_create(ctypes.byref(h), 128, 24, signs, lam) == -2     # group
+    assert lib.kvq_plan_create_transform(ctypes.byref(h), 128, 32, signs, lam, 2) == -2  # transform
+    assert lib.kvq_plan_transform(None) == -1
     bad = (ctypes.c_int8 * 128)(*([1] * 127 + [0]))
     assert lib.kvq_plan_create(ctypes.byref(h), 128, 32, bad, lam) == -1       # sign value
     neg = (ctypes.c_float * 128)(*([1.0] * 127 + [-1.0]))
