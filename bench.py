@@ -180,9 +180,10 @@ def oracle_sample(wl, seed: int, layer: int = 0):
     v = kvgen.kv_numpy(wl, "v", (1, wl.h_kv, T, D), seed=seed, layer=layer)
     q = kvgen.q_numpy((1, wl.h_q, D), seed=seed, layer=layer)
     t0 = time.perf_counter()
-    ek = oracle.encode(k, ks, kl, G)
-    ev = oracle.encode(v, vs, vl, G)
-    oracle.attend_decode_int4(q, ek["packed"], ek["scales"], ev["packed"], ev["scales"], (ks, kl), (vs, vl), [T], G)
+    ek = oracle.encode(k, ks, kl, G, TRANSFORM)
+    ev = oracle.encode(v, vs, vl, G, TRANSFORM)
+    oracle.attend_decode_int4(q, ek["packed"], ek["scales"], ev["packed"], ev["scales"], (ks, kl), (vs, vl), [T], G,
+                              transform=TRANSFORM)
     dt = time.perf_counter() - t0
     return 2 * wl.h_kv * T, dt
 
@@ -235,9 +236,13 @@ def run_reference(args, rank: int, world: int):
     return 0
 
 
+# the plans' rotation: "srft" (the pages' method, the default) or "srht" (--transform)
+TRANSFORM = "srft"
+
+
 def _config(wl):
     return {"workload": "gemma3-1b-prefill: encode K+V of 26 layers x 4096 tokens, then 1-token int4 decode "
-                        "attention per layer",
+                        "attention per layer", "transform": TRANSFORM,
             "layers": wl.layers, "kv_heads": wl.h_kv, "q_heads": wl.h_q, "head_dim": wl.head_dim,
             "batch": wl.batch, "prefix": wl.contexts[0], "group": wl.group,
             "l2": f"inputs rotate over {N_INPUT_SETS} distinct input sets (3 x 109 MB) so each step reads HBM"}
@@ -269,7 +274,7 @@ def run_kvq(args, rank: int, world: int):
     for l in range(L):
         for kind in ("k", "v"):
             s, lam = kvgen.plan_params(D, seed=seed, layer=l, kind=kind)
-            plans.append(kvq.Plan(s, lam, group=G))
+            plans.append(kvq.Plan(s, lam, group=G, transform=TRANSFORM))
     X = []
     for i in range(N_INPUT_SETS):
         x = torch.empty((NJ, Hkv, T, D), dtype=torch.float16, device=dev)
@@ -398,11 +403,13 @@ def run_kvq(args, rank: int, world: int):
     src = "measured (MEASURED_PEAKS.json hbm_gbs, burst copy)" if peak_kind == "measured" else "fallback 6.65 TB/s"
     tc = kvq.get_encode_path() != "fft" and G == 32
     # the tensor-core encode's own work: Y = X [W_hi; W_lo]^T, 2 x D x 2D flops per vector
-    # (context for the HBM roofline: at D = 256 this product, not HBM, bounds the kernel)
+    # (SRHT plans: the exact W, 2 x D x D) -- context for the HBM roofline: at D = 256 the
+    # hi/lo product, not HBM, bounds the SRFT kernel
     tensor = None
     if tc:
-        tflops = vec_step * 4 * D * D / (enc_avg * 1e-3) / 1e12
-        tensor = {"flops_per_vec": 4 * D * D, "achieved_TFLOP_s": tflops,
+        fpv = (2 if TRANSFORM == "srht" else 4) * D * D
+        tflops = vec_step * fpv / (enc_avg * 1e-3) / 1e12
+        tensor = {"flops_per_vec": fpv, "achieved_TFLOP_s": tflops,
                   "peak_TFLOP_s": _tensor_peak(), "frac": tflops / _tensor_peak(),
                   "peak_source": "measured (MEASURED_PEAKS.json bf16_tflops_sustained; fp16 runs at the bf16 rate)"}
     if enc_avg >= att_avg:
@@ -504,8 +511,8 @@ def run_decode_workload(args, rank: int, world: int):
         T_cap = T + 2
         plans, caches, caches16 = [], [], []
         for l in range(distinct):
-            pk = kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=l, kind="k"))
-            pv = kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=l, kind="v"))
+            pk = kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=l, kind="k"), transform=TRANSFORM)
+            pv = kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=l, kind="v"), transform=TRANSFORM)
             plans.append((pk, pv))
             c = {}
             for kind, pl in (("k", pk), ("v", pv)):
@@ -589,7 +596,7 @@ def run_decode_workload(args, rank: int, world: int):
     if sb:
         # streaming encode: one token per step for each of sb sequences x Hkv heads x {K, V}
         # (one grouped launch per step; a few MB, so this measures latency, not HBM)
-        pk, pv = (kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=0, kind=k)) for k in ("k", "v"))
+        pk, pv = (kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=0, kind=k), transform=TRANSFORM) for k in ("k", "v"))
         xk = kvgen.kv_torch(wl, "k", (sb, Hkv, 1, D), dev, seed=seed, layer=0, salt=77)
         xv = kvgen.kv_torch(wl, "v", (sb, Hkv, 1, D), dev, seed=seed, layer=0, salt=78)
         kc = torch.zeros((sb, Hkv, 2, D // 2), dtype=torch.uint8, device=dev)
@@ -611,7 +618,8 @@ def run_decode_workload(args, rank: int, world: int):
     line = {"metric": METRIC, "value": big["int4_attn_GB_s"], "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": big["int4_step_ms"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": args.workload, "layers": layers, "kv_heads": Hkv, "q_heads": Hq, "head_dim": D,
+            "config": {"workload": args.workload, "transform": TRANSFORM, "layers": layers, "kv_heads": Hkv,
+                       "q_heads": Hq, "head_dim": D,
                        "batch": B, "contexts": list(contexts), "group": G},
             "cases": cases}
     if stream_enc is not None:
@@ -635,7 +643,11 @@ def main(argv=None):
                     help="distinct per-layer caches cycled through a decode step (each > L2 for the big shapes)")
     ap.add_argument("--ncu", action="store_true",
                     help="profiling mode: run --steps eager steps without timing, for ncu captures")
+    ap.add_argument("--transform", default="srft", choices=["srft", "srht"],
+                    help="the plans' rotation: srft (the pages' method) or srht (the Hadamard variant)")
     args = ap.parse_args(argv)
+    global TRANSFORM
+    TRANSFORM = args.transform
     if args.warmup < 3:
         args.warmup = 3
     rank = int(os.environ.get("RANK", "0"))

@@ -236,12 +236,17 @@ kvq_status kvq_plan_create_transform(kvq_plan** out, int D, int G, const int8_t*
   // fp16 pair (value = hi + lo to ~2^-22 |W|), laid out per 128-channel half h as
   // 128 hi rows then 128 lo rows: row 256 h + r = hi of channel 128 h + r,
   // row 256 h + 128 + r = lo of the same channel.
-  std::vector<uint16_t> wt((size_t)2 * D * D);
+  // SRHT plans: W = H diag(s) exactly (entries +-1; D rows, D columns), the factor
+  // lambda_c / sqrt(D) is applied by the kernel's epilogue.
+  std::vector<uint16_t> wt(hadamard ? (size_t)D * D : (size_t)2 * D * D);
   for (int c = 0; c < D; ++c) {
     const int h = c / 128, rr = c % 128;
     for (int n = 0; n < D; ++n) {
-      const double r = hadamard ? kvq::hadamard_value(c, n) / std::sqrt((double)D) : kvq::basis_value(c, n, D);
-      const double w = (double)lambda[c] * r * (double)signs[n];
+      if (hadamard) {
+        wt[(size_t)c * D + n] = kvq::half_bits((float)(kvq::hadamard_value(c, n) * (double)signs[n]));
+        continue;
+      }
+      const double w = (double)lambda[c] * kvq::basis_value(c, n, D) * (double)signs[n];
       const uint16_t hi = kvq::half_bits((float)w);
       const uint16_t lo = kvq::half_bits((float)(w - (double)kvq::half_value(hi)));
       wt[(size_t)(256 * h + rr) * D + n] = hi;

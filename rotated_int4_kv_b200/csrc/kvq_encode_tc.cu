@@ -28,6 +28,12 @@
 // Two TMEM accumulators (2 x D columns) let the epilogue of tile i overlap the
 // MMAs of tile i + 1. Every wait is bounded; a CTA that gives up raises a device
 // error flag and still deallocates its TMEM.
+//
+// Exact W (EX, plans of the SRHT variant): W = H diag(s) has entries +-1, exact in
+// fp16, so one product per K step gives Y exactly up to the fp32 accumulation; the
+// per-channel factor lambda_c / sqrt(D) is applied in the epilogue. An MMA then
+// covers all D channels (N = D), one CTA per tile at either head dim, half the
+// tensor work of the hi/lo product.
 #include <algorithm>
 #include <cstdio>
 #include <mutex>
@@ -50,9 +56,10 @@ constexpr int kTcMaxJobs = 64;
 
 struct alignas(64) TcJob {
   CUtensorMap xmap;  // x as [rows][D] fp16, box {64, 128}, 128-byte swizzle
-  CUtensorMap wmap;  // W as [2D][D] fp16 (hi rows, then lo rows), box {64, 2D}, 128-byte swizzle
+  CUtensorMap wmap;  // W as [2D][D] fp16 (hi rows, then lo rows; EX: [D][D]), box {64, N}, 128-byte swizzle
   uint8_t* codes;    // [BH][T_cap][D/2]
   uint16_t* scales;  // [BH][T_cap][D/32]
+  const float* chan; // EX: the per-channel factors lambda_c / sqrt(D)
   int rows, n, T_cap, pos, tile0;  // rows = B*H*n; tile0 = first global tile of the job
 };
 
@@ -62,16 +69,16 @@ struct TcBatch {
   int njobs, ntiles;
 };
 
-template <int D>
+template <int D, bool EX>
 struct TcCfg {
   static constexpr int KC = D / 64;                  // 64-wide K chunks (one 128-byte swizzle atom each)
-  static constexpr int kSplit = D / 128;             // CTAs per tile (channel halves)
+  static constexpr int kSplit = EX ? 1 : D / 128;    // CTAs per tile (channel halves)
   static constexpr int kChunkA = kTcRows * 128;      // one K chunk of a 128-row X tile: 16 KB
-  static constexpr int kN = 256;                     // MMA N: 128 W_hi rows then 128 W_lo rows
-  static constexpr int kChunkW = kN * 128;           // one K chunk of [W_hi; W_lo]: 32 KB
-  static constexpr int kW = KC * kChunkW;            // 64 KB (D = 128) or 128 KB (D = 256)
-  static constexpr int kChunks = D == 128 ? 10 : 6;  // X ring depth in K chunks
-  static constexpr int kTmemCols = 2 * kN;           // two accumulators of 256 fp32 columns
+  static constexpr int kN = EX ? D : 256;            // MMA N: D exact rows, or 128 W_hi rows then 128 W_lo rows
+  static constexpr int kChunkW = kN * 128;           // one K chunk of W
+  static constexpr int kW = KC * kChunkW;            // 64 KB (D = 128) or 128 KB (D = 256); EX: 32 / 128 KB
+  static constexpr int kChunks = (EX && D == 128) ? 12 : (D == 128 ? 10 : 6);  // X ring depth in K chunks
+  static constexpr int kTmemCols = 2 * kN;           // two accumulators of N fp32 columns
   static constexpr int kBars = 8 * (2 * kChunks + 4 + 3) + 16;
   static constexpr int kSmem = kW + kChunks * kChunkA + kBars + 1024;
   static_assert(kSmem <= 227 * 1024, "shared memory");
@@ -82,9 +89,9 @@ __device__ __forceinline__ int job_of(const TcJob* jobs, int njobs, int job, int
   return job;
 }
 
-template <int D, int MAXJ>
+template <int D, bool EX, int MAXJ>
 __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_constant__ TcBatch<MAXJ> bt) {
-  using C = TcCfg<D>;
+  using C = TcCfg<D, EX>;
   constexpr int kTcChunks = C::kChunks;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -238,8 +245,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
   } else {
     // ------------------------------------------------------------ epilogue
     // warp w: TMEM lanes 32 (w % 4) .. + 31 (one vector per thread), channel groups
-    // [h * NGH, (h + 1) * NGH) with h = (w - 2) / 4
-    constexpr int NGH = 2;  // groups per thread: 128 channels per CTA, two threads per vector
+    // [h * NGH, (h + 1) * NGH) of the CTA's channels with h = (w - 2) / 4
+    constexpr int NGH = EX ? D / 64 : 2;  // groups per thread: two threads per vector
     const int q = warp & 3;
     const int h = (warp - 2) >> 2;
     int job = ntile > 0 ? job_of(bt.j, bt.njobs, 0, t_begin) : 0;
@@ -259,37 +266,75 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
       const int bh = valid ? r / J.n : 0;
       const size_t orow = (size_t)bh * J.T_cap + J.pos + (r - bh * J.n);
       const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * C::kN + 32 * NGH * h);
-      float y[NGH][32], ylo[NGH][32];
-#pragma unroll
-      for (int g = 0; g < NGH; ++g) {
-        tmem_ld32(ta + 32 * g, y[g]);
-        tmem_ld32(ta + 128 + 32 * g, ylo[g]);
-      }
-      tmem_ld_wait();
-#pragma unroll
-      for (int g = 0; g < NGH; ++g) {
-        tmem_regs_fence(y[g]);
-        tmem_regs_fence(ylo[g]);
-      }
-      // the accumulator may be overwritten as soon as every epilogue warp has its values
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&tempty[a]);
       uint32_t sb[NGH];
+      if constexpr (EX) {
+        // Y exact up to the fp32 accumulation; y = Y * lambda_c / sqrt(D)
+        float y[NGH][32];
 #pragma unroll
-      for (int g = 0; g < NGH; ++g) {
+        for (int g = 0; g < NGH; ++g) tmem_ld32(ta + 32 * g, y[g]);
+        tmem_ld_wait();
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          const float2 v = __fadd2_rn(make_float2(y[g][e], y[g][e + 1]), make_float2(ylo[g][e], ylo[g][e + 1]));
-          y[g][e] = v.x;
-          y[g][e + 1] = v.y;
+        for (int g = 0; g < NGH; ++g) tmem_regs_fence(y[g]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[a]);
+#pragma unroll
+        for (int g = 0; g < NGH; ++g) {
+          const float4* f4 = reinterpret_cast<const float4*>(J.chan + 32 * (NGH * h + g));
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 f = __ldg(f4 + e);
+            y[g][4 * e] *= f.x;
+            y[g][4 * e + 1] *= f.y;
+            y[g][4 * e + 2] *= f.z;
+            y[g][4 * e + 3] *= f.w;
+          }
+          uint32_t w[4];
+          quantize_group<32>(y[g], w, sb[g]);
+          if (valid)
+            reinterpret_cast<uint4*>(J.codes + orow * (D / 2))[NGH * h + g] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        uint32_t w[4];
-        quantize_group<32>(y[g], w, sb[g]);
-        if (valid)
-          reinterpret_cast<uint4*>(J.codes + orow * (D / 2))[4 * half + NGH * h + g] = make_uint4(w[0], w[1], w[2], w[3]);
+        if (valid) {
+          if constexpr (NGH == 4) {
+            reinterpret_cast<uint2*>(J.scales + orow * (D / 32))[h] = make_uint2(sb[0] | (sb[1] << 16),
+                                                                                 sb[2] | (sb[3] << 16));
+          } else {
+            reinterpret_cast<uint32_t*>(J.scales + orow * (D / 32))[h] = sb[0] | (sb[1] << 16);
+          }
+        }
+      } else {
+        float y[NGH][32], ylo[NGH][32];
+#pragma unroll
+        for (int g = 0; g < NGH; ++g) {
+          tmem_ld32(ta + 32 * g, y[g]);
+          tmem_ld32(ta + 128 + 32 * g, ylo[g]);
+        }
+        tmem_ld_wait();
+#pragma unroll
+        for (int g = 0; g < NGH; ++g) {
+          tmem_regs_fence(y[g]);
+          tmem_regs_fence(ylo[g]);
+        }
+        // the accumulator may be overwritten as soon as every epilogue warp has its values
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tempty[a]);
+#pragma unroll
+        for (int g = 0; g < NGH; ++g) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 2) {
+            const float2 v = __fadd2_rn(make_float2(y[g][e], y[g][e + 1]), make_float2(ylo[g][e], ylo[g][e + 1]));
+            y[g][e] = v.x;
+            y[g][e + 1] = v.y;
+          }
+          uint32_t w[4];
+          quantize_group<32>(y[g], w, sb[g]);
+          if (valid)
+            reinterpret_cast<uint4*>(J.codes + orow * (D / 2))[4 * half + NGH * h + g] =
+                make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        if (valid) reinterpret_cast<uint32_t*>(J.scales + orow * (D / 32))[2 * half + h] = sb[0] | (sb[1] << 16);
       }
-      if (valid) reinterpret_cast<uint32_t*>(J.scales + orow * (D / 32))[2 * half + h] = sb[0] | (sb[1] << 16);
     }
   }
 
@@ -306,10 +351,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
 void tc_prepare() {
   static std::once_flag once;
   std::call_once(once, [] {
-    cudaFuncSetAttribute(encode_tc_kernel<128, kTcMaxJobs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         TcCfg<128>::kSmem);
-    cudaFuncSetAttribute(encode_tc_kernel<256, kTcMaxJobs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         TcCfg<256>::kSmem);
+    cudaFuncSetAttribute(encode_tc_kernel<128, false, kTcMaxJobs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         TcCfg<128, false>::kSmem);
+    cudaFuncSetAttribute(encode_tc_kernel<256, false, kTcMaxJobs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         TcCfg<256, false>::kSmem);
+    cudaFuncSetAttribute(encode_tc_kernel<128, true, kTcMaxJobs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         TcCfg<128, true>::kSmem);
+    cudaFuncSetAttribute(encode_tc_kernel<256, true, kTcMaxJobs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         TcCfg<256, true>::kSmem);
   });
 }
 
@@ -320,6 +369,7 @@ bool encode_tc_supported(int D, int G) { return (D == 128 || D == 256) && G == 3
 // Grouped launch over jobs of one head_dim (128 or 256, group 32); jobs with no rows are skipped.
 kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t strm) {
   const int D = jobs[0].plan->D;
+  const bool ex = jobs[0].plan->xform == 1;  // SRHT: exact W
   tc_prepare();
   int i0 = 0;
   while (i0 < njobs) {
@@ -338,15 +388,17 @@ kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t 
       kvq_status st = encode_tiled(&J.xmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, j.x, xd, xs, xb,
                                    CU_TENSOR_MAP_SWIZZLE_128B, "encode x");
       if (st != KVQ_OK) return st;
-      // W = Lambda F_r diag(s): per 128-channel half, 128 hi rows then 128 lo rows, D columns
-      const uint64_t wd[2] = {(uint64_t)D, (uint64_t)(2 * D)};
+      // W = Lambda F_r diag(s): per 128-channel half, 128 hi rows then 128 lo rows, D
+      // columns; exact W (SRHT): H diag(s), D rows (channels), D columns
+      const uint64_t wd[2] = {(uint64_t)D, (uint64_t)(ex ? D : 2 * D)};
       const uint64_t ws[1] = {(uint64_t)D * 2};
-      const uint32_t wb[2] = {64u, 256u};
+      const uint32_t wb[2] = {64u, (uint32_t)(ex ? D : 256)};
       st = encode_tiled(&J.wmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, j.plan->wt_dev, wd, ws, wb,
                         CU_TENSOR_MAP_SWIZZLE_128B, "encode weights");
       if (st != KVQ_OK) return st;
       J.codes = j.codes;
       J.scales = j.scales;
+      J.chan = j.plan->enc_dev->chan;
       J.rows = (int)rows;
       J.n = j.n;
       J.T_cap = j.T_cap;
@@ -374,14 +426,23 @@ kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t 
     cfg.attrs = attr;
     cfg.numAttrs = 1;
     cudaError_t e;
-    if (D == 128) {
+    if (ex) {
       cfg.gridDim = dim3(std::min(tiles, sms));
-      cfg.dynamicSmemBytes = TcCfg<128>::kSmem;
-      e = cudaLaunchKernelEx(&cfg, encode_tc_kernel<128, kTcMaxJobs>, bt);
+      if (D == 128) {
+        cfg.dynamicSmemBytes = TcCfg<128, true>::kSmem;
+        e = cudaLaunchKernelEx(&cfg, encode_tc_kernel<128, true, kTcMaxJobs>, bt);
+      } else {
+        cfg.dynamicSmemBytes = TcCfg<256, true>::kSmem;
+        e = cudaLaunchKernelEx(&cfg, encode_tc_kernel<256, true, kTcMaxJobs>, bt);
+      }
+    } else if (D == 128) {
+      cfg.gridDim = dim3(std::min(tiles, sms));
+      cfg.dynamicSmemBytes = TcCfg<128, false>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, encode_tc_kernel<128, false, kTcMaxJobs>, bt);
     } else {
       cfg.gridDim = dim3(2 * std::min(tiles, sms / 2));
-      cfg.dynamicSmemBytes = TcCfg<256>::kSmem;
-      e = cudaLaunchKernelEx(&cfg, encode_tc_kernel<256, kTcMaxJobs>, bt);
+      cfg.dynamicSmemBytes = TcCfg<256, false>::kSmem;
+      e = cudaLaunchKernelEx(&cfg, encode_tc_kernel<256, false, kTcMaxJobs>, bt);
     }
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("encode (tensor cores) launch: ") + cudaGetErrorString(e));
