@@ -421,7 +421,7 @@ kvq_status kvq_attend_decode(const kvq_plan* pk, const kvq_plan* pv, const uint1
   if (!pk || !pv) return fail(KVQ_ERR_INVALID_ARG, "attend: null plan");
   if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device || pk->xform != pv->xform)
     return fail(KVQ_ERR_INVALID_ARG, "attend: K and V plans differ in head_dim, group, transform or device");
-  if (pk->G != 32) return fail(KVQ_ERR_UNSUPPORTED, "attend: group must be 32");
+  if (pk->G != 32 && pk->G != 16) return fail(KVQ_ERR_UNSUPPORTED, "attend: group must be 32 or 16");
   kvq_status st = check_attend_common(B, Hq, Hkv, pk->D, T_cap, T_len, q, out, ws, ws_bytes);
   if (st != KVQ_OK || B == 0) return st;
   if (!kc || !ks || !vc || !vs) return fail(KVQ_ERR_INVALID_ARG, "attend: null cache buffer");
@@ -440,7 +440,7 @@ kvq_status kvq_attend_decode_append(const kvq_plan* pk, const kvq_plan* pv, cons
   if (!pk || !pv) return fail(KVQ_ERR_INVALID_ARG, "attend_append: null plan");
   if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device || pk->xform != pv->xform)
     return fail(KVQ_ERR_INVALID_ARG, "attend_append: K and V plans differ in head_dim, group, transform or device");
-  if (pk->G != 32) return fail(KVQ_ERR_UNSUPPORTED, "attend_append: group must be 32");
+  if (pk->G != 32 && pk->G != 16) return fail(KVQ_ERR_UNSUPPORTED, "attend_append: group must be 32 or 16");
   if (pos < 0) return fail(KVQ_ERR_INVALID_ARG, "attend_append: pos < 0");
   if (pos >= T_cap) return fail(KVQ_ERR_CAPACITY, "attend_append: pos + 1 > T_cap");
   kvq_status st = check_attend_common(B, Hq, Hkv, pk->D, T_cap, pos + 1, q, out, ws, ws_bytes);
@@ -472,7 +472,7 @@ kvq_status kvq_attend_decode_batch(const kvq_attend_job* jobs, int njobs, int B,
         j.pk->device != p0->device || j.pv->device != p0->device || j.pk->xform != p0->xform ||
         j.pv->xform != p0->xform)
       return fail(KVQ_ERR_INVALID_ARG, tag + "plans differ in head_dim, group, transform or device");
-    if (j.pk->G != 32) return fail(KVQ_ERR_UNSUPPORTED, tag + "group must be 32");
+    if (j.pk->G != 32 && j.pk->G != 16) return fail(KVQ_ERR_UNSUPPORTED, tag + "group must be 32 or 16");
     kvq_status st = check_attend_common(B, Hq, Hkv, p0->D, T_cap, T_len, j.q, j.out, ws, ws_bytes);
     if (st != KVQ_OK) return fail(st, tag + kvq_last_error());
     if (B == 0) continue;
@@ -499,7 +499,7 @@ kvq_status kvq_attend_decode_noalloc(const kvq_plan* pk, const kvq_plan* pv, con
   if (!pk || !pv) return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: null plan");
   if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device || pk->xform != pv->xform)
     return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: K and V plans differ in head_dim, group, transform or device");
-  if (pk->G != 32) return fail(KVQ_ERR_UNSUPPORTED, "attend_noalloc: group must be 32");
+  if (pk->G != 32 && pk->G != 16) return fail(KVQ_ERR_UNSUPPORTED, "attend_noalloc: group must be 32 or 16");
   if (B < 0 || Hq <= 0 || Hkv <= 0 || T_cap < 0) return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: bad sizes");
   if (Hq % Hkv) return fail(KVQ_ERR_UNSUPPORTED, "attend_noalloc: Hq must be a multiple of Hkv");
   if (T_cap & 1) return fail(KVQ_ERR_ALIGNMENT, "attend_noalloc: T_cap must be even");

@@ -59,9 +59,11 @@ constexpr int kMaxClusterThroughput = 4;
 constexpr int kMaxMerge = kMaxSplitsCfg / 4;  // cluster partials per unit merged through the workspace
 constexpr int kMaxJobs = 32;                // problems per launch of a batch (job table in parameter space)
 
-template <int D, bool INT4>
+template <int D, bool INT4, int G = 32>
 struct Cfg {
-  static constexpr int NG = D / 32;                        // scale groups (int4)
+  static_assert(G == 32 || G == 16, "group size");
+  static constexpr int NC = D / 32;                        // 32-channel chunks of a code row (16 bytes each)
+  static constexpr int NG = INT4 ? D / G : NC;             // scale groups per token (int4)
   static constexpr int kRowBytes = INT4 ? D / 2 : 2 * D;   // bytes per token row of K (and V)
   // consumer warps (plus one producer warp); resident CTAs per SM for the launch bounds
   static constexpr int kCWarps = 4;
@@ -94,7 +96,7 @@ struct Cfg {
   static constexpr int kConsts = INT4 ? 2 * (kChanBytes + kSgnBytes) : 0;
   // B fragments of the score product, one 16-byte entry per (k step, lane):
   // (hi01, hi23, lo01, lo23) -- read from shared memory at each use
-  static constexpr int kKSteps = INT4 ? 2 * NG : D / 16;
+  static constexpr int kKSteps = INT4 ? 2 * NC : D / 16;
   static constexpr int kQf = kKSteps * 32 * 16;
   // fused append: the new K and V rows (fp16 [2][D]); at D = 128 they are staged in the
   // B-fragment buffer (built only after the append's encode), at D = 256 (whose query
@@ -584,14 +586,15 @@ __device__ __forceinline__ void unrotate_out_eo(const float* om, int heads, cons
   }
 }
 
-template <int D, bool INT4, int MAXJ>
-__global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinBlocks))
+template <int D, bool INT4, int MAXJ, int G = 32>
+__global__ void __launch_bounds__((Cfg<D, INT4, G>::kThreads), (Cfg<D, INT4, G>::kMinBlocks))
     attend_kernel(const __grid_constant__ AttnJobs<MAXJ> jt, const __grid_constant__ AttnParams p) {
-  using C = Cfg<D, INT4>;
+  using C = Cfg<D, INT4, G>;
   constexpr int kCWarps = C::kCWarps;
   constexpr int kThreads = C::kThreads;
   static_assert(D == 256 || kCWarps == 4, "the D = 128 rotation helpers take four consumer warps");
   constexpr int NG = C::NG;
+  constexpr int NC = C::NC;
   constexpr int MT = D / 16;  // channel m-tiles of the PV product
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -777,21 +780,25 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
         consumer_sync<kCWarps>();
         if (threadIdx.x < 2 * NG) {
           const int r = threadIdx.x / NG, grp = threadIdx.x - r * NG;
-          float* yg = ybuf + r * D + 32 * grp;
-          float y[32];
+          float* yg = ybuf + r * D + G * grp;
+          float y[G];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) y[i] = yg[i];
-          uint32_t wd[4], sb;
-          quantize_group<32>(y, wd, sb);
+          for (int i = 0; i < G; ++i) y[i] = yg[i];
+          uint32_t wd[G / 8], sb;
+          quantize_group<G>(y, wd, sb);
           if (ht == 0) {
             const size_t crow = (size_t)bk * p.T_cap + p.append_pos;
-            *reinterpret_cast<uint4*>((r ? p.vc_out : p.kc_out) + crow * (D / 2) + 16 * grp) =
-                make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            uint8_t* cdst = (r ? p.vc_out : p.kc_out) + crow * (D / 2) + (G / 2) * grp;
+            if constexpr (G == 32) {
+              *reinterpret_cast<uint4*>(cdst) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+            } else {
+              *reinterpret_cast<uint2*>(cdst) = make_uint2(wd[0], wd[1]);
+            }
             (r ? p.vs_out : p.ks_out)[crow * NG + grp] = (uint16_t)sb;
           }
           const float sc = __half2float(__ushort_as_half((unsigned short)sb));
 #pragma unroll
-          for (int w = 0; w < 4; ++w) {
+          for (int w = 0; w < G / 8; ++w) {
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const int nib = (int)((wd[w] >> (4 * e)) & 15u);
@@ -887,7 +894,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
             }
           }
   #pragma unroll
-          for (int gp = 0; gp < NG / 2; ++gp) {  // two groups per ldmatrix.x4
+          for (int gp = 0; gp < NC / 2; ++gp) {  // two 32-channel chunks per ldmatrix.x4
             const int mi = lane >> 3;
             const int row = r0s + ((mi & 1) << 3) + (lane & 7);
             const int chunk = 2 * gp + (mi >> 1);
@@ -900,9 +907,33 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
             nib8_to_h2(w2, hA1);
             nib8_to_h2(w3, hB1);
             const int G0 = 2 * gp, G1 = 2 * gp + 1;
-            float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
             const uint4 f0 = qf[(2 * G0) * 32 + lane], f1 = qf[(2 * G0 + 1) * 32 + lane];
             const uint4 f2 = qf[(2 * G1) * 32 + lane], f3 = qf[(2 * G1 + 1) * 32 + lane];
+            if constexpr (G == 16) {
+              // a chunk holds two scale groups; lane c's channels (8c .. 8c+7 of the chunk)
+              // lie in sub-group c / 2, so masking the B operand by lane splits the product
+              const uint32_t m0 = (c >> 1) ? 0u : 0xffffffffu, m1 = ~m0;
+              auto chunk = [&](const uint32_t (&hA)[4], const uint32_t (&hB)[4], const uint4 fa, const uint4 fb,
+                               int CH) {
+                float a[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                  const uint32_t m = j ? m1 : m0;
+                  mma_16816(a[j], hA[0], hB[0], hA[1], hB[1], fa.x & m, fa.y & m);
+                  mma_16816(a[j], hA[0], hB[0], hA[1], hB[1], fa.z & m, fa.w & m);
+                  mma_16816(a[j], hA[2], hB[2], hA[3], hB[3], fb.x & m, fb.y & m);
+                  mma_16816(a[j], hA[2], hB[2], hA[3], hB[3], fb.z & m, fb.w & m);
+                }
+                scs[0] = fmaf(skA[2 * CH], a[0][0], fmaf(skA[2 * CH + 1], a[1][0], scs[0]));
+                scs[1] = fmaf(skA[2 * CH], a[0][1], fmaf(skA[2 * CH + 1], a[1][1], scs[1]));
+                scs[2] = fmaf(skB[2 * CH], a[0][2], fmaf(skB[2 * CH + 1], a[1][2], scs[2]));
+                scs[3] = fmaf(skB[2 * CH], a[0][3], fmaf(skB[2 * CH + 1], a[1][3], scs[3]));
+              };
+              chunk(hA0, hB0, f0, f1, G0);
+              chunk(hA1, hB1, f2, f3, G1);
+              continue;
+            }
+            float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
             mma_16816(a0, hA0[0], hB0[0], hA0[1], hB0[1], f0.x, f0.y);
             mma_16816(a0, hA0[0], hB0[0], hA0[1], hB0[1], f0.z, f0.w);
             mma_16816(a0, hA0[2], hB0[2], hA0[3], hB0[3], f1.x, f1.y);
@@ -1016,7 +1047,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
             }
           }
   #pragma unroll
-          for (int gp = 0; gp < NG / 2; ++gp) {
+          for (int gp = 0; gp < NC / 2; ++gp) {
             const int mi = lane >> 3;
             const int row = r0s + ((mi & 1) << 3) + (lane & 7);
             const int chunk = 2 * gp + (mi >> 1);
@@ -1025,19 +1056,35 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
             ldmatrix_x4_trans(w0, w1, w2, w3, smem_u32(vt + row * C::kRowBytes + pch * 16));
   #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const int G = 2 * gp + h;
+              const int CH = 2 * gp + h;  // the 32-channel chunk
+              uint32_t lo[4], hi[4];
+              nib8_to_h2(h ? w2 : w0, lo);  // tokens 2c, 2c+1: channels 4g .. 4g+3 of the chunk
+              nib8_to_h2(h ? w3 : w1, hi);  // tokens 2c+8, 2c+9
+              if constexpr (G == 16) {
+                // lane g's channels lie in sub-group g / 4 of the chunk: one product per
+                // sub-group (its V scales in B) with the other sub-group's rows masked out
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                  const uint32_t sel = j ? 0x7632u : 0x5410u;
+                  const uint32_t s01 = prmt(sw[0][CH], sw[1][CH], sel);
+                  const uint32_t s89 = prmt(sw[2][CH], sw[3][CH], sel);
+                  const uint32_t b0 = h2_bits(__hmul2(bits_h2(pb0[sb]), bits_h2(s01)));
+                  const uint32_t b1 = h2_bits(__hmul2(bits_h2(pb1[sb]), bits_h2(s89)));
+                  const uint32_t m = ((g >> 2) == j) ? 0xffffffffu : 0u;
+                  mma_16816(o_acc[2 * CH], lo[0] & m, lo[1] & m, hi[0] & m, hi[1] & m, b0, b1);
+                  mma_16816(o_acc[2 * CH + 1], lo[2] & m, lo[3] & m, hi[2] & m, hi[3] & m, b0, b1);
+                }
+                continue;
+              }
               // V-scale pairs for this group: (s[2c], s[2c+1]) and (s[2c+8], s[2c+9])
-              const uint32_t sel = (G & 1) ? 0x7632u : 0x5410u;
-              const uint32_t s01 = prmt(sw[0][G >> 1], sw[1][G >> 1], sel);
-              const uint32_t s89 = prmt(sw[2][G >> 1], sw[3][G >> 1], sel);
+              const uint32_t sel = (CH & 1) ? 0x7632u : 0x5410u;
+              const uint32_t s01 = prmt(sw[0][CH >> 1], sw[1][CH >> 1], sel);
+              const uint32_t s89 = prmt(sw[2][CH >> 1], sw[3][CH >> 1], sel);
               const uint32_t b0 = h2_bits(__hmul2(bits_h2(pb0[sb]), bits_h2(s01)));
               const uint32_t b1 = h2_bits(__hmul2(bits_h2(pb1[sb]), bits_h2(s89)));
-              uint32_t lo[4], hi[4];
-              nib8_to_h2(h ? w2 : w0, lo);  // tokens 2c, 2c+1: channels 4g .. 4g+3 of group G
-              nib8_to_h2(h ? w3 : w1, hi);  // tokens 2c+8, 2c+9
               // M-tile X: rows g -> ch 4g, g+8 -> ch 4g+1 ; M-tile Y: ch 4g+2, 4g+3
-              mma_16816(o_acc[2 * G], lo[0], lo[1], hi[0], hi[1], b0, b1);
-              mma_16816(o_acc[2 * G + 1], lo[2], lo[3], hi[2], hi[3], b0, b1);
+              mma_16816(o_acc[2 * CH], lo[0], lo[1], hi[0], hi[1], b0, b1);
+              mma_16816(o_acc[2 * CH + 1], lo[2], lo[3], hi[2], hi[3], b0, b1);
             }
           }
         } else {
@@ -1126,8 +1173,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4>::kThreads), (Cfg<D, INT4>::kMinB
     for (int mt = 0; mt < MT; ++mt) {
       int ch0, ch1;  // channels held in rows g and g+8 of m-tile mt
       if constexpr (INT4) {
-        const int G = mt >> 1;
-        ch0 = G * 32 + 4 * g + ((mt & 1) ? 2 : 0);
+        ch0 = (mt >> 1) * 32 + 4 * g + ((mt & 1) ? 2 : 0);
         ch1 = ch0 + 1;
       } else {
         ch0 = mt * 16 + g;
@@ -1348,13 +1394,13 @@ struct Occupancy {
   int cap[kMaxCluster + 1];
 };
 
-template <int D, bool INT4, int MAXJ>
+template <int D, bool INT4, int MAXJ, int G = 32>
 const Occupancy& occupancy() {
-  using C = Cfg<D, INT4>;
+  using C = Cfg<D, INT4, G>;
   static Occupancy occ{};
   static std::once_flag once;
   std::call_once(once, [] {
-    auto kern = attend_kernel<D, INT4, MAXJ>;
+    auto kern = attend_kernel<D, INT4, MAXJ, G>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     int nb = 0;
@@ -1495,9 +1541,9 @@ size_t ws_bytes_for(int B, int Hq, int Hkv, int D, int ncl, int HT) {
 
 // Tensor maps and pointers of one problem. Rows of the code (or fp16) maps are
 // (b, kv head, token) rows; scale maps have one row of T_cap * D/32 halves per (b, kv head).
-template <int D, bool INT4>
+template <int D, bool INT4, int G = 32>
 kvq_status make_job(const AttendJobHost& h, int B, int Hkv, int T_cap, AttnJob* j) {
-  using C = Cfg<D, INT4>;
+  using C = Cfg<D, INT4, G>;
   const uint64_t rows = (uint64_t)B * Hkv * T_cap;
   kvq_status st;
   if (INT4) {
@@ -1559,20 +1605,20 @@ struct AppendHost {
 
 // One launch over nj <= MAXJ problems of equal shape (with app: the fused append, T_len =
 // the tokens already cached = app->pos).
-template <int D, bool INT4, int MAXJ>
+template <int D, bool INT4, int MAXJ, int G = 32>
 kvq_status launch_chunk(const AttendJobHost* jobs, int nj, int B, int Hq, int Hkv, int T_cap, const int32_t* seq_lens,
                         int T_len, float sigma, void* ws, size_t ws_bytes, cudaStream_t strm,
                         const AppendHost* app = nullptr) {
-  using C = Cfg<D, INT4>;
+  using C = Cfg<D, INT4, G>;
   const int T_split = seq_lens ? T_cap : T_len;
   const int Bj = nj * B;  // the jobs of a launch split like a larger batch
-  SplitPlan sp = choose_split(Bj, Hq, Hkv, T_split, occupancy<D, INT4, MAXJ>(), C::kTile, C::kStageNs);
+  SplitPlan sp = choose_split(Bj, Hq, Hkv, T_split, occupancy<D, INT4, MAXJ, G>(), C::kTile, C::kStageNs);
   const size_t units = (size_t)Bj * Hkv * sp.HT;
   const size_t need = ws_bytes_for(Bj, Hq, Hkv, D, sp.S / sp.C, sp.HT);
   if (ws_bytes < need) return fail(KVQ_ERR_WORKSPACE, "attend: workspace too small for this split");
   AttnJobs<MAXJ> jt;
   for (int i = 0; i < nj; ++i) {
-    const kvq_status st = make_job<D, INT4>(jobs[i], B, Hkv, T_cap, &jt.j[i]);
+    const kvq_status st = make_job<D, INT4, G>(jobs[i], B, Hkv, T_cap, &jt.j[i]);
     if (st != KVQ_OK) return st;
   }
   AttnParams prm{};
@@ -1620,22 +1666,23 @@ kvq_status launch_chunk(const AttendJobHost* jobs, int nj, int B, int Hq, int Hk
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, attend_kernel<D, INT4, MAXJ>, jt, prm);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, attend_kernel<D, INT4, MAXJ, G>, jt, prm);
   if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
   return KVQ_OK;
 }
 
 // Launches of up to kMaxJobs problems each, in stream order; they reuse the
 // workspace from its start (every launch leaves its counters at zero).
-template <int D, bool INT4>
+template <int D, bool INT4, int G = 32>
 kvq_status run_attend(const AttendJobHost* jobs, int njobs, int B, int Hq, int Hkv, int T_cap,
                       const int32_t* seq_lens, int T_len, float sigma, void* ws, size_t ws_bytes, cudaStream_t strm) {
   if (njobs == 1)
-    return launch_chunk<D, INT4, 1>(jobs, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, strm);
+    return launch_chunk<D, INT4, 1, G>(jobs, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, strm);
   for (int j0 = 0; j0 < njobs; j0 += kMaxJobs) {
     const int nj = std::min(kMaxJobs, njobs - j0);
     const kvq_status st =
-        launch_chunk<D, INT4, kMaxJobs>(jobs + j0, nj, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, strm);
+        launch_chunk<D, INT4, kMaxJobs, G>(jobs + j0, nj, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes,
+                                           strm);
     if (st != KVQ_OK) return st;
   }
   return KVQ_OK;
@@ -1665,9 +1712,14 @@ kvq_status launch_attend_int4(const kvq_plan* pk, const kvq_plan* pv, const uint
 kvq_status launch_attend_int4_batch(const AttendJobHost* jobs, int njobs, int B, int Hq, int Hkv, int T_cap,
                                     const int32_t* seq_lens, int T_len, float sigma, void* ws, size_t ws_bytes,
                                     cudaStream_t s) {
-  if (jobs[0].pk->D == 128)
-    return run_attend<128, true>(jobs, njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
-  return run_attend<256, true>(jobs, njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
+  const int D = jobs[0].pk->D, G = jobs[0].pk->G;
+  if (D == 128 && G == 32)
+    return run_attend<128, true, 32>(jobs, njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
+  if (D == 256 && G == 32)
+    return run_attend<256, true, 32>(jobs, njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
+  if (D == 128)
+    return run_attend<128, true, 16>(jobs, njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
+  return run_attend<256, true, 16>(jobs, njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
 }
 
 kvq_status launch_attend_int4_append(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q, const uint16_t* k_new,
@@ -1676,9 +1728,13 @@ kvq_status launch_attend_int4_append(const kvq_plan* pk, const kvq_plan* pv, con
                                      size_t ws_bytes, cudaStream_t s) {
   const AttendJobHost job{pk, pv, q, kc, ks, vc, vs, out};
   const AppendHost app{k_new, v_new, kc, ks, vc, vs, pos};
+  if (pk->D == 128 && pk->G == 32)
+    return launch_chunk<128, true, 1, 32>(&job, 1, B, Hq, Hkv, T_cap, nullptr, pos, sigma, ws, ws_bytes, s, &app);
+  if (pk->D == 256 && pk->G == 32)
+    return launch_chunk<256, true, 1, 32>(&job, 1, B, Hq, Hkv, T_cap, nullptr, pos, sigma, ws, ws_bytes, s, &app);
   if (pk->D == 128)
-    return launch_chunk<128, true, 1>(&job, 1, B, Hq, Hkv, T_cap, nullptr, pos, sigma, ws, ws_bytes, s, &app);
-  return launch_chunk<256, true, 1>(&job, 1, B, Hq, Hkv, T_cap, nullptr, pos, sigma, ws, ws_bytes, s, &app);
+    return launch_chunk<128, true, 1, 16>(&job, 1, B, Hq, Hkv, T_cap, nullptr, pos, sigma, ws, ws_bytes, s, &app);
+  return launch_chunk<256, true, 1, 16>(&job, 1, B, Hq, Hkv, T_cap, nullptr, pos, sigma, ws, ws_bytes, s, &app);
 }
 
 kvq_status launch_attend_fp16(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq, int Hkv, int D,
@@ -1728,7 +1784,9 @@ kvq_status launch_attend_int4_noalloc(const kvq_plan* pk, const kvq_plan* pv, co
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(KVQ_ERR_DEVICE, "attend_noalloc: no current device");
   const int D = pk->D;
   // the exact split the launch will choose, hence the exact scratch it needs
-  const Occupancy& occ = D == 128 ? occupancy<128, true, 1>() : occupancy<256, true, 1>();
+  const int G = pk->G;
+  const Occupancy& occ = D == 128 ? (G == 32 ? occupancy<128, true, 1, 32>() : occupancy<128, true, 1, 16>())
+                                  : (G == 32 ? occupancy<256, true, 1, 32>() : occupancy<256, true, 1, 16>());
   const SplitPlan sp = choose_split(B, Hq, Hkv, seq_lens ? T_cap : T_len, occ, Cfg<128, true>::kTile,
                                     D == 128 ? Cfg<128, true>::kStageNs : Cfg<256, true>::kStageNs);
   const size_t need = ws_bytes_for(B, Hq, Hkv, D, sp.S / sp.C, sp.HT);
@@ -1744,9 +1802,17 @@ kvq_status launch_attend_int4_noalloc(const kvq_plan* pk, const kvq_plan* pv, co
   const cudaError_t e = cudaMemsetAsync(scratch, 0, ws_cnt_bytes(units), s);
   if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("attend_noalloc: memset: ") + cudaGetErrorString(e));
   const AttendJobHost job{pk, pv, q, kc, ks, vc, vs, out};
+  if (D == 128 && G == 32)
+    return run_attend<128, true, 32>(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, scratch, kNoAllocScratchBytes,
+                                     s);
+  if (D == 256 && G == 32)
+    return run_attend<256, true, 32>(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, scratch, kNoAllocScratchBytes,
+                                     s);
   if (D == 128)
-    return run_attend<128, true>(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, scratch, kNoAllocScratchBytes, s);
-  return run_attend<256, true>(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, scratch, kNoAllocScratchBytes, s);
+    return run_attend<128, true, 16>(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, scratch, kNoAllocScratchBytes,
+                                     s);
+  return run_attend<256, true, 16>(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, scratch, kNoAllocScratchBytes,
+                                   s);
 }
 
 uint32_t attend_error_flags(bool clear) {

@@ -330,3 +330,69 @@ def test_attend_append_rejects_bad_positions(kvq):
         kvq.attend_decode_append(pk, pv, q, kn, kn, codes, scales, codes.clone(), scales.clone(), T_cap)
     with pytest.raises(kvq.KvqError, match="INVALID_ARG"):
         kvq.attend_decode_append(pk, pv, q, kn, kn, codes, scales, codes.clone(), scales.clone(), -1)
+
+
+G16_CASES = [
+    # (workload, B, Hkv, Hq, T_cap, lens)
+    ("qwen", 1, 2, 12, 1024, None),
+    ("qwen", 2, 2, 12, 300, [300, 41]),
+    ("longctx", 1, 1, 16, 200, None),           # two head tiles
+    ("gemma", 1, 1, 4, 2048, None),             # D = 256
+    ("gemma", 2, 2, 6, 334, [333, 17]),
+]
+
+
+@pytest.mark.parametrize("case", G16_CASES, ids=_ids(G16_CASES))
+def test_attend_group16_matches_oracle(kvq, case):
+    """Scale groups of 16 channels (the pages' "Methodik" 3 figure): attention and the fused
+    append on G = 16 caches, against the oracle with G = 16."""
+    from tests.parity import BOUNDARY_TALLY, check_encode
+
+    wl_name, B, Hkv, Hq, T_cap, lens = case
+    wl = kvgen.WORKLOADS[wl_name]
+    D, G = wl.head_dim, 16
+    dev = torch.device("cuda")
+    cache = {}
+    for kind in ("k", "v"):
+        s, lam = kvgen.plan_params(D, seed=27, kind=kind)
+        plan = kvq.Plan(s, lam, G)
+        x = torch.from_numpy(kvgen.kv_numpy(wl, kind, (B, Hkv, T_cap - 1, D), seed=27)).to(dev)
+        codes = torch.zeros((B, Hkv, T_cap, D // 2), dtype=torch.uint8, device=dev)
+        scales = torch.zeros((B, Hkv, T_cap, D // G), dtype=torch.float16, device=dev)
+        kvq.encode(plan, x, codes, scales, 0)
+        cache[kind] = dict(plan=plan, params=(s, lam), codes=codes, scales=scales)
+    k, v = cache["k"], cache["v"]
+    q16 = kvgen.q_numpy((B, Hq, D), salt=14)
+    q = torch.from_numpy(q16).to(dev)
+    lens_np = [T_cap - 1] * B if lens is None else [min(L, T_cap - 1) for L in lens]
+    sl = torch.tensor(lens_np, dtype=torch.int32, device=dev)
+    out = kvq.attend_decode(k["plan"], v["plan"], q, k["codes"], k["scales"], v["codes"], v["scales"], seq_lens=sl)
+    torch.cuda.synchronize()
+    assert kvq.poll_device_errors() == 0
+
+    def oracle_out(lens_):
+        return oracle.attend_decode_int4(q16, k["codes"].cpu().numpy(), k["scales"].cpu().numpy(),
+                                         v["codes"].cpu().numpy(), v["scales"].cpu().numpy(), k["params"],
+                                         v["params"], lens_, G)
+
+    check_rel_l2(out.cpu().numpy().astype(np.float64).reshape(-1, D), oracle_out(lens_np).reshape(-1, D),
+                 label=f"G16 {case}")
+    if lens is None:
+        # the fused append at pos = T_cap - 1 with G = 16
+        new = {kind: kvgen.kv_numpy(wl, kind, (B, Hkv, D), seed=28) for kind in ("k", "v")}
+        pos = T_cap - 1
+        out2 = kvq.attend_decode_append(k["plan"], v["plan"], q, torch.from_numpy(new["k"]).to(dev),
+                                        torch.from_numpy(new["v"]).to(dev), k["codes"], k["scales"], v["codes"],
+                                        v["scales"], pos)
+        torch.cuda.synchronize()
+        assert kvq.poll_device_errors() == 0
+        for kind in ("k", "v"):
+            c = cache[kind]
+            nb, na = check_encode(new[kind][:, :, None], c["params"][0], c["params"][1], G,
+                                  c["codes"][:, :, pos:pos + 1].cpu().numpy(),
+                                  c["scales"][:, :, pos:pos + 1].cpu().numpy(), label=f"G16 append {kind}",
+                                  count_only=True)
+            BOUNDARY_TALLY["bad"] += nb
+            BOUNDARY_TALLY["all"] += na
+        check_rel_l2(out2.cpu().numpy().astype(np.float64).reshape(-1, D), oracle_out([pos + 1] * B).reshape(-1, D),
+                     label=f"G16 append {case}")
