@@ -143,8 +143,8 @@ kvq_status kvq_encode_batch(const kvq_encode_job* jobs, int njobs, void* stream)
  * kvq_set_encode_path / kvq_get_encode_path -- which kernel kvq_encode and
  * kvq_encode_batch run (process-wide setting; not on the pages):
  *   0  default: the tensor-core encode (tcgen05 GEMM against W = Lambda F_r diag(s)
- *      held as an fp16 hi + lo pair) where it exists (head_dim 128, group 32),
- *      else the register-FFT encode;
+ *      held as an fp16 hi + lo pair; for SRHT plans the exact W = H diag(s)), which
+ *      covers head_dim 128 and 256 with group 32 or 16;
  *   1  always the register-FFT encode (one radix-2 real FFT per vector in registers);
  *   2  always the tensor-core encode (KVQ_ERR_UNSUPPORTED where it does not exist).
  * Both produce codes and scales that meet the same acceptance rule against the

@@ -82,7 +82,7 @@ kvq_status dispatch_encode(const kvq_encode_job* jobs, int njobs, cudaStream_t s
   const int path = g_encode_path.load();
   const bool tc = encode_tc_supported(p->D, p->G) && p->wt_dev != nullptr;
   if (path == 2 && !tc)
-    return fail(KVQ_ERR_UNSUPPORTED, "encode: the tensor-core path supports head_dim 128 with group 32 only");
+    return fail(KVQ_ERR_UNSUPPORTED, "encode: the tensor-core path supports head_dim 128 or 256 with group 32 or 16");
   if (tc && path != 1) return launch_encode_tc(jobs, njobs, s);
   return launch_encode_jobs(jobs, njobs, s);
 }

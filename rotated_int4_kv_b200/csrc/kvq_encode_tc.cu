@@ -58,7 +58,7 @@ struct alignas(64) TcJob {
   CUtensorMap xmap;  // x as [rows][D] fp16, box {64, 128}, 128-byte swizzle
   CUtensorMap wmap;  // W as [2D][D] fp16 (hi rows, then lo rows; EX: [D][D]), box {64, N}, 128-byte swizzle
   uint8_t* codes;    // [BH][T_cap][D/2]
-  uint16_t* scales;  // [BH][T_cap][D/32]
+  uint16_t* scales;  // [BH][T_cap][D/G]
   const float* chan; // EX: the per-channel factors lambda_c / sqrt(D)
   int rows, n, T_cap, pos, tile0;  // rows = B*H*n; tile0 = first global tile of the job
 };
@@ -89,7 +89,40 @@ __device__ __forceinline__ int job_of(const TcJob* jobs, int njobs, int job, int
   return job;
 }
 
-template <int D, bool EX, int MAXJ>
+// The quantiser over one 32-channel chunk: one group of 32 or two of 16 (sb: their scales).
+template <int G>
+__device__ __forceinline__ void quantize_chunk(const float (&y)[32], uint32_t (&w)[4], uint32_t (&sb)[32 / G]) {
+  if constexpr (G == 32) {
+    quantize_group<32>(y, w, sb[0]);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      float yh[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) yh[i] = y[16 * j + i];
+      uint32_t wh[2];
+      quantize_group<16>(yh, wh, sb[j]);
+      w[2 * j] = wh[0];
+      w[2 * j + 1] = wh[1];
+    }
+  }
+}
+
+// n consecutive fp16 scale bits (n = 2, 4 or 8) to one 4-, 8- or 16-byte store
+template <int N>
+__device__ __forceinline__ void store_scales(uint16_t* dst, const uint32_t (&sb)[N]) {
+  static_assert(N == 2 || N == 4 || N == 8, "scale count");
+  if constexpr (N == 2) {
+    *reinterpret_cast<uint32_t*>(dst) = sb[0] | (sb[1] << 16);
+  } else if constexpr (N == 4) {
+    *reinterpret_cast<uint2*>(dst) = make_uint2(sb[0] | (sb[1] << 16), sb[2] | (sb[3] << 16));
+  } else {
+    *reinterpret_cast<uint4*>(dst) = make_uint4(sb[0] | (sb[1] << 16), sb[2] | (sb[3] << 16), sb[4] | (sb[5] << 16),
+                                                sb[6] | (sb[7] << 16));
+  }
+}
+
+template <int D, bool EX, int G, int MAXJ>
 __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_constant__ TcBatch<MAXJ> bt) {
   using C = TcCfg<D, EX>;
   constexpr int kTcChunks = C::kChunks;
@@ -246,7 +279,8 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
     // ------------------------------------------------------------ epilogue
     // warp w: TMEM lanes 32 (w % 4) .. + 31 (one vector per thread), channel groups
     // [h * NGH, (h + 1) * NGH) of the CTA's channels with h = (w - 2) / 4
-    constexpr int NGH = EX ? D / 64 : 2;  // groups per thread: two threads per vector
+    constexpr int NGH = EX ? D / 64 : 2;  // 32-channel chunks per thread: two threads per vector
+    constexpr int SPC = 32 / G;            // scale groups per chunk
     const int q = warp & 3;
     const int h = (warp - 2) >> 2;
     int job = ntile > 0 ? job_of(bt.j, bt.njobs, 0, t_begin) : 0;
@@ -266,7 +300,7 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
       const int bh = valid ? r / J.n : 0;
       const size_t orow = (size_t)bh * J.T_cap + J.pos + (r - bh * J.n);
       const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * C::kN + 32 * NGH * h);
-      uint32_t sb[NGH];
+      uint32_t sb[NGH * SPC];
       if constexpr (EX) {
         // Y exact up to the fp32 accumulation; y = Y * lambda_c / sqrt(D)
         float y[NGH][32];
@@ -289,19 +323,14 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
             y[g][4 * e + 2] *= f.z;
             y[g][4 * e + 3] *= f.w;
           }
-          uint32_t w[4];
-          quantize_group<32>(y[g], w, sb[g]);
+          uint32_t w[4], sg[SPC];
+          quantize_chunk<G>(y[g], w, sg);
+#pragma unroll
+          for (int j = 0; j < SPC; ++j) sb[SPC * g + j] = sg[j];
           if (valid)
             reinterpret_cast<uint4*>(J.codes + orow * (D / 2))[NGH * h + g] = make_uint4(w[0], w[1], w[2], w[3]);
         }
-        if (valid) {
-          if constexpr (NGH == 4) {
-            reinterpret_cast<uint2*>(J.scales + orow * (D / 32))[h] = make_uint2(sb[0] | (sb[1] << 16),
-                                                                                 sb[2] | (sb[3] << 16));
-          } else {
-            reinterpret_cast<uint32_t*>(J.scales + orow * (D / 32))[h] = sb[0] | (sb[1] << 16);
-          }
-        }
+        if (valid) store_scales<NGH * SPC>(J.scales + orow * (D / G) + NGH * SPC * h, sb);
       } else {
         float y[NGH][32], ylo[NGH][32];
 #pragma unroll
@@ -327,13 +356,15 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
             y[g][e] = v.x;
             y[g][e + 1] = v.y;
           }
-          uint32_t w[4];
-          quantize_group<32>(y[g], w, sb[g]);
+          uint32_t w[4], sg[SPC];
+          quantize_chunk<G>(y[g], w, sg);
+#pragma unroll
+          for (int j = 0; j < SPC; ++j) sb[SPC * g + j] = sg[j];
           if (valid)
             reinterpret_cast<uint4*>(J.codes + orow * (D / 2))[4 * half + NGH * h + g] =
                 make_uint4(w[0], w[1], w[2], w[3]);
         }
-        if (valid) reinterpret_cast<uint32_t*>(J.scales + orow * (D / 32))[2 * half + h] = sb[0] | (sb[1] << 16);
+        if (valid) store_scales<NGH * SPC>(J.scales + orow * (D / G) + SPC * (4 * half + NGH * h), sb);
       }
     }
   }
@@ -348,23 +379,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
 }
 
 
+template <int D, bool EX, int G>
+void tc_prepare_one() {
+  cudaFuncSetAttribute(encode_tc_kernel<D, EX, G, kTcMaxJobs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                       TcCfg<D, EX>::kSmem);
+}
+
 void tc_prepare() {
   static std::once_flag once;
   std::call_once(once, [] {
-    cudaFuncSetAttribute(encode_tc_kernel<128, false, kTcMaxJobs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         TcCfg<128, false>::kSmem);
-    cudaFuncSetAttribute(encode_tc_kernel<256, false, kTcMaxJobs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         TcCfg<256, false>::kSmem);
-    cudaFuncSetAttribute(encode_tc_kernel<128, true, kTcMaxJobs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         TcCfg<128, true>::kSmem);
-    cudaFuncSetAttribute(encode_tc_kernel<256, true, kTcMaxJobs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         TcCfg<256, true>::kSmem);
+    tc_prepare_one<128, false, 32>();
+    tc_prepare_one<256, false, 32>();
+    tc_prepare_one<128, true, 32>();
+    tc_prepare_one<256, true, 32>();
+    tc_prepare_one<128, false, 16>();
+    tc_prepare_one<256, false, 16>();
+    tc_prepare_one<128, true, 16>();
+    tc_prepare_one<256, true, 16>();
   });
+}
+
+template <int D, bool EX, int G>
+cudaError_t tc_launch(cudaLaunchConfig_t cfg, const TcBatch<kTcMaxJobs>& bt, int tiles, int sms) {
+  cfg.gridDim = dim3(TcCfg<D, EX>::kSplit == 2 ? 2 * std::min(tiles, sms / 2) : std::min(tiles, sms));
+  cfg.dynamicSmemBytes = TcCfg<D, EX>::kSmem;
+  return cudaLaunchKernelEx(&cfg, encode_tc_kernel<D, EX, G, kTcMaxJobs>, bt);
 }
 
 }  // namespace
 
-bool encode_tc_supported(int D, int G) { return (D == 128 || D == 256) && G == 32; }
+bool encode_tc_supported(int D, int G) { return (D == 128 || D == 256) && (G == 32 || G == 16); }
 
 // Grouped launch over jobs of one head_dim (128 or 256, group 32); jobs with no rows are skipped.
 kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t strm) {
@@ -425,24 +469,16 @@ kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    const int G = jobs[0].plan->G;
     cudaError_t e;
-    if (ex) {
-      cfg.gridDim = dim3(std::min(tiles, sms));
-      if (D == 128) {
-        cfg.dynamicSmemBytes = TcCfg<128, true>::kSmem;
-        e = cudaLaunchKernelEx(&cfg, encode_tc_kernel<128, true, kTcMaxJobs>, bt);
-      } else {
-        cfg.dynamicSmemBytes = TcCfg<256, true>::kSmem;
-        e = cudaLaunchKernelEx(&cfg, encode_tc_kernel<256, true, kTcMaxJobs>, bt);
-      }
-    } else if (D == 128) {
-      cfg.gridDim = dim3(std::min(tiles, sms));
-      cfg.dynamicSmemBytes = TcCfg<128, false>::kSmem;
-      e = cudaLaunchKernelEx(&cfg, encode_tc_kernel<128, false, kTcMaxJobs>, bt);
+    if (G == 32) {
+      e = ex ? (D == 128 ? tc_launch<128, true, 32>(cfg, bt, tiles, sms) : tc_launch<256, true, 32>(cfg, bt, tiles, sms))
+             : (D == 128 ? tc_launch<128, false, 32>(cfg, bt, tiles, sms)
+                         : tc_launch<256, false, 32>(cfg, bt, tiles, sms));
     } else {
-      cfg.gridDim = dim3(2 * std::min(tiles, sms / 2));
-      cfg.dynamicSmemBytes = TcCfg<256, false>::kSmem;
-      e = cudaLaunchKernelEx(&cfg, encode_tc_kernel<256, false, kTcMaxJobs>, bt);
+      e = ex ? (D == 128 ? tc_launch<128, true, 16>(cfg, bt, tiles, sms) : tc_launch<256, true, 16>(cfg, bt, tiles, sms))
+             : (D == 128 ? tc_launch<128, false, 16>(cfg, bt, tiles, sms)
+                         : tc_launch<256, false, 16>(cfg, bt, tiles, sms));
     }
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("encode (tensor cores) launch: ") + cudaGetErrorString(e));

@@ -29,8 +29,6 @@ def _plan(kvq, D, kind, layer=0, G=32, seed=61):
 @pytest.mark.parametrize("wl_name,B,H,n,G", [("qwen", 2, 2, 130, 32), ("gemma", 1, 1, 300, 32), ("toy", 1, 1, 77, 16),
                                              ("gemma", 2, 1, 65, 16)])
 def test_srht_encode_decode(kvq, path, wl_name, B, H, n, G):
-    if path == "tensor" and G != 32:
-        pytest.skip("the tensor-core encode takes group 32")
     wl = kvgen.WORKLOADS[wl_name]
     D = wl.head_dim
     plan, (s, lam) = _plan(kvq, D, "k", G=G)
