@@ -224,6 +224,37 @@ kvq_status kvq_attend_decode_append(const kvq_plan* pk, const kvq_plan* pv, cons
                                     uint16_t* out, void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * kvq_attend_decode_partial -- sequence-sharded (context-parallel) decode, step 1: the
+ * attention of kvq_attend_decode over cached tokens t_begin .. t_end - 1 only, left as
+ * each query head's softmax partial in the rotated domain instead of an output (a GPU
+ * holding one slice of a long context attends over its slice; the slices' partials are
+ * exchanged, e.g. by an all-gather, and merged by kvq_attend_combine). Not on the pages.
+ *   partial   fp32 [B, Hq, D + 4]: per query head m (the maximum of the scores, in
+ *             base-2 units of softmax_scale * score), l (sum of 2^(score - m)), two pad
+ *             floats, o_t[D] = sum 2^(score - m) cV * scaleV (rotated domain, not
+ *             normalised). A head with no tokens gets m = -inf, l = 0, o_t = 0.
+ *   t_begin   even, 0 <= t_begin <= t_end <= T_cap; the same range for every batch entry.
+ *   other arguments as kvq_attend_decode (no seq_lens).
+ * Errors: as kvq_attend_decode.
+ */
+kvq_status kvq_attend_decode_partial(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q,
+                                     const uint8_t* k_codes, const uint16_t* k_scales,
+                                     const uint8_t* v_codes, const uint16_t* v_scales, int B, int Hq,
+                                     int Hkv, int T_cap, int t_begin, int t_end, float softmax_scale,
+                                     float* partial, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * kvq_attend_combine -- step 2: merges n_parts partials of the same query heads (fp32
+ * [n_parts, B, Hq, D + 4], e.g. gathered from the GPUs of a context-parallel group) by
+ * the log-sum-exp rule, M = max m_r, L = sum l_r 2^(m_r - M), O = sum o_r 2^(m_r - M),
+ * and un-rotates O / L with the V plan: the result equals kvq_attend_decode over the
+ * union of the ranges up to fp32 rounding. 1 <= n_parts <= 64.
+ *   out   fp16 [B, Hq, D]. Errors: INVALID_ARG, UNSUPPORTED, ALIGNMENT, DEVICE, CUDA.
+ */
+kvq_status kvq_attend_combine(const kvq_plan* pv, const float* partials, int n_parts, int B, int Hq,
+                              uint16_t* out, void* stream);
+
+/*
  * kvq_attend_decode_batch -- kvq_attend_decode for many independent problems of one
  * shape in one grouped launch (up to 32 per launch; more are run as consecutive
  * launches on the stream), e.g. the decode attention of every layer of a model

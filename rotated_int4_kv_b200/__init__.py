@@ -5,12 +5,14 @@ The compute path lives in ``libkvq.so`` (hand-written CUDA for sm_100a, C ABI in
 """
 from ._lib import LIB_PATH, KvqError, lib  # noqa: F401
 from .cache import Int4KVCache  # noqa: F401
-from .api import (Plan, attend_decode, attend_decode_append, attend_decode_batch, attend_decode_noalloc,  # noqa: F401
-                  attend_decode_ref,
+from .api import (Plan, attend_combine, attend_decode, attend_decode_append, attend_decode_batch,  # noqa: F401
+                  attend_decode_context_parallel, attend_decode_noalloc, attend_decode_partial, attend_decode_ref,
+                  gather_partials,
                   decode, encode, encode_batch, get_encode_path, make_workspace, poll_device_errors, set_encode_path,
                   workspace_size)
 
-__all__ = ["Plan", "Int4KVCache", "encode", "encode_batch", "decode", "attend_decode", "attend_decode_append", "attend_decode_batch",
+__all__ = ["Plan", "Int4KVCache", "attend_decode_partial", "attend_combine", "gather_partials",
+           "attend_decode_context_parallel", "encode", "encode_batch", "decode", "attend_decode", "attend_decode_append", "attend_decode_batch",
            "attend_decode_noalloc", "attend_decode_ref", "workspace_size", "make_workspace", "poll_device_errors",
            "set_encode_path", "get_encode_path",
            "KvqError", "LIB_PATH", "lib"]

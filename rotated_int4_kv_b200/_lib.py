@@ -51,6 +51,8 @@ def _load() -> ctypes.CDLL:
         "kvq_workspace_size": (S, [I, I, I, I, I]),
         "kvq_attend_decode": (I, [P, P, P, P, P, P, P, I, I, I, I, P, I, F, P, P, S, P]),
         "kvq_attend_decode_append": (I, [P, P, P, P, P, P, P, P, P, I, I, I, I, I, F, P, P, S, P]),
+        "kvq_attend_decode_partial": (I, [P, P, P, P, P, P, P, I, I, I, I, I, I, F, P, P, S, P]),
+        "kvq_attend_combine": (I, [P, P, I, I, I, P, P]),
         "kvq_attend_decode_ref": (I, [P, P, P, I, I, I, I, I, P, I, F, P, P, S, P]),
         "kvq_attend_decode_noalloc": (I, [P, P, P, P, P, P, P, I, I, I, I, P, I, F, P, P]),
         "kvq_attend_decode_batch": (I, [ctypes.POINTER(AttendJob), I, I, I, I, I, P, I, F, P, S, P]),

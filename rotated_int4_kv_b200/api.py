@@ -195,6 +195,66 @@ def attend_decode_append(pk: Plan, pv: Plan, q, k_new, v_new, k_codes, k_scales,
     return out
 
 
+def attend_decode_partial(pk: Plan, pv: Plan, q, k_codes, k_scales, v_codes, v_scales, t_begin: int, t_end: int,
+                          softmax_scale: float = 0.0, partial=None, workspace=None, stream=None) -> torch.Tensor:
+    """Sequence-sharded decode, step 1: the softmax partial of every query head over
+    cached tokens [t_begin, t_end) (fp32 [B, Hq, D + 4]; see kvq_attend_decode_partial)."""
+    B, Hq, D = q.shape
+    _, Hkv, T_cap, _ = k_codes.shape
+    _need(q, "q", torch.float16)
+    for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
+        _need(t, name, torch.uint8, (B, Hkv, T_cap, D // 2))
+    for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
+        _need(t, name, torch.float16, (B, Hkv, T_cap, D // pk.group))
+    if partial is None:
+        partial = torch.empty((B, Hq, D + 4), dtype=torch.float32, device=q.device)
+    _need(partial, "partial", torch.float32, (B, Hq, D + 4))
+    if workspace is None:
+        workspace = make_workspace(B, Hq, Hkv, D, T_cap, q.device)
+    check(lib.kvq_attend_decode_partial(pk.handle, pv.handle, _ptr(q), _ptr(k_codes), _ptr(k_scales), _ptr(v_codes),
+                                        _ptr(v_scales), B, Hq, Hkv, T_cap, int(t_begin), int(t_end),
+                                        float(softmax_scale), _ptr(partial), _ptr(workspace), workspace.numel(),
+                                        _stream(stream)), "kvq_attend_decode_partial")
+    return partial
+
+
+def attend_combine(pv: Plan, partials, out=None, stream=None) -> torch.Tensor:
+    """Sequence-sharded decode, step 2: merge partials fp32 [N, B, Hq, D + 4] and un-rotate
+    (see kvq_attend_combine); returns fp16 [B, Hq, D]."""
+    N, B, Hq, D4 = partials.shape
+    D = D4 - 4
+    _need(partials, "partials", torch.float32)
+    if out is None:
+        out = torch.empty((B, Hq, D), dtype=torch.float16, device=partials.device)
+    _need(out, "out", torch.float16, (B, Hq, D))
+    check(lib.kvq_attend_combine(pv.handle, _ptr(partials), N, B, Hq, _ptr(out), _stream(stream)),
+          "kvq_attend_combine")
+    return out
+
+
+def gather_partials(partial: torch.Tensor, group=None) -> torch.Tensor:
+    """All-gather of one softmax partial per rank of a context-parallel group (NCCL on
+    GPUs; any torch.distributed backend): returns [world, *partial.shape], rank order."""
+    import torch.distributed as dist
+
+    world = dist.get_world_size(group)
+    bufs = [torch.empty_like(partial) for _ in range(world)]
+    dist.all_gather(bufs, partial.contiguous(), group=group)
+    return torch.stack(bufs)
+
+
+def attend_decode_context_parallel(pk: Plan, pv: Plan, q, k_codes, k_scales, v_codes, v_scales, t_begin: int,
+                                   t_end: int, group=None, softmax_scale: float = 0.0, out=None,
+                                   workspace=None) -> torch.Tensor:
+    """Decode attention over a sequence sharded across the ranks of ``group``: each rank
+    holds its slice [t_begin, t_end) of every (b, kv head) in its caches and passes the
+    same q; the partials are all-gathered ((D + 4) * 4 bytes per query head per rank) and
+    every rank merges them into the same output."""
+    part = attend_decode_partial(pk, pv, q, k_codes, k_scales, v_codes, v_scales, t_begin, t_end,
+                                 softmax_scale=softmax_scale, workspace=workspace)
+    return attend_combine(pv, gather_partials(part, group), out=out)
+
+
 def attend_decode_batch(jobs, seq_lens=None, T_len=None, softmax_scale: float = 0.0, workspace=None,
                         stream=None) -> list:
     """Grouped int4 decode attention: ``jobs`` is a sequence of

@@ -456,6 +456,41 @@ kvq_status kvq_attend_decode_append(const kvq_plan* pk, const kvq_plan* pv, cons
                                         ws, ws_bytes, (cudaStream_t)stream);
 }
 
+kvq_status kvq_attend_decode_partial(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q, const uint8_t* kc,
+                                     const uint16_t* ks, const uint8_t* vc, const uint16_t* vs, int B, int Hq, int Hkv,
+                                     int T_cap, int t_begin, int t_end, float sigma, float* partial, void* ws,
+                                     size_t ws_bytes, void* stream) {
+  if (!pk || !pv) return fail(KVQ_ERR_INVALID_ARG, "attend_partial: null plan");
+  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device || pk->xform != pv->xform)
+    return fail(KVQ_ERR_INVALID_ARG, "attend_partial: K and V plans differ in head_dim, group, transform or device");
+  if (pk->G != 32 && pk->G != 16) return fail(KVQ_ERR_UNSUPPORTED, "attend_partial: group must be 32 or 16");
+  if (t_begin < 0 || t_end < t_begin) return fail(KVQ_ERR_INVALID_ARG, "attend_partial: need 0 <= t_begin <= t_end");
+  if (t_end > T_cap) return fail(KVQ_ERR_CAPACITY, "attend_partial: t_end > T_cap");
+  if (t_begin & 1) return fail(KVQ_ERR_ALIGNMENT, "attend_partial: t_begin must be even");
+  kvq_status st = check_attend_common(B, Hq, Hkv, pk->D, T_cap, t_end - t_begin, q, partial, ws, ws_bytes);
+  if (st != KVQ_OK || B == 0) return st;
+  if (!kc || !ks || !vc || !vs) return fail(KVQ_ERR_INVALID_ARG, "attend_partial: null cache buffer");
+  if (!kvq::aligned16(kc) || !kvq::aligned16(ks) || !kvq::aligned16(vc) || !kvq::aligned16(vs))
+    return fail(KVQ_ERR_ALIGNMENT, "attend_partial: cache buffers must be 16-byte aligned");
+  st = kvq::check_plan_device(pk);
+  if (st != KVQ_OK) return st;
+  return kvq::launch_attend_int4_partial(pk, pv, q, kc, ks, vc, vs, B, Hq, Hkv, T_cap, t_begin, t_end, sigma, partial,
+                                         ws, ws_bytes, (cudaStream_t)stream);
+}
+
+kvq_status kvq_attend_combine(const kvq_plan* pv, const float* partials, int n_parts, int B, int Hq, uint16_t* out,
+                              void* stream) {
+  if (!pv) return fail(KVQ_ERR_INVALID_ARG, "attend_combine: null plan");
+  if (n_parts < 1 || B < 0 || Hq <= 0) return fail(KVQ_ERR_INVALID_ARG, "attend_combine: bad sizes");
+  if (B == 0) return KVQ_OK;
+  if (!partials || !out) return fail(KVQ_ERR_INVALID_ARG, "attend_combine: null buffer");
+  if (!kvq::aligned16(partials) || !kvq::aligned16(out))
+    return fail(KVQ_ERR_ALIGNMENT, "attend_combine: buffers must be 16-byte aligned");
+  kvq_status st = kvq::check_plan_device(pv);
+  if (st != KVQ_OK) return st;
+  return kvq::launch_attend_combine(pv, partials, n_parts, B, Hq, out, (cudaStream_t)stream);
+}
+
 kvq_status kvq_attend_decode_batch(const kvq_attend_job* jobs, int njobs, int B, int Hq, int Hkv, int T_cap,
                                    const int32_t* seq_lens, int T_len, float sigma, void* ws, size_t ws_bytes,
                                    void* stream) {

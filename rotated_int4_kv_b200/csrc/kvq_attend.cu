@@ -133,6 +133,12 @@ struct AttnParams {
   uint16_t* vs_out;
   int append_pos;
   int xform;  // the plans' kvq_transform (0 SRFT, 1 SRHT)
+  // sequence-sharded (context-parallel) decode: the tokens streamed are
+  // [t_base, t_base + T_len) of every (b, kv head); with part_out set the result of
+  // each query head is not un-rotated but written as its softmax partial
+  // (m, l, pad, pad, o_t[D]) in fp32, m in base-2 units of the scaled scores
+  int t_base;
+  float* part_out;
 };
 
 // One attention problem of a launch: its caches (as tensor maps), query, output
@@ -715,19 +721,21 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G>::kThreads), (Cfg<D, INT4, G>:
         mbar_arrive_expect_tx(&full[s], C::kStageBytes);
         const uint64_t pol = l2_evict_first_policy();
         if constexpr (INT4) {
-          tma_load_2d_hint(st, &J.kmap, &full[s], 0, row0 + t0, pol);
-          tma_load_2d_hint(st + C::kKBytes, &J.vmap, &full[s], 0, row0 + t0, pol);
+          tma_load_2d_hint(st, &J.kmap, &full[s], 0, row0 + p.t_base + t0, pol);
+          tma_load_2d_hint(st + C::kKBytes, &J.vmap, &full[s], 0, row0 + p.t_base + t0, pol);
 #pragma unroll
           for (int j = 0; j < C::kScaleLoads; ++j) {
-            tma_load_2d(st + 2 * C::kKBytes + j * C::kScaleBox * 2, &J.ksmap, &full[s], t0 * NG + j * C::kScaleBox, bk);
+            tma_load_2d(st + 2 * C::kKBytes + j * C::kScaleBox * 2, &J.ksmap, &full[s],
+                        (p.t_base + t0) * NG + j * C::kScaleBox, bk);
             tma_load_2d(st + 2 * C::kKBytes + C::kSBytes + j * C::kScaleBox * 2, &J.vsmap, &full[s],
-                        t0 * NG + j * C::kScaleBox, bk);
+                        (p.t_base + t0) * NG + j * C::kScaleBox, bk);
           }
         } else {
 #pragma unroll
           for (int j = 0; j < D / 64; ++j) {
-            tma_load_2d_hint(st + j * C::kTile * 128, &J.kmap, &full[s], 64 * j, row0 + t0, pol);
-            tma_load_2d_hint(st + C::kKBytes + j * C::kTile * 128, &J.vmap, &full[s], 64 * j, row0 + t0, pol);
+            tma_load_2d_hint(st + j * C::kTile * 128, &J.kmap, &full[s], 64 * j, row0 + p.t_base + t0, pol);
+            tma_load_2d_hint(st + C::kKBytes + j * C::kTile * 128, &J.vmap, &full[s], 64 * j, row0 + p.t_base + t0,
+                             pol);
           }
         }
       }
@@ -1358,6 +1366,15 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G>::kThreads), (Cfg<D, INT4, G>:
   }
 
   // ------------------------------------------------------------ normalise, un-rotate, store fp16
+  if (INT4 && p.part_out) {
+    // sequence-sharded decode: the unit's softmax partial, rotated domain, unnormalised
+    float* pb = p.part_out + ((size_t)b * p.Hq + hq0) * (D + 4);
+    for (int i = threadIdx.x; i < heads * (D + 4); i += kThreads) {
+      const int h = i / (D + 4), e = i - h * (D + 4);
+      pb[i] = e == 0 ? mrg[h] : (e == 1 ? mrg[kHT + h] : (e < 4 ? 0.0f : om[h * D + e - 4]));
+    }
+    return;
+  }
   uint16_t* ob = J.out + ((size_t)b * p.Hq + hq0) * D;
   if constexpr (C::kMmaRot) {
     if constexpr (D == 128) {
@@ -1376,6 +1393,104 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G>::kThreads), (Cfg<D, INT4, G>:
       const float r = L > 0.0f ? 1.0f / L : 0.0f;
       reinterpret_cast<uint32_t*>(ob)[i] = pack_half2(om[2 * i] * r, om[2 * i + 1] * r);
     }
+  }
+}
+
+// ---------------------------------------------------------------- partial combine
+// Sequence-sharded decode: the N softmax partials of a query head (rotated domain,
+// fp32 [N][B][Hq][D + 4] rows m, l, pad, pad, o_t[D]) merge by the log-sum-exp rule,
+// M = max m_r, L = sum l_r 2^(m_r - M), O = sum o_r 2^(m_r - M), and O / L is un-rotated
+// with the V plan as in the attention kernel. One CTA (four warps) per (8-head tile, b).
+constexpr int kCombineThreads = 128;
+constexpr int kMaxParts = 64;
+
+template <int D>
+struct CombineSmem {
+  static constexpr int kRot = 4 * 128 * 128;           // F128 (or H128) hi/lo, 128-byte swizzle
+  static constexpr int kOm = kHT * D * 4;              // merged o_t
+  static constexpr int kXb = kHT * D * 4;              // un-rotated output
+  static constexpr int kEo = D == 256 ? 2 * 8 * 128 * 4 : 0;
+  static constexpr int kW = kMaxParts * kHT * 4;       // merge weights
+  static constexpr int kConsts = D * 4 + D * 2;        // V plan: dg / lambda, sign masks
+  static constexpr int kBytes = kRot + kOm + kXb + kEo + kW + kConsts + 16 * 4 + 64 + 1024;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kCombineThreads) combine_kernel(const __grid_constant__ CUtensorMap rotmap,
+                                                                  const CodecConsts* vd, const float* parts, int N,
+                                                                  int B, int Hq, uint16_t* out, int xform) {
+  using C = CombineSmem<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* srot = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  float* om = reinterpret_cast<float*>(srot + C::kRot);
+  float* xb = om + kHT * D;
+  float* eo = xb + kHT * D;
+  float* wsm = eo + C::kEo / 4;
+  float* vch = wsm + kMaxParts * kHT;
+  uint32_t* vsg = reinterpret_cast<uint32_t*>(vch + D);
+  float* mrg = reinterpret_cast<float*>(vsg + D / 2);
+  uint64_t* bar = reinterpret_cast<uint64_t*>(mrg + 16);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.y, h0 = blockIdx.x * kHT;
+  const int heads = min(kHT, Hq - h0);
+  const bool hada = xform == 1;
+  if (threadIdx.x == 0) {
+    mbar_init(bar, 1);
+    fence_mbarrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    mbar_arrive_expect_tx(bar, (uint32_t)(C::kRot + C::kConsts));
+#pragma unroll
+    for (int hl = 0; hl < 2; ++hl)
+#pragma unroll
+      for (int kc = 0; kc < 2; ++kc) tma_load_2d(srot + (2 * hl + kc) * 16384, &rotmap, bar, 64 * kc, 128 * hl);
+    bulk_load(vch, vd->chan, D * 4, bar);
+    bulk_load(vsg, vd->sgn, D * 2, bar);
+  }
+  const size_t rstride = (size_t)B * Hq * (D + 4);  // one partial to the next
+  const float* pb = parts + ((size_t)b * Hq + h0) * (D + 4);
+  if (threadIdx.x < kHT) {
+    const int h = threadIdx.x;
+    float M = -INFINITY, L = 0.0f;
+    if (h < heads) {
+      for (int r = 0; r < N; ++r) M = fmaxf(M, pb[r * rstride + (size_t)h * (D + 4)]);
+      for (int r = 0; r < N; ++r) {
+        const float mr = pb[r * rstride + (size_t)h * (D + 4)];
+        const float w = (M == -INFINITY || mr == -INFINITY) ? 0.0f : fast_exp2(mr - M);
+        wsm[r * kHT + h] = w;
+        L = fmaf(w, pb[r * rstride + (size_t)h * (D + 4) + 1], L);
+      }
+    }
+    mrg[h] = M;
+    mrg[kHT + h] = L;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < heads * D / 4; i += kCombineThreads) {
+    const int h = (4 * i) / D, c4 = i - h * (D / 4);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int r = 0; r < N; ++r) {
+      const float w = wsm[r * kHT + h];
+      const float4 v = __ldg(reinterpret_cast<const float4*>(pb + r * rstride + (size_t)h * (D + 4) + 4) + c4);
+      acc.x = fmaf(w, v.x, acc.x);
+      acc.y = fmaf(w, v.y, acc.y);
+      acc.z = fmaf(w, v.z, acc.z);
+      acc.w = fmaf(w, v.w, acc.w);
+    }
+    reinterpret_cast<float4*>(om)[i] = acc;
+  }
+  if (!mbar_wait_bounded(bar, 0) && threadIdx.x == 0) atomicOr(&g_attend_err, kErrTimeoutLoad);
+  __syncthreads();
+  if constexpr (D == 128) {
+    unrotate_out_f128(om, heads, mrg + kHT, vch, srot, xb, warp, lane, hada);
+  } else {
+    unrotate_out_eo<4>(om, heads, mrg + kHT, vch, srot, eo, xb, warp, lane, hada);
+  }
+  __syncthreads();
+  uint16_t* ob = out + ((size_t)b * Hq + h0) * D;
+  for (int i = threadIdx.x; i < heads * D / 2; i += kCombineThreads) {
+    const int j = i % (D / 2);
+    reinterpret_cast<uint32_t*>(ob)[i] = pack_half2(xb[2 * i], xb[2 * i + 1]) ^ vsg[j];
   }
 }
 
@@ -1603,12 +1718,19 @@ struct AppendHost {
   int pos;
 };
 
+// A sequence-sharded call: the token range's start and the partials' destination.
+struct RangeHost {
+  int t_base;
+  float* part_out;
+};
+
 // One launch over nj <= MAXJ problems of equal shape (with app: the fused append, T_len =
-// the tokens already cached = app->pos).
+// the tokens already cached = app->pos; with range: tokens [t_base, t_base + T_len) and
+// softmax partials instead of outputs).
 template <int D, bool INT4, int MAXJ, int G = 32>
 kvq_status launch_chunk(const AttendJobHost* jobs, int nj, int B, int Hq, int Hkv, int T_cap, const int32_t* seq_lens,
                         int T_len, float sigma, void* ws, size_t ws_bytes, cudaStream_t strm,
-                        const AppendHost* app = nullptr) {
+                        const AppendHost* app = nullptr, const RangeHost* range = nullptr) {
   using C = Cfg<D, INT4, G>;
   const int T_split = seq_lens ? T_cap : T_len;
   const int Bj = nj * B;  // the jobs of a launch split like a larger batch
@@ -1639,6 +1761,12 @@ kvq_status launch_chunk(const AttendJobHost* jobs, int nj, int B, int Hq, int Hk
   prm.part = reinterpret_cast<float*>(wsb + ws_cnt_bytes(units));
   prm.append_pos = -1;
   prm.xform = INT4 ? jobs[0].pk->xform : 0;
+  prm.t_base = 0;
+  prm.part_out = nullptr;
+  if (range) {
+    prm.t_base = range->t_base;
+    prm.part_out = range->part_out;
+  }
   if (app) {
     prm.k_new = app->k_new;
     prm.v_new = app->v_new;
@@ -1735,6 +1863,52 @@ kvq_status launch_attend_int4_append(const kvq_plan* pk, const kvq_plan* pv, con
   if (pk->D == 128)
     return launch_chunk<128, true, 1, 16>(&job, 1, B, Hq, Hkv, T_cap, nullptr, pos, sigma, ws, ws_bytes, s, &app);
   return launch_chunk<256, true, 1, 16>(&job, 1, B, Hq, Hkv, T_cap, nullptr, pos, sigma, ws, ws_bytes, s, &app);
+}
+
+kvq_status launch_attend_int4_partial(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q, const uint8_t* kc,
+                                      const uint16_t* ks, const uint8_t* vc, const uint16_t* vs, int B, int Hq,
+                                      int Hkv, int T_cap, int t_begin, int t_end, float sigma, float* part, void* ws,
+                                      size_t ws_bytes, cudaStream_t s) {
+  const AttendJobHost job{pk, pv, q, kc, ks, vc, vs, nullptr};
+  const RangeHost rg{t_begin, part};
+  const int T = t_end - t_begin;
+  if (pk->D == 128 && pk->G == 32)
+    return launch_chunk<128, true, 1, 32>(&job, 1, B, Hq, Hkv, T_cap, nullptr, T, sigma, ws, ws_bytes, s, nullptr, &rg);
+  if (pk->D == 256 && pk->G == 32)
+    return launch_chunk<256, true, 1, 32>(&job, 1, B, Hq, Hkv, T_cap, nullptr, T, sigma, ws, ws_bytes, s, nullptr, &rg);
+  if (pk->D == 128)
+    return launch_chunk<128, true, 1, 16>(&job, 1, B, Hq, Hkv, T_cap, nullptr, T, sigma, ws, ws_bytes, s, nullptr, &rg);
+  return launch_chunk<256, true, 1, 16>(&job, 1, B, Hq, Hkv, T_cap, nullptr, T, sigma, ws, ws_bytes, s, nullptr, &rg);
+}
+
+namespace {
+template <int D>
+kvq_status run_combine(const kvq_plan* pv, const float* parts, int N, int B, int Hq, uint16_t* out, cudaStream_t s) {
+  static std::once_flag once;
+  std::call_once(once, [] {
+    cudaFuncSetAttribute(combine_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, CombineSmem<D>::kBytes);
+  });
+  CUtensorMap rotmap;
+  const uint64_t rd[2] = {128u, 256u};
+  const uint64_t rs[1] = {256u};
+  const uint32_t rb[2] = {64u, 128u};
+  kvq_status st = encode_tiled(&rotmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, pv->rot_dev, rd, rs, rb,
+                               CU_TENSOR_MAP_SWIZZLE_128B, "F128");
+  if (st != KVQ_OK) return st;
+  const dim3 grid((unsigned)((Hq + kHT - 1) / kHT), (unsigned)B);
+  combine_kernel<D><<<grid, kCombineThreads, CombineSmem<D>::kBytes, s>>>(rotmap, pv->dec_dev, parts, N, B, Hq, out,
+                                                                          pv->xform);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("combine launch: ") + cudaGetErrorString(e));
+  return KVQ_OK;
+}
+}  // namespace
+
+kvq_status launch_attend_combine(const kvq_plan* pv, const float* parts, int N, int B, int Hq, uint16_t* out,
+                                 cudaStream_t s) {
+  if (N > kMaxParts) return fail(KVQ_ERR_UNSUPPORTED, "attend_combine: more than 64 partials");
+  if (pv->D == 128) return run_combine<128>(pv, parts, N, B, Hq, out, s);
+  return run_combine<256>(pv, parts, N, B, Hq, out, s);
 }
 
 kvq_status launch_attend_fp16(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq, int Hkv, int D,

@@ -102,6 +102,12 @@ kvq_status launch_attend_int4_append(const kvq_plan* pk, const kvq_plan* pv, con
                                      const uint16_t* v_new, uint8_t* kc, uint16_t* ks, uint8_t* vc, uint16_t* vs, int B,
                                      int Hq, int Hkv, int T_cap, int pos, float sigma, uint16_t* out, void* ws,
                                      size_t ws_bytes, cudaStream_t s);
+kvq_status launch_attend_int4_partial(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q, const uint8_t* kc,
+                                      const uint16_t* ks, const uint8_t* vc, const uint16_t* vs, int B, int Hq,
+                                      int Hkv, int T_cap, int t_begin, int t_end, float sigma, float* part, void* ws,
+                                      size_t ws_bytes, cudaStream_t s);
+kvq_status launch_attend_combine(const kvq_plan* pv, const float* parts, int N, int B, int Hq, uint16_t* out,
+                                 cudaStream_t s);
 kvq_status launch_attend_fp16(const uint16_t* q, const uint16_t* k, const uint16_t* v, int B, int Hq,
                               int Hkv, int D, int T_cap, const int32_t* seq_lens, int T_len, float sigma,
                               uint16_t* out, void* ws, size_t ws_bytes, cudaStream_t s);

@@ -51,6 +51,9 @@ def test_status_strings_and_host_checks():
     assert lib.kvq_attend_decode_append(None, None, None, None, None, None, None, None, None, 1, 4, 1, 64, 10,
                                         ctypes.c_float(0), None, None, 0, None) == -1
     assert b"null plan" in lib.kvq_last_error()
+    assert lib.kvq_attend_decode_partial(None, None, None, None, None, None, None, 1, 4, 1, 64, 0, 32,
+                                         ctypes.c_float(0), None, None, 0, None) == -1
+    assert lib.kvq_attend_combine(None, None, 2, 1, 4, None, None) == -1
     assert lib.kvq_encode_batch(None, -1, None) == -1
     assert lib.kvq_encode_batch(None, 0, None) == 0
     assert lib.kvq_attend_decode_batch(None, -1, 1, 4, 1, 64, None, 64, ctypes.c_float(0), None, 0, None) == -1
