@@ -58,9 +58,9 @@ KERNEL_SOURCES = {
 }
 NCU_TRAFFIC = {
     # kernel -> (source digest at capture time, bytes per launch)
-    "encode": ("800dad8c026c", 115282176),       # register-FFT encode, Gemma step (52 jobs)
-    "encode_tc": ("424d112ae180", 124641024),    # tensor-core encode, Gemma step (52 jobs)
-    "attend": ("71f8ac5bccce", 32592896),        # grouped int4 attention, Gemma step (26 jobs)
+    "encode": ("e66cb71d3607", 112104533),       # register-FFT encode, Gemma step (52 jobs)
+    "encode_tc": ("32a6058a33bc", 124299349),    # tensor-core encode, Gemma step (52 jobs)
+    "attend": ("4d35af3b22da", 32610219),        # grouped int4 attention, Gemma step (26 jobs)
 }
 
 
@@ -263,6 +263,7 @@ def run_kvq(args, rank: int, world: int):
     local = int(os.environ.get("LOCAL_RANK", "0"))
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
+    kvq.set_encode_path(args.encode_path)
     wl = kvgen.WORKLOADS[WORKLOAD]
     L, Hkv, Hq, D, T, G = wl.layers, wl.h_kv, wl.h_q, wl.head_dim, wl.contexts[0], wl.group
     seed = kvgen.DEFAULT_SEED + 1000 * rank
@@ -428,7 +429,7 @@ def run_kvq(args, rank: int, world: int):
         res = {
             "metric": METRIC, "value": value, "unit": "Mvec/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": _config(wl),
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": dict(_config(wl), encode_path=args.encode_path),
             "encode": {"kernel_us": 1e3 * enc_avg, "ns_per_vec": 1e6 * enc_avg / vec_step,
                        "Mvec_s": vec_step / (enc_avg * 1e-3) / 1e6, "GB_s": enc_gbs,
                        "frac_hbm": enc_gbs / hbm, "frac_hbm_8TBs_nominal": enc_gbs / 8000.0,
@@ -645,6 +646,9 @@ def main(argv=None):
                     help="profiling mode: run --steps eager steps without timing, for ncu captures")
     ap.add_argument("--transform", default="srft", choices=["srft", "srht"],
                     help="the plans' rotation: srft (the pages' method) or srht (the Hadamard variant)")
+    ap.add_argument("--encode-path", default="auto", choices=["auto", "fft", "tensor"],
+                    help="encode kernel of the prefill step: tensor cores where supported (auto), "
+                         "the register FFT, or tensor cores only")
     args = ap.parse_args(argv)
     global TRANSFORM
     TRANSFORM = args.transform
