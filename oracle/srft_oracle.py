@@ -35,6 +35,11 @@ Readings taken where the pages leave a step open:
     the quantiser divides by that stored fp16 scale.
   * Codes: round half to even, clamped to [-7, 7]; a zero scale gives zero
     codes. Two's-complement nibbles, even element in the low nibble.
+  * int8 codes ([M2] names "signed int4/int8" as the rounding target and
+    defines int8 no further): the same steps with 127 in place of 7 (scale =
+    fp16_rne(min(absmax/127, 65504)), codes clamped to [-127, 127], -128 never
+    produced), one two's-complement byte per code, channel i at byte i. Every
+    function taking ``bits`` accepts 4 (default) or 8.
   * Decode: x_hat = diag(s) F_r^T (c * scale / lambda).
   * Attention (not on the pages): softmax(sigma <q, x_hat_K>) weighted sum of
     x_hat_V, sigma = 1/sqrt(D) by default; query head h reads KV head
@@ -58,6 +63,13 @@ import numpy as np
 
 FP16_MAX = 65504.0
 QMAX = 7
+
+
+def qmax(bits: int = 4) -> int:
+    """Largest code magnitude of a signed b-bit code with symmetric range: 7 or 127."""
+    if bits not in (4, 8):
+        raise ValueError("bits must be 4 or 8")
+    return (1 << (bits - 1)) - 1
 
 
 # ---------------------------------------------------------------------------
@@ -143,18 +155,18 @@ def fp16_rne(v) -> np.ndarray:
     return np.asarray(v, dtype=np.float64).astype(np.float16).astype(np.float64)
 
 
-def group_scales(y: np.ndarray, G: int) -> np.ndarray:
-    """Per-group abs-max scale: fp16_rne(min(absmax/7, 65504)); fp16 array [..., D/G]."""
+def group_scales(y: np.ndarray, G: int, bits: int = 4) -> np.ndarray:
+    """Per-group abs-max scale: fp16_rne(min(absmax/qmax, 65504)); fp16 array [..., D/G]."""
     y = np.asarray(y, dtype=np.float64)
     D = y.shape[-1]
     if D % G:
         raise ValueError("G must divide D")
     a = np.abs(y).reshape(y.shape[:-1] + (D // G, G)).max(axis=-1)
-    return np.minimum(a / QMAX, FP16_MAX).astype(np.float16)
+    return np.minimum(a / qmax(bits), FP16_MAX).astype(np.float16)
 
 
-def quantize(y: np.ndarray, scales16: np.ndarray, G: int):
-    """Signed int4 codes c = clamp(rint(y / scale), -7, 7); 0 where scale == 0.
+def quantize(y: np.ndarray, scales16: np.ndarray, G: int, bits: int = 4):
+    """Signed codes c = clamp(rint(y / scale), -qmax, qmax); 0 where scale == 0.
 
     Returns (codes int8 [..., D], pre-rounding values y/scale fp64 [..., D]).
     """
@@ -163,7 +175,7 @@ def quantize(y: np.ndarray, scales16: np.ndarray, G: int):
     sc = np.repeat(np.asarray(scales16, dtype=np.float64), G, axis=-1)
     with np.errstate(divide="ignore", invalid="ignore"):
         u = np.where(sc > 0, y / np.where(sc > 0, sc, 1.0), 0.0)
-    codes = np.clip(np.rint(u), -QMAX, QMAX).astype(np.int8)
+    codes = np.clip(np.rint(u), -qmax(bits), qmax(bits)).astype(np.int8)
     assert codes.shape[-1] == D
     return codes, u
 
@@ -189,16 +201,32 @@ def unpack_nibbles(packed: np.ndarray) -> np.ndarray:
     return out
 
 
-def encode(x: np.ndarray, signs: np.ndarray, lam: np.ndarray, G: int = 32, transform: str = "srft"):
+def pack_codes(codes: np.ndarray, bits: int = 4) -> np.ndarray:
+    """Stored code bytes: nibble pairs (bits = 4) or one two's-complement byte per code (bits = 8)."""
+    if qmax(bits) == 7:
+        return pack_nibbles(codes)
+    return (np.asarray(codes, dtype=np.int64) & 0xFF).astype(np.uint8)
+
+
+def unpack_codes(packed: np.ndarray, bits: int = 4) -> np.ndarray:
+    """Inverse of pack_codes: signed codes, int8 [..., D]."""
+    if qmax(bits) == 7:
+        return unpack_nibbles(packed)
+    b = np.asarray(packed, dtype=np.int64)
+    return np.where(b >= 128, b - 256, b).astype(np.int8)
+
+
+def encode(x: np.ndarray, signs: np.ndarray, lam: np.ndarray, G: int = 32, transform: str = "srft",
+           bits: int = 4):
     """The encode path of [ABS]/[M2] over the last axis.
 
-    Returns dict(packed=uint8 [..., D/2], scales=float16 [..., D/G],
+    Returns dict(packed=uint8 [..., D*bits/8], scales=float16 [..., D/G],
     codes=int8 [..., D], y=fp64 [..., D], u=fp64 pre-rounding y/scale).
     """
     y = srft_forward(x, signs, lam, transform)
-    scales = group_scales(y, G)
-    codes, u = quantize(y, scales, G)
-    return {"packed": pack_nibbles(codes), "scales": scales, "codes": codes, "y": y, "u": u}
+    scales = group_scales(y, G, bits)
+    codes, u = quantize(y, scales, G, bits)
+    return {"packed": pack_codes(codes, bits), "scales": scales, "codes": codes, "y": y, "u": u}
 
 
 def dequantize(codes: np.ndarray, scales16: np.ndarray, G: int) -> np.ndarray:
@@ -208,14 +236,15 @@ def dequantize(codes: np.ndarray, scales16: np.ndarray, G: int) -> np.ndarray:
 
 
 def decode(packed: np.ndarray, scales16: np.ndarray, signs: np.ndarray, lam: np.ndarray,
-           G: int = 32, transform: str = "srft") -> np.ndarray:
+           G: int = 32, transform: str = "srft", bits: int = 4) -> np.ndarray:
     """x_hat = R^T (c*scale / lambda), fp64 [..., D]."""
-    return srft_inverse(dequantize(unpack_nibbles(packed), scales16, G), signs, lam, transform)
+    return srft_inverse(dequantize(unpack_codes(packed, bits), scales16, G), signs, lam, transform)
 
 
-def compressed_bytes_per_vector(D: int, G: int) -> int:
-    """D/2 bytes of codes plus one fp16 scale per group [RES]."""
-    return D // 2 + 2 * (D // G)
+def compressed_bytes_per_vector(D: int, G: int, bits: int = 4) -> int:
+    """D*bits/8 bytes of codes plus one fp16 scale per group [RES]."""
+    qmax(bits)
+    return D * bits // 8 + 2 * (D // G)
 
 
 # ---------------------------------------------------------------------------
@@ -223,10 +252,10 @@ def compressed_bytes_per_vector(D: int, G: int) -> int:
 # ---------------------------------------------------------------------------
 
 def encode_into_cache(x: np.ndarray, signs, lam, G: int, codes_cache: np.ndarray,
-                      scales_cache: np.ndarray, pos: int) -> None:
+                      scales_cache: np.ndarray, pos: int, transform: str = "srft", bits: int = 4) -> None:
     """Encode x [B, H, n, D] and write rows pos..pos+n-1 of the cache in place."""
     n = x.shape[2]
-    enc = encode(x, signs, lam, G)
+    enc = encode(x, signs, lam, G, transform, bits)
     codes_cache[:, :, pos:pos + n, :] = enc["packed"]
     scales_cache[:, :, pos:pos + n, :] = enc["scales"]
 
@@ -266,20 +295,21 @@ def attend_decode(q: np.ndarray, k_hat: np.ndarray, v_hat: np.ndarray, seq_lens,
 
 
 def attend_decode_int4(q, k_packed, k_scales, v_packed, v_scales, k_params, v_params, seq_lens,
-                       G: int = 32, sigma: float | None = None, transform: str = "srft") -> np.ndarray:
-    """Attention over a packed int4 cache: decode K and V, then attend_decode.
+                       G: int = 32, sigma: float | None = None, transform: str = "srft",
+                       bits: int = 4) -> np.ndarray:
+    """Attention over a packed int4 (or int8) cache: decode K and V, then attend_decode.
 
     k_params / v_params = (signs, lambda) of the K and V transforms.
     """
     T = int(np.max(seq_lens))
-    kh = decode(k_packed[:, :, :T], k_scales[:, :, :T], k_params[0], k_params[1], G, transform)
-    vh = decode(v_packed[:, :, :T], v_scales[:, :, :T], v_params[0], v_params[1], G, transform)
+    kh = decode(k_packed[:, :, :T], k_scales[:, :, :T], k_params[0], k_params[1], G, transform, bits)
+    vh = decode(v_packed[:, :, :T], v_scales[:, :, :T], v_params[0], v_params[1], G, transform, bits)
     return attend_decode(q, kh, vh, seq_lens, sigma)
 
 
 def attend_decode_int4_rotated(q, k_packed, k_scales, v_packed, v_scales, k_params, v_params,
                                seq_lens, G: int = 32, sigma: float | None = None,
-                               transform: str = "srft") -> np.ndarray:
+                               transform: str = "srft", bits: int = 4) -> np.ndarray:
     """The same attention computed in the rotated domain.
 
     q_t = Lambda_K^-1 R_K q; score_t = sigma * sum_g scale_{t,g} sum_{i in g} q_t[i] c_t[i];
@@ -303,8 +333,8 @@ def attend_decode_int4_rotated(q, k_packed, k_scales, v_packed, v_scales, k_para
         for h in range(Hq):
             kv = h // grp
             qt = (Rk @ q[b, h]) / lk
-            ck = dequantize(unpack_nibbles(k_packed[b, kv, :T]), k_scales[b, kv, :T], G)
-            cv = dequantize(unpack_nibbles(v_packed[b, kv, :T]), v_scales[b, kv, :T], G)
+            ck = dequantize(unpack_codes(k_packed[b, kv, :T], bits), k_scales[b, kv, :T], G)
+            cv = dequantize(unpack_codes(v_packed[b, kv, :T], bits), v_scales[b, kv, :T], G)
             ot = _softmax_weighted(sigma * (ck @ qt), cv)
             out[b, h] = Rv.T @ (ot / lv)
     return out
