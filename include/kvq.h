@@ -96,6 +96,25 @@ kvq_status kvq_plan_create_transform(kvq_plan** out, int head_dim, int group, co
 /* The plan's kvq_transform value; -1 for a NULL plan. */
 int kvq_plan_transform(const kvq_plan* plan);
 
+/*
+ * kvq_plan_create_ex -- kvq_plan_create_transform with the code width chosen ([M2]
+ * rounds "to signed int4/int8"):
+ *   bits  4: codes clamp(rint(y / scale), -7, 7) with scale = fp16_rn(min(absmax/7,
+ *            65504)), two per byte (nibble pairs, as kvq_encode describes);
+ *         8: the same with 127 in place of 7 (scale = fp16_rn(min(absmax/127, 65504)),
+ *            codes in [-127, 127]), one two's-complement byte per channel, channel i at
+ *            byte i. Every "D/2" code row below is then D bytes.
+ *   Other values: UNSUPPORTED. int8 plans are served by the tensor-core encode (the
+ *   register-FFT path, kvq_set_encode_path(1), returns UNSUPPORTED for them), decode
+ *   and every attention entry point; both plans of an attention call, and all jobs of
+ *   a batch, must share the code width.
+ */
+kvq_status kvq_plan_create_ex(kvq_plan** out, int head_dim, int group, const int8_t* signs_host,
+                              const float* lambda_host, int transform, int bits);
+
+/* The plan's code width (4 or 8); -1 for a NULL plan. */
+int kvq_plan_bits(const kvq_plan* plan);
+
 /* Frees the plan and its device block. Passing NULL is a no-op. The caller must
  * ensure no launch that uses the plan is still pending. */
 kvq_status kvq_plan_destroy(kvq_plan* plan);

@@ -42,6 +42,8 @@ def _load() -> ctypes.CDLL:
         "kvq_plan_create": (I, [ctypes.POINTER(P), I, I, P, P]),
         "kvq_plan_create_transform": (I, [ctypes.POINTER(P), I, I, P, P, I]),
         "kvq_plan_transform": (I, [P]),
+        "kvq_plan_create_ex": (I, [ctypes.POINTER(P), I, I, P, P, I, I]),
+        "kvq_plan_bits": (I, [P]),
         "kvq_plan_destroy": (I, [P]),
         "kvq_plan_head_dim": (I, [P]),
         "kvq_plan_group": (I, [P]),

@@ -40,9 +40,11 @@ TRANSFORMS = {"srft": 0, "srht": 1}
 
 class Plan:
     """A (sign vector s, lambda) transform plan on the current CUDA device; transform
-    "srft" (the pages' method, default) or "srht" (the Hadamard variant)."""
+    "srft" (the pages' method, default) or "srht" (the Hadamard variant); bits 4 (int4
+    codes, two per byte, default) or 8 (int8 codes, one byte each). Code buffers hold
+    head_dim * bits / 8 bytes per cached vector."""
 
-    def __init__(self, signs, lam, group: int = 32, transform: str = "srft"):
+    def __init__(self, signs, lam, group: int = 32, transform: str = "srft", bits: int = 4):
         s = np.ascontiguousarray(np.asarray(signs, dtype=np.int8))
         l = np.ascontiguousarray(np.asarray(lam, dtype=np.float32))
         if s.ndim != 1 or l.shape != s.shape:
@@ -52,12 +54,17 @@ class Plan:
         self.head_dim = int(s.shape[0])
         self.group = int(group)
         self.transform = transform
+        self.bits = int(bits)
         self._h = ctypes.c_void_p()
-        check(lib.kvq_plan_create_transform(ctypes.byref(self._h), self.head_dim, self.group,
-                                            s.ctypes.data_as(ctypes.c_void_p), l.ctypes.data_as(ctypes.c_void_p),
-                                            TRANSFORMS[transform]),
-              "kvq_plan_create_transform")
+        check(lib.kvq_plan_create_ex(ctypes.byref(self._h), self.head_dim, self.group,
+                                     s.ctypes.data_as(ctypes.c_void_p), l.ctypes.data_as(ctypes.c_void_p),
+                                     TRANSFORMS[transform], self.bits),
+              "kvq_plan_create_ex")
         self._lib = lib
+
+    @property
+    def code_row_bytes(self) -> int:
+        return self.head_dim * self.bits // 8
 
     @property
     def handle(self) -> ctypes.c_void_p:
@@ -81,7 +88,7 @@ def encode(plan: Plan, x: torch.Tensor, codes: torch.Tensor, scales: torch.Tenso
     B, H, n, D = x.shape
     T_cap = codes.shape[2]
     _need(x, "x", torch.float16)
-    _need(codes, "codes", torch.uint8, (B, H, T_cap, D // 2))
+    _need(codes, "codes", torch.uint8, (B, H, T_cap, D * plan.bits // 8))
     _need(scales, "scales", torch.float16, (B, H, T_cap, D // plan.group))
     check(lib.kvq_encode(plan.handle, _ptr(x), B, H, n, _ptr(codes), _ptr(scales), T_cap, int(pos),
                          _stream(stream)), "kvq_encode")
@@ -95,7 +102,7 @@ def encode_batch(jobs, stream=None) -> None:
         B, H, n, D = x.shape
         T_cap = codes.shape[2]
         _need(x, f"jobs[{i}].x", torch.float16)
-        _need(codes, f"jobs[{i}].codes", torch.uint8, (B, H, T_cap, D // 2))
+        _need(codes, f"jobs[{i}].codes", torch.uint8, (B, H, T_cap, D * plan.bits // 8))
         _need(scales, f"jobs[{i}].scales", torch.float16, (B, H, T_cap, D // plan.group))
         arr[i] = EncodeJob(plan.handle.value, x.data_ptr(), codes.data_ptr(), scales.data_ptr(), B, H, n, T_cap,
                            int(pos))
@@ -119,9 +126,9 @@ def get_encode_path() -> str:
 def decode(plan: Plan, codes: torch.Tensor, scales: torch.Tensor, t0: int, n: int, out: torch.Tensor = None,
            stream=None) -> torch.Tensor:
     """Decode cache rows t0..t0+n-1 into fp16 [B, H, n, D]."""
-    B, H, T_cap, half = codes.shape
-    D = 2 * half
-    _need(codes, "codes", torch.uint8)
+    B, H, T_cap, _ = codes.shape
+    D = plan.head_dim
+    _need(codes, "codes", torch.uint8, (B, H, T_cap, plan.code_row_bytes))
     _need(scales, "scales", torch.float16, (B, H, T_cap, D // plan.group))
     if out is None:
         out = torch.empty((B, H, n, D), dtype=torch.float16, device=codes.device)
@@ -148,7 +155,7 @@ def attend_decode(pk: Plan, pv: Plan, q, k_codes, k_scales, v_codes, v_scales, s
     _, Hkv, T_cap, half = k_codes.shape
     _need(q, "q", torch.float16)
     for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
-        _need(t, name, torch.uint8, (B, Hkv, T_cap, D // 2))
+        _need(t, name, torch.uint8, (B, Hkv, T_cap, D * pk.bits // 8))
     for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
         _need(t, name, torch.float16, (B, Hkv, T_cap, D // pk.group))
     if seq_lens is not None:
@@ -180,7 +187,7 @@ def attend_decode_append(pk: Plan, pv: Plan, q, k_new, v_new, k_codes, k_scales,
             raise ValueError(f"{name}: expected shape {(B, Hkv, D)}, got {tuple(t.shape)}")
         _need(t, name, torch.float16)
     for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
-        _need(t, name, torch.uint8, (B, Hkv, T_cap, D // 2))
+        _need(t, name, torch.uint8, (B, Hkv, T_cap, D * pk.bits // 8))
     for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
         _need(t, name, torch.float16, (B, Hkv, T_cap, D // pk.group))
     if out is None:
@@ -203,7 +210,7 @@ def attend_decode_partial(pk: Plan, pv: Plan, q, k_codes, k_scales, v_codes, v_s
     _, Hkv, T_cap, _ = k_codes.shape
     _need(q, "q", torch.float16)
     for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
-        _need(t, name, torch.uint8, (B, Hkv, T_cap, D // 2))
+        _need(t, name, torch.uint8, (B, Hkv, T_cap, D * pk.bits // 8))
     for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
         _need(t, name, torch.float16, (B, Hkv, T_cap, D // pk.group))
     if partial is None:
@@ -274,7 +281,7 @@ def attend_decode_batch(jobs, seq_lens=None, T_len=None, softmax_scale: float = 
                                                                              device=q.device)
         _need(q, f"jobs[{i}].q", torch.float16, (B, Hq, D))
         for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
-            _need(t, f"jobs[{i}].{name}", torch.uint8, (B, Hkv, T_cap, D // 2))
+            _need(t, f"jobs[{i}].{name}", torch.uint8, (B, Hkv, T_cap, D * pk.bits // 8))
         for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
             _need(t, f"jobs[{i}].{name}", torch.float16, (B, Hkv, T_cap, D // pk.group))
         _need(out, f"jobs[{i}].out", torch.float16, (B, Hq, D))
@@ -302,7 +309,7 @@ def attend_decode_noalloc(pk: Plan, pv: Plan, q, k_codes, k_scales, v_codes, v_s
     _, Hkv, T_cap, half = k_codes.shape
     _need(q, "q", torch.float16)
     for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
-        _need(t, name, torch.uint8, (B, Hkv, T_cap, D // 2))
+        _need(t, name, torch.uint8, (B, Hkv, T_cap, D * pk.bits // 8))
     for name, t in (("k_scales", k_scales), ("v_scales", v_scales)):
         _need(t, name, torch.float16, (B, Hkv, T_cap, D // pk.group))
     if seq_lens is not None:

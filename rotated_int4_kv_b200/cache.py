@@ -19,16 +19,18 @@ class Int4KVCache:
     """Per-layer int4 K and V caches of ``capacity`` tokens for ``batch`` sequences.
 
     ``k_params`` / ``v_params``: one (signs, lambda) pair for every layer, or a list of
-    ``layers`` pairs (K and V get separate transforms); ``transform`` "srft" or "srht".
-    All sequences of the batch share the write position of a layer.
+    ``layers`` pairs (K and V get separate transforms); ``transform`` "srft" or "srht";
+    ``bits`` 4 (int4 codes) or 8 (int8 codes). All sequences of the batch share the
+    write position of a layer.
     """
 
     def __init__(self, layers: int, batch: int, kv_heads: int, head_dim: int, capacity: int, k_params, v_params,
-                 device=None, group: int = 32, transform: str = "srft"):
+                 device=None, group: int = 32, transform: str = "srft", bits: int = 4):
         if layers <= 0 or batch <= 0 or kv_heads <= 0 or capacity <= 0:
             raise ValueError("layers, batch, kv_heads and capacity must be positive")
         self.device = torch.device(device) if device is not None else torch.device("cuda")
         self.layers, self.batch, self.kv_heads, self.head_dim, self.group = layers, batch, kv_heads, head_dim, group
+        self.bits = bits
         self.capacity = capacity + (capacity & 1)  # the attention kernels fetch scale rows in 16-byte units
 
         def per_layer(params):
@@ -41,9 +43,9 @@ class Int4KVCache:
             return list(params)
 
         with torch.cuda.device(self.device):
-            self.k_plans = [Plan(s, lam, group, transform) for s, lam in per_layer(k_params)]
-            self.v_plans = [Plan(s, lam, group, transform) for s, lam in per_layer(v_params)]
-        shape_c = (batch, kv_heads, self.capacity, head_dim // 2)
+            self.k_plans = [Plan(s, lam, group, transform, bits) for s, lam in per_layer(k_params)]
+            self.v_plans = [Plan(s, lam, group, transform, bits) for s, lam in per_layer(v_params)]
+        shape_c = (batch, kv_heads, self.capacity, head_dim * bits // 8)
         shape_s = (batch, kv_heads, self.capacity, head_dim // group)
         self.k_codes = [torch.zeros(shape_c, dtype=torch.uint8, device=self.device) for _ in range(layers)]
         self.v_codes = [torch.zeros(shape_c, dtype=torch.uint8, device=self.device) for _ in range(layers)]
@@ -66,12 +68,12 @@ class Int4KVCache:
         return per * self.layers
 
     @staticmethod
-    def compression_ratio(head_dim: int, group: int = 32) -> float:
-        """fp16 K/V bytes over int4 code + fp16 scale bytes for the same tokens (3.56 at G = 32)."""
-        return (2 * head_dim) / (head_dim // 2 + 2 * (head_dim // group))
+    def compression_ratio(head_dim: int, group: int = 32, bits: int = 4) -> float:
+        """fp16 K/V bytes over code + fp16 scale bytes for the same tokens (int4: 3.56 at G = 32)."""
+        return (2 * head_dim) / (head_dim * bits // 8 + 2 * (head_dim // group))
 
     def compression_vs_fp16(self) -> float:
-        return self.compression_ratio(self.head_dim, self.group)
+        return self.compression_ratio(self.head_dim, self.group, self.bits)
 
     def _workspace(self, q_heads: int) -> torch.Tensor:
         ws = self._ws.get(q_heads)

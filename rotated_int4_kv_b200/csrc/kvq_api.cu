@@ -84,6 +84,7 @@ kvq_status dispatch_encode(const kvq_encode_job* jobs, int njobs, cudaStream_t s
   if (path == 2 && !tc)
     return fail(KVQ_ERR_UNSUPPORTED, "encode: the tensor-core path supports head_dim 128 or 256 with group 32 or 16");
   if (tc && path != 1) return launch_encode_tc(jobs, njobs, s);
+  if (p->bits != 4) return fail(KVQ_ERR_UNSUPPORTED, "encode: the register-FFT path writes int4 codes only");
   return launch_encode_jobs(jobs, njobs, s);
 }
 
@@ -195,10 +196,18 @@ kvq_status kvq_plan_create(kvq_plan** out, int D, int G, const int8_t* signs, co
 
 int kvq_plan_transform(const kvq_plan* p) { return p ? p->xform : -1; }
 
+int kvq_plan_bits(const kvq_plan* p) { return p ? p->bits : -1; }
+
 kvq_status kvq_plan_create_transform(kvq_plan** out, int D, int G, const int8_t* signs, const float* lambda,
                                      int transform) {
+  return kvq_plan_create_ex(out, D, G, signs, lambda, transform, 4);
+}
+
+kvq_status kvq_plan_create_ex(kvq_plan** out, int D, int G, const int8_t* signs, const float* lambda, int transform,
+                              int bits) {
   if (!out || !signs || !lambda) return fail(KVQ_ERR_INVALID_ARG, "plan_create: null argument");
   *out = nullptr;
+  if (bits != 4 && bits != 8) return fail(KVQ_ERR_UNSUPPORTED, "plan_create: bits must be 4 or 8");
   if (transform != KVQ_TRANSFORM_SRFT && transform != KVQ_TRANSFORM_SRHT)
     return fail(KVQ_ERR_UNSUPPORTED, "plan_create: transform must be KVQ_TRANSFORM_SRFT or KVQ_TRANSFORM_SRHT");
   const bool hadamard = transform == KVQ_TRANSFORM_SRHT;
@@ -220,6 +229,7 @@ kvq_status kvq_plan_create_transform(kvq_plan** out, int D, int G, const int8_t*
   p->G = G;
   p->device = dev;
   p->xform = transform;
+  p->bits = bits;
   // per-channel factor of the rotation's unnormalised rows: the real DFT's dg_c, or
   // 1/sqrt(D) for every Hadamard row
   for (int c = 0; c < D; ++c) {
@@ -361,8 +371,8 @@ kvq_status kvq_encode_batch(const kvq_encode_job* jobs, int njobs, void* stream)
       kvq_status st = kvq::check_plan_device(p0);
       if (st != KVQ_OK) return st;
     } else if (j.plan->D != p0->D || j.plan->G != p0->G || j.plan->device != p0->device ||
-               j.plan->xform != p0->xform) {
-      return fail(KVQ_ERR_INVALID_ARG, w + "all jobs must share head_dim, group, transform and device");
+               j.plan->xform != p0->xform || j.plan->bits != p0->bits) {
+      return fail(KVQ_ERR_INVALID_ARG, w + "all jobs must share head_dim, group, transform, code width and device");
     }
     live.push_back(j);
   }
@@ -419,8 +429,9 @@ kvq_status kvq_attend_decode(const kvq_plan* pk, const kvq_plan* pv, const uint1
                              int T_cap, const int32_t* seq_lens, int T_len, float sigma, uint16_t* out,
                              void* ws, size_t ws_bytes, void* stream) {
   if (!pk || !pv) return fail(KVQ_ERR_INVALID_ARG, "attend: null plan");
-  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device || pk->xform != pv->xform)
-    return fail(KVQ_ERR_INVALID_ARG, "attend: K and V plans differ in head_dim, group, transform or device");
+  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device || pk->xform != pv->xform ||
+      pk->bits != pv->bits)
+    return fail(KVQ_ERR_INVALID_ARG, "attend: K and V plans differ in head_dim, group, transform, code width or device");
   if (pk->G != 32 && pk->G != 16) return fail(KVQ_ERR_UNSUPPORTED, "attend: group must be 32 or 16");
   kvq_status st = check_attend_common(B, Hq, Hkv, pk->D, T_cap, T_len, q, out, ws, ws_bytes);
   if (st != KVQ_OK || B == 0) return st;
@@ -438,8 +449,9 @@ kvq_status kvq_attend_decode_append(const kvq_plan* pk, const kvq_plan* pv, cons
                                     int Hq, int Hkv, int T_cap, int pos, float sigma, uint16_t* out, void* ws,
                                     size_t ws_bytes, void* stream) {
   if (!pk || !pv) return fail(KVQ_ERR_INVALID_ARG, "attend_append: null plan");
-  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device || pk->xform != pv->xform)
-    return fail(KVQ_ERR_INVALID_ARG, "attend_append: K and V plans differ in head_dim, group, transform or device");
+  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device || pk->xform != pv->xform ||
+      pk->bits != pv->bits)
+    return fail(KVQ_ERR_INVALID_ARG, "attend_append: K and V plans differ in head_dim, group, transform, code width or device");
   if (pk->G != 32 && pk->G != 16) return fail(KVQ_ERR_UNSUPPORTED, "attend_append: group must be 32 or 16");
   if (pos < 0) return fail(KVQ_ERR_INVALID_ARG, "attend_append: pos < 0");
   if (pos >= T_cap) return fail(KVQ_ERR_CAPACITY, "attend_append: pos + 1 > T_cap");
@@ -461,8 +473,9 @@ kvq_status kvq_attend_decode_partial(const kvq_plan* pk, const kvq_plan* pv, con
                                      int T_cap, int t_begin, int t_end, float sigma, float* partial, void* ws,
                                      size_t ws_bytes, void* stream) {
   if (!pk || !pv) return fail(KVQ_ERR_INVALID_ARG, "attend_partial: null plan");
-  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device || pk->xform != pv->xform)
-    return fail(KVQ_ERR_INVALID_ARG, "attend_partial: K and V plans differ in head_dim, group, transform or device");
+  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device || pk->xform != pv->xform ||
+      pk->bits != pv->bits)
+    return fail(KVQ_ERR_INVALID_ARG, "attend_partial: K and V plans differ in head_dim, group, transform, code width or device");
   if (pk->G != 32 && pk->G != 16) return fail(KVQ_ERR_UNSUPPORTED, "attend_partial: group must be 32 or 16");
   if (t_begin < 0 || t_end < t_begin) return fail(KVQ_ERR_INVALID_ARG, "attend_partial: need 0 <= t_begin <= t_end");
   if (t_end > T_cap) return fail(KVQ_ERR_CAPACITY, "attend_partial: t_end > T_cap");
@@ -505,8 +518,8 @@ kvq_status kvq_attend_decode_batch(const kvq_attend_job* jobs, int njobs, int B,
     if (!j.pk || !j.pv) return fail(KVQ_ERR_INVALID_ARG, tag + "null plan");
     if (j.pk->D != p0->D || j.pv->D != p0->D || j.pk->G != p0->G || j.pv->G != p0->G ||
         j.pk->device != p0->device || j.pv->device != p0->device || j.pk->xform != p0->xform ||
-        j.pv->xform != p0->xform)
-      return fail(KVQ_ERR_INVALID_ARG, tag + "plans differ in head_dim, group, transform or device");
+        j.pv->xform != p0->xform || j.pk->bits != p0->bits || j.pv->bits != p0->bits)
+      return fail(KVQ_ERR_INVALID_ARG, tag + "plans differ in head_dim, group, transform, code width or device");
     if (j.pk->G != 32 && j.pk->G != 16) return fail(KVQ_ERR_UNSUPPORTED, tag + "group must be 32 or 16");
     kvq_status st = check_attend_common(B, Hq, Hkv, p0->D, T_cap, T_len, j.q, j.out, ws, ws_bytes);
     if (st != KVQ_OK) return fail(st, tag + kvq_last_error());
@@ -532,8 +545,9 @@ kvq_status kvq_attend_decode_noalloc(const kvq_plan* pk, const kvq_plan* pv, con
                                      int Hkv, int T_cap, const int32_t* seq_lens, int T_len, float sigma,
                                      uint16_t* out, void* stream) {
   if (!pk || !pv) return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: null plan");
-  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device || pk->xform != pv->xform)
-    return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: K and V plans differ in head_dim, group, transform or device");
+  if (pk->D != pv->D || pk->G != pv->G || pk->device != pv->device || pk->xform != pv->xform ||
+      pk->bits != pv->bits)
+    return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: K and V plans differ in head_dim, group, transform, code width or device");
   if (pk->G != 32 && pk->G != 16) return fail(KVQ_ERR_UNSUPPORTED, "attend_noalloc: group must be 32 or 16");
   if (B < 0 || Hq <= 0 || Hkv <= 0 || T_cap < 0) return fail(KVQ_ERR_INVALID_ARG, "attend_noalloc: bad sizes");
   if (Hq % Hkv) return fail(KVQ_ERR_UNSUPPORTED, "attend_noalloc: Hq must be a multiple of Hkv");

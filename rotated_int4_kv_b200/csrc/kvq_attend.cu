@@ -59,26 +59,29 @@ constexpr int kMaxClusterThroughput = 4;
 constexpr int kMaxMerge = kMaxSplitsCfg / 4;  // cluster partials per unit merged through the workspace
 constexpr int kMaxJobs = 32;                // problems per launch of a batch (job table in parameter space)
 
-template <int D, bool INT4, int G = 32>
+template <int D, bool INT4, int G = 32, int BITS = 4>
 struct Cfg {
   static_assert(G == 32 || G == 16, "group size");
-  static constexpr int NC = D / 32;                        // 32-channel chunks of a code row (16 bytes each)
-  static constexpr int NG = INT4 ? D / G : NC;             // scale groups per token (int4)
-  static constexpr int kRowBytes = INT4 ? D / 2 : 2 * D;   // bytes per token row of K (and V)
+  static_assert(BITS == 4 || BITS == 8, "code width");
+  static constexpr int NC = D / 32;                        // 32-channel chunks of a code row (16 or 32 bytes)
+  static constexpr int NG = INT4 ? D / G : NC;             // scale groups per token (quantised caches)
+  static constexpr int kRowBytes = INT4 ? D * BITS / 8 : 2 * D;  // bytes per token row of K (and V)
   // consumer warps (plus one producer warp); resident CTAs per SM for the launch bounds
   static constexpr int kCWarps = 4;
   static constexpr int kThreads = (kCWarps + 1) * 32;
   static constexpr int kMinBlocks = D == 128 ? 2 : 1;
   // each consumer warp takes kSub subtiles of 16 tokens per stage (two independent
-  // instruction streams for the int4 path, whose per-token work is latency-bound)
-  static constexpr int kSub = INT4 ? 2 : 1;
+  // instruction streams for the int4 path, whose per-token work is latency-bound; one
+  // for int8, whose rows are twice as long)
+  static constexpr int kSub = (INT4 && BITS == 4) ? 2 : 1;
   static constexpr int kTile = 16 * kCWarps * kSub;        // tokens per stage
   static constexpr int kKBytes = kTile * kRowBytes;
   static constexpr int kSBytes = INT4 ? kTile * NG * 2 : 0;
   static constexpr int kStageBytes = 2 * kKBytes + 2 * kSBytes;
   static constexpr int kStages = INT4 ? 2 : (D == 128 ? 3 : 2);
   // latency of one stage when the kernel is latency-bound (ns, measured; split planning)
-  static constexpr long kStageNs = INT4 ? (D == 128 ? 750 : 1350) : (D == 128 ? 200 : 570);
+  static constexpr long kStageNs =
+      INT4 ? (BITS == 4 ? (D == 128 ? 750 : 1350) : (D == 128 ? 450 : 800)) : (D == 128 ? 200 : 570);
   static constexpr int kScaleBox = (kTile * NG) < 256 ? kTile * NG : 256;  // halves per scale TMA box
   static constexpr int kScaleLoads = INT4 ? (kTile * NG) / kScaleBox : 0;
   static constexpr int kRing = kStages * kStageBytes;
@@ -110,6 +113,8 @@ struct Cfg {
   static constexpr int kRot = kMmaRot ? 4 * 128 * 128 : 0;
   static constexpr int kSmem = kRotOff + kRot + 1024;
   static_assert(2 * kStages * 8 + 3 * 8 + 4 <= kBars, "barrier region");
+  // 128-byte-swizzled code boxes start on 1024-byte boundaries
+  static_assert(kKBytes % 1024 == 0 && kStageBytes % 1024 == 0, "stage layout");
   // the merge weights of up to kMaxMerge partials reuse the (dead) B fragments
   static_assert(kQf >= 2 * kMaxMerge * kHT * 4, "merge scratch");
   static_assert(kHT * D <= kCWarps * (2 * kHT + kHT * D), "output scratch");
@@ -186,6 +191,23 @@ __device__ __forceinline__ void nib8_to_h2(uint32_t w, uint32_t (&h)[4]) {
   h[1] = h2_bits(__hfma2(bits_h2(b), k16, k72));
   h[2] = h2_bits(__hsub2(bits_h2(c), k1032));
   h[3] = h2_bits(__hfma2(bits_h2(d), k16, k72));
+}
+
+// Two fp16x2 pairs of exact integer codes from one word of four int8 codes (two's
+// complement): (b0, b2) and (b1, b3). Each permute forms 0x6400 | (byte ^ 0x80) per
+// half, the fp16 value 1024 + 128 + code; one fp16 subtraction removes the offset.
+__device__ __forceinline__ void byte4_to_h2(uint32_t w, uint32_t (&h)[2]) {
+  const __half2 k1152 = __floats2half2_rn(1152.0f, 1152.0f);
+  const uint32_t x = w ^ 0x80808080u;
+  h[0] = h2_bits(__hsub2(bits_h2(prmt(x, 0x64646464u, 0x4240u)), k1152));
+  h[1] = h2_bits(__hsub2(bits_h2(prmt(x, 0x64646464u, 0x4341u)), k1152));
+}
+
+// Shared-memory offset of 16-byte column cc of token row `row` in a stage of int8 code
+// rows: 128-byte boxes (one per 128 channels) of kTile rows, 128-byte swizzle.
+template <int kTile>
+__device__ __forceinline__ int code8_off(int row, int cc) {
+  return (cc >> 3) * kTile * 128 + row * 128 + (((cc & 7) ^ (row & 7)) << 4);
 }
 
 template <int NW>
@@ -592,10 +614,10 @@ __device__ __forceinline__ void unrotate_out_eo(const float* om, int heads, cons
   }
 }
 
-template <int D, bool INT4, int MAXJ, int G = 32>
-__global__ void __launch_bounds__((Cfg<D, INT4, G>::kThreads), (Cfg<D, INT4, G>::kMinBlocks))
+template <int D, bool INT4, int MAXJ, int G = 32, int BITS = 4>
+__global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT4, G, BITS>::kMinBlocks))
     attend_kernel(const __grid_constant__ AttnJobs<MAXJ> jt, const __grid_constant__ AttnParams p) {
-  using C = Cfg<D, INT4, G>;
+  using C = Cfg<D, INT4, G, BITS>;
   constexpr int kCWarps = C::kCWarps;
   constexpr int kThreads = C::kThreads;
   static_assert(D == 256 || kCWarps == 4, "the D = 128 rotation helpers take four consumer warps");
@@ -721,8 +743,17 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G>::kThreads), (Cfg<D, INT4, G>:
         mbar_arrive_expect_tx(&full[s], C::kStageBytes);
         const uint64_t pol = l2_evict_first_policy();
         if constexpr (INT4) {
-          tma_load_2d_hint(st, &J.kmap, &full[s], 0, row0 + p.t_base + t0, pol);
-          tma_load_2d_hint(st + C::kKBytes, &J.vmap, &full[s], 0, row0 + p.t_base + t0, pol);
+          if constexpr (BITS == 4) {
+            tma_load_2d_hint(st, &J.kmap, &full[s], 0, row0 + p.t_base + t0, pol);
+            tma_load_2d_hint(st + C::kKBytes, &J.vmap, &full[s], 0, row0 + p.t_base + t0, pol);
+          } else {
+#pragma unroll
+            for (int j = 0; j < D / 128; ++j) {
+              tma_load_2d_hint(st + j * C::kTile * 128, &J.kmap, &full[s], 128 * j, row0 + p.t_base + t0, pol);
+              tma_load_2d_hint(st + C::kKBytes + j * C::kTile * 128, &J.vmap, &full[s], 128 * j,
+                               row0 + p.t_base + t0, pol);
+            }
+          }
 #pragma unroll
           for (int j = 0; j < C::kScaleLoads; ++j) {
             tma_load_2d(st + 2 * C::kKBytes + j * C::kScaleBox * 2, &J.ksmap, &full[s],
@@ -792,12 +823,16 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G>::kThreads), (Cfg<D, INT4, G>:
           float y[G];
 #pragma unroll
           for (int i = 0; i < G; ++i) y[i] = yg[i];
-          uint32_t wd[G / 8], sb;
-          quantize_group<G>(y, wd, sb);
+          constexpr int kGW = G * BITS / 32;  // code words of one group
+          uint32_t wd[kGW], sb;
+          quantize_group<G, BITS>(y, wd, sb);
           if (ht == 0) {
             const size_t crow = (size_t)bk * p.T_cap + p.append_pos;
-            uint8_t* cdst = (r ? p.vc_out : p.kc_out) + crow * (D / 2) + (G / 2) * grp;
-            if constexpr (G == 32) {
+            uint8_t* cdst = (r ? p.vc_out : p.kc_out) + crow * (D * BITS / 8) + (G * BITS / 8) * grp;
+            if constexpr (kGW == 8) {
+              reinterpret_cast<uint4*>(cdst)[0] = make_uint4(wd[0], wd[1], wd[2], wd[3]);
+              reinterpret_cast<uint4*>(cdst)[1] = make_uint4(wd[4], wd[5], wd[6], wd[7]);
+            } else if constexpr (kGW == 4) {
               *reinterpret_cast<uint4*>(cdst) = make_uint4(wd[0], wd[1], wd[2], wd[3]);
             } else {
               *reinterpret_cast<uint2*>(cdst) = make_uint2(wd[0], wd[1]);
@@ -805,12 +840,19 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G>::kThreads), (Cfg<D, INT4, G>:
             (r ? p.vs_out : p.ks_out)[crow * NG + grp] = (uint16_t)sb;
           }
           const float sc = __half2float(__ushort_as_half((unsigned short)sb));
+          constexpr int kPer = 32 / BITS;  // codes per word
 #pragma unroll
-          for (int w = 0; w < G / 8; ++w) {
+          for (int w = 0; w < kGW; ++w) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int nib = (int)((wd[w] >> (4 * e)) & 15u);
-              yg[8 * w + e] = (float)(nib >= 8 ? nib - 16 : nib) * sc;
+            for (int e = 0; e < kPer; ++e) {
+              int code;
+              if constexpr (BITS == 4) {
+                const int nib = (int)((wd[w] >> (4 * e)) & 15u);
+                code = nib >= 8 ? nib - 16 : nib;
+              } else {
+                code = (int)(int8_t)((wd[w] >> (8 * e)) & 255u);
+              }
+              yg[kPer * w + e] = (float)code * sc;
             }
           }
         }
@@ -832,7 +874,14 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G>::kThreads), (Cfg<D, INT4, G>:
       const float* qh = qt + g * D;
       for (int ks = warp; ks < kKSteps; ks += kCWarps) {
         int ch[4];
-        if constexpr (INT4) {
+        if constexpr (INT4 && BITS == 8) {
+          // channels 16 ks .. 16 ks + 15: slots (2c, 2c+1) <- (4c, 4c+2), (2c+8, 2c+9) <- (4c+1, 4c+3)
+          const int base = 16 * ks + 4 * c;
+          ch[0] = base;
+          ch[1] = base + 2;
+          ch[2] = base + 1;
+          ch[3] = base + 3;
+        } else if constexpr (INT4) {
           // group G = ks/2; step A: (8c, 8c+4 | 8c+1, 8c+5); step B: (8c+2, 8c+6 | 8c+3, 8c+7)
           const int base = (ks >> 1) * 32 + 8 * c + ((ks & 1) ? 2 : 0);
           ch[0] = base;
@@ -901,6 +950,34 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G>::kThreads), (Cfg<D, INT4, G>:
               skB[2 * q2 + 1] = fb.y;
             }
           }
+          if constexpr (BITS == 8) {
+            // one 32-channel chunk (two 16-byte columns) per ldmatrix.x4; each k step of
+            // 16 channels is one product with the hi and one with the lo query half
+#pragma unroll
+            for (int ch = 0; ch < NC; ++ch) {
+              const int mi = lane >> 3;
+              const int row = r0s + ((mi & 1) << 3) + (lane & 7);
+              uint32_t w0, w1, w2, w3;  // (tok g, ch 0-15) (tok g+8, ch 0-15) (tok g, ch 16-31) (tok g+8, ch 16-31)
+              ldmatrix_x4(w0, w1, w2, w3, smem_u32(kt + code8_off<C::kTile>(row, 2 * ch + (mi >> 1))));
+              uint32_t e0[2], e1[2], e2[2], e3[2];
+              byte4_to_h2(w0, e0);
+              byte4_to_h2(w1, e1);
+              byte4_to_h2(w2, e2);
+              byte4_to_h2(w3, e3);
+              const uint4 f0 = qf[(2 * ch) * 32 + lane], f1 = qf[(2 * ch + 1) * 32 + lane];
+              float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
+              mma_16816(a0, e0[0], e1[0], e0[1], e1[1], f0.x, f0.y);
+              mma_16816(a0, e0[0], e1[0], e0[1], e1[1], f0.z, f0.w);
+              mma_16816(a1, e2[0], e3[0], e2[1], e3[1], f1.x, f1.y);
+              mma_16816(a1, e2[0], e3[0], e2[1], e3[1], f1.z, f1.w);
+              // scale groups of the two 16-channel halves: the chunk's one group (G = 32) or two
+              const int q0 = G == 32 ? ch : 2 * ch, q1 = G == 32 ? ch : 2 * ch + 1;
+              scs[0] = fmaf(skA[q0], a0[0], fmaf(skA[q1], a1[0], scs[0]));
+              scs[1] = fmaf(skA[q0], a0[1], fmaf(skA[q1], a1[1], scs[1]));
+              scs[2] = fmaf(skB[q0], a0[2], fmaf(skB[q1], a1[2], scs[2]));
+              scs[3] = fmaf(skB[q0], a0[3], fmaf(skB[q1], a1[3], scs[3]));
+            }
+          } else {
   #pragma unroll
           for (int gp = 0; gp < NC / 2; ++gp) {  // two 32-channel chunks per ldmatrix.x4
             const int mi = lane >> 3;
@@ -954,6 +1031,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G>::kThreads), (Cfg<D, INT4, G>:
             scs[1] = fmaf(skA[G0], a0[1], fmaf(skA[G1], a1[1], scs[1]));
             scs[2] = fmaf(skB[G0], a0[2], fmaf(skB[G1], a1[2], scs[2]));
             scs[3] = fmaf(skB[G0], a0[3], fmaf(skB[G1], a1[3], scs[3]));
+          }
           }
         } else {
           const uint8_t* kt = st;
@@ -1054,6 +1132,31 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G>::kThreads), (Cfg<D, INT4, G>:
               for (int q2 = 0; q2 < NG / 2; ++q2) sw[e][q2] = valid ? sp[q2] : 0u;
             }
           }
+          if constexpr (BITS == 8) {
+            // transposed 8x8 blocks of 2-byte units: lane (g, c) holds tokens 2c, 2c+1 of
+            // channels 2g, 2g+1 per word; M rows g / g+8 of m-tile 2 ch + h are the channels
+            // 32 ch + 16 h + 2g / + 1
+#pragma unroll
+            for (int ch = 0; ch < NC; ++ch) {
+              const int mi = lane >> 3;
+              const int row = r0s + ((mi & 1) << 3) + (lane & 7);
+              uint32_t w0, w1, w2, w3;  // (tok 0-7, ch 0-15) (tok 8-15, ch 0-15) (tok 0-7, ch 16-31) (tok 8-15, ch 16-31)
+              ldmatrix_x4_trans(w0, w1, w2, w3, smem_u32(vt + code8_off<C::kTile>(row, 2 * ch + (mi >> 1))));
+#pragma unroll
+              for (int h = 0; h < 2; ++h) {
+                const int grp = G == 32 ? ch : 2 * ch + h;
+                uint32_t lo[2], hi[2];
+                byte4_to_h2(h ? w2 : w0, lo);  // tokens 2c, 2c+1
+                byte4_to_h2(h ? w3 : w1, hi);  // tokens 2c+8, 2c+9
+                const uint32_t sel = (grp & 1) ? 0x7632u : 0x5410u;
+                const uint32_t s01 = prmt(sw[0][grp >> 1], sw[1][grp >> 1], sel);
+                const uint32_t s89 = prmt(sw[2][grp >> 1], sw[3][grp >> 1], sel);
+                const uint32_t b0 = h2_bits(__hmul2(bits_h2(pb0[sb]), bits_h2(s01)));
+                const uint32_t b1 = h2_bits(__hmul2(bits_h2(pb1[sb]), bits_h2(s89)));
+                mma_16816(o_acc[2 * ch + h], lo[0], lo[1], hi[0], hi[1], b0, b1);
+              }
+            }
+          } else {
   #pragma unroll
           for (int gp = 0; gp < NC / 2; ++gp) {
             const int mi = lane >> 3;
@@ -1094,6 +1197,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G>::kThreads), (Cfg<D, INT4, G>:
               mma_16816(o_acc[2 * CH], lo[0], lo[1], hi[0], hi[1], b0, b1);
               mma_16816(o_acc[2 * CH + 1], lo[2], lo[3], hi[2], hi[3], b0, b1);
             }
+          }
           }
         } else {
           const uint8_t* vt = st + C::kKBytes;
@@ -1139,7 +1243,8 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G>::kThreads), (Cfg<D, INT4, G>:
         }
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-          const int ch0 = (mt >> 1) * 32 + 4 * g + ((mt & 1) ? 2 : 0), ch1 = ch0 + 1;
+          const int ch0 = BITS == 8 ? 16 * mt + 2 * g : (mt >> 1) * 32 + 4 * g + ((mt & 1) ? 2 : 0);
+          const int ch1 = ch0 + 1;
           o_acc[mt][0] = fmaf(o_acc[mt][0], al[0], pn[0] * vhat[ch0]);
           o_acc[mt][1] = fmaf(o_acc[mt][1], al[1], pn[1] * vhat[ch0]);
           o_acc[mt][2] = fmaf(o_acc[mt][2], al[0], pn[0] * vhat[ch1]);
@@ -1180,7 +1285,10 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G>::kThreads), (Cfg<D, INT4, G>:
 #pragma unroll
     for (int mt = 0; mt < MT; ++mt) {
       int ch0, ch1;  // channels held in rows g and g+8 of m-tile mt
-      if constexpr (INT4) {
+      if constexpr (INT4 && BITS == 8) {
+        ch0 = 16 * mt + 2 * g;
+        ch1 = ch0 + 1;
+      } else if constexpr (INT4) {
         ch0 = (mt >> 1) * 32 + 4 * g + ((mt & 1) ? 2 : 0);
         ch1 = ch0 + 1;
       } else {
@@ -1509,13 +1617,13 @@ struct Occupancy {
   int cap[kMaxCluster + 1];
 };
 
-template <int D, bool INT4, int MAXJ, int G = 32>
+template <int D, bool INT4, int MAXJ, int G = 32, int BITS = 4>
 const Occupancy& occupancy() {
-  using C = Cfg<D, INT4, G>;
+  using C = Cfg<D, INT4, G, BITS>;
   static Occupancy occ{};
   static std::once_flag once;
   std::call_once(once, [] {
-    auto kern = attend_kernel<D, INT4, MAXJ, G>;
+    auto kern = attend_kernel<D, INT4, MAXJ, G, BITS>;
     cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
     cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     int nb = 0;
@@ -1656,16 +1764,19 @@ size_t ws_bytes_for(int B, int Hq, int Hkv, int D, int ncl, int HT) {
 
 // Tensor maps and pointers of one problem. Rows of the code (or fp16) maps are
 // (b, kv head, token) rows; scale maps have one row of T_cap * D/32 halves per (b, kv head).
-template <int D, bool INT4, int G = 32>
+template <int D, bool INT4, int G = 32, int BITS = 4>
 kvq_status make_job(const AttendJobHost& h, int B, int Hkv, int T_cap, AttnJob* j) {
-  using C = Cfg<D, INT4, G>;
+  using C = Cfg<D, INT4, G, BITS>;
   const uint64_t rows = (uint64_t)B * Hkv * T_cap;
   kvq_status st;
   if (INT4) {
-    const uint64_t dims[2] = {(uint64_t)D / 2, rows};
-    const uint64_t strides[1] = {(uint64_t)D / 2};
-    const uint32_t box[2] = {(uint32_t)D / 2, (uint32_t)C::kTile};
-    const CUtensorMapSwizzle sw = D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+    // code rows of RB bytes: int4 one box per row (64-byte swizzle for 64-byte rows),
+    // int8 boxes of 128 bytes (one per 128 channels)
+    constexpr int RB = D * BITS / 8;
+    const uint64_t dims[2] = {(uint64_t)RB, rows};
+    const uint64_t strides[1] = {(uint64_t)RB};
+    const uint32_t box[2] = {(uint32_t)(RB < 128 ? RB : 128), (uint32_t)C::kTile};
+    const CUtensorMapSwizzle sw = RB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
     st = encode_tiled(&j->kmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, h.kc, dims, strides, box, sw, "K codes");
     if (st == KVQ_OK) st = encode_tiled(&j->vmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, h.vc, dims, strides, box, sw, "V codes");
     if (st != KVQ_OK) return st;
@@ -1727,20 +1838,20 @@ struct RangeHost {
 // One launch over nj <= MAXJ problems of equal shape (with app: the fused append, T_len =
 // the tokens already cached = app->pos; with range: tokens [t_base, t_base + T_len) and
 // softmax partials instead of outputs).
-template <int D, bool INT4, int MAXJ, int G = 32>
+template <int D, bool INT4, int MAXJ, int G = 32, int BITS = 4>
 kvq_status launch_chunk(const AttendJobHost* jobs, int nj, int B, int Hq, int Hkv, int T_cap, const int32_t* seq_lens,
                         int T_len, float sigma, void* ws, size_t ws_bytes, cudaStream_t strm,
                         const AppendHost* app = nullptr, const RangeHost* range = nullptr) {
-  using C = Cfg<D, INT4, G>;
+  using C = Cfg<D, INT4, G, BITS>;
   const int T_split = seq_lens ? T_cap : T_len;
   const int Bj = nj * B;  // the jobs of a launch split like a larger batch
-  SplitPlan sp = choose_split(Bj, Hq, Hkv, T_split, occupancy<D, INT4, MAXJ, G>(), C::kTile, C::kStageNs);
+  SplitPlan sp = choose_split(Bj, Hq, Hkv, T_split, occupancy<D, INT4, MAXJ, G, BITS>(), C::kTile, C::kStageNs);
   const size_t units = (size_t)Bj * Hkv * sp.HT;
   const size_t need = ws_bytes_for(Bj, Hq, Hkv, D, sp.S / sp.C, sp.HT);
   if (ws_bytes < need) return fail(KVQ_ERR_WORKSPACE, "attend: workspace too small for this split");
   AttnJobs<MAXJ> jt;
   for (int i = 0; i < nj; ++i) {
-    const kvq_status st = make_job<D, INT4, G>(jobs[i], B, Hkv, T_cap, &jt.j[i]);
+    const kvq_status st = make_job<D, INT4, G, BITS>(jobs[i], B, Hkv, T_cap, &jt.j[i]);
     if (st != KVQ_OK) return st;
   }
   AttnParams prm{};
@@ -1794,23 +1905,23 @@ kvq_status launch_chunk(const AttendJobHost* jobs, int nj, int B, int Hq, int Hk
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, attend_kernel<D, INT4, MAXJ, G>, jt, prm);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, attend_kernel<D, INT4, MAXJ, G, BITS>, jt, prm);
   if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("attend launch: ") + cudaGetErrorString(e));
   return KVQ_OK;
 }
 
 // Launches of up to kMaxJobs problems each, in stream order; they reuse the
 // workspace from its start (every launch leaves its counters at zero).
-template <int D, bool INT4, int G = 32>
+template <int D, bool INT4, int G = 32, int BITS = 4>
 kvq_status run_attend(const AttendJobHost* jobs, int njobs, int B, int Hq, int Hkv, int T_cap,
                       const int32_t* seq_lens, int T_len, float sigma, void* ws, size_t ws_bytes, cudaStream_t strm) {
   if (njobs == 1)
-    return launch_chunk<D, INT4, 1, G>(jobs, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, strm);
+    return launch_chunk<D, INT4, 1, G, BITS>(jobs, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, strm);
   for (int j0 = 0; j0 < njobs; j0 += kMaxJobs) {
     const int nj = std::min(kMaxJobs, njobs - j0);
     const kvq_status st =
-        launch_chunk<D, INT4, kMaxJobs, G>(jobs + j0, nj, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes,
-                                           strm);
+        launch_chunk<D, INT4, kMaxJobs, G, BITS>(jobs + j0, nj, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws,
+                                                 ws_bytes, strm);
     if (st != KVQ_OK) return st;
   }
   return KVQ_OK;
@@ -1840,14 +1951,11 @@ kvq_status launch_attend_int4(const kvq_plan* pk, const kvq_plan* pv, const uint
 kvq_status launch_attend_int4_batch(const AttendJobHost* jobs, int njobs, int B, int Hq, int Hkv, int T_cap,
                                     const int32_t* seq_lens, int T_len, float sigma, void* ws, size_t ws_bytes,
                                     cudaStream_t s) {
-  const int D = jobs[0].pk->D, G = jobs[0].pk->G;
-  if (D == 128 && G == 32)
-    return run_attend<128, true, 32>(jobs, njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
-  if (D == 256 && G == 32)
-    return run_attend<256, true, 32>(jobs, njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
-  if (D == 128)
-    return run_attend<128, true, 16>(jobs, njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
-  return run_attend<256, true, 16>(jobs, njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
+  const kvq_plan* pk = jobs[0].pk;
+  return dispatch_dgb(pk->D, pk->G, pk->bits, [&](auto d, auto g, auto b) {
+    return run_attend<decltype(d)::value, true, decltype(g)::value, decltype(b)::value>(
+        jobs, njobs, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, ws, ws_bytes, s);
+  });
 }
 
 kvq_status launch_attend_int4_append(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q, const uint16_t* k_new,
@@ -1856,13 +1964,10 @@ kvq_status launch_attend_int4_append(const kvq_plan* pk, const kvq_plan* pv, con
                                      size_t ws_bytes, cudaStream_t s) {
   const AttendJobHost job{pk, pv, q, kc, ks, vc, vs, out};
   const AppendHost app{k_new, v_new, kc, ks, vc, vs, pos};
-  if (pk->D == 128 && pk->G == 32)
-    return launch_chunk<128, true, 1, 32>(&job, 1, B, Hq, Hkv, T_cap, nullptr, pos, sigma, ws, ws_bytes, s, &app);
-  if (pk->D == 256 && pk->G == 32)
-    return launch_chunk<256, true, 1, 32>(&job, 1, B, Hq, Hkv, T_cap, nullptr, pos, sigma, ws, ws_bytes, s, &app);
-  if (pk->D == 128)
-    return launch_chunk<128, true, 1, 16>(&job, 1, B, Hq, Hkv, T_cap, nullptr, pos, sigma, ws, ws_bytes, s, &app);
-  return launch_chunk<256, true, 1, 16>(&job, 1, B, Hq, Hkv, T_cap, nullptr, pos, sigma, ws, ws_bytes, s, &app);
+  return dispatch_dgb(pk->D, pk->G, pk->bits, [&](auto d, auto g, auto b) {
+    return launch_chunk<decltype(d)::value, true, 1, decltype(g)::value, decltype(b)::value>(
+        &job, 1, B, Hq, Hkv, T_cap, nullptr, pos, sigma, ws, ws_bytes, s, &app);
+  });
 }
 
 kvq_status launch_attend_int4_partial(const kvq_plan* pk, const kvq_plan* pv, const uint16_t* q, const uint8_t* kc,
@@ -1872,13 +1977,10 @@ kvq_status launch_attend_int4_partial(const kvq_plan* pk, const kvq_plan* pv, co
   const AttendJobHost job{pk, pv, q, kc, ks, vc, vs, nullptr};
   const RangeHost rg{t_begin, part};
   const int T = t_end - t_begin;
-  if (pk->D == 128 && pk->G == 32)
-    return launch_chunk<128, true, 1, 32>(&job, 1, B, Hq, Hkv, T_cap, nullptr, T, sigma, ws, ws_bytes, s, nullptr, &rg);
-  if (pk->D == 256 && pk->G == 32)
-    return launch_chunk<256, true, 1, 32>(&job, 1, B, Hq, Hkv, T_cap, nullptr, T, sigma, ws, ws_bytes, s, nullptr, &rg);
-  if (pk->D == 128)
-    return launch_chunk<128, true, 1, 16>(&job, 1, B, Hq, Hkv, T_cap, nullptr, T, sigma, ws, ws_bytes, s, nullptr, &rg);
-  return launch_chunk<256, true, 1, 16>(&job, 1, B, Hq, Hkv, T_cap, nullptr, T, sigma, ws, ws_bytes, s, nullptr, &rg);
+  return dispatch_dgb(pk->D, pk->G, pk->bits, [&](auto d, auto g, auto b) {
+    return launch_chunk<decltype(d)::value, true, 1, decltype(g)::value, decltype(b)::value>(
+        &job, 1, B, Hq, Hkv, T_cap, nullptr, T, sigma, ws, ws_bytes, s, nullptr, &rg);
+  });
 }
 
 namespace {
@@ -1958,11 +2060,12 @@ kvq_status launch_attend_int4_noalloc(const kvq_plan* pk, const kvq_plan* pv, co
   if (cudaGetDevice(&dev) != cudaSuccess) return fail(KVQ_ERR_DEVICE, "attend_noalloc: no current device");
   const int D = pk->D;
   // the exact split the launch will choose, hence the exact scratch it needs
-  const int G = pk->G;
-  const Occupancy& occ = D == 128 ? (G == 32 ? occupancy<128, true, 1, 32>() : occupancy<128, true, 1, 16>())
-                                  : (G == 32 ? occupancy<256, true, 1, 32>() : occupancy<256, true, 1, 16>());
-  const SplitPlan sp = choose_split(B, Hq, Hkv, seq_lens ? T_cap : T_len, occ, Cfg<128, true>::kTile,
-                                    D == 128 ? Cfg<128, true>::kStageNs : Cfg<256, true>::kStageNs);
+  const SplitPlan sp = dispatch_dgb(D, pk->G, pk->bits, [&](auto d, auto g, auto b) {
+    constexpr int kD = decltype(d)::value, kG = decltype(g)::value, kB = decltype(b)::value;
+    using C = Cfg<kD, true, kG, kB>;
+    return choose_split(B, Hq, Hkv, seq_lens ? T_cap : T_len, occupancy<kD, true, 1, kG, kB>(), C::kTile,
+                        C::kStageNs);
+  });
   const size_t need = ws_bytes_for(B, Hq, Hkv, D, sp.S / sp.C, sp.HT);
   if (need > kNoAllocScratchBytes)
     return fail(KVQ_ERR_WORKSPACE, "attend_noalloc: these shapes need " + std::to_string(need) +
@@ -1976,17 +2079,8 @@ kvq_status launch_attend_int4_noalloc(const kvq_plan* pk, const kvq_plan* pv, co
   const cudaError_t e = cudaMemsetAsync(scratch, 0, ws_cnt_bytes(units), s);
   if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("attend_noalloc: memset: ") + cudaGetErrorString(e));
   const AttendJobHost job{pk, pv, q, kc, ks, vc, vs, out};
-  if (D == 128 && G == 32)
-    return run_attend<128, true, 32>(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, scratch, kNoAllocScratchBytes,
-                                     s);
-  if (D == 256 && G == 32)
-    return run_attend<256, true, 32>(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, scratch, kNoAllocScratchBytes,
-                                     s);
-  if (D == 128)
-    return run_attend<128, true, 16>(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, scratch, kNoAllocScratchBytes,
-                                     s);
-  return run_attend<256, true, 16>(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, scratch, kNoAllocScratchBytes,
-                                   s);
+  return launch_attend_int4_batch(&job, 1, B, Hq, Hkv, T_cap, seq_lens, T_len, sigma, scratch, kNoAllocScratchBytes,
+                                  s);
 }
 
 uint32_t attend_error_flags(bool clear) {

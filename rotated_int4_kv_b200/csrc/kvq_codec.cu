@@ -399,20 +399,20 @@ __global__ void __launch_bounds__(kNT, 3) encode_kernel(const __grid_constant__ 
 }
 
 // ---------------------------------------------------------------- decode
-template <int D>
+template <int D, int BITS>
 struct DecSmem {
-  static constexpr int kCStage = kNT * D / 2;  // packed code tile
+  static constexpr int kCStage = kNT * D * BITS / 8;  // code tile (int8: D / 128 boxes of 128-byte rows)
   static constexpr int kXTile = kNT * D * 2;   // fp16 output tile
   static constexpr int kStages = D == 128 ? 2 : 1;
   static constexpr int kBytes = kStages * kCStage + kXTile + 64 + 1024;
 };
 
-template <int D, int G, int XF>
+template <int D, int G, int XF, int BITS>
 __global__ void __launch_bounds__(kNT, kMinBlocks<D>) decode_kernel(const __grid_constant__ CUtensorMap cmap,
                                                      const __grid_constant__ CUtensorMap omap,
                                                      const __grid_constant__ CodecConsts cc, TileGeom geom,
                                                      const uint16_t* __restrict__ scales, int T_cap, int t0_cache) {
-  using L = DecSmem<D>;
+  using L = DecSmem<D, BITS>;
   constexpr int kBoxes = D / 64;
   constexpr int kBoxBytes = kNT * 128;
   constexpr int kNG = D / G;
@@ -437,7 +437,13 @@ __global__ void __launch_bounds__(kNT, kMinBlocks<D>) decode_kernel(const __grid
     int bh0, t0;
     tile_origin(geom, tile, bh0, t0);
     mbar_arrive_expect_tx(&bar[stage], L::kCStage);
-    tma_load_3d(cs + stage * L::kCStage, &cmap, &bar[stage], 0, t0_cache + t0, bh0);
+    if constexpr (BITS == 4) {
+      tma_load_3d(cs + stage * L::kCStage, &cmap, &bar[stage], 0, t0_cache + t0, bh0);
+    } else {
+#pragma unroll
+      for (int bx = 0; bx < D / 128; ++bx)
+        tma_load_3d(cs + stage * L::kCStage + bx * kNT * 128, &cmap, &bar[stage], 128 * bx, t0_cache + t0, bh0);
+    }
   };
   if (tid == 0) {
     for (int s = 0; s < L::kStages; ++s) {
@@ -490,13 +496,23 @@ __global__ void __launch_bounds__(kNT, kMinBlocks<D>) decode_kernel(const __grid
       atomicOr(&g_codec_err, kErrTimeoutLoad);
       return;
     }
-    uint32_t words[D / 8];
-    {
+    uint32_t words[D * BITS / 32];
+    if constexpr (BITS == 4) {
       const uint8_t* row = cs + stage * L::kCStage + tid * (D / 2);
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         const int pc = (D == 128) ? (c ^ ((tid >> 1) & 3)) : (c ^ (tid & 7));
         const uint4 w = *reinterpret_cast<const uint4*>(row + pc * 16);
+        words[4 * c] = w.x;
+        words[4 * c + 1] = w.y;
+        words[4 * c + 2] = w.z;
+        words[4 * c + 3] = w.w;
+      }
+    } else {
+#pragma unroll
+      for (int c = 0; c < D / 16; ++c) {  // 16-byte chunk c of the row: box c / 8, swizzled column
+        const uint8_t* row = cs + stage * L::kCStage + (c >> 3) * kNT * 128 + tid * 128;
+        const uint4 w = *reinterpret_cast<const uint4*>(row + (((c & 7) ^ (tid & 7)) << 4));
         words[4 * c] = w.x;
         words[4 * c + 1] = w.y;
         words[4 * c + 2] = w.z;
@@ -508,15 +524,18 @@ __global__ void __launch_bounds__(kNT, kMinBlocks<D>) decode_kernel(const __grid
       const int nxt = tile + L::kStages * stride;
       if (nxt < geom.n_tiles) issue(nxt, stage);
     }
-    // unpack: code c = (nibble ^ 8) - 8 exactly, via the fp32 magic constant
+    // unpack: code c = (nibble ^ 8) - 8 (int8: (byte ^ 128) - 128) exactly, via the fp32
+    // magic constant
     float v[D];
+    constexpr int kPer = 32 / BITS;  // codes per word
 #pragma unroll
-    for (int w = 0; w < D / 8; ++w) {
-      const uint32_t u = words[w] ^ 0x88888888u;
+    for (int w = 0; w < D / kPer; ++w) {
+      const uint32_t u = words[w] ^ (BITS == 4 ? 0x88888888u : 0x80808080u);
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int c = 8 * w + j;
-        const float code = __uint_as_float(((u >> (4 * j)) & 0xFu) | 0x4B400000u) - 12582920.0f;
+      for (int j = 0; j < kPer; ++j) {
+        const int c = kPer * w + j;
+        const float code = __uint_as_float(((u >> (BITS * j)) & ((1u << BITS) - 1u)) | 0x4B400000u) -
+                           (BITS == 4 ? 12582920.0f : 12583040.0f);
         v[XF == 1 ? c : slot_of_channel(c, D)] = code * (sc[c / G] * cc.chan[c]);
       }
     }
@@ -652,18 +671,19 @@ kvq_status run_encode(const kvq_encode_job* jobs, int njobs, cudaStream_t s) {
   return KVQ_OK;
 }
 
-template <int D, int G, int XF>
+template <int D, int G, int XF, int BITS>
 kvq_status run_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* scales, int B, int H, int T_cap,
                       int t0, int n, uint16_t* out, cudaStream_t s) {
   const int BH = B * H;
   TileGeom geom = make_geom(BH, n);
   CUtensorMap cmap, omap;
   {
-    const uint64_t dims[3] = {(uint64_t)D / 2, (uint64_t)T_cap, (uint64_t)BH};
-    const uint64_t strides[2] = {(uint64_t)D / 2, (uint64_t)(D / 2) * T_cap};
-    const uint32_t box[3] = {(uint32_t)D / 2, (uint32_t)geom.T_box, (uint32_t)geom.BH_box};
+    constexpr int RB = D * BITS / 8;  // code bytes per row
+    const uint64_t dims[3] = {(uint64_t)RB, (uint64_t)T_cap, (uint64_t)BH};
+    const uint64_t strides[2] = {(uint64_t)RB, (uint64_t)RB * T_cap};
+    const uint32_t box[3] = {(uint32_t)(RB < 128 ? RB : 128), (uint32_t)geom.T_box, (uint32_t)geom.BH_box};
     kvq_status st = encode_tiled(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, codes, dims, strides, box,
-                                 D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, "code cache");
+                                 RB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, "code cache");
     if (st != KVQ_OK) return st;
   }
   {
@@ -674,15 +694,15 @@ kvq_status run_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* s
                                  CU_TENSOR_MAP_SWIZZLE_128B, "decode output");
     if (st != KVQ_OK) return st;
   }
-  constexpr int smem = DecSmem<D>::kBytes;
+  constexpr int smem = DecSmem<D, BITS>::kBytes;
   static int blocks_per_sm = -1;
   static std::once_flag once;
   std::call_once(once, [&] {
-    cudaFuncSetAttribute(decode_kernel<D, G, XF>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    blocks_per_sm = occupancy_blocks(decode_kernel<D, G, XF>, smem);
+    cudaFuncSetAttribute(decode_kernel<D, G, XF, BITS>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    blocks_per_sm = occupancy_blocks(decode_kernel<D, G, XF, BITS>, smem);
   });
   const int grid = std::min(geom.n_tiles, blocks_per_sm * num_sms(p->device));
-  decode_kernel<D, G, XF><<<grid, kNT, smem, s>>>(cmap, omap, p->dec, geom, scales, T_cap, t0);
+  decode_kernel<D, G, XF, BITS><<<grid, kNT, smem, s>>>(cmap, omap, p->dec, geom, scales, T_cap, t0);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("decode launch: ") + cudaGetErrorString(e));
   return KVQ_OK;
@@ -707,11 +727,10 @@ kvq_status launch_encode_jobs(const kvq_encode_job* jobs, int njobs, cudaStream_
 template <int XF>
 kvq_status launch_decode_xf(const kvq_plan* p, const uint8_t* codes, const uint16_t* scales, int B, int H, int T_cap,
                             int t0, int n, uint16_t* out, cudaStream_t s) {
-  if (p->D == 128 && p->G == 32) return run_decode<128, 32, XF>(p, codes, scales, B, H, T_cap, t0, n, out, s);
-  if (p->D == 256 && p->G == 32) return run_decode<256, 32, XF>(p, codes, scales, B, H, T_cap, t0, n, out, s);
-  if (p->D == 128 && p->G == 16) return run_decode<128, 16, XF>(p, codes, scales, B, H, T_cap, t0, n, out, s);
-  if (p->D == 256 && p->G == 16) return run_decode<256, 16, XF>(p, codes, scales, B, H, T_cap, t0, n, out, s);
-  return fail(KVQ_ERR_UNSUPPORTED, "decode: unsupported (head_dim, group)");
+  return dispatch_dgb(p->D, p->G, p->bits, [&](auto d, auto g, auto b) {
+    return run_decode<decltype(d)::value, decltype(g)::value, XF, decltype(b)::value>(p, codes, scales, B, H, T_cap,
+                                                                                      t0, n, out, s);
+  });
 }
 
 kvq_status launch_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* scales, int B, int H, int T_cap,

@@ -57,7 +57,7 @@ constexpr int kTcMaxJobs = 64;
 struct alignas(64) TcJob {
   CUtensorMap xmap;  // x as [rows][D] fp16, box {64, 128}, 128-byte swizzle
   CUtensorMap wmap;  // W as [2D][D] fp16 (hi rows, then lo rows; EX: [D][D]), box {64, N}, 128-byte swizzle
-  uint8_t* codes;    // [BH][T_cap][D/2]
+  uint8_t* codes;    // [BH][T_cap][D * BITS / 8]
   uint16_t* scales;  // [BH][T_cap][D/G]
   const float* chan; // EX: the per-channel factors lambda_c / sqrt(D)
   int rows, n, T_cap, pos, tile0;  // rows = B*H*n; tile0 = first global tile of the job
@@ -89,22 +89,35 @@ __device__ __forceinline__ int job_of(const TcJob* jobs, int njobs, int job, int
   return job;
 }
 
-// The quantiser over one 32-channel chunk: one group of 32 or two of 16 (sb: their scales).
-template <int G>
-__device__ __forceinline__ void quantize_chunk(const float (&y)[32], uint32_t (&w)[4], uint32_t (&sb)[32 / G]) {
+// The quantiser over one 32-channel chunk: one group of 32 or two of 16 (sb: their
+// scales); BITS code words (the chunk's 16 or 32 code bytes).
+template <int G, int BITS>
+__device__ __forceinline__ void quantize_chunk(const float (&y)[32], uint32_t (&w)[BITS], uint32_t (&sb)[32 / G]) {
   if constexpr (G == 32) {
-    quantize_group<32>(y, w, sb[0]);
+    quantize_group<32, BITS>(y, w, sb[0]);
   } else {
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
       float yh[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) yh[i] = y[16 * j + i];
-      uint32_t wh[2];
-      quantize_group<16>(yh, wh, sb[j]);
-      w[2 * j] = wh[0];
-      w[2 * j + 1] = wh[1];
+      uint32_t wh[BITS / 2];
+      quantize_group<16, BITS>(yh, wh, sb[j]);
+#pragma unroll
+      for (int i = 0; i < BITS / 2; ++i) w[(BITS / 2) * j + i] = wh[i];
     }
+  }
+}
+
+// the code bytes of 32-channel chunk k of cache row `orow` (16 or 32 bytes)
+template <int D, int BITS>
+__device__ __forceinline__ void store_chunk(uint8_t* codes, size_t orow, int k, const uint32_t (&w)[BITS]) {
+  uint4* row = reinterpret_cast<uint4*>(codes + orow * (D * BITS / 8));
+  if constexpr (BITS == 4) {
+    row[k] = make_uint4(w[0], w[1], w[2], w[3]);
+  } else {
+    row[2 * k] = make_uint4(w[0], w[1], w[2], w[3]);
+    row[2 * k + 1] = make_uint4(w[4], w[5], w[6], w[7]);
   }
 }
 
@@ -122,7 +135,7 @@ __device__ __forceinline__ void store_scales(uint16_t* dst, const uint32_t (&sb)
   }
 }
 
-template <int D, bool EX, int G, int MAXJ>
+template <int D, bool EX, int G, int BITS, int MAXJ>
 __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_constant__ TcBatch<MAXJ> bt) {
   using C = TcCfg<D, EX>;
   constexpr int kTcChunks = C::kChunks;
@@ -323,12 +336,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
             y[g][4 * e + 2] *= f.z;
             y[g][4 * e + 3] *= f.w;
           }
-          uint32_t w[4], sg[SPC];
-          quantize_chunk<G>(y[g], w, sg);
+          uint32_t w[BITS], sg[SPC];
+          quantize_chunk<G, BITS>(y[g], w, sg);
 #pragma unroll
           for (int j = 0; j < SPC; ++j) sb[SPC * g + j] = sg[j];
-          if (valid)
-            reinterpret_cast<uint4*>(J.codes + orow * (D / 2))[NGH * h + g] = make_uint4(w[0], w[1], w[2], w[3]);
+          if (valid) store_chunk<D, BITS>(J.codes, orow, NGH * h + g, w);
         }
         if (valid) store_scales<NGH * SPC>(J.scales + orow * (D / G) + NGH * SPC * h, sb);
       } else {
@@ -356,13 +368,11 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
             y[g][e] = v.x;
             y[g][e + 1] = v.y;
           }
-          uint32_t w[4], sg[SPC];
-          quantize_chunk<G>(y[g], w, sg);
+          uint32_t w[BITS], sg[SPC];
+          quantize_chunk<G, BITS>(y[g], w, sg);
 #pragma unroll
           for (int j = 0; j < SPC; ++j) sb[SPC * g + j] = sg[j];
-          if (valid)
-            reinterpret_cast<uint4*>(J.codes + orow * (D / 2))[4 * half + NGH * h + g] =
-                make_uint4(w[0], w[1], w[2], w[3]);
+          if (valid) store_chunk<D, BITS>(J.codes, orow, 4 * half + NGH * h + g, w);
         }
         if (valid) store_scales<NGH * SPC>(J.scales + orow * (D / G) + SPC * (4 * half + NGH * h), sb);
       }
@@ -379,38 +389,36 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
 }
 
 
-template <int D, bool EX, int G>
-void tc_prepare_one() {
-  cudaFuncSetAttribute(encode_tc_kernel<D, EX, G, kTcMaxJobs>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                       TcCfg<D, EX>::kSmem);
-}
-
 void tc_prepare() {
   static std::once_flag once;
   std::call_once(once, [] {
-    tc_prepare_one<128, false, 32>();
-    tc_prepare_one<256, false, 32>();
-    tc_prepare_one<128, true, 32>();
-    tc_prepare_one<256, true, 32>();
-    tc_prepare_one<128, false, 16>();
-    tc_prepare_one<256, false, 16>();
-    tc_prepare_one<128, true, 16>();
-    tc_prepare_one<256, true, 16>();
+    for (int bits : {4, 8})
+      for (int D : {128, 256})
+        for (int G : {32, 16})
+          dispatch_dgb(D, G, bits, [](auto d, auto g, auto b) {
+            constexpr int kD = decltype(d)::value, kG = decltype(g)::value, kB = decltype(b)::value;
+            cudaFuncSetAttribute(encode_tc_kernel<kD, false, kG, kB, kTcMaxJobs>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<kD, false>::kSmem);
+            cudaFuncSetAttribute(encode_tc_kernel<kD, true, kG, kB, kTcMaxJobs>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<kD, true>::kSmem);
+            return 0;
+          });
   });
 }
 
-template <int D, bool EX, int G>
+template <int D, bool EX, int G, int BITS>
 cudaError_t tc_launch(cudaLaunchConfig_t cfg, const TcBatch<kTcMaxJobs>& bt, int tiles, int sms) {
   cfg.gridDim = dim3(TcCfg<D, EX>::kSplit == 2 ? 2 * std::min(tiles, sms / 2) : std::min(tiles, sms));
   cfg.dynamicSmemBytes = TcCfg<D, EX>::kSmem;
-  return cudaLaunchKernelEx(&cfg, encode_tc_kernel<D, EX, G, kTcMaxJobs>, bt);
+  return cudaLaunchKernelEx(&cfg, encode_tc_kernel<D, EX, G, BITS, kTcMaxJobs>, bt);
 }
 
 }  // namespace
 
 bool encode_tc_supported(int D, int G) { return (D == 128 || D == 256) && (G == 32 || G == 16); }
 
-// Grouped launch over jobs of one head_dim (128 or 256, group 32); jobs with no rows are skipped.
+// Grouped launch over jobs of one head_dim (128 or 256), group (32 or 16), transform and
+// code width (4 or 8 bits); jobs with no rows are skipped.
 kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t strm) {
   const int D = jobs[0].plan->D;
   const bool ex = jobs[0].plan->xform == 1;  // SRHT: exact W
@@ -469,17 +477,10 @@ kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t 
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    const int G = jobs[0].plan->G;
-    cudaError_t e;
-    if (G == 32) {
-      e = ex ? (D == 128 ? tc_launch<128, true, 32>(cfg, bt, tiles, sms) : tc_launch<256, true, 32>(cfg, bt, tiles, sms))
-             : (D == 128 ? tc_launch<128, false, 32>(cfg, bt, tiles, sms)
-                         : tc_launch<256, false, 32>(cfg, bt, tiles, sms));
-    } else {
-      e = ex ? (D == 128 ? tc_launch<128, true, 16>(cfg, bt, tiles, sms) : tc_launch<256, true, 16>(cfg, bt, tiles, sms))
-             : (D == 128 ? tc_launch<128, false, 16>(cfg, bt, tiles, sms)
-                         : tc_launch<256, false, 16>(cfg, bt, tiles, sms));
-    }
+    cudaError_t e = dispatch_dgb(D, jobs[0].plan->G, jobs[0].plan->bits, [&](auto d, auto g, auto b) {
+      constexpr int kD = decltype(d)::value, kG = decltype(g)::value, kB = decltype(b)::value;
+      return ex ? tc_launch<kD, true, kG, kB>(cfg, bt, tiles, sms) : tc_launch<kD, false, kG, kB>(cfg, bt, tiles, sms);
+    });
     if (e == cudaSuccess) e = cudaGetLastError();
     if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("encode (tensor cores) launch: ") + cudaGetErrorString(e));
   }

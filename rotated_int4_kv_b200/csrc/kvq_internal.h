@@ -8,6 +8,7 @@
 #include <stdint.h>
 
 #include <string>
+#include <type_traits>
 
 #include "../../include/kvq.h"
 
@@ -29,6 +30,7 @@ struct kvq_plan {
   int G = 0;
   int device = -1;
   int xform = 0;           // kvq_transform: 0 SRFT, 1 SRHT
+  int bits = 4;            // code width: 4 (nibble pairs) or 8 (one byte per channel)
   kvq::CodecConsts enc{};  // lambda_c * dg_c
   kvq::CodecConsts dec{};  // dg_c / lambda_c
   // Device block: copies of `enc` and `dec` for kernels that serve several plans
@@ -46,6 +48,24 @@ struct kvq_plan {
 };
 
 namespace kvq {
+
+// Bytes of one cached vector's codes.
+inline int code_row_bytes(const kvq_plan* p) { return p->D * p->bits / 8; }
+
+template <int V>
+using IC = std::integral_constant<int, V>;
+
+// Calls f(IC<D>, IC<G>, IC<BITS>) for the quantiser configurations the kernels are
+// built for (D 128 | 256, G 32 | 16, BITS 4 | 8); fails with `what` otherwise.
+template <typename F>
+auto dispatch_dgb(int D, int G, int bits, F&& f) -> decltype(f(IC<128>{}, IC<32>{}, IC<4>{})) {
+  if (bits == 4) {
+    if (D == 128) return G == 32 ? f(IC<128>{}, IC<32>{}, IC<4>{}) : f(IC<128>{}, IC<16>{}, IC<4>{});
+    return G == 32 ? f(IC<256>{}, IC<32>{}, IC<4>{}) : f(IC<256>{}, IC<16>{}, IC<4>{});
+  }
+  if (D == 128) return G == 32 ? f(IC<128>{}, IC<32>{}, IC<8>{}) : f(IC<128>{}, IC<16>{}, IC<8>{});
+  return G == 32 ? f(IC<256>{}, IC<32>{}, IC<8>{}) : f(IC<256>{}, IC<16>{}, IC<8>{});
+}
 
 // thread-local last-error text
 void set_error(const std::string& msg);

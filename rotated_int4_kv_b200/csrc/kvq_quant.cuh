@@ -1,12 +1,14 @@
 // kvq_quant.cuh -- per-group quantisation of rotated, lambda-scaled channels to
-// signed int4 ("When Quantization Is Free", gist.science/de/paper/2605.05699,
-// "Methodik" 2: per-group abs-max scale, symmetric int4 codes, nibble packing).
+// signed int4 or int8 ("When Quantization Is Free", gist.science/de/paper/2605.05699,
+// "Methodik" 2: per-group abs-max scale, rounding to signed int4/int8, nibble packing).
 //
-// scale = fp16_rn(min(absmax / 7, 65504)); code = clamp(rint(y / scale), -7, 7)
+// int4: scale = fp16_rn(min(absmax / 7, 65504)); code = clamp(rint(y / scale), -7, 7)
 // (0 where the scale is 0), two's-complement nibbles, even channel in the low
 // nibble. The rounding is the fp32 "magic number" FMA: y * (1/scale) + (1.5 * 2^23
 // + 8) leaves code + 8 in the low four mantissa bits (round to nearest even), so
 // packing is integer shifts and a byte permute.
+// int8: the same with 127 in place of 7 and 1.5 * 2^23 + 128 (code + 128 in the low
+// byte), one two's-complement byte per channel.
 #pragma once
 
 #include <cuda_fp16.h>
@@ -51,11 +53,41 @@ __device__ __forceinline__ float absmax(const float (&y)[G]) {
   }
 }
 
-// One group of G values (already lambda-scaled): G/8 packed code words and the
-// fp16 scale bits.
-template <int G>
-__device__ __forceinline__ void quantize_group(const float (&y)[G], uint32_t (&words)[G / 8], uint32_t& sbits) {
+constexpr float kMagic8 = 12583040.0f;    // 1.5 * 2^23 + 128: bits = 0x4B400080 + code
+constexpr float kMagic8Lo = 12582913.0f;  // code -127
+constexpr float kMagic8Hi = 12583167.0f;  // code +127
+
+// One group of G values (already lambda-scaled): G * BITS / 32 code words (nibble
+// pairs for BITS = 4, bytes for BITS = 8) and the fp16 scale bits.
+template <int G, int BITS = 4>
+__device__ __forceinline__ void quantize_group(const float (&y)[G], uint32_t (&words)[G * BITS / 32],
+                                               uint32_t& sbits) {
+  static_assert(BITS == 4 || BITS == 8, "code width");
   const float a = absmax<G>(y);
+  if constexpr (BITS == 8) {
+    const float sf = fminf(__fdiv_rn(a, 127.0f), 65504.0f);
+    const __half hs = __float2half_rn(sf);
+    const float sq = __half2float(hs);
+    const float inv = sq > 0.0f ? __frcp_rn(sq) : 0.0f;
+    sbits = __half_as_ushort(hs);
+    uint32_t bits[G];
+    if (a * inv < 127.5f) {
+#pragma unroll
+      for (int i = 0; i < G; ++i) bits[i] = __float_as_uint(fmaf(y[i], inv, kMagic8));
+    } else {
+#pragma unroll
+      for (int i = 0; i < G; ++i)
+        bits[i] = __float_as_uint(fminf(fmaxf(fmaf(y[i], inv, kMagic8), kMagic8Lo), kMagic8Hi));
+    }
+    // low byte of each word = code + 128 (1..255): four bytes per word, then the sign flip
+#pragma unroll
+    for (int w = 0; w < G / 4; ++w) {
+      const uint32_t lo = prmt(bits[4 * w], bits[4 * w + 1], 0x3340u);
+      const uint32_t hi = prmt(bits[4 * w + 2], bits[4 * w + 3], 0x3340u);
+      words[w] = prmt(lo, hi, 0x5410u) ^ 0x80808080u;
+    }
+    return;
+  }
   const float sf = fminf(__fdiv_rn(a, 7.0f), 65504.0f);
   const __half hs = __float2half_rn(sf);
   const float sq = __half2float(hs);

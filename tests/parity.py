@@ -22,20 +22,20 @@ REL_L2 = 2e-3
 BOUNDARY_TALLY = {"bad": 0, "all": 0}
 
 
-def check_encode(x16, signs, lam, G, gpu_packed, gpu_scales, label="", count_only=False, transform="srft"):
-    """x16 [..., D] fp16 (numpy), gpu_packed [..., D/2] u8, gpu_scales [..., D/G] fp16.
+def check_encode(x16, signs, lam, G, gpu_packed, gpu_scales, label="", count_only=False, transform="srft", bits=4):
+    """x16 [..., D] fp16 (numpy), gpu_packed [..., D*bits/8] u8, gpu_scales [..., D/G] fp16.
 
     Returns (boundary mismatches, elements). With count_only the 1e-5 fraction is
     left to the caller, which applies it to all elements of its run (the rule bounds
     the fraction over all elements, not per small piece)."""
     x16 = np.asarray(x16)
     y = oracle.srft_forward(x16, signs, lam, transform)
-    so = oracle.group_scales(y, G).astype(np.float64)
+    so = oracle.group_scales(y, G, bits).astype(np.float64)
     sg = np.asarray(gpu_scales).astype(np.float64)
     bad_scale = np.abs(sg - so) > SCALE_RTOL * np.abs(so)
     assert not bad_scale.any(), f"{label}: {bad_scale.sum()} scales off (e.g. gpu {sg[bad_scale][:4]} vs {so[bad_scale][:4]})"
-    codes_o, u = oracle.quantize(y, np.asarray(gpu_scales), G)
-    codes_g = oracle.unpack_nibbles(np.asarray(gpu_packed))
+    codes_o, u = oracle.quantize(y, np.asarray(gpu_scales), G, bits)
+    codes_g = oracle.unpack_codes(np.asarray(gpu_packed), bits)
     mism = codes_o != codes_g
     dist = np.abs(np.abs(u - np.floor(u)) - 0.5)
     n_m = int(mism.sum())

@@ -22,7 +22,7 @@ def test_header_declares_the_boundary():
               "kvq_workspace_size", "kvq_attend_decode", "kvq_attend_decode_ref", "kvq_status_string",
               "kvq_last_error", "kvq_poll_device_errors", "kvq_attend_decode_batch",
               "kvq_attend_decode_noalloc", "kvq_attend_decode_append", "kvq_plan_create_transform",
-              "kvq_plan_transform"):
+              "kvq_plan_transform", "kvq_plan_create_ex", "kvq_plan_bits"):
         assert n in names
 
 
@@ -68,6 +68,9 @@ def test_status_strings_and_host_checks():
     assert lib.kvq_plan_create(ctypes.byref(h), 128, 24, signs, lam) == -2     # group
     assert lib.kvq_plan_create_transform(ctypes.byref(h), 128, 32, signs, lam, 2) == -2  # transform
     assert lib.kvq_plan_transform(None) == -1
+    assert lib.kvq_plan_create_ex(ctypes.byref(h), 128, 32, signs, lam, 0, 5) == -2  # code width
+    assert b"bits" in lib.kvq_last_error()
+    assert lib.kvq_plan_bits(None) == -1
     bad = (ctypes.c_int8 * 128)(*([1] * 127 + [0]))
     assert lib.kvq_plan_create(ctypes.byref(h), 128, 32, bad, lam) == -1       # sign value
     neg = (ctypes.c_float * 128)(*([1.0] * 127 + [-1.0]))

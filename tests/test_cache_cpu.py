@@ -13,6 +13,9 @@ def test_compression_ratio_matches_pages_and_oracle():
     assert Int4KVCache.compression_ratio(128, 32) == pytest.approx(16 / (4 + 16 / 32))
     assert Int4KVCache.compression_ratio(256, 32) == pytest.approx(3.5556, abs=1e-4)
     assert Int4KVCache.compression_ratio(128, 16) == pytest.approx(3.2)
+    # int8 codes: 2D / (D + 2D/G)
+    assert Int4KVCache.compression_ratio(128, 32, 8) == pytest.approx(256 / 136)
+    assert Int4KVCache.compression_ratio(256, 16, 8) == pytest.approx(2 * 256 / oracle.compressed_bytes_per_vector(256, 16, 8))
     for D in (128, 256):
         for G in (16, 32):
             assert Int4KVCache.compression_ratio(D, G) == pytest.approx(2 * D / oracle.compressed_bytes_per_vector(D, G))
