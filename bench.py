@@ -36,6 +36,8 @@ import kvgen  # noqa: E402
 METRIC = "encode Mvec/s (ns/vec) and int4 decode-attn GB/s, % of B200 HBM roofline"
 WORKLOAD = "gemma"
 N_INPUT_SETS = 3
+TRANSFORM = "srft"
+BITS = 4
 
 
 def _peaks():
@@ -86,13 +88,16 @@ def _source_digest(kind: str) -> str:
 
 
 def _ncu_traffic(kind: str):
+    # captured on the default step (SRFT plans, int4 codes); other variants have no figure
+    if TRANSFORM != "srft" or BITS != 4:
+        return None
     rec = NCU_TRAFFIC.get(kind)
     return rec[1] if rec is not None and rec[0] == _source_digest(kind) else None
 
 
-def _algo_bytes(D: int, G: int = 32):
-    vec = 2 * D + D // 2 + 2 * (D // G)          # encode: fp16 in + codes + scales out
-    tok = 2 * (D // 2 + 2 * (D // G))            # int4 attention: K and V codes + scales per token x kv head
+def _algo_bytes(D: int, G: int = 32, bits: int = 4):
+    vec = 2 * D + D * bits // 8 + 2 * (D // G)   # encode: fp16 in + codes + scales out
+    tok = 2 * (D * bits // 8 + 2 * (D // G))     # quantised attention: K and V codes + scales per token x kv head
     return vec, tok
 
 
@@ -180,10 +185,10 @@ def oracle_sample(wl, seed: int, layer: int = 0):
     v = kvgen.kv_numpy(wl, "v", (1, wl.h_kv, T, D), seed=seed, layer=layer)
     q = kvgen.q_numpy((1, wl.h_q, D), seed=seed, layer=layer)
     t0 = time.perf_counter()
-    ek = oracle.encode(k, ks, kl, G, TRANSFORM)
-    ev = oracle.encode(v, vs, vl, G, TRANSFORM)
+    ek = oracle.encode(k, ks, kl, G, TRANSFORM, BITS)
+    ev = oracle.encode(v, vs, vl, G, TRANSFORM, BITS)
     oracle.attend_decode_int4(q, ek["packed"], ek["scales"], ev["packed"], ev["scales"], (ks, kl), (vs, vl), [T], G,
-                              transform=TRANSFORM)
+                              transform=TRANSFORM, bits=BITS)
     dt = time.perf_counter() - t0
     return 2 * wl.h_kv * T, dt
 
@@ -206,7 +211,7 @@ def cpu_baseline(wl, budget_s: float = 10.0):
         n += 1
     return {"value": vecs / secs / 1e6, "unit": "Mvec/s", "cores": _blas_threads(), "kind": "oracle",
             "sample": f"{n} x one layer of the step (K+V encode of {2 * wl.h_kv * wl.contexts[0]} vectors, D="
-                      f"{wl.head_dim}, plus the 1-token int4 attention over {wl.contexts[0]} tokens), "
+                      f"{wl.head_dim}, plus the 1-token int{BITS} attention over {wl.contexts[0]} tokens), "
                       f"{secs:.1f} s of host time"}
 
 
@@ -242,7 +247,7 @@ TRANSFORM = "srft"
 
 def _config(wl):
     return {"workload": "gemma3-1b-prefill: encode K+V of 26 layers x 4096 tokens, then 1-token int4 decode "
-                        "attention per layer", "transform": TRANSFORM,
+                        "attention per layer", "transform": TRANSFORM, "bits": BITS,
             "layers": wl.layers, "kv_heads": wl.h_kv, "q_heads": wl.h_q, "head_dim": wl.head_dim,
             "batch": wl.batch, "prefix": wl.contexts[0], "group": wl.group,
             "l2": f"inputs rotate over {N_INPUT_SETS} distinct input sets (3 x 109 MB) so each step reads HBM"}
@@ -268,21 +273,21 @@ def run_kvq(args, rank: int, world: int):
     L, Hkv, Hq, D, T, G = wl.layers, wl.h_kv, wl.h_q, wl.head_dim, wl.contexts[0], wl.group
     seed = kvgen.DEFAULT_SEED + 1000 * rank
     NJ = 2 * L
-    vec_b, tok_b = _algo_bytes(D, G)
+    vec_b, tok_b = _algo_bytes(D, G, BITS)
 
     # plans (per layer and K/V), inputs, caches
     plans = []
     for l in range(L):
         for kind in ("k", "v"):
             s, lam = kvgen.plan_params(D, seed=seed, layer=l, kind=kind)
-            plans.append(kvq.Plan(s, lam, group=G, transform=TRANSFORM))
+            plans.append(kvq.Plan(s, lam, group=G, transform=TRANSFORM, bits=BITS))
     X = []
     for i in range(N_INPUT_SETS):
         x = torch.empty((NJ, Hkv, T, D), dtype=torch.float16, device=dev)
         for j in range(NJ):
             kvgen.kv_torch(wl, "kv"[j % 2], (1, Hkv, T, D), dev, seed=seed, layer=j // 2, salt=i, out=x[j:j + 1])
         X.append(x)
-    codes = torch.empty((NJ, Hkv, T, D // 2), dtype=torch.uint8, device=dev)
+    codes = torch.empty((NJ, Hkv, T, D * BITS // 8), dtype=torch.uint8, device=dev)
     scales = torch.empty((NJ, Hkv, T, D // G), dtype=torch.float16, device=dev)
     q = torch.stack([kvgen.q_torch((1, Hq, D), dev, seed=seed, layer=l) for l in range(L)])  # [L, 1, Hq, D]
     out = torch.empty((L, 1, Hq, D), dtype=torch.float16, device=dev)
@@ -421,7 +426,7 @@ def run_kvq(args, rank: int, world: int):
                 "share": enc_avg / (enc_avg + att_avg), "peak_source": src}
     else:
         roof = {"bound": "hbm", "achieved": att_gbs, "peak": hbm, "unit": "GB/s", "frac": att_gbs / hbm,
-                "traffic": _ncu_traffic("attend"), "kernel": f"attend_kernel<{D},int4,32>",
+                "traffic": _ncu_traffic("attend"), "kernel": f"attend_kernel<{D},{'int4' if BITS == 4 else 'int8'},{G}>",
                 "share": att_avg / (enc_avg + att_avg), "peak_source": src}
     res = None
     if rank == 0:
@@ -442,7 +447,7 @@ def run_kvq(args, rank: int, world: int):
                 "encode": {"kernel": roof["kernel"] if enc_avg >= att_avg else "encode", "us": 1e3 * enc_avg,
                            "achieved_GB_s": enc_gbs, "frac": enc_gbs / hbm, "share": enc_avg / (enc_avg + att_avg),
                            "tensor": tensor},
-                "attention": {"kernel": f"attend_kernel<{D},int4,32>", "us": 1e3 * att_avg, "achieved_GB_s": att_gbs,
+                "attention": {"kernel": f"attend_kernel<{D},{'int4' if BITS == 4 else 'int8'},{G}>", "us": 1e3 * att_avg, "achieved_GB_s": att_gbs,
                               "frac": att_gbs / hbm, "share": att_avg / (enc_avg + att_avg),
                               "traffic": _ncu_traffic("attend")},
             },
@@ -503,7 +508,7 @@ def run_decode_workload(args, rank: int, world: int):
     D, Hkv, Hq, B, G = wl.head_dim, wl.h_kv, wl.h_q, wl.batch, wl.group
     seed = kvgen.DEFAULT_SEED + 1000 * rank
     hbm, _ = _peaks()
-    vec_b, tok_b = _algo_bytes(D, G)
+    vec_b, tok_b = _algo_bytes(D, G, BITS)
     contexts = wl.contexts if args.contexts is None else tuple(int(c) for c in args.contexts.split(","))
     layers = wl.layers if args.layers is None else args.layers
     distinct = min(layers, max(1, args.distinct_layers))
@@ -512,12 +517,12 @@ def run_decode_workload(args, rank: int, world: int):
         T_cap = T + 2
         plans, caches, caches16 = [], [], []
         for l in range(distinct):
-            pk = kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=l, kind="k"), transform=TRANSFORM)
-            pv = kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=l, kind="v"), transform=TRANSFORM)
+            pk = kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=l, kind="k"), transform=TRANSFORM, bits=BITS)
+            pv = kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=l, kind="v"), transform=TRANSFORM, bits=BITS)
             plans.append((pk, pv))
             c = {}
             for kind, pl in (("k", pk), ("v", pv)):
-                codes = torch.zeros((B, Hkv, T_cap, D // 2), dtype=torch.uint8, device=dev)
+                codes = torch.zeros((B, Hkv, T_cap, D * BITS // 8), dtype=torch.uint8, device=dev)
                 scales = torch.zeros((B, Hkv, T_cap, D // G), dtype=torch.float16, device=dev)
                 x16 = torch.zeros((B, Hkv, T_cap, D), dtype=torch.float16, device=dev)
                 for b in range(B):
@@ -597,15 +602,16 @@ def run_decode_workload(args, rank: int, world: int):
     if sb:
         # streaming encode: one token per step for each of sb sequences x Hkv heads x {K, V}
         # (one grouped launch per step; a few MB, so this measures latency, not HBM)
-        pk, pv = (kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=0, kind=k), transform=TRANSFORM) for k in ("k", "v"))
+        pk, pv = (kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=0, kind=k), transform=TRANSFORM, bits=BITS)
+                  for k in ("k", "v"))
         xk = kvgen.kv_torch(wl, "k", (sb, Hkv, 1, D), dev, seed=seed, layer=0, salt=77)
         xv = kvgen.kv_torch(wl, "v", (sb, Hkv, 1, D), dev, seed=seed, layer=0, salt=78)
-        kc = torch.zeros((sb, Hkv, 2, D // 2), dtype=torch.uint8, device=dev)
+        kc = torch.zeros((sb, Hkv, 2, D * BITS // 8), dtype=torch.uint8, device=dev)
         ks = torch.zeros((sb, Hkv, 2, D // G), dtype=torch.float16, device=dev)
         vc, vs = torch.zeros_like(kc), torch.zeros_like(ks)
         nvec = 2 * sb * Hkv
         stream_enc = {"sequences": sb, "vectors_per_step": nvec, "l2": "inputs fit in L2: launch latency"}
-        for path in ("tensor", "fft"):
+        for path in (("tensor", "fft") if BITS == 4 else ("tensor",)):  # the FFT encode writes int4 only
             kvq.set_encode_path(path)
             try:
                 ms_e = _graph_time(torch, lambda: kvq.encode_batch([(pk, xk, kc, ks, 0), (pv, xv, vc, vs, 0)]),
@@ -619,7 +625,7 @@ def run_decode_workload(args, rank: int, world: int):
     line = {"metric": METRIC, "value": big["int4_attn_GB_s"], "unit": "GB/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": big["int4_step_ms"],
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": args.workload, "transform": TRANSFORM, "layers": layers, "kv_heads": Hkv,
+            "config": {"workload": args.workload, "transform": TRANSFORM, "bits": BITS, "layers": layers, "kv_heads": Hkv,
                        "q_heads": Hq, "head_dim": D,
                        "batch": B, "contexts": list(contexts), "group": G},
             "cases": cases}
@@ -646,12 +652,15 @@ def main(argv=None):
                     help="profiling mode: run --steps eager steps without timing, for ncu captures")
     ap.add_argument("--transform", default="srft", choices=["srft", "srht"],
                     help="the plans' rotation: srft (the pages' method) or srht (the Hadamard variant)")
+    ap.add_argument("--bits", type=int, default=4, choices=[4, 8],
+                    help="code width of the plans: 4 (the pages' int4, default) or 8 (int8 codes)")
     ap.add_argument("--encode-path", default="auto", choices=["auto", "fft", "tensor"],
                     help="encode kernel of the prefill step: tensor cores where supported (auto), "
                          "the register FFT, or tensor cores only")
     args = ap.parse_args(argv)
-    global TRANSFORM
+    global TRANSFORM, BITS
     TRANSFORM = args.transform
+    BITS = args.bits
     if args.warmup < 3:
         args.warmup = 3
     rank = int(os.environ.get("RANK", "0"))
