@@ -1065,21 +1065,26 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
           if (!vb) s2[sb][2] = s2[sb][3] = -INFINITY;
         }
       }
-      // ---- online softmax over the warp's SUB x 16 tokens (exact running max per head column)
+      // ---- online softmax over the warp's SUB x 16 tokens. The reference m_run of each head
+      // column is a ceiling: every score so far is <= m_run, so p = 2^(s - m_run) <= 1. It
+      // moves (column maxima across the lanes, rescale of o and l) only when a score of this
+      // stage exceeds it, and then to the new maximum plus kHeadroom, so that the next small
+      // rises of the maximum cost one vote and no shuffles.
+      constexpr float kHeadroom = 3.0f;
       float mx0 = fmaxf(s2[0][0], s2[0][2]), mx1 = fmaxf(s2[0][1], s2[0][3]);
 #pragma unroll
       for (int sb = 1; sb < SUB; ++sb) {
         mx0 = fmaxf(mx0, fmaxf(s2[sb][0], s2[sb][2]));
         mx1 = fmaxf(mx1, fmaxf(s2[sb][1], s2[sb][3]));
       }
+      if (__any_sync(0xffffffffu, (mx0 > m_run[0]) || (mx1 > m_run[1]))) {
 #pragma unroll
-      for (int off = 4; off < 32; off <<= 1) {
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-      }
-      const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
-      const bool grow = (mn0 > m_run[0]) || (mn1 > m_run[1]);
-      if (__any_sync(0xffffffffu, grow)) {
+        for (int off = 4; off < 32; off <<= 1) {
+          mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+          mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+        }
+        const float mn0 = mx0 > m_run[0] ? mx0 + kHeadroom : m_run[0];
+        const float mn1 = mx1 > m_run[1] ? mx1 + kHeadroom : m_run[1];
         const float al0 = mn0 == -INFINITY ? 1.0f : fast_exp2(m_run[0] - mn0);
         const float al1 = mn1 == -INFINITY ? 1.0f : fast_exp2(m_run[1] - mn1);
         l_run[0] *= al0;
