@@ -611,7 +611,7 @@ def run_decode_workload(args, rank: int, world: int):
         vc, vs = torch.zeros_like(kc), torch.zeros_like(ks)
         nvec = 2 * sb * Hkv
         stream_enc = {"sequences": sb, "vectors_per_step": nvec, "l2": "inputs fit in L2: launch latency"}
-        for path in (("tensor", "fft") if BITS == 4 else ("tensor",)):  # the FFT encode writes int4 only
+        for path in ("tensor", "fft"):
             kvq.set_encode_path(path)
             try:
                 ms_e = _graph_time(torch, lambda: kvq.encode_batch([(pk, xk, kc, ks, 0), (pv, xv, vc, vs, 0)]),

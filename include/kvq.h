@@ -104,10 +104,9 @@ int kvq_plan_transform(const kvq_plan* plan);
  *         8: the same with 127 in place of 7 (scale = fp16_rn(min(absmax/127, 65504)),
  *            codes in [-127, 127]), one two's-complement byte per channel, channel i at
  *            byte i. Every "D/2" code row below is then D bytes.
- *   Other values: UNSUPPORTED. int8 plans are served by the tensor-core encode (the
- *   register-FFT path, kvq_set_encode_path(1), returns UNSUPPORTED for them), decode
- *   and every attention entry point; both plans of an attention call, and all jobs of
- *   a batch, must share the code width.
+ *   Other values: UNSUPPORTED. int8 plans are served by both encode paths, decode and
+ *   every attention entry point; both plans of an attention call, and all jobs of a
+ *   batch, must share the code width.
  */
 kvq_status kvq_plan_create_ex(kvq_plan** out, int head_dim, int group, const int8_t* signs_host,
                               const float* lambda_host, int transform, int bits);

@@ -84,7 +84,6 @@ kvq_status dispatch_encode(const kvq_encode_job* jobs, int njobs, cudaStream_t s
   if (path == 2 && !tc)
     return fail(KVQ_ERR_UNSUPPORTED, "encode: the tensor-core path supports head_dim 128 or 256 with group 32 or 16");
   if (tc && path != 1) return launch_encode_tc(jobs, njobs, s);
-  if (p->bits != 4) return fail(KVQ_ERR_UNSUPPORTED, "encode: the register-FFT path writes int4 codes only");
   return launch_encode_jobs(jobs, njobs, s);
 }
 

@@ -136,11 +136,12 @@ __device__ __forceinline__ uint32_t atom_add_acq_rel(uint32_t* p, uint32_t v) {
   return old;
 }
 
-// lambda, per-group abs-max, fp16 scale, int4 rounding and nibble packing of
-// NV channel values (NV/G groups); lam points at the lambda*dg of those channels.
-template <int NV, int G>
+// lambda, per-group abs-max, fp16 scale, rounding and packing (int4 nibble pairs or
+// int8 bytes) of NV channel values (NV/G groups); lam points at the lambda*dg of those
+// channels.
+template <int NV, int G, int BITS>
 __device__ __forceinline__ void quantize_pack(const float (&v)[NV], const float* __restrict__ lam,
-                                              uint32_t (&words)[NV / 8], uint32_t (&sbits)[NV / G]) {
+                                              uint32_t (&words)[NV * BITS / 32], uint32_t (&sbits)[NV / G]) {
 #pragma unroll
   for (int g = 0; g < NV / G; ++g) {
     float y[G];
@@ -152,14 +153,15 @@ __device__ __forceinline__ void quantize_pack(const float (&v)[NV], const float*
       y[4 * i4 + 2] = v[g * G + 4 * i4 + 2] * l4.z;
       y[4 * i4 + 3] = v[g * G + 4 * i4 + 3] * l4.w;
     }
-    uint32_t w[G / 8];
-    quantize_group<G>(y, w, sbits[g]);
+    constexpr int kGW = G * BITS / 32;
+    uint32_t w[kGW];
+    quantize_group<G, BITS>(y, w, sbits[g]);
 #pragma unroll
-    for (int i = 0; i < G / 8; ++i) words[g * (G / 8) + i] = w[i];
+    for (int i = 0; i < kGW; ++i) words[g * kGW + i] = w[i];
   }
 }
 
-template <int D>
+template <int D, int BITS>
 struct EncCfg {
   static constexpr int kTPV = D / 128;                 // threads per vector
   static constexpr int kRows = kNT / kTPV;             // vectors per tile
@@ -167,14 +169,15 @@ struct EncCfg {
   static constexpr int kXStage = kRows * D * 2;        // 32 KB
   static constexpr int kBoxBytes = kRows * 128;        // one 64-half box
   static constexpr int kStages = 2;
-  static constexpr int kCWarp = kRowsW * D / 2;        // per-warp code staging (2 KB)
+  static constexpr int kRowBytes = D * BITS / 8;       // code bytes per vector
+  static constexpr int kCWarp = kRowsW * kRowBytes;    // per-warp code staging (2 or 4 KB)
   static constexpr int kBytes = kStages * kXStage + 4 * kCWarp + 64 + 1024;
 };
 
 // XF: 0 = SRFT (real FFT in registers), 1 = SRHT (Walsh-Hadamard butterflies).
-template <int D, int G, int XF, int MAXJ>
+template <int D, int G, int XF, int BITS, int MAXJ>
 __global__ void __launch_bounds__(kNT, 3) encode_kernel(const __grid_constant__ EncBatch<MAXJ> P) {
-  using C = EncCfg<D>;
+  using C = EncCfg<D, BITS>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* xs = smem;
@@ -267,7 +270,8 @@ __global__ void __launch_bounds__(kNT, 3) encode_kernel(const __grid_constant__ 
       }
     }
     // ---- transform (packed f32x2 halves + scalar top stage), lambda, quantise, pack
-    uint32_t words[16];
+    constexpr int kHW = 64 * BITS / 32;  // code words of one 64-channel half
+    uint32_t words[2 * kHW];
     uint32_t sbits[128 / G];
     int cb_lo, cb_hi;  // first channels of the two 64-channel halves this thread owns
     if constexpr (XF == 1) {
@@ -306,13 +310,13 @@ __global__ void __launch_bounds__(kNT, 3) encode_kernel(const __grid_constant__ 
         lo[i] = vv[i];
         hi[i] = vv[64 + i];
       }
-      uint32_t wl[8], wh[8], sl[64 / G], sh[64 / G];
-      quantize_pack<64, G>(lo, J.cc->chan + cb_lo, wl, sl);
-      quantize_pack<64, G>(hi, J.cc->chan + cb_hi, wh, sh);
+      uint32_t wl[kHW], wh[kHW], sl[64 / G], sh[64 / G];
+      quantize_pack<64, G, BITS>(lo, J.cc->chan + cb_lo, wl, sl);
+      quantize_pack<64, G, BITS>(hi, J.cc->chan + cb_hi, wh, sh);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < kHW; ++i) {
         words[i] = wl[i];
-        words[8 + i] = wh[i];
+        words[kHW + i] = wh[i];
       }
 #pragma unroll
       for (int i = 0; i < 64 / G; ++i) {
@@ -324,7 +328,7 @@ __global__ void __launch_bounds__(kNT, 3) encode_kernel(const __grid_constant__ 
       float vv[128];
 #pragma unroll
       for (int c = 0; c < 128; ++c) vv[c] = slotv(v, slot_of_channel(c, 128));
-      quantize_pack<128, G>(vv, J.cc->chan, words, sbits);
+      quantize_pack<128, G, BITS>(vv, J.cc->chan, words, sbits);
       cb_lo = 0;
       cb_hi = 64;
     } else {
@@ -339,13 +343,13 @@ __global__ void __launch_bounds__(kNT, 3) encode_kernel(const __grid_constant__ 
         lo[i] = vv[i];
         hi[i] = vv[64 + i];
       }
-      uint32_t wl[8], wh[8], sl[64 / G], sh[64 / G];
-      quantize_pack<64, G>(lo, J.cc->chan + cb_lo, wl, sl);
-      quantize_pack<64, G>(hi, J.cc->chan + cb_hi, wh, sh);
+      uint32_t wl[kHW], wh[kHW], sl[64 / G], sh[64 / G];
+      quantize_pack<64, G, BITS>(lo, J.cc->chan + cb_lo, wl, sl);
+      quantize_pack<64, G, BITS>(hi, J.cc->chan + cb_hi, wh, sh);
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
+      for (int i = 0; i < kHW; ++i) {
         words[i] = wl[i];
-        words[8 + i] = wh[i];
+        words[kHW + i] = wh[i];
       }
 #pragma unroll
       for (int i = 0; i < 64 / G; ++i) {
@@ -375,15 +379,21 @@ __global__ void __launch_bounds__(kNT, 3) encode_kernel(const __grid_constant__ 
     __syncwarp();
     {
       const int rw = r - warp * C::kRowsW;  // row within the warp's slice
-      uint8_t* row = cs + rw * (D / 2);
+      constexpr int kHC = 64 * BITS / 8 / 16;  // 16-byte chunks per 64-channel half (2 or 4)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
 #pragma unroll
-        for (int c2 = 0; c2 < 2; ++c2) {  // 16-byte chunks = 32 channels
-          const int ch = (h ? cb_hi : cb_lo) / 32 + c2;
-          const int pc = (D == 128) ? (ch ^ ((rw >> 1) & 3)) : (ch ^ (rw & 7));
-          const int wi = 8 * h + 4 * c2;
-          *reinterpret_cast<uint4*>(row + pc * 16) = make_uint4(words[wi], words[wi + 1], words[wi + 2], words[wi + 3]);
+        for (int c2 = 0; c2 < kHC; ++c2) {
+          const int ch = (h ? cb_hi : cb_lo) * BITS / 128 + c2;  // 16-byte chunk of the code row
+          const int wi = kHW * h + 4 * c2;
+          uint8_t* dst;
+          if constexpr (BITS == 4) {  // one box per row (64- or 128-byte swizzle)
+            const int pc = (D == 128) ? (ch ^ ((rw >> 1) & 3)) : (ch ^ (rw & 7));
+            dst = cs + rw * (D / 2) + pc * 16;
+          } else {  // 128-byte boxes of the warp's rows (128-byte swizzle)
+            dst = cs + (ch >> 3) * (C::kRowsW * 128) + rw * 128 + (((ch & 7) ^ (rw & 7)) << 4);
+          }
+          *reinterpret_cast<uint4*>(dst) = make_uint4(words[wi], words[wi + 1], words[wi + 2], words[wi + 3]);
         }
       }
     }
@@ -391,7 +401,10 @@ __global__ void __launch_bounds__(kNT, 3) encode_kernel(const __grid_constant__ 
     __syncwarp();
     if (lane == 0) {
       const int r0 = warp * C::kRowsW;  // the warp's rows: a {Tw, RowsW/Tw} box of the tile
-      tma_store_3d(&J.cmap, cs, 0, J.pos + t0 + (r0 & (J.T_box - 1)), bh0 + (r0 >> J.t_shift));
+#pragma unroll
+      for (int bx = 0; bx < (BITS == 4 ? 1 : D / 128); ++bx)
+        tma_store_3d(&J.cmap, cs + bx * (C::kRowsW * 128), 128 * bx, J.pos + t0 + (r0 & (J.T_box - 1)),
+                     bh0 + (r0 >> J.t_shift));
       bulk_commit_group();
     }
   }
@@ -597,8 +610,9 @@ int occupancy_blocks(K kernel, int smem_bytes) {
   return nb;
 }
 
-template <int D, int G, int XF, int MAXJ>
+template <int D, int G, int XF, int BITS, int MAXJ>
 kvq_status run_encode_chunk(const kvq_encode_job* jobs, int nj, cudaStream_t s) {
+  using C = EncCfg<D, BITS>;
   EncBatch<MAXJ> P;
   memset(&P, 0, sizeof(P));
   int tiles = 0;
@@ -606,8 +620,8 @@ kvq_status run_encode_chunk(const kvq_encode_job* jobs, int nj, cudaStream_t s) 
     const kvq_encode_job& q = jobs[i];
     EncJob& J = P.jobs[i];
     const int BH = q.B * q.H;
-    TileGeom geom = make_geom(BH, q.n, EncCfg<D>::kRows);
-    const int RW = EncCfg<D>::kRowsW;
+    TileGeom geom = make_geom(BH, q.n, C::kRows);
+    const int RW = C::kRowsW;
     const int Tw = std::min(geom.T_box, RW);
     {
       const uint64_t dims[3] = {(uint64_t)D, (uint64_t)q.n, (uint64_t)BH};
@@ -618,11 +632,12 @@ kvq_status run_encode_chunk(const kvq_encode_job* jobs, int nj, cudaStream_t s) 
       if (st != KVQ_OK) return st;
     }
     {
-      const uint64_t dims[3] = {(uint64_t)D / 2, (uint64_t)(q.pos + q.n), (uint64_t)BH};
-      const uint64_t strides[2] = {(uint64_t)D / 2, (uint64_t)(D / 2) * q.T_cap};
-      const uint32_t box[3] = {(uint32_t)D / 2, (uint32_t)Tw, (uint32_t)(RW / Tw)};
+      constexpr int RB = C::kRowBytes;
+      const uint64_t dims[3] = {(uint64_t)RB, (uint64_t)(q.pos + q.n), (uint64_t)BH};
+      const uint64_t strides[2] = {(uint64_t)RB, (uint64_t)RB * q.T_cap};
+      const uint32_t box[3] = {(uint32_t)(RB < 128 ? RB : 128), (uint32_t)Tw, (uint32_t)(RW / Tw)};
       kvq_status st = encode_tiled(&J.cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q.codes, dims, strides, box,
-                                   D == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, "code cache");
+                                   RB == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, "code cache");
       if (st != KVQ_OK) return st;
     }
     J.cc = q.plan->enc_dev;
@@ -641,8 +656,8 @@ kvq_status run_encode_chunk(const kvq_encode_job* jobs, int nj, cudaStream_t s) 
   }
   P.njobs = nj;
   P.total_tiles = tiles;
-  void (*kern)(const EncBatch<MAXJ>) = encode_kernel<D, G, XF, MAXJ>;
-  const int smem = EncCfg<D>::kBytes;
+  void (*kern)(const EncBatch<MAXJ>) = encode_kernel<D, G, XF, BITS, MAXJ>;
+  const int smem = C::kBytes;
   static int blocks_per_sm = -1;
   static std::once_flag once;
   std::call_once(once, [&] {
@@ -660,12 +675,12 @@ kvq_status run_encode_chunk(const kvq_encode_job* jobs, int nj, cudaStream_t s) 
 
 constexpr int kMaxJobs = 64;
 
-template <int D, int G, int XF>
+template <int D, int G, int XF, int BITS>
 kvq_status run_encode(const kvq_encode_job* jobs, int njobs, cudaStream_t s) {
-  if (njobs == 1) return run_encode_chunk<D, G, XF, 1>(jobs, 1, s);
+  if (njobs == 1) return run_encode_chunk<D, G, XF, BITS, 1>(jobs, 1, s);
   for (int i = 0; i < njobs; i += kMaxJobs) {
     const int nj = std::min(kMaxJobs, njobs - i);
-    kvq_status st = run_encode_chunk<D, G, XF, kMaxJobs>(jobs + i, nj, s);
+    kvq_status st = run_encode_chunk<D, G, XF, BITS, kMaxJobs>(jobs + i, nj, s);
     if (st != KVQ_OK) return st;
   }
   return KVQ_OK;
@@ -712,11 +727,9 @@ kvq_status run_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* s
 
 template <int XF>
 kvq_status launch_encode_xf(const kvq_encode_job* jobs, int njobs, int D, int G, cudaStream_t s) {
-  if (D == 128 && G == 32) return run_encode<128, 32, XF>(jobs, njobs, s);
-  if (D == 256 && G == 32) return run_encode<256, 32, XF>(jobs, njobs, s);
-  if (D == 128 && G == 16) return run_encode<128, 16, XF>(jobs, njobs, s);
-  if (D == 256 && G == 16) return run_encode<256, 16, XF>(jobs, njobs, s);
-  return fail(KVQ_ERR_UNSUPPORTED, "encode: unsupported (head_dim, group)");
+  return dispatch_dgb(D, G, jobs[0].plan->bits, [&](auto d, auto g, auto b) {
+    return run_encode<decltype(d)::value, decltype(g)::value, XF, decltype(b)::value>(jobs, njobs, s);
+  });
 }
 
 kvq_status launch_encode_jobs(const kvq_encode_job* jobs, int njobs, cudaStream_t s) {

@@ -3,8 +3,8 @@ int8 here is the int4 quantiser with 127 in place of 7 and one byte per code) on
 entry point that serves them, against the oracle with bits = 8: the tensor-core encode
 (D = 128 / 256, G = 32 / 16, SRFT / SRHT), decode, decode attention (GQA, ragged
 lengths, several tiles and a ragged tail, batched jobs, the allocation-free variant),
-the fused append, sequence-sharded partials and the cache wrapper. The register-FFT
-encode writes int4 codes only and must refuse int8 plans."""
+the fused append, sequence-sharded partials and the cache wrapper; both encode paths
+(tensor cores, register FFT)."""
 import numpy as np
 import pytest
 
@@ -29,10 +29,11 @@ def _plan(kvq, D, kind, G=32, xf="srft", layer=0, seed=81):
     return kvq.Plan(s, lam, G, xf, BITS), (s, lam)
 
 
+@pytest.mark.parametrize("path", ["tensor", "fft"])
 @pytest.mark.parametrize("xf", ["srft", "srht"])
 @pytest.mark.parametrize("wl_name,B,H,n,G", [("qwen", 2, 2, 130, 32), ("gemma", 1, 1, 300, 32), ("toy", 1, 1, 77, 16),
                                              ("gemma", 2, 1, 65, 16), ("mistral", 1, 3, 513, 32)])
-def test_int8_encode_decode(kvq, xf, wl_name, B, H, n, G):
+def test_int8_encode_decode(kvq, path, xf, wl_name, B, H, n, G):
     wl = kvgen.WORKLOADS[wl_name]
     D = wl.head_dim
     plan, (s, lam) = _plan(kvq, D, "k", G, xf)
@@ -41,11 +42,15 @@ def test_int8_encode_decode(kvq, xf, wl_name, B, H, n, G):
     T_cap, pos = n + 6, 3
     codes = torch.full((B, H, T_cap, D), 0xA5, dtype=torch.uint8, device="cuda")
     scales = torch.full((B, H, T_cap, D // G), 7.0, dtype=torch.float16, device="cuda")
-    kvq.encode(plan, torch.from_numpy(x16).cuda(), codes, scales, pos)
+    kvq.set_encode_path(path)
+    try:
+        kvq.encode(plan, torch.from_numpy(x16).cuda(), codes, scales, pos)
+    finally:
+        kvq.set_encode_path("auto")
     torch.cuda.synchronize()
     assert kvq.poll_device_errors() == 0
     c, sc = codes.cpu().numpy(), scales.cpu().numpy()
-    nb, na = check_encode(x16, s, lam, G, c[:, :, pos:pos + n], sc[:, :, pos:pos + n], label=f"{wl_name} {xf}",
+    nb, na = check_encode(x16, s, lam, G, c[:, :, pos:pos + n], sc[:, :, pos:pos + n], label=f"{wl_name} {xf} {path}",
                           count_only=True, transform=xf, bits=BITS)
     TALLY["bad"] += nb
     TALLY["all"] += na
@@ -82,18 +87,11 @@ def test_int8_grouped_encode_batch(kvq):
         TALLY["all"] += na
 
 
-def test_int8_refused_by_the_fft_encode_and_mixed_widths(kvq):
+def test_int8_and_int4_plans_do_not_mix(kvq):
     D = 128
     plan, _ = _plan(kvq, D, "k")
-    x = torch.zeros((1, 1, 4, D), dtype=torch.float16, device="cuda")
     codes = torch.zeros((1, 1, 4, D), dtype=torch.uint8, device="cuda")
     scales = torch.zeros((1, 1, 4, D // 32), dtype=torch.float16, device="cuda")
-    kvq.set_encode_path("fft")
-    try:
-        with pytest.raises(kvq.KvqError, match="UNSUPPORTED"):
-            kvq.encode(plan, x, codes, scales, 0)
-    finally:
-        kvq.set_encode_path("auto")
     s, lam = kvgen.plan_params(D, kind="v")
     pv4 = kvq.Plan(s, lam)  # int4
     q = torch.zeros((1, 4, D), dtype=torch.float16, device="cuda")
