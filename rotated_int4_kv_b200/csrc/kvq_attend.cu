@@ -1732,23 +1732,32 @@ SplitPlan choose_split(int B, int Hq, int Hkv, int T, const Occupancy& occ, int 
   } else {
     // estimated time in stage-times: rounds of resident CTAs x (stages per split +
     // the per-CTA fixed cost), plus the workspace merge when a unit has several clusters
+    // cluster candidates: the default rule (a divisor up to 4), and one cluster spanning
+    // every split (up to 8), which saves the workspace merge when its CTAs fit in the
+    // same number of rounds
     long best_t = -1;
     for (int S = 1; S <= s_cap; ++S) {
       const int Sr = realised(S);
       if (!mergeable(Sr)) continue;
-      const int C = cluster_for(Sr, cmax);
-      const long rounds = (units * Sr + occ.cap[C] - 1) / occ.cap[C];
-      const long t = rounds * ((ntile + S - 1) / S + kFixedTiles) + (Sr / C > 1 ? kMergeTiles : 0);
-      if (best_t < 0 || t < best_t) {
-        best_t = t;
-        best = S;
+      const int cands[2] = {cluster_for(Sr, cmax), Sr <= kMaxCluster ? Sr : 0};
+      for (const int C : cands) {
+        if (C < 1) continue;
+        const long rounds = (units * Sr + occ.cap[C] - 1) / occ.cap[C];
+        const long t = rounds * ((ntile + S - 1) / S + kFixedTiles) + (Sr / C > 1 ? kMergeTiles : 0);
+        if (best_t < 0 || t < best_t) {
+          best_t = t;
+          best = S;
+          best_c = C == cluster_for(Sr, cmax) ? 0 : C;
+        }
       }
     }
   }
   const int tiles_per = (ntile + best - 1) / best;
   sp.tps = tiles_per * tile;
   if (best_c > 0) {
-    sp.S = best;
+    // latency regime: S as chosen (trailing splits may be empty, C divides S); throughput
+    // regime: the realised split count, which the one-cluster candidate C equals
+    sp.S = latency ? best : (ntile + tiles_per - 1) / tiles_per;
     sp.C = best_c;
   } else {
     sp.S = (ntile + tiles_per - 1) / tiles_per;
