@@ -66,15 +66,21 @@ struct Cfg {
   static constexpr int NC = D / 32;                        // 32-channel chunks of a code row (16 or 32 bytes)
   static constexpr int NG = INT4 ? D / G : NC;             // scale groups per token (quantised caches)
   static constexpr int kRowBytes = INT4 ? D * BITS / 8 : 2 * D;  // bytes per token row of K (and V)
-  // consumer warps (plus one producer warp); resident CTAs per SM for the launch bounds
-  static constexpr int kCWarps = 4;
+  // consumer warps (plus one producer warp); resident CTAs per SM for the launch bounds.
+  // kTWarps groups of tokens; with kCSplit = 2 (D = 256 int4) each group is a warp pair,
+  // one warp per 128-channel half: the pair trades partial scores through shared memory
+  // and each warp converts, multiplies and accumulates only its half (twice the warps per
+  // SM, half the latency chain per warp)
+  static constexpr int kCSplit = (INT4 && BITS == 4 && D == 256) ? 2 : 1;
+  static constexpr int kTWarps = 4;
+  static constexpr int kCWarps = kTWarps * kCSplit;
   static constexpr int kThreads = (kCWarps + 1) * 32;
   static constexpr int kMinBlocks = D == 128 ? 2 : 1;
   // each consumer warp takes kSub subtiles of 16 tokens per stage (two independent
   // instruction streams for the int4 path, whose per-token work is latency-bound; one
   // for int8, whose rows are twice as long)
   static constexpr int kSub = (INT4 && BITS == 4) ? 2 : 1;
-  static constexpr int kTile = 16 * kCWarps * kSub;        // tokens per stage
+  static constexpr int kTile = 16 * kTWarps * kSub;        // tokens per stage
   static constexpr int kKBytes = kTile * kRowBytes;
   static constexpr int kSBytes = INT4 ? kTile * NG * 2 : 0;
   static constexpr int kStageBytes = 2 * kKBytes + 2 * kSBytes;
@@ -87,7 +93,7 @@ struct Cfg {
   static constexpr int kRing = kStages * kStageBytes;
   // tail scratch (reuses the ring): the warps' partials, this CTA's partial, the merged
   // (M, L) and the warps' (m, l); the un-rotated output reuses the warp partials
-  static constexpr int kTail = ((kCWarps + 1) * (2 * kHT + kHT * D) + 2 * kHT + kCWarps * 2 * kHT) * 4;
+  static constexpr int kTail = ((kTWarps + 1) * (2 * kHT + kHT * D) + 2 * kHT + kTWarps * 2 * kHT) * 4;
   static constexpr int kScratch = kRing > kTail ? kRing : kTail;
   static constexpr int kQt = kHT * D * 4;                  // fp32 q_t (or merged o_t) [8][D]
   // staged at kernel start by bulk copies: the tile's query rows (fp16 [8][D]) and,
@@ -105,11 +111,15 @@ struct Cfg {
   // B-fragment buffer (built only after the append's encode), at D = 256 (whose query
   // rotation uses that buffer as scratch) in a region of their own
   static constexpr int kApp = (INT4 && D == 256) ? 2 * D * 2 : 0;
+  // warp pairs: partial scores [stage parity][group][half][subtile][lane] float4, then
+  // one mbarrier per (stage parity, group) on which both warps' 64 threads meet
+  static constexpr int kXchData = kCSplit > 1 ? 2 * kTWarps * 2 * kSub * 32 * 16 : 0;
+  static constexpr int kXch = kCSplit > 1 ? kXchData + 2 * kTWarps * 8 : 0;
   static constexpr int kBars = 128;        // full[], empty[], const, rotation, cluster rdy / got barriers, flag
   // D = 128 int4: the plan's rotation matrix (hi, lo) for the query, then the V plan's
   // transpose for the output, as [hi/lo][64-column chunk][128 rows][128 B] (128-byte swizzle)
   static constexpr bool kMmaRot = INT4;   // F128 (D = 256: even/odd split)
-  static constexpr int kRotOff = (kScratch + kQt + kQs + kConsts + kQf + kApp + kBars + 1023) / 1024 * 1024;
+  static constexpr int kRotOff = (kScratch + kQt + kQs + kConsts + kQf + kApp + kXch + kBars + 1023) / 1024 * 1024;
   static constexpr int kRot = kMmaRot ? 4 * 128 * 128 : 0;
   static constexpr int kSmem = kRotOff + kRot + 1024;
   static_assert(2 * kStages * 8 + 3 * 8 + 4 <= kBars, "barrier region");
@@ -117,7 +127,7 @@ struct Cfg {
   static_assert(kKBytes % 1024 == 0 && kStageBytes % 1024 == 0, "stage layout");
   // the merge weights of up to kMaxMerge partials reuse the (dead) B fragments
   static_assert(kQf >= 2 * kMaxMerge * kHT * 4, "merge scratch");
-  static_assert(kHT * D <= kCWarps * (2 * kHT + kHT * D), "output scratch");
+  static_assert(kHT * D <= kTWarps * (2 * kHT + kHT * D), "output scratch");
 };
 
 struct AttnParams {
@@ -624,6 +634,8 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
   constexpr int NG = C::NG;
   constexpr int NC = C::NC;
   constexpr int MT = D / 16;  // channel m-tiles of the PV product
+  constexpr int kTWarps = C::kTWarps, kCSplit = C::kCSplit;
+  constexpr int MTH = MT / kCSplit;  // m-tiles of this warp's channel half
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
@@ -637,7 +649,10 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
   uint4* qf = reinterpret_cast<uint4*>(smem + C::kScratch + C::kQt + C::kQs + C::kConsts);
   uint16_t* app_in = reinterpret_cast<uint16_t*>(D == 128 ? smem + C::kScratch + C::kQt + C::kQs + C::kConsts
                                                                 : smem + C::kScratch + C::kQt + C::kQs + C::kConsts + C::kQf);
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kScratch + C::kQt + C::kQs + C::kConsts + C::kQf + C::kApp);
+  float4* xch = reinterpret_cast<float4*>(smem + C::kScratch + C::kQt + C::kQs + C::kConsts + C::kQf + C::kApp);
+  uint64_t* xbar = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(xch) + C::kXchData);  // [2][groups]
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + C::kScratch + C::kQt + C::kQs + C::kConsts + C::kQf + C::kApp +
+                                               C::kXch);
   uint64_t* empty = full + C::kStages;
   uint64_t* cbar = empty + C::kStages;
   uint64_t* rdy = cbar + 1;   // cluster peers: the leader has read this CTA's partial
@@ -648,6 +663,9 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int g = lane >> 2, c = lane & 3;
+  const int tw = warp % kTWarps;              // consumer warps: the token group
+  const int chh = warp / kTWarps;             // and the channel half (0 without the pair split)
+  const int mo = chh * MTH;                   // first m-tile of the half
   const int split = blockIdx.x, ht = blockIdx.y;
   const int job = MAXJ == 1 ? 0 : (int)blockIdx.z / (p.B * p.Hkv);
   const int bk = (int)blockIdx.z - job * (p.B * p.Hkv);
@@ -668,6 +686,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
       mbar_init(&empty[s], kCWarps);
     }
     mbar_init(cbar, 1);
+    for (int x = 0; x < (kCSplit > 1 ? 2 * kTWarps : 0); ++x) mbar_init(&xbar[x], 64);
     mbar_init(rdy, 1);
     mbar_init(got, cluster_nctarank() > 1 ? cluster_nctarank() - 1 : 1);
     fence_mbarrier_init();
@@ -716,9 +735,9 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
   // per-warp softmax state (consumer warps): heads 2c, 2c+1
   float m_run[2] = {-INFINITY, -INFINITY};
   float l_run[2] = {0.0f, 0.0f};
-  float o_acc[MT][4];
+  float o_acc[MTH][4];
 #pragma unroll
-  for (int i = 0; i < MT; ++i) o_acc[i][0] = o_acc[i][1] = o_acc[i][2] = o_acc[i][3] = 0.0f;
+  for (int i = 0; i < MTH; ++i) o_acc[i][0] = o_acc[i][1] = o_acc[i][2] = o_acc[i][3] = 0.0f;
   bool ok = true;
 
   if (warp == kCWarps) {
@@ -916,7 +935,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
       const uint8_t* st = ring + s * C::kStageBytes;
       // this warp's SUB subtiles of 16 tokens: stage rows (SUB warp + sb) 16 .. + 15
       constexpr int SUB = C::kSub;
-      if (t_begin + i * C::kTile + warp * SUB * 16 >= t_end) {
+      if (t_begin + i * C::kTile + tw * SUB * 16 >= t_end) {
         // none of the warp's tokens is in range (the ragged last stage): nothing to add
         __syncwarp();
         if (lane == 0) mbar_arrive(&empty[s]);
@@ -927,7 +946,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
       float sc[SUB][4];
 #pragma unroll
       for (int sb = 0; sb < SUB; ++sb) {
-        const int r0s = (warp * SUB + sb) * 16;
+        const int r0s = (tw * SUB + sb) * 16;
         tw0[sb] = t_begin + i * C::kTile + r0s;
         partial[sb] = tw0[sb] + 16 > t_end;
         float scs[4] = {0.f, 0.f, 0.f, 0.f};
@@ -936,12 +955,13 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
           const uint8_t* kt = st;
           const uint8_t* ks = st + 2 * C::kKBytes;
           // scales of tokens r0+g and r0+g+8
-          float skA[NG], skB[NG];
+          constexpr int NGL = NG / kCSplit;  // scale groups of this warp's channel half
+          float skA[NGL], skB[NGL];
           {
-            const uint16_t* sa = reinterpret_cast<const uint16_t*>(ks) + (r0s + g) * NG;
-            const uint16_t* sb = reinterpret_cast<const uint16_t*>(ks) + (r0s + g + 8) * NG;
+            const uint16_t* sa = reinterpret_cast<const uint16_t*>(ks) + (r0s + g) * NG + chh * NGL;
+            const uint16_t* sb = reinterpret_cast<const uint16_t*>(ks) + (r0s + g + 8) * NG + chh * NGL;
   #pragma unroll
-            for (int q2 = 0; q2 < NG / 2; ++q2) {
+            for (int q2 = 0; q2 < NGL / 2; ++q2) {
               const float2 fa = __half22float2(bits_h2(reinterpret_cast<const uint32_t*>(sa)[q2]));
               const float2 fb = __half22float2(bits_h2(reinterpret_cast<const uint32_t*>(sb)[q2]));
               skA[2 * q2] = fa.x;
@@ -979,7 +999,8 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
             }
           } else {
   #pragma unroll
-          for (int gp = 0; gp < NC / 2; ++gp) {  // two 32-channel chunks per ldmatrix.x4
+          for (int gpl = 0; gpl < NC / 2 / kCSplit; ++gpl) {  // two 32-channel chunks per ldmatrix.x4
+            const int gp = chh * (NC / 2 / kCSplit) + gpl;     // (of this warp's channel half)
             const int mi = lane >> 3;
             const int row = r0s + ((mi & 1) << 3) + (lane & 7);
             const int chunk = 2 * gp + (mi >> 1);
@@ -991,7 +1012,8 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
             nib8_to_h2(w1, hB0);
             nib8_to_h2(w2, hA1);
             nib8_to_h2(w3, hB1);
-            const int G0 = 2 * gp, G1 = 2 * gp + 1;
+            const int G0 = 2 * gp, G1 = 2 * gp + 1;      // chunks of the row (query fragments)
+            const int L0 = 2 * gpl, L1 = 2 * gpl + 1;    // the same within the half (scales)
             const uint4 f0 = qf[(2 * G0) * 32 + lane], f1 = qf[(2 * G0 + 1) * 32 + lane];
             const uint4 f2 = qf[(2 * G1) * 32 + lane], f3 = qf[(2 * G1 + 1) * 32 + lane];
             if constexpr (G == 16) {
@@ -1014,8 +1036,8 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
                 scs[2] = fmaf(skB[2 * CH], a[0][2], fmaf(skB[2 * CH + 1], a[1][2], scs[2]));
                 scs[3] = fmaf(skB[2 * CH], a[0][3], fmaf(skB[2 * CH + 1], a[1][3], scs[3]));
               };
-              chunk(hA0, hB0, f0, f1, G0);
-              chunk(hA1, hB1, f2, f3, G1);
+              chunk(hA0, hB0, f0, f1, L0);
+              chunk(hA1, hB1, f2, f3, L1);
               continue;
             }
             float a0[4] = {0.f, 0.f, 0.f, 0.f}, a1[4] = {0.f, 0.f, 0.f, 0.f};
@@ -1027,10 +1049,10 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
             mma_16816(a1, hA1[0], hB1[0], hA1[1], hB1[1], f2.z, f2.w);
             mma_16816(a1, hA1[2], hB1[2], hA1[3], hB1[3], f3.x, f3.y);
             mma_16816(a1, hA1[2], hB1[2], hA1[3], hB1[3], f3.z, f3.w);
-            scs[0] = fmaf(skA[G0], a0[0], fmaf(skA[G1], a1[0], scs[0]));
-            scs[1] = fmaf(skA[G0], a0[1], fmaf(skA[G1], a1[1], scs[1]));
-            scs[2] = fmaf(skB[G0], a0[2], fmaf(skB[G1], a1[2], scs[2]));
-            scs[3] = fmaf(skB[G0], a0[3], fmaf(skB[G1], a1[3], scs[3]));
+            scs[0] = fmaf(skA[L0], a0[0], fmaf(skA[L1], a1[0], scs[0]));
+            scs[1] = fmaf(skA[L0], a0[1], fmaf(skA[L1], a1[1], scs[1]));
+            scs[2] = fmaf(skB[L0], a0[2], fmaf(skB[L1], a1[2], scs[2]));
+            scs[3] = fmaf(skB[L0], a0[3], fmaf(skB[L1], a1[3], scs[3]));
           }
           }
         } else {
@@ -1052,6 +1074,32 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
 
 #pragma unroll
         for (int e = 0; e < 4; ++e) sc[sb][e] = scs[e];
+      }
+      if constexpr (kCSplit == 2) {
+        // the pair's partial scores over the two channel halves: publish, meet, add (the
+        // sum is the same in both warps: fp addition commutes); slots alternate by stage,
+        // so a slot is rewritten only after the partner passed the next meeting
+        float4* mine = xch + ((((i & 1) * kTWarps + tw) * 2 + chh) * SUB) * 32;
+        const float4* other = xch + ((((i & 1) * kTWarps + tw) * 2 + (chh ^ 1)) * SUB) * 32;
+#pragma unroll
+        for (int sb = 0; sb < SUB; ++sb) mine[sb * 32 + lane] = make_float4(sc[sb][0], sc[sb][1], sc[sb][2], sc[sb][3]);
+        // every thread of the pair arrives (release of its own stores) and waits (acquire),
+        // bounded: a partner that gave up a wait cannot hold this warp
+        uint64_t* xb = &xbar[(i & 1) * kTWarps + tw];
+        mbar_arrive(xb);
+        if (!__all_sync(0xffffffffu, mbar_wait_bounded(xb, (i >> 1) & 1))) {  // warp-uniform outcome
+          atomicOr(&g_attend_err, kErrTimeoutLoad);
+          ok = false;
+          break;
+        }
+#pragma unroll
+        for (int sb = 0; sb < SUB; ++sb) {
+          const float4 v = other[sb * 32 + lane];
+          sc[sb][0] += v.x;
+          sc[sb][1] += v.y;
+          sc[sb][2] += v.z;
+          sc[sb][3] += v.w;
+        }
       }
       // base-2 scores with masking of tokens outside [t_begin, t_end)
       float s2[SUB][4];
@@ -1090,7 +1138,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
         l_run[0] *= al0;
         l_run[1] *= al1;
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
+        for (int mt = 0; mt < MTH; ++mt) {
           o_acc[mt][0] *= al0;
           o_acc[mt][1] *= al1;
           o_acc[mt][2] *= al0;
@@ -1120,21 +1168,22 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
       }
 #pragma unroll
       for (int sb = 0; sb < SUB; ++sb) {
-        const int r0s = (warp * SUB + sb) * 16;
+        const int r0s = (tw * SUB + sb) * 16;
         // ---- PV: O^T[channel][head] += V^T[channel][token] P[token][head]
         if constexpr (INT4) {
           const uint8_t* vt = st + C::kKBytes;
           const uint16_t* vs = reinterpret_cast<const uint16_t*>(st + 2 * C::kKBytes + C::kSBytes);
           // V scales of tokens 2c, 2c+1, 2c+8, 2c+9 (rows of this warp), paired per group
-          uint32_t sw[4][NG / 2];
+          constexpr int NGLV = NG / kCSplit;  // scale groups of this warp's channel half
+          uint32_t sw[4][NGLV / 2];
           {
             const int toks[4] = {2 * c, 2 * c + 1, 2 * c + 8, 2 * c + 9};
   #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const uint32_t* sp = reinterpret_cast<const uint32_t*>(vs + (r0s + toks[e]) * NG);
+              const uint32_t* sp = reinterpret_cast<const uint32_t*>(vs + (r0s + toks[e]) * NG + chh * NGLV);
               const bool valid = !partial[sb] || (tw0[sb] + toks[e] < t_end);
   #pragma unroll
-              for (int q2 = 0; q2 < NG / 2; ++q2) sw[e][q2] = valid ? sp[q2] : 0u;
+              for (int q2 = 0; q2 < NGLV / 2; ++q2) sw[e][q2] = valid ? sp[q2] : 0u;
             }
           }
           if constexpr (BITS == 8) {
@@ -1163,7 +1212,8 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
             }
           } else {
   #pragma unroll
-          for (int gp = 0; gp < NC / 2; ++gp) {
+          for (int gpl = 0; gpl < NC / 2 / kCSplit; ++gpl) {
+            const int gp = chh * (NC / 2 / kCSplit) + gpl;  // (of this warp's channel half)
             const int mi = lane >> 3;
             const int row = r0s + ((mi & 1) << 3) + (lane & 7);
             const int chunk = 2 * gp + (mi >> 1);
@@ -1172,7 +1222,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
             ldmatrix_x4_trans(w0, w1, w2, w3, smem_u32(vt + row * C::kRowBytes + pch * 16));
   #pragma unroll
             for (int h = 0; h < 2; ++h) {
-              const int CH = 2 * gp + h;  // the 32-channel chunk
+              const int CH = 2 * gpl + h;  // the 32-channel chunk within the half (registers)
               uint32_t lo[4], hi[4];
               nib8_to_h2(h ? w2 : w0, lo);  // tokens 2c, 2c+1: channels 4g .. 4g+3 of the chunk
               nib8_to_h2(h ? w3 : w1, hi);  // tokens 2c+8, 2c+9
@@ -1232,9 +1282,10 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
       l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
     }
     if constexpr (INT4) {
-      if (app && warp == 0) {
-        // the appended token: one more element of warp 0's online softmax (scores and
-        // dequantised V row from (1b); l is the warp total here, so every lane adds p)
+      if (app && tw == 0) {
+        // the appended token: one more element of token group 0's online softmax (scores
+        // and dequantised V row from (1b); l is the warp total here, so every lane adds p;
+        // with the pair split both warps of the group add it, each to its channel half)
         const float* vhat = ybuf + D;
         float pn[2], al[2];
 #pragma unroll
@@ -1247,13 +1298,14 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
           m_run[e] = mn;
         }
 #pragma unroll
-        for (int mt = 0; mt < MT; ++mt) {
+        for (int ml = 0; ml < MTH; ++ml) {
+          const int mt = mo + ml;  // the m-tile's place in the whole row
           const int ch0 = BITS == 8 ? 16 * mt + 2 * g : (mt >> 1) * 32 + 4 * g + ((mt & 1) ? 2 : 0);
           const int ch1 = ch0 + 1;
-          o_acc[mt][0] = fmaf(o_acc[mt][0], al[0], pn[0] * vhat[ch0]);
-          o_acc[mt][1] = fmaf(o_acc[mt][1], al[1], pn[1] * vhat[ch0]);
-          o_acc[mt][2] = fmaf(o_acc[mt][2], al[0], pn[0] * vhat[ch1]);
-          o_acc[mt][3] = fmaf(o_acc[mt][3], al[1], pn[1] * vhat[ch1]);
+          o_acc[ml][0] = fmaf(o_acc[ml][0], al[0], pn[0] * vhat[ch0]);
+          o_acc[ml][1] = fmaf(o_acc[ml][1], al[1], pn[1] * vhat[ch0]);
+          o_acc[ml][2] = fmaf(o_acc[ml][2], al[0], pn[0] * vhat[ch1]);
+          o_acc[ml][3] = fmaf(o_acc[ml][3], al[1], pn[1] * vhat[ch1]);
         }
       }
     }
@@ -1264,16 +1316,18 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
   // ------------------------------------------------------------ merge the warps (ring is free now)
   // Each warp rescales its (m, l, o) to the CTA maximum M = max_w m_w, then the CTA
   // partial is O = sum_w o_w 2^(m_w - M), L = sum_w l_w 2^(m_w - M).
+  // (per token group: the two warps of a pair hold the same m and l and one channel
+  // half of o each)
   constexpr int PART = 2 * kHT + kHT * D;        // m[8] | l[8] | o[8][D]
-  float* wst = reinterpret_cast<float*>(ring);  // [warp][PART] (o only)
-  float* cpart = wst + kCWarps * PART;           // this CTA's partial [PART]
+  float* wst = reinterpret_cast<float*>(ring);  // [group][PART] (o only)
+  float* cpart = wst + kTWarps * PART;           // this CTA's partial [PART]
   float* mrg = cpart + PART;                     // merged (M, L) [2][8]
-  float* wml = mrg + 2 * kHT;                    // the warps' (m, l) [warp][2][8]
-  if (warp < kCWarps && g == 0) {
-    wml[warp * 2 * kHT + 2 * c] = m_run[0];
-    wml[warp * 2 * kHT + 2 * c + 1] = m_run[1];
-    wml[warp * 2 * kHT + kHT + 2 * c] = l_run[0];
-    wml[warp * 2 * kHT + kHT + 2 * c + 1] = l_run[1];
+  float* wml = mrg + 2 * kHT;                    // the groups' (m, l) [group][2][8]
+  if (warp < kCWarps && chh == 0 && g == 0) {
+    wml[tw * 2 * kHT + 2 * c] = m_run[0];
+    wml[tw * 2 * kHT + 2 * c + 1] = m_run[1];
+    wml[tw * 2 * kHT + kHT + 2 * c] = l_run[0];
+    wml[tw * 2 * kHT + kHT + 2 * c + 1] = l_run[1];
   }
   __syncthreads();
   if (warp < kCWarps) {
@@ -1283,12 +1337,13 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
       const int h = 2 * c + e;
       float M = -INFINITY;
 #pragma unroll
-      for (int w = 0; w < kCWarps; ++w) M = fmaxf(M, wml[w * 2 * kHT + h]);
+      for (int w = 0; w < kTWarps; ++w) M = fmaxf(M, wml[w * 2 * kHT + h]);
       sc[e] = m_run[e] == -INFINITY ? 0.0f : fast_exp2(m_run[e] - M);
     }
-    float* wo = wst + warp * PART + 2 * kHT;
+    float* wo = wst + tw * PART + 2 * kHT;
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
+    for (int ml = 0; ml < MTH; ++ml) {
+      const int mt = mo + ml;
       int ch0, ch1;  // channels held in rows g and g+8 of m-tile mt
       if constexpr (INT4 && BITS == 8) {
         ch0 = 16 * mt + 2 * g;
@@ -1300,20 +1355,20 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
         ch0 = mt * 16 + g;
         ch1 = ch0 + 8;
       }
-      wo[(2 * c) * D + ch0] = o_acc[mt][0] * sc[0];
-      wo[(2 * c + 1) * D + ch0] = o_acc[mt][1] * sc[1];
-      wo[(2 * c) * D + ch1] = o_acc[mt][2] * sc[0];
-      wo[(2 * c + 1) * D + ch1] = o_acc[mt][3] * sc[1];
+      wo[(2 * c) * D + ch0] = o_acc[ml][0] * sc[0];
+      wo[(2 * c + 1) * D + ch0] = o_acc[ml][1] * sc[1];
+      wo[(2 * c) * D + ch1] = o_acc[ml][2] * sc[0];
+      wo[(2 * c + 1) * D + ch1] = o_acc[ml][3] * sc[1];
     }
   } else if (lane < kHT) {
     const int h = lane;
     float M = -INFINITY;
 #pragma unroll
-    for (int w = 0; w < kCWarps; ++w) M = fmaxf(M, wml[w * 2 * kHT + h]);
+    for (int w = 0; w < kTWarps; ++w) M = fmaxf(M, wml[w * 2 * kHT + h]);
     float L = 0.0f;
     if (M != -INFINITY) {
 #pragma unroll
-      for (int w = 0; w < kCWarps; ++w) {
+      for (int w = 0; w < kTWarps; ++w) {
         const float mw = wml[w * 2 * kHT + h];
         if (mw != -INFINITY) L += wml[w * 2 * kHT + kHT + h] * fast_exp2(mw - M);
       }
@@ -1325,7 +1380,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
   for (int i = threadIdx.x; i < heads * D / 4; i += kThreads) {
     float4 acc = reinterpret_cast<const float4*>(wst + 2 * kHT)[i];
 #pragma unroll
-    for (int w = 1; w < kCWarps; ++w) {
+    for (int w = 1; w < kTWarps; ++w) {
       const float4 v = reinterpret_cast<const float4*>(wst + w * PART + 2 * kHT)[i];
       acc.x += v.x;
       acc.y += v.y;
