@@ -421,8 +421,8 @@ def run_kvq(args, rank: int, world: int):
     if enc_avg >= att_avg:
         roof = {"bound": "hbm", "achieved": enc_gbs, "peak": hbm, "unit": "GB/s", "frac": enc_gbs / hbm,
                 "traffic": _ncu_traffic("encode_tc" if tc else "encode"),
-                "kernel": f"encode_tc_kernel<{D},64>" if tc
-                else f"encode_kernel<{D},{G},64>",
+                "kernel": f"encode_tc_kernel<{D},{int(TRANSFORM == 'srht')},{G},{BITS},64>" if tc
+                else f"encode_kernel<{D},{G},{int(TRANSFORM == 'srht')},{BITS},64>",
                 "share": enc_avg / (enc_avg + att_avg), "peak_source": src}
     else:
         roof = {"bound": "hbm", "achieved": att_gbs, "peak": hbm, "unit": "GB/s", "frac": att_gbs / hbm,
