@@ -202,17 +202,32 @@ def _blas_threads():
         return os.cpu_count() or 1
 
 
-def cpu_baseline(wl, budget_s: float = 10.0):
-    vecs, secs, n = 0, 0.0, 0
-    while secs < budget_s or n < 1:
-        v, dt = oracle_sample(wl, seed=kvgen.DEFAULT_SEED, layer=n % wl.layers)
-        vecs += v
-        secs += dt
-        n += 1
-    return {"value": vecs / secs / 1e6, "unit": "Mvec/s", "cores": _blas_threads(), "kind": "oracle",
+def cpu_baseline(wl, budget_s: float = 10.0, single_budget_s: float = 5.0):
+    """The oracle on the host's cores (BLAS threads = all cores), plus the same sample with
+    one BLAS thread."""
+    def run(budget):
+        vecs, secs, n = 0, 0.0, 0
+        while secs < budget or n < 1:
+            v, dt = oracle_sample(wl, seed=kvgen.DEFAULT_SEED, layer=n % wl.layers)
+            vecs += v
+            secs += dt
+            n += 1
+        return vecs / secs / 1e6, n, secs
+
+    value, n, secs = run(budget_s)
+    single = None
+    try:
+        from threadpoolctl import threadpool_limits
+        with threadpool_limits(limits=1):
+            v1, n1, s1 = run(single_budget_s)
+        single = {"value": v1, "cores": 1, "sample": f"{n1} layers, {s1:.1f} s"}
+    except ImportError:
+        pass
+    return {"value": value, "unit": "Mvec/s", "cores": _blas_threads(), "kind": "oracle",
             "sample": f"{n} x one layer of the step (K+V encode of {2 * wl.h_kv * wl.contexts[0]} vectors, D="
                       f"{wl.head_dim}, plus the 1-token int{BITS} attention over {wl.contexts[0]} tokens), "
-                      f"{secs:.1f} s of host time"}
+                      f"{secs:.1f} s of host time",
+            "single_thread": single}
 
 
 # ---------------------------------------------------------------- reference arm
@@ -398,6 +413,16 @@ def run_kvq(args, rank: int, world: int):
     h2d = x_dev.numel() * 2 + q.numel() * 2
     d2h = out.numel() * 2
 
+    # ---- decode (the inverse, not part of the step): one launch over the step's 52 packed
+    # caches as a batch of 52 (the first plan's s and lambda for all: a throughput figure;
+    # its parity is tested per plan). Codes and scales (30.7 MB) were just written and may
+    # be L2-resident; the 109 MB fp16 output streams to HBM.
+    dec_out = torch.empty((NJ, Hkv, T, D), dtype=torch.float16, device=dev)
+    ms_dec = _graph_time(torch, lambda: kvq.decode(plans[0], codes, scales, 0, T, out=dec_out), 20, 3)
+    ms_dec = max_over_ranks([ms_dec], dist, dev)[0]
+    del dec_out
+    assert kvq.poll_device_errors() == 0
+
     vec_step = NJ * Hkv * T
     value = job_throughput(world, vec_step, ms, args.steps)
     hbm, peak_kind = _peaks()
@@ -451,6 +476,10 @@ def run_kvq(args, rank: int, world: int):
                               "frac": att_gbs / hbm, "share": att_avg / (enc_avg + att_avg),
                               "traffic": _ncu_traffic("attend")},
             },
+            "decode": {"kernel_us": 1e3 * ms_dec, "ns_per_vec": 1e6 * ms_dec / vec_step,
+                       "GB_s": vec_step * vec_b / (ms_dec * 1e-3) / 1e9,
+                       "frac_hbm": vec_step * vec_b / (ms_dec * 1e-3) / 1e9 / hbm, "bytes_per_vec": vec_b,
+                       "note": "one launch over the 52 caches of the step; input may be L2-resident"},
             "cpu_baseline": cpu,
             "e2e": {"value": world * vec_step / (e2e_ms * 1e-3) / 1e6, "unit": "Mvec/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
