@@ -32,6 +32,9 @@
  *      x / out vectors   fp16 [B, H, n, D]
  *      codes cache       u8   [B, H, T_cap, D/2]   two's-complement nibbles,
  *                                                  channel 2j in the low nibble of byte j
+ *                                                  (int8 plans, kvq_plan_create_ex:
+ *                                                  [B, H, T_cap, D], one byte per channel;
+ *                                                  every "D/2" below is then D)
  *      scales cache      fp16 [B, H, T_cap, D/G]   scale of channels [gG, gG+G)
  *      q                 fp16 [B, Hq, D]
  *      attention out     fp16 [B, Hq, D]

@@ -164,7 +164,7 @@ struct alignas(64) AttnJob {
   CUtensorMap rotmap;                    // int4: F128 (hi/lo rows), from the K plan
   const uint16_t* q;
   uint16_t* out;
-  const CodecConsts* ke;  // K plan: sign masks (int4 only)
+  const CodecConsts* ke;  // K plan: sign masks (quantised caches only)
   const CodecConsts* kd;  // K plan: dg / lambda per channel
   const CodecConsts* vd;  // V plan: dg / lambda per channel, sign masks
 };
@@ -245,7 +245,6 @@ __device__ __forceinline__ int chan_of_slot128(int j) { return j == 0 ? 0 : (j =
 // the channel of row j of the resident matrix: the real DFT's slot order, or (hada:
 // SRHT plans, the matrix is the Hadamard matrix) the identity
 __device__ __forceinline__ int chan_of_row128(int j, bool hada) { return hada ? j : chan_of_slot128(j); }
-__device__ __forceinline__ int slot_of_chan128(int c) { return c == 0 ? 0 : (c == 127 ? 1 : c + 1); }
 
 // X[j][r] = sum_m F128[j][m] x'_r[m] for up to eight fp16 rows x_r (x'_r = x_r with the
 // sign mask sgn_of(r) applied to its fp16 pairs, exact), on the tensor cores:

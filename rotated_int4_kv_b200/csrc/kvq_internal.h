@@ -94,7 +94,8 @@ kvq_status launch_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t
                          int T_cap, int t0, int n, uint16_t* out, cudaStream_t s);
 
 // attention launchers (kvq_attend.cu)
-// One decode-attention problem: plans (int4 only), query, caches, output.
+// One decode-attention problem: plans (quantised caches; none for the fp16 comparator),
+// query, caches, output.
 struct AttendJobHost {
   const kvq_plan* pk;
   const kvq_plan* pv;
