@@ -13,6 +13,10 @@ import oracle
 SCALE_RTOL = 1e-3
 BOUNDARY_BAND = 1e-4
 MAX_BOUNDARY_FRAC = 1e-5
+# int8 codes: the same band, the fraction scaled by qmax / 7 = 127 / 7. The rule is stated
+# for int4 codes; with 18x finer bins relative to y, the same relative error of the GPU's
+# fp32 transform puts 18x more elements within the band of a rounding boundary.
+MAX_BOUNDARY_FRAC_INT8 = MAX_BOUNDARY_FRAC * 127 / 7
 REL_L2 = 2e-3
 
 

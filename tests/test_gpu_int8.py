@@ -10,7 +10,7 @@ import pytest
 
 import kvgen
 import oracle
-from tests.parity import MAX_BOUNDARY_FRAC, check_encode, check_rel_l2
+from tests.parity import MAX_BOUNDARY_FRAC_INT8, check_encode, check_rel_l2
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -261,4 +261,4 @@ def test_int8_cache_wrapper(kvq):
 def test_int8_boundary_fraction_over_all_cases():
     if TALLY["all"] == 0:
         pytest.skip("no int8 encode ran")
-    assert TALLY["bad"] <= MAX_BOUNDARY_FRAC * TALLY["all"], TALLY
+    assert TALLY["bad"] <= MAX_BOUNDARY_FRAC_INT8 * TALLY["all"], TALLY
