@@ -83,3 +83,53 @@ def test_random_shape(c):
         ref = oracle.attend_decode_int4(q16[b:b + 1], kc[b:b + 1], ks[b:b + 1], vc[b:b + 1], vs[b:b + 1], k[1], v[1],
                                         [lens[b]], G, transform=xf, bits=bits)
         check_rel_l2(got[b:b + 1].reshape(-1, D), ref.reshape(-1, D), label=f"b{b} T{lens[b]}")
+
+
+APPEND_CASES = [c for i, c in enumerate(CASES) if i % 2 == 0]
+
+
+@pytest.mark.parametrize("c", APPEND_CASES, ids=[f"D{c['D']}-i{c['bits']}-G{c['G']}-{c['xf']}-B{c['B']}-kv{c['Hkv']}"
+                                                  f"-q{c['Hq']}-T{c['T_cap']}" for c in APPEND_CASES])
+def test_random_append_and_partials(c):
+    """The fused append at a random position, then the sequence split into random slices
+    (partials + combine), both against the oracle on the GPU's own cache."""
+    import rotated_int4_kv_b200 as kvq
+
+    D, bits, G, xf, B, Hkv, Hq, T_cap = (c[k] for k in ("D", "bits", "G", "xf", "B", "Hkv", "Hq", "T_cap"))
+    wl = kvgen.WORKLOADS["qwen" if D == 128 else "gemma"]
+    dev = torch.device("cuda")
+    rng = np.random.default_rng(c["seed"] + 7)
+    pos = int(rng.integers(0, T_cap))  # the new token's row; rows [0, pos) are cached
+    cache = {}
+    for kind in ("k", "v"):
+        s, lam = kvgen.plan_params(D, seed=c["seed"], kind=kind)
+        plan = kvq.Plan(s, lam, G, xf, bits)
+        codes = torch.zeros((B, Hkv, T_cap, D * bits // 8), dtype=torch.uint8, device=dev)
+        scales = torch.zeros((B, Hkv, T_cap, D // G), dtype=torch.float16, device=dev)
+        if pos:
+            x16 = kvgen.kv_numpy(wl, kind, (B, Hkv, pos, D), seed=c["seed"])
+            kvq.encode(plan, torch.from_numpy(x16).to(dev), codes, scales, 0)
+        new = kvgen.kv_numpy(wl, kind, (B, Hkv, D), seed=c["seed"], salt=5)
+        cache[kind] = (plan, (s, lam), codes, scales, new)
+    q16 = kvgen.q_numpy((B, Hq, D), seed=c["seed"], salt=3)
+    q = torch.from_numpy(q16).to(dev)
+    k, v = cache["k"], cache["v"]
+    out = kvq.attend_decode_append(k[0], v[0], q, torch.from_numpy(k[4]).to(dev), torch.from_numpy(v[4]).to(dev),
+                                   k[2], k[3], v[2], v[3], pos)
+    torch.cuda.synchronize()
+    assert kvq.poll_device_errors() == 0
+    kc, ks, vc, vs = (t.cpu().numpy() for t in (k[2], k[3], v[2], v[3]))
+    T = pos + 1
+    ref = oracle.attend_decode_int4(q16, kc, ks, vc, vs, k[1], v[1], [T] * B, G, transform=xf, bits=bits)
+    check_rel_l2(out.cpu().numpy().astype(np.float64).reshape(-1, D), ref.reshape(-1, D), label=f"append pos {pos}")
+    # the same T tokens in random slices (even starts), merged by the combine kernel
+    cuts = sorted({0, T} | {2 * int(x) for x in rng.integers(0, T // 2 + 1, size=int(rng.integers(1, 4)))})
+    cuts = [x for x in cuts if x <= T]
+    if cuts[-1] != T:
+        cuts.append(T)
+    parts = [kvq.attend_decode_partial(k[0], v[0], q, k[2], k[3], v[2], v[3], cuts[j], cuts[j + 1])
+             for j in range(len(cuts) - 1)]
+    merged = kvq.attend_combine(v[0], torch.stack(parts))
+    torch.cuda.synchronize()
+    assert kvq.poll_device_errors() == 0
+    check_rel_l2(merged.cpu().numpy().astype(np.float64).reshape(-1, D), ref.reshape(-1, D), label=f"slices {cuts}")
