@@ -86,6 +86,7 @@ def encode(plan: Plan, x: torch.Tensor, codes: torch.Tensor, scales: torch.Tenso
            stream=None) -> None:
     """Encode x [B, H, n, D] fp16 into cache rows pos..pos+n-1 of codes / scales."""
     B, H, n, D = x.shape
+    _same_dim(D, plan)
     T_cap = codes.shape[2]
     _need(x, "x", torch.float16)
     _need(codes, "codes", torch.uint8, (B, H, T_cap, D * plan.bits // 8))
@@ -100,6 +101,7 @@ def encode_batch(jobs, stream=None) -> None:
     arr = (EncodeJob * max(1, len(jobs)))()
     for i, (plan, x, codes, scales, pos) in enumerate(jobs):
         B, H, n, D = x.shape
+        _same_dim(D, plan)
         T_cap = codes.shape[2]
         _need(x, f"jobs[{i}].x", torch.float16)
         _need(codes, f"jobs[{i}].codes", torch.uint8, (B, H, T_cap, D * plan.bits // 8))
@@ -138,6 +140,14 @@ def decode(plan: Plan, codes: torch.Tensor, scales: torch.Tensor, t0: int, n: in
     return out
 
 
+def _same_dim(D: int, *plans) -> None:
+    """The C ABI sizes every row by the plan's head_dim; a tensor of another head_dim
+    would be read or written past its end, so it is refused here."""
+    for pl in plans:
+        if pl.head_dim != D:
+            raise ValueError(f"tensor head_dim {D} does not match the plan's head_dim {pl.head_dim}")
+
+
 def workspace_size(B: int, Hq: int, Hkv: int, head_dim: int, T_cap: int) -> int:
     return int(lib.kvq_workspace_size(B, Hq, Hkv, head_dim, T_cap))
 
@@ -152,6 +162,7 @@ def attend_decode(pk: Plan, pv: Plan, q, k_codes, k_scales, v_codes, v_scales, s
                   softmax_scale: float = 0.0, out=None, workspace=None, stream=None) -> torch.Tensor:
     """One-query decode attention on the packed int4 cache (rotated domain)."""
     B, Hq, D = q.shape
+    _same_dim(D, pk, pv)
     _, Hkv, T_cap, half = k_codes.shape
     _need(q, "q", torch.float16)
     for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
@@ -180,6 +191,7 @@ def attend_decode_append(pk: Plan, pv: Plan, q, k_new, v_new, k_codes, k_scales,
     [B, Hkv, D] or [B, Hkv, 1, D]) into the caches at token ``pos`` and attend over
     tokens 0 .. pos (see kvq_attend_decode_append)."""
     B, Hq, D = q.shape
+    _same_dim(D, pk, pv)
     _, Hkv, T_cap, _ = k_codes.shape
     _need(q, "q", torch.float16)
     for name, t in (("k_new", k_new), ("v_new", v_new)):
@@ -207,6 +219,7 @@ def attend_decode_partial(pk: Plan, pv: Plan, q, k_codes, k_scales, v_codes, v_s
     """Sequence-sharded decode, step 1: the softmax partial of every query head over
     cached tokens [t_begin, t_end) (fp32 [B, Hq, D + 4]; see kvq_attend_decode_partial)."""
     B, Hq, D = q.shape
+    _same_dim(D, pk, pv)
     _, Hkv, T_cap, _ = k_codes.shape
     _need(q, "q", torch.float16)
     for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):
@@ -230,6 +243,7 @@ def attend_combine(pv: Plan, partials, out=None, stream=None) -> torch.Tensor:
     (see kvq_attend_combine); returns fp16 [B, Hq, D]."""
     N, B, Hq, D4 = partials.shape
     D = D4 - 4
+    _same_dim(D, pv)
     _need(partials, "partials", torch.float32)
     if out is None:
         out = torch.empty((B, Hq, D), dtype=torch.float16, device=partials.device)
@@ -277,6 +291,7 @@ def attend_decode_batch(jobs, seq_lens=None, T_len=None, softmax_scale: float = 
     outs = []
     for i, job in enumerate(jobs):
         pk, pv, q, k_codes, k_scales, v_codes, v_scales = job[:7]
+        _same_dim(D, pk, pv)
         out = job[7] if len(job) > 7 and job[7] is not None else torch.empty((B, Hq, D), dtype=torch.float16,
                                                                              device=q.device)
         _need(q, f"jobs[{i}].q", torch.float16, (B, Hq, D))
@@ -306,6 +321,7 @@ def attend_decode_noalloc(pk: Plan, pv: Plan, q, k_codes, k_scales, v_codes, v_s
     allocate device memory; its scratch is a static array inside the library
     (8 MiB, shared by all calls: calls that overlap on the GPU race)."""
     B, Hq, D = q.shape
+    _same_dim(D, pk, pv)
     _, Hkv, T_cap, half = k_codes.shape
     _need(q, "q", torch.float16)
     for name, t in (("k_codes", k_codes), ("v_codes", v_codes)):

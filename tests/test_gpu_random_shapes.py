@@ -133,3 +133,25 @@ def test_random_append_and_partials(c):
     torch.cuda.synchronize()
     assert kvq.poll_device_errors() == 0
     check_rel_l2(merged.cpu().numpy().astype(np.float64).reshape(-1, D), ref.reshape(-1, D), label=f"slices {cuts}")
+
+
+def test_head_dim_mismatch_is_refused():
+    """The C ABI sizes rows by the plan's head_dim: the binding refuses tensors of another
+    head_dim before anything is launched."""
+    import rotated_int4_kv_b200 as kvq
+
+    pk = kvq.Plan(*kvgen.plan_params(128, kind="k"))
+    pv = kvq.Plan(*kvgen.plan_params(128, kind="v"))
+    dev = torch.device("cuda")
+    x = torch.zeros((1, 1, 4, 64), dtype=torch.float16, device=dev)
+    codes = torch.zeros((1, 1, 4, 32), dtype=torch.uint8, device=dev)
+    scales = torch.zeros((1, 1, 4, 2), dtype=torch.float16, device=dev)
+    with pytest.raises(ValueError, match="head_dim"):
+        kvq.encode(pk, x, codes, scales)
+    q = torch.zeros((1, 4, 64), dtype=torch.float16, device=dev)
+    with pytest.raises(ValueError, match="head_dim"):
+        kvq.attend_decode(pk, pv, q, codes, scales, codes, scales, T_len=4)
+    with pytest.raises(ValueError, match="head_dim"):
+        kvq.attend_decode_batch([(pk, pv, q, codes, scales, codes, scales)], T_len=4)
+    with pytest.raises(ValueError, match="head_dim"):
+        kvq.attend_combine(pv, torch.zeros((2, 1, 4, 68), dtype=torch.float32, device=dev))
