@@ -52,8 +52,10 @@ Readings taken where the pages leave a step open:
     pack steps. Every function taking ``transform`` accepts "srft" (default)
     or "srht".
 
-Parity pins: every function here is checked in ``tests/test_oracle_pins.py``
-against closed forms, brute force and invariants (see that file).
+Parity pins: every function here is checked against closed forms, brute force and
+invariants in ``tests/test_oracle_pins.py`` (the SRFT path), ``tests/test_oracle_srht_pins.py``
+(the Hadamard variant) and ``tests/test_oracle_int8_pins.py`` (int8 codes), each with
+planted mistakes that the pins must reject.
 """
 from __future__ import annotations
 
