@@ -495,37 +495,32 @@ __device__ __forceinline__ void rotate_query_eo(const uint16_t* qs, int heads, c
 // Transpose of rotate_query_eo for the output (sign applied at the fp16 store):
 // Z_c = (dg / lambda)_c o_t[c] / L; (E', O') = combine^T(Z); x_even = F128^T E',
 // x_odd = F128^T O' on the tensor cores (ldmatrix.trans of the resident F128; E', O'
-// enter as fp16 hi + lo). eo: fp32 scratch [2][8][128]. All 160 threads call it.
+// enter as fp16 hi + lo). eo: fp32 scratch [2][8][128]. The NW warps' threads, and only
+// they, call it (it synchronises them on named barrier 1).
 template <int NW>
 __device__ __forceinline__ void unrotate_out_eo(const float* om, int heads, const float* Lh, const float* vch,
                                                 const uint8_t* srot, float* eo, float* xb, int warp, int lane,
                                                 bool hada) {
-  const int t = threadIdx.x;
+  // the prep is spread over the NW warps' threads, one (frequency, head) pair each
   if (hada) {
     // Hadamard (SRHT plans), the transpose of X[2k + b] = E_k + (-1)^b O_k:
     // E'_k = Z_2k + Z_2k+1, O'_k = Z_2k - Z_2k+1
-    if (t < 128) {
-      const int k = t;
-#pragma unroll
-      for (int h = 0; h < 8; ++h) {
-        float e = 0.0f, o = 0.0f;
-        if (h < heads) {
-          const float L = Lh[h];
-          const float r = L > 0.0f ? 1.0f / L : 0.0f;
-          const float z0 = om[h * 256 + 2 * k] * vch[2 * k] * r, z1 = om[h * 256 + 2 * k + 1] * vch[2 * k + 1] * r;
-          e = z0 + z1;
-          o = z0 - z1;
-        }
-        eo[h * 128 + k] = e;
-        eo[1024 + h * 128 + k] = o;
+    for (int it = threadIdx.x; it < 128 * 8; it += NW * 32) {
+      const int h = it >> 7, k = it & 127;
+      float e = 0.0f, o = 0.0f;
+      if (h < heads) {
+        const float L = Lh[h];
+        const float r = L > 0.0f ? 1.0f / L : 0.0f;
+        const float z0 = om[h * 256 + 2 * k] * vch[2 * k] * r, z1 = om[h * 256 + 2 * k + 1] * vch[2 * k + 1] * r;
+        e = z0 + z1;
+        o = z0 - z1;
       }
+      eo[h * 128 + k] = e;
+      eo[1024 + h * 128 + k] = o;
     }
-  } else if (t <= 64) {  // k = t
-    const int k = t;
-    float sn, cs;
-    sincospif((float)k / 128.0f, &sn, &cs);
-#pragma unroll
-    for (int h = 0; h < 8; ++h) {
+  } else {
+    for (int it = threadIdx.x; it < 65 * 8; it += NW * 32) {  // k = 0 .. 64
+      const int h = it / 65, k = it - 65 * h;
       float* E = eo + h * 128;
       float* O = eo + 1024 + h * 128;
       if (h >= heads) {
@@ -534,6 +529,8 @@ __device__ __forceinline__ void unrotate_out_eo(const float* om, int heads, cons
         else { E[2 * k] = E[2 * k + 1] = O[2 * k] = O[2 * k + 1] = 0.0f; }
         continue;
       }
+      float sn, cs;
+      sincospif((float)k / 128.0f, &sn, &cs);
       const float L = Lh[h];
       const float r = L > 0.0f ? 1.0f / L : 0.0f;
       const float* o = om + h * 256;
@@ -556,7 +553,7 @@ __device__ __forceinline__ void unrotate_out_eo(const float* om, int heads, cons
       }
     }
   }
-  __syncthreads();
+  consumer_sync<NW>();
   if (warp < NW) {
     const int g = lane >> 2, cq = lane & 3;
     const int mi = lane >> 3;
@@ -1450,21 +1447,29 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
       mrg[kHT + threadIdx.x] = 0.0f;
     }
     __syncthreads();
-    if (csize > 1 && threadIdx.x == 0)
-      for (int r = 1; r < csize; ++r) mbar_arrive_remote(mapa_shared(smem_u32(rdy), (uint32_t)r));
+    // The producer warp, idle from here on, tells the peers that their shared memory may
+    // go (lane r to peer r) and leaves; the consumer warps finish the CTA without waiting
+    // for those remote arrivals. Every load from the peers has returned its value (consumed
+    // before the barrier above), so the signal orders nothing and needs no release.
+    if (warp == kCWarps) {
+      if (lane >= 1 && lane < csize) mbar_arrive_remote_relaxed(mapa_shared(smem_u32(rdy), (uint32_t)lane));
+      return;
+    }
   }
+  // below: consumer warps only
+  constexpr int kCThreads = kCWarps * 32;
   float* wsm = reinterpret_cast<float*>(qf);       // [n][8] weights (workspace merge scratch)
   float* lsm = wsm + kMaxMerge * kHT;              // [n][8]
   float* xb = wst;                                 // [8][D] un-rotated output (fp32), over the dead warp partials
   // merge n partials (pointer of partial r from `at`) into (mrg, om) -- om unnormalised, relative to M
   auto merge = [&](int n, auto at) {
-    for (int i = threadIdx.x; i < n * kHT; i += kThreads) {
+    for (int i = threadIdx.x; i < n * kHT; i += kCThreads) {
       const int r = i / kHT, h = i - r * kHT;
       const float* pr = at(r);
       wsm[i] = __ldcg(pr + h);
       lsm[i] = __ldcg(pr + kHT + h);
     }
-    __syncthreads();
+    consumer_sync<kCWarps>();
     if (threadIdx.x < kHT) {
       const int h = threadIdx.x;
       float M = -INFINITY;
@@ -1479,8 +1484,8 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
       mrg[h] = M;
       mrg[kHT + h] = L;
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < heads * D / 4; i += kThreads) {
+    consumer_sync<kCWarps>();
+    for (int i = threadIdx.x; i < heads * D / 4; i += kCThreads) {
       const int h = (4 * i) / D;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       // eight partials' loads in flight at a time (one L2 round trip per eight)
@@ -1502,22 +1507,19 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
       }
       reinterpret_cast<float4*>(om)[i] = acc;
     }
-    __syncthreads();
+    consumer_sync<kCWarps>();
   };
-  // the producer warp reads staged constants below: observe their barrier too
-  if (warp == kCWarps && !mbar_wait_bounded(cbar, 0)) atomicOr(&g_attend_err, kErrTimeoutLoad);
-
   // ------------------------------------------------------------ more than one cluster per unit: global merge
   const int ncl = p.S / csize;
   if (ncl > 1) {
     const int cl = split / csize;
     float* gpart = p.part + ((size_t)unit * ncl + cl) * PART;
-    for (int i = threadIdx.x; i < kHT * 2; i += kThreads) __stcg(gpart + i, mrg[i]);
-    for (int i = threadIdx.x; i < heads * D / 4; i += kThreads)
+    for (int i = threadIdx.x; i < kHT * 2; i += kCThreads) __stcg(gpart + i, mrg[i]);
+    for (int i = threadIdx.x; i < heads * D / 4; i += kCThreads)
       __stcg(reinterpret_cast<float4*>(gpart + 2 * kHT) + i, reinterpret_cast<const float4*>(om)[i]);
     // bar.sync orders every thread's stores before thread 0's device-scope fence and
     // counter increment; the last leader fences again before reading the others' partials.
-    __syncthreads();
+    consumer_sync<kCWarps>();
     if (threadIdx.x == 0) {
       __threadfence();
       const int prev = atomicAdd(p.cnt + unit, 1);
@@ -1525,7 +1527,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
       if (last) __threadfence();
       *flag = last;
     }
-    __syncthreads();
+    consumer_sync<kCWarps>();
     if (*flag == 0) return;
     if (threadIdx.x == 0) p.cnt[unit] = 0;  // leave the counter at zero for the next call
     const float* gbase = p.part + (size_t)unit * ncl * PART;
@@ -1536,7 +1538,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
   if (INT4 && p.part_out) {
     // sequence-sharded decode: the unit's softmax partial, rotated domain, unnormalised
     float* pb = p.part_out + ((size_t)b * p.Hq + hq0) * (D + 4);
-    for (int i = threadIdx.x; i < heads * (D + 4); i += kThreads) {
+    for (int i = threadIdx.x; i < heads * (D + 4); i += kCThreads) {
       const int h = i / (D + 4), e = i - h * (D + 4);
       pb[i] = e == 0 ? mrg[h] : (e == 1 ? mrg[kHT + h] : (e < 4 ? 0.0f : om[h * D + e - 4]));
     }
@@ -1549,13 +1551,13 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
     } else {
       unrotate_out_eo<kCWarps>(om, heads, mrg + kHT, vch, srot, reinterpret_cast<float*>(qf), xb, warp, lane, hada);
     }
-    __syncthreads();
-    for (int i = threadIdx.x; i < heads * D / 2; i += kThreads) {
+    consumer_sync<kCWarps>();
+    for (int i = threadIdx.x; i < heads * D / 2; i += kCThreads) {
       const int j = i % (D / 2);
       reinterpret_cast<uint32_t*>(ob)[i] = pack_half2(xb[2 * i], xb[2 * i + 1]) ^ vsg[j];
     }
   } else {
-    for (int i = threadIdx.x; i < heads * D / 2; i += kThreads) {
+    for (int i = threadIdx.x; i < heads * D / 2; i += kCThreads) {
       const float L = mrg[kHT + (2 * i) / D];
       const float r = L > 0.0f ? 1.0f / L : 0.0f;
       reinterpret_cast<uint32_t*>(ob)[i] = pack_half2(om[2 * i] * r, om[2 * i + 1] * r);
