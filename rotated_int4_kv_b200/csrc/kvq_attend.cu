@@ -225,6 +225,13 @@ __device__ __forceinline__ void consumer_sync() { asm volatile("bar.sync 1, %0;"
 
 __device__ __forceinline__ float fast_exp2(float x) { return ex2_approx(x); }
 
+// A remote mbarrier arrival without release semantics: for a signal that orders no
+// memory operation of the arriving CTA ("your shared memory may go", sent after every
+// load from it has returned its value).
+__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
 // split an fp32 into fp16 hi + lo (hi = rn(x), lo = rn(x - hi))
 __device__ __forceinline__ void split_h(float x, __half& hi, __half& lo) {
   hi = __float2half_rn(x);

@@ -97,12 +97,6 @@ __device__ __forceinline__ uint32_t mapa_shared(uint32_t smem_addr, uint32_t ran
 __device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
-// The same arrival without release semantics: for a signal that orders no memory
-// operation of the arriving CTA (e.g. "your shared memory may go", sent after every
-// load from it has returned its value).
-__device__ __forceinline__ void mbar_arrive_remote_relaxed(uint32_t cluster_addr) {
-  asm volatile("mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
-}
 
 // Wait on a local mbarrier whose phase another CTA of the cluster completes (acquire
 // at cluster scope); bounded like mbar_wait_bounded.
