@@ -1413,34 +1413,49 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
   float* om = qt;                                  // merged o_t [8][D] (fp32)
   {
     const uint32_t cbase = smem_u32(cpart);
-    for (int i = threadIdx.x; i < heads * D / 4; i += kThreads) {
+    // two float4 items per thread and round (8 heads x D / 4 items may exceed the block),
+    // all their loads issued before any is used: one distributed-shared-memory round trip
+    // per round
+    constexpr int kItems = kHT * D / 4;
+    constexpr int kPer = kItems > kThreads ? 2 : 1;
+    const int nitems = heads * D / 4;
+    for (int base = 0; base < nitems; base += kPer * kThreads) {
+    float mr[kPer][kMaxCluster], lr[kPer][kMaxCluster];
+    float4 vr[kPer][kMaxCluster];
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = base + threadIdx.x + u * kThreads;
       const int h = (4 * i) / D;
-      float mr[kMaxCluster], lr[kMaxCluster];
-      float4 vr[kMaxCluster];
 #pragma unroll
       for (int r = 0; r < kMaxCluster; ++r) {
-        if (r < csize) {
+        if (r < csize && i < nitems) {
           const uint32_t a = mapa_shared(cbase, (uint32_t)r);
-          mr[r] = ld_dsmem_f32(a + 4 * h);
-          lr[r] = ld_dsmem_f32(a + 4 * (kHT + h));
-          vr[r] = ld_dsmem_f32x4(a + 4 * (2 * kHT) + 16 * i);
+          mr[u][r] = ld_dsmem_f32(a + 4 * h);
+          lr[u][r] = ld_dsmem_f32(a + 4 * (kHT + h));
+          vr[u][r] = ld_dsmem_f32x4(a + 4 * (2 * kHT) + 16 * i);
         }
       }
+    }
+#pragma unroll
+    for (int u = 0; u < kPer; ++u) {
+      const int i = base + threadIdx.x + u * kThreads;
+      if (i >= nitems) continue;
+      const int h = (4 * i) / D;
       float M = -INFINITY;
 #pragma unroll
       for (int r = 0; r < kMaxCluster; ++r)
-        if (r < csize) M = fmaxf(M, mr[r]);
+        if (r < csize) M = fmaxf(M, mr[u][r]);
       float L = 0.0f;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
       for (int r = 0; r < kMaxCluster; ++r) {
         if (r < csize) {
-          const float w = (M == -INFINITY || mr[r] == -INFINITY) ? 0.0f : fast_exp2(mr[r] - M);
-          L = fmaf(w, lr[r], L);
-          acc.x = fmaf(w, vr[r].x, acc.x);
-          acc.y = fmaf(w, vr[r].y, acc.y);
-          acc.z = fmaf(w, vr[r].z, acc.z);
-          acc.w = fmaf(w, vr[r].w, acc.w);
+          const float w = (M == -INFINITY || mr[u][r] == -INFINITY) ? 0.0f : fast_exp2(mr[u][r] - M);
+          L = fmaf(w, lr[u][r], L);
+          acc.x = fmaf(w, vr[u][r].x, acc.x);
+          acc.y = fmaf(w, vr[u][r].y, acc.y);
+          acc.z = fmaf(w, vr[u][r].z, acc.z);
+          acc.w = fmaf(w, vr[u][r].w, acc.w);
         }
       }
       reinterpret_cast<float4*>(om)[i] = acc;
@@ -1448,6 +1463,7 @@ __global__ void __launch_bounds__((Cfg<D, INT4, G, BITS>::kThreads), (Cfg<D, INT
         mrg[h] = M;
         mrg[kHT + h] = L;
       }
+    }
     }
     if (threadIdx.x >= heads && threadIdx.x < kHT) {  // head rows past the group: empty
       mrg[threadIdx.x] = -INFINITY;
