@@ -62,7 +62,7 @@ NCU_TRAFFIC = {
     # kernel -> (source digest at capture time, bytes per launch)
     "encode": ("e66cb71d3607", 112104533),       # register-FFT encode, Gemma step (52 jobs)
     "encode_tc": ("ba92cae89f03", 124381952),    # tensor-core encode, Gemma step (52 jobs)
-    "attend": ("304d3f084c13", 32594944),        # grouped int4 attention, Gemma step (26 jobs)
+    "attend": ("fe582db1b810", 32586240),        # grouped int4 attention, Gemma step (26 jobs)
 }
 
 
