@@ -95,6 +95,20 @@ def _ncu_traffic(kind: str):
     return rec[1] if rec is not None and rec[0] == _source_digest(kind) else None
 
 
+# DRAM traffic per launch of the int4 attention kernel at the attention arms' shapes
+# (one ncu capture each, keyed like NCU_TRAFFIC by the kernel sources' digest)
+NCU_TRAFFIC_ATTN = {
+    # arm -> (source digest at capture time, bytes per launch)
+}
+
+
+def _ncu_traffic_attn(arm: str):
+    if TRANSFORM != "srft" or BITS != 4:
+        return None
+    rec = NCU_TRAFFIC_ATTN.get(arm)
+    return rec[1] if rec is not None and rec[0] == _source_digest("attend") else None
+
+
 def _algo_bytes(D: int, G: int = 32, bits: int = 4):
     vec = 2 * D + D * bits // 8 + 2 * (D // G)   # encode: fp16 in + codes + scales out
     tok = 2 * (D * bits // 8 + 2 * (D // G))     # quantised attention: K and V codes + scales per token x kv head
@@ -223,7 +237,8 @@ def cpu_baseline(wl, budget_s: float = 10.0, single_budget_s: float = 5.0):
         single = {"value": v1, "cores": 1, "sample": f"{n1} layers, {s1:.1f} s"}
     except ImportError:
         pass
-    return {"value": value, "unit": "Mvec/s", "cores": _blas_threads(), "kind": "oracle",
+    return {"value": value, "unit": "Mvec/s", "cores": _blas_threads(), "os_cpu_count": os.cpu_count(),
+            "kind": "oracle",
             "sample": f"{n} x one layer of the step (K+V encode of {2 * wl.h_kv * wl.contexts[0]} vectors, D="
                       f"{wl.head_dim}, plus the 1-token int{BITS} attention over {wl.contexts[0]} tokens), "
                       f"{secs:.1f} s of host time",
@@ -248,9 +263,12 @@ def run_reference(args, rank: int, world: int):
     line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "Mvec/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * secs / max(1, args.steps),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": _config(wl),
-            "cpu_baseline": {"value": val, "unit": "Mvec/s", "cores": _blas_threads(), "kind": "oracle",
-                             "sample": sample},
+            "config": dict(_config(wl), encode_path=args.encode_path),
+            "step_sample": {"layers_per_timed_step": 1, "layers_per_gpu_step": wl.layers,
+                            "note": "each timed step of this arm is one layer of the workload on the host; "
+                                    "value (Mvec/s) is per vector and so comparable, ms_per_step is not"},
+            "cpu_baseline": {"value": val, "unit": "Mvec/s", "cores": _blas_threads(),
+                             "os_cpu_count": os.cpu_count(), "kind": "oracle", "sample": sample},
             "e2e": {"value": val, "unit": "Mvec/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -423,6 +441,25 @@ def run_kvq(args, rank: int, world: int):
     del dec_out
     assert kvq.poll_device_errors() == 0
 
+    # ---- the attention half of the metric at bandwidth-bound and latency-bound shapes:
+    # int4 against the fp16 comparator on identical shapes (decode_case), each a CUDA
+    # graph of back-to-back calls; the big caches (604 MB int4 / 2.15 GB fp16) exceed L2
+    attn_arms = None
+    if not args.skip_attention_arms:
+        attn_arms = {}
+        for key, wname, T, layers, distinct, variants in (
+                ("mistral_32k", "mistral", 32768, 4, 1, False),
+                ("longctx_128k", "longctx", 131072, 4, 1, False),
+                ("qwen_1k_step", "qwen", 1024, 28, 4, True),
+                ("qwen_4k_step", "qwen", 4096, 28, 4, True)):
+            case = decode_case(kvq, torch, kvgen.WORKLOADS[wname], T, layers, distinct, args.steps, args.warmup,
+                               seed, dev, step_variants=variants)
+            for f in ("int4_attn_ms", "fp16_attn_ms"):
+                case[f] = max_over_ranks([case[f]], dist, dev)[0]
+            case["attn_speedup"] = case["fp16_attn_ms"] / case["int4_attn_ms"]
+            case["int4_traffic_bytes_per_launch"] = _ncu_traffic_attn(key)
+            attn_arms[key] = case
+
     vec_step = NJ * Hkv * T
     value = job_throughput(world, vec_step, ms, args.steps)
     hbm, peak_kind = _peaks()
@@ -480,6 +517,7 @@ def run_kvq(args, rank: int, world: int):
                        "GB_s": vec_step * vec_b / (ms_dec * 1e-3) / 1e9,
                        "frac_hbm": vec_step * vec_b / (ms_dec * 1e-3) / 1e9 / hbm, "bytes_per_vec": vec_b,
                        "note": "one launch over the 52 caches of the step; input may be L2-resident"},
+            "attention_arms": attn_arms,
             "cpu_baseline": cpu,
             "e2e": {"value": world * vec_step / (e2e_ms * 1e-3) / 1e6, "unit": "Mvec/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
@@ -520,11 +558,113 @@ def _graph_time(torch, fn, steps, warmup):
     return a.elapsed_time(b) / steps
 
 
+def decode_case(kvq, torch, wl, T, layers, distinct, steps, warmup, seed, dev, batch=None, step_variants=True):
+    """One context length of a decode-step workload: int4 against the fp16 comparator.
+
+    Per layer (a CUDA graph of `layers` layers cycling over `distinct` caches): the int4
+    step is one fused launch (kvq_attend_decode_append: the new token's K/V encoded at T,
+    attention over T + 1); the two-launch int4 step (encode, then attention) beside it;
+    the fp16 step is two one-token append copies + the fp16 attention kernel. Attention
+    alone is timed for both caches. With step_variants=False only the two attention-alone
+    graphs run (bandwidth-bound shapes, where the append is noise)."""
+    D, Hkv, Hq, G = wl.head_dim, wl.h_kv, wl.h_q, wl.group
+    B = wl.batch if batch is None else batch
+    vec_b, tok_b = _algo_bytes(D, G, BITS)
+    hbm, _ = _peaks()
+    T_cap = T + 2
+    plans, caches, k16s, v16s = [], [], [], []
+    for l in range(distinct):
+        pk = kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=l, kind="k"), transform=TRANSFORM, bits=BITS)
+        pv = kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=l, kind="v"), transform=TRANSFORM, bits=BITS)
+        plans.append((pk, pv))
+        c = {}
+        for kind, pl in (("k", pk), ("v", pv)):
+            codes = torch.zeros((B, Hkv, T_cap, D * BITS // 8), dtype=torch.uint8, device=dev)
+            scales = torch.zeros((B, Hkv, T_cap, D // G), dtype=torch.float16, device=dev)
+            x16 = torch.zeros((B, Hkv, T_cap, D), dtype=torch.float16, device=dev)
+            for b in range(B):
+                kvgen.kv_torch(wl, kind, (1, Hkv, T, D), dev, seed=seed, layer=l, salt=b, out=x16[b:b + 1, :, :T])
+                kvq.encode(pl, x16[b:b + 1, :, :T].contiguous(), codes[b:b + 1], scales[b:b + 1], 0)
+            c[kind] = (codes, scales)
+            (k16s if kind == "k" else v16s).append(x16)
+        caches.append(c)
+    q = [kvgen.q_torch((B, Hq, D), dev, seed=seed, layer=l) for l in range(distinct)]
+    newk = [kvgen.kv_torch(wl, "k", (B, Hkv, 1, D), dev, seed=seed, layer=l, salt=99) for l in range(distinct)]
+    newv = [kvgen.kv_torch(wl, "v", (B, Hkv, 1, D), dev, seed=seed, layer=l, salt=98) for l in range(distinct)]
+    out = torch.empty((B, Hq, D), dtype=torch.float16, device=dev)
+    ws = [kvq.make_workspace(B, Hq, Hkv, D, T_cap, dev) for _ in range(distinct)]
+
+    def step_int4():
+        # one launch per layer: the new token's K/V encoded at T and attention over T + 1
+        for l in range(layers):
+            d = l % distinct
+            pk, pv = plans[d]
+            kc, ks = caches[d]["k"]
+            vc, vs = caches[d]["v"]
+            kvq.attend_decode_append(pk, pv, q[d], newk[d], newv[d], kc, ks, vc, vs, T, out=out, workspace=ws[d])
+
+    def step_int4_two_launches():
+        for l in range(layers):
+            d = l % distinct
+            pk, pv = plans[d]
+            kc, ks = caches[d]["k"]
+            vc, vs = caches[d]["v"]
+            kvq.encode_batch([(pk, newk[d], kc, ks, T), (pv, newv[d], vc, vs, T)])
+            kvq.attend_decode(pk, pv, q[d], kc, ks, vc, vs, T_len=T + 1, out=out, workspace=ws[d])
+
+    def step_fp16():
+        for l in range(layers):
+            d = l % distinct
+            k16s[d][:, :, T:T + 1].copy_(newk[d])
+            v16s[d][:, :, T:T + 1].copy_(newv[d])
+            kvq.attend_decode_ref(q[d], k16s[d], v16s[d], T_len=T + 1, out=out, workspace=ws[d])
+
+    def attn_only_int4():
+        for l in range(layers):
+            d = l % distinct
+            pk, pv = plans[d]
+            kvq.attend_decode(pk, pv, q[d], *caches[d]["k"], *caches[d]["v"], T_len=T + 1, out=out,
+                              workspace=ws[d])
+
+    def attn_only_fp16():
+        for l in range(layers):
+            d = l % distinct
+            kvq.attend_decode_ref(q[d], k16s[d], v16s[d], T_len=T + 1, out=out, workspace=ws[d])
+
+    a4 = _graph_time(torch, attn_only_int4, steps, warmup)
+    a16 = _graph_time(torch, attn_only_fp16, steps, warmup)
+    tokheads = layers * B * Hkv * (T + 1)
+    S, C, _ = kvq.attend_split_info(B, Hq, Hkv, D, T + 1, G, BITS)
+    case = {
+        "T": T, "batch": B, "kv_heads": Hkv, "q_heads": Hq, "head_dim": D, "layers": layers,
+        "distinct_layer_caches": distinct,
+        "int4_attn_ms": a4, "fp16_attn_ms": a16, "attn_speedup": a16 / a4,
+        "int4_us_per_layer": 1e3 * a4 / layers, "fp16_us_per_layer": 1e3 * a16 / layers,
+        "int4_tokens_heads_per_s": tokheads / (a4 * 1e-3),
+        "int4_attn_GB_s": tokheads * tok_b / (a4 * 1e-3) / 1e9,
+        "int4_frac_hbm": tokheads * tok_b / (a4 * 1e-3) / 1e9 / hbm,
+        "fp16_attn_GB_s": tokheads * 4 * D / (a16 * 1e-3) / 1e9,
+        "fp16_frac_hbm": tokheads * 4 * D / (a16 * 1e-3) / 1e9 / hbm,
+        "bytes_per_token_head": tok_b, "int4_split": {"splits": S, "cluster": C},
+        "l2": ("working set > L2 (HBM-bound)" if distinct * B * Hkv * T * tok_b > 126e6
+               else "working set fits in L2: latency of an L2-warm decode loop"),
+    }
+    if step_variants:
+        ms4 = _graph_time(torch, step_int4, steps, warmup)
+        ms4_2 = _graph_time(torch, step_int4_two_launches, steps, warmup)
+        ms16 = _graph_time(torch, step_fp16, steps, warmup)
+        case.update({"int4_step_ms": ms4, "int4_step_two_launch_ms": ms4_2, "fp16_step_ms": ms16,
+                     "step_speedup": ms16 / ms4, "int4_step_us_per_layer": 1e3 * ms4 / layers,
+                     "fp16_step_us_per_layer": 1e3 * ms16 / layers})
+    assert kvq.poll_device_errors() == 0
+    del caches, k16s, v16s, plans, ws
+    torch.cuda.empty_cache()
+    return case
+
+
 def run_decode_workload(args, rank: int, world: int):
     """Decode-step workloads: per layer, append one token of K and V to the cache and run
-    one-query decode attention over it, int4 against the fp16 comparator. int4 step = one
-    fused launch (kvq_attend_decode_append; the two-launch step, encode then attention,
-    is reported beside it); fp16 step = one-token K/V append copies + fp16 attention.
+    one-query decode attention over it, int4 against the fp16 comparator (decode_case).
     Steps are CUDA graphs."""
     import torch
 
@@ -536,96 +676,11 @@ def run_decode_workload(args, rank: int, world: int):
     wl = kvgen.WORKLOADS[args.workload]
     D, Hkv, Hq, B, G = wl.head_dim, wl.h_kv, wl.h_q, wl.batch, wl.group
     seed = kvgen.DEFAULT_SEED + 1000 * rank
-    hbm, _ = _peaks()
     vec_b, tok_b = _algo_bytes(D, G, BITS)
     contexts = wl.contexts if args.contexts is None else tuple(int(c) for c in args.contexts.split(","))
     layers = wl.layers if args.layers is None else args.layers
     distinct = min(layers, max(1, args.distinct_layers))
-    cases = []
-    for T in contexts:
-        T_cap = T + 2
-        plans, caches, caches16 = [], [], []
-        for l in range(distinct):
-            pk = kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=l, kind="k"), transform=TRANSFORM, bits=BITS)
-            pv = kvq.Plan(*kvgen.plan_params(D, seed=seed, layer=l, kind="v"), transform=TRANSFORM, bits=BITS)
-            plans.append((pk, pv))
-            c = {}
-            for kind, pl in (("k", pk), ("v", pv)):
-                codes = torch.zeros((B, Hkv, T_cap, D * BITS // 8), dtype=torch.uint8, device=dev)
-                scales = torch.zeros((B, Hkv, T_cap, D // G), dtype=torch.float16, device=dev)
-                x16 = torch.zeros((B, Hkv, T_cap, D), dtype=torch.float16, device=dev)
-                for b in range(B):
-                    kvgen.kv_torch(wl, kind, (1, Hkv, T, D), dev, seed=seed, layer=l, salt=b, out=x16[b:b + 1, :, :T])
-                    kvq.encode(pl, x16[b:b + 1, :, :T].contiguous(), codes[b:b + 1], scales[b:b + 1], 0)
-                c[kind] = (codes, scales)
-                caches16.append(x16) if kind == "k" else caches16.append(x16)
-            caches.append(c)
-        k16s = caches16[0::2]
-        v16s = caches16[1::2]
-        q = [kvgen.q_torch((B, Hq, D), dev, seed=seed, layer=l) for l in range(distinct)]
-        newk = [kvgen.kv_torch(wl, "k", (B, Hkv, 1, D), dev, seed=seed, layer=l, salt=99) for l in range(distinct)]
-        newv = [kvgen.kv_torch(wl, "v", (B, Hkv, 1, D), dev, seed=seed, layer=l, salt=98) for l in range(distinct)]
-        out = torch.empty((B, Hq, D), dtype=torch.float16, device=dev)
-        ws = [kvq.make_workspace(B, Hq, Hkv, D, T_cap, dev) for _ in range(distinct)]
-
-        def step_int4():
-            # one launch per layer: the new token's K/V encoded at T and attention over T + 1
-            for l in range(layers):
-                d = l % distinct
-                pk, pv = plans[d]
-                kc, ks = caches[d]["k"]
-                vc, vs = caches[d]["v"]
-                kvq.attend_decode_append(pk, pv, q[d], newk[d], newv[d], kc, ks, vc, vs, T, out=out, workspace=ws[d])
-
-        def step_int4_two_launches():
-            for l in range(layers):
-                d = l % distinct
-                pk, pv = plans[d]
-                kc, ks = caches[d]["k"]
-                vc, vs = caches[d]["v"]
-                kvq.encode_batch([(pk, newk[d], kc, ks, T), (pv, newv[d], vc, vs, T)])
-                kvq.attend_decode(pk, pv, q[d], kc, ks, vc, vs, T_len=T + 1, out=out, workspace=ws[d])
-
-        def step_fp16():
-            for l in range(layers):
-                d = l % distinct
-                k16s[d][:, :, T:T + 1].copy_(newk[d])
-                v16s[d][:, :, T:T + 1].copy_(newv[d])
-                kvq.attend_decode_ref(q[d], k16s[d], v16s[d], T_len=T + 1, out=out, workspace=ws[d])
-
-        def attn_only_int4():
-            for l in range(layers):
-                d = l % distinct
-                pk, pv = plans[d]
-                kvq.attend_decode(pk, pv, q[d], *caches[d]["k"], *caches[d]["v"], T_len=T + 1, out=out,
-                                  workspace=ws[d])
-
-        def attn_only_fp16():
-            for l in range(layers):
-                d = l % distinct
-                kvq.attend_decode_ref(q[d], k16s[d], v16s[d], T_len=T + 1, out=out, workspace=ws[d])
-
-        ms4 = _graph_time(torch, step_int4, args.steps, args.warmup)
-        ms4_2 = _graph_time(torch, step_int4_two_launches, args.steps, args.warmup)
-        ms16 = _graph_time(torch, step_fp16, args.steps, args.warmup)
-        a4 = _graph_time(torch, attn_only_int4, args.steps, args.warmup)
-        a16 = _graph_time(torch, attn_only_fp16, args.steps, args.warmup)
-        assert kvq.poll_device_errors() == 0
-        tokheads = layers * B * Hkv * (T + 1)
-        cases.append({
-            "T": T, "layers": layers, "distinct_layer_caches": distinct,
-            "int4_step_ms": ms4, "int4_step_two_launch_ms": ms4_2, "fp16_step_ms": ms16, "step_speedup": ms16 / ms4,
-            "int4_attn_ms": a4, "fp16_attn_ms": a16, "attn_speedup": a16 / a4,
-            "int4_tokens_heads_per_s": tokheads / (a4 * 1e-3),
-            "int4_attn_GB_s": tokheads * tok_b / (a4 * 1e-3) / 1e9,
-            "int4_frac_hbm": tokheads * tok_b / (a4 * 1e-3) / 1e9 / hbm,
-            "fp16_attn_GB_s": tokheads * 4 * D / (a16 * 1e-3) / 1e9,
-            "fp16_frac_hbm": tokheads * 4 * D / (a16 * 1e-3) / 1e9 / hbm,
-            "l2": ("working set > L2 (HBM-bound)" if distinct * B * Hkv * T * tok_b > 126e6
-                   else "working set fits in L2: latency of an L2-warm decode loop"),
-        })
-        del caches, caches16, k16s, v16s
-        torch.cuda.empty_cache()
+    cases = [decode_case(kvq, torch, wl, T, layers, distinct, args.steps, args.warmup, seed, dev) for T in contexts]
     stream_enc = None
     sb = wl.extra.get("stream_batch") if wl.extra else None
     if sb:
@@ -683,6 +738,8 @@ def main(argv=None):
                     help="the plans' rotation: srft (the pages' method) or srht (the Hadamard variant)")
     ap.add_argument("--bits", type=int, default=4, choices=[4, 8],
                     help="code width of the plans: 4 (the pages' int4, default) or 8 (int8 codes)")
+    ap.add_argument("--skip-attention-arms", action="store_true",
+                    help="default workload: leave out the int4-vs-fp16 attention arms (Mistral 32K, 128K, Qwen step)")
     ap.add_argument("--encode-path", default="auto", choices=["auto", "fft", "tensor"],
                     help="encode kernel of the prefill step: tensor cores where supported (auto), "
                          "the register FFT, or tensor cores only")

@@ -3,13 +3,16 @@
  *
  * The method is the fused KV-cache compression of "When Quantization Is Free:
  * An int4 KV Cache That Outruns fp16 on Apple Silicon" (arXiv 2605.05699):
- *   [ABS] paperdance.org/p/2605.05699, abstract: sign-randomised FFT + per-channel
- *         lambda + per-group abs-max + int4 nibble pack, in one fused kernel.
- *   [M1]  gist.science/de/paper/2605.05699, "Methodik" 1: SRFT(x) = pack(F . diag(s) . x),
- *         F the unitary DFT, s a fixed random +/-1 vector.
- *   [M2]  same page, "Methodik" 2: load + sign, FFT passes, Hermitian unpack to a real
- *         representation, per-channel lambda, per-group abs-max, signed int4
- *         rounding, two codes per byte.
+ *   [ABS] paperdance.org/p/2605.05699, English abstract: one fused kernel does the whole
+ *         encode -- a random-sign FFT, one factor per channel, one absolute-maximum
+ *         scale per channel group, and two 4-bit codes packed into each byte.
+ *   [M1]  gist.science/de/paper/2605.05699, "Methodik" 1: the rotation is the unitary
+ *         DFT F applied after a fixed random +/-1 sign vector s, the complex result
+ *         packed to real values.
+ *   [M2]  same page, "Methodik" 2: the kernel's steps in order -- signs applied on
+ *         load, the FFT butterflies, the Hermitian-symmetric spectrum unpacked to real
+ *         values, the per-channel factor, the group abs-max and rounding to signed
+ *         4-bit (or 8-bit) integers, and nibble packing.
  * The read path (decode, decode attention on the packed cache) is not on the
  * pages; it is the inverse transform and softmax attention taken in the rotated
  * domain, valid because F is unitary (<q, R^T y> = <R q, y>).
@@ -228,8 +231,9 @@ kvq_status kvq_attend_decode(const kvq_plan* pk, const kvq_plan* pv, const uint1
  * kvq_encode with n = 1 at `pos` stores, up to fp32 rounding of the transform: a
  * code may differ only where the pre-rounding value lies at a rounding boundary),
  * and the query attends over tokens 0 .. pos, the new one included, as
- * kvq_attend_decode with T_len = pos + 1 (the SURVEY's "fused append"; the pages
- * encode each new token with the same fused kernel as a prefill, [M2]).
+ * kvq_attend_decode with T_len = pos + 1. The new token's encode is folded into the
+ * attention launch; the pages run the same fused encode for a decoded token as for a
+ * prefill, [M2].
  *   k_new, v_new   fp16 [B, Hkv, D], the new token's rows (original domain).
  *   k_codes, k_scales, v_codes, v_scales   the caches as in kvq_attend_decode,
  *              written at token pos (every (b, kv head)), read at tokens < pos.
@@ -342,6 +346,37 @@ kvq_status kvq_attend_decode_ref(const uint16_t* q, const uint16_t* k, const uin
                                  int Hq, int Hkv, int head_dim, int T_cap,
                                  const int32_t* seq_lens, int T_len, float softmax_scale,
                                  uint16_t* out, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * kvq_attend_split_info -- the sequence split the attention entry points choose for
+ * these shapes on the current device (not on the pages; a planning query, e.g. to
+ * size buffers or to check which merge path a call takes). One unit is one (batch
+ * entry, kv head, tile of up to 8 query heads); its tokens are cut into *splits
+ * contiguous ranges, one CTA each; groups of *cluster CTAs merge their softmax
+ * partials through distributed shared memory, and a unit with *splits / *cluster > 1
+ * also merges its cluster partials through the workspace.
+ *   B, Hq, Hkv, head_dim   as in kvq_attend_decode (one problem, not a batch of jobs).
+ *   group, bits   the plans' group (32 or 16) and code width (4 or 8); bits = 16 asks
+ *                 for kvq_attend_decode_ref's fp16 kernel (group ignored).
+ *   T             the token count the split is chosen from: T_cap when seq_lens is
+ *                 passed, else T_len (kvq_attend_decode_append: pos; _partial:
+ *                 t_end - t_begin).
+ *   splits, cluster, head_tiles   host outputs; any may be NULL.
+ * Errors: INVALID_ARG, UNSUPPORTED, DEVICE (no sm_100 device current).
+ */
+kvq_status kvq_attend_split_info(int B, int Hq, int Hkv, int head_dim, int group, int bits, int T,
+                                 int* splits, int* cluster, int* head_tiles);
+
+/*
+ * kvq_debug_wait_timeout -- a self-test of the kernels' failure path (not on the
+ * pages): launches one CTA on `stream` that waits, through the same bounded wait the
+ * kernels use, on an mbarrier that nothing will complete, with a budget of limit_us
+ * microseconds (1 .. 1e6) instead of 1 s. When the budget runs out the CTA raises
+ * flag 1 (the flag of a TMA load that never arrived) and exits; the context stays
+ * usable. kvq_poll_device_errors then reports the flag. Errors: INVALID_ARG, DEVICE,
+ * CUDA.
+ */
+kvq_status kvq_debug_wait_timeout(uint32_t limit_us, void* stream);
 
 /*
  * kvq_poll_device_errors -- synchronises the current device, then returns (in

@@ -10,11 +10,13 @@ Sources, cited by page and section (the pages are web renderings of the paper
 "When Quantization Is Free: An int4 KV Cache That Outruns fp16 on Apple
 Silicon", arXiv 2605.05699):
 
-  [ABS]  paperdance.org/p/2605.05699 -- the English abstract: the fused kernel is
-         "sign-randomized FFT + per-channel lambda + per-group abs-max + int4
-         nibble pack"; 3x persistent compression.
-  [M1]   gist.science/de/paper/2605.05699, "Methodik" 1 (SRFT): SRFT(x) =
-         pack(F . diag(s) . x), F the unitary DFT, s a fixed random sign vector.
+  [ABS]  paperdance.org/p/2605.05699 -- the English abstract: one fused kernel
+         applies a random-sign FFT, a factor per channel and an absolute-maximum
+         scale per channel group, and packs two 4-bit codes per byte; the cache
+         stays about 3x smaller than fp16.
+  [M1]   gist.science/de/paper/2605.05699, "Methodik" 1 (SRFT): the unitary DFT F
+         applied after a fixed random +-1 sign vector s, its complex output packed
+         to real values.
   [M2]   same page, "Methodik" 2 (fused kernel), its five steps: load and sign
          multiply; FFT passes; Hermitian unpack into a real representation;
          per-channel lambda, per-group abs-max reduction and rounding to signed
@@ -37,7 +39,7 @@ Readings taken where the pages leave a step open:
     codes. Two's-complement nibbles, even element in the low nibble.
   * int8 codes ([M2] names "signed int4/int8" as the rounding target and
     defines int8 no further): the same steps with 127 in place of 7 (scale =
-    fp16_rne(min(absmax/127, 65504)), codes clamped to [-127, 127], -128 never
+    fp16 round-to-nearest-even of min(absmax/127, 65504), codes clamped to [-127, 127], -128 never
     produced), one two's-complement byte per code, channel i at byte i. Every
     function taking ``bits`` accepts 4 (default) or 8.
   * Decode: x_hat = diag(s) F_r^T (c * scale / lambda).
@@ -152,13 +154,8 @@ def srft_inverse(y: np.ndarray, signs: np.ndarray, lam: np.ndarray, transform: s
 # The quantiser [M2], [M3]
 # ---------------------------------------------------------------------------
 
-def fp16_rne(v) -> np.ndarray:
-    """Round fp64 values to the nearest fp16 (ties to even); returned as fp64."""
-    return np.asarray(v, dtype=np.float64).astype(np.float16).astype(np.float64)
-
-
 def group_scales(y: np.ndarray, G: int, bits: int = 4) -> np.ndarray:
-    """Per-group abs-max scale: fp16_rne(min(absmax/qmax, 65504)); fp16 array [..., D/G]."""
+    """Per-group abs-max scale: min(absmax/qmax, 65504) rounded to fp16 (ties to even); fp16 array [..., D/G]."""
     y = np.asarray(y, dtype=np.float64)
     D = y.shape[-1]
     if D % G:
@@ -247,19 +244,6 @@ def compressed_bytes_per_vector(D: int, G: int, bits: int = 4) -> int:
     """D*bits/8 bytes of codes plus one fp16 scale per group [RES]."""
     qmax(bits)
     return D * bits // 8 + 2 * (D // G)
-
-
-# ---------------------------------------------------------------------------
-# Cache helpers: the [B, H, T_cap, ...] layout written at token offset pos
-# ---------------------------------------------------------------------------
-
-def encode_into_cache(x: np.ndarray, signs, lam, G: int, codes_cache: np.ndarray,
-                      scales_cache: np.ndarray, pos: int, transform: str = "srft", bits: int = 4) -> None:
-    """Encode x [B, H, n, D] and write rows pos..pos+n-1 of the cache in place."""
-    n = x.shape[2]
-    enc = encode(x, signs, lam, G, transform, bits)
-    codes_cache[:, :, pos:pos + n, :] = enc["packed"]
-    scales_cache[:, :, pos:pos + n, :] = enc["scales"]
 
 
 # ---------------------------------------------------------------------------

@@ -59,6 +59,8 @@ def _load() -> ctypes.CDLL:
         "kvq_attend_decode_noalloc": (I, [P, P, P, P, P, P, P, I, I, I, I, P, I, F, P, P]),
         "kvq_attend_decode_batch": (I, [ctypes.POINTER(AttendJob), I, I, I, I, I, P, I, F, P, S, P]),
         "kvq_poll_device_errors": (I, [U32P]),
+        "kvq_attend_split_info": (I, [I, I, I, I, I, I, I, ctypes.POINTER(I), ctypes.POINTER(I), ctypes.POINTER(I)]),
+        "kvq_debug_wait_timeout": (I, [ctypes.c_uint32, P]),
         "kvq_set_encode_path": (I, [I]),
         "kvq_get_encode_path": (I, []),
         "kvq_status_string": (ctypes.c_char_p, [I]),

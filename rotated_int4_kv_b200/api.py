@@ -369,3 +369,20 @@ def poll_device_errors() -> int:
     flags = ctypes.c_uint32(0)
     check(lib.kvq_poll_device_errors(ctypes.byref(flags)), "kvq_poll_device_errors")
     return int(flags.value)
+
+
+def attend_split_info(B: int, Hq: int, Hkv: int, head_dim: int, T: int, group: int = 32, bits: int = 4):
+    """(splits, cluster, head_tiles) that the attention entry points choose for these
+    shapes on the current device (bits 16 = the fp16 comparator). A unit whose
+    splits / cluster > 1 merges its cluster partials through the workspace."""
+    s, c, h = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    check(lib.kvq_attend_split_info(B, Hq, Hkv, head_dim, group, bits, T, ctypes.byref(s), ctypes.byref(c),
+                                    ctypes.byref(h)), "kvq_attend_split_info")
+    return int(s.value), int(c.value), int(h.value)
+
+
+def debug_wait_timeout(limit_us: int, stream=None) -> None:
+    """Launch the library's bounded-wait self-test: one CTA waits on a barrier that never
+    completes with a budget of limit_us, then raises the load-timeout flag (1) that
+    :func:`poll_device_errors` reports."""
+    check(lib.kvq_debug_wait_timeout(int(limit_us), _stream(stream)), "kvq_debug_wait_timeout")

@@ -578,6 +578,29 @@ kvq_status kvq_attend_decode_ref(const uint16_t* q, const uint16_t* k, const uin
                                  (cudaStream_t)stream);
 }
 
+kvq_status kvq_attend_split_info(int B, int Hq, int Hkv, int D, int G, int bits, int T, int* splits, int* cluster,
+                                 int* head_tiles) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || T < 0) return fail(KVQ_ERR_INVALID_ARG, "split_info: bad sizes");
+  if (Hq % Hkv) return fail(KVQ_ERR_UNSUPPORTED, "split_info: Hq must be a multiple of Hkv");
+  if (D != 128 && D != 256) return fail(KVQ_ERR_UNSUPPORTED, "split_info: head_dim must be 128 or 256");
+  if (bits != 4 && bits != 8 && bits != 16) return fail(KVQ_ERR_UNSUPPORTED, "split_info: bits must be 4, 8 or 16");
+  if (bits != 16 && G != 32 && G != 16) return fail(KVQ_ERR_UNSUPPORTED, "split_info: group must be 32 or 16");
+  int dev = -1;
+  cudaDeviceProp prop{};
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaGetDeviceProperties(&prop, dev) != cudaSuccess || prop.major != 10)
+    return fail(KVQ_ERR_DEVICE, "split_info: needs a current compute capability 10.x (sm_100) device");
+  return kvq::attend_split_info(B, Hq, Hkv, D, G, bits, T, splits, cluster, head_tiles);
+}
+
+kvq_status kvq_debug_wait_timeout(uint32_t limit_us, void* stream) {
+  if (limit_us == 0 || limit_us > 1000000u) return fail(KVQ_ERR_INVALID_ARG, "debug_wait_timeout: limit_us must be in [1, 1e6]");
+  int dev = -1;
+  cudaDeviceProp prop{};
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaGetDeviceProperties(&prop, dev) != cudaSuccess || prop.major != 10)
+    return fail(KVQ_ERR_DEVICE, "debug_wait_timeout: needs a current compute capability 10.x (sm_100) device");
+  return kvq::launch_wait_probe(limit_us, (cudaStream_t)stream);
+}
+
 kvq_status kvq_poll_device_errors(uint32_t* flags) {
   if (cudaDeviceSynchronize() != cudaSuccess) return fail(KVQ_ERR_CUDA, "poll: device synchronize failed");
   const uint32_t f = kvq::codec_error_flags(true) | kvq::attend_error_flags(true) | kvq::encode_tc_error_flags(true);

@@ -2176,6 +2176,52 @@ kvq_status launch_attend_int4_noalloc(const kvq_plan* pk, const kvq_plan* pv, co
                                   s);
 }
 
+// ---------------------------------------------------------------- split query
+kvq_status attend_split_info(int B, int Hq, int Hkv, int D, int G, int bits, int T, int* splits, int* cluster,
+                             int* head_tiles) {
+  SplitPlan sp{};
+  if (bits == 16) {
+    if (D == 128) {
+      using C = Cfg<128, false>;
+      sp = choose_split(B, Hq, Hkv, T, occupancy<128, false, 1>(), C::kTile, C::kStageNs);
+    } else {
+      using C = Cfg<256, false>;
+      sp = choose_split(B, Hq, Hkv, T, occupancy<256, false, 1>(), C::kTile, C::kStageNs);
+    }
+  } else {
+    sp = dispatch_dgb(D, G, bits, [&](auto d, auto g, auto b) {
+      constexpr int kD = decltype(d)::value, kG = decltype(g)::value, kB = decltype(b)::value;
+      using C = Cfg<kD, true, kG, kB>;
+      return choose_split(B, Hq, Hkv, T, occupancy<kD, true, 1, kG, kB>(), C::kTile, C::kStageNs);
+    });
+  }
+  if (splits) *splits = sp.S;
+  if (cluster) *cluster = sp.C;
+  if (head_tiles) *head_tiles = sp.HT;
+  return KVQ_OK;
+}
+
+// ---------------------------------------------------------------- bounded-wait probe
+// One CTA arms an mbarrier with a transaction count that no copy will ever satisfy
+// and waits on it through the library's bounded wait with a short budget; when the
+// budget runs out it raises the same error flag a stalled TMA load raises in the
+// kernels above and returns. Nothing is loaded, so nothing is left in flight.
+__global__ void wait_probe_kernel(uint64_t limit_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x != 0) return;
+  mbar_init(&bar, 1);
+  fence_mbarrier_init();
+  mbar_arrive_expect_tx(&bar, 16);
+  if (!mbar_wait_bounded(&bar, 0, limit_ns)) atomicOr(&g_attend_err, kErrTimeoutLoad);
+}
+
+kvq_status launch_wait_probe(uint32_t limit_us, cudaStream_t s) {
+  wait_probe_kernel<<<1, 32, 0, s>>>((uint64_t)limit_us * 1000ull);
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return fail(KVQ_ERR_CUDA, std::string("wait probe launch: ") + cudaGetErrorString(e));
+  return KVQ_OK;
+}
+
 uint32_t attend_error_flags(bool clear) {
   uint32_t v = 0;
   cudaMemcpyFromSymbol(&v, g_attend_err, sizeof(v));

@@ -133,6 +133,10 @@ kvq_status launch_attend_fp16(const uint16_t* q, const uint16_t* k, const uint16
                               int Hkv, int D, int T_cap, const int32_t* seq_lens, int T_len, float sigma,
                               uint16_t* out, void* ws, size_t ws_bytes, cudaStream_t s);
 
+kvq_status attend_split_info(int B, int Hq, int Hkv, int D, int G, int bits, int T, int* splits, int* cluster,
+                             int* head_tiles);
+kvq_status launch_wait_probe(uint32_t limit_us, cudaStream_t s);
+
 // device error word (bit flags raised by kernels that gave up a bounded wait)
 uint32_t* device_error_word();
 

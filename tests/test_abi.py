@@ -22,7 +22,8 @@ def test_header_declares_the_boundary():
               "kvq_workspace_size", "kvq_attend_decode", "kvq_attend_decode_ref", "kvq_status_string",
               "kvq_last_error", "kvq_poll_device_errors", "kvq_attend_decode_batch",
               "kvq_attend_decode_noalloc", "kvq_attend_decode_append", "kvq_plan_create_transform",
-              "kvq_plan_transform", "kvq_plan_create_ex", "kvq_plan_bits"):
+              "kvq_plan_transform", "kvq_plan_create_ex", "kvq_plan_bits", "kvq_attend_split_info",
+              "kvq_debug_wait_timeout"):
         assert n in names
 
 
@@ -58,6 +59,13 @@ def test_status_strings_and_host_checks():
     assert lib.kvq_encode_batch(None, 0, None) == 0
     assert lib.kvq_attend_decode_batch(None, -1, 1, 4, 1, 64, None, 64, ctypes.c_float(0), None, 0, None) == -1
     assert lib.kvq_attend_decode_batch(None, 0, 1, 4, 1, 64, None, 64, ctypes.c_float(0), None, 0, None) == 0
+    # planning query and the wait self-test: argument checks before any device call
+    assert lib.kvq_attend_split_info(0, 8, 1, 128, 32, 4, 1024, None, None, None) == -1
+    assert lib.kvq_attend_split_info(1, 6, 4, 128, 32, 4, 1024, None, None, None) == -2
+    assert lib.kvq_attend_split_info(1, 8, 1, 96, 32, 4, 1024, None, None, None) == -2
+    assert lib.kvq_attend_split_info(1, 8, 1, 128, 32, 5, 1024, None, None, None) == -2
+    assert lib.kvq_debug_wait_timeout(0, None) == -1
+    assert lib.kvq_debug_wait_timeout(2000000, None) == -1
     jobs = (kvq_lib.AttendJob * 2)()  # null plans: refused before any CUDA call
     assert lib.kvq_attend_decode_batch(jobs, 2, 1, 4, 1, 64, None, 64, ctypes.c_float(0), None, 0, None) == -1
     assert b"job 0" in lib.kvq_last_error()

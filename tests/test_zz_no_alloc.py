@@ -23,7 +23,7 @@ def _cache(kvq, wl, B, Hkv, T, seed):
     out = {}
     for kind in ("k", "v"):
         plan = kvq.Plan(*kvgen.plan_params(D, seed=seed, kind=kind))
-        x = torch.from_numpy(kvgen.kv_numpy(wl, kind, (B, Hkv, T, D), seed=seed)).to(dev)
+        x = kvgen.kv_torch(wl, kind, (B, Hkv, T, D), dev, seed=seed)
         codes = torch.zeros((B, Hkv, T, D // 2), dtype=torch.uint8, device=dev)
         scales = torch.zeros((B, Hkv, T, D // 32), dtype=torch.float16, device=dev)
         kvq.encode(plan, x, codes, scales, 0)
@@ -31,15 +31,21 @@ def _cache(kvq, wl, B, Hkv, T, seed):
     return out
 
 
-@pytest.mark.parametrize("name,B,Hkv,Hq,T,lens", [
-    ("qwen", 2, 2, 12, 1000, [1000, 377]),
-    ("gemma", 1, 1, 4, 4096, None),
+@pytest.mark.parametrize("name,B,Hkv,Hq,T,lens,multi", [
+    ("qwen", 2, 2, 12, 1000, [1000, 377], False),
+    ("gemma", 1, 1, 4, 4096, None, False),
+    # one unit over 128K tokens: its splits span several clusters, so the cluster
+    # partials are written to and merged from the static scratch, not only the counters
+    ("longctx", 1, 1, 8, 131072, None, True),
 ])
-def test_noalloc_matches_workspace_entry_point_twice(name, B, Hkv, Hq, T, lens):
+def test_noalloc_matches_workspace_entry_point_twice(name, B, Hkv, Hq, T, lens, multi):
     import rotated_int4_kv_b200 as kvq
 
     wl = kvgen.WORKLOADS[name]
     D = wl.head_dim
+    if multi:
+        S, C, _ = kvq.attend_split_info(B, Hq, Hkv, D, T)
+        assert S // C > 1, f"split {S} in clusters of {C}: the scratch's partial region would not be used"
     c = _cache(kvq, wl, B, Hkv, T, seed=41)
     q = torch.from_numpy(kvgen.q_numpy((B, Hq, D), salt=13)).cuda()
     sl = None if lens is None else torch.tensor(lens, dtype=torch.int32, device="cuda")
