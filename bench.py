@@ -56,6 +56,7 @@ def _peaks():
 KERNEL_SOURCES = {
     "encode": ["kvq_codec.cu", "kvq_ptx.cuh", "srft_fft.cuh", "kvq_internal.h"],
     "encode_tc": ["kvq_encode_tc.cu", "kvq_ptx.cuh", "kvq_quant.cuh", "kvq_internal.h"],
+    "encode_split": ["kvq_encode_tc.cu", "kvq_ptx.cuh", "kvq_quant.cuh", "kvq_internal.h", "srft_fft.cuh"],
     "attend": ["kvq_attend.cu", "kvq_ptx.cuh", "kvq_quant.cuh", "kvq_internal.h"],
 }
 NCU_TRAFFIC = {
@@ -107,6 +108,20 @@ def _ncu_traffic_attn(arm: str):
         return None
     rec = NCU_TRAFFIC_ATTN.get(arm)
     return rec[1] if rec is not None and rec[0] == _source_digest("attend") else None
+
+
+def _encode_kernel(path: str, D: int, G: int):
+    """(traffic key, kernel name, tensor flops per vector or None) of the encode `path` runs.
+    Mirrors the library's dispatch: "auto" is the dense tensor-core product. Tensor work
+    per vector: the dense
+    product X [W_hi; W_lo]^T is 2 x D x 2D flops (SRHT: the exact W, 2 x D x D); the split
+    is two 128-point products (E, O), each hi + lo: 2 x 2 x 2 x 128 x 128 = 2 D^2 at D = 256."""
+    xf = int(TRANSFORM == "srht")
+    if path == "fft":
+        return "encode", f"encode_kernel<{D},{G},{xf},{BITS},64>", None
+    if path == "split":
+        return "encode_split", f"encode_split_kernel<{G},{BITS},64>", 2 * D * D
+    return "encode_tc", f"encode_tc_kernel<{D},{xf},{G},{BITS},64>", (2 if xf else 4) * D * D
 
 
 def _algo_bytes(D: int, G: int = 32, bits: int = 4):
@@ -469,22 +484,17 @@ def run_kvq(args, rank: int, world: int):
     clocks = clk.summary(wall0 - 1.0, wall1 + 0.2)
     # roofline of the kernel with the larger share of the step (each phase is one launch)
     src = "measured (MEASURED_PEAKS.json hbm_gbs, burst copy)" if peak_kind == "measured" else "fallback 6.65 TB/s"
-    tc = kvq.get_encode_path() != "fft" and G == 32
-    # the tensor-core encode's own work: Y = X [W_hi; W_lo]^T, 2 x D x 2D flops per vector
-    # (SRHT plans: the exact W, 2 x D x D) -- context for the HBM roofline: at D = 256 the
-    # hi/lo product, not HBM, bounds the SRFT kernel
+    enc_key, enc_kernel, fpv = _encode_kernel(kvq.get_encode_path(), D, G)
+    # the tensor-core encode's own work (context for the HBM roofline)
     tensor = None
-    if tc:
-        fpv = (2 if TRANSFORM == "srht" else 4) * D * D
+    if fpv is not None:
         tflops = vec_step * fpv / (enc_avg * 1e-3) / 1e12
         tensor = {"flops_per_vec": fpv, "achieved_TFLOP_s": tflops,
                   "peak_TFLOP_s": _tensor_peak(), "frac": tflops / _tensor_peak(),
                   "peak_source": "measured (MEASURED_PEAKS.json bf16_tflops_sustained; fp16 runs at the bf16 rate)"}
     if enc_avg >= att_avg:
         roof = {"bound": "hbm", "achieved": enc_gbs, "peak": hbm, "unit": "GB/s", "frac": enc_gbs / hbm,
-                "traffic": _ncu_traffic("encode_tc" if tc else "encode"),
-                "kernel": f"encode_tc_kernel<{D},{int(TRANSFORM == 'srht')},{G},{BITS},64>" if tc
-                else f"encode_kernel<{D},{G},{int(TRANSFORM == 'srht')},{BITS},64>",
+                "traffic": _ncu_traffic(enc_key), "kernel": enc_kernel,
                 "share": enc_avg / (enc_avg + att_avg), "peak_source": src}
     else:
         roof = {"bound": "hbm", "achieved": att_gbs, "peak": hbm, "unit": "GB/s", "frac": att_gbs / hbm,
@@ -506,7 +516,7 @@ def run_kvq(args, rank: int, world: int):
                           "frac_hbm": att_gbs / hbm, "bytes_per_token_head": tok_b},
             "roofline": roof,
             "kernels": {  # both launches of the step, each timed with CUDA events on its stream
-                "encode": {"kernel": roof["kernel"] if enc_avg >= att_avg else "encode", "us": 1e3 * enc_avg,
+                "encode": {"kernel": enc_kernel, "us": 1e3 * enc_avg, "traffic": _ncu_traffic(enc_key),
                            "achieved_GB_s": enc_gbs, "frac": enc_gbs / hbm, "share": enc_avg / (enc_avg + att_avg),
                            "tensor": tensor},
                 "attention": {"kernel": f"attend_kernel<{D},{'int4' if BITS == 4 else 'int8'},{G}>", "us": 1e3 * att_avg, "achieved_GB_s": att_gbs,
@@ -740,9 +750,10 @@ def main(argv=None):
                     help="code width of the plans: 4 (the pages' int4, default) or 8 (int8 codes)")
     ap.add_argument("--skip-attention-arms", action="store_true",
                     help="default workload: leave out the int4-vs-fp16 attention arms (Mistral 32K, 128K, Qwen step)")
-    ap.add_argument("--encode-path", default="auto", choices=["auto", "fft", "tensor"],
+    ap.add_argument("--encode-path", default="auto", choices=["auto", "fft", "tensor", "split"],
                     help="encode kernel of the prefill step: tensor cores where supported (auto), "
-                         "the register FFT, or tensor cores only")
+                         "the register FFT, the dense tensor-core product, or the radix-2 split "
+                         "(head_dim 256 SRFT)")
     args = ap.parse_args(argv)
     global TRANSFORM, BITS
     TRANSFORM = args.transform

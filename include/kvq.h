@@ -166,15 +166,19 @@ kvq_status kvq_encode_batch(const kvq_encode_job* jobs, int njobs, void* stream)
 /*
  * kvq_set_encode_path / kvq_get_encode_path -- which kernel kvq_encode and
  * kvq_encode_batch run (process-wide setting; not on the pages):
- *   0  default: the tensor-core encode (tcgen05 GEMM against W = Lambda F_r diag(s)
- *      held as an fp16 hi + lo pair; for SRHT plans the exact W = H diag(s)), which
- *      covers head_dim 128 and 256 with group 32 or 16;
+ *   0  default: the dense tensor-core encode (path 2) where it exists;
  *   1  always the register-FFT encode (one radix-2 real FFT per vector in registers);
- *   2  always the tensor-core encode (KVQ_ERR_UNSUPPORTED where it does not exist).
+ *   2  the dense tensor-core encode (tcgen05 GEMM against W = Lambda F_r diag(s) held
+ *      as an fp16 hi + lo pair; for SRHT plans the exact W = H diag(s)), head_dim 128
+ *      and 256 with group 32 or 16;
+ *   3  the radix-2 split on the tensor cores: the two 128-point real DFTs of the even
+ *      and odd samples as products against the plan-independent F128 (fp16 hi + lo),
+ *      joined by one radix-2 step (half the tensor work of path 2); head_dim 256 SRFT
+ *      plans only (KVQ_ERR_UNSUPPORTED otherwise).
  * Both produce codes and scales that meet the same acceptance rule against the
  * fp64 definition; they may differ from each other only at rounding boundaries.
  * Set it between launches, not while another thread is encoding.
- * Errors: INVALID_ARG for a value other than 0, 1, 2.
+ * Errors: INVALID_ARG for a value other than 0, 1, 2, 3.
  */
 kvq_status kvq_set_encode_path(int path);
 int kvq_get_encode_path(void);

@@ -111,12 +111,13 @@ def encode_batch(jobs, stream=None) -> None:
     check(lib.kvq_encode_batch(arr, len(jobs), _stream(stream)), "kvq_encode_batch")
 
 
-ENCODE_PATHS = {"auto": 0, "fft": 1, "tensor": 2}
+ENCODE_PATHS = {"auto": 0, "fft": 1, "tensor": 2, "split": 3}
 
 
 def set_encode_path(path: str) -> None:
     """Select the encode kernel: "auto" (tensor cores where supported), "fft"
-    (register FFT) or "tensor" (tensor cores only)."""
+    (register FFT), "tensor" (tensor cores, dense product) or "split" (tensor cores,
+    radix-2 split; head_dim 256 SRFT plans only)."""
     check(lib.kvq_set_encode_path(ENCODE_PATHS[path]), "kvq_set_encode_path")
 
 

@@ -83,7 +83,12 @@ kvq_status dispatch_encode(const kvq_encode_job* jobs, int njobs, cudaStream_t s
   const bool tc = encode_tc_supported(p->D, p->G) && p->wt_dev != nullptr;
   if (path == 2 && !tc)
     return fail(KVQ_ERR_UNSUPPORTED, "encode: the tensor-core path supports head_dim 128 or 256 with group 32 or 16");
-  if (tc && path != 1) return launch_encode_tc(jobs, njobs, s);
+  if (path == 3) {
+    if (!encode_split_supported(p))
+      return fail(KVQ_ERR_UNSUPPORTED, "encode: the radix-2 split path serves head_dim 256 SRFT plans");
+    return launch_encode_tc(jobs, njobs, s, true);
+  }
+  if (tc && path != 1) return launch_encode_tc(jobs, njobs, s, false);
   return launch_encode_jobs(jobs, njobs, s);
 }
 
@@ -380,7 +385,7 @@ kvq_status kvq_encode_batch(const kvq_encode_job* jobs, int njobs, void* stream)
 }
 
 kvq_status kvq_set_encode_path(int path) {
-  if (path < 0 || path > 2) return fail(KVQ_ERR_INVALID_ARG, "set_encode_path: path must be 0, 1 or 2");
+  if (path < 0 || path > 3) return fail(KVQ_ERR_INVALID_ARG, "set_encode_path: path must be 0, 1, 2 or 3");
   kvq::g_encode_path.store(path);
   return KVQ_OK;
 }

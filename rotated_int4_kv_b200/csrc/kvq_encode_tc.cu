@@ -37,10 +37,12 @@
 #include <algorithm>
 #include <cstdio>
 #include <mutex>
+#include <utility>
 
 #include "kvq_internal.h"
 #include "kvq_ptx.cuh"
 #include "kvq_quant.cuh"
+#include "srft_fft.cuh"
 
 namespace kvq {
 
@@ -59,7 +61,8 @@ struct alignas(64) TcJob {
   CUtensorMap wmap;  // W as [2D][D] fp16 (hi rows, then lo rows; EX: [D][D]), box {64, N}, 128-byte swizzle
   uint8_t* codes;    // [BH][T_cap][D * BITS / 8]
   uint16_t* scales;  // [BH][T_cap][D/G]
-  const float* chan; // EX: the per-channel factors lambda_c / sqrt(D)
+  const float* chan; // EX: the per-channel factors lambda_c / sqrt(D); split: lambda_c dg_c
+  const uint32_t* sgn;  // split: sign masks, one per fp16 pair of samples
   int rows, n, T_cap, pos, tile0;  // rows = B*H*n; tile0 = first global tile of the job
 };
 
@@ -389,6 +392,380 @@ __global__ void __launch_bounds__(kTcThreads, 1) encode_tc_kernel(const __grid_c
 }
 
 
+// ============================================================================ D = 256, radix-2 split
+// The SRFT at D = 256 by one radix-2 decimation in time, with the two half-length
+// transforms on the tensor cores (half the tensor work of the dense hi/lo product).
+// With x' = s (.) x and the unnormalised 128-point real spectra (slot order: slot 0 =
+// X_0, slot 1 = X_64, slot 2k = Re X_k, slot 2k+1 = Im X_k)
+//   E = F128 x'_even,  O = F128 x'_odd,
+//   X_k = E_k + W^k O_k,  X_{128-k} = conj(E_k - W^k O_k),  W = e^{-2 pi i / 256},
+// and y_c = lambda_c dg_c (Re or Im of X at channel c's frequency). F128 is the plan-
+// independent matrix the attention kernels use (fp16 hi + lo, exact to ~2^-22), so
+// it is loaded once per CTA and never reloaded when the job changes; each plan's
+// signs are applied while the samples are separated, and its factors in the epilogue.
+//   warp 0      TMA: F128 (resident), each tile's plan constants (bulk copies into one
+//               of three slots), a ring of 16 KB chunks (128 rows x 64 samples) of x;
+//   warp 1      TMEM (E and O of two tiles: 512 columns) and the MMA thread: per tile
+//               2 x 2 x 4 K steps of M = 128, N = 128 (hi, then lo into the same
+//               accumulator);
+//   warps 2-9   workers, per tile i: first the separation of tile i + 1 -- thread
+//               (row r, half j) applies the signs to row r of chunk pair j (samples
+//               128j .. 128j + 127) and rewrites it in place as the 64 even samples
+//               (chunk 2j: E's inputs 64j .. 64j + 63) and the 64 odd ones, so the MMAs
+//               of tile i + 1 run during the epilogue of tile i; then the epilogue of
+//               tile i -- thread (row, h) forms X_k and X_{128-k} for k = 16 g .. 16 g + 16
+//               of its group pairs g = 2h, 2h + 1 (channel chunks g and 7 - g) with
+//               compile-time twiddles, applies the factors and quantises.
+constexpr int kSpRing = 9;     // ring depth in chunks (a tile is four)
+constexpr int kSpWork = 8;     // worker warps: the separation of tile i + 1, then the epilogue of tile i
+constexpr int kSpThreads = 32 * (2 + kSpWork);
+constexpr int kSpChunk = kTcRows * 128;        // 16 KB
+constexpr int kSpF = 2 * (256 * 128);          // F128 [hi; lo] (256 rows) x 2 K-chunks of 64: 64 KB
+constexpr int kSpCst = 256 * 4 + 128 * 4;      // a tile's plan constants: lambda_c dg_c [256], sign masks [128]
+// constant slots: tiles i (epilogue) and i + 1 (separation) are in use while tile i + 2's
+// constants load, so that load never waits for the epilogue just finishing
+constexpr int kSpCstSlots = 3;
+constexpr int kSpBars = 8 * (3 * kSpRing + 2 * 2 + 2 * kSpCstSlots + 2) + 16;
+constexpr int kSpSmem = kSpF + kSpRing * kSpChunk + kSpCstSlots * kSpCst + kSpBars + 1024;
+static_assert(kSpSmem <= 227 * 1024, "shared memory");
+
+// 16 bytes of shared memory, loaded where written (volatile: loop-invariant loads of the
+// sign masks would otherwise be hoisted out of the row loop and held in 128 registers)
+__device__ __forceinline__ uint4 lds128_here(const void* p) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(smem_u32(p)));
+  return v;
+}
+
+// byte offset of 16-byte unit u of row r in a 128-byte-swizzled chunk (1024-byte aligned)
+__device__ __forceinline__ uint32_t sw128_off(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
+
+// Frequency k = 16 GP + TT of a group pair: X_k = E_k + W^k O_k (SIDE 0) or X_{128-k} =
+// conj(E_k - W^k O_k) (SIDE 1), W = e^{-2 pi i / 256}, times the channel factors, into the
+// chunk's local channels.
+template <int GP, int TT, int SIDE>
+__device__ __forceinline__ void split_freq(const float (&e)[32], const float (&o)[32], float e32, float e33, float o32,
+                                           float o33, const float* cc, float (&y)[32]) {
+  float er, ei, orr, oi;
+  if constexpr (TT < 16) {
+    er = e[2 * TT];
+    orr = o[2 * TT];
+    // k = 0: slot 1 holds X_64, and Im X_0 = 0
+    ei = (GP == 0 && TT == 0) ? 0.0f : e[2 * TT + 1];
+    oi = (GP == 0 && TT == 0) ? 0.0f : o[2 * TT + 1];
+  } else if constexpr (GP < 3) {
+    er = e32;
+    ei = e33;
+    orr = o32;
+    oi = o33;
+  } else {  // k = 64: E_64 and O_64 are real
+    er = e33;
+    ei = 0.0f;
+    orr = o33;
+    oi = 0.0f;
+  }
+  constexpr float c = static_cast<float>(cos2pi_frac(16 * GP + TT, 256));
+  constexpr float sn = static_cast<float>(sin2pi_frac(16 * GP + TT, 256));
+  const float xr = fmaf(c, orr, fmaf(sn, oi, er));   // Re X_k = Re (E + W^k O)
+  const float xi = fmaf(c, oi, fmaf(-sn, orr, ei));  // Im X_k
+  if constexpr (SIDE == 0) {
+    // channel 2k - 1 = Re X_k (local 2TT - 1), 2k = Im X_k (local 2TT); local 0 of chunk 0 is X_0
+    if constexpr (TT >= 1) y[2 * TT - 1] = xr * cc[2 * TT - 1];
+    if constexpr (TT <= 15) y[2 * TT] = (GP == 0 && TT == 0 ? xr : xi) * cc[2 * TT];
+  } else {
+    // Re X_{128-k} = 2 Re E - Re X_k at local 31 - 2TT, Im X_{128-k} = Im X_k - 2 Im E at 32 - 2TT
+    if constexpr (TT <= 15) y[31 - 2 * TT] = fmaf(2.0f, er, -xr) * cc[31 - 2 * TT];
+    if constexpr (TT >= 1) y[32 - 2 * TT] = fmaf(-2.0f, ei, xi) * cc[32 - 2 * TT];
+  }
+}
+
+template <int GP, int SIDE, int... TT>
+__device__ __forceinline__ void split_freqs(std::integer_sequence<int, TT...>, const float (&e)[32], const float (&o)[32],
+                                            float e32, float e33, float o32, float o33, const float* cc,
+                                            float (&y)[32]) {
+  (split_freq<GP, TT, SIDE>(e, o, e32, e33, o32, o33, cc, y), ...);
+}
+
+// One channel chunk of a tile row: SIDE 0 = chunk GP, from X_k (k = 16 GP + tt, tt = 0..16);
+// SIDE 1 = chunk 7 - GP, from X_{128-k} (the same E_k, O_k). E and O are (re)loaded from TMEM
+// for each side, which keeps one side's values live at a time (a CTA of ten warps gets at
+// most 168 registers a thread). sb collects the chunk's scale bits at sb[SPC * slot].
+template <int GP, int SIDE, int G, int BITS>
+__device__ __forceinline__ void split_side(uint32_t ta, const float* chan, uint8_t* codes, size_t orow, bool valid,
+                                           uint32_t (&sb)[64 / G], int slot, uint64_t* tempty, bool release) {
+  constexpr int SPC = 32 / G;
+  float e[32], o[32], e32, e33, o32, o33;
+  tmem_ld32(ta + 32 * GP, e);
+  tmem_ld32(ta + 128 + 32 * GP, o);
+  // k = 16 GP + 16: slots (2k, 2k + 1), or for GP = 3 the real X_64 in slot 1 (read with slot 0)
+  constexpr int xc = GP < 3 ? 32 * GP + 32 : 0;
+  tmem_ld2(ta + xc, e32, e33);
+  tmem_ld2(ta + 128 + xc, o32, o33);
+  tmem_ld_wait();
+  tmem_regs_fence(e);
+  tmem_regs_fence(o);
+  tmem_regs_fence(e32);
+  tmem_regs_fence(e33);
+  tmem_regs_fence(o32);
+  tmem_regs_fence(o33);
+  if (release) {  // every TMEM value of this tile is in registers: the accumulator may be reused
+    tc_fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(tempty);
+  }
+  const float* cc = chan + 32 * (SIDE == 0 ? GP : 7 - GP);
+  float y[32];
+  // frequencies k = 16 GP + TT, TT = 0..16, with their twiddles as compile-time constants
+  split_freqs<GP, SIDE>(std::make_integer_sequence<int, 17>{}, e, o, e32, e33, o32, o33, cc, y);
+  uint32_t w[BITS], sg[SPC];
+  quantize_chunk<G, BITS>(y, w, sg);
+#pragma unroll
+  for (int j = 0; j < SPC; ++j) sb[SPC * slot + j] = sg[j];
+  if (valid) store_chunk<256, BITS>(codes, orow, SIDE == 0 ? GP : 7 - GP, w);
+}
+
+// Group pair GP of a tile row: chunks GP and 7 - GP (scale bits into sb_lo / sb_hi: the chunks
+// (2h, 2h + 1) and (6 - 2h, 7 - 2h), h = GP / 2).
+template <int GP, int G, int BITS>
+__device__ __forceinline__ void split_pair(uint32_t ta, const float* chan, uint8_t* codes, size_t orow, bool valid,
+                                           uint32_t (&sb_lo)[64 / G], uint32_t (&sb_hi)[64 / G], uint64_t* tempty,
+                                           bool release) {
+  split_side<GP, 0, G, BITS>(ta, chan, codes, orow, valid, sb_lo, GP & 1, tempty, false);
+  split_side<GP, 1, G, BITS>(ta, chan, codes, orow, valid, sb_hi, 1 - (GP & 1), tempty, release);
+}
+
+template <int G, int BITS, int MAXJ>
+__global__ void __launch_bounds__(kSpThreads, 1) encode_split_kernel(const __grid_constant__ TcBatch<MAXJ> bt) {
+  constexpr int SPC = 32 / G;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sF = sm;
+  uint8_t* sR = sF + kSpF;
+  uint8_t* sC = sR + kSpRing * kSpChunk;
+  uint64_t* rfull = reinterpret_cast<uint64_t*>(sC + kSpCstSlots * kSpCst);  // [ring] a chunk landed
+  uint64_t* rdone = rfull + kSpRing;                                // [ring] a chunk separated
+  uint64_t* rempty = rdone + kSpRing;                               // [ring] the MMAs read it
+  uint64_t* tfull = rempty + kSpRing;  // [2] accumulators ready
+  uint64_t* tempty = tfull + 2;        // [2] accumulators drained
+  uint64_t* cfull = tempty + 2;                // [slots] a tile's plan constants landed
+  uint64_t* cempty = cfull + kSpCstSlots;      // [slots] the workers are done with them
+  uint64_t* ffull = cempty + kSpCstSlots;      // F128 landed
+  uint64_t* mdone = ffull + 1;         // every MMA of this CTA completed
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(mdone + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int per = (bt.ntiles + (int)gridDim.x - 1) / (int)gridDim.x;
+  const int t_begin = (int)blockIdx.x * per;
+  const int t_end = min(t_begin + per, bt.ntiles);
+  const int ntile = max(0, t_end - t_begin);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kSpRing; ++s) {
+      mbar_init(&rfull[s], 1);
+      mbar_init(&rdone[s], kSpWork / 2);  // the four worker warps of that chunk pair
+      mbar_init(&rempty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tfull[b], 1);
+      mbar_init(&tempty[b], kSpWork);
+    }
+    for (int b = 0; b < kSpCstSlots; ++b) {
+      mbar_init(&cfull[b], 1);
+      mbar_init(&cempty[b], kSpWork);
+    }
+    mbar_init(ffull, 1);
+    mbar_init(mdone, 1);
+    fence_mbarrier_init();
+  }
+  grid_dep_launch();
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0 && ntile > 0) {
+      const uint64_t pol = l2_evict_first_policy();
+      int job = job_of(bt.j, bt.njobs, 0, t_begin);
+      // F128 is a constant of every plan (written when the plan is made): loaded while
+      // the previous kernel in the stream finishes; the inputs only after it
+      mbar_arrive_expect_tx(ffull, kSpF);
+      tma_load_2d(sF, &bt.j[job].wmap, ffull, 0, 0);
+      tma_load_2d(sF + kSpF / 2, &bt.j[job].wmap, ffull, 64, 0);
+      grid_dep_wait();
+      bool ok = true;
+      for (int i = 0; i < ntile && ok; ++i) {
+        const int t = t_begin + i;
+        job = job_of(bt.j, bt.njobs, job, t);
+        const TcJob& J = bt.j[job];
+        const int row = (t - J.tile0) * kTcRows;
+        const int cs = i % kSpCstSlots;
+        if (i >= kSpCstSlots && !mbar_wait_bounded(&cempty[cs], ((i / kSpCstSlots) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&cfull[cs], kSpCst);
+        bulk_load(sC + cs * kSpCst, J.chan, 256 * 4, &cfull[cs]);
+        bulk_load(sC + cs * kSpCst + 256 * 4, J.sgn, 128 * 4, &cfull[cs]);
+#pragma unroll
+        for (int kc = 0; kc < 4; ++kc) {
+          const int c = 4 * i + kc, s = c % kSpRing;
+          if (c >= kSpRing && !mbar_wait_bounded(&rempty[s], ((c / kSpRing) - 1) & 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&rfull[s], kSpChunk);
+          tma_load_2d_hint(sR + s * kSpChunk, &J.xmap, &rfull[s], kc * 64, row, pol);
+        }
+      }
+      if (!ok) atomicOr(&g_enc_tc_err, kErrTimeoutLoad);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && ntile > 0) {
+      constexpr uint32_t idesc = umma_idesc_f16(kTcRows, 128);
+      bool ok = mbar_wait_bounded(ffull, 0);
+      for (int i = 0; i < ntile && ok; ++i) {
+        const int a = i & 1;
+        if (i >= 2 && !mbar_wait_bounded(&tempty[a], ((i >> 1) - 1) & 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t f0 = smem_u32(sF);
+#pragma unroll
+        for (int j = 0; j < 2 && ok; ++j) {
+#pragma unroll
+          for (int eo = 0; eo < 2; ++eo) {  // E's inputs 64j .. 64j + 63 in chunk 4i + 2j, O's in the next
+            const int c = 4 * i + 2 * j + eo, s = c % kSpRing;
+            if (!mbar_wait_bounded(&rdone[s], (c / kSpRing) & 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t d = tmem + (uint32_t)(a * 256 + eo * 128);
+            const uint32_t a0 = smem_u32(sR + s * kSpChunk);
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk) {  // K = 16 per MMA: 32 bytes along the swizzled row
+              const uint64_t ad = umma_desc_sw128(a0 + kk * 32);
+              const uint32_t fb = f0 + j * (kSpF / 2) + kk * 32;
+              umma_f16(d, ad, umma_desc_sw128(fb), idesc, (j | kk) != 0);        // F128 hi rows
+              umma_f16(d, ad, umma_desc_sw128(fb + 128 * 128), idesc, true);    // F128 lo rows
+            }
+            umma_commit(&rempty[s]);  // the chunk is free once these MMAs have read it
+          }
+        }
+        if (!ok) break;
+        umma_commit(&tfull[a]);
+      }
+      if (!ok) atomicOr(&g_enc_tc_err, kErrTimeoutLoad);
+      // TMEM is released below: wait (bounded) until every MMA of this CTA has completed
+      umma_commit(mdone);
+      if (!mbar_wait_bounded(mdone, 0)) atomicOr(&g_enc_tc_err, kErrTimeoutLoad);
+    }
+  } else {
+    // ------------------------------------------------------------ workers
+    const int wi = warp - 2;
+    const int q = warp & 3;        // TMEM lane quarter of this warp (epilogue)
+    const int h = wi >> 2;         // epilogue: group pairs 2h and 2h + 1; separation: chunk pair h
+    const int srow = 32 * (wi & 3) + lane;  // separation: the row this thread rewrites
+    // signs + even/odd separation of row srow of chunk pair h of tile i, in place
+    auto separate = [&](int i) -> bool {
+      const int cs = i % kSpCstSlots;
+      if (!mbar_wait_bounded(&cfull[cs], (i / kSpCstSlots) & 1)) return false;
+      const uint4* sg4 = reinterpret_cast<const uint4*>(sC + cs * kSpCst + 256 * 4);  // 8 samples per uint4
+      const int c0 = 4 * i + 2 * h;  // chunks c0 (samples 128h .. +63) and c0 + 1 (128h + 64 .. +127)
+      const int s0 = c0 % kSpRing, s1 = (c0 + 1) % kSpRing;
+      if (!(mbar_wait_bounded(&rfull[s0], (c0 / kSpRing) & 1) && mbar_wait_bounded(&rfull[s1], ((c0 + 1) / kSpRing) & 1)))
+        return false;
+      uint8_t* p0 = sR + s0 * kSpChunk;
+      uint8_t* p1 = sR + s1 * kSpChunk;
+      uint4 in[16];  // this row's 128 samples, signs applied
+#pragma unroll
+      for (int u = 0; u < 16; ++u) {
+        uint4 v = *reinterpret_cast<const uint4*>((u < 8 ? p0 : p1) + sw128_off(srow, u & 7));
+        const uint4 m = sg4[16 * h + u];
+        v.x ^= m.x;
+        v.y ^= m.y;
+        v.z ^= m.z;
+        v.w ^= m.w;
+        in[u] = v;
+      }
+#pragma unroll
+      for (int v = 0; v < 8; ++v) {  // unit v: samples 128h + 16v .. + 15 -> 8 even, 8 odd
+        const uint4 A = in[2 * v], B = in[2 * v + 1];
+        *reinterpret_cast<uint4*>(p0 + sw128_off(srow, v)) =
+            make_uint4(prmt(A.x, A.y, 0x5410u), prmt(A.z, A.w, 0x5410u), prmt(B.x, B.y, 0x5410u),
+                       prmt(B.z, B.w, 0x5410u));
+        *reinterpret_cast<uint4*>(p1 + sw128_off(srow, v)) =
+            make_uint4(prmt(A.x, A.y, 0x7632u), prmt(A.z, A.w, 0x7632u), prmt(B.x, B.y, 0x7632u),
+                       prmt(B.z, B.w, 0x7632u));
+      }
+      fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor cores
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&rdone[s0]);
+        mbar_arrive(&rdone[s1]);
+      }
+      return true;
+    };
+    bool ok = ntile > 0 ? __all_sync(0xffffffffu, separate(0)) : true;
+    int job = ntile > 0 ? job_of(bt.j, bt.njobs, 0, t_begin) : 0;
+    for (int i = 0; i < ntile && ok; ++i) {
+      if (i + 1 < ntile && !__all_sync(0xffffffffu, separate(i + 1))) {
+        ok = false;
+        break;
+      }
+      const int t = t_begin + i;
+      job = job_of(bt.j, bt.njobs, job, t);
+      const TcJob& J = bt.j[job];
+      const int a = i & 1;
+      // warp-uniform outcome: the tcgen05.ld below needs the whole warp
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(&tfull[a], (i >> 1) & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int r = (t - J.tile0) * kTcRows + 32 * q + lane;
+      const bool valid = r < J.rows;
+      const int bh = valid ? r / J.n : 0;
+      const size_t orow = (size_t)bh * J.T_cap + J.pos + (r - bh * J.n);
+      const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 256);
+      const float* chan = reinterpret_cast<const float*>(sC + (i % kSpCstSlots) * kSpCst);
+      uint32_t sb_lo[2 * SPC], sb_hi[2 * SPC];
+      if (h == 0) {
+        split_pair<0, G, BITS>(ta, chan, J.codes, orow, valid, sb_lo, sb_hi, &tempty[a], false);
+        split_pair<1, G, BITS>(ta, chan, J.codes, orow, valid, sb_lo, sb_hi, &tempty[a], true);
+      } else {
+        split_pair<2, G, BITS>(ta, chan, J.codes, orow, valid, sb_lo, sb_hi, &tempty[a], false);
+        split_pair<3, G, BITS>(ta, chan, J.codes, orow, valid, sb_lo, sb_hi, &tempty[a], true);
+      }
+      if (valid) {
+        uint16_t* sr = J.scales + orow * (256 / G);
+        store_scales<2 * SPC>(sr + SPC * 2 * h, sb_lo);
+        store_scales<2 * SPC>(sr + SPC * (6 - 2 * h), sb_hi);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&cempty[i % kSpCstSlots]);
+    }
+    if (!ok && lane == 0) atomicOr(&g_enc_tc_err, kErrTimeoutLoad);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+
 void tc_prepare() {
   static std::once_flag once;
   std::call_once(once, [] {
@@ -401,6 +778,9 @@ void tc_prepare() {
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<kD, false>::kSmem);
             cudaFuncSetAttribute(encode_tc_kernel<kD, true, kG, kB, kTcMaxJobs>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, TcCfg<kD, true>::kSmem);
+            if constexpr (kD == 256)
+              cudaFuncSetAttribute(encode_split_kernel<kG, kB, kTcMaxJobs>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kSpSmem);
             return 0;
           });
   });
@@ -413,15 +793,28 @@ cudaError_t tc_launch(cudaLaunchConfig_t cfg, const TcBatch<kTcMaxJobs>& bt, int
   return cudaLaunchKernelEx(&cfg, encode_tc_kernel<D, EX, G, BITS, kTcMaxJobs>, bt);
 }
 
+template <int G, int BITS>
+cudaError_t split_launch(cudaLaunchConfig_t cfg, const TcBatch<kTcMaxJobs>& bt, int tiles, int sms) {
+  cfg.gridDim = dim3(std::min(tiles, sms));
+  cfg.blockDim = dim3(kSpThreads);
+  cfg.dynamicSmemBytes = kSpSmem;
+  return cudaLaunchKernelEx(&cfg, encode_split_kernel<G, BITS, kTcMaxJobs>, bt);
+}
+
 }  // namespace
 
 bool encode_tc_supported(int D, int G) { return (D == 128 || D == 256) && (G == 32 || G == 16); }
 
+bool encode_split_supported(const kvq_plan* p) { return p->D == 256 && p->xform == 0 && (p->G == 32 || p->G == 16); }
+
 // Grouped launch over jobs of one head_dim (128 or 256), group (32 or 16), transform and
-// code width (4 or 8 bits); jobs with no rows are skipped.
-kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t strm) {
+// code width (4 or 8 bits); jobs with no rows are skipped. split: the radix-2 split
+// kernel (D = 256, SRFT plans) instead of the dense product.
+kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t strm, bool split) {
   const int D = jobs[0].plan->D;
   const bool ex = jobs[0].plan->xform == 1;  // SRHT: exact W
+  if (split && !encode_split_supported(jobs[0].plan))
+    return fail(KVQ_ERR_UNSUPPORTED, "encode: the radix-2 split kernel serves head_dim 256 SRFT plans");
   tc_prepare();
   int i0 = 0;
   while (i0 < njobs) {
@@ -442,15 +835,25 @@ kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t 
       if (st != KVQ_OK) return st;
       // W = Lambda F_r diag(s): per 128-channel half, 128 hi rows then 128 lo rows, D
       // columns; exact W (SRHT): H diag(s), D rows (channels), D columns
-      const uint64_t wd[2] = {(uint64_t)D, (uint64_t)(ex ? D : 2 * D)};
-      const uint64_t ws[1] = {(uint64_t)D * 2};
-      const uint32_t wb[2] = {64u, (uint32_t)(ex ? D : 256)};
-      st = encode_tiled(&J.wmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, j.plan->wt_dev, wd, ws, wb,
-                        CU_TENSOR_MAP_SWIZZLE_128B, "encode weights");
+      // split: F128 [hi 128 rows; lo 128 rows] x 128 columns (the plan-independent operand)
+      if (split) {
+        const uint64_t fd[2] = {128u, 256u};
+        const uint64_t fs[1] = {256u};
+        const uint32_t fb[2] = {64u, 256u};
+        st = encode_tiled(&J.wmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, j.plan->rot_dev, fd, fs, fb,
+                          CU_TENSOR_MAP_SWIZZLE_128B, "encode F128");
+      } else {
+        const uint64_t wd[2] = {(uint64_t)D, (uint64_t)(ex ? D : 2 * D)};
+        const uint64_t ws[1] = {(uint64_t)D * 2};
+        const uint32_t wb[2] = {64u, (uint32_t)(ex ? D : 256)};
+        st = encode_tiled(&J.wmap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, j.plan->wt_dev, wd, ws, wb,
+                          CU_TENSOR_MAP_SWIZZLE_128B, "encode weights");
+      }
       if (st != KVQ_OK) return st;
       J.codes = j.codes;
       J.scales = j.scales;
       J.chan = j.plan->enc_dev->chan;
+      J.sgn = j.plan->enc_dev->sgn;
       J.rows = (int)rows;
       J.n = j.n;
       J.T_cap = j.T_cap;
@@ -479,6 +882,7 @@ kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t 
     cfg.numAttrs = 1;
     cudaError_t e = dispatch_dgb(D, jobs[0].plan->G, jobs[0].plan->bits, [&](auto d, auto g, auto b) {
       constexpr int kD = decltype(d)::value, kG = decltype(g)::value, kB = decltype(b)::value;
+      if (split) return split_launch<kG, kB>(cfg, bt, tiles, sms);
       return ex ? tc_launch<kD, true, kG, kB>(cfg, bt, tiles, sms) : tc_launch<kD, false, kG, kB>(cfg, bt, tiles, sms);
     });
     if (e == cudaSuccess) e = cudaGetLastError();

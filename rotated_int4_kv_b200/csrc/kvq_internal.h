@@ -82,9 +82,12 @@ kvq_status check_plan_device(const kvq_plan* p);
 
 // tensor-core encode (kvq_encode_tc.cu)
 bool encode_tc_supported(int D, int G);
-kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t s);
+bool encode_split_supported(const kvq_plan* p);
+kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t s, bool split);
 uint32_t encode_tc_error_flags(bool clear);
-// encode path: 0 = tensor cores where supported, else the register FFT; 1 = register FFT; 2 = tensor cores
+// encode path: 0 = tensor cores where supported (the radix-2 split kernel for head_dim 256 SRFT
+// plans), else the register FFT; 1 = register FFT; 2 = tensor cores, dense product; 3 = tensor
+// cores, radix-2 split (head_dim 256 SRFT only)
 int encode_path();
 kvq_status dispatch_encode(const kvq_encode_job* jobs, int njobs, cudaStream_t s);
 

@@ -45,7 +45,7 @@ CASES = [
 
 
 _TALLY = BOUNDARY_TALLY  # shared with the fused-append tests
-PATHS = ["fft", "tensor"]
+PATHS = ["fft", "tensor", "split"]  # split: the radix-2 split kernel (head_dim 256 SRFT plans)
 
 
 @pytest.fixture
@@ -61,6 +61,8 @@ def test_encode_matches_oracle(kvq, case, encode_path):
     wl_name, B, H, n, T_cap, pos, G = case
     wl = kvgen.WORKLOADS[wl_name]
     D = wl.head_dim
+    if encode_path == "split" and D != 256:
+        pytest.skip("the radix-2 split kernel serves head_dim 256")
     s, lam = kvgen.plan_params(D, seed=11)
     plan = kvq.Plan(s, lam, group=G)
     x16 = kvgen.kv_numpy(wl, "k", (B, H, n, D), seed=12)
@@ -215,3 +217,17 @@ def test_encode_batch_rejects_mixed_head_dims(kvq):
     with pytest.raises(kvq.KvqError) as e:
         kvq.encode_batch([j1, j2])
     assert e.value.status == -1
+
+
+def test_split_path_refuses_other_plans(kvq):
+    dev = torch.device("cuda")
+    plan = kvq.Plan(*kvgen.plan_params(128))
+    codes = torch.zeros((1, 1, 4, 64), dtype=torch.uint8, device=dev)
+    scales = torch.zeros((1, 1, 4, 4), dtype=torch.float16, device=dev)
+    kvq.set_encode_path("split")
+    try:
+        with pytest.raises(kvq.KvqError) as e:
+            kvq.encode(plan, torch.zeros((1, 1, 4, 128), dtype=torch.float16, device=dev), codes, scales, 0)
+    finally:
+        kvq.set_encode_path("auto")
+    assert e.value.status == -2

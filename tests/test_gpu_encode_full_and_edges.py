@@ -4,13 +4,14 @@
   (26 layers x K and V, each 4096 vectors of D = 256, int4 codes, SRFT plans with
   their own s and lambda). The same launch runs here on both encode paths, and every
   row of every job -- so the first and last tile of each job and the rows on both
-  sides of every 128-row tile boundary -- is checked against the oracle.
+  sides of every 128-row tile boundary -- is checked against the oracle, on every
+  encode path (auto, register FFT, dense tensor-core product, radix-2 split).
 * The quantiser's edge cases ("Methodik" 2 of gist.science/de/paper/2605.05699:
   per-group abs-max scale and rounding to signed int4), whose oracle behaviour the
   pins in tests/test_oracle_pins.py fix: groups whose absmax / 7 exceeds the fp16
   range (scale clamped to 65504, codes clamped to +-7), groups small enough for an
   fp16-subnormal scale (codes clamped where the coarse scale would round to 8), and
-  all-zero vectors (zero scale, zero codes). They run through both encode paths at
+  all-zero vectors (zero scale, zero codes). They run through every encode path at
   both head dims and through the fused append of kvq_attend_decode_append.
 """
 import numpy as np
@@ -41,7 +42,7 @@ def encode_path(kvq, request):
     kvq.set_encode_path("auto")
 
 
-@pytest.mark.parametrize("encode_path", ["auto", "fft"], indirect=True)
+@pytest.mark.parametrize("encode_path", ["auto", "fft", "tensor", "split"], indirect=True)
 def test_gemma_step_grouped_encode_every_row(kvq, encode_path):
     """The benchmark's encode launch (bench.py, default workload, rank 0, first input set)."""
     wl = kvgen.WORKLOADS["gemma"]
@@ -111,9 +112,11 @@ def _expect_edge_effects(x16, s, lam, G, scales):
     assert zero_rows.any() and (sc[zero_rows] == 0).all()
 
 
-@pytest.mark.parametrize("encode_path", ["tensor", "fft"], indirect=True)
+@pytest.mark.parametrize("encode_path", ["tensor", "fft", "split"], indirect=True)
 @pytest.mark.parametrize("D", [128, 256])
 def test_quantiser_edges_on_both_encode_paths(kvq, encode_path, D):
+    if encode_path == "split" and D != 256:
+        pytest.skip("the radix-2 split kernel serves head_dim 256")
     s, lam = kvgen.plan_params(D, seed=31, kind="k")
     plan = kvq.Plan(s, lam)
     x16 = edge_vectors(D, lam, s, n_each=40, seed=D)
