@@ -440,98 +440,112 @@ __device__ __forceinline__ uint4 lds128_here(const void* p) {
 // byte offset of 16-byte unit u of row r in a 128-byte-swizzled chunk (1024-byte aligned)
 __device__ __forceinline__ uint32_t sw128_off(int r, int u) { return (uint32_t)(r * 128 + ((u ^ (r & 7)) << 4)); }
 
-// Frequency k = 16 GP + TT of a group pair: X_k = E_k + W^k O_k (SIDE 0) or X_{128-k} =
-// conj(E_k - W^k O_k) (SIDE 1), W = e^{-2 pi i / 256}, times the channel factors, into the
-// chunk's local channels.
-template <int GP, int TT, int SIDE>
-__device__ __forceinline__ void split_freq(const float (&e)[32], const float (&o)[32], float e32, float e33, float o32,
-                                           float o33, const float* cc, float (&y)[32]) {
+// (cos, sin)(2 pi k / 256) for k = 16 GP + TT, at [17 GP + TT] (GP = 0..3, TT = 0..16);
+// written once per device from the same exact-octant Taylor evaluation as the
+// compile-time twiddles of the register FFT
+__constant__ float2 c_split_tw[4 * 17];
+
+// Frequency k = 16 GP + TT of a group pair: X_k = E_k + W^k O_k into chunk GP (y0) and
+// X_{128-k} = conj(E_k - W^k O_k) into chunk 7 - GP (y1), W = e^{-2 pi i / 256}, each value
+// times its channel factor. GP is a runtime value (one code path for every pair).
+template <int TT>
+__device__ __forceinline__ void split_freq(int GP, const float (&e)[32], const float (&o)[32], float e32, float e33,
+                                           float o32, float o33, const float* c0, const float* c1, float (&y0)[32],
+                                           float (&y1)[32]) {
   float er, ei, orr, oi;
-  if constexpr (TT < 16) {
-    er = e[2 * TT];
-    orr = o[2 * TT];
+  if constexpr (TT == 0) {
     // k = 0: slot 1 holds X_64, and Im X_0 = 0
-    ei = (GP == 0 && TT == 0) ? 0.0f : e[2 * TT + 1];
-    oi = (GP == 0 && TT == 0) ? 0.0f : o[2 * TT + 1];
-  } else if constexpr (GP < 3) {
-    er = e32;
-    ei = e33;
-    orr = o32;
-    oi = o33;
-  } else {  // k = 64: E_64 and O_64 are real
-    er = e33;
-    ei = 0.0f;
-    orr = o33;
-    oi = 0.0f;
-  }
-  constexpr float c = static_cast<float>(cos2pi_frac(16 * GP + TT, 256));
-  constexpr float sn = static_cast<float>(sin2pi_frac(16 * GP + TT, 256));
-  const float xr = fmaf(c, orr, fmaf(sn, oi, er));   // Re X_k = Re (E + W^k O)
-  const float xi = fmaf(c, oi, fmaf(-sn, orr, ei));  // Im X_k
-  if constexpr (SIDE == 0) {
-    // channel 2k - 1 = Re X_k (local 2TT - 1), 2k = Im X_k (local 2TT); local 0 of chunk 0 is X_0
-    if constexpr (TT >= 1) y[2 * TT - 1] = xr * cc[2 * TT - 1];
-    if constexpr (TT <= 15) y[2 * TT] = (GP == 0 && TT == 0 ? xr : xi) * cc[2 * TT];
+    er = e[0];
+    orr = o[0];
+    ei = GP == 0 ? 0.0f : e[1];
+    oi = GP == 0 ? 0.0f : o[1];
+  } else if constexpr (TT < 16) {
+    er = e[2 * TT];
+    ei = e[2 * TT + 1];
+    orr = o[2 * TT];
+    oi = o[2 * TT + 1];
   } else {
-    // Re X_{128-k} = 2 Re E - Re X_k at local 31 - 2TT, Im X_{128-k} = Im X_k - 2 Im E at 32 - 2TT
-    if constexpr (TT <= 15) y[31 - 2 * TT] = fmaf(2.0f, er, -xr) * cc[31 - 2 * TT];
-    if constexpr (TT >= 1) y[32 - 2 * TT] = fmaf(-2.0f, ei, xi) * cc[32 - 2 * TT];
+    // k = 16 GP + 16: slots (2k, 2k + 1), or for GP = 3 the real E_64 and O_64 (slot 1)
+    const bool ny = GP == 3;
+    er = ny ? e33 : e32;
+    ei = ny ? 0.0f : e33;
+    orr = ny ? o33 : o32;
+    oi = ny ? 0.0f : o33;
+  }
+  const float2 w = c_split_tw[17 * GP + TT];
+  const float xr = fmaf(w.x, orr, fmaf(w.y, oi, er));   // Re X_k = Re (E + W^k O)
+  const float xi = fmaf(w.x, oi, fmaf(-w.y, orr, ei));  // Im X_k
+  // chunk GP: channel 2k - 1 = Re X_k (local 2TT - 1), 2k = Im X_k (local 2TT); local 0 of chunk 0 is X_0
+  if constexpr (TT >= 1) y0[2 * TT - 1] = xr * c0[2 * TT - 1];
+  if constexpr (TT == 0) y0[0] = (GP == 0 ? xr : xi) * c0[0];
+  else if constexpr (TT <= 15) y0[2 * TT] = xi * c0[2 * TT];
+  // chunk 7 - GP: Re X_{128-k} = 2 Re E - Re X_k at local 31 - 2TT, Im X_{128-k} = Im X_k - 2 Im E at 32 - 2TT
+  if constexpr (TT <= 15) y1[31 - 2 * TT] = fmaf(2.0f, er, -xr) * c1[31 - 2 * TT];
+  if constexpr (TT >= 1) y1[32 - 2 * TT] = fmaf(-2.0f, ei, xi) * c1[32 - 2 * TT];
+}
+
+template <int... TT>
+__device__ __forceinline__ void split_freqs(std::integer_sequence<int, TT...>, int GP, const float (&e)[32],
+                                            const float (&o)[32], float e32, float e33, float o32, float o33,
+                                            const float* c0, const float* c1, float (&y0)[32], float (&y1)[32]) {
+  (split_freq<TT>(GP, e, o, e32, e33, o32, o33, c0, c1, y0, y1), ...);
+}
+
+// Quantise and store one channel chunk of a tile row (codes and scale bits).
+template <int G, int BITS>
+__device__ __forceinline__ void split_store(const float (&y)[32], int chunk, uint8_t* codes, uint16_t* srow,
+                                            bool valid) {
+  constexpr int SPC = 32 / G;
+  uint32_t w[BITS], sg[SPC];
+  quantize_chunk<G, BITS>(y, w, sg);
+  if (valid) {
+    store_chunk<256, BITS>(codes, 0, chunk, w);
+    if constexpr (SPC == 1) srow[chunk] = (uint16_t)sg[0];
+    else *reinterpret_cast<uint32_t*>(srow + 2 * chunk) = sg[0] | (sg[1] << 16);
   }
 }
 
-template <int GP, int SIDE, int... TT>
-__device__ __forceinline__ void split_freqs(std::integer_sequence<int, TT...>, const float (&e)[32], const float (&o)[32],
-                                            float e32, float e33, float o32, float o33, const float* cc,
-                                            float (&y)[32]) {
-  (split_freq<GP, TT, SIDE>(e, o, e32, e33, o32, o33, cc, y), ...);
+// E_k and O_k (k = 16 GP + tt, tt = 0..16) of one tile row, issued as TMEM loads (the
+// caller waits with tmem_ld_wait before using them)
+struct SplitIn {
+  float e[32], o[32], e32, e33, o32, o33;
+};
+__device__ __forceinline__ void split_load(SplitIn& v, int GP, uint32_t ta) {
+  tmem_ld32(ta + 32 * GP, v.e);
+  tmem_ld32(ta + 128 + 32 * GP, v.o);
+  // k = 16 GP + 16: slots (2k, 2k + 1), or for GP = 3 the real X_64 in slot 1 (read with slot 0)
+  const uint32_t xc = GP < 3 ? 32 * GP + 32 : 0;
+  tmem_ld2(ta + xc, v.e32, v.e33);
+  tmem_ld2(ta + 128 + xc, v.o32, v.o33);
+}
+__device__ __forceinline__ void split_fence(SplitIn& v) {
+  tmem_regs_fence(v.e);
+  tmem_regs_fence(v.o);
+  tmem_regs_fence(v.e32);
+  tmem_regs_fence(v.e33);
+  tmem_regs_fence(v.o32);
+  tmem_regs_fence(v.o33);
 }
 
-// One channel chunk of a tile row: SIDE 0 = chunk GP, from X_k (k = 16 GP + tt, tt = 0..16);
-// SIDE 1 = chunk 7 - GP, from X_{128-k} (the same E_k, O_k). E and O are (re)loaded from TMEM
-// for each side, which keeps one side's values live at a time (a CTA of ten warps gets at
-// most 168 registers a thread). sb collects the chunk's scale bits at sb[SPC * slot].
-template <int GP, int SIDE, int G, int BITS>
-__device__ __forceinline__ void split_side(uint32_t ta, const float* chan, uint8_t* codes, size_t orow, bool valid,
-                                           uint32_t (&sb)[64 / G], int slot, uint64_t* tempty, bool release) {
-  constexpr int SPC = 32 / G;
-  float e[32], o[32], e32, e33, o32, o33;
-  tmem_ld32(ta + 32 * GP, e);
-  tmem_ld32(ta + 128 + 32 * GP, o);
-  // k = 16 GP + 16: slots (2k, 2k + 1), or for GP = 3 the real X_64 in slot 1 (read with slot 0)
-  constexpr int xc = GP < 3 ? 32 * GP + 32 : 0;
-  tmem_ld2(ta + xc, e32, e33);
-  tmem_ld2(ta + 128 + xc, o32, o33);
+// Group pair GP of a tile row: channel chunks GP (from X_k, k = 16 GP + tt, tt = 0..16) and
+// 7 - GP (from X_{128-k}), both formed from one TMEM load of E_k and O_k.
+template <int G, int BITS>
+__device__ __forceinline__ void split_pair(int GP, uint32_t ta, const float* chan, uint8_t* codes, uint16_t* srow,
+                                           bool valid, uint64_t* tempty, bool release) {
+  SplitIn v;
+  split_load(v, GP, ta);
   tmem_ld_wait();
-  tmem_regs_fence(e);
-  tmem_regs_fence(o);
-  tmem_regs_fence(e32);
-  tmem_regs_fence(e33);
-  tmem_regs_fence(o32);
-  tmem_regs_fence(o33);
+  split_fence(v);
   if (release) {  // every TMEM value of this tile is in registers: the accumulator may be reused
     tc_fence_before();
     __syncwarp();
     if ((threadIdx.x & 31) == 0) mbar_arrive(tempty);
   }
-  const float* cc = chan + 32 * (SIDE == 0 ? GP : 7 - GP);
-  float y[32];
-  // frequencies k = 16 GP + TT, TT = 0..16, with their twiddles as compile-time constants
-  split_freqs<GP, SIDE>(std::make_integer_sequence<int, 17>{}, e, o, e32, e33, o32, o33, cc, y);
-  uint32_t w[BITS], sg[SPC];
-  quantize_chunk<G, BITS>(y, w, sg);
-#pragma unroll
-  for (int j = 0; j < SPC; ++j) sb[SPC * slot + j] = sg[j];
-  if (valid) store_chunk<256, BITS>(codes, orow, SIDE == 0 ? GP : 7 - GP, w);
-}
-
-// Group pair GP of a tile row: chunks GP and 7 - GP (scale bits into sb_lo / sb_hi: the chunks
-// (2h, 2h + 1) and (6 - 2h, 7 - 2h), h = GP / 2).
-template <int GP, int G, int BITS>
-__device__ __forceinline__ void split_pair(uint32_t ta, const float* chan, uint8_t* codes, size_t orow, bool valid,
-                                           uint32_t (&sb_lo)[64 / G], uint32_t (&sb_hi)[64 / G], uint64_t* tempty,
-                                           bool release) {
-  split_side<GP, 0, G, BITS>(ta, chan, codes, orow, valid, sb_lo, GP & 1, tempty, false);
-  split_side<GP, 1, G, BITS>(ta, chan, codes, orow, valid, sb_hi, 1 - (GP & 1), tempty, release);
+  float y0[32], y1[32];
+  split_freqs(std::make_integer_sequence<int, 17>{}, GP, v.e, v.o, v.e32, v.e33, v.o32, v.o33, chan + 32 * GP,
+              chan + 32 * (7 - GP), y0, y1);
+  split_store<G, BITS>(y0, GP, codes, srow, valid);
+  split_store<G, BITS>(y1, 7 - GP, codes, srow, valid);
 }
 
 template <int G, int BITS, int MAXJ>
@@ -737,19 +751,12 @@ __global__ void __launch_bounds__(kSpThreads, 1) encode_split_kernel(const __gri
       const size_t orow = (size_t)bh * J.T_cap + J.pos + (r - bh * J.n);
       const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(a * 256);
       const float* chan = reinterpret_cast<const float*>(sC + (i % kSpCstSlots) * kSpCst);
-      uint32_t sb_lo[2 * SPC], sb_hi[2 * SPC];
-      if (h == 0) {
-        split_pair<0, G, BITS>(ta, chan, J.codes, orow, valid, sb_lo, sb_hi, &tempty[a], false);
-        split_pair<1, G, BITS>(ta, chan, J.codes, orow, valid, sb_lo, sb_hi, &tempty[a], true);
-      } else {
-        split_pair<2, G, BITS>(ta, chan, J.codes, orow, valid, sb_lo, sb_hi, &tempty[a], false);
-        split_pair<3, G, BITS>(ta, chan, J.codes, orow, valid, sb_lo, sb_hi, &tempty[a], true);
-      }
-      if (valid) {
-        uint16_t* sr = J.scales + orow * (256 / G);
-        store_scales<2 * SPC>(sr + SPC * 2 * h, sb_lo);
-        store_scales<2 * SPC>(sr + SPC * (6 - 2 * h), sb_hi);
-      }
+      uint8_t* crow = J.codes + orow * (256 * BITS / 8);
+      uint16_t* srow = J.scales + orow * (256 / G);
+      // group pairs 2h and 2h + 1 in turn (one code path: the i-cache holds the whole loop)
+#pragma unroll 1
+      for (int pp = 0; pp < 2; ++pp)
+        split_pair<G, BITS>(2 * h + pp, ta, chan, crow, srow, valid, &tempty[a], pp == 1);
       __syncwarp();
       if (lane == 0) mbar_arrive(&cempty[i % kSpCstSlots]);
     }
@@ -765,6 +772,26 @@ __global__ void __launch_bounds__(kSpThreads, 1) encode_split_kernel(const __gri
   }
 }
 
+
+// the split kernel's twiddle table, once per device (the set-up of its first launch there)
+kvq_status split_twiddles() {
+  static std::mutex mu;
+  static bool done[64] = {false};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return fail(KVQ_ERR_DEVICE, "encode: no device");
+  std::lock_guard<std::mutex> lk(mu);
+  if (!done[dev]) {
+    float2 tw[4 * 17];
+    for (int gp = 0; gp < 4; ++gp)
+      for (int tt = 0; tt <= 16; ++tt)
+        tw[17 * gp + tt] = make_float2(static_cast<float>(cos2pi_frac(16 * gp + tt, 256)),
+                                       static_cast<float>(sin2pi_frac(16 * gp + tt, 256)));
+    if (cudaMemcpyToSymbol(c_split_tw, tw, sizeof(tw)) != cudaSuccess)
+      return fail(KVQ_ERR_CUDA, "encode: twiddle table upload failed");
+    done[dev] = true;
+  }
+  return KVQ_OK;
+}
 
 void tc_prepare() {
   static std::once_flag once;
@@ -816,6 +843,10 @@ kvq_status launch_encode_tc(const kvq_encode_job* jobs, int njobs, cudaStream_t 
   if (split && !encode_split_supported(jobs[0].plan))
     return fail(KVQ_ERR_UNSUPPORTED, "encode: the radix-2 split kernel serves head_dim 256 SRFT plans");
   tc_prepare();
+  if (split) {
+    const kvq_status st = split_twiddles();
+    if (st != KVQ_OK) return st;
+  }
   int i0 = 0;
   while (i0 < njobs) {
     TcBatch<kTcMaxJobs> bt{};
