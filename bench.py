@@ -63,7 +63,7 @@ NCU_TRAFFIC = {
     # kernel -> (source digest at capture time, bytes per launch)
     "encode": ("e66cb71d3607", 112104533),       # register-FFT encode, Gemma step (52 jobs)
     "encode_tc": ("ba92cae89f03", 124381952),    # tensor-core encode, Gemma step (52 jobs)
-    "attend": ("fe582db1b810", 32586240),        # grouped int4 attention, Gemma step (26 jobs)
+    "attend": ("a86a9a2072fd", 32586240),        # grouped int4 attention, Gemma step (26 jobs)
 }
 
 
@@ -99,7 +99,9 @@ def _ncu_traffic(kind: str):
 # DRAM traffic per launch of the int4 attention kernel at the attention arms' shapes
 # (one ncu capture each, keyed like NCU_TRAFFIC by the kernel sources' digest)
 NCU_TRAFFIC_ATTN = {
-    # arm -> (source digest at capture time, bytes per launch)
+    # arm -> (source digest at capture time, bytes per launch): int4 attention, one layer
+    "mistral_32k": ("a86a9a2072fd", 606671488),   # B=16, 8/32 heads, 32769 tokens: median read + write of 6 launches
+    "longctx_128k": ("a86a9a2072fd", 605072256),  # B=4, 8/64 heads, 131073 tokens: median read + write of 6 launches
 }
 
 
@@ -415,7 +417,6 @@ def run_kvq(args, rank: int, world: int):
     if dist is not None:
         dist.barrier()
     wall1 = time.time()
-    clk.stop()
     ms = t_start.elapsed_time(t_end)
     enc_ms = [a.elapsed_time(b) for a, b in zip(ev_a, ev_b)]
     att_ms = [ev_b[s].elapsed_time(ev_a[s + 1]) for s in range(args.steps - 1)] + [ev_b[-1].elapsed_time(t_end)]
@@ -460,6 +461,7 @@ def run_kvq(args, rank: int, world: int):
     # int4 against the fp16 comparator on identical shapes (decode_case), each a CUDA
     # graph of back-to-back calls; the big caches (604 MB int4 / 2.15 GB fp16) exceed L2
     attn_arms = None
+    arms0 = time.time()
     if not args.skip_attention_arms:
         attn_arms = {}
         for key, wname, T, layers, distinct, variants in (
@@ -474,6 +476,12 @@ def run_kvq(args, rank: int, world: int):
             case["attn_speedup"] = case["fp16_attn_ms"] / case["int4_attn_ms"]
             case["int4_traffic_bytes_per_launch"] = _ncu_traffic_attn(key)
             attn_arms[key] = case
+    arms1 = time.time()
+    clk.stop()
+    if attn_arms is not None:
+        arm_clocks = clk.summary(arms0, arms1)
+        attn_arms["clocks"] = {"sm_mhz": arm_clocks["sm_mhz"], "sm_max_mhz": arm_clocks["sm_max_mhz"],
+                               "reasons": arm_clocks["reasons"], "samples": arm_clocks["samples"]}
 
     vec_step = NJ * Hkv * T
     value = job_throughput(world, vec_step, ms, args.steps)
