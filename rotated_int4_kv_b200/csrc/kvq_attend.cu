@@ -1748,7 +1748,10 @@ const Occupancy& occupancy() {
 // (C = the largest divisor of S up to 8 in the latency regime, up to 4 in the
 // throughput regime, where large clusters constrain scheduling more than they
 // save) that merge through distributed shared memory; when S > C the S / C
-// cluster partials (<= kMaxMerge) merge through the workspace.
+// cluster partials (<= kMaxMerge) merge through the workspace. The throughput regime
+// also weighs one cluster spanning all S splits and no cluster at all (C = 1): the
+// latter lets S fill every resident slot when no cluster size divides it (e.g. 9
+// splits of 4 x 8 units = 288 of 296 slots at 128K tokens instead of 8 = 256).
 // (all in tokens; a stage is 64 or 128 tokens depending on the kernel)
 constexpr int kMinTokensPerSplit = 128;
 constexpr int kMaxSplits = kMaxSplitsCfg;
@@ -1818,7 +1821,9 @@ SplitPlan choose_split(int B, int Hq, int Hkv, int T, const Occupancy& occ, int 
     for (int S = 1; S <= s_cap; ++S) {
       const int Sr = realised(S);
       if (!mergeable(Sr)) continue;
-      const int cands[2] = {cluster_for(Sr, cmax), Sr <= kMaxCluster ? Sr : 0};
+      // ... and no cluster at all (every split's partial through the workspace), which lets
+      // the split count use every resident slot when no cluster size divides it well
+      const int cands[3] = {cluster_for(Sr, cmax), Sr <= kMaxCluster ? Sr : 0, Sr <= kMaxMerge ? 1 : 0};
       for (const int C : cands) {
         if (C < 1) continue;
         const long rounds = (units * Sr + occ.cap[C] - 1) / occ.cap[C];
