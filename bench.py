@@ -58,6 +58,7 @@ KERNEL_SOURCES = {
     "encode_tc": ["kvq_encode_tc.cu", "kvq_ptx.cuh", "kvq_quant.cuh", "kvq_internal.h"],
     "encode_split": ["kvq_encode_tc.cu", "kvq_ptx.cuh", "kvq_quant.cuh", "kvq_internal.h", "srft_fft.cuh"],
     "attend": ["kvq_attend.cu", "kvq_ptx.cuh", "kvq_quant.cuh", "kvq_internal.h"],
+    "decode_tc": ["kvq_decode_tc.cu", "kvq_ptx.cuh", "kvq_internal.h"],
 }
 NCU_TRAFFIC = {
     # kernel -> (source digest at capture time, bytes per launch)
@@ -447,14 +448,26 @@ def run_kvq(args, rank: int, world: int):
     h2d = x_dev.numel() * 2 + q.numel() * 2
     d2h = out.numel() * 2
 
-    # ---- decode (the inverse, not part of the step): one launch over the step's 52 packed
-    # caches as a batch of 52 (the first plan's s and lambda for all: a throughput figure;
-    # its parity is tested per plan). Codes and scales (30.7 MB) were just written and may
-    # be L2-resident; the 109 MB fp16 output streams to HBM.
+    # ---- decode (the inverse, not part of the step): one launch over 52 packed caches of
+    # the step's shape as a batch of 52, one plan for all (the same launch is checked row by
+    # row against the oracle). The caches of the three input sets (3 x 30.7 MB) are decoded
+    # in turn, so each launch reads codes that 218 MB of other traffic has pushed out of L2;
+    # the 109 MB fp16 output streams to HBM.
+    kvq.set_decode_path(args.decode_path)
+    dec_sets = []
+    for i in range(N_INPUT_SETS):
+        dc, dsc = torch.empty_like(codes), torch.empty_like(scales)
+        kvq.encode(plans[0], X[i], dc, dsc, 0)
+        dec_sets.append((dc, dsc))
     dec_out = torch.empty((NJ, Hkv, T, D), dtype=torch.float16, device=dev)
-    ms_dec = _graph_time(torch, lambda: kvq.decode(plans[0], codes, scales, 0, T, out=dec_out), 20, 3)
+
+    def dec_all():
+        for dc, dsc in dec_sets:
+            kvq.decode(plans[0], dc, dsc, 0, T, out=dec_out)
+
+    ms_dec = _graph_time(torch, dec_all, 20, 3) / N_INPUT_SETS
     ms_dec = max_over_ranks([ms_dec], dist, dev)[0]
-    del dec_out
+    del dec_out, dec_sets
     assert kvq.poll_device_errors() == 0
 
     # ---- the attention half of the metric at bandwidth-bound and latency-bound shapes:
@@ -534,7 +547,12 @@ def run_kvq(args, rank: int, world: int):
             "decode": {"kernel_us": 1e3 * ms_dec, "ns_per_vec": 1e6 * ms_dec / vec_step,
                        "GB_s": vec_step * vec_b / (ms_dec * 1e-3) / 1e9,
                        "frac_hbm": vec_step * vec_b / (ms_dec * 1e-3) / 1e9 / hbm, "bytes_per_vec": vec_b,
-                       "note": "one launch over the 52 caches of the step; input may be L2-resident"},
+                       "kernel": (f"decode_tc_kernel<{D},{BITS},{G}>" if args.decode_path == "tensor"
+                                  else f"decode_kernel<{D},{G},{BITS}>"),
+                       "path": args.decode_path,
+                       "traffic": _ncu_traffic("decode_tc") if args.decode_path == "tensor" else None,
+                       "l2": "one launch over 52 caches of the step's shape; three cache sets decoded in turn "
+                             "(codes read from HBM)"},
             "attention_arms": attn_arms,
             "cpu_baseline": cpu,
             "e2e": {"value": world * vec_step / (e2e_ms * 1e-3) / 1e6, "unit": "Mvec/s",
@@ -758,6 +776,8 @@ def main(argv=None):
                     help="code width of the plans: 4 (the pages' int4, default) or 8 (int8 codes)")
     ap.add_argument("--skip-attention-arms", action="store_true",
                     help="default workload: leave out the int4-vs-fp16 attention arms (Mistral 32K, 128K, Qwen step)")
+    ap.add_argument("--decode-path", default="tensor", choices=["tensor", "fft"],
+                    help="kvq_decode kernel for the decode measurement (not part of the timed step)")
     ap.add_argument("--encode-path", default="auto", choices=["auto", "fft", "tensor", "split"],
                     help="encode kernel of the prefill step: tensor cores where supported (auto), "
                          "the register FFT, the dense tensor-core product, or the radix-2 split "

@@ -185,12 +185,33 @@ int kvq_get_encode_path(void);
 
 /*
  * kvq_decode -- the inverse: x_hat = diag(s) . F_r^T . (c * scale / lambda), rounded
- * to fp16, for cache rows t0 .. t0+n-1 of every (b, h).
- *   out  fp16 [B, H, n, D] contiguous.
+ * to fp16, for cache rows t0 .. t0+n-1 of every (b, h). The encode's definition
+ * ("When Quantization Is Free", gist.science/de/paper/2605.05699, "Methodik" 1-2) is
+ * a linear map up to the quantiser, so this is its exact inverse applied to the
+ * dequantised values; the pages use the same read-back for their error figures.
+ *   codes, scales  the cache as written by kvq_encode (device, 16-byte aligned);
+ *   out  fp16 [B, H, n, D] contiguous (device, 16-byte aligned), written, never read.
+ * Default kernel (kvq_set_decode_path): the tensor-core product against the plan's fp16
+ * decode matrix, within 5e-4 relative L2 of the fp64 result per vector (the fp16 output
+ * alone rounds at 2^-11 relative); path 1 runs the register inverse FFT in fp32.
  * Errors: INVALID_ARG, ALIGNMENT, CAPACITY, DEVICE, CUDA.
  */
 kvq_status kvq_decode(const kvq_plan* plan, const uint8_t* codes, const uint16_t* scales, int B,
                       int H, int T_cap, int t0, int n, uint16_t* out, void* stream);
+
+/*
+ * kvq_set_decode_path / kvq_get_decode_path -- which kernel kvq_decode runs
+ * (process-wide setting; not on the pages):
+ *   0  default: tensor cores -- the codes dequantised to fp16 (code times the group
+ *      scale, normalised per vector by a power of two), one tcgen05 product against
+ *      W_dec = diag(s) Q^T Lambda^-1 in fp16 (built with the plan), fp32 accumulation;
+ *   1  the register inverse FFT (SRFT) or Walsh-Hadamard butterflies (SRHT) in fp32.
+ * Both serve every plan (head_dim 128 / 256, group 32 / 16, int4 / int8, SRFT / SRHT).
+ * Set it between launches, not while another thread is decoding.
+ * Errors: INVALID_ARG for a value other than 0, 1.
+ */
+kvq_status kvq_set_decode_path(int path);
+int kvq_get_decode_path(void);
 
 /*
  * kvq_workspace_size -- bytes of device workspace that kvq_attend_decode and

@@ -63,6 +63,8 @@ def _load() -> ctypes.CDLL:
         "kvq_debug_wait_timeout": (I, [ctypes.c_uint32, P]),
         "kvq_set_encode_path": (I, [I]),
         "kvq_get_encode_path": (I, []),
+        "kvq_set_decode_path": (I, [I]),
+        "kvq_get_decode_path": (I, []),
         "kvq_status_string": (ctypes.c_char_p, [I]),
         "kvq_last_error": (ctypes.c_char_p, []),
     }

@@ -126,6 +126,21 @@ def get_encode_path() -> str:
     return {n: k for k, n in ENCODE_PATHS.items()}[v]
 
 
+DECODE_PATHS = {"tensor": 0, "fft": 1}
+
+
+def set_decode_path(path: str) -> None:
+    """Select the decode kernel: "tensor" (default: fp16 dequantised codes times the
+    plan's fp16 decode matrix on the tensor cores) or "fft" (register inverse transform
+    in fp32)."""
+    check(lib.kvq_set_decode_path(DECODE_PATHS[path]), "kvq_set_decode_path")
+
+
+def get_decode_path() -> str:
+    v = int(lib.kvq_get_decode_path())
+    return {n: k for k, n in DECODE_PATHS.items()}[v]
+
+
 def decode(plan: Plan, codes: torch.Tensor, scales: torch.Tensor, t0: int, n: int, out: torch.Tensor = None,
            stream=None) -> torch.Tensor:
     """Decode cache rows t0..t0+n-1 into fp16 [B, H, n, D]."""

@@ -18,7 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libkvq.so")
-SOURCES = ["kvq_api.cu", "kvq_codec.cu", "kvq_encode_tc.cu", "kvq_attend.cu"]
+SOURCES = ["kvq_api.cu", "kvq_codec.cu", "kvq_encode_tc.cu", "kvq_decode_tc.cu", "kvq_attend.cu"]
 HEADERS = ["kvq_internal.h", "kvq_ptx.cuh", "kvq_quant.cuh", "srft_fft.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxed-constexpr",

@@ -76,6 +76,10 @@ std::atomic<int> g_encode_path{0};
 
 int encode_path() { return g_encode_path.load(); }
 
+std::atomic<int> g_decode_path{0};
+
+int decode_path() { return g_decode_path.load(); }
+
 // All jobs share head_dim and group (checked by the callers).
 kvq_status dispatch_encode(const kvq_encode_job* jobs, int njobs, cudaStream_t s) {
   const kvq_plan* p = jobs[0].plan;
@@ -293,10 +297,21 @@ kvq_status kvq_plan_create_ex(kvq_plan** out, int D, int G, const int8_t* signs,
         rot[(size_t)(M + j) * M + m] = lo;
       }
   }
+  // tensor-core decode operand: W_dec = diag(s) Q^T Lambda^-1 (row n = output sample n,
+  // column = channel), one fp16 rounding per entry; the columns of each 16-byte unit in
+  // the order the kernel's dequantiser writes the channels (decode_unit_channel)
+  std::vector<uint16_t> wdec((size_t)D * D);
+  for (int n = 0; n < D; ++n)
+    for (int k = 0; k < D; ++k) {
+      const int c = (k & ~7) + kvq::decode_unit_channel(k & 7, bits);
+      const double q = hadamard ? kvq::hadamard_value(c, n) / std::sqrt((double)D) : kvq::basis_value(c, n, D);
+      wdec[(size_t)n * D + k] = kvq::half_bits((float)((double)signs[n] * q / (double)lambda[c]));
+    }
   constexpr size_t kWtOff = 4096;  // after the two CodecConsts copies, 16-byte aligned for TMA
   static_assert(2 * sizeof(kvq::CodecConsts) <= kWtOff, "plan block layout");
   const size_t rot_off = kWtOff + wt.size() * 2;
-  const size_t bytes = rot_off + rot.size() * 2;
+  const size_t wdec_off = rot_off + rot.size() * 2;
+  const size_t bytes = wdec_off + wdec.size() * 2;
   void* blk = nullptr;
   if (cudaMalloc(&blk, bytes) != cudaSuccess) {
     delete p;
@@ -308,7 +323,8 @@ kvq_status kvq_plan_create_ex(kvq_plan** out, int D, int G, const int8_t* signs,
       (!wt.empty() &&
        cudaMemcpy((char*)blk + kWtOff, wt.data(), wt.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess) ||
       (!rot.empty() &&
-       cudaMemcpy((char*)blk + rot_off, rot.data(), rot.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess)) {
+       cudaMemcpy((char*)blk + rot_off, rot.data(), rot.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess) ||
+      cudaMemcpy((char*)blk + wdec_off, wdec.data(), wdec.size() * 2, cudaMemcpyHostToDevice) != cudaSuccess) {
     cudaFree(blk);
     delete p;
     return fail(KVQ_ERR_CUDA, "plan_create: upload failed");
@@ -318,6 +334,7 @@ kvq_status kvq_plan_create_ex(kvq_plan** out, int D, int G, const int8_t* signs,
   p->dec_dev = reinterpret_cast<const kvq::CodecConsts*>((char*)blk + sizeof(kvq::CodecConsts));
   p->wt_dev = wt.empty() ? nullptr : reinterpret_cast<const uint16_t*>((char*)blk + kWtOff);
   p->rot_dev = reinterpret_cast<const uint16_t*>((char*)blk + rot_off);
+  p->wdec_dev = reinterpret_cast<const uint16_t*>((char*)blk + wdec_off);
   *out = p;
   return KVQ_OK;
 }
@@ -392,6 +409,14 @@ kvq_status kvq_set_encode_path(int path) {
 
 int kvq_get_encode_path(void) { return kvq::g_encode_path.load(); }
 
+kvq_status kvq_set_decode_path(int path) {
+  if (path < 0 || path > 1) return fail(KVQ_ERR_INVALID_ARG, "set_decode_path: path must be 0 or 1");
+  kvq::g_decode_path.store(path);
+  return KVQ_OK;
+}
+
+int kvq_get_decode_path(void) { return kvq::g_decode_path.load(); }
+
 kvq_status kvq_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* scales, int B, int H, int T_cap,
                       int t0, int n, uint16_t* out, void* stream) {
   if (!p) return fail(KVQ_ERR_INVALID_ARG, "decode: null plan");
@@ -404,6 +429,8 @@ kvq_status kvq_decode(const kvq_plan* p, const uint8_t* codes, const uint16_t* s
   if ((long)B * H > (1L << 30) || (long)T_cap * B * H > (1L << 40)) return fail(KVQ_ERR_INVALID_ARG, "decode: too large");
   kvq_status st = kvq::check_plan_device(p);
   if (st != KVQ_OK) return st;
+  if (kvq::decode_path() == 0)
+    return kvq::launch_decode_tc(p, codes, scales, B, H, T_cap, t0, n, out, (cudaStream_t)stream);
   return kvq::launch_decode(p, codes, scales, B, H, T_cap, t0, n, out, (cudaStream_t)stream);
 }
 
@@ -608,7 +635,8 @@ kvq_status kvq_debug_wait_timeout(uint32_t limit_us, void* stream) {
 
 kvq_status kvq_poll_device_errors(uint32_t* flags) {
   if (cudaDeviceSynchronize() != cudaSuccess) return fail(KVQ_ERR_CUDA, "poll: device synchronize failed");
-  const uint32_t f = kvq::codec_error_flags(true) | kvq::attend_error_flags(true) | kvq::encode_tc_error_flags(true);
+  const uint32_t f = kvq::codec_error_flags(true) | kvq::attend_error_flags(true) | kvq::encode_tc_error_flags(true) |
+                     kvq::decode_tc_error_flags(true);
   if (flags) *flags = f;
   return KVQ_OK;
 }

@@ -45,6 +45,9 @@ struct kvq_plan {
   // slot order, fp16 hi rows [128] then lo rows [128] (plan-independent; the attention
   // kernels apply the plans' signs and per-channel factors around it).
   const uint16_t* rot_dev = nullptr;
+  // Tensor-core decode operand in the same block: W_dec = diag(s) Q^T Lambda^-1 as fp16,
+  // D rows (output samples) x D columns (channels, in the dequantiser's pair order).
+  const uint16_t* wdec_dev = nullptr;
 };
 
 namespace kvq {
@@ -90,6 +93,20 @@ uint32_t encode_tc_error_flags(bool clear);
 // cores, radix-2 split (head_dim 256 SRFT only)
 int encode_path();
 kvq_status dispatch_encode(const kvq_encode_job* jobs, int njobs, cudaStream_t s);
+
+// tensor-core decode (kvq_decode_tc.cu)
+kvq_status launch_decode_tc(const kvq_plan* p, const uint8_t* codes, const uint16_t* scales, int B, int H,
+                            int T_cap, int t0, int n, uint16_t* out, cudaStream_t s);
+uint32_t decode_tc_error_flags(bool clear);
+// decode path: 0 = tensor cores (default), 1 = register FFT
+int decode_path();
+// K position p (0..7) of a 16-byte unit of the tensor-core decode's fp16 operand -> the
+// channel offset within the unit's eight channels (the dequantiser's pair order)
+inline int decode_unit_channel(int p, int bits) {
+  if (bits == 4) return (p & 1) ? (p >> 1) + 4 : (p >> 1);  // pairs (j, j + 4) of one 32-bit word
+  static const int k8[8] = {0, 2, 1, 3, 4, 6, 5, 7};       // pairs (0, 2), (1, 3) of each word
+  return k8[p];
+}
 
 // codec launchers (kvq_codec.cu)
 kvq_status launch_encode_jobs(const kvq_encode_job* jobs, int njobs, cudaStream_t s);

@@ -23,7 +23,7 @@ def test_header_declares_the_boundary():
               "kvq_last_error", "kvq_poll_device_errors", "kvq_attend_decode_batch",
               "kvq_attend_decode_noalloc", "kvq_attend_decode_append", "kvq_plan_create_transform",
               "kvq_plan_transform", "kvq_plan_create_ex", "kvq_plan_bits", "kvq_attend_split_info",
-              "kvq_debug_wait_timeout"):
+              "kvq_debug_wait_timeout", "kvq_set_decode_path", "kvq_get_decode_path"):
         assert n in names
 
 
@@ -64,6 +64,12 @@ def test_status_strings_and_host_checks():
     assert lib.kvq_attend_split_info(1, 6, 4, 128, 32, 4, 1024, None, None, None) == -2
     assert lib.kvq_attend_split_info(1, 8, 1, 96, 32, 4, 1024, None, None, None) == -2
     assert lib.kvq_attend_split_info(1, 8, 1, 128, 32, 5, 1024, None, None, None) == -2
+    # decode kernel selection: 0 (tensor cores, the default) or 1 (register FFT)
+    assert lib.kvq_get_decode_path() == 0
+    assert lib.kvq_set_decode_path(2) == -1 and lib.kvq_set_decode_path(-1) == -1
+    assert lib.kvq_get_decode_path() == 0
+    assert lib.kvq_set_decode_path(1) == 0 and lib.kvq_get_decode_path() == 1
+    assert lib.kvq_set_decode_path(0) == 0
     assert lib.kvq_debug_wait_timeout(0, None) == -1
     assert lib.kvq_debug_wait_timeout(2000000, None) == -1
     jobs = (kvq_lib.AttendJob * 2)()  # null plans: refused before any CUDA call
