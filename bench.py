@@ -63,8 +63,11 @@ KERNEL_SOURCES = {
 NCU_TRAFFIC = {
     # kernel -> (source digest at capture time, bytes per launch)
     "encode": ("e66cb71d3607", 112104533),       # register-FFT encode, Gemma step (52 jobs)
-    "encode_tc": ("ba92cae89f03", 124381952),    # tensor-core encode, Gemma step (52 jobs)
-    "attend": ("a86a9a2072fd", 32586240),        # grouped int4 attention, Gemma step (26 jobs)
+    "encode_tc": ("4a3236741c4b", 124388608),    # tensor-core encode, Gemma step (52 jobs)
+    "attend": ("a61a78c8ce3e", 32586240),        # grouped int4 attention, Gemma step (26 jobs)
+    # tensor-core decode of the step's 52 caches: 30.85 MB read + 51.41 MB written during the launch
+    # (the rest of its 109 MB output is written back from L2 after it ends)
+    "decode_tc": ("db5404aad09c", 82263936),
 }
 
 
@@ -101,8 +104,8 @@ def _ncu_traffic(kind: str):
 # (one ncu capture each, keyed like NCU_TRAFFIC by the kernel sources' digest)
 NCU_TRAFFIC_ATTN = {
     # arm -> (source digest at capture time, bytes per launch): int4 attention, one layer
-    "mistral_32k": ("a86a9a2072fd", 606671488),   # B=16, 8/32 heads, 32769 tokens: median read + write of 6 launches
-    "longctx_128k": ("a86a9a2072fd", 605072256),  # B=4, 8/64 heads, 131073 tokens: median read + write of 6 launches
+    "mistral_32k": ("a61a78c8ce3e", 606666368),   # B=16, 8/32 heads, 32769 tokens: median read + write of 6 launches
+    "longctx_128k": ("a61a78c8ce3e", 605429376),  # B=4, 8/64 heads, 131073 tokens: median read + write of 6 launches
 }
 
 
@@ -364,8 +367,16 @@ def run_kvq(args, rank: int, world: int):
         for s in range(args.steps):
             kvq.encode_batch(jobs_for(s % N_INPUT_SETS))
             attn_phase()
+        # then the decode launch of the measurement below (not part of the step), once per
+        # step, over the step's 52 packed caches with one plan (same shape and traffic)
+        kvq.set_decode_path(args.decode_path)
+        dec_out = torch.empty((NJ, Hkv, T, D), dtype=torch.float16, device=dev)
+        for s in range(args.steps):
+            kvq.decode(plans[0], codes, scales, 0, T, out=dec_out)
         torch.cuda.synchronize()
-        print(json.dumps({"ncu_mode": True, "steps": args.steps, "launches_per_step": 2}), flush=True)
+        assert kvq.poll_device_errors() == 0
+        print(json.dumps({"ncu_mode": True, "steps": args.steps, "launches_per_step": 2,
+                          "decode_launches": args.steps}), flush=True)
         return 0
 
     g_enc, g_att = [], []
