@@ -73,8 +73,19 @@ struct DtCfg {
   static constexpr int kTmemCols = 2 * D;
   static constexpr int kWordsPerChunk = 2 * BITS;    // code words per K chunk (64 channels)
   static constexpr int kBars = 8 * (2 * kRing + 2 * 2 + 2 * 2 + 2) + 16;
-  static constexpr int kSmem = kB + kCSlots * kCodeTile + kRing * kChunkA + kOut + kBars + 1024;
-  static_assert(kSmem <= 227 * 1024, "shared memory");
+  static constexpr int kBase = kB + kCSlots * kCodeTile + kRing * kChunkA + kOut + kBars;
+  static constexpr int kLimit = 227 * 1024;
+  // the dequantisers' scale rows of the next tile, one per vector (async copies), where the
+  // shared memory allows; otherwise they load them into registers
+  template <int G>
+  static constexpr int kScaleSlot = (kBase + kDtRows * (D / G) * 2 <= kLimit) ? kDtRows * (D / G) * 2 : 0;
+  // 1024 bytes of slack for aligning the base where they fit; without them the kernel checks
+  // that the base is 1024-byte aligned and refuses to run (error flag) if it is not
+  template <int G>
+  static constexpr int kSlack = (kBase + kScaleSlot<G> + 1024 <= kLimit) ? 1024 : 0;
+  template <int G>
+  static constexpr int kSmem = kBase + kScaleSlot<G> + kSlack<G>;
+  static_assert(kBase <= kLimit, "shared memory");
 };
 
 struct DtParams {
@@ -124,6 +135,25 @@ __device__ __forceinline__ void prefetch_scales(const DtParams& P, int bh, int t
   }
 }
 
+// Async copy of the scales of cache row (bh, t0 + t) into dst (zeros outside the job: a
+// copy of zero source bytes fills its destination with zeros and reads nothing).
+template <int NS>
+__device__ __forceinline__ void cp_async_scales(uint32_t* dst, const DtParams& P, int bh, int t) {
+  const bool in = bh < P.BH && t < P.n;
+  const uint16_t* sp = in ? P.scales + ((size_t)bh * P.T_cap + P.t0 + t) * (size_t)(2 * NS) : P.scales;
+  if constexpr (NS == 2) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(smem_u32(dst)), "l"(sp), "r"(in ? 8 : 0)
+                 : "memory");
+  } else {
+#pragma unroll
+    for (int i = 0; i < NS / 4; ++i)
+      asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst + 4 * i)), "l"(sp + 8 * i),
+                   "r"(in ? 16 : 0)
+                   : "memory");
+  }
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 // The row's power-of-two normaliser: e with max scale * 2^-e in [1, 2) (e = -14 when
 // the largest scale is zero or an fp16 subnormal). Returns 2^-e; alpha = 2^e.
 template <int NS>
@@ -152,12 +182,20 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
   using C = DtCfg<D, BITS>;
   constexpr int NS = D / G / 2;
   extern __shared__ uint8_t smem_raw[];
+  constexpr int kSS = C::template kScaleSlot<G>;
+  if constexpr (C::template kSlack<G> == 0) {
+    if (smem_u32(smem_raw) & 1023u) {  // uniform across the CTA: no barrier or TMEM touched yet
+      if (threadIdx.x == 0) atomicOr(&g_dec_tc_err, kErrTimeoutLoad);
+      return;
+    }
+  }
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sB = sm;
   uint8_t* sC = sB + C::kB;
   uint8_t* sA = sC + C::kCSlots * C::kCodeTile;
   uint8_t* sO = sA + C::kRing * C::kChunkA;
-  uint64_t* afull = reinterpret_cast<uint64_t*>(sO + C::kOut);
+  uint32_t* sS = reinterpret_cast<uint32_t*>(sO + C::kOut);  // scale slot (kSS bytes)
+  uint64_t* afull = reinterpret_cast<uint64_t*>(sO + C::kOut + kSS);
   uint64_t* aempty = afull + C::kRing;
   uint64_t* cfull = aempty + C::kRing;
   uint64_t* cfree = cfull + 2;
@@ -281,12 +319,35 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
         sg[2 * j + 1] = (uint32_t)__half_as_ushort(h1) * 0x10001u;
       }
     };
+    // the next tile's scale row: an async copy into this row's place in the scale slot when
+    // there is one (an arrival with release semantics does not wait for it, unlike a load in
+    // flight), else a cache prefetch now and a load at the end of the tile
+    uint32_t* srow = sS + row * NS;
+    auto next_scales = [&](int i) {
+      int bh0, tt0;
+      dt_tile_origin(P, t_begin + i, bh0, tt0);
+      if constexpr (kSS > 0) {
+        cp_async_scales<NS>(srow, P, bh0 + bh_l, tt0 + t_l);
+      } else {
+        prefetch_scales<NS>(P, bh0 + bh_l, tt0 + t_l);
+      }
+    };
+    auto take_scales = [&](int i, uint32_t (&sc)[NS]) {
+      if constexpr (kSS > 0) {
+        cp_async_wait_all();
+#pragma unroll
+        for (int j = 0; j < NS; ++j) sc[j] = srow[j];
+      } else {
+        int bh0, tt0;
+        dt_tile_origin(P, t_begin + i, bh0, tt0);
+        load_scales<NS>(P, bh0 + bh_l, tt0 + t_l, sc);
+      }
+    };
     uint32_t sg[2 * NS];
     if (ntile > 0) {
-      int bh0, tt0;
       uint32_t sc[NS];
-      dt_tile_origin(P, t_begin, bh0, tt0);
-      load_scales<NS>(P, bh0 + bh_l, tt0 + t_l, sc);
+      next_scales(0);
+      take_scales(0, sc);
       factors(sc, sg);
     }
     for (int i = 0; i < ntile; ++i) {
@@ -296,11 +357,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
         if (lane == 0) atomicOr(&g_dec_tc_err, kErrTimeoutLoad);
         break;
       }
-      if (i + 1 < ntile) {  // the next tile's scales, loaded after this tile's last arrival
-        int bh0, tt0;
-        dt_tile_origin(P, t_begin + i + 1, bh0, tt0);
-        prefetch_scales<NS>(P, bh0 + bh_l, tt0 + t_l);
-      }
+      if (i + 1 < ntile) next_scales(i + 1);
       bool ok = true;
 #pragma unroll
       for (int kc = 0; kc < C::KC; ++kc) {
@@ -368,12 +425,10 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
         break;
       }
       if (i + 1 < ntile) {
-        // the next tile's scales are loaded after this tile's last arrival: a release arrival
-        // waits for every load of its thread still in flight
-        int bh0, tt0;
+        // the next tile's factors, after this tile's last arrival: a release arrival waits
+        // for every load of its thread still in flight
         uint32_t sn[NS];
-        dt_tile_origin(P, t_begin + i + 1, bh0, tt0);
-        load_scales<NS>(P, bh0 + bh_l, tt0 + t_l, sn);
+        take_scales(i + 1, sn);
         factors(sn, sg);
       }
     }
@@ -483,12 +538,13 @@ cudaError_t dt_launch(const DtParams& P, int sms, cudaStream_t strm) {
   using C = DtCfg<D, BITS>;
   static std::once_flag once;
   std::call_once(once, [] {
-    cudaFuncSetAttribute(decode_tc_kernel<D, BITS, G>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
+    cudaFuncSetAttribute(decode_tc_kernel<D, BITS, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         C::template kSmem<G>);
   });
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(std::min(P.ntiles, sms));
   cfg.blockDim = dim3(kDtThreads);
-  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.dynamicSmemBytes = C::template kSmem<G>;
   cfg.stream = strm;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
