@@ -29,8 +29,8 @@
 //               scales by a direct load (one tile ahead), its codes from the slot ->
 //               exact fp16 integers (one lop3 per pair) -> times the normalised scale
 //               (fp16x2) -> 16-byte stores into the 128-byte-swizzled K-major layout of a
-//               ring of 16 KB K chunks (three at D = 256, so that the dequantisers run two
-//               chunks ahead of the MMAs), freed by the MMAs that read them;
+//               ring of 16 KB K chunks (three at D = 256, six at D = 128; two chunks per
+//               step at D = 128: one wait, one proxy fence), freed by the MMAs that read them;
 //   warps 6-13  epilogue, two per TMEM lane quarter (32 rows, half of the D columns
 //               each): 32 columns per step (the next step's TMEM load in flight) -> times
 //               2^e -> fp16 -> a swizzled 2 KB staging tile (two per warp at D = 128) ->
@@ -359,37 +359,48 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
       }
       if (i + 1 < ntile) next_scales(i + 1);
       bool ok = true;
+      // CPS K chunks per step: one wait for their ring slots, one proxy fence and CPS
+      // arrivals per step, their conversions interleaved (more independent work per warp).
+      // Pairs need a ring of at least four chunks: with three, waiting for two free slots
+      // cuts the dequantisers' lead over the MMAs (measured slower at D = 256).
+      constexpr int CPS = C::kRing >= 4 ? 2 : 1;
 #pragma unroll
-      for (int kc = 0; kc < C::KC; ++kc) {
-        const int c = i * C::KC + kc, s = c % C::kRing;
-        // this chunk's code words (8 for int4, 16 for int8) from 16-byte pieces of the row
+      for (int kp = 0; kp < C::KC; kp += CPS) {
+        const int c0 = i * C::KC + kp;
+        // the step's code words (8 per chunk for int4, 16 for int8) from 16-byte pieces of the row
         constexpr int WPC = C::kWordsPerChunk;
-        uint32_t w[WPC];
+        uint32_t w[CPS * WPC];
 #pragma unroll
-        for (int pc = 0; pc < WPC / 4; ++pc) {
-          const uint4 v = code_piece<D, BITS>(cs, row, (WPC / 4) * kc + pc);
+        for (int pc = 0; pc < CPS * WPC / 4; ++pc) {
+          const uint4 v = code_piece<D, BITS>(cs, row, (WPC / 4) * kp + pc);
           w[4 * pc] = v.x;
           w[4 * pc + 1] = v.y;
           w[4 * pc + 2] = v.z;
           w[4 * pc + 3] = v.w;
         }
-        if (kc == C::KC - 1) {  // every code of this tile has been read: release the slot
+        if (kp + CPS == C::KC) {  // every code of this tile has been read: release the slot
           __syncwarp();
           if (lane == 0) mbar_arrive(&cfree[slot]);
         }
-        if (!__all_sync(0xffffffffu, c < C::kRing || mbar_wait_bounded(&aempty[s], ((c / C::kRing) - 1) & 1))) {
+        bool free_ok = true;
+#pragma unroll
+        for (int j = 0; j < CPS; ++j) {
+          const int c = c0 + j;
+          free_ok = free_ok && (c < C::kRing || mbar_wait_bounded(&aempty[c % C::kRing], ((c / C::kRing) - 1) & 1));
+        }
+        if (!__all_sync(0xffffffffu, free_ok)) {
           ok = false;
           break;
         }
-        uint8_t* dst = sA + s * C::kChunkA + row * 128;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {  // 16-byte unit u: K positions 8u .. 8u + 7 of the chunk
-          const int U = 8 * kc + u;    // unit of the row: channels 8U .. 8U + 7
+        for (int uu = 0; uu < 8 * CPS; ++uu) {  // unit uu % 8 of chunk kp + uu / 8: K positions 8u .. 8u + 7
+          const int u = uu & 7;
+          const int U = 8 * kp + uu;           // unit of the row: channels 8U .. 8U + 7
           const __half2 sc = *reinterpret_cast<const __half2*>(&sg[(8 * U) / G]);
           uint32_t h[4];
           if constexpr (BITS == 4) {
             // word U holds channels 8U .. 8U + 7 (nibble j = channel 8U + j); pair p = (j, j + 4)
-            const uint32_t x = w[u] ^ 0x88888888u;  // nibble + 8 in 0 .. 15
+            const uint32_t x = w[uu] ^ 0x88888888u;  // nibble + 8 in 0 .. 15
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
               const uint32_t m = lop3_and_or(x >> (4 * p), 0x000F000Fu, 0x64006400u);  // 1024 + code + 8
@@ -403,7 +414,7 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
             // pairs (0, 2), (1, 3) of each word
 #pragma unroll
             for (int q = 0; q < 2; ++q) {
-              const uint32_t x = w[2 * u + q] ^ 0x80808080u;  // byte + 128 in 1 .. 255
+              const uint32_t x = w[2 * uu + q] ^ 0x80808080u;  // byte + 128 in 1 .. 255
 #pragma unroll
               for (int p = 0; p < 2; ++p) {
                 const uint32_t m = lop3_and_or(x >> (8 * p), 0x00FF00FFu, 0x64006400u);  // 1024 + code + 128
@@ -414,11 +425,15 @@ __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_c
               }
             }
           }
+          uint8_t* dst = sA + ((c0 + uu / 8) % C::kRing) * C::kChunkA + row * 128;
           *reinterpret_cast<uint4*>(dst + ((u ^ sw) << 4)) = make_uint4(h[0], h[1], h[2], h[3]);
         }
         fence_proxy_async_smem();  // the stores above are read by the tensor cores (async proxy)
         __syncwarp();
-        if (lane == 0) mbar_arrive(&afull[s]);
+        if (lane == 0) {
+#pragma unroll
+          for (int j = 0; j < CPS; ++j) mbar_arrive(&afull[(c0 + j) % C::kRing]);
+        }
       }
       if (!ok) {
         if (lane == 0) atomicOr(&g_dec_tc_err, kErrTimeoutLoad);
