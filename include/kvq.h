@@ -188,7 +188,8 @@ int kvq_get_encode_path(void);
  * to fp16, for cache rows t0 .. t0+n-1 of every (b, h). The encode's definition
  * ("When Quantization Is Free", gist.science/de/paper/2605.05699, "Methodik" 1-2) is
  * a linear map up to the quantiser, so this is its exact inverse applied to the
- * dequantised values; the pages use the same read-back for their error figures.
+ * dequantised values (the pages describe no decode kernel; this one follows from that
+ * definition).
  *   codes, scales  the cache as written by kvq_encode (device, 16-byte aligned);
  *   out  fp16 [B, H, n, D] contiguous (device, 16-byte aligned), written, never read.
  * Default kernel (kvq_set_decode_path): the tensor-core product against the plan's fp16
