@@ -26,7 +26,10 @@
 //   warp 1      TMEM (two accumulators of D columns) and the single MMA thread: per
 //               tile D/64 K chunks of four M = 128, N = D, K = 16 products;
 //   warps 2-5   dequantisers, one thread per vector (tile row 32 (w - 2) + lane): its
-//               scales by a direct load (one tile ahead), its codes from the slot ->
+//               next tile's scales by an async copy into a shared slot at tile start (a
+//               release arrival waits for loads in flight but not for async copies; where
+//               the slot does not fit, a cache prefetch and a load after the tile's last
+//               arrival), its codes from the code slot ->
 //               exact fp16 integers (one lop3 per pair) -> times the normalised scale
 //               (fp16x2) -> 16-byte stores into the 128-byte-swizzled K-major layout of a
 //               ring of 16 KB K chunks (three at D = 256, six at D = 128; two chunks per
