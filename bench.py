@@ -67,7 +67,7 @@ NCU_TRAFFIC = {
     "attend": ("a61a78c8ce3e", 32586240),        # grouped int4 attention, Gemma step (26 jobs)
     # tensor-core decode of the step's 52 caches: 30.85 MB read + 51.41 MB written during the launch
     # (the rest of its 109 MB output is written back from L2 after it ends)
-    "decode_tc": ("c2a91d5d429a", 82238976),
+    "decode_tc": ("171497c41872", 83871360),
 }
 
 

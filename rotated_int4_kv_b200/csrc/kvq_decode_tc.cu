@@ -184,7 +184,7 @@ template <int D, int BITS, int G>
 __global__ void __launch_bounds__(kDtThreads, 1) decode_tc_kernel(const __grid_constant__ DtParams P) {
   using C = DtCfg<D, BITS>;
   constexpr int NS = D / G / 2;
-  extern __shared__ uint8_t smem_raw[];
+  extern __shared__ __align__(1024) uint8_t smem_raw[];  // 128-byte swizzle atoms need 1024-byte alignment
   constexpr int kSS = C::template kScaleSlot<G>;
   if constexpr (C::template kSlack<G> == 0) {
     if (smem_u32(smem_raw) & 1023u) {  // uniform across the CTA: no barrier or TMEM touched yet
